@@ -1,0 +1,384 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with
+a hand-derived value (``tests/golden``), a closed form, an invariant, or a
+brute-force numpy computation written independently of the oracle's C code.
+``test_oracle_pins.py`` runs them; ``test_oracle_mutations.py`` plants bugs in
+the oracle and checks that at least one pin catches each.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# independent numpy brute force (fp64)
+# ---------------------------------------------------------------------------
+def np_attend(q, K, V, scale):
+    s = scale * (K.astype(np.float64) @ q.astype(np.float64))
+    m = s.max()
+    w = np.exp(s - m)
+    return (w @ V.astype(np.float64)) / w.sum(), m + np.log(w.sum())
+
+
+def np_bound(q, kmin, kmax):
+    q = q.astype(np.float64)
+    return np.maximum(q * kmax.astype(np.float64), q * kmin.astype(np.float64)).sum(-1)
+
+
+def rand_shape(rng, S=2, Hq=4, Hkv=2, d=16, L=45, ps=4, B=6, A=2, budget=12, scale=None):
+    return oracle.shape(S, Hq, Hkv, d, L, ps, B, A, budget,
+                        scale if scale is not None else float(np.float32(0.37)))
+
+
+def rand_inputs(rng, sh):
+    f = lambda *s: rng.standard_normal(s).astype(np.float32)
+    Qp = f(sh.S, sh.Hq, sh.B, sh.d)
+    Qc = Qp + np.float32(0.01) * f(sh.S, sh.Hq, sh.B, sh.d)
+    # give a few tokens per head a large change
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            idx = rng.choice(sh.B, size=min(sh.A + 1, sh.B), replace=False)
+            Qc[s, h, idx] += f(len(idx), sh.d)
+    return {"Qc": Qc.astype(np.float32), "Qp": Qp, "K": f(sh.S, sh.Hkv, sh.L, sh.d),
+            "V": f(sh.S, sh.Hkv, sh.L, sh.d), "Kb": f(sh.S, sh.Hkv, sh.B, sh.d),
+            "Vb": f(sh.S, sh.Hkv, sh.B, sh.d)}
+
+
+def close(a, b, tol, what):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3g} > {tol}"
+
+
+# ---------------------------------------------------------------------------
+# golden, hand-derived
+# ---------------------------------------------------------------------------
+def pin_golden_attention():
+    g = golden("attention_two_keys.json")
+    o, lse = oracle.attend_tokens(np.array(g["q"]), np.array(g["K"]), np.array(g["V"]),
+                                  [0, 1], g["scale"])
+    close(o, g["expect_o"], 1e-7, "golden attention o")
+    close(lse, g["expect_lse"], 1e-7, "golden attention lse")
+
+
+def pin_golden_merge():
+    g = golden("merge_two_parts.json")
+    o, lse = oracle.merge(g["o1"], g["l1"], g["o2"], g["l2"])
+    close(o, g["expect_o"], 1e-12, "golden merge o")
+    close(lse, g["expect_lse"], 1e-12, "golden merge lse")
+
+
+def pin_golden_bound():
+    g = golden("quest_bound_pages.json")
+    K = np.array(g["K"], np.float32)
+    d = K.shape[1]
+    sh = oracle.shape(1, 1, 1, d, K.shape[0], g["page_size"], 1, 1, 2)
+    kmin, kmax = oracle.build_meta(sh, K[None, None])
+    close(kmin[0, 0], g["expect_kmin"], 0, "golden kmin")
+    close(kmax[0, 0], g["expect_kmax"], 0, "golden kmax")
+    U = oracle.bound_scores(np.array(g["q"], np.float32), kmin[0, 0], kmax[0, 0])
+    close(U, g["expect_U"], 0, "golden bound")
+    for k, pages in g["expect_topk"].items():
+        got = oracle.topk_pages(U, int(k))
+        assert list(got) == pages, f"golden top-{k}: {list(got)} != {pages}"
+
+
+def pin_golden_locality():
+    g = golden("locality_active.json")
+    Qc = np.array(g["Qc"], np.float32)[None, None]
+    Qp = np.array(g["Qp"], np.float32)[None, None]
+    B, d = Qc.shape[2], Qc.shape[3]
+    sh = oracle.shape(1, 1, 1, d, 1, 1, B, 1, 1)
+    mse = oracle.locality(sh, Qc, Qp)
+    close(mse[0, 0], g["expect_mse"], 0, "golden mse")
+    for a, toks in g["expect_active"].items():
+        sh.A = int(a)
+        got = oracle.active(sh, mse)
+        assert list(got[0, 0]) == toks, f"golden active top-{a}: {list(got[0, 0])} != {toks}"
+
+
+# ---------------------------------------------------------------------------
+# brute force / closed forms / invariants
+# ---------------------------------------------------------------------------
+def pin_meta_bruteforce():
+    rng = np.random.default_rng(11)
+    sh = rand_shape(rng, L=45, ps=4)      # 12 pages, last one holds 1 token
+    K = rng.standard_normal((sh.S, sh.Hkv, sh.L, sh.d)).astype(np.float32)
+    kmin, kmax = oracle.build_meta(sh, K)
+    P = oracle.n_pages(sh)
+    for p in range(P):
+        blk = K[:, :, p * sh.ps:min((p + 1) * sh.ps, sh.L), :]
+        close(kmin[:, :, p], blk.min(axis=2), 0, f"kmin page {p}")
+        close(kmax[:, :, p], blk.max(axis=2), 0, f"kmax page {p}")
+        assert np.all(kmin[:, :, p, None] <= blk) and np.all(blk <= kmax[:, :, p, None])
+
+
+def pin_attend_numpy():
+    rng = np.random.default_rng(12)
+    d, n = 24, 57
+    q = rng.standard_normal(d).astype(np.float32)
+    K = (3 * rng.standard_normal((n, d))).astype(np.float32)
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    tok = rng.choice(n, size=31, replace=False)
+    scale = 0.29
+    o, lse = oracle.attend_tokens(q, K, V, tok, scale)
+    ro, rl = np_attend(q, K[tok], V[tok], np.float64(np.float32(scale)))
+    close(o, ro, 1e-12, "attend o vs numpy")
+    close(lse, rl, 1e-12, "attend lse vs numpy")
+
+
+def pin_merge_concat():
+    """merge(attn(q,K1,V1), attn(q,K2,V2)) == attn(q, K1+K2, V1+V2)."""
+    rng = np.random.default_rng(13)
+    d = 32
+    q = rng.standard_normal(d).astype(np.float32)
+    K = (2 * rng.standard_normal((40, d))).astype(np.float32)
+    V = rng.standard_normal((40, d)).astype(np.float32)
+    scale = 0.5
+    o1, l1 = oracle.attend_tokens(q, K, V, np.arange(0, 13), scale)
+    o2, l2 = oracle.attend_tokens(q, K, V, np.arange(13, 40), scale)
+    o, lse = oracle.merge(o1, l1, o2, l2)
+    ro, rl = np_attend(q, K, V, scale)
+    close(o, ro, 1e-12, "merge == attention over the union (o)")
+    close(lse, rl, 1e-12, "merge == attention over the union (lse)")
+
+
+def pin_bound_upper():
+    """U(q,p) >= max_{j in p} q.k_j for every page."""
+    rng = np.random.default_rng(14)
+    d, ps, P = 64, 16, 40
+    for trial in range(4):
+        K = rng.standard_normal((P * ps, d)).astype(np.float32)
+        q = rng.standard_normal(d).astype(np.float32)
+        sh = oracle.shape(1, 1, 1, d, P * ps, ps, 1, 1, ps)
+        kmin, kmax = oracle.build_meta(sh, K[None, None])
+        U = oracle.bound_scores(q, kmin[0, 0], kmax[0, 0]).astype(np.float64)
+        true = (K.astype(np.float64) @ q.astype(np.float64)).reshape(P, ps).max(1)
+        tol = 1e-5 * (np.abs(q) @ np.maximum(np.abs(kmax[0, 0]), np.abs(kmin[0, 0])).T)
+        assert np.all(U >= true - tol), f"bound below true max by {np.max(true - U):.3g}"
+        close(U, np_bound(q, kmin[0, 0], kmax[0, 0]), float(np.max(tol)), "bound vs fp64")
+
+
+def pin_bound_ps1_exact():
+    """Page size 1: the bound is q.k itself; top-k pages = exact top-k tokens.
+    Small integers keep every fp32 product and partial sum exact."""
+    rng = np.random.default_rng(15)
+    d, L = 32, 300
+    K = rng.integers(-8, 9, size=(L, d)).astype(np.float32)
+    q = rng.integers(-8, 9, size=d).astype(np.float32)
+    sh = oracle.shape(1, 1, 1, d, L, 1, 1, 1, 1)
+    kmin, kmax = oracle.build_meta(sh, K[None, None])
+    U = oracle.bound_scores(q, kmin[0, 0], kmax[0, 0])
+    exact = K.astype(np.int64) @ q.astype(np.int64)
+    close(U, exact, 0, "ps=1 bound == q.k")
+    for k in (1, 5, 17):
+        order = np.lexsort((np.arange(L), -exact))  # score desc, index asc
+        want = np.sort(order[:k])
+        got = oracle.topk_pages(U, k)
+        assert list(got) == list(want), f"ps=1 top-{k}: {got} != {want}"
+
+
+def pin_locality_numpy():
+    rng = np.random.default_rng(16)
+    sh = rand_shape(rng, B=12, A=3, d=128)
+    x = rand_inputs(rng, sh)
+    mse = oracle.locality(sh, x["Qc"], x["Qp"])
+    ref = ((x["Qc"].astype(np.float64) - x["Qp"].astype(np.float64)) ** 2).mean(-1)
+    assert np.all(np.abs(mse - ref) <= 1e-5 * ref + 1e-12), "mse vs fp64"
+    act = oracle.active(sh, mse)
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            order = np.lexsort((np.arange(sh.B), -ref[s, h]))
+            gaps = np.abs(np.diff(np.sort(ref[s, h])))
+            if gaps.min() > 1e-4 * ref[s, h].max():
+                assert list(act[s, h]) == sorted(order[:sh.A]), "active set vs fp64 ranking"
+
+
+def pin_planted_recovery():
+    """Planted actives (drift 1.0 vs 0.01) are recovered exactly on the tiny
+    workload and on the first heads of the GQA workload."""
+    from sparse_long_context_mse_b200 import synth
+    for n in (0, 1):
+        cfg = synth.config(n)
+        if n == 1:
+            cfg = cfg.with_(prefix_len=64)
+        q = synth.gen_queries(cfg)
+        sh = oracle.shape_of(cfg)
+        mse = oracle.locality(sh, q["q"][1], q["q"][0])
+        act = oracle.active(sh, mse)
+        planted = q["planted"][0].numpy()
+        for s in range(cfg.num_seqs):
+            for h in range(cfg.n_q_heads):
+                want = list(np.nonzero(planted[s, h])[0])
+                assert list(act[s, h]) == want, f"cfg{n} s{s} h{h}: {list(act[s, h])} != {want}"
+
+
+def _np_dense_all(sh, x):
+    """numpy: prefix attention per row, and attention over prefix + block."""
+    G = sh.Hq // sh.Hkv
+    o_p = np.zeros((sh.S, sh.Hq, sh.B, sh.d))
+    l_p = np.zeros((sh.S, sh.Hq, sh.B))
+    full = np.zeros_like(o_p)
+    full_l = np.zeros_like(l_p)
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            g = h // G
+            Kc = np.concatenate([x["K"][s, g], x["Kb"][s, g]])
+            Vc = np.concatenate([x["V"][s, g], x["Vb"][s, g]])
+            for t in range(sh.B):
+                q = x["Qc"][s, h, t]
+                o_p[s, h, t], l_p[s, h, t] = np_attend(q, x["K"][s, g], x["V"][s, g], sh.scale)
+                full[s, h, t], full_l[s, h, t] = np_attend(q, Kc, Vc, sh.scale)
+    return o_p, l_p, full, full_l
+
+
+def pin_dense_prefix_numpy():
+    rng = np.random.default_rng(17)
+    sh = rand_shape(rng)
+    x = rand_inputs(rng, sh)
+    r = oracle.dense_prefix(sh, x["Qc"], x["K"], x["V"], x["Kb"], x["Vb"])
+    o_p, l_p, full, full_l = _np_dense_all(sh, x)
+    close(r["o_p"], o_p, 1e-6, "dense o_p vs numpy")
+    close(r["l_p"], l_p, 1e-6, "dense L_p vs numpy")
+    close(r["out"], full, 1e-6, "dense out == attention over prefix+block")
+    close(r["lse"], full_l, 1e-5, "dense lse == logsumexp over prefix+block")
+
+
+def pin_gqa_mapping():
+    """Query head h reads KV head h // G: make the KV heads very different."""
+    rng = np.random.default_rng(18)
+    sh = rand_shape(rng, S=1, Hq=6, Hkv=3, L=20, B=3)
+    x = rand_inputs(rng, sh)
+    for g in range(sh.Hkv):
+        x["V"][0, g] += np.float32(10.0 * (g + 1))
+    r = oracle.dense_prefix(sh, x["Qc"], x["K"], x["V"], x["Kb"], x["Vb"])
+    o_p, l_p, _, _ = _np_dense_all(sh, x)
+    close(r["o_p"], o_p, 1e-5, "GQA mapping (o_p)")
+
+
+def _step_inputs(seed, **kw):
+    rng = np.random.default_rng(seed)
+    sh = rand_shape(rng, **kw)
+    x = rand_inputs(rng, sh)
+    kmin, kmax = oracle.build_meta(sh, x["K"])
+    cache = oracle.dense_prefix(sh, x["Qp"], x["K"], x["V"], x["Kb"], x["Vb"])
+    return sh, x, kmin, kmax, cache
+
+
+def pin_step_dense_equiv():
+    """|A| = B and a budget covering the prefix: LoSA == dense attention."""
+    sh, x, kmin, kmax, cache = _step_inputs(19, A=6, B=6, budget=10_000)
+    r = oracle.step(sh, x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                    cache["o_p"], cache["l_p"])
+    o_p, l_p, full, full_l = _np_dense_all(sh, x)
+    close(r["o_p"], o_p, 1e-6, "dense-equivalent step o_p")
+    close(r["l_p"], l_p, 1e-5, "dense-equivalent step L_p")
+    close(r["out"], full, 1e-6, "dense-equivalent step out")
+    P = oracle.n_pages(sh)
+    assert np.all(r["union_count"] == P)
+
+
+def _np_suffix(sh, x, s, h, t):
+    G = sh.Hq // sh.Hkv
+    return np_attend(x["Qc"][s, h, t], x["Kb"][s, h // G], x["Vb"][s, h // G], sh.scale)
+
+
+def _np_merge(o1, l1, o2, l2):
+    m = max(l1, l2)
+    a, b = np.exp(l1 - m), np.exp(l2 - m)
+    return (a * o1 + b * o2) / (a + b), m + np.log(a + b)
+
+
+def pin_step_stable_rows():
+    """Stable rows: cache bitwise unchanged, out = merge(cached, fresh suffix)."""
+    sh, x, kmin, kmax, cache = _step_inputs(20)
+    r = oracle.step(sh, x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                    cache["o_p"], cache["l_p"])
+    n_stable = 0
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            act = set(r["active_idx"][s, h].tolist())
+            for t in range(sh.B):
+                if t in act:
+                    continue
+                n_stable += 1
+                assert np.array_equal(r["o_p"][s, h, t].view(np.uint32),
+                                      cache["o_p"][s, h, t].view(np.uint32))
+                assert r["l_p"][s, h, t].view(np.uint32) == cache["l_p"][s, h, t].view(np.uint32)
+                os_, ls = _np_suffix(sh, x, s, h, t)
+                o, l = _np_merge(cache["o_p"][s, h, t].astype(np.float64),
+                                 float(cache["l_p"][s, h, t]), os_, ls)
+                close(r["out"][s, h, t], o, 1e-6, "stable row out")
+                close(r["lse"][s, h, t], l, 1e-5, "stable row lse")
+    assert n_stable == sh.S * sh.Hq * (sh.B - sh.A)
+
+
+def pin_step_zero_active():
+    sh, x, kmin, kmax, cache = _step_inputs(21, A=0)
+    r = oracle.step(sh, x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                    cache["o_p"], cache["l_p"])
+    assert np.array_equal(r["o_p"], cache["o_p"]) and np.array_equal(r["l_p"], cache["l_p"])
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            for t in range(sh.B):
+                os_, ls = _np_suffix(sh, x, s, h, t)
+                o, _ = _np_merge(cache["o_p"][s, h, t].astype(np.float64),
+                                 float(cache["l_p"][s, h, t]), os_, ls)
+                close(r["out"][s, h, t], o, 1e-6, "|A|=0 row out")
+    assert np.all(r["union_count"] == 0)
+
+
+def pin_step_active_rows_bruteforce():
+    """Active rows: pages are a top-k of the fp64 bound (ties within rounding
+    allowed), o_p/L_p equal numpy attention over those pages' tokens, and the
+    union count equals a brute-force set union with k <= U <= min(P, R k)."""
+    sh, x, kmin, kmax, cache = _step_inputs(22, L=93, ps=4, B=8, A=3, budget=16)
+    r = oracle.step(sh, x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                    cache["o_p"], cache["l_p"])
+    G = sh.Hq // sh.Hkv
+    k = oracle.pages_per_row(sh)
+    P = oracle.n_pages(sh)
+    for s in range(sh.S):
+        unions = [set() for _ in range(sh.Hkv)]
+        for h in range(sh.Hq):
+            g = h // G
+            for a, t in enumerate(r["active_idx"][s, h]):
+                q = x["Qc"][s, h, t]
+                U = np_bound(q, kmin[s, g], kmax[s, g])
+                pages = r["page_idx"][s, h, a]
+                assert len(set(pages.tolist())) == k and list(pages) == sorted(pages)
+                kth = np.sort(U)[::-1][k - 1]
+                tol = 1e-5 * np.abs(U).max()
+                assert np.all(U[pages] >= kth - tol), "selected page below the k-th bound"
+                others = np.setdiff1d(np.arange(P), pages)
+                assert np.all(U[others] <= kth + tol), "unselected page above the k-th bound"
+                tok = np.concatenate([np.arange(p * sh.ps, min((p + 1) * sh.ps, sh.L))
+                                      for p in pages])
+                o, l = np_attend(q, x["K"][s, g][tok], x["V"][s, g][tok], sh.scale)
+                close(r["o_p"][s, h, t], o, 1e-6, "active row o_p")
+                close(r["l_p"][s, h, t], l, 1e-5, "active row L_p")
+                os_, ls = _np_suffix(sh, x, s, h, t)
+                om, _ = _np_merge(r["o_p"][s, h, t].astype(np.float64), float(r["l_p"][s, h, t]),
+                                  os_, ls)
+                close(r["out"][s, h, t], om, 1e-6, "active row out")
+                unions[g].update(pages.tolist())
+        for g in range(sh.Hkv):
+            assert r["union_count"][s, g] == len(unions[g]), "union count vs set union"
+            assert k <= r["union_count"][s, g] <= min(P, G * sh.A * k)
+
+
+PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]
