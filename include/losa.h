@@ -1,0 +1,185 @@
+/*
+ * losa.h -- C ABI of the LoSA per-denoising-step attention library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * LoSA ("LoSA: Locality Aware Sparse Attention for Block-Wise Diffusion
+ * Language Models") speeds up the prefix attention of block-wise diffusion
+ * LMs.  Between two denoising steps only a few block tokens change much
+ * (paper, "locality of representation changes"), so each step
+ *
+ *   1. scores every block token by the MSE between its current and previous
+ *      query and keeps the top-|A| per query head as "active";
+ *   2. picks, for each active query only, the top-k prefix pages by the QUEST
+ *      bound sum_i max(q_i*kmax_i, q_i*kmin_i) over per-page key min/max,
+ *      k = budget / page_size;
+ *   3. loads the union of those pages once per GQA group and recomputes the
+ *      prefix output o_p and log-normaliser L_p of the active tokens over
+ *      their own pages; stable tokens reuse last step's o_p, L_p untouched;
+ *   4. attends every block token densely to the block's own keys (o_s, L_s);
+ *   5. merges prefix and suffix with the online-softmax (log-sum-exp) merge.
+ *
+ * The first denoising step of a block is a dense pass over the whole prefix
+ * that fills the cache for every block token (paper, limitations: the
+ * cold-start dense step), and the page min/max metadata is built once per
+ * prefix.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *   in the row-major layouts given below (innermost index last), 16-byte
+ *   aligned.  The library never allocates or frees memory and keeps no state
+ *   between calls; the workspace is caller-owned scratch.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *   legacy default stream).  Host-side validation happens before any launch;
+ *   a call that returns an error has launched nothing, except LOSA_ERR_CUDA
+ *   after a failed launch.
+ * - Element types: LOSA_BF16 (bfloat16) or LOSA_F32 (float) for Q, K, V and
+ *   the page metadata; the cached prefix state, the outputs and all
+ *   accumulation are fp32.
+ * - Sizes:  S sequences, Hq query heads, Hkv KV heads (G = Hq / Hkv query
+ *   heads share KV head g = h / G), d = head_dim, L = prefix_len,
+ *   ps = page_size, P = ceil(L / ps) pages (the last may be partial),
+ *   B = block_size, A = n_active, k = min(token_budget / ps, P).
+ */
+#ifndef LOSA_H_
+#define LOSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ----------------------------------------------------- */
+#define LOSA_OK                 0
+#define LOSA_ERR_INVALID_ARG    1  /* null/misaligned pointer, inconsistent sizes      */
+#define LOSA_ERR_UNSUPPORTED    2  /* valid but outside what the kernels implement     */
+#define LOSA_ERR_CUDA           3  /* a CUDA launch failed (message: losa_last_error)  */
+#define LOSA_ERR_DEVICE_TIMEOUT 4  /* a bounded device-side wait gave up               */
+#define LOSA_ERR_DEVICE_BOUNDS  5  /* a device-side index check failed (access skipped)*/
+
+/* ---- element types ---------------------------------------------------- */
+#define LOSA_F32  0
+#define LOSA_BF16 1
+
+/* ---- workspace kinds -------------------------------------------------- */
+#define LOSA_WS_DENSE 0
+#define LOSA_WS_STEP  1
+
+/* Problem shape shared by every call.  Limits checked by the library:
+ * head_dim == 128, page_size == 16 (LOSA_ERR_UNSUPPORTED otherwise);
+ * 1 <= block_size <= 32; G * block_size <= 128; 0 <= n_active <= block_size;
+ * n_active > 0 needs k >= 1; k <= 64 unless k == P (every page selected). */
+typedef struct {
+    int32_t num_seqs;      /* S                                           */
+    int32_t n_q_heads;     /* Hq                                          */
+    int32_t n_kv_heads;    /* Hkv, Hq % Hkv == 0                          */
+    int32_t head_dim;      /* d                                           */
+    int32_t prefix_len;    /* L >= 1                                      */
+    int32_t page_size;     /* ps                                          */
+    int32_t block_size;    /* B                                           */
+    int32_t n_active;      /* |A| per query head                          */
+    int32_t token_budget;  /* prefix tokens each active query may attend  */
+    float   scale;         /* softmax scale; 0 selects 1/sqrt(d)          */
+    int32_t dtype;         /* LOSA_F32 or LOSA_BF16                       */
+} losa_shape;
+
+/* Bytes of page metadata for `shape` (the size of `page_meta` below). */
+size_t losa_page_meta_size(const losa_shape* shape);
+
+/* Bytes of workspace needed by losa_dense_prefix (which = LOSA_WS_DENSE) or
+ * losa_step (LOSA_WS_STEP).  0 for an invalid shape. */
+size_t losa_workspace_size(const losa_shape* shape, int which);
+
+/*
+ * Page metadata build (once per prefix): for every page and channel, the min
+ * and max of the keys of the page's valid tokens -- what the QUEST bound
+ * needs (paper, methodology: QUEST-style page selection over KV pages).
+ *
+ *   k_prefix   [S][Hkv][L][d]   keys, element type `dtype`
+ *   page_meta  out, losa_page_meta_size() bytes, element type `dtype`:
+ *              for page p of (s, g), a record of 2*d elements -- kmin[0..d)
+ *              then kmax[0..d) -- at record index (s*Hkv + g)*P + p.  Inside
+ *              a record the 16-byte chunks are stored XOR-swizzled: logical
+ *              chunk c sits at chunk position c ^ (p & 7).  (This keeps the
+ *              scoring kernel's shared-memory reads free of bank conflicts.)
+ * Min/max introduce no rounding: the values are exact copies of key values.
+ */
+int losa_build_page_meta(const losa_shape* shape, const void* k_prefix, void* page_meta,
+                         void* stream);
+
+/*
+ * Cold-start dense pass (first denoising step of a block; paper,
+ * limitations): every block token attends to the whole prefix, which fills
+ * the cached prefix state of every row; then dense suffix attention over the
+ * block and the log-sum-exp merge give the step output.
+ *
+ *   q          [S][Hq][B][d]    queries of this step
+ *   k_prefix,
+ *   v_prefix   [S][Hkv][L][d]
+ *   k_blk,
+ *   v_blk      [S][Hkv][B][d]   the block's own keys/values
+ *   o_p        out [S][Hq][B][d] fp32  prefix output, all rows
+ *   l_p        out [S][Hq][B]    fp32  prefix log-normaliser (natural log)
+ *   out        out [S][Hq][B][d] fp32  attention over prefix + block
+ *   out_lse    out [S][Hq][B]    fp32  its log-normaliser; may be NULL
+ *   workspace  >= losa_workspace_size(shape, LOSA_WS_DENSE) bytes, 256-byte
+ *              aligned; contents on entry are irrelevant.
+ */
+int losa_dense_prefix(const losa_shape* shape, const void* q, const void* k_prefix,
+                      const void* v_prefix, const void* k_blk, const void* v_blk, float* o_p,
+                      float* l_p, float* out, float* out_lse, void* workspace, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * One LoSA denoising step (steps 2..T of a block; paper, methodology).
+ *
+ *   q_cur      [S][Hq][B][d]    this step's queries
+ *   q_prev     [S][Hq][B][d]    the previous step's queries (caller rotates)
+ *   k_prefix,
+ *   v_prefix   [S][Hkv][L][d]
+ *   page_meta  from losa_build_page_meta on the same k_prefix
+ *   k_blk,
+ *   v_blk      [S][Hkv][B][d]
+ *   o_p, l_p   in/out cached prefix state [S][Hq][B][d], [S][Hq][B] fp32:
+ *              rows of active tokens are overwritten with their sparse
+ *              prefix result; rows of stable tokens are not written at all.
+ *   out        out [S][Hq][B][d] fp32; must not alias any input
+ *   out_lse    out [S][Hq][B] fp32; may be NULL
+ *   active_idx optional out [S][Hq][A] int32: active tokens, ascending
+ *   page_idx   optional out [S][Hq][A][k] int32: each active row's pages,
+ *              ascending
+ *   union_count optional out [S][Hkv] int32: distinct pages loaded per
+ *              (sequence, KV head) -- the union over its G*A active rows
+ *   workspace  >= losa_workspace_size(shape, LOSA_WS_STEP) bytes, 256-byte
+ *              aligned; contents on entry are irrelevant.
+ * Selection rules: the active set is the top-A tokens by MSE (fp32, channels
+ * summed in order), ties to the lower token index; pages are the top-k by the
+ * bound (ties to the lower page index, -0 == +0).  n_active == 0 is legal
+ * (every row reuses its cache); n_active == B with k == P equals dense
+ * attention.
+ */
+int losa_step(const losa_shape* shape, const void* q_cur, const void* q_prev,
+              const void* k_prefix, const void* v_prefix, const void* page_meta,
+              const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
+              float* out_lse, int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
+              void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the device-side status recorded in the
+ * workspace by the last call that used it (LOSA_OK, LOSA_ERR_DEVICE_TIMEOUT
+ * or LOSA_ERR_DEVICE_BOUNDS) and clears it.  LOSA_ERR_CUDA if the copy
+ * fails. */
+int losa_read_device_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* losa_status_string(int status);
+
+/* Message of the last LOSA_ERR_CUDA on the calling thread ("" if none). */
+const char* losa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOSA_H_ */

@@ -1,0 +1,156 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every symbol the
+header declares, and its host-side validation returns the documented codes
+before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_long_context_mse_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "losa.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return api.lib()
+
+
+def header_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(losa_[a-z_]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = header_functions()
+    assert set(declared) == set(api.EXPORTS)
+    for name in declared:
+        assert hasattr(L, name), name
+    nm = subprocess.run(["nm", "-D", "--defined-only", api.LIB_PATH], capture_output=True,
+                        text=True).stdout
+    for name in declared:
+        assert re.search(rf"\bT {name}\b", nm), f"{name} not exported"
+
+
+def test_library_is_sm100a_only():
+    # the build targets sm_100a only (no other SASS, no PTX for JIT)
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH)
+
+
+def S(**kw):
+    base = dict(num_seqs=1, n_q_heads=32, n_kv_heads=8, head_dim=128, prefix_len=65536,
+                page_size=16, block_size=16, n_active=4, token_budget=128, dtype="bf16")
+    base.update(kw)
+    return api.make_shape(**base)
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert api.status_string(code)
+    assert api.status_string(99) == "unknown status"
+
+
+def test_sizes(L):
+    sh = S()
+    P = 4096
+    assert api.page_meta_size(sh) == 8 * P * 2 * 128 * 2
+    assert api.page_meta_size(S(dtype="f32")) == 8 * P * 2 * 128 * 4
+    assert api.page_meta_size(S(prefix_len=65537)) == 8 * (P + 1) * 2 * 128 * 2
+    for which in (api.LOSA_WS_DENSE, api.LOSA_WS_STEP):
+        n = api.workspace_size(sh, which)
+        assert n > 0 and n % 256 == 0
+    assert api.workspace_size(sh, 7) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_q_heads=30), api.LOSA_ERR_INVALID_ARG),          # Hq % Hkv != 0
+    (dict(n_active=17), api.LOSA_ERR_INVALID_ARG),           # |A| > B
+    (dict(n_active=-1), api.LOSA_ERR_INVALID_ARG),
+    (dict(prefix_len=0), api.LOSA_ERR_INVALID_ARG),
+    (dict(token_budget=8), api.LOSA_ERR_INVALID_ARG),         # k = 0 with |A| > 0
+    (dict(scale=-1.0), api.LOSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), api.LOSA_ERR_INVALID_ARG),
+    (dict(head_dim=64), api.LOSA_ERR_UNSUPPORTED),
+    (dict(page_size=32), api.LOSA_ERR_UNSUPPORTED),
+    (dict(dtype=7), api.LOSA_ERR_UNSUPPORTED),
+    (dict(block_size=64, n_active=4), api.LOSA_ERR_UNSUPPORTED),   # B > 32
+    (dict(n_q_heads=64, n_kv_heads=2, block_size=8), api.LOSA_ERR_UNSUPPORTED),  # G*B > 128
+    (dict(token_budget=16 * 65), api.LOSA_ERR_UNSUPPORTED),  # 64 < k < P
+])
+def test_shape_validation(L, kw, code):
+    if kw.get("dtype") == 7:
+        sh = S()
+        sh.dtype = 7
+    else:
+        sh = S(**kw)
+    assert api.workspace_size(sh, api.LOSA_WS_STEP) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    rc = L.losa_step(ctypes.byref(sh), *([fake] * 10), None, None, None, None, fake,
+                     1 << 40, None)
+    assert rc == code
+    rc = L.losa_build_page_meta(ctypes.byref(sh), fake, ctypes.c_void_p(1 << 30), None)
+    assert rc == code
+
+
+def test_legal_edge_shapes_size(L):
+    # |A| = 0 with a zero budget, and k == P beyond 64 (every page), are legal
+    assert api.workspace_size(S(n_active=0, token_budget=0), api.LOSA_WS_STEP) > 0
+    assert api.workspace_size(S(prefix_len=4096, token_budget=4096), api.LOSA_WS_STEP) > 0
+    assert api.workspace_size(S(n_q_heads=8, n_kv_heads=1, block_size=16, n_active=16),
+                              api.LOSA_WS_STEP) > 0
+
+
+def _step_args(ptrs):
+    return [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
+
+
+def test_pointer_validation(L):
+    sh = S()
+    ws_n = api.workspace_size(sh, api.LOSA_WS_STEP)
+    base = [0x100000 * (i + 1) for i in range(10)] + [None, None, None, None, 0x7f0000000000]
+
+    def call(ptrs, ws_bytes=ws_n):
+        return L.losa_step(ctypes.byref(sh), *_step_args(ptrs), ws_bytes, None)
+
+    for i in range(10):  # each required pointer: null, then misaligned
+        p = list(base)
+        p[i] = None
+        assert call(p) == api.LOSA_ERR_INVALID_ARG
+        p[i] = base[i] + 8
+        assert call(p) == api.LOSA_ERR_INVALID_ARG
+    p = list(base)
+    p[14] = base[14] + 128               # workspace not 256-byte aligned
+    assert call(p) == api.LOSA_ERR_INVALID_ARG
+    assert call(base, ws_n - 1) == api.LOSA_ERR_INVALID_ARG   # workspace too small
+    p = list(base)
+    p[11] = 0x900004                     # optional output misaligned
+    assert call(p) == api.LOSA_ERR_INVALID_ARG
+    p = list(base)
+    p[9] = p[0]                          # out aliases q_cur
+    assert call(p) == api.LOSA_ERR_INVALID_ARG
+    assert L.losa_step(None, *_step_args(base), ws_n, None) == api.LOSA_ERR_INVALID_ARG
+
+
+def test_dense_pointer_validation(L):
+    sh = S()
+    ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)
+    base = [0x100000 * (i + 1) for i in range(9)] + [0x7f0000000000]
+    for i in range(8):
+        p = list(base)
+        p[i] = None
+        rc = L.losa_dense_prefix(ctypes.byref(sh), *_step_args(p), ws_n, None)
+        assert rc == api.LOSA_ERR_INVALID_ARG
+    rc = L.losa_dense_prefix(ctypes.byref(sh), *_step_args(base), ws_n - 256, None)
+    assert rc == api.LOSA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        api.lib()
