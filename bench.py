@@ -273,13 +273,16 @@ def run_losa(args):
     warm_replays = max(3, -(-args.warmup // per_replay))
     replays = max(1, -(-args.steps // per_replay))
     steps_timed = replays * per_replay
-    for _ in range(warm_replays):
-        graph.replay()
+    # graph.replay() launches on the current stream: keep it `stream`, the
+    # stream the events are recorded on
+    with torch.cuda.stream(stream):
+        for _ in range(warm_replays):
+            graph.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
         ev0.record(stream)
         for _ in range(replays):
             graph.replay()
@@ -349,14 +352,15 @@ def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):
         stream.synchronize()
         with torch.cuda.graph(g, stream=stream):
             fn()
-        for _ in range(2):
-            g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
         torch.cuda.synchronize()
         ms = max_over_ranks(e0.elapsed_time(e1), world) / reps
         del g

@@ -19,7 +19,6 @@ constexpr int kMaxB = 32;       // block tokens (one warp lane per token)
 constexpr int kMaxRowsPerGroup = 128;  // G*B (and hence G*A) per KV head
 constexpr int kMaxK = 64;       // pages per active row unless every page is taken
 constexpr int kPartStride = kD + 4;    // floats per split-softmax partial: m, l, pad, pad, acc[d]
-constexpr size_t kMaxDynSmem = 227 * 1024;  // opt-in shared memory per CTA (sm_100)
 constexpr int kMaxDevices = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

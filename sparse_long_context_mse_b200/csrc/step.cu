@@ -439,7 +439,9 @@ __global__ void __launch_bounds__(128)
 // Raises the dynamic shared-memory limit of the kernels that need more than
 // 48 KB, once per device (the first call on a device should come before any
 // stream capture).
-int set_kernel_attributes() {
+int g_max_dyn[kMaxDevices] = {};  // smallest dynamic-smem limit granted, per device
+
+int set_kernel_attributes(size_t* max_dyn) {
   static std::mutex mu;
   static bool done[kMaxDevices] = {};
   int dev = 0;
@@ -447,16 +449,27 @@ int set_kernel_attributes() {
   if (e != cudaSuccess) return record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return LOSA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(mu);
-  if (done[dev]) return LOSA_OK;
+  if (done[dev]) {
+    *max_dyn = static_cast<size_t>(g_max_dyn[dev]);
+    return LOSA_OK;
+  }
   const void* fns[] = {reinterpret_cast<const void*>(score_kernel),
                        reinterpret_cast<const void*>(select_kernel),
                        reinterpret_cast<const void*>(gather_kernel)};
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return record_cuda_error(e);
   for (const void* f : fns) {
-    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kMaxDynSmem));
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, f);
     if (e != cudaSuccess) return record_cuda_error(e);
+    const int dyn = optin - static_cast<int>(fa.sharedSizeBytes);
+    e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    g_max_dyn[dev] = dyn < g_max_dyn[dev] || g_max_dyn[dev] == 0 ? dyn : g_max_dyn[dev];
   }
   done[dev] = true;
+  *max_dyn = static_cast<size_t>(g_max_dyn[dev]);
   return LOSA_OK;
 }
 
@@ -497,23 +510,24 @@ extern "C" int losa_step(const losa_shape* shape, const void* q_cur, const void*
   int32_t* ucount = reinterpret_cast<int32_t*>(ws + d.off_ucount);
   float* part = reinterpret_cast<float*>(ws + d.off_part);
 
-  rc = set_kernel_attributes();
+  size_t max_dyn = 0;
+  rc = set_kernel_attributes(&max_dyn);
   if (rc != LOSA_OK) return rc;
+  // every limit is checked before the first launch
+  const size_t smem_score = static_cast<size_t>(d.R) * (kD + kScoreThreads) * sizeof(float);
+  const size_t smem_sel = 2 * static_cast<size_t>((d.P + 31) / 32) * sizeof(uint32_t);
+  const size_t smem_g = static_cast<size_t>(kGatherWarps) * 2 * kPS * kD * sizeof(float);
+  const int ublocks = (d.Umax + kGatherWarps - 1) / kGatherWarps;
+  if (smem_score > max_dyn || smem_sel > max_dyn || smem_g > max_dyn || ublocks > 65535)
+    return LOSA_ERR_UNSUPPORTED;
+
   active_kernel<<<d.S * d.Hq, 128, 0, st>>>(q_cur, q_prev, act_tok, act_slot, active_idx, d);
   if (d.A > 0) {
-    if (!d.all_pages) {
-      const size_t smem = static_cast<size_t>(d.R) * (kD + kScoreThreads) * sizeof(float);
-      if (smem > kMaxDynSmem) return LOSA_ERR_UNSUPPORTED;
-      score_kernel<<<dim3(d.nchunk, d.S * d.Hkv), kScoreThreads, smem, st>>>(q_cur, page_meta,
-                                                                             act_tok, cand, d);
-    }
-    const size_t smem_sel = 2 * static_cast<size_t>((d.P + 31) / 32) * sizeof(uint32_t);
-    if (smem_sel > kMaxDynSmem) return LOSA_ERR_UNSUPPORTED;
+    if (!d.all_pages)
+      score_kernel<<<dim3(d.nchunk, d.S * d.Hkv), kScoreThreads, smem_score, st>>>(
+          q_cur, page_meta, act_tok, cand, d);
     select_kernel<<<d.S * d.Hkv, kSelectThreads, smem_sel, st>>>(
         cand, sel, uni, umask, ucount, page_idx, union_count, d, status);
-    const int ublocks = (d.Umax + kGatherWarps - 1) / kGatherWarps;
-    if (ublocks > 65535) return LOSA_ERR_UNSUPPORTED;
-    const size_t smem_g = static_cast<size_t>(kGatherWarps) * 2 * kPS * kD * sizeof(float);
     gather_kernel<<<dim3(d.S * d.Hkv, ublocks), kGatherWarps * 32, smem_g, st>>>(
         q_cur, k_prefix, v_prefix, act_tok, sel, uni, umask, ucount, part, d, status);
   } else if (union_count) {
