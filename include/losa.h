@@ -28,7 +28,8 @@
  * - All tensor pointers are DEVICE pointers owned by the caller, contiguous
  *   in the row-major layouts given below (innermost index last), 16-byte
  *   aligned.  The library never allocates or frees memory and keeps no state
- *   between calls; the workspace is caller-owned scratch.
+ *   between calls; the workspace is caller-owned scratch (losa_step_noalloc
+ *   alone uses a fixed array owned by the library instead).
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *   legacy default stream).  Host-side validation happens before any launch;
  *   a call that returns an error has launched nothing, except LOSA_ERR_CUDA
@@ -165,6 +166,40 @@ int losa_step(const losa_shape* shape, const void* q_cur, const void* q_prev,
               const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
               float* out_lse, int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
               void* workspace, size_t ws_bytes, void* stream);
+
+/* Size of the scratch array behind losa_step_noalloc: 8 MiB per GPU. */
+#define LOSA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/*
+ * losa_step for callers that cannot allocate device memory.  The paper has
+ * no counterpart to this entry point; it exists for callers such as a plugin
+ * inside a host framework whose caching allocator already owns the GPU's
+ * memory (where a raw cudaMalloc fails or fragments that pool), or a
+ * latency-critical loop that must not call cudaMalloc/cudaFree because they
+ * can synchronise the device.
+ *
+ * Same arguments and results as losa_step, minus `workspace`/`ws_bytes`: the
+ * scratch is a LOSA_NOALLOC_SCRATCH_BYTES array in device global memory that
+ * belongs to this library.  Every GPU that loads the library holds that
+ * array until the process exits.  This function itself allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).
+ *  - Shapes whose losa_workspace_size(shape, LOSA_WS_STEP) exceeds
+ *    LOSA_NOALLOC_SCRATCH_BYTES are rejected with LOSA_ERR_UNSUPPORTED before
+ *    anything is launched.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture on that device.
+ *  - All calls on a device share the one array, which keeps whatever the
+ *    last call left in it (losa_step needs nothing there to start at zero).
+ *    Calls that can overlap on the GPU -- on different streams without an
+ *    ordering between them -- race on the array and give wrong results;
+ *    order them on one stream or with events.
+ */
+int losa_step_noalloc(const losa_shape* shape, const void* q_cur, const void* q_prev,
+                      const void* k_prefix, const void* v_prefix, const void* page_meta,
+                      const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
+                      float* out_lse, int32_t* active_idx, int32_t* page_idx,
+                      int32_t* union_count, void* stream);
 
 /* Synchronises `stream`, then returns the device-side status recorded in the
  * workspace by the last call that used it (LOSA_OK, LOSA_ERR_DEVICE_TIMEOUT

@@ -30,8 +30,11 @@ LOSA_WS_STEP = 1
 
 #: every symbol ``include/losa.h`` declares
 EXPORTS = ("losa_page_meta_size", "losa_workspace_size", "losa_build_page_meta",
-           "losa_dense_prefix", "losa_step", "losa_read_device_status", "losa_status_string",
-           "losa_last_error")
+           "losa_dense_prefix", "losa_step", "losa_step_noalloc", "losa_read_device_status",
+           "losa_status_string", "losa_last_error")
+
+#: size of the library-owned scratch behind ``losa_step_noalloc``
+NOALLOC_SCRATCH_BYTES = 8 * 1024 * 1024
 
 
 class LosaError(RuntimeError):
@@ -105,6 +108,8 @@ def lib():
         L.losa_dense_prefix.restype = i32
         L.losa_step.argtypes = [sp] + [vp] * 14 + [vp, sz, vp]
         L.losa_step.restype = i32
+        L.losa_step_noalloc.argtypes = [sp] + [vp] * 14 + [vp]
+        L.losa_step_noalloc.restype = i32
         L.losa_read_device_status.argtypes = [vp, vp]
         L.losa_read_device_status.restype = i32
         L.losa_status_string.argtypes = [i32]
@@ -223,6 +228,33 @@ def step(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, 
             _ptr(union_count, (sh.num_seqs, sh.n_kv_heads), torch.int32, "union_count", dev),
             _ptr(workspace, None, torch.uint8, "workspace", dev)]
     _check(lib().losa_step(ctypes.byref(sh), *args, workspace.numel(), _stream(stream)))
+
+
+def step_noalloc(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
+                 l_p, out, out_lse, active_idx=None, page_idx=None, union_count=None,
+                 stream=None):
+    """``losa_step_noalloc``: one step without a caller workspace, for callers
+    that cannot allocate device memory (the library's own fixed scratch array
+    is used; shapes needing more than ``NOALLOC_SCRATCH_BYTES`` are refused).
+    Calls that may overlap on the GPU race on that array."""
+    dev = _device_of(q_cur)
+    dt = sh.torch_dtype
+    qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.prefix_len, sh.head_dim)
+    kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
+    rs = qs[:3]
+    A, k = sh.n_active, sh.pages_per_row
+    args = [_ptr(q_cur, qs, dt, "q_cur", dev), _ptr(q_prev, qs, dt, "q_prev", dev),
+            _ptr(k_prefix, kv, dt, "k_prefix", dev), _ptr(v_prefix, kv, dt, "v_prefix", dev),
+            _ptr(page_meta, (page_meta_size(sh),), torch.uint8, "page_meta", dev),
+            _ptr(k_blk, kb, dt, "k_blk", dev), _ptr(v_blk, kb, dt, "v_blk", dev),
+            _ptr(o_p, qs, torch.float32, "o_p", dev), _ptr(l_p, rs, torch.float32, "l_p", dev),
+            _ptr(out, qs, torch.float32, "out", dev),
+            _ptr(out_lse, rs, torch.float32, "out_lse", dev),
+            _ptr(active_idx, (sh.num_seqs, sh.n_q_heads, A), torch.int32, "active_idx", dev),
+            _ptr(page_idx, (sh.num_seqs, sh.n_q_heads, A, k), torch.int32, "page_idx", dev),
+            _ptr(union_count, (sh.num_seqs, sh.n_kv_heads), torch.int32, "union_count", dev)]
+    _check(lib().losa_step_noalloc(ctypes.byref(sh), *args, _stream(stream)))
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
