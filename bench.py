@@ -188,10 +188,8 @@ def step_bytes(sh, union_counts, esz):
 
 
 def launches_per_step(sh):
-    """Kernels one losa_step launches (mirrors the library's launch sequence)."""
-    if sh.n_active == 0:
-        return 2
-    return 5 if sh.pages_per_row < sh.n_pages else 4
+    """Kernels one losa_step launches: the fused step is a single launch."""
+    return 1
 
 
 # ---------------------------------------------------------------------------

@@ -85,26 +85,14 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
     return LOSA_OK;
   }
   if (which != LOSA_WS_STEP) return LOSA_ERR_INVALID_ARG;
-  d->chunk_pages = 128;
-  d->nchunk = (d->P + d->chunk_pages - 1) / d->chunk_pages;
+  // step: status word + one online-softmax partial per (group, active row,
+  // selected page)
   const size_t R = static_cast<size_t>(d->R), K = static_cast<size_t>(d->k);
-  d->off_act_tok = off;
-  off += align256(static_cast<size_t>(d->S) * d->Hq * d->A * sizeof(int32_t));
-  d->off_act_slot = off;
-  off += align256(static_cast<size_t>(d->S) * d->Hq * d->B * sizeof(int32_t));
-  d->off_cand = off;
-  if (!d->all_pages) off += align256(SG * d->nchunk * R * K * sizeof(unsigned long long));
-  d->off_sel = off;
-  off += align256(SG * R * K * sizeof(int32_t));
-  d->off_union = off;
-  off += align256(SG * d->Umax * sizeof(int32_t));
-  d->off_mask = off;
-  off += align256(SG * d->Umax * d->MW * sizeof(uint32_t));
-  d->off_ucount = off;
-  off += align256(SG * sizeof(int32_t));
   d->off_part = off;
   off += align256(SG * R * K * kPartStride * sizeof(float));
   d->total = off;
+  // the fused step keeps each group's selection state in shared memory
+  if (!fused_step_fits(*d, kB200MaxDynSmem)) return LOSA_ERR_UNSUPPORTED;
   return LOSA_OK;
 }
 

@@ -31,12 +31,10 @@ struct Dims {
   int all_pages;          // k == P: every page is selected, no scoring needed
   float scale;            // softmax scale (natural-log units)
   float scale_log2;       // scale * log2(e): scores in base-2 units
-  // scoring chunks (step) / prefix splits (dense)
-  int nchunk, chunk_pages;
+  // prefix splits (dense)
   int nsplit, split_pages;
   // workspace byte offsets
-  size_t off_status, off_act_tok, off_act_slot, off_cand, off_sel, off_union, off_mask,
-      off_ucount, off_part, total;
+  size_t off_status, off_part, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).
@@ -215,6 +213,16 @@ inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 }
 
 int make_dims(const losa_shape* sh, int which, Dims* d);
+// Whether the fused step kernel's shared-memory plan fits in `max_dyn` bytes.
+bool fused_step_fits(const Dims& d, int max_dyn);
+// Dynamic shared memory a B200 CTA may opt in to (227 KB).
+constexpr int kB200MaxDynSmem = 232448;
+// The fused step kernel (step_fused.cu); arguments already validated.
+int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
+                      const void* v_prefix, const void* page_meta, const void* k_blk,
+                      const void* v_blk, float* o_p, float* l_p, float* out, float* out_lse,
+                      int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
+                      void* workspace, cudaStream_t st);
 int record_cuda_error(cudaError_t e);  // stores the message, returns LOSA_ERR_CUDA
 int num_sms();
 

@@ -101,8 +101,12 @@ def test_legal_edge_shapes_size(L):
     # |A| = 0 with a zero budget, and k == P beyond 64 (every page), are legal
     assert api.workspace_size(S(n_active=0, token_budget=0), api.LOSA_WS_STEP) > 0
     assert api.workspace_size(S(prefix_len=4096, token_budget=4096), api.LOSA_WS_STEP) > 0
+    assert api.workspace_size(S(n_q_heads=8, n_kv_heads=1, block_size=16, n_active=16,
+                                prefix_len=3000), api.LOSA_WS_STEP) > 0
+    # 128 active rows per KV head over a 64K prefix: the per-group selection
+    # state no longer fits in one CTA's shared memory
     assert api.workspace_size(S(n_q_heads=8, n_kv_heads=1, block_size=16, n_active=16),
-                              api.LOSA_WS_STEP) > 0
+                              api.LOSA_WS_STEP) == 0
 
 
 def _step_args(ptrs):
