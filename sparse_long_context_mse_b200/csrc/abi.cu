@@ -1,5 +1,6 @@
 // abi.cu -- host side of the C ABI: shape validation, workspace layout,
 // status reporting.  No kernel lives here.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <string>
@@ -85,11 +86,24 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
     return LOSA_OK;
   }
   if (which != LOSA_WS_STEP) return LOSA_ERR_INVALID_ARG;
-  // step: status word + one online-softmax partial per (group, active row,
-  // selected page)
+  // step: the scan splits each group's pages into chunks so that the whole
+  // grid covers the SMs once; a chunk's bound scores live in shared memory
   const size_t R = static_cast<size_t>(d->R), K = static_cast<size_t>(d->k);
-  d->off_part = off;
-  off += align256(SG * R * K * kPartStride * sizeof(float));
+  {
+    const long long per_group = std::max<long long>(1, kSizingSms / static_cast<long long>(SG));
+    long long chunk = (P + per_group - 1) / per_group;
+    chunk = (chunk + 7) / 8 * 8;
+    const long long cap = std::max<long long>(8, (16384 / std::max(d->R, 1)) / 8 * 8);
+    chunk = std::min(chunk, cap);
+    d->chunk_pages = static_cast<int>(chunk);
+    d->nchunk = static_cast<int>((P + chunk - 1) / chunk);
+  }
+  // workspace: status word, the active tokens of every group, and the chunk
+  // candidates (selection keys) of every (group, chunk, active row)
+  d->off_act = off;
+  off += align256(SG * R * sizeof(int32_t));
+  d->off_cand = off;
+  off += align256(SG * d->nchunk * R * K * sizeof(unsigned long long));
   d->total = off;
   // the fused step keeps each group's selection state in shared memory
   if (!fused_step_fits(*d, kB200MaxDynSmem)) return LOSA_ERR_UNSUPPORTED;

@@ -31,10 +31,11 @@ struct Dims {
   int all_pages;          // k == P: every page is selected, no scoring needed
   float scale;            // softmax scale (natural-log units)
   float scale_log2;       // scale * log2(e): scores in base-2 units
-  // prefix splits (dense)
+  // prefix splits (dense pass); page chunks of the step's scan
   int nsplit, split_pages;
+  int nchunk, chunk_pages;
   // workspace byte offsets
-  size_t off_status, off_part, total;
+  size_t off_status, off_part, off_act, off_cand, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).

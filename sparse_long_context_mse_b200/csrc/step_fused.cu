@@ -1,4 +1,4 @@
-// step_fused.cu -- one LoSA denoising step as a single kernel launch.
+// step_fused.cu -- one LoSA denoising step in two kernel launches.
 //
 // LoSA paper, methodology: locality pruning (MSE of Q_t vs Q_{t-1}, top-|A|
 // per head), reuse of the cached prefix state for stable tokens, QUEST page
@@ -6,37 +6,33 @@
 // prefix attention, dense intra-block suffix, online-softmax merge, cache
 // update.
 //
-// One thread-block cluster of CL CTAs serves one (sequence, KV head) group;
-// CTA `rank` of the cluster owns pages [rank*chunk, (rank+1)*chunk) of the
-// group's prefix.  Phases (one CTA's view):
-//
-//   P0  issue bulk (TMA) copies of this CTA's page-metadata chunk into a
-//       shared-memory ring; meanwhile compute the group's active set (every
-//       CTA computes it, identically), the suffix of the stable rows this CTA
-//       owns (written out at once) and of its active rows (kept in smem);
-//   P1  QUEST bound of every page of the chunk for the group's R active rows:
-//       bf16 -- tensor cores, U = [q-|q+] . [kmin;kmax] (mma.sync m16n8k16,
-//       exact products, fp32 accumulation); fp32 -- CUDA cores, the sum in
-//       channel order with one rounding per operation;
-//   P2  chunk-local top-k per row (selection keys: score, then lower page);
-//   --  cluster barrier
-//   P3  rows are dealt to CTAs (r % CL); each merges its rows' CL candidate
-//       lists through distributed shared memory into the row's top-k pages;
-//   --  cluster barrier
-//   P4  every CTA reads all rows' page lists, builds the group's union
-//       (bitmap, ascending) and the row mask of each union page; union slot u
-//       belongs to CTA u % CL;
-//   P5  each CTA bulk-copies its union pages' K and V (each page read once
-//       for the whole GQA group) and writes an online-softmax partial
-//       (m, l, acc) for every row whose mask holds the page;
-//   --  cluster barrier
-//   P6  each CTA combines the partials of its active rows, writes their new
-//       o_p / L_p to the cache and merges them with their suffix.
+// K1 `losa_scan_kernel` -- a flat grid over every SM: each CTA owns one chunk
+//    of one (sequence, KV head) group's pages.  It bulk-copies (TMA) the
+//    chunk's page metadata into a shared-memory ring and meanwhile computes
+//    the group's active set (every CTA of the group computes it, identically)
+//    and finishes its share of the group's stable rows (suffix attention over
+//    the block, merge with the untouched cache).  Then the QUEST bound of the
+//    chunk's pages for the group's R active rows -- bf16: tensor cores,
+//    U = [q- | q+] . [kmin ; kmax] with mma.sync m16n8k16 (exact products,
+//    fp32 accumulation); fp32: CUDA cores, the sum in channel order with one
+//    rounding per operation -- and a chunk-local top-k per row, written to the
+//    workspace.
+// K2 `losa_gather_kernel` -- one thread-block cluster per group, launched
+//    with programmatic dependent launch behind K1.  Rows are dealt to the
+//    cluster's CTAs; each merges its rows' chunk candidates into the row's
+//    top-k pages; every CTA then builds the group's page union (bitmap,
+//    ascending, with a row mask per page) from the rows' lists in
+//    distributed shared memory; union slot u belongs to CTA u % CL, which
+//    bulk-copies the page's K and V once for the whole GQA group and folds
+//    the page into an online-softmax partial per row; finally each CTA
+//    combines its rows' partials from every CTA of the cluster (distributed
+//    shared memory), writes the new o_p / L_p to the cache and merges them
+//    with the suffix.
 //
 // Every wait on a bulk copy is bounded (clock64); a wait that gives up sets
-// LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA keeps going through
-// every cluster barrier without doing further work, so the cluster never
-// deadlocks.  There is no other cross-CTA wait.
+// LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA skips the rest of
+// its work but still takes part in every cluster barrier, so the cluster
+// never deadlocks.  There is no other cross-CTA wait.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -58,41 +54,7 @@ constexpr int kMaxStages = kMaxRingBytes / kStageBytes;
 constexpr int kCandCap = 64;                     // per-warp compaction buffer
 constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
 constexpr int kMaxCluster = 16;
-
-struct Layout {  // dynamic shared-memory byte offsets
-  int ring, scores, qrows, kbv, cand, sel_own, sel_all, bitmap, wbase, lpages, masks, sfx, cbuf,
-      ps, misc, mbar, total;
-};
-
-struct Params {
-  const void* qc;
-  const void* qp;
-  const void* K;
-  const void* V;
-  const char* meta;
-  const void* kb;
-  const void* vb;
-  float* o_p;
-  float* l_p;
-  float* out;
-  float* out_lse;
-  int32_t* active_idx;
-  int32_t* page_idx;
-  int32_t* union_count;
-  float* part;
-  int* status;
-  Dims d;
-  int CL;           // CTAs per cluster (per group)
-  int chunk;        // pages per CTA (multiple of 8)
-  int tile;         // pages per ring stage
-  int rec;          // bytes per metadata record
-  int sc_stride;    // floats per score row
-  int stages;       // metadata ring stages (ring = stages * 32 KiB)
-  int gslots;       // gather slots per gathering warp
-  int gwarps;       // warps that gather union pages
-  int max_lp;       // max union pages per CTA
-  Layout lo;
-};
+constexpr int kMaxGatherPages = 16;              // pages in flight per K2 CTA
 
 // ---------------------------------------------------------------------------
 // PTX wrappers: mbarrier, bulk copy, ldmatrix, mma
@@ -305,125 +267,260 @@ __device__ void warp_topk(KeyFn key, int n, int k, unsigned long long* out,
 }
 
 // ---------------------------------------------------------------------------
-// The kernel
+// Register top-k: KP (power of two) selection keys per thread, descending.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void cas_desc(unsigned long long& a, unsigned long long& b) {
+  const bool sw = a < b;
+  const unsigned long long hi = sw ? b : a, lo = sw ? a : b;
+  a = hi;
+  b = lo;
+}
+
+template <int KP>
+__device__ __forceinline__ void bitonic_sort_desc(unsigned long long (&x)[KP]) {
+#pragma unroll
+  for (int size = 2; size <= KP; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+      for (int i = 0; i < KP; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0) cas_desc(x[i], x[j]);
+          else cas_desc(x[j], x[i]);
+        }
+      }
+    }
+  }
+}
+
+// x <- the KP largest of x and y (both descending); result descending.  The
+// element-wise max of x and reversed y is bitonic and holds exactly the top
+// KP; half-cleaners sort it.
+template <int KP>
+__device__ __forceinline__ void merge_top(unsigned long long (&x)[KP],
+                                          const unsigned long long (&y)[KP]) {
+#pragma unroll
+  for (int i = 0; i < KP; ++i) x[i] = umax64(x[i], y[KP - 1 - i]);
+#pragma unroll
+  for (int stride = KP >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+      const int j = i ^ stride;
+      if (j > i) cas_desc(x[i], x[j]);
+    }
+  }
+}
+
+// Merge the lists of `width` consecutive lanes (power of two <= 32); every
+// lane of the group ends with the group's top KP.
+template <int KP>
+__device__ __forceinline__ void group_merge(unsigned long long (&x)[KP], int width) {
+  for (int off = 1; off < width; off <<= 1) {
+    unsigned long long y[KP];
+#pragma unroll
+    for (int i = 0; i < KP; ++i) y[i] = __shfl_xor_sync(0xffffffffu, x[i], off);
+    merge_top<KP>(x, y);
+  }
+}
+
+// Top-KP of the keys key(i), i = j, j + stride, j + 2*stride, ... < n, held by
+// one thread (descending, 0 = empty).
+template <int KP, typename KeyFn>
+__device__ __forceinline__ void thread_topk(KeyFn key, int j, int stride, int n,
+                                            unsigned long long (&x)[KP]) {
+#pragma unroll
+  for (int i = 0; i < KP; ++i) x[i] = 0ull;
+  for (int base = j; base < n; base += stride * KP) {
+    unsigned long long y[KP];
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+      const int idx = base + i * stride;
+      y[i] = idx < n ? key(idx) : 0ull;
+    }
+    bitonic_sort_desc<KP>(y);
+    merge_top<KP>(x, y);
+  }
+}
+
+int pow2_floor(int x) {
+  int p = 1;
+  while (p * 2 <= x) p *= 2;
+  return p;
+}
+int align_up(int x, int a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// K1: scan
+// ---------------------------------------------------------------------------
+struct ScanLayout {
+  int ring, scores, qrows, qstage, misc, ps, cbuf, mbar, total;
+};
+
+struct ScanParams {
+  const void* qc;
+  const void* qp;
+  const char* meta;
+  const void* kb;
+  const void* vb;
+  const float* o_p;
+  const float* l_p;
+  float* out;
+  float* out_lse;
+  int32_t* active_idx;
+  int32_t* union_count;
+  int32_t* act_tok_g;              // workspace [S*Hkv][R]
+  unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
+  int* status;
+  Dims d;
+  int rec;        // bytes per metadata record
+  int tile;       // pages per ring stage
+  int stages;     // ring stages
+  int sc_stride;  // floats per score row
+  int qw;         // 32-bit words per staged query row (padded)
+  int kp;         // register top-k width (2..16), 0 = warp fallback
+  int tpr;        // threads per row for the chunk top-k
+  ScanLayout lo;
+};
+
+template <int DT, int KP>
+__device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* sc, int R, int k,
+                                           int npages, int p0, unsigned long long* dst_base,
+                                           unsigned long long* cbuf) {
+  const int tid = threadIdx.x;
+  if (KP > 0) {
+    const int tpr = prm.tpr;
+    const int r = tid / tpr, j = tid % tpr;
+    const int rr = r < R ? r : 0;  // idle rows work on row 0 and write nothing
+    const float* row = sc + rr * prm.sc_stride;
+    unsigned long long x[KP > 0 ? KP : 1];
+    thread_topk<(KP > 0 ? KP : 1)>([&](int i) { return sel_key(row[i], p0 + i); }, j, tpr, npages,
+                                   x);
+    group_merge<(KP > 0 ? KP : 1)>(x, tpr);
+    if (r < R && j == 0) {
+      unsigned long long* dst = dst_base + static_cast<size_t>(r) * k;
+#pragma unroll
+      for (int i = 0; i < (KP > 0 ? KP : 1); ++i)
+        if (i < k) dst[i] = x[i];
+    }
+  } else {
+    const int warp = tid >> 5;
+    for (int r = warp; r < R; r += kWarps) {
+      const float* row = sc + r * prm.sc_stride;
+      warp_topk([&](int i) { return sel_key(row[i], p0 + i); }, npages, k,
+                cbuf + (kWarps + warp) * kCandCap, cbuf + warp * kCandCap);
+      __syncwarp();
+      const int lane = tid & 31;
+      for (int i = lane; i < k; i += 32)
+        dst_base[static_cast<size_t>(r) * k + i] = cbuf[(kWarps + warp) * kCandCap + i];
+      __syncwarp();
+    }
+  }
+}
+
 template <int DT>
-__global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm) {
+__global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams prm) {
   extern __shared__ __align__(1024) char smem[];
-  cg::cluster_group cluster = cg::this_cluster();
   const Dims& d = prm.d;
-  const Layout& lo = prm.lo;
+  const ScanLayout& lo = prm.lo;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int CL = prm.CL;
+  const int chunk = blockIdx.x, nchunk = gridDim.x;
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
   const int esz = DT == LOSA_BF16 ? 2 : 4;
+  const int GB = G * B;
+  const int Bpad = (B + kPS - 1) / kPS * kPS;
+  const int qw = prm.qw;
+
+  // let the gather kernel be scheduled as soon as resources free up; it
+  // waits for this grid's completion before reading anything written here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   char* ring = smem + lo.ring;
   float* sc = reinterpret_cast<float*>(smem + lo.scores);
+  char* kbv = smem + lo.scores;  // block K then V (element type); aliases sc
   char* qrows = smem + lo.qrows;
-  char* kbv = smem + lo.scores;  // [Bpad][kD] K then V, element type (aliases sc)
-  unsigned long long* cand = reinterpret_cast<unsigned long long*>(smem + lo.cand);
-  int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
-  int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel_all);
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + lo.bitmap);
-  int32_t* wbase = reinterpret_cast<int32_t*>(smem + lo.wbase);
-  int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
-  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
-  float* sfx = reinterpret_cast<float*>(smem + lo.sfx);
-  unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
-  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
+  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.qstage);  // [GB][qw]
+  uint32_t* qps = qcs + GB * qw;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
+  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
+  unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
-  // misc: [0] failed flag, [1] union size, [2] local pages, [3..3+kMaxB*? ) act
   int32_t* s_fail = misc;
-  int32_t* s_U = misc + 1;
-  int32_t* s_nlp = misc + 2;
-  float* s_mse = reinterpret_cast<float*>(misc + 4);   // [G*B]
-  int32_t* act_slot = misc + 4 + kMaxRowsPerGroup;     // [G*B] slot or -1
-  int32_t* act_tok = act_slot + kMaxRowsPerGroup;      // [G][A] -> [R]
+  float* s_mse = reinterpret_cast<float*>(misc + 4);
+  int32_t* act_slot = misc + 4 + kMaxRowsPerGroup;
+  int32_t* act_tok = act_slot + kMaxRowsPerGroup;
 
-  const int p0 = rank * prm.chunk;
-  const int npages = max(0, min(d.P, p0 + prm.chunk) - p0);
+  const int p0 = chunk * d.chunk_pages;
+  const int npages = max(0, min(d.P, p0 + d.chunk_pages) - p0);
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
-  const bool scan = A > 0 && !d.all_pages;
+  const bool scan = A > 0 && !d.all_pages && npages > 0;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.P * prm.rec;
+  // stable token-rows of the group handled here: i = chunk + n * nchunk
+  const int n_stable_mine = GB > chunk ? (GB - chunk + nchunk - 1) / nchunk : 0;
+  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
 
-  // ---- P0: barriers, first metadata copies --------------------------------
   if (tid == 0) {
-    for (int i = 0; i < kMaxStages + kWarps * 2; ++i) mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-  }
-  __syncthreads();
-  if (tid == 0 && scan) {
-    for (int t = 0; t < min(ntiles, prm.stages); ++t) {
-      const int np = min(prm.tile, npages - t * prm.tile);
-      const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
-      mbar_expect_tx(&mbar[t], bytes);
-      bulk_g2s(ring + t * kStageBytes, meta_g + static_cast<size_t>(p0 + t * prm.tile) * prm.rec,
-               bytes, &mbar[t]);
+    if (scan) {
+      for (int t = 0; t < min(ntiles, prm.stages); ++t) {
+        const int np = min(prm.tile, npages - t * prm.tile);
+        const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
+        mbar_expect_tx(&mbar[t], bytes);
+        bulk_g2s(ring + t * kStageBytes,
+                 meta_g + static_cast<size_t>(p0 + t * prm.tile) * prm.rec, bytes, &mbar[t]);
+      }
+    }
+    if (n_stable_mine > 0) {  // the block's own K/V for the suffix
+      mbar_expect_tx(&mbar[kMaxStages], 2 * blk_bytes);
+      const size_t off = static_cast<size_t>(sg) * B * kD * esz;
+      bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxStages]);
+      bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
+               &mbar[kMaxStages]);
     }
   }
 
-  // ---- P0: locality score and active set (every CTA, identical) -----------
-  const int GB = G * B;
+  // ---- stage the group's current / previous queries (coalesced), padded
+  // rows so that one thread walking its row in channel order hits every bank
+  {
+    const int cpr = kD * esz / 16;  // 16-byte chunks per row
+    const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
+    const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
+    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + base);
+    for (int e = tid; e < GB * cpr; e += kThreads) {
+      const int row = e / cpr, c = e % cpr;
+      const uint4 a = gc[e], b = gp[e];
+      uint32_t* x = qcs + row * qw + 4 * c;
+      uint32_t* y = qps + row * qw + 4 * c;
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
+    }
+  }
+  __syncthreads();
+
+  // ---- locality score: fp32, one rounding per operation, channels in order
   if (tid < GB) {
-    const int hl = tid / B, t = tid % B;
-    const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
+    const uint32_t* x = qcs + tid * qw;
+    const uint32_t* y = qps + tid * qw;
     float acc = 0.f;
     if (DT == LOSA_BF16) {
-      const uint4* a4 = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + row * kD * 2);
-      const uint4* b4 = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + row * kD * 2);
-#pragma unroll 4
-      for (int c = 0; c < kD / 8; ++c) {
-        const uint4 x = a4[c], y = b4[c];
-        const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float d0 = __fsub_rn(__uint_as_float(xs[u] << 16), __uint_as_float(ys[u] << 16));
-          acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-          const float d1 = __fsub_rn(__uint_as_float(xs[u] & 0xffff0000u),
-                                     __uint_as_float(ys[u] & 0xffff0000u));
-          acc = __fadd_rn(acc, __fmul_rn(d1, d1));
-        }
+      for (int w = 0; w < kD / 2; ++w) {
+        const uint32_t a = x[w], b = y[w];
+        const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
+        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
+        const float d1 = __fsub_rn(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u));
+        acc = __fadd_rn(acc, __fmul_rn(d1, d1));
       }
     } else {
-      const float4* a4 = reinterpret_cast<const float4*>(static_cast<const float*>(prm.qc) + row * kD);
-      const float4* b4 = reinterpret_cast<const float4*>(static_cast<const float*>(prm.qp) + row * kD);
-      for (int c = 0; c < kD / 4; ++c) {
-        const float4 x = a4[c], y = b4[c];
-        const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float d0 = __fsub_rn(xs[u], ys[u]);
-          acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-        }
+      for (int w = 0; w < kD; ++w) {
+        const float d0 = __fsub_rn(__uint_as_float(x[w]), __uint_as_float(y[w]));
+        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
       }
     }
     s_mse[tid] = __fdiv_rn(acc, static_cast<float>(kD));
-  }
-  // block K/V of the group -> smem in the element type, rows >= B zero (this
-  // area is reused for the bound scores once the suffix is done)
-  const int Bpad = (B + kPS - 1) / kPS * kPS;
-  {
-    const int chunks = Bpad * kD * esz / 16;  // 16-byte chunks per tensor
-    const char* kg = static_cast<const char*>(prm.kb) + static_cast<size_t>(sg) * B * kD * esz;
-    const char* vg = static_cast<const char*>(prm.vb) + static_cast<size_t>(sg) * B * kD * esz;
-    char* kd = reinterpret_cast<char*>(kbv);
-    char* vd = kd + Bpad * kD * esz;
-    const int valid = B * kD * esz / 16;
-    for (int e = tid; e < chunks; e += kThreads) {
-      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-      if (e < valid) {
-        a = reinterpret_cast<const uint4*>(kg)[e];
-        b = reinterpret_cast<const uint4*>(vg)[e];
-      }
-      reinterpret_cast<uint4*>(kd)[e] = a;
-      reinterpret_cast<uint4*>(vd)[e] = b;
-    }
   }
   __syncthreads();
   if (tid < GB) {  // rank within the head: ties go to the lower token index
@@ -448,37 +545,40 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
   __syncthreads();
   if (tid < GB && act_slot[tid] >= 0) {
     const int hl = tid / B, t = tid % B;
-    act_tok[hl * A + act_slot[tid]] = t;
-    if (rank == 0 && prm.active_idx)
-      prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = t;
+    const int r = hl * A + act_slot[tid];
+    act_tok[r] = t;
+    if (chunk == 0) {
+      prm.act_tok_g[static_cast<size_t>(sg) * R + r] = t;
+      if (prm.active_idx)
+        prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = t;
+    }
   }
+  if (chunk == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
   __syncthreads();
 
-  // active rows' query vectors for the bound: bf16 -> [R16][256] = [q- | q+]
-  // (swizzled 16-byte chunks for ldmatrix); fp32 -> [R][128] plain
+  // ---- active rows' queries for the bound: bf16 -> [R16][256] = [q- | q+]
+  // in swizzled 16-byte chunks (ldmatrix); fp32 -> [R][128]
   const int R16 = (R + 15) / 16 * 16;
   if (scan) {
     if (DT == LOSA_BF16) {
       for (int e = tid; e < R16 * 32; e += kThreads) {
-        const int r = e / 32, c = e % 32;  // 16-byte chunk c of row r (8 bf16)
+        const int r = e / 32, c = e % 32;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (r < R) {
-          const int hl = r / A, t = act_tok[r];
-          const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-          const uint4 q = *reinterpret_cast<const uint4*>(
-              static_cast<const char*>(prm.qc) + row * kD * 2 + (c & 15) * 16);
-          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+          const int row = (r / A) * B + act_tok[r];
+          const uint32_t* src = qcs + row * qw + 4 * (c & 15);
           uint32_t o[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            uint32_t lo16 = w[u] & 0xffffu, hi16 = w[u] >> 16;
-            const bool neg_lo = lo16 & 0x8000u, neg_hi = hi16 & 0x8000u;
+            const uint32_t w = src[u];
+            uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
+            const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
             if (c < 16) {  // q- = min(q, 0)
-              lo16 = neg_lo ? lo16 : 0u;
-              hi16 = neg_hi ? hi16 : 0u;
-            } else {       // q+ = max(q, 0)
-              lo16 = neg_lo ? 0u : lo16;
-              hi16 = neg_hi ? 0u : hi16;
+              lo16 = nl ? lo16 : 0u;
+              hi16 = nh ? hi16 : 0u;
+            } else {  // q+ = max(q, 0)
+              lo16 = nl ? 0u : lo16;
+              hi16 = nh ? 0u : hi16;
             }
             o[u] = lo16 | (hi16 << 16);
           }
@@ -487,47 +587,46 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
         *reinterpret_cast<uint4*>(qrows + r * 512 + ((c ^ (r & 7)) << 4)) = v;
       }
     } else {
-      for (int e = tid; e < R * kD / 4; e += kThreads) {
-        const int r = e / (kD / 4), c = (e % (kD / 4)) * 4;
-        const int hl = r / A, t = act_tok[r];
-        const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-        *reinterpret_cast<float4*>(qrows + (r * kD + c) * 4) = ld4(prm.qc, row * kD + c, DT);
+      for (int e = tid; e < R * kD; e += kThreads) {
+        const int r = e / kD, c = e % kD;
+        const int row = (r / A) * B + act_tok[r];
+        reinterpret_cast<uint32_t*>(qrows)[r * kD + c] = qcs[row * qw + c];
       }
     }
   }
 
-  // suffix of this CTA's rows: stable token-rows i with i % CL == rank are
-  // finished here; active rows r with r % CL == rank keep (o_s, L_s) in smem
-  // for the final merge
-  {
-    float* psw = Ps + warp * 16;
-    const char* kbs = reinterpret_cast<const char*>(kbv);
-    const char* vbs = kbs + Bpad * kD * esz;
-    const int nstable_mine = (GB - rank + CL - 1) / CL;
-    const int nactive_mine = R > rank ? (R - rank + CL - 1) / CL : 0;
-    for (int job = warp; job < nstable_mine + nactive_mine; job += kWarps) {
-      int hl, t, r = -1;
-      if (job < nstable_mine) {
-        const int i = rank + job * CL;
+  // ---- this CTA's stable rows: suffix over the block, merge with the cache
+  if (n_stable_mine > 0) {
+    const bool ok = mbar_wait(&mbar[kMaxStages], 0);
+    if (!ok) {
+      if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+    } else {
+      float* psw = Ps + warp * 16;
+      const char* kbs = kbv;
+      const char* vbs = kbv + Bpad * kD * esz;
+      for (int n = warp; n < n_stable_mine; n += kWarps) {
+        const int i = chunk + n * nchunk;
         if (act_slot[i] >= 0) continue;
-        hl = i / B;
-        t = i % B;
-      } else {
-        r = rank + (job - nstable_mine) * CL;
-        hl = r / A;
-        t = act_tok[r];
-      }
-      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-      const float4 q = ld4(prm.qc, row * kD + 4 * lane, DT);
-      float m = -INFINITY, l = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j0 = 0; j0 < B; j0 += kPS)
-        attend_page<DT>(q, kbs + j0 * kD * esz, vbs + j0 * kD * esz, min(kPS, B - j0),
-                        d.scale_log2, m, l, acc, psw);
-      const float inv = 1.f / l;
-      const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      const float Ls = (m + __log2f(l)) * kLn2;
-      if (r < 0) {
+        const int hl = i / B, t = i % B;
+        const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
+        float4 q;
+        if (DT == LOSA_BF16) {
+          const uint32_t w0 = qcs[i * qw + 2 * lane], w1 = qcs[i * qw + 2 * lane + 1];
+          q = make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
+                          __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
+        } else {
+          const uint32_t* w = qcs + i * qw + 4 * lane;
+          q = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
+                          __uint_as_float(w[3]));
+        }
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          attend_page<DT>(q, kbs + j0 * kD * esz, vbs + j0 * kD * esz, min(kPS, B - j0),
+                          d.scale_log2, m, l, acc, psw);
+        const float inv = 1.f / l;
+        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        const float Ls = (m + __log2f(l)) * kLn2;
         const float4 op = *reinterpret_cast<const float4*>(prm.o_p + row * kD + 4 * lane);
         const float Lp = prm.l_p[row];
         float4 o;
@@ -535,146 +634,268 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
         lse_merge(op, Lp, os, Ls, o, L);
         *reinterpret_cast<float4*>(prm.out + row * kD + 4 * lane) = o;
         if (prm.out_lse && lane == 0) prm.out_lse[row] = L;
-      } else {
-        float* dst = sfx + (r / CL) * kPartStride;
-        if (lane == 0) dst[0] = Ls;
-        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
       }
     }
   }
-  __syncthreads();
+  __syncthreads();  // the block K/V area becomes the score area below
+  if (!scan) return;
 
-  // ---- P1: bound scores of the chunk --------------------------------------
-  if (scan) {
-    for (int t = 0; t < ntiles; ++t) {
-      const int st = t % prm.stages;
-      const uint32_t parity = (t / prm.stages) & 1;
-      if (!mbar_wait(&mbar[st], parity)) {
-        atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-        *s_fail = 1;
-      }
-      __syncthreads();
-      if (*s_fail) break;
-      const char* tile = ring + st * kStageBytes;
-      const int np = min(prm.tile, npages - t * prm.tile);
-      const int pl0 = t * prm.tile;  // chunk-local index of the tile's first page
-      if (DT == LOSA_BF16) {
-        const int ntn = (np + 7) / 8, ntm = R16 / 16;
-        const int g4 = lane >> 2, t4 = lane & 3;
-        for (int job = warp; job < ntn * ntm; job += kWarps) {
-          const int nt = job % ntn, mt = job / ntn;
-          float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // ---- bound scores of the chunk
+  const int ntm = R16 / 16;
+  for (int t = 0; t < ntiles; ++t) {
+    const int st = t % prm.stages;
+    const uint32_t parity = (t / prm.stages) & 1;
+    if (!mbar_wait(&mbar[st], parity)) {
+      atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+      *s_fail = 1;
+    }
+    __syncthreads();
+    if (*s_fail) return;  // no cluster here: leaving early is safe
+    const char* tile = ring + st * kStageBytes;
+    const int np = min(prm.tile, npages - t * prm.tile);
+    const int pl0 = t * prm.tile;
+    if (DT == LOSA_BF16) {
+      const int ntn = (np + 7) / 8;
+      const int g4 = lane >> 2, t4 = lane & 3;
+      for (int job = warp; job < ntn * ntm; job += kWarps) {
+        const int nt = job % ntn, mt = job / ntn;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int ks = 0; ks < 16; ks += 2) {
-            uint32_t b[4];
-            {
-              const int mi = lane >> 3, pg = nt * 8 + (lane & 7);
-              const int ch = ks * 2 + mi;
-              ldsm_x4(su32(tile + pg * 512 + ((ch ^ (pg & 7)) << 4)), b[0], b[1], b[2], b[3]);
-            }
+        for (int ks = 0; ks < 16; ks += 2) {
+          uint32_t b[4];
+          {
+            const int mi = lane >> 3, pg = nt * 8 + (lane & 7);
+            const int ch = ks * 2 + mi;
+            ldsm_x4(su32(tile + pg * 512 + ((ch ^ (pg & 7)) << 4)), b[0], b[1], b[2], b[3]);
+          }
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              uint32_t a[4];
-              const int mi = lane >> 3;
-              const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
-              const int ch = (ks + kk) * 2 + (mi >> 1);
-              ldsm_x4(su32(qrows + row * 512 + ((ch ^ (row & 7)) << 4)), a[0], a[1], a[2], a[3]);
-              mma_bf16(acc, a, b[2 * kk], b[2 * kk + 1]);
-            }
-          }
-          const int r0 = mt * 16 + g4, pc = pl0 + nt * 8 + 2 * t4;
-          if (r0 < R) {
-            sc[r0 * prm.sc_stride + pc] = acc[0];
-            sc[r0 * prm.sc_stride + pc + 1] = acc[1];
-          }
-          if (r0 + 8 < R) {
-            sc[(r0 + 8) * prm.sc_stride + pc] = acc[2];
-            sc[(r0 + 8) * prm.sc_stride + pc + 1] = acc[3];
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t a[4];
+            const int mi = lane >> 3;
+            const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
+            const int ch = (ks + kk) * 2 + (mi >> 1);
+            ldsm_x4(su32(qrows + row * 512 + ((ch ^ (row & 7)) << 4)), a[0], a[1], a[2], a[3]);
+            mma_bf16(acc, a, b[2 * kk], b[2 * kk + 1]);
           }
         }
-      } else {
-        // fp32: exact sum in channel order, one rounding per operation
-        for (int e = tid; e < np * R; e += kThreads) {
-          const int pl = e % np, r = e / np;
-          const int pg = p0 + pl0 + pl;
-          const char* recp = tile + pl * prm.rec;
-          const float* q = reinterpret_cast<const float*>(qrows) + r * kD;
-          float acc = 0.f;
-          for (int c = 0; c < kD / 4; ++c) {
-            const float4 mn = *reinterpret_cast<const float4*>(recp + meta_swz(16u * c, pg));
-            const float4 mx =
-                *reinterpret_cast<const float4*>(recp + meta_swz(16u * (c + kD / 4), pg));
-            const float mns[4] = {mn.x, mn.y, mn.z, mn.w}, mxs[4] = {mx.x, mx.y, mx.z, mx.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float qi = q[4 * c + u];
-              acc = __fadd_rn(acc, fmaxf(__fmul_rn(qi, mxs[u]), __fmul_rn(qi, mns[u])));
-            }
-          }
-          sc[r * prm.sc_stride + pl0 + pl] = acc;
+        const int r0 = mt * 16 + g4, pc = pl0 + nt * 8 + 2 * t4;
+        if (r0 < R) {
+          sc[r0 * prm.sc_stride + pc] = acc[0];
+          sc[r0 * prm.sc_stride + pc + 1] = acc[1];
+        }
+        if (r0 + 8 < R) {
+          sc[(r0 + 8) * prm.sc_stride + pc] = acc[2];
+          sc[(r0 + 8) * prm.sc_stride + pc + 1] = acc[3];
         }
       }
-      __syncthreads();
-      if (tid == 0 && t + prm.stages < ntiles) {  // refill the stage just consumed
-        const int tn = t + prm.stages;
-        const int npn = min(prm.tile, npages - tn * prm.tile);
-        const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
-        mbar_expect_tx(&mbar[st], bytes);
-        bulk_g2s(ring + st * kStageBytes,
-                 meta_g + static_cast<size_t>(p0 + tn * prm.tile) * prm.rec, bytes, &mbar[st]);
+    } else {
+      for (int e = tid; e < np * R; e += kThreads) {
+        const int pl = e % np, r = e / np;
+        const int pg = p0 + pl0 + pl;
+        const char* recp = tile + pl * prm.rec;
+        const float* q = reinterpret_cast<const float*>(qrows) + r * kD;
+        float acc = 0.f;
+        for (int c = 0; c < kD / 4; ++c) {
+          const float4 mn = *reinterpret_cast<const float4*>(recp + meta_swz(16u * c, pg));
+          const float4 mx = *reinterpret_cast<const float4*>(recp + meta_swz(16u * (c + kD / 4), pg));
+          const float mns[4] = {mn.x, mn.y, mn.z, mn.w}, mxs[4] = {mx.x, mx.y, mx.z, mx.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float qi = q[4 * c + u];
+            acc = __fadd_rn(acc, fmaxf(__fmul_rn(qi, mxs[u]), __fmul_rn(qi, mns[u])));
+          }
+        }
+        sc[r * prm.sc_stride + pl0 + pl] = acc;
       }
     }
-    // ---- P2: chunk-local top-k per row ------------------------------------
-    if (!*s_fail) {
-      for (int r = warp; r < R; r += kWarps) {
-        const float* row = sc + r * prm.sc_stride;
-        warp_topk([&](int i) { return sel_key(row[i], p0 + i); }, npages, k, cand + r * k,
-                  cbuf + warp * kCandCap);
-      }
+    __syncthreads();
+    if (tid == 0 && t + prm.stages < ntiles) {  // refill the stage just consumed
+      const int tn = t + prm.stages;
+      const int npn = min(prm.tile, npages - tn * prm.tile);
+      const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
+      mbar_expect_tx(&mbar[st], bytes);
+      bulk_g2s(ring + st * kStageBytes, meta_g + static_cast<size_t>(p0 + tn * prm.tile) * prm.rec,
+               bytes, &mbar[st]);
     }
   }
-  __syncthreads();
-  cluster.sync();
 
-  // ---- P3: merge of the CL candidate lists of this CTA's rows --------------
-  if (A > 0) {
-    if (!d.all_pages) {
-      for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
-        unsigned long long* best = cbuf + (kWarps + warp) * kCandCap;  // k <= 64
-        const unsigned long long* remote[kMaxCluster];
-        for (int c = 0; c < CL; ++c) remote[c] = cluster.map_shared_rank(cand, c) + r * k;
-        warp_topk([&](int i) { return remote[i / k][i % k]; }, CL * k, k, best,
-                  cbuf + warp * kCandCap);
-        // the k pages in ascending order
-        int32_t* dst = sel_own + (r / CL) * k;
-        for (int j = lane; j < k; j += 32) {
-          const int pj = key_index(best[j]);
-          int rk = 0;
-          for (int u = 0; u < k; ++u) rk += key_index(best[u]) < pj;
-          dst[rk] = pj;
-          if (prm.page_idx) {
-            const int hl = r / A, a = r % A;
-            prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + rk] = pj;
-          }
-        }
-        __syncwarp();
-      }
-    } else if (prm.page_idx) {
-      for (int e = tid; e < R * k; e += kThreads) {
-        const int r = e / k;
-        if (r % CL != rank) continue;
-        const int hl = r / A, a = r % A;
-        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + e % k] = e % k;
-      }
-    }
+  // ---- chunk-local top-k per row -> workspace
+  unsigned long long* dst = prm.cand + (static_cast<size_t>(sg) * nchunk + chunk) * R * k;
+  switch (prm.kp) {
+    case 2: chunk_topk<DT, 2>(prm, sc, R, k, npages, p0, dst, cbuf); break;
+    case 4: chunk_topk<DT, 4>(prm, sc, R, k, npages, p0, dst, cbuf); break;
+    case 8: chunk_topk<DT, 8>(prm, sc, R, k, npages, p0, dst, cbuf); break;
+    case 16: chunk_topk<DT, 16>(prm, sc, R, k, npages, p0, dst, cbuf); break;
+    default: chunk_topk<DT, 0>(prm, sc, R, k, npages, p0, dst, cbuf); break;
   }
-  __syncthreads();
-  cluster.sync();
+}
 
-  // ---- P4: union of the group's pages and this CTA's share ------------------
+// ---------------------------------------------------------------------------
+// K2: select, union, gather, combine
+// ---------------------------------------------------------------------------
+struct GatherLayout {
+  int slots, kbv, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, misc, ps, cbuf, mbar,
+      total;
+};
+
+struct GatherParams {
+  const void* qc;
+  const void* K;
+  const void* V;
+  const void* kb;
+  const void* vb;
+  float* o_p;
+  float* l_p;
+  float* out;
+  float* out_lse;
+  int32_t* page_idx;
+  int32_t* union_count;
+  const int32_t* act_tok_g;
+  const unsigned long long* cand;
+  int* status;
+  Dims d;
+  int CL;        // CTAs per cluster
+  int max_lp;    // max union pages per CTA
+  int ngp;       // pages in flight per CTA
+  int kp;        // register top-k width for the merge (0 = warp fallback)
+  GatherLayout lo;
+};
+
+template <int KP>
+__device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg,
+                                          unsigned long long* best, unsigned long long* cbuf) {
+  const Dims& d = prm.d;
+  const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
+  const unsigned long long* base = prm.cand + static_cast<size_t>(sg) * nc * R * k;
+  if (KP > 0) {
+    unsigned long long x[KP > 0 ? KP : 1];
+#pragma unroll
+    for (int i = 0; i < (KP > 0 ? KP : 1); ++i) x[i] = 0ull;
+    for (int c = lane; c < nc; c += 32) {
+      unsigned long long y[KP > 0 ? KP : 1];
+      const unsigned long long* lst = base + (static_cast<size_t>(c) * R + r) * k;
+#pragma unroll
+      for (int i = 0; i < (KP > 0 ? KP : 1); ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
+      merge_top<(KP > 0 ? KP : 1)>(x, y);
+    }
+    group_merge<(KP > 0 ? KP : 1)>(x, 32);
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < (KP > 0 ? KP : 1); ++i)
+        if (i < k) best[i] = x[i];
+    }
+    __syncwarp();
+  } else {
+    warp_topk([&](int i) { return __ldcg(base + (static_cast<size_t>(i / k) * R + r) * k + i % k); },
+              nc * k, k, best, cbuf);
+    __syncwarp();
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherParams prm) {
+  extern __shared__ __align__(1024) char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const Dims& d = prm.d;
+  const GatherLayout& lo = prm.lo;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int CL = prm.CL;
+  const int sg = blockIdx.y;
+  const int s = sg / d.Hkv, g = sg % d.Hkv;
+  const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
+  const int esz = DT == LOSA_BF16 ? 2 : 4;
+  const int Bpad = (B + kPS - 1) / kPS * kPS;
+  const int pbytes = kPS * kD * esz;
   const int nwords = (d.P + 31) / 32;
-  if (A > 0 && d.all_pages) {
-    // every row takes every page: the union is the whole prefix
+
+  char* slots = smem + lo.slots;
+  char* kbv = smem + lo.kbv;
+  char* qa = smem + lo.qa;  // [R][kD] active rows' queries, element type
+  int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
+  int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel_all);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + lo.bitmap);
+  int32_t* wbase = reinterpret_cast<int32_t*>(smem + lo.wbase);
+  int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
+  float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
+  int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
+  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
+  unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
+  int32_t* s_fail = misc;
+  int32_t* s_U = misc + 1;
+  int32_t* s_nlp = misc + 2;
+  int32_t* act_tok = misc + 4;  // [R]
+  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
+
+  if (tid == 0) {
+    for (int i = 0; i < kMaxGatherPages + 1; ++i) mbar_init(&mbar[i], 1);
+    fence_mbar_init();
+    *s_fail = 0;
+    // the block's own K/V (not written by the scan kernel)
+    mbar_expect_tx(&mbar[kMaxGatherPages], 2 * blk_bytes);
+    const size_t off = static_cast<size_t>(sg) * B * kD * esz;
+    bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxGatherPages]);
+    bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
+             &mbar[kMaxGatherPages]);
+  }
+  for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
+    part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+
+  // everything below reads what the scan kernel wrote
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  for (int r = tid; r < R; r += kThreads) act_tok[r] = __ldcg(prm.act_tok_g + static_cast<size_t>(sg) * R + r);
+  __syncthreads();
+  {  // active rows' queries
+    const int cpr = kD * esz / 16;
+    for (int e = tid; e < R * cpr; e += kThreads) {
+      const int r = e / cpr, c = e % cpr;
+      const int hl = r / A;
+      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + act_tok[r];
+      reinterpret_cast<uint4*>(qa)[e] =
+          reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + row * kD * esz)[c];
+    }
+  }
+
+  // ---- this CTA's rows (r % CL == rank): merge of the chunk candidates
+  if (!d.all_pages) {
+    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
+      unsigned long long* best = cbuf + (kWarps + warp) * kCandCap;
+      switch (prm.kp) {
+        case 2: merge_row<2>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+        case 4: merge_row<4>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+        case 8: merge_row<8>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+        case 16: merge_row<16>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+        default: merge_row<0>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+      }
+      int32_t* dst = sel_own + (r / CL) * k;
+      for (int j = lane; j < k; j += 32) {  // pages in ascending order
+        const int pj = key_index(best[j]);
+        int rk = 0;
+        for (int u = 0; u < k; ++u) rk += key_index(best[u]) < pj;
+        dst[rk] = pj;
+        if (prm.page_idx) {
+          const int hl = r / A, a = r % A;
+          prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + rk] = pj;
+        }
+      }
+      __syncwarp();
+    }
+  } else if (prm.page_idx) {
+    for (int e = tid; e < R * k; e += kThreads) {
+      const int r = e / k;
+      if (r % CL != rank) continue;
+      const int hl = r / A, a = r % A;
+      prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + e % k] = e % k;
+    }
+  }
+  __syncthreads();
+  cluster.sync();
+
+  // ---- union of the group's pages and this CTA's share
+  if (d.all_pages) {
     const int U = d.P;
     const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
     if (tid == 0) {
@@ -687,7 +908,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
       const int nb = min(32, R - 32 * w);
       masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
     }
-  } else if (A > 0) {
+  } else {
     for (int e = tid; e < R * k; e += kThreads) {
       const int r = e / k, j = e % k;
       sel_all[e] = cluster.map_shared_rank(sel_own, r % CL)[(r / CL) * k + j];
@@ -700,8 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
       else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
     }
     __syncthreads();
-    // exclusive prefix of word popcounts (warp 0; words dealt in runs per lane)
-    if (warp == 0) {
+    if (warp == 0) {  // exclusive prefix of word popcounts
       const int per = (nwords + 31) / 32;
       const int w0 = lane * per, w1 = min(nwords, w0 + per);
       int sum = 0;
@@ -748,107 +968,88 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
       if (u / CL < prm.max_lp) atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
       else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
     }
-  } else if (tid == 0 && rank == 0 && prm.union_count) {
-    prm.union_count[sg] = 0;
   }
   __syncthreads();
 
-  // ---- P5: gather this CTA's union pages ------------------------------------
-  if (A > 0 && !*s_fail && warp < prm.gwarps) {
+  // ---- gather: this CTA's union pages, in batches of ngp; warp w folds the
+  // pages of rows r = w, w + 8, ... into their partials (one writer per row)
+  {
     const int nlp = min(*s_nlp, prm.max_lp);
-    const int gw = prm.gwarps;
-    const int pbytes = kPS * kD * esz;  // one of K, V of a full page
-    char* slots = ring + warp * prm.gslots * 2 * pbytes;
-    uint64_t* wbar = mbar + kMaxStages + warp * 2;
-    const int mine = warp < nlp ? (nlp - warp + gw - 1) / gw : 0;
-    auto issue = [&](int i) {  // i-th page of this warp into slot i % gslots
-      const int p = lpages[warp + i * gw];
-      const int ntok = min(kPS, d.L - p * kPS);
-      const uint32_t bytes = static_cast<uint32_t>(ntok * kD * esz);
-      char* dst = slots + (i % prm.gslots) * 2 * pbytes;
-      const size_t off = (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS) * kD * esz;
-      mbar_expect_tx(&wbar[i % prm.gslots], 2 * bytes);
-      bulk_g2s(dst, static_cast<const char*>(prm.K) + off, bytes, &wbar[i % prm.gslots]);
-      bulk_g2s(dst + pbytes, static_cast<const char*>(prm.V) + off, bytes, &wbar[i % prm.gslots]);
-    };
-    if (lane == 0)
-      for (int i = 0; i < min(mine, prm.gslots); ++i) issue(i);
-    float* psw = Ps + warp * 16;
-    for (int i = 0; i < mine; ++i) {
-      const int ul = warp + i * gw;
-      const int p = lpages[ul];
-      const int ntok = min(kPS, d.L - p * kPS);
-      // every lane waits on the slot's barrier (acquire by each reader)
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&wbar[i % prm.gslots], (i / prm.gslots) & 1));
-      if (!ok) {
-        if (lane == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-        break;
-      }
-      const char* Ks = slots + (i % prm.gslots) * 2 * pbytes;
-      const char* Vs = Ks + pbytes;
-      const uint32_t* mk = masks + ul * d.MW;
-      for (int w = 0; w < d.MW; ++w) {
-        uint32_t bits = mk[w];
-        while (bits) {
-          const int r = w * 32 + __ffs(bits) - 1;
-          bits &= bits - 1;
-          const int hl = r / A, t = act_tok[r];
-          const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-          const float4 q = ld4(prm.qc, row * kD + 4 * lane, DT);
-          float m = -INFINITY, l = 0.f;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          // zero rows beyond ntok are masked by attend_page (score -inf, p = 0)
-          attend_page<DT>(q, Ks, Vs, ntok, d.scale_log2, m, l, acc, psw);
-          // slot of page p in row r's ascending list
-          int lo_ = p;
-          if (!d.all_pages) {
-            const int32_t* lst = sel_all + r * k;
-            int hi_ = k;
-            lo_ = 0;
-            while (lo_ < hi_) {
-              const int mid = (lo_ + hi_) >> 1;
-              if (lst[mid] < p) lo_ = mid + 1;
-              else hi_ = mid;
-            }
-            if (lo_ < k && lst[lo_] != p) lo_ = k;
-          }
-          if (lo_ >= k) {
-            if (lane == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-            continue;
-          }
-          float* dst = prm.part + ((static_cast<size_t>(sg) * R + r) * k + lo_) * kPartStride;
-          if (lane == 0) {
-            dst[0] = m;
-            dst[1] = l;
-          }
-          *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = acc;
+    for (int b0 = 0; b0 < nlp && !*s_fail; b0 += prm.ngp) {
+      const int nb = min(prm.ngp, nlp - b0);
+      const int batch = b0 / prm.ngp;
+      if (tid == 0) {
+        for (int i = 0; i < nb; ++i) {
+          const int p = lpages[b0 + i];
+          const int ntok = min(kPS, d.L - p * kPS);
+          const uint32_t bytes = static_cast<uint32_t>(ntok * kD * esz);
+          const size_t off = (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS) * kD * esz;
+          char* dst = slots + i * 2 * pbytes;
+          mbar_expect_tx(&mbar[i], 2 * bytes);
+          bulk_g2s(dst, static_cast<const char*>(prm.K) + off, bytes, &mbar[i]);
+          bulk_g2s(dst + pbytes, static_cast<const char*>(prm.V) + off, bytes, &mbar[i]);
         }
       }
-      __syncwarp();
-      if (lane == 0 && i + prm.gslots < mine) issue(i + prm.gslots);
+      float* psw = Ps + warp * 16;
+      for (int r = warp; r < R; r += kWarps) {
+        bool have = false;
+        for (int i = 0; i < nb; ++i) have |= (masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u;
+        if (!have) continue;
+        float4 q = row4<DT>(qa, r, lane);
+        float* pr = part + r * kPartStride;
+        float m = pr[0], l = pr[1];
+        float4 acc = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+        for (int i = 0; i < nb; ++i) {
+          if (!((masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u)) continue;
+          if (!__all_sync(0xffffffffu, mbar_wait(&mbar[i], batch & 1))) {
+            if (lane == 0) {
+              atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+              *s_fail = 1;
+            }
+            break;
+          }
+          const int p = lpages[b0 + i];
+          const char* Ks = slots + i * 2 * pbytes;
+          attend_page<DT>(q, Ks, Ks + pbytes, min(kPS, d.L - p * kPS), d.scale_log2, m, l, acc,
+                          psw);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          pr[0] = m;
+          pr[1] = l;
+        }
+        *reinterpret_cast<float4*>(pr + 4 + 4 * lane) = acc;
+      }
+      // every barrier of this batch completes (waited by the warps that use
+      // its page) before the slots are refilled
+      for (int i = tid; i < nb; i += kThreads)
+        if (!mbar_wait(&mbar[i], batch & 1)) *s_fail = 1;
+      __syncthreads();
     }
   }
-  __threadfence();
   __syncthreads();
   cluster.sync();
 
-  // ---- P6: combine, cache write-back, merge with the suffix ----------------
-  if (A > 0 && !*s_fail) {
-    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
-      const float* src0 = prm.part + (static_cast<size_t>(sg) * R + r) * k * kPartStride;
+  // ---- combine every CTA's partial of this CTA's rows, cache write-back,
+  // suffix and merge
+  // the block K/V copy is always waited for (no copy may land after exit)
+  const bool blk_ok = mbar_wait(&mbar[kMaxGatherPages], 0);
+  if (!*s_fail) {
+    float* psw = Ps + warp * 16;
+    for (int r = rank + CL * warp; r < R && blk_ok; r += CL * kWarps) {
       float M = -INFINITY;
-      for (int j = 0; j < k; ++j) M = fmaxf(M, __ldcg(src0 + static_cast<size_t>(j) * kPartStride));
+      for (int c = 0; c < CL; ++c) M = fmaxf(M, cluster.map_shared_rank(part, c)[r * kPartStride]);
       float lsum = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j = 0; j < k; ++j) {
-        const float* src = src0 + static_cast<size_t>(j) * kPartStride;
-        const float w = exp2f(__ldcg(src) - M);
-        lsum += w * __ldcg(src + 1);
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(src + 4 + 4 * lane));
-        acc.x += w * x.x;
-        acc.y += w * x.y;
-        acc.z += w * x.z;
-        acc.w += w * x.w;
+      for (int c = 0; c < CL; ++c) {  // fixed order: deterministic
+        const float* pr = cluster.map_shared_rank(part, c) + r * kPartStride;
+        const float w = exp2f(pr[0] - M);
+        lsum += w * pr[1];
+        const float4 a = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+        acc.x += w * a.x;
+        acc.y += w * a.y;
+        acc.z += w * a.z;
+        acc.w += w * a.w;
       }
       const float inv = 1.f / lsum;
       const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
@@ -857,102 +1058,133 @@ __global__ void __launch_bounds__(kThreads, 1) losa_step_kernel(const Params prm
       const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
       *reinterpret_cast<float4*>(prm.o_p + row * kD + 4 * lane) = op;
       if (lane == 0) prm.l_p[row] = Lp;
-      const float* sx = sfx + (r / CL) * kPartStride;
-      const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
+      // suffix of the active row over the block's own keys
+      const float4 q = row4<DT>(qa, r, lane);
+      float m2 = -INFINITY, l2 = 0.f;
+      float4 a2 = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < B; j0 += kPS)
+        attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
+                        d.scale_log2, m2, l2, a2, psw);
+      const float inv2 = 1.f / l2;
+      const float4 os = make_float4(a2.x * inv2, a2.y * inv2, a2.z * inv2, a2.w * inv2);
+      const float Ls = (m2 + __log2f(l2)) * kLn2;
       float4 o;
       float L;
-      lse_merge(op, Lp, os, sx[0], o, L);
+      lse_merge(op, Lp, os, Ls, o, L);
       *reinterpret_cast<float4*>(prm.out + row * kD + 4 * lane) = o;
       if (prm.out_lse && lane == 0) prm.out_lse[row] = L;
     }
+    if (!blk_ok && tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
   }
+  // no CTA may leave while others can still read its shared memory
+  cluster.sync();
+}
+// ---------------------------------------------------------------------------
+// host side: launch geometry, shared-memory layouts, attributes
+// ---------------------------------------------------------------------------
+constexpr int kGatherSmemTarget = 110 * 1024;  // two gather CTAs per SM
+
+int topk_width(int k) {
+  if (k <= 2) return 2;
+  if (k <= 4) return 4;
+  if (k <= 8) return 8;
+  if (k <= 16) return 16;
+  return 0;  // warp fallback
 }
 
-// ---------------------------------------------------------------------------
-// host side: launch geometry, shared-memory layout, attributes
-// ---------------------------------------------------------------------------
-int align_up(int x, int a) { return (x + a - 1) / a * a; }
-
-bool plan_with_ring(const Dims& d, Params* prm, int ring_bytes, int max_dyn, int max_cluster) {
+bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   prm->d = d;
   prm->rec = 2 * kD * d.esz;
   prm->tile = kStageBytes / prm->rec;  // 64 (bf16) or 32 (fp32) pages per stage
-  const int chunk = align_up((d.P + max_cluster - 1) / max_cluster, 8);
-  const int CL = (d.P + chunk - 1) / chunk;
-  prm->chunk = chunk;
-  prm->CL = CL;
-  prm->stages = ring_bytes / kStageBytes;
-  prm->sc_stride = align_up(chunk, 4) + 4;
-  const int pbytes = kPS * kD * d.esz;
-  prm->gwarps = std::min(kWarps, ring_bytes / (2 * pbytes));
-  if (prm->gwarps < 1) return false;
-  prm->gslots = std::min(2, ring_bytes / (prm->gwarps * 2 * pbytes));
-  prm->max_lp = (d.Umax + CL - 1) / CL;
-  const bool scan = d.A > 0 && !d.all_pages;
-  if (scan && d.k > kCandCap) return false;
+  prm->sc_stride = align_up(d.chunk_pages, 4) + 4;
+  prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
+  prm->kp = topk_width(d.k);
+  prm->tpr = d.R > 0 ? std::min(32, pow2_floor(std::max(1, kThreads / d.R))) : 1;
+  const bool selects = d.A > 0 && !d.all_pages;
+  if (selects && prm->kp == 0 && d.k > kCandCap) return false;
   const int R16 = (d.R + 15) / 16 * 16;
   const int Bpad = (d.B + kPS - 1) / kPS * kPS;
-  const int nwords = (d.P + 31) / 32;
-  const int rows_per_cta = (d.R + CL - 1) / CL;
-  Layout& lo = prm->lo;
-  int off = 0;
-  auto take = [&](long long bytes, int align) {
-    off = align_up(off, align);
-    const int o = off;
-    off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
-    return o;
-  };
-  lo.ring = take(ring_bytes, 1024);
-  lo.scores = take(std::max<long long>(scan ? 4LL * d.R * prm->sc_stride : 0,
-                                       2LL * Bpad * kD * d.esz), 16);
-  lo.qrows = take(scan ? R16 * 512 : 0, 128);
-  lo.kbv = lo.scores;
-  lo.cand = take(scan ? 8LL * d.R * d.k : 0, 16);
-  lo.sel_own = take(scan ? 4LL * rows_per_cta * d.k : 0, 16);
-  lo.sel_all = take(d.all_pages ? 0 : 4LL * d.R * d.k, 16);
-  lo.bitmap = take(nwords * 4, 16);
-  lo.wbase = take(nwords * 4, 16);
-  lo.lpages = take(prm->max_lp * 4, 16);
-  lo.masks = take(4LL * prm->max_lp * d.MW, 16);
-  lo.sfx = take(4LL * rows_per_cta * kPartStride, 16);
-  lo.cbuf = take(2 * kWarps * kCandCap * 8, 16);
-  lo.ps = take(kWarps * 16 * 4, 16);
-  lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
-  lo.mbar = take((kMaxStages + kWarps * 2) * 8, 8);
-  lo.total = off;
-  return lo.total <= max_dyn;
-}
-
-// Largest metadata ring (128, 96 or 64 KiB) whose plan fits.
-bool plan(const Dims& d, Params* prm, int max_dyn, int max_cluster = kMaxCluster) {
-  for (int ring = kMaxRingBytes; ring >= 64 * 1024; ring -= 32 * 1024)
-    if (plan_with_ring(d, prm, ring, max_dyn, max_cluster)) return true;
+  const int GB = d.G * d.B;
+  for (int ring = kMaxRingBytes; ring >= 64 * 1024; ring -= 32 * 1024) {
+    ScanLayout& lo = prm->lo;
+    int off = 0;
+    auto take = [&](long long bytes, int align) {
+      off = align_up(off, align);
+      const int o = off;
+      off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
+      return o;
+    };
+    lo.ring = take(ring, 1024);
+    lo.scores = take(std::max(4LL * d.R * prm->sc_stride, 2LL * Bpad * kD * d.esz), 16);
+    lo.qrows = take(R16 * 512, 128);
+    lo.qstage = take(2LL * GB * prm->qw * 4, 16);
+    lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
+    lo.ps = take(kWarps * 16 * 4, 16);
+    lo.cbuf = take(selects && prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
+    lo.mbar = take((kMaxStages + 1) * 8, 8);
+    lo.total = off;
+    prm->stages = ring / kStageBytes;
+    if (lo.total <= max_dyn) return true;
+  }
   return false;
 }
 
-}  // namespace
-
-// Whether the fused step's shared-memory plan fits `max_dyn` bytes.
-bool fused_step_fits(const Dims& d, int max_dyn) {
-  Params prm;
-  return plan(d, &prm, max_dyn);
+bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster) {
+  prm->d = d;
+  int CL = std::min(max_cluster, std::max(1, d.Umax));
+  prm->CL = CL;
+  prm->max_lp = (d.Umax + CL - 1) / CL;
+  prm->kp = topk_width(d.k);
+  if (!d.all_pages && prm->kp == 0 && d.k > kCandCap) return false;
+  const int Bpad = (d.B + kPS - 1) / kPS * kPS;
+  const int nwords = (d.P + 31) / 32;
+  const int pbytes = kPS * kD * d.esz;
+  const int rows_per_cta = (d.R + CL - 1) / CL;
+  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
+    GatherLayout& lo = prm->lo;
+    int off = 0;
+    auto take = [&](long long bytes, int align) {
+      off = align_up(off, align);
+      const int o = off;
+      off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
+      return o;
+    };
+    lo.slots = take(2LL * ngp * pbytes, 1024);
+    lo.kbv = take(2LL * Bpad * kD * d.esz, 16);
+    lo.qa = take(1LL * d.R * kD * d.esz, 16);
+    lo.sel_own = take(d.all_pages ? 0 : 4LL * rows_per_cta * d.k, 16);
+    lo.sel_all = take(d.all_pages ? 0 : 4LL * d.R * d.k, 16);
+    lo.bitmap = take(nwords * 4, 16);
+    lo.wbase = take(nwords * 4, 16);
+    lo.lpages = take(prm->max_lp * 4, 16);
+    lo.masks = take(4LL * prm->max_lp * d.MW, 16);
+    lo.part = take(4LL * d.R * kPartStride, 16);
+    lo.misc = take((4 + kMaxRowsPerGroup) * 4, 16);
+    lo.ps = take(kWarps * 16 * 4, 16);
+    // per-warp merge output (always) and compaction buffer (warp fallback)
+    lo.cbuf = take(2 * kWarps * kCandCap * 8, 16);
+    lo.mbar = take((kMaxGatherPages + 1) * 8, 8);
+    lo.total = off;
+    prm->ngp = ngp;
+    if (lo.total <= std::min(max_dyn, kGatherSmemTarget) || (ngp == 1 && lo.total <= max_dyn))
+      return true;
+  }
+  return false;
 }
-
-namespace {
 
 std::mutex g_attr_mu;
 bool g_attr_done[kMaxDevices] = {};
 int g_attr_dyn[kMaxDevices] = {};
 int g_attr_cluster[kMaxDevices] = {};
 
-// Largest cluster size (16 or 8) of which at least one cluster of
-// full-shared-memory CTAs can be resident on the device.
-int probe_cluster(int dyn) {
-  for (int cl = kMaxCluster; cl >= 8; cl /= 2) {
+// Largest cluster size (16, 8, 4) of which at least one cluster of gather
+// CTAs can be resident on the device.
+int probe_cluster() {
+  for (int cl = kMaxCluster; cl >= 4; cl /= 2) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cl, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
+    cfg.dynamicSmemBytes = static_cast<size_t>(kGatherSmemTarget);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cl;
@@ -961,12 +1193,12 @@ int probe_cluster(int dyn) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, losa_step_kernel<LOSA_BF16>, &cfg) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&n, losa_gather_kernel<LOSA_BF16>, &cfg) == cudaSuccess &&
         n > 0)
       return cl;
     cudaGetLastError();  // clear a refused query
   }
-  return 8;
+  return 4;
 }
 
 int ensure_attributes(int* max_dyn, int* max_cluster) {
@@ -979,22 +1211,26 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
     int optin = 0;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return record_cuda_error(e);
-    const void* fns[] = {reinterpret_cast<const void*>(losa_step_kernel<LOSA_BF16>),
-                         reinterpret_cast<const void*>(losa_step_kernel<LOSA_F32>)};
+    const void* fns[] = {reinterpret_cast<const void*>(losa_scan_kernel<LOSA_BF16>),
+                         reinterpret_cast<const void*>(losa_scan_kernel<LOSA_F32>),
+                         reinterpret_cast<const void*>(losa_gather_kernel<LOSA_BF16>),
+                         reinterpret_cast<const void*>(losa_gather_kernel<LOSA_F32>)};
     int dyn = optin;
-    for (const void* f : fns) {
+    for (int i = 0; i < 4; ++i) {
       cudaFuncAttributes fa;
-      e = cudaFuncGetAttributes(&fa, f);
+      e = cudaFuncGetAttributes(&fa, fns[i]);
       if (e != cudaSuccess) return record_cuda_error(e);
       const int mine = optin - static_cast<int>(fa.sharedSizeBytes);
-      e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
+      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
       if (e != cudaSuccess) return record_cuda_error(e);
-      e = cudaFuncSetAttribute(f, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return record_cuda_error(e);
-      dyn = mine < dyn ? mine : dyn;
+      if (i >= 2) {
+        e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return record_cuda_error(e);
+      }
+      dyn = std::min(dyn, mine);
     }
     g_attr_dyn[dev] = dyn;
-    g_attr_cluster[dev] = probe_cluster(dyn);
+    g_attr_cluster[dev] = probe_cluster();
     g_attr_done[dev] = true;
   }
   *max_dyn = g_attr_dyn[dev];
@@ -1004,7 +1240,12 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
 
 }  // namespace
 
-// Plans and launches the fused step (host validation already done).
+bool fused_step_fits(const Dims& d, int max_dyn) {
+  ScanParams sp;
+  GatherParams gp;
+  return plan_scan(d, &sp, max_dyn) && (d.A == 0 || plan_gather(d, &gp, max_dyn, kMaxCluster));
+}
+
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
                       const void* v_prefix, const void* page_meta, const void* k_blk,
                       const void* v_blk, float* o_p, float* l_p, float* out, float* out_lse,
@@ -1013,41 +1254,70 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   int max_dyn = 0, max_cluster = kMaxCluster;
   int rc = ensure_attributes(&max_dyn, &max_cluster);
   if (rc != LOSA_OK) return rc;
-  Params prm;
-  if (!plan(d, &prm, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
-  if (d.S * d.Hkv > 65535) return LOSA_ERR_UNSUPPORTED;
+  ScanParams sp;
+  GatherParams gp;
+  if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
+  if (d.A > 0 && !plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
+  if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
   char* ws = static_cast<char*>(workspace);
-  prm.qc = q_cur;
-  prm.qp = q_prev;
-  prm.K = k_prefix;
-  prm.V = v_prefix;
-  prm.meta = static_cast<const char*>(page_meta);
-  prm.kb = k_blk;
-  prm.vb = v_blk;
-  prm.o_p = o_p;
-  prm.l_p = l_p;
-  prm.out = out;
-  prm.out_lse = out_lse;
-  prm.active_idx = active_idx;
-  prm.page_idx = page_idx;
-  prm.union_count = union_count;
-  prm.part = reinterpret_cast<float*>(ws + d.off_part);
-  prm.status = reinterpret_cast<int*>(ws + d.off_status);
+  int* status = reinterpret_cast<int*>(ws + d.off_status);
+  int32_t* act_tok = reinterpret_cast<int32_t*>(ws + d.off_act);
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(prm.CL, d.S * d.Hkv, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(prm.lo.total);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  sp.qc = q_cur;
+  sp.qp = q_prev;
+  sp.meta = static_cast<const char*>(page_meta);
+  sp.kb = k_blk;
+  sp.vb = v_blk;
+  sp.o_p = o_p;
+  sp.l_p = l_p;
+  sp.out = out;
+  sp.out_lse = out_lse;
+  sp.active_idx = active_idx;
+  sp.union_count = union_count;
+  sp.act_tok_g = act_tok;
+  sp.cand = cand;
+  sp.status = status;
+  cudaLaunchConfig_t c1 = {};
+  c1.gridDim = dim3(d.nchunk, d.S * d.Hkv, 1);
+  c1.blockDim = dim3(kThreads, 1, 1);
+  c1.dynamicSmemBytes = static_cast<size_t>(sp.lo.total);
+  c1.stream = st;
+  cudaError_t e = d.dtype == LOSA_BF16 ? cudaLaunchKernelEx(&c1, losa_scan_kernel<LOSA_BF16>, sp)
+                                       : cudaLaunchKernelEx(&c1, losa_scan_kernel<LOSA_F32>, sp);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  if (d.A == 0) return LOSA_OK;
+
+  gp.qc = q_cur;
+  gp.K = k_prefix;
+  gp.V = v_prefix;
+  gp.kb = k_blk;
+  gp.vb = v_blk;
+  gp.o_p = o_p;
+  gp.l_p = l_p;
+  gp.out = out;
+  gp.out_lse = out_lse;
+  gp.page_idx = page_idx;
+  gp.union_count = union_count;
+  gp.act_tok_g = act_tok;
+  gp.cand = cand;
+  gp.status = status;
+  cudaLaunchConfig_t c2 = {};
+  c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
+  c2.blockDim = dim3(kThreads, 1, 1);
+  c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
+  c2.stream = st;
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = prm.CL;
+  attr[0].val.clusterDim.x = gp.CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = d.dtype == LOSA_BF16 ? cudaLaunchKernelEx(&cfg, losa_step_kernel<LOSA_BF16>, prm)
-                                       : cudaLaunchKernelEx(&cfg, losa_step_kernel<LOSA_F32>, prm);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  c2.attrs = attr;
+  c2.numAttrs = 2;
+  e = d.dtype == LOSA_BF16 ? cudaLaunchKernelEx(&c2, losa_gather_kernel<LOSA_BF16>, gp)
+                           : cudaLaunchKernelEx(&c2, losa_gather_kernel<LOSA_F32>, gp);
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
 

@@ -62,10 +62,10 @@ def test_noalloc_matches_workspace_step_on_two_calls():
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
-    # eight 32K sequences with B = 32 need more step workspace than the fixed
-    # array holds: refused before anything is launched (fake pointers are
-    # never dereferenced)
-    sh = api.shape_of(synth.config(3))
+    # sixteen 64K sequences with every block token active and a 1024-token
+    # budget need more step workspace than the fixed array holds: refused
+    # before anything is launched (the fake pointers are never dereferenced)
+    sh = api.make_shape(16, 32, 8, 128, 65536, 16, 16, 16, 1024)
     assert api.workspace_size(sh, api.LOSA_WS_STEP) > api.NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(1 << 20)
     rc = api.lib().losa_step_noalloc(ctypes.byref(sh), *([fake] * 10), None, None, None, None,
