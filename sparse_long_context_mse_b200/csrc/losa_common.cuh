@@ -190,7 +190,7 @@ __device__ __forceinline__ void lse_merge(float4 o1, float L1, float4 o2, float 
                                           float& L) {
   const float m = fmaxf(L1, L2);
   const float a = __expf(L1 - m), b = __expf(L2 - m);
-  const float inv = 1.f / (a + b);
+  const float inv = __frcp_rn(a + b);
   o.x = (a * o1.x + b * o2.x) * inv;
   o.y = (a * o1.y + b * o2.y) * inv;
   o.z = (a * o1.z + b * o2.z) * inv;

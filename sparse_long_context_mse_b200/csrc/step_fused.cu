@@ -39,6 +39,7 @@
 #include <mutex>
 
 #include "losa_common.cuh"
+#include "ptx.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -52,68 +53,8 @@ constexpr int kMaxRingBytes = 128 * 1024;
 constexpr int kStageBytes = 32 * 1024;
 constexpr int kMaxStages = kMaxRingBytes / kStageBytes;
 constexpr int kCandCap = 64;                     // per-warp compaction buffer
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
 constexpr int kMaxCluster = 16;
 constexpr int kMaxGatherPages = 16;              // pages in flight per K2 CTA
-
-// ---------------------------------------------------------------------------
-// PTX wrappers: mbarrier, bulk copy, ldmatrix, mma
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t su32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-// Non-multicast bulk copy global -> this CTA's shared memory.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(su32(dst)),
-      "l"(src), "r"(bytes), "r"(su32(bar))
-      : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(su32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait for phase `parity` of `bar`; false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
-  return true;
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
   return a > b ? a : b;
@@ -134,7 +75,7 @@ __device__ __forceinline__ float4 row4(const char* base, int j, int lane) {
 // Online-softmax update of one row (lane owns 4 channels) with `ntok` <= 16
 // keys/values of a page held in shared memory in element type DT.
 template <int DT>
-__device__ __forceinline__ void attend_page(float4 q, const char* Ks, const char* Vs, int ntok,
+__device__ __noinline__ void attend_page(float4 q, const char* Ks, const char* Vs, int ntok,
                                             float scale_log2, float& m, float& l, float4& acc,
                                             float* Ps) {
   const int lane = threadIdx.x & 31;
@@ -343,6 +284,72 @@ __device__ __forceinline__ void thread_topk(KeyFn key, int j, int stride, int n,
   }
 }
 
+// Top-k (k <= W) of the keys held by a group of W lanes (W a power of two;
+// groups are aligned inside the warp).  Lane j of a group holds the keys
+// key(i) for i = j, j + W, ... < n (0 = no key).  The threshold tau is the
+// k-th largest of the group's lane maxima: at least k keys reach it, so every
+// key of the top k does too.  The keys >= tau (at most `cap`) are compacted
+// into buf and rank-sorted into out[0..k).  Returns false, for every lane of
+// the warp and before writing anything, if an active group of the warp had
+// more than `cap` survivors.
+template <typename KeyFn>
+__device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long long* buf,
+                                  unsigned long long* out, int cap, bool active) {
+  const int lane = threadIdx.x & 31;
+  const int j = lane & (W - 1);
+  unsigned long long lmax = 0ull;
+#pragma unroll 1
+  for (int i = j; i < n; i += W) lmax = umax64(lmax, key(i));
+  unsigned long long v = lmax;  // bitonic sort of the lane maxima, descending
+#pragma unroll 1
+  for (int size = 2; size <= W; size <<= 1) {
+#pragma unroll 1
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool dir = (j & size) == 0, lower = (j & stride) == 0;
+      v = (lower == dir) ? umax64(v, o) : (v < o ? v : o);
+    }
+  }
+  const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1, W);
+  int cnt = 0;
+#pragma unroll 1
+  for (int i = j; i < n; i += W) {
+    const unsigned long long x = key(i);
+    cnt += (x >= tau && x != 0ull);
+  }
+  int incl = cnt;
+#pragma unroll 1
+  for (int o = 1; o < W; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o, W);
+    if (j >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, W - 1, W);
+  if (!__all_sync(0xffffffffu, !active || total <= cap)) return false;
+  if (active) {
+    int pos = incl - cnt;
+#pragma unroll 1
+    for (int i = j; i < n; i += W) {
+      const unsigned long long x = key(i);
+      if (x >= tau && x != 0ull) buf[pos++] = x;
+    }
+  }
+  __syncwarp();
+  if (active) {
+#pragma unroll 1
+    for (int t = j; t < total; t += W) {
+      const unsigned long long x = buf[t];
+      int rank = 0;
+#pragma unroll 4
+      for (int m = 0; m < total; ++m) rank += buf[m] > x;
+      if (rank < k) out[rank] = x;
+    }
+#pragma unroll 1
+    for (int t = total + j; t < k; t += W) out[t] = 0ull;
+  }
+  __syncwarp();
+  return true;
+}
+
 int pow2_floor(int x) {
   int p = 1;
   while (p * 2 <= x) p *= 2;
@@ -354,22 +361,13 @@ int align_up(int x, int a) { return (x + a - 1) / a * a; }
 // K1: scan
 // ---------------------------------------------------------------------------
 struct ScanLayout {
-  int ring, scores, qrows, qstage, misc, ps, cbuf, mbar, total;
+  int ring, scores, qrows, misc, fbuf, cbuf, mbar, total;
 };
 
 struct ScanParams {
   const void* qc;
   const void* qp;
   const char* meta;
-  const void* kb;
-  const void* vb;
-  const float* o_p;
-  const float* l_p;
-  float* out;
-  float* out_lse;
-  int32_t* active_idx;
-  int32_t* union_count;
-  int32_t* act_tok_g;              // workspace [S*Hkv][R]
   unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
   int* status;
   Dims d;
@@ -383,34 +381,46 @@ struct ScanParams {
   ScanLayout lo;
 };
 
+// Chunk-local top-k of every active row -> dst_base[r][0..k).  Fast path
+// (k <= 16): the threshold filter over a group of W >= k lanes per row, rows
+// in passes of kThreads / W; a warp whose groups overflow the filter buffer
+// falls back to register sort-and-merge.  k > 16: one warp per row.
 template <int DT, int KP>
 __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* sc, int R, int k,
                                            int npages, int p0, unsigned long long* dst_base,
-                                           unsigned long long* cbuf) {
+                                           unsigned long long* fbuf, unsigned long long* cbuf) {
   const int tid = threadIdx.x;
   if (KP > 0) {
-    const int tpr = prm.tpr;
-    const int r = tid / tpr, j = tid % tpr;
-    const int rr = r < R ? r : 0;  // idle rows work on row 0 and write nothing
-    const float* row = sc + rr * prm.sc_stride;
-    unsigned long long x[KP > 0 ? KP : 1];
-    thread_topk<(KP > 0 ? KP : 1)>([&](int i) { return sel_key(row[i], p0 + i); }, j, tpr, npages,
-                                   x);
-    group_merge<(KP > 0 ? KP : 1)>(x, tpr);
-    if (r < R && j == 0) {
-      unsigned long long* dst = dst_base + static_cast<size_t>(r) * k;
+    const int W = prm.tpr;
+    const int rows_per_pass = kThreads / W;
+#pragma unroll 1
+    for (int r0 = 0; r0 < R; r0 += rows_per_pass) {
+      const int r = r0 + tid / W;
+      const bool active = r < R;
+      const float* row = sc + (active ? r : 0) * prm.sc_stride;
+      unsigned long long* out = dst_base + static_cast<size_t>(active ? r : 0) * k;
+      auto key = [&](int i) { return sel_key(row[i], p0 + i); };
+      if (!group_topk_filter(key, npages, W, k, fbuf + (tid / W) * kCandCap, out, kCandCap,
+                             active)) {
+        unsigned long long x[KP > 0 ? KP : 1];
+        thread_topk<(KP > 0 ? KP : 1)>(key, tid & (W - 1), W, npages, x);
+        group_merge<(KP > 0 ? KP : 1)>(x, W);
+        if (active && (tid & (W - 1)) == 0) {
 #pragma unroll
-      for (int i = 0; i < (KP > 0 ? KP : 1); ++i)
-        if (i < k) dst[i] = x[i];
+          for (int i = 0; i < (KP > 0 ? KP : 1); ++i)
+            if (i < k) out[i] = x[i];
+        }
+      }
     }
   } else {
-    const int warp = tid >> 5;
+    const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll 1
     for (int r = warp; r < R; r += kWarps) {
       const float* row = sc + r * prm.sc_stride;
       warp_topk([&](int i) { return sel_key(row[i], p0 + i); }, npages, k,
                 cbuf + (kWarps + warp) * kCandCap, cbuf + warp * kCandCap);
       __syncwarp();
-      const int lane = tid & 31;
+#pragma unroll 1
       for (int i = lane; i < k; i += 32)
         dst_base[static_cast<size_t>(r) * k + i] = cbuf[(kWarps + warp) * kCandCap + i];
       __syncwarp();
@@ -418,7 +428,7 @@ __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* s
   }
 }
 
-template <int DT>
+template <int DT, int KP>
 __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams prm) {
   extern __shared__ __align__(1024) char smem[];
   const Dims& d = prm.d;
@@ -428,23 +438,20 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
-  const int esz = DT == LOSA_BF16 ? 2 : 4;
   const int GB = G * B;
-  const int Bpad = (B + kPS - 1) / kPS * kPS;
   const int qw = prm.qw;
 
-  // let the gather kernel be scheduled as soon as resources free up; it
-  // waits for this grid's completion before reading anything written here
+  // let the gather kernel start its own preparation now; it waits for this
+  // grid's completion before it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   char* ring = smem + lo.ring;
   float* sc = reinterpret_cast<float*>(smem + lo.scores);
-  char* kbv = smem + lo.scores;  // block K then V (element type); aliases sc
-  char* qrows = smem + lo.qrows;
-  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.qstage);  // [GB][qw]
+  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.scores);  // staging; aliases sc
   uint32_t* qps = qcs + GB * qw;
+  char* qrows = smem + lo.qrows;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
-  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
+  unsigned long long* fbuf = reinterpret_cast<unsigned long long*>(smem + lo.fbuf);
   unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
   int32_t* s_fail = misc;
@@ -455,41 +462,32 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int p0 = chunk * d.chunk_pages;
   const int npages = max(0, min(d.P, p0 + d.chunk_pages) - p0);
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
-  const bool scan = A > 0 && !d.all_pages && npages > 0;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.P * prm.rec;
-  // stable token-rows of the group handled here: i = chunk + n * nchunk
-  const int n_stable_mine = GB > chunk ? (GB - chunk + nchunk - 1) / nchunk : 0;
-  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
+  if (npages == 0) return;
 
   if (tid == 0) {
-    for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxStages; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    if (scan) {
-      for (int t = 0; t < min(ntiles, prm.stages); ++t) {
-        const int np = min(prm.tile, npages - t * prm.tile);
-        const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
-        mbar_expect_tx(&mbar[t], bytes);
-        bulk_g2s(ring + t * kStageBytes,
-                 meta_g + static_cast<size_t>(p0 + t * prm.tile) * prm.rec, bytes, &mbar[t]);
-      }
-    }
-    if (n_stable_mine > 0) {  // the block's own K/V for the suffix
-      mbar_expect_tx(&mbar[kMaxStages], 2 * blk_bytes);
-      const size_t off = static_cast<size_t>(sg) * B * kD * esz;
-      bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxStages]);
-      bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
-               &mbar[kMaxStages]);
+#pragma unroll 1
+    for (int t = 0; t < min(ntiles, prm.stages); ++t) {
+      const int np = min(prm.tile, npages - t * prm.tile);
+      const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
+      mbar_expect_tx(&mbar[t], bytes);
+      bulk_g2s(ring + t * kStageBytes, meta_g + static_cast<size_t>(p0 + t * prm.tile) * prm.rec,
+               bytes, &mbar[t]);
     }
   }
 
   // ---- stage the group's current / previous queries (coalesced), padded
   // rows so that one thread walking its row in channel order hits every bank
   {
+    const int esz = DT == LOSA_BF16 ? 2 : 4;
     const int cpr = kD * esz / 16;  // 16-byte chunks per row
     const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
     const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
     const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + base);
+#pragma unroll 2
     for (int e = tid; e < GB * cpr; e += kThreads) {
       const int row = e / cpr, c = e % cpr;
       const uint4 a = gc[e], b = gp[e];
@@ -507,6 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     const uint32_t* y = qps + tid * qw;
     float acc = 0.f;
     if (DT == LOSA_BF16) {
+#pragma unroll 8
       for (int w = 0; w < kD / 2; ++w) {
         const uint32_t a = x[w], b = y[w];
         const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
@@ -515,18 +514,20 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
         acc = __fadd_rn(acc, __fmul_rn(d1, d1));
       }
     } else {
+#pragma unroll 8
       for (int w = 0; w < kD; ++w) {
         const float d0 = __fsub_rn(__uint_as_float(x[w]), __uint_as_float(y[w]));
         acc = __fadd_rn(acc, __fmul_rn(d0, d0));
       }
     }
-    s_mse[tid] = __fdiv_rn(acc, static_cast<float>(kD));
+    s_mse[tid] = acc * (1.0f / kD);  // exact: kD is a power of two
   }
   __syncthreads();
   if (tid < GB) {  // rank within the head: ties go to the lower token index
     const int hl = tid / B, t = tid % B;
     const float x = s_mse[tid];
     int rk = 0;
+#pragma unroll 4
     for (int u = 0; u < B; ++u) {
       const float y = s_mse[hl * B + u];
       rk += (y > x) || (y == x && u < t);
@@ -538,110 +539,58 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   if (tid < GB && act_slot[tid]) {  // slot = active tokens before t in the head
     const int hl = tid / B, t = tid % B;
     my_slot = 0;
+#pragma unroll 1
     for (int u = 0; u < t; ++u) my_slot += act_slot[hl * B + u];
   }
   __syncthreads();
   if (tid < GB) act_slot[tid] = my_slot;
   __syncthreads();
-  if (tid < GB && act_slot[tid] >= 0) {
-    const int hl = tid / B, t = tid % B;
-    const int r = hl * A + act_slot[tid];
-    act_tok[r] = t;
-    if (chunk == 0) {
-      prm.act_tok_g[static_cast<size_t>(sg) * R + r] = t;
-      if (prm.active_idx)
-        prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = t;
-    }
-  }
-  if (chunk == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
+  if (tid < GB && act_slot[tid] >= 0) act_tok[(tid / B) * A + act_slot[tid]] = tid % B;
   __syncthreads();
 
   // ---- active rows' queries for the bound: bf16 -> [R16][256] = [q- | q+]
   // in swizzled 16-byte chunks (ldmatrix); fp32 -> [R][128]
   const int R16 = (R + 15) / 16 * 16;
-  if (scan) {
-    if (DT == LOSA_BF16) {
-      for (int e = tid; e < R16 * 32; e += kThreads) {
-        const int r = e / 32, c = e % 32;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < R) {
-          const int row = (r / A) * B + act_tok[r];
-          const uint32_t* src = qcs + row * qw + 4 * (c & 15);
-          uint32_t o[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t w = src[u];
-            uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
-            const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
-            if (c < 16) {  // q- = min(q, 0)
-              lo16 = nl ? lo16 : 0u;
-              hi16 = nh ? hi16 : 0u;
-            } else {  // q+ = max(q, 0)
-              lo16 = nl ? 0u : lo16;
-              hi16 = nh ? 0u : hi16;
-            }
-            o[u] = lo16 | (hi16 << 16);
-          }
-          v = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        *reinterpret_cast<uint4*>(qrows + r * 512 + ((c ^ (r & 7)) << 4)) = v;
-      }
-    } else {
-      for (int e = tid; e < R * kD; e += kThreads) {
-        const int r = e / kD, c = e % kD;
+  if (DT == LOSA_BF16) {
+#pragma unroll 1
+    for (int e = tid; e < R16 * 32; e += kThreads) {
+      const int r = e / 32, c = e % 32;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < R) {
         const int row = (r / A) * B + act_tok[r];
-        reinterpret_cast<uint32_t*>(qrows)[r * kD + c] = qcs[row * qw + c];
-      }
-    }
-  }
-
-  // ---- this CTA's stable rows: suffix over the block, merge with the cache
-  if (n_stable_mine > 0) {
-    const bool ok = mbar_wait(&mbar[kMaxStages], 0);
-    if (!ok) {
-      if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-    } else {
-      float* psw = Ps + warp * 16;
-      const char* kbs = kbv;
-      const char* vbs = kbv + Bpad * kD * esz;
-      for (int n = warp; n < n_stable_mine; n += kWarps) {
-        const int i = chunk + n * nchunk;
-        if (act_slot[i] >= 0) continue;
-        const int hl = i / B, t = i % B;
-        const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-        float4 q;
-        if (DT == LOSA_BF16) {
-          const uint32_t w0 = qcs[i * qw + 2 * lane], w1 = qcs[i * qw + 2 * lane + 1];
-          q = make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
-                          __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
-        } else {
-          const uint32_t* w = qcs + i * qw + 4 * lane;
-          q = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
-                          __uint_as_float(w[3]));
+        const uint32_t* src = qcs + row * qw + 4 * (c & 15);
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t w = src[u];
+          uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
+          const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
+          if (c < 16) {  // q- = min(q, 0)
+            lo16 = nl ? lo16 : 0u;
+            hi16 = nh ? hi16 : 0u;
+          } else {  // q+ = max(q, 0)
+            lo16 = nl ? 0u : lo16;
+            hi16 = nh ? 0u : hi16;
+          }
+          o[u] = lo16 | (hi16 << 16);
         }
-        float m = -INFINITY, l = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j0 = 0; j0 < B; j0 += kPS)
-          attend_page<DT>(q, kbs + j0 * kD * esz, vbs + j0 * kD * esz, min(kPS, B - j0),
-                          d.scale_log2, m, l, acc, psw);
-        const float inv = 1.f / l;
-        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        const float Ls = (m + __log2f(l)) * kLn2;
-        const float4 op = *reinterpret_cast<const float4*>(prm.o_p + row * kD + 4 * lane);
-        const float Lp = prm.l_p[row];
-        float4 o;
-        float L;
-        lse_merge(op, Lp, os, Ls, o, L);
-        *reinterpret_cast<float4*>(prm.out + row * kD + 4 * lane) = o;
-        if (prm.out_lse && lane == 0) prm.out_lse[row] = L;
+        v = make_uint4(o[0], o[1], o[2], o[3]);
       }
+      *reinterpret_cast<uint4*>(qrows + r * 512 + ((c ^ (r & 7)) << 4)) = v;
+    }
+  } else {
+#pragma unroll 1
+    for (int e = tid; e < R * kD; e += kThreads) {
+      const int r = e / kD, c = e % kD;
+      const int row = (r / A) * B + act_tok[r];
+      reinterpret_cast<uint32_t*>(qrows)[r * kD + c] = qcs[row * qw + c];
     }
   }
-  __syncthreads();  // the block K/V area becomes the score area below
-  if (!scan) return;
+  __syncthreads();  // the staging area becomes the score area below
 
   // ---- bound scores of the chunk
   const int ntm = R16 / 16;
+#pragma unroll 1
   for (int t = 0; t < ntiles; ++t) {
     const int st = t % prm.stages;
     const uint32_t parity = (t / prm.stages) & 1;
@@ -657,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     if (DT == LOSA_BF16) {
       const int ntn = (np + 7) / 8;
       const int g4 = lane >> 2, t4 = lane & 3;
+#pragma unroll 1
       for (int job = warp; job < ntn * ntm; job += kWarps) {
         const int nt = job % ntn, mt = job / ntn;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -689,12 +639,14 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
         }
       }
     } else {
+#pragma unroll 1
       for (int e = tid; e < np * R; e += kThreads) {
         const int pl = e % np, r = e / np;
         const int pg = p0 + pl0 + pl;
         const char* recp = tile + pl * prm.rec;
         const float* q = reinterpret_cast<const float*>(qrows) + r * kD;
         float acc = 0.f;
+#pragma unroll 1
         for (int c = 0; c < kD / 4; ++c) {
           const float4 mn = *reinterpret_cast<const float4*>(recp + meta_swz(16u * c, pg));
           const float4 mx = *reinterpret_cast<const float4*>(recp + meta_swz(16u * (c + kD / 4), pg));
@@ -721,25 +673,20 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
 
   // ---- chunk-local top-k per row -> workspace
   unsigned long long* dst = prm.cand + (static_cast<size_t>(sg) * nchunk + chunk) * R * k;
-  switch (prm.kp) {
-    case 2: chunk_topk<DT, 2>(prm, sc, R, k, npages, p0, dst, cbuf); break;
-    case 4: chunk_topk<DT, 4>(prm, sc, R, k, npages, p0, dst, cbuf); break;
-    case 8: chunk_topk<DT, 8>(prm, sc, R, k, npages, p0, dst, cbuf); break;
-    case 16: chunk_topk<DT, 16>(prm, sc, R, k, npages, p0, dst, cbuf); break;
-    default: chunk_topk<DT, 0>(prm, sc, R, k, npages, p0, dst, cbuf); break;
-  }
+  chunk_topk<DT, KP>(prm, sc, R, k, npages, p0, dst, fbuf, cbuf);
 }
 
 // ---------------------------------------------------------------------------
-// K2: select, union, gather, combine
+// K2: active set, suffix, stable rows; then select, union, gather, combine
 // ---------------------------------------------------------------------------
 struct GatherLayout {
-  int slots, kbv, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, misc, ps, cbuf, mbar,
-      total;
+  int stage, kbv, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, sfx, misc, ps, mbuf,
+      mbar, total;
 };
 
 struct GatherParams {
   const void* qc;
+  const void* qp;
   const void* K;
   const void* V;
   const void* kb;
@@ -748,51 +695,112 @@ struct GatherParams {
   float* l_p;
   float* out;
   float* out_lse;
+  int32_t* active_idx;
   int32_t* page_idx;
   int32_t* union_count;
-  const int32_t* act_tok_g;
   const unsigned long long* cand;
   int* status;
   Dims d;
   int CL;        // CTAs per cluster
   int max_lp;    // max union pages per CTA
   int ngp;       // pages in flight per CTA
-  int kp;        // register top-k width for the merge (0 = warp fallback)
+  int qw;        // 32-bit words per staged query row (padded)
   GatherLayout lo;
 };
 
+// The k best chunk candidates of row r (keys, descending) -> out[0..k).
+// Fast path: lane c holds chunk c's sorted list; threshold = k-th largest
+// list head; the survivors are rank-sorted.  Fallback: sort-and-merge trees
+// or k rounds of warp argmax.
 template <int KP>
 __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg,
-                                          unsigned long long* best, unsigned long long* cbuf) {
+                                          unsigned long long* out, unsigned long long* fb) {
   const Dims& d = prm.d;
   const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
   const unsigned long long* base = prm.cand + static_cast<size_t>(sg) * nc * R * k;
   if (KP > 0) {
-    unsigned long long x[KP > 0 ? KP : 1];
+    constexpr int KQ = KP > 0 ? KP : 1;
+    unsigned long long x[KQ];
+    {
+      const unsigned long long* lst = base + (static_cast<size_t>(lane) * R + r) * k;
 #pragma unroll
-    for (int i = 0; i < (KP > 0 ? KP : 1); ++i) x[i] = 0ull;
-    for (int c = lane; c < nc; c += 32) {
-      unsigned long long y[KP > 0 ? KP : 1];
+      for (int i = 0; i < KQ; ++i) x[i] = (lane < nc && i < k) ? __ldcg(lst + i) : 0ull;
+    }
+#pragma unroll 1
+    for (int c = lane + 32; c < nc; c += 32) {  // more than 32 chunks: fold lists
+      unsigned long long y[KQ];
       const unsigned long long* lst = base + (static_cast<size_t>(c) * R + r) * k;
 #pragma unroll
-      for (int i = 0; i < (KP > 0 ? KP : 1); ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
-      merge_top<(KP > 0 ? KP : 1)>(x, y);
+      for (int i = 0; i < KQ; ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
+      merge_top<KQ>(x, y);
     }
-    group_merge<(KP > 0 ? KP : 1)>(x, 32);
-    if (lane == 0) {
+    // threshold from the list heads (every list is sorted, descending)
+    unsigned long long v = x[0];
+#pragma unroll 1
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll 1
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
+        const bool dir = (lane & size) == 0, lower = (lane & stride) == 0;
+        v = (lower == dir) ? umax64(v, o) : (v < o ? v : o);
+      }
+    }
+    const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1);
+    int cnt = 0;
 #pragma unroll
-      for (int i = 0; i < (KP > 0 ? KP : 1); ++i)
-        if (i < k) best[i] = x[i];
+    for (int i = 0; i < KQ; ++i) cnt += (x[i] >= tau && x[i] != 0ull);
+    int incl = cnt;
+#pragma unroll 1
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= kCandCap) {
+      int pos = incl - cnt;
+#pragma unroll
+      for (int i = 0; i < KQ; ++i)
+        if (x[i] >= tau && x[i] != 0ull) fb[pos++] = x[i];
+      __syncwarp();
+#pragma unroll 1
+      for (int t = lane; t < total; t += 32) {
+        const unsigned long long y = fb[t];
+        int rank = 0;
+#pragma unroll 4
+        for (int m = 0; m < total; ++m) rank += fb[m] > y;
+        if (rank < k) out[rank] = y;
+      }
+#pragma unroll 1
+      for (int t = total + lane; t < k; t += 32) out[t] = 0ull;
+    } else {
+      group_merge<KQ>(x, 32);
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < KQ; ++i)
+          if (i < k) out[i] = x[i];
+      }
     }
     __syncwarp();
   } else {
     warp_topk([&](int i) { return __ldcg(base + (static_cast<size_t>(i / k) * R + r) * k + i % k); },
-              nc * k, k, best, cbuf);
+              nc * k, k, out, fb);
     __syncwarp();
   }
 }
 
 template <int DT>
+__device__ __forceinline__ float4 qrow4(const uint32_t* qs, int row, int qw, int lane) {
+  if (DT == LOSA_BF16) {
+    const uint32_t w0 = qs[row * qw + 2 * lane], w1 = qs[row * qw + 2 * lane + 1];
+    return make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
+                       __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
+  }
+  const uint32_t* w = qs + row * qw + 4 * lane;
+  return make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
+                     __uint_as_float(w[3]));
+}
+
+template <int DT, int KP>
 __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherParams prm) {
   extern __shared__ __align__(1024) char smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -808,8 +816,12 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   const int Bpad = (B + kPS - 1) / kPS * kPS;
   const int pbytes = kPS * kD * esz;
   const int nwords = (d.P + 31) / 32;
+  const int GB = G * B;
+  const int qw = prm.qw;
 
-  char* slots = smem + lo.slots;
+  char* slots = smem + lo.stage;  // gather pages, once the staged queries are done with
+  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.stage);
+  uint32_t* qps = qcs + GB * qw;
   char* kbv = smem + lo.kbv;
   char* qa = smem + lo.qa;  // [R][kD] active rows' queries, element type
   int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
@@ -819,61 +831,179 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
+  float* sfx = reinterpret_cast<float*>(smem + lo.sfx);    // this CTA's active rows' suffix
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
-  unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
+  unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
   int32_t* s_fail = misc;
   int32_t* s_U = misc + 1;
   int32_t* s_nlp = misc + 2;
-  int32_t* act_tok = misc + 4;  // [R]
+  float* s_mse = reinterpret_cast<float*>(misc + 4);
+  int32_t* act_slot = misc + 4 + kMaxRowsPerGroup;
+  int32_t* act_tok = act_slot + kMaxRowsPerGroup;
   const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
+  float* psw = Ps + warp * 16;
 
+  // ================= preparation (independent of the scan kernel) ==========
   if (tid == 0) {
     for (int i = 0; i < kMaxGatherPages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    // the block's own K/V (not written by the scan kernel)
-    mbar_expect_tx(&mbar[kMaxGatherPages], 2 * blk_bytes);
+    mbar_expect_tx(&mbar[kMaxGatherPages], 2 * blk_bytes);  // the block's own K/V
     const size_t off = static_cast<size_t>(sg) * B * kD * esz;
     bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxGatherPages]);
     bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
              &mbar[kMaxGatherPages]);
   }
-  for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
-    part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
-
-  // everything below reads what the scan kernel wrote
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  for (int r = tid; r < R; r += kThreads) act_tok[r] = __ldcg(prm.act_tok_g + static_cast<size_t>(sg) * R + r);
-  __syncthreads();
-  {  // active rows' queries
+  {  // stage the group's current / previous queries (padded rows)
     const int cpr = kD * esz / 16;
-    for (int e = tid; e < R * cpr; e += kThreads) {
-      const int r = e / cpr, c = e % cpr;
-      const int hl = r / A;
-      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + act_tok[r];
-      reinterpret_cast<uint4*>(qa)[e] =
-          reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + row * kD * esz)[c];
+    const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
+    const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
+    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + base);
+#pragma unroll 2
+    for (int e = tid; e < GB * cpr; e += kThreads) {
+      const int row = e / cpr, c = e % cpr;
+      const uint4 a = gc[e], b = gp[e];
+      uint32_t* x = qcs + row * qw + 4 * c;
+      uint32_t* y = qps + row * qw + 4 * c;
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
     }
   }
-
-  // ---- this CTA's rows (r % CL == rank): merge of the chunk candidates
-  if (!d.all_pages) {
-    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
-      unsigned long long* best = cbuf + (kWarps + warp) * kCandCap;
-      switch (prm.kp) {
-        case 2: merge_row<2>(prm, r, sg, best, cbuf + warp * kCandCap); break;
-        case 4: merge_row<4>(prm, r, sg, best, cbuf + warp * kCandCap); break;
-        case 8: merge_row<8>(prm, r, sg, best, cbuf + warp * kCandCap); break;
-        case 16: merge_row<16>(prm, r, sg, best, cbuf + warp * kCandCap); break;
-        default: merge_row<0>(prm, r, sg, best, cbuf + warp * kCandCap); break;
+#pragma unroll 1
+  for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
+    part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+  __syncthreads();
+  // locality score (fp32, one rounding per operation, channels in order) and
+  // active set -- the same computation, in the same order, as the scan kernel
+  if (tid < GB) {
+    const uint32_t* x = qcs + tid * qw;
+    const uint32_t* y = qps + tid * qw;
+    float acc = 0.f;
+    if (DT == LOSA_BF16) {
+#pragma unroll 8
+      for (int w = 0; w < kD / 2; ++w) {
+        const uint32_t a = x[w], b = y[w];
+        const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
+        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
+        const float d1 = __fsub_rn(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u));
+        acc = __fadd_rn(acc, __fmul_rn(d1, d1));
       }
+    } else {
+#pragma unroll 8
+      for (int w = 0; w < kD; ++w) {
+        const float d0 = __fsub_rn(__uint_as_float(x[w]), __uint_as_float(y[w]));
+        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
+      }
+    }
+    s_mse[tid] = acc * (1.0f / kD);
+  }
+  __syncthreads();
+  if (tid < GB) {
+    const int hl = tid / B, t = tid % B;
+    const float x = s_mse[tid];
+    int rk = 0;
+#pragma unroll 4
+    for (int u = 0; u < B; ++u) {
+      const float y = s_mse[hl * B + u];
+      rk += (y > x) || (y == x && u < t);
+    }
+    act_slot[tid] = rk < A ? 1 : 0;
+  }
+  __syncthreads();
+  int my_slot = -1;
+  if (tid < GB && act_slot[tid]) {
+    const int hl = tid / B, t = tid % B;
+    my_slot = 0;
+#pragma unroll 1
+    for (int u = 0; u < t; ++u) my_slot += act_slot[hl * B + u];
+  }
+  __syncthreads();
+  if (tid < GB) act_slot[tid] = my_slot;
+  __syncthreads();
+  if (tid < GB && act_slot[tid] >= 0) {
+    const int hl = tid / B;
+    act_tok[hl * A + act_slot[tid]] = tid % B;
+    if (rank == 0 && prm.active_idx)
+      prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = tid % B;
+  }
+  if (rank == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
+  __syncthreads();
+  {  // active rows' queries in the element type
+    const int wpr = kD * esz / 4;  // 32-bit words per row
+#pragma unroll 1
+    for (int e = tid; e < R * wpr; e += kThreads) {
+      const int r = e / wpr, w = e % wpr;
+      const int row = (r / A) * B + act_tok[r];
+      reinterpret_cast<uint32_t*>(qa)[e] = qcs[row * qw + w];
+    }
+  }
+  // suffix over the block: stable token-rows i with i % CL == rank are
+  // finished here (merge with their untouched cache); active rows r with
+  // r % CL == rank keep (o_s, L_s) for the final merge
+  const bool blk_ok = mbar_wait(&mbar[kMaxGatherPages], 0);
+  if (!blk_ok && tid == 0) {
+    atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+    *s_fail = 1;
+  }
+  if (blk_ok) {
+    const int n_st = GB > rank ? (GB - rank + CL - 1) / CL : 0;
+    const int n_ac = R > rank ? (R - rank + CL - 1) / CL : 0;
+#pragma unroll 1
+    for (int job = warp; job < n_st + n_ac; job += kWarps) {
+      int row, r = -1;
+      if (job < n_st) {
+        const int i = rank + job * CL;
+        if (act_slot[i] >= 0) continue;
+        row = i;
+      } else {
+        r = rank + (job - n_st) * CL;
+        row = (r / A) * B + act_tok[r];
+      }
+      const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G) * B + row;
+      const float4 q = qrow4<DT>(qcs, row, qw, lane);
+      float m = -INFINITY, l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int j0 = 0; j0 < B; j0 += kPS)
+        attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
+                        d.scale_log2, m, l, acc, psw);
+      const float inv = __frcp_rn(l);
+      const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      const float Ls = (m + __log2f(l)) * kLn2;
+      if (r < 0) {
+        const float4 op = *reinterpret_cast<const float4*>(prm.o_p + grow * kD + 4 * lane);
+        float4 o;
+        float L;
+        lse_merge(op, prm.l_p[grow], os, Ls, o, L);
+        *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
+        if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+      } else {
+        float* dst = sfx + (r / CL) * kPartStride;
+        if (lane == 0) dst[0] = Ls;
+        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
+      }
+    }
+  }
+  if (A == 0) return;  // every row was stable; no cluster exchange follows
+  __syncthreads();
+
+  // ================= after the scan kernel ==================================
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- this CTA's rows (r % CL == rank): the row's k pages
+  if (!d.all_pages) {
+#pragma unroll 1
+    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
+      unsigned long long* best = mbuf + (kWarps + warp) * kCandCap;
+      merge_row<KP>(prm, r, sg, best, mbuf + warp * kCandCap);
       int32_t* dst = sel_own + (r / CL) * k;
+#pragma unroll 1
       for (int j = lane; j < k; j += 32) {  // pages in ascending order
         const int pj = key_index(best[j]);
         int rk = 0;
+#pragma unroll 4
         for (int u = 0; u < k; ++u) rk += key_index(best[u]) < pj;
         dst[rk] = pj;
         if (prm.page_idx) {
@@ -884,11 +1014,12 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       __syncwarp();
     }
   } else if (prm.page_idx) {
-    for (int e = tid; e < R * k; e += kThreads) {
-      const int r = e / k;
-      if (r % CL != rank) continue;
+#pragma unroll 1
+    for (int r = rank; r < R; r += CL) {
       const int hl = r / A, a = r % A;
-      prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + e % k] = e % k;
+#pragma unroll 1
+      for (int j = tid; j < k; j += kThreads)
+        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + j] = j;
     }
   }
   __syncthreads();
@@ -902,19 +1033,26 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       *s_nlp = nlp;
       if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
     }
+#pragma unroll 1
     for (int j = tid; j < min(nlp, prm.max_lp); j += kThreads) lpages[j] = rank + j * CL;
+#pragma unroll 1
     for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) {
       const int w = e % d.MW;
       const int nb = min(32, R - 32 * w);
       masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
     }
   } else {
+    const int rows_own = (R + CL - 1) / CL;
+#pragma unroll 1
     for (int e = tid; e < R * k; e += kThreads) {
-      const int r = e / k, j = e % k;
+      const int r = e / k, j = e - r * k;
       sel_all[e] = cluster.map_shared_rank(sel_own, r % CL)[(r / CL) * k + j];
     }
+    (void)rows_own;
+#pragma unroll 1
     for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
     __syncthreads();
+#pragma unroll 1
     for (int e = tid; e < R * k; e += kThreads) {
       const int p = sel_all[e];
       if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
@@ -925,14 +1063,16 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       const int per = (nwords + 31) / 32;
       const int w0 = lane * per, w1 = min(nwords, w0 + per);
       int sum = 0;
+#pragma unroll 1
       for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
       int incl = sum;
-#pragma unroll
+#pragma unroll 1
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
       int run = incl - sum;
+#pragma unroll 1
       for (int w = w0; w < w1; ++w) {
         wbase[w] = run;
         run += __popc(bitmap[w]);
@@ -946,9 +1086,11 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       *s_nlp = nlp;
       if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
     }
+#pragma unroll 1
     for (int w = tid; w < nwords; w += kThreads) {
       uint32_t bits = bitmap[w];
       int pos = wbase[w];
+#pragma unroll 1
       while (bits) {
         const int b = __ffs(bits) - 1;
         bits &= bits - 1;
@@ -956,8 +1098,10 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
         ++pos;
       }
     }
+#pragma unroll 1
     for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) masks[e] = 0u;
     __syncthreads();
+#pragma unroll 1
     for (int e = tid; e < R * k; e += kThreads) {
       const int p = sel_all[e];
       if (p < 0 || p >= d.P) continue;
@@ -975,10 +1119,12 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   // pages of rows r = w, w + 8, ... into their partials (one writer per row)
   {
     const int nlp = min(*s_nlp, prm.max_lp);
+#pragma unroll 1
     for (int b0 = 0; b0 < nlp && !*s_fail; b0 += prm.ngp) {
       const int nb = min(prm.ngp, nlp - b0);
       const int batch = b0 / prm.ngp;
       if (tid == 0) {
+#pragma unroll 1
         for (int i = 0; i < nb; ++i) {
           const int p = lpages[b0 + i];
           const int ntok = min(kPS, d.L - p * kPS);
@@ -990,15 +1136,17 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
           bulk_g2s(dst + pbytes, static_cast<const char*>(prm.V) + off, bytes, &mbar[i]);
         }
       }
-      float* psw = Ps + warp * 16;
+#pragma unroll 1
       for (int r = warp; r < R; r += kWarps) {
         bool have = false;
+#pragma unroll 1
         for (int i = 0; i < nb; ++i) have |= (masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u;
         if (!have) continue;
-        float4 q = row4<DT>(qa, r, lane);
+        const float4 q = row4<DT>(qa, r, lane);
         float* pr = part + r * kPartStride;
         float m = pr[0], l = pr[1];
         float4 acc = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+#pragma unroll 1
         for (int i = 0; i < nb; ++i) {
           if (!((masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u)) continue;
           if (!__all_sync(0xffffffffu, mbar_wait(&mbar[i], batch & 1))) {
@@ -1020,8 +1168,8 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
         }
         *reinterpret_cast<float4*>(pr + 4 + 4 * lane) = acc;
       }
-      // every barrier of this batch completes (waited by the warps that use
-      // its page) before the slots are refilled
+      // every copy of this batch has landed before the slots are refilled
+#pragma unroll 1
       for (int i = tid; i < nb; i += kThreads)
         if (!mbar_wait(&mbar[i], batch & 1)) *s_fail = 1;
       __syncthreads();
@@ -1031,19 +1179,21 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   cluster.sync();
 
   // ---- combine every CTA's partial of this CTA's rows, cache write-back,
-  // suffix and merge
-  // the block K/V copy is always waited for (no copy may land after exit)
-  const bool blk_ok = mbar_wait(&mbar[kMaxGatherPages], 0);
+  // merge with the suffix
   if (!*s_fail) {
-    float* psw = Ps + warp * 16;
-    for (int r = rank + CL * warp; r < R && blk_ok; r += CL * kWarps) {
+#pragma unroll 1
+    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
       float M = -INFINITY;
+#pragma unroll 1
       for (int c = 0; c < CL; ++c) M = fmaxf(M, cluster.map_shared_rank(part, c)[r * kPartStride]);
       float lsum = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
       for (int c = 0; c < CL; ++c) {  // fixed order: deterministic
         const float* pr = cluster.map_shared_rank(part, c) + r * kPartStride;
-        const float w = exp2f(pr[0] - M);
+        const float mc = pr[0];
+        if (mc == -INFINITY) continue;  // this CTA held none of the row's pages
+        const float w = exp2f(mc - M);
         lsum += w * pr[1];
         const float4 a = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
         acc.x += w * a.x;
@@ -1051,34 +1201,26 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
         acc.z += w * a.z;
         acc.w += w * a.w;
       }
-      const float inv = 1.f / lsum;
+      const float inv = __frcp_rn(lsum);
       const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
       const float Lp = (M + __log2f(lsum)) * kLn2;
       const int hl = r / A, t = act_tok[r];
-      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-      *reinterpret_cast<float4*>(prm.o_p + row * kD + 4 * lane) = op;
-      if (lane == 0) prm.l_p[row] = Lp;
-      // suffix of the active row over the block's own keys
-      const float4 q = row4<DT>(qa, r, lane);
-      float m2 = -INFINITY, l2 = 0.f;
-      float4 a2 = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int j0 = 0; j0 < B; j0 += kPS)
-        attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
-                        d.scale_log2, m2, l2, a2, psw);
-      const float inv2 = 1.f / l2;
-      const float4 os = make_float4(a2.x * inv2, a2.y * inv2, a2.z * inv2, a2.w * inv2);
-      const float Ls = (m2 + __log2f(l2)) * kLn2;
+      const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
+      *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
+      if (lane == 0) prm.l_p[grow] = Lp;
+      const float* sx = sfx + (r / CL) * kPartStride;
+      const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
       float4 o;
       float L;
-      lse_merge(op, Lp, os, Ls, o, L);
-      *reinterpret_cast<float4*>(prm.out + row * kD + 4 * lane) = o;
-      if (prm.out_lse && lane == 0) prm.out_lse[row] = L;
+      lse_merge(op, Lp, os, sx[0], o, L);
+      *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
+      if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
     }
-    if (!blk_ok && tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
   }
   // no CTA may leave while others can still read its shared memory
   cluster.sync();
 }
+
 // ---------------------------------------------------------------------------
 // host side: launch geometry, shared-memory layouts, attributes
 // ---------------------------------------------------------------------------
@@ -1099,11 +1241,13 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   prm->sc_stride = align_up(d.chunk_pages, 4) + 4;
   prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
   prm->kp = topk_width(d.k);
-  prm->tpr = d.R > 0 ? std::min(32, pow2_floor(std::max(1, kThreads / d.R))) : 1;
-  const bool selects = d.A > 0 && !d.all_pages;
-  if (selects && prm->kp == 0 && d.k > kCandCap) return false;
+  // a row's top-k group: at least k lanes, and enough lanes to cover the
+  // CTA's rows in few passes
+  prm->tpr = std::min(32, std::max(pow2_floor(std::max(1, kThreads / std::max(d.R, 1))),
+                                   d.k <= 1 ? 1 : pow2_floor(2 * d.k - 1)));
+  if (prm->kp > 0 && prm->tpr < d.k) return false;
+  if (prm->kp == 0 && d.k > kCandCap) return false;
   const int R16 = (d.R + 15) / 16 * 16;
-  const int Bpad = (d.B + kPS - 1) / kPS * kPS;
   const int GB = d.G * d.B;
   for (int ring = kMaxRingBytes; ring >= 64 * 1024; ring -= 32 * 1024) {
     ScanLayout& lo = prm->lo;
@@ -1115,13 +1259,13 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
       return o;
     };
     lo.ring = take(ring, 1024);
-    lo.scores = take(std::max(4LL * d.R * prm->sc_stride, 2LL * Bpad * kD * d.esz), 16);
+    // scores, or (before the scan) the staged queries
+    lo.scores = take(std::max(4LL * d.R * prm->sc_stride, 2LL * GB * prm->qw * 4), 16);
     lo.qrows = take(R16 * 512, 128);
-    lo.qstage = take(2LL * GB * prm->qw * 4, 16);
     lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
-    lo.ps = take(kWarps * 16 * 4, 16);
-    lo.cbuf = take(selects && prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
-    lo.mbar = take((kMaxStages + 1) * 8, 8);
+    lo.fbuf = take(prm->kp > 0 ? 8LL * (kThreads / prm->tpr) * kCandCap : 0, 16);
+    lo.cbuf = take(prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
+    lo.mbar = take(kMaxStages * 8, 8);
     lo.total = off;
     prm->stages = ring / kStageBytes;
     if (lo.total <= max_dyn) return true;
@@ -1131,15 +1275,16 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
 
 bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster) {
   prm->d = d;
-  int CL = std::min(max_cluster, std::max(1, d.Umax));
+  const int CL = std::min(max_cluster, std::max(1, std::max(d.Umax, 1)));
   prm->CL = CL;
   prm->max_lp = (d.Umax + CL - 1) / CL;
-  prm->kp = topk_width(d.k);
-  if (!d.all_pages && prm->kp == 0 && d.k > kCandCap) return false;
+  prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
+  if (!d.all_pages && d.A > 0 && topk_width(d.k) == 0 && d.k > kCandCap) return false;
   const int Bpad = (d.B + kPS - 1) / kPS * kPS;
   const int nwords = (d.P + 31) / 32;
   const int pbytes = kPS * kD * d.esz;
   const int rows_per_cta = (d.R + CL - 1) / CL;
+  const int GB = d.G * d.B;
   for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
     GatherLayout& lo = prm->lo;
     int off = 0;
@@ -1149,7 +1294,8 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster)
       off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
       return o;
     };
-    lo.slots = take(2LL * ngp * pbytes, 1024);
+    // staged queries first, gather pages later
+    lo.stage = take(std::max(2LL * ngp * pbytes, 2LL * GB * prm->qw * 4), 1024);
     lo.kbv = take(2LL * Bpad * kD * d.esz, 16);
     lo.qa = take(1LL * d.R * kD * d.esz, 16);
     lo.sel_own = take(d.all_pages ? 0 : 4LL * rows_per_cta * d.k, 16);
@@ -1159,10 +1305,10 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster)
     lo.lpages = take(prm->max_lp * 4, 16);
     lo.masks = take(4LL * prm->max_lp * d.MW, 16);
     lo.part = take(4LL * d.R * kPartStride, 16);
-    lo.misc = take((4 + kMaxRowsPerGroup) * 4, 16);
+    lo.sfx = take(4LL * rows_per_cta * kPartStride, 16);
+    lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
     lo.ps = take(kWarps * 16 * 4, 16);
-    // per-warp merge output (always) and compaction buffer (warp fallback)
-    lo.cbuf = take(2 * kWarps * kCandCap * 8, 16);
+    lo.mbuf = take(2 * kWarps * kCandCap * 8, 16);
     lo.mbar = take((kMaxGatherPages + 1) * 8, 8);
     lo.total = off;
     prm->ngp = ngp;
@@ -1193,12 +1339,42 @@ int probe_cluster() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, losa_gather_kernel<LOSA_BF16>, &cfg) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&n, losa_gather_kernel<LOSA_BF16, 8>, &cfg) == cudaSuccess &&
         n > 0)
       return cl;
     cudaGetLastError();  // clear a refused query
   }
   return 4;
+}
+
+template <int DT, int KP>
+cudaError_t set_attrs_one(int optin, int* dyn) {
+  const void* fns[2] = {reinterpret_cast<const void*>(losa_scan_kernel<DT, KP>),
+                        reinterpret_cast<const void*>(losa_gather_kernel<DT, KP>)};
+  for (int i = 0; i < 2; ++i) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, fns[i]);
+    if (e != cudaSuccess) return e;
+    const int mine = optin - static_cast<int>(fa.sharedSizeBytes);
+    e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
+    if (e != cudaSuccess) return e;
+    if (i == 1) {
+      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    *dyn = std::min(*dyn, mine);
+  }
+  return cudaSuccess;
+}
+
+template <int DT>
+cudaError_t set_attrs_dt(int optin, int* dyn) {
+  cudaError_t e;
+  if ((e = set_attrs_one<DT, 0>(optin, dyn)) != cudaSuccess) return e;
+  if ((e = set_attrs_one<DT, 2>(optin, dyn)) != cudaSuccess) return e;
+  if ((e = set_attrs_one<DT, 4>(optin, dyn)) != cudaSuccess) return e;
+  if ((e = set_attrs_one<DT, 8>(optin, dyn)) != cudaSuccess) return e;
+  return set_attrs_one<DT, 16>(optin, dyn);
 }
 
 int ensure_attributes(int* max_dyn, int* max_cluster) {
@@ -1211,24 +1387,9 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
     int optin = 0;
     e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e != cudaSuccess) return record_cuda_error(e);
-    const void* fns[] = {reinterpret_cast<const void*>(losa_scan_kernel<LOSA_BF16>),
-                         reinterpret_cast<const void*>(losa_scan_kernel<LOSA_F32>),
-                         reinterpret_cast<const void*>(losa_gather_kernel<LOSA_BF16>),
-                         reinterpret_cast<const void*>(losa_gather_kernel<LOSA_F32>)};
     int dyn = optin;
-    for (int i = 0; i < 4; ++i) {
-      cudaFuncAttributes fa;
-      e = cudaFuncGetAttributes(&fa, fns[i]);
-      if (e != cudaSuccess) return record_cuda_error(e);
-      const int mine = optin - static_cast<int>(fa.sharedSizeBytes);
-      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
-      if (e != cudaSuccess) return record_cuda_error(e);
-      if (i >= 2) {
-        e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return record_cuda_error(e);
-      }
-      dyn = std::min(dyn, mine);
-    }
+    if ((e = set_attrs_dt<LOSA_BF16>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
+    if ((e = set_attrs_dt<LOSA_F32>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
     g_attr_dyn[dev] = dyn;
     g_attr_cluster[dev] = probe_cluster();
     g_attr_done[dev] = true;
@@ -1238,12 +1399,35 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
   return LOSA_OK;
 }
 
+template <int DT, int KP>
+cudaError_t launch_pair(const cudaLaunchConfig_t* c1, const ScanParams& sp,
+                        const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+  if (c1) {
+    const cudaError_t e = cudaLaunchKernelEx(c1, losa_scan_kernel<DT, KP>, sp);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
+}
+
+template <int DT>
+cudaError_t launch_dt(int kp, const cudaLaunchConfig_t* c1, const ScanParams& sp,
+                      const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+  switch (kp) {
+    case 2: return launch_pair<DT, 2>(c1, sp, c2, gp);
+    case 4: return launch_pair<DT, 4>(c1, sp, c2, gp);
+    case 8: return launch_pair<DT, 8>(c1, sp, c2, gp);
+    case 16: return launch_pair<DT, 16>(c1, sp, c2, gp);
+    default: return launch_pair<DT, 0>(c1, sp, c2, gp);
+  }
+}
+
 }  // namespace
 
 bool fused_step_fits(const Dims& d, int max_dyn) {
   ScanParams sp;
   GatherParams gp;
-  return plan_scan(d, &sp, max_dyn) && (d.A == 0 || plan_gather(d, &gp, max_dyn, kMaxCluster));
+  const bool scan = d.A > 0 && !d.all_pages;
+  return (!scan || plan_scan(d, &sp, max_dyn)) && plan_gather(d, &gp, max_dyn, kMaxCluster);
 }
 
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
@@ -1256,39 +1440,27 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   if (rc != LOSA_OK) return rc;
   ScanParams sp;
   GatherParams gp;
-  if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
-  if (d.A > 0 && !plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
+  if (d.A > 0 && !d.all_pages && !plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
+  if (!plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
   if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
   char* ws = static_cast<char*>(workspace);
   int* status = reinterpret_cast<int*>(ws + d.off_status);
-  int32_t* act_tok = reinterpret_cast<int32_t*>(ws + d.off_act);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
 
   sp.qc = q_cur;
   sp.qp = q_prev;
   sp.meta = static_cast<const char*>(page_meta);
-  sp.kb = k_blk;
-  sp.vb = v_blk;
-  sp.o_p = o_p;
-  sp.l_p = l_p;
-  sp.out = out;
-  sp.out_lse = out_lse;
-  sp.active_idx = active_idx;
-  sp.union_count = union_count;
-  sp.act_tok_g = act_tok;
   sp.cand = cand;
   sp.status = status;
+  const bool scan = d.A > 0 && !d.all_pages;
   cudaLaunchConfig_t c1 = {};
   c1.gridDim = dim3(d.nchunk, d.S * d.Hkv, 1);
   c1.blockDim = dim3(kThreads, 1, 1);
   c1.dynamicSmemBytes = static_cast<size_t>(sp.lo.total);
   c1.stream = st;
-  cudaError_t e = d.dtype == LOSA_BF16 ? cudaLaunchKernelEx(&c1, losa_scan_kernel<LOSA_BF16>, sp)
-                                       : cudaLaunchKernelEx(&c1, losa_scan_kernel<LOSA_F32>, sp);
-  if (e != cudaSuccess) return record_cuda_error(e);
-  if (d.A == 0) return LOSA_OK;
 
   gp.qc = q_cur;
+  gp.qp = q_prev;
   gp.K = k_prefix;
   gp.V = v_prefix;
   gp.kb = k_blk;
@@ -1297,17 +1469,17 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   gp.l_p = l_p;
   gp.out = out;
   gp.out_lse = out_lse;
+  gp.active_idx = active_idx;
   gp.page_idx = page_idx;
   gp.union_count = union_count;
-  gp.act_tok_g = act_tok;
   gp.cand = cand;
   gp.status = status;
   cudaLaunchConfig_t c2 = {};
+  cudaLaunchAttribute attr[2];
   c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
   c2.blockDim = dim3(kThreads, 1, 1);
   c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
   c2.stream = st;
-  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = gp.CL;
   attr[0].val.clusterDim.y = 1;
@@ -1315,9 +1487,12 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   c2.attrs = attr;
-  c2.numAttrs = 2;
-  e = d.dtype == LOSA_BF16 ? cudaLaunchKernelEx(&c2, losa_gather_kernel<LOSA_BF16>, gp)
-                           : cudaLaunchKernelEx(&c2, losa_gather_kernel<LOSA_F32>, gp);
+  c2.numAttrs = scan ? 2 : 1;  // overlap with the scan kernel it depends on
+  // one top-k width per compiled kernel: the selection code of the others is
+  // never fetched
+  const int kp = scan ? sp.kp : 2;
+  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, scan ? &c1 : nullptr, sp, c2, gp)
+                                             : launch_dt<LOSA_F32>(kp, scan ? &c1 : nullptr, sp, c2, gp);
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
 
