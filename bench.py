@@ -188,8 +188,9 @@ def step_bytes(sh, union_counts, esz):
 
 
 def launches_per_step(sh):
-    """Kernels one losa_step launches: the fused step is a single launch."""
-    return 1
+    """Kernels one losa_step launches: the scan kernel always, the gather
+    kernel whenever some query row is active."""
+    return 2 if sh.n_active > 0 else 1
 
 
 # ---------------------------------------------------------------------------

@@ -10,8 +10,10 @@
 //    of one (sequence, KV head) group's pages.  It bulk-copies (TMA) the
 //    chunk's page metadata into a shared-memory ring and meanwhile computes
 //    the group's active set (every CTA of the group computes it, identically)
-//    and finishes its share of the group's stable rows (suffix attention over
-//    the block, merge with the untouched cache).  Then the QUEST bound of the
+//    and the suffix attention over the block of its share of the group's
+//    token rows: stable rows are finished here (merge with the untouched
+//    cache), active rows leave their suffix partial in the workspace.  With
+//    no active row (or k = P) that is all.  Otherwise the QUEST bound of the
 //    chunk's pages for the group's R active rows -- bf16: tensor cores,
 //    U = [q- | q+] . [kmin ; kmax] with mma.sync m16n8k16 (exact products,
 //    fp32 accumulation); fp32: CUDA cores, the sum in channel order with one
@@ -27,7 +29,7 @@
 //    the page into an online-softmax partial per row; finally each CTA
 //    combines its rows' partials from every CTA of the cluster (distributed
 //    shared memory), writes the new o_p / L_p to the cache and merges them
-//    with the suffix.
+//    with the suffix partial.  K2 is launched only when some row is active.
 //
 // Every wait on a bulk copy is bounded (clock64); a wait that gives up sets
 // LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA skips the rest of
@@ -295,11 +297,18 @@ __device__ __forceinline__ void thread_topk(KeyFn key, int j, int stride, int n,
 template <typename KeyFn>
 __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long long* buf,
                                   unsigned long long* out, int cap, bool active) {
+  constexpr int kNV = 32;  // keys a lane keeps in registers
   const int lane = threadIdx.x & 31;
   const int j = lane & (W - 1);
+  if (n > W * kNV) return false;  // (uniform) the caller's other path handles it
+  unsigned long long kx[kNV];
   unsigned long long lmax = 0ull;
-#pragma unroll 1
-  for (int i = j; i < n; i += W) lmax = umax64(lmax, key(i));
+#pragma unroll
+  for (int t = 0; t < kNV; ++t) {
+    const int i = j + t * W;
+    kx[t] = i < n ? key(i) : 0ull;
+    lmax = umax64(lmax, kx[t]);
+  }
   unsigned long long v = lmax;  // bitonic sort of the lane maxima, descending
 #pragma unroll 1
   for (int size = 2; size <= W; size <<= 1) {
@@ -312,11 +321,8 @@ __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long 
   }
   const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1, W);
   int cnt = 0;
-#pragma unroll 1
-  for (int i = j; i < n; i += W) {
-    const unsigned long long x = key(i);
-    cnt += (x >= tau && x != 0ull);
-  }
+#pragma unroll
+  for (int t = 0; t < kNV; ++t) cnt += (kx[t] >= tau && kx[t] != 0ull);
   int incl = cnt;
 #pragma unroll 1
   for (int o = 1; o < W; o <<= 1) {
@@ -327,11 +333,9 @@ __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long 
   if (!__all_sync(0xffffffffu, !active || total <= cap)) return false;
   if (active) {
     int pos = incl - cnt;
-#pragma unroll 1
-    for (int i = j; i < n; i += W) {
-      const unsigned long long x = key(i);
-      if (x >= tau && x != 0ull) buf[pos++] = x;
-    }
+#pragma unroll
+    for (int t = 0; t < kNV; ++t)
+      if (kx[t] >= tau && kx[t] != 0ull) buf[pos++] = kx[t];
   }
   __syncwarp();
   if (active) {
@@ -339,7 +343,7 @@ __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long 
     for (int t = j; t < total; t += W) {
       const unsigned long long x = buf[t];
       int rank = 0;
-#pragma unroll 4
+#pragma unroll 8
       for (int m = 0; m < total; ++m) rank += buf[m] > x;
       if (rank < k) out[rank] = x;
     }
@@ -361,13 +365,23 @@ int align_up(int x, int a) { return (x + a - 1) / a * a; }
 // K1: scan
 // ---------------------------------------------------------------------------
 struct ScanLayout {
-  int ring, scores, qrows, misc, fbuf, cbuf, mbar, total;
+  int ring, scores, kbv, qrows, misc, ps, fbuf, cbuf, mbar, total;
 };
 
 struct ScanParams {
   const void* qc;
   const void* qp;
   const char* meta;
+  const void* kb;
+  const void* vb;
+  const float* o_p;
+  const float* l_p;
+  float* out;
+  float* out_lse;
+  int32_t* active_idx;
+  int32_t* union_count;
+  int32_t* act_tok_g;              // workspace [S*Hkv][R]
+  float* sfx_g;                    // workspace [S*Hkv][R][kPartStride]: active rows' suffix
   unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
   int* status;
   Dims d;
@@ -440,6 +454,8 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
   const int GB = G * B;
   const int qw = prm.qw;
+  const int esz = DT == LOSA_BF16 ? 2 : 4;
+  const int Bpad = (B + kPS - 1) / kPS * kPS;
 
   // let the gather kernel start its own preparation now; it waits for this
   // grid's completion before it reads anything written here
@@ -449,7 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   float* sc = reinterpret_cast<float*>(smem + lo.scores);
   uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.scores);  // staging; aliases sc
   uint32_t* qps = qcs + GB * qw;
+  char* kbv = smem + lo.kbv;  // the block's own K then V (element type)
   char* qrows = smem + lo.qrows;
+  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   unsigned long long* fbuf = reinterpret_cast<unsigned long long*>(smem + lo.fbuf);
   unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
@@ -463,14 +481,24 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int npages = max(0, min(d.P, p0 + d.chunk_pages) - p0);
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.P * prm.rec;
-  if (npages == 0) return;
+  const bool scan = A > 0 && !d.all_pages && npages > 0;
+  // token-rows of the group whose suffix this CTA computes: i = chunk + n * nchunk
+  const int n_mine = GB > chunk ? (GB - chunk + nchunk - 1) / nchunk : 0;
+  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
 
   if (tid == 0) {
-    for (int i = 0; i < kMaxStages; ++i) mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
+    if (n_mine > 0) {
+      mbar_expect_tx(&mbar[kMaxStages], 2 * blk_bytes);
+      const size_t off = static_cast<size_t>(sg) * B * kD * esz;
+      bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxStages]);
+      bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
+               &mbar[kMaxStages]);
+    }
 #pragma unroll 1
-    for (int t = 0; t < min(ntiles, prm.stages); ++t) {
+    for (int t = 0; scan && t < min(ntiles, prm.stages); ++t) {
       const int np = min(prm.tile, npages - t * prm.tile);
       const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
       mbar_expect_tx(&mbar[t], bytes);
@@ -482,7 +510,6 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   // ---- stage the group's current / previous queries (coalesced), padded
   // rows so that one thread walking its row in channel order hits every bank
   {
-    const int esz = DT == LOSA_BF16 ? 2 : 4;
     const int cpr = kD * esz / 16;  // 16-byte chunks per row
     const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
     const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
@@ -545,8 +572,66 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   __syncthreads();
   if (tid < GB) act_slot[tid] = my_slot;
   __syncthreads();
-  if (tid < GB && act_slot[tid] >= 0) act_tok[(tid / B) * A + act_slot[tid]] = tid % B;
+  if (tid < GB && act_slot[tid] >= 0) {
+    const int hl = tid / B, r = hl * A + act_slot[tid];
+    act_tok[r] = tid % B;
+    if (chunk == 0) {
+      prm.act_tok_g[static_cast<size_t>(sg) * R + r] = tid % B;
+      if (prm.active_idx)
+        prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = tid % B;
+    }
+  }
+  if (chunk == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
   __syncthreads();
+
+  // ---- suffix over the block of this CTA's token-rows (hidden under the
+  // metadata stream): stable rows are finished here (merge with their
+  // untouched cache); active rows leave (o_s, L_s) in the workspace
+  if (n_mine > 0) {
+    if (!mbar_wait(&mbar[kMaxStages], 0)) {
+      if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+    } else {
+      float* psw = Ps + warp * 16;
+#pragma unroll 1
+      for (int n = warp; n < n_mine; n += kWarps) {
+        const int i = chunk + n * nchunk;
+        const int slot = act_slot[i];
+        const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G) * B + i;
+        float4 q;
+        if (DT == LOSA_BF16) {
+          const uint32_t w0 = qcs[i * qw + 2 * lane], w1 = qcs[i * qw + 2 * lane + 1];
+          q = make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
+                          __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
+        } else {
+          const uint32_t* w = qcs + i * qw + 4 * lane;
+          q = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
+                          __uint_as_float(w[3]));
+        }
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
+                          d.scale_log2, m, l, acc, psw);
+        const float inv = __frcp_rn(l);
+        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        const float Ls = (m + __log2f(l)) * kLn2;
+        if (slot < 0) {
+          const float4 op = *reinterpret_cast<const float4*>(prm.o_p + grow * kD + 4 * lane);
+          float4 o;
+          float L;
+          lse_merge(op, prm.l_p[grow], os, Ls, o, L);
+          *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
+          if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+        } else {
+          float* dst = prm.sfx_g + (static_cast<size_t>(sg) * R + (i / B) * A + slot) * kPartStride;
+          if (lane == 0) dst[0] = Ls;
+          *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
+        }
+      }
+    }
+  }
+  if (!scan) return;
 
   // ---- active rows' queries for the bound: bf16 -> [R16][256] = [q- | q+]
   // in swizzled 16-byte chunks (ldmatrix); fp32 -> [R][128]
@@ -677,20 +762,17 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
 }
 
 // ---------------------------------------------------------------------------
-// K2: active set, suffix, stable rows; then select, union, gather, combine
+// K2: select, union, gather, combine
 // ---------------------------------------------------------------------------
 struct GatherLayout {
-  int stage, kbv, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, sfx, misc, ps, mbuf,
-      mbar, total;
+  int stage, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf, mbar,
+      total;
 };
 
 struct GatherParams {
   const void* qc;
-  const void* qp;
   const void* K;
   const void* V;
-  const void* kb;
-  const void* vb;
   float* o_p;
   float* l_p;
   float* out;
@@ -698,6 +780,8 @@ struct GatherParams {
   int32_t* active_idx;
   int32_t* page_idx;
   int32_t* union_count;
+  const int32_t* act_tok_g;
+  const float* sfx_g;
   const unsigned long long* cand;
   int* status;
   Dims d;
@@ -813,16 +897,10 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
   const int esz = DT == LOSA_BF16 ? 2 : 4;
-  const int Bpad = (B + kPS - 1) / kPS * kPS;
   const int pbytes = kPS * kD * esz;
   const int nwords = (d.P + 31) / 32;
-  const int GB = G * B;
-  const int qw = prm.qw;
 
-  char* slots = smem + lo.stage;  // gather pages, once the staged queries are done with
-  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.stage);
-  uint32_t* qps = qcs + GB * qw;
-  char* kbv = smem + lo.kbv;
+  char* slots = smem + lo.stage;  // gather pages
   char* qa = smem + lo.qa;  // [R][kD] active rows' queries, element type
   int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
   int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel_all);
@@ -831,7 +909,6 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
-  float* sfx = reinterpret_cast<float*>(smem + lo.sfx);    // this CTA's active rows' suffix
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
@@ -839,158 +916,35 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   int32_t* s_fail = misc;
   int32_t* s_U = misc + 1;
   int32_t* s_nlp = misc + 2;
-  float* s_mse = reinterpret_cast<float*>(misc + 4);
-  int32_t* act_slot = misc + 4 + kMaxRowsPerGroup;
-  int32_t* act_tok = act_slot + kMaxRowsPerGroup;
-  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
+  int32_t* act_tok = misc + 4;  // [R]
   float* psw = Ps + warp * 16;
 
-  // ================= preparation (independent of the scan kernel) ==========
   if (tid == 0) {
-    for (int i = 0; i < kMaxGatherPages + 1; ++i) mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxGatherPages; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    mbar_expect_tx(&mbar[kMaxGatherPages], 2 * blk_bytes);  // the block's own K/V
-    const size_t off = static_cast<size_t>(sg) * B * kD * esz;
-    bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxGatherPages]);
-    bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
-             &mbar[kMaxGatherPages]);
-  }
-  {  // stage the group's current / previous queries (padded rows)
-    const int cpr = kD * esz / 16;
-    const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
-    const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
-    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + base);
-#pragma unroll 2
-    for (int e = tid; e < GB * cpr; e += kThreads) {
-      const int row = e / cpr, c = e % cpr;
-      const uint4 a = gc[e], b = gp[e];
-      uint32_t* x = qcs + row * qw + 4 * c;
-      uint32_t* y = qps + row * qw + 4 * c;
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
-    }
   }
 #pragma unroll 1
   for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
     part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
-  __syncthreads();
-  // locality score (fp32, one rounding per operation, channels in order) and
-  // active set -- the same computation, in the same order, as the scan kernel
-  if (tid < GB) {
-    const uint32_t* x = qcs + tid * qw;
-    const uint32_t* y = qps + tid * qw;
-    float acc = 0.f;
-    if (DT == LOSA_BF16) {
-#pragma unroll 8
-      for (int w = 0; w < kD / 2; ++w) {
-        const uint32_t a = x[w], b = y[w];
-        const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
-        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-        const float d1 = __fsub_rn(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u));
-        acc = __fadd_rn(acc, __fmul_rn(d1, d1));
-      }
-    } else {
-#pragma unroll 8
-      for (int w = 0; w < kD; ++w) {
-        const float d0 = __fsub_rn(__uint_as_float(x[w]), __uint_as_float(y[w]));
-        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-      }
-    }
-    s_mse[tid] = acc * (1.0f / kD);
-  }
-  __syncthreads();
-  if (tid < GB) {
-    const int hl = tid / B, t = tid % B;
-    const float x = s_mse[tid];
-    int rk = 0;
-#pragma unroll 4
-    for (int u = 0; u < B; ++u) {
-      const float y = s_mse[hl * B + u];
-      rk += (y > x) || (y == x && u < t);
-    }
-    act_slot[tid] = rk < A ? 1 : 0;
-  }
-  __syncthreads();
-  int my_slot = -1;
-  if (tid < GB && act_slot[tid]) {
-    const int hl = tid / B, t = tid % B;
-    my_slot = 0;
-#pragma unroll 1
-    for (int u = 0; u < t; ++u) my_slot += act_slot[hl * B + u];
-  }
-  __syncthreads();
-  if (tid < GB) act_slot[tid] = my_slot;
-  __syncthreads();
-  if (tid < GB && act_slot[tid] >= 0) {
-    const int hl = tid / B;
-    act_tok[hl * A + act_slot[tid]] = tid % B;
-    if (rank == 0 && prm.active_idx)
-      prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = tid % B;
-  }
-  if (rank == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
-  __syncthreads();
-  {  // active rows' queries in the element type
-    const int wpr = kD * esz / 4;  // 32-bit words per row
-#pragma unroll 1
-    for (int e = tid; e < R * wpr; e += kThreads) {
-      const int r = e / wpr, w = e % wpr;
-      const int row = (r / A) * B + act_tok[r];
-      reinterpret_cast<uint32_t*>(qa)[e] = qcs[row * qw + w];
-    }
-  }
-  // suffix over the block: stable token-rows i with i % CL == rank are
-  // finished here (merge with their untouched cache); active rows r with
-  // r % CL == rank keep (o_s, L_s) for the final merge
-  const bool blk_ok = mbar_wait(&mbar[kMaxGatherPages], 0);
-  if (!blk_ok && tid == 0) {
-    atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-    *s_fail = 1;
-  }
-  if (blk_ok) {
-    const int n_st = GB > rank ? (GB - rank + CL - 1) / CL : 0;
-    const int n_ac = R > rank ? (R - rank + CL - 1) / CL : 0;
-#pragma unroll 1
-    for (int job = warp; job < n_st + n_ac; job += kWarps) {
-      int row, r = -1;
-      if (job < n_st) {
-        const int i = rank + job * CL;
-        if (act_slot[i] >= 0) continue;
-        row = i;
-      } else {
-        r = rank + (job - n_st) * CL;
-        row = (r / A) * B + act_tok[r];
-      }
-      const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G) * B + row;
-      const float4 q = qrow4<DT>(qcs, row, qw, lane);
-      float m = -INFINITY, l = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-      for (int j0 = 0; j0 < B; j0 += kPS)
-        attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
-                        d.scale_log2, m, l, acc, psw);
-      const float inv = __frcp_rn(l);
-      const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      const float Ls = (m + __log2f(l)) * kLn2;
-      if (r < 0) {
-        const float4 op = *reinterpret_cast<const float4*>(prm.o_p + grow * kD + 4 * lane);
-        float4 o;
-        float L;
-        lse_merge(op, prm.l_p[grow], os, Ls, o, L);
-        *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
-        if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
-      } else {
-        float* dst = sfx + (r / CL) * kPartStride;
-        if (lane == 0) dst[0] = Ls;
-        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
-      }
-    }
-  }
-  if (A == 0) return;  // every row was stable; no cluster exchange follows
-  __syncthreads();
 
-  // ================= after the scan kernel ==================================
+  // everything below reads what the scan kernel wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
+
+#pragma unroll 1
+  for (int r = tid; r < R; r += kThreads)
+    act_tok[r] = __ldcg(prm.act_tok_g + static_cast<size_t>(sg) * R + r);
+  __syncthreads();
+  {  // active rows' queries (element type)
+    const int cpr = kD * esz / 16;
+#pragma unroll 1
+    for (int e = tid; e < R * cpr; e += kThreads) {
+      const int r = e / cpr, c = e - r * cpr;
+      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + r / A) * B + act_tok[r];
+      reinterpret_cast<uint4*>(qa)[e] =
+          reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + row * kD * esz)[c];
+    }
+  }
 
   // ---- this CTA's rows (r % CL == rank): the row's k pages
   if (!d.all_pages) {
@@ -1208,11 +1162,11 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
       *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
       if (lane == 0) prm.l_p[grow] = Lp;
-      const float* sx = sfx + (r / CL) * kPartStride;
-      const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
+      const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
+      const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4 + 4 * lane));
       float4 o;
       float L;
-      lse_merge(op, Lp, os, sx[0], o, L);
+      lse_merge(op, Lp, os, __ldcg(sx), o, L);
       *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
       if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
     }
@@ -1245,8 +1199,9 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   // CTA's rows in few passes
   prm->tpr = std::min(32, std::max(pow2_floor(std::max(1, kThreads / std::max(d.R, 1))),
                                    d.k <= 1 ? 1 : pow2_floor(2 * d.k - 1)));
-  if (prm->kp > 0 && prm->tpr < d.k) return false;
-  if (prm->kp == 0 && d.k > kCandCap) return false;
+  const bool selects = d.A > 0 && !d.all_pages;
+  if (selects && prm->kp > 0 && prm->tpr < d.k) return false;
+  if (selects && prm->kp == 0 && d.k > kCandCap) return false;
   const int R16 = (d.R + 15) / 16 * 16;
   const int GB = d.G * d.B;
   for (int ring = kMaxRingBytes; ring >= 64 * 1024; ring -= 32 * 1024) {
@@ -1261,11 +1216,13 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
     lo.ring = take(ring, 1024);
     // scores, or (before the scan) the staged queries
     lo.scores = take(std::max(4LL * d.R * prm->sc_stride, 2LL * GB * prm->qw * 4), 16);
+    lo.kbv = take(2LL * ((d.B + kPS - 1) / kPS * kPS) * kD * d.esz, 16);
     lo.qrows = take(R16 * 512, 128);
     lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
+    lo.ps = take(kWarps * 16 * 4, 16);
     lo.fbuf = take(prm->kp > 0 ? 8LL * (kThreads / prm->tpr) * kCandCap : 0, 16);
     lo.cbuf = take(prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
-    lo.mbar = take(kMaxStages * 8, 8);
+    lo.mbar = take((kMaxStages + 1) * 8, 8);
     lo.total = off;
     prm->stages = ring / kStageBytes;
     if (lo.total <= max_dyn) return true;
@@ -1280,11 +1237,9 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster)
   prm->max_lp = (d.Umax + CL - 1) / CL;
   prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
   if (!d.all_pages && d.A > 0 && topk_width(d.k) == 0 && d.k > kCandCap) return false;
-  const int Bpad = (d.B + kPS - 1) / kPS * kPS;
   const int nwords = (d.P + 31) / 32;
   const int pbytes = kPS * kD * d.esz;
   const int rows_per_cta = (d.R + CL - 1) / CL;
-  const int GB = d.G * d.B;
   for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
     GatherLayout& lo = prm->lo;
     int off = 0;
@@ -1294,9 +1249,7 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster)
       off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
       return o;
     };
-    // staged queries first, gather pages later
-    lo.stage = take(std::max(2LL * ngp * pbytes, 2LL * GB * prm->qw * 4), 1024);
-    lo.kbv = take(2LL * Bpad * kD * d.esz, 16);
+    lo.stage = take(2LL * ngp * pbytes, 1024);
     lo.qa = take(1LL * d.R * kD * d.esz, 16);
     lo.sel_own = take(d.all_pages ? 0 : 4LL * rows_per_cta * d.k, 16);
     lo.sel_all = take(d.all_pages ? 0 : 4LL * d.R * d.k, 16);
@@ -1305,11 +1258,10 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster)
     lo.lpages = take(prm->max_lp * 4, 16);
     lo.masks = take(4LL * prm->max_lp * d.MW, 16);
     lo.part = take(4LL * d.R * kPartStride, 16);
-    lo.sfx = take(4LL * rows_per_cta * kPartStride, 16);
-    lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
+    lo.misc = take((4 + kMaxRowsPerGroup) * 4, 16);
     lo.ps = take(kWarps * 16 * 4, 16);
     lo.mbuf = take(2 * kWarps * kCandCap * 8, 16);
-    lo.mbar = take((kMaxGatherPages + 1) * 8, 8);
+    lo.mbar = take(kMaxGatherPages * 8, 8);
     lo.total = off;
     prm->ngp = ngp;
     if (lo.total <= std::min(max_dyn, kGatherSmemTarget) || (ngp == 1 && lo.total <= max_dyn))
@@ -1400,18 +1352,16 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
 }
 
 template <int DT, int KP>
-cudaError_t launch_pair(const cudaLaunchConfig_t* c1, const ScanParams& sp,
-                        const cudaLaunchConfig_t& c2, const GatherParams& gp) {
-  if (c1) {
-    const cudaError_t e = cudaLaunchKernelEx(c1, losa_scan_kernel<DT, KP>, sp);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
+cudaError_t launch_pair(const cudaLaunchConfig_t& c1, const ScanParams& sp,
+                        const cudaLaunchConfig_t* c2, const GatherParams& gp) {
+  const cudaError_t e = cudaLaunchKernelEx(&c1, losa_scan_kernel<DT, KP>, sp);
+  if (e != cudaSuccess || !c2) return e;
+  return cudaLaunchKernelEx(c2, losa_gather_kernel<DT, KP>, gp);
 }
 
 template <int DT>
-cudaError_t launch_dt(int kp, const cudaLaunchConfig_t* c1, const ScanParams& sp,
-                      const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+cudaError_t launch_dt(int kp, const cudaLaunchConfig_t& c1, const ScanParams& sp,
+                      const cudaLaunchConfig_t* c2, const GatherParams& gp) {
   switch (kp) {
     case 2: return launch_pair<DT, 2>(c1, sp, c2, gp);
     case 4: return launch_pair<DT, 4>(c1, sp, c2, gp);
@@ -1426,8 +1376,7 @@ cudaError_t launch_dt(int kp, const cudaLaunchConfig_t* c1, const ScanParams& sp
 bool fused_step_fits(const Dims& d, int max_dyn) {
   ScanParams sp;
   GatherParams gp;
-  const bool scan = d.A > 0 && !d.all_pages;
-  return (!scan || plan_scan(d, &sp, max_dyn)) && plan_gather(d, &gp, max_dyn, kMaxCluster);
+  return plan_scan(d, &sp, max_dyn) && (d.A == 0 || plan_gather(d, &gp, max_dyn, kMaxCluster));
 }
 
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
@@ -1440,19 +1389,30 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   if (rc != LOSA_OK) return rc;
   ScanParams sp;
   GatherParams gp;
-  if (d.A > 0 && !d.all_pages && !plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
-  if (!plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
+  if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
+  if (d.A > 0 && !plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
   if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
   char* ws = static_cast<char*>(workspace);
   int* status = reinterpret_cast<int*>(ws + d.off_status);
+  int32_t* act_tok = reinterpret_cast<int32_t*>(ws + d.off_act);
+  float* sfx = reinterpret_cast<float*>(ws + d.off_sfx);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
 
   sp.qc = q_cur;
   sp.qp = q_prev;
   sp.meta = static_cast<const char*>(page_meta);
+  sp.kb = k_blk;
+  sp.vb = v_blk;
+  sp.o_p = o_p;
+  sp.l_p = l_p;
+  sp.out = out;
+  sp.out_lse = out_lse;
+  sp.active_idx = active_idx;
+  sp.union_count = union_count;
+  sp.act_tok_g = act_tok;
+  sp.sfx_g = sfx;
   sp.cand = cand;
   sp.status = status;
-  const bool scan = d.A > 0 && !d.all_pages;
   cudaLaunchConfig_t c1 = {};
   c1.gridDim = dim3(d.nchunk, d.S * d.Hkv, 1);
   c1.blockDim = dim3(kThreads, 1, 1);
@@ -1460,39 +1420,40 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   c1.stream = st;
 
   gp.qc = q_cur;
-  gp.qp = q_prev;
   gp.K = k_prefix;
   gp.V = v_prefix;
-  gp.kb = k_blk;
-  gp.vb = v_blk;
   gp.o_p = o_p;
   gp.l_p = l_p;
   gp.out = out;
   gp.out_lse = out_lse;
-  gp.active_idx = active_idx;
   gp.page_idx = page_idx;
   gp.union_count = union_count;
+  gp.act_tok_g = act_tok;
+  gp.sfx_g = sfx;
   gp.cand = cand;
   gp.status = status;
   cudaLaunchConfig_t c2 = {};
   cudaLaunchAttribute attr[2];
-  c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
-  c2.blockDim = dim3(kThreads, 1, 1);
-  c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
-  c2.stream = st;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = gp.CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  c2.attrs = attr;
-  c2.numAttrs = scan ? 2 : 1;  // overlap with the scan kernel it depends on
+  if (d.A > 0) {
+    c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
+    c2.blockDim = dim3(kThreads, 1, 1);
+    c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
+    c2.stream = st;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = gp.CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
+    c2.attrs = attr;
+    c2.numAttrs = 2;
+  }
   // one top-k width per compiled kernel: the selection code of the others is
   // never fetched
-  const int kp = scan ? sp.kp : 2;
-  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, scan ? &c1 : nullptr, sp, c2, gp)
-                                             : launch_dt<LOSA_F32>(kp, scan ? &c1 : nullptr, sp, c2, gp);
+  const int kp = (d.A > 0 && !d.all_pages) ? sp.kp : 2;
+  const cudaLaunchConfig_t* c2p = d.A > 0 ? &c2 : nullptr;
+  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, c1, sp, c2p, gp)
+                                             : launch_dt<LOSA_F32>(kp, c1, sp, c2p, gp);
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
 
