@@ -98,13 +98,11 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
     d->chunk_pages = static_cast<int>(chunk);
     d->nchunk = static_cast<int>((P + chunk - 1) / chunk);
   }
-  // workspace: status word, the active tokens of every group, the active
-  // rows' suffix attention, and the chunk candidates (selection keys) of
-  // every (group, chunk, active row)
+  // workspace: status word, the active set of every group (active tokens,
+  // then every token's active slot or -1), and the chunk candidates
+  // (selection keys) of every (group, chunk, active row)
   d->off_act = off;
-  off += align256(SG * R * sizeof(int32_t));
-  d->off_sfx = off;
-  off += align256(SG * R * kPartStride * sizeof(float));
+  off += align256(SG * (R + static_cast<size_t>(G) * d->B) * sizeof(int32_t));
   d->off_cand = off;
   off += align256(SG * d->nchunk * R * K * sizeof(unsigned long long));
   d->total = off;

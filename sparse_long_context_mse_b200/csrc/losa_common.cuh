@@ -35,7 +35,7 @@ struct Dims {
   int nsplit, split_pages;
   int nchunk, chunk_pages;
   // workspace byte offsets
-  size_t off_status, off_part, off_act, off_sfx, off_cand, total;
+  size_t off_status, off_part, off_act, off_cand, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).

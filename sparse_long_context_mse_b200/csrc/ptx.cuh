@@ -1,5 +1,6 @@
 // ptx.cuh -- inline-PTX wrappers shared by the LoSA kernels (sm_100a):
-// mbarriers, non-multicast bulk copies (TMA), cp.async, ldmatrix, mma.sync.
+// mbarriers, non-multicast bulk copies (TMA), cp.async, ldmatrix, mma.sync,
+// cluster barriers.
 #pragma once
 
 #include <stdint.h>
@@ -77,12 +78,29 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
                "r"(src_bytes)
                : "memory");
 }
+// 4-byte global -> shared copy (for sources that need not be 16-byte aligned).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Thread-block-cluster barrier, split into its two halves.  Every thread of
+// every CTA of the cluster arrives, then waits; the release/acquire pair
+// orders shared-memory writes made before the arrive (including writes to
+// other CTAs' shared memory) before reads made after the wait.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Two fp32 values -> packed bf16x2 (round to nearest even), low half first.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -6,35 +6,38 @@
 // prefix attention, dense intra-block suffix, online-softmax merge, cache
 // update.
 //
-// K1 `losa_scan_kernel` -- a flat grid over every SM: each CTA owns one chunk
-//    of one (sequence, KV head) group's pages.  It bulk-copies (TMA) the
-//    chunk's page metadata into a shared-memory ring and meanwhile computes
-//    the group's active set (every CTA of the group computes it, identically)
-//    and the suffix attention over the block of its share of the group's
-//    token rows: stable rows are finished here (merge with the untouched
-//    cache), active rows leave their suffix partial in the workspace.  With
-//    no active row (or k = P) that is all.  Otherwise the QUEST bound of the
-//    chunk's pages for the group's R active rows -- bf16: tensor cores,
-//    U = [q- | q+] . [kmin ; kmax] with mma.sync m16n8k16 (exact products,
-//    fp32 accumulation); fp32: CUDA cores, the sum in channel order with one
-//    rounding per operation -- and a chunk-local top-k per row, written to the
-//    workspace.
+// K1 `losa_scan_kernel` -- a flat grid over the SMs: each CTA owns one chunk
+//    of one (sequence, KV head) group's pages.  At launch it bulk-copies (TMA)
+//    the group's current and previous queries and the chunk's page metadata
+//    into shared memory; the locality score (lanes split a row's channels)
+//    and the active set (one warp per head, lane = token) follow as soon as
+//    the queries land, then the QUEST bound of the chunk's pages for the
+//    group's R active rows -- bf16: tensor cores, U = [q- | q+] . [kmin ;
+//    kmax] with mma.sync m16n8k16 (exact products, fp32 accumulation, the
+//    A operand held in registers); fp32: CUDA cores, the sum in channel order
+//    with one rounding per operation -- and a chunk-local top-k per row into
+//    the workspace.  The first CTA of a group also stores the active set.
 // K2 `losa_gather_kernel` -- one thread-block cluster per group, launched
-//    with programmatic dependent launch behind K1.  Rows are dealt to the
-//    cluster's CTAs; each merges its rows' chunk candidates into the row's
-//    top-k pages; every CTA then builds the group's page union (bitmap,
-//    ascending, with a row mask per page) from the rows' lists in
-//    distributed shared memory; union slot u belongs to CTA u % CL, which
-//    bulk-copies the page's K and V once for the whole GQA group and folds
-//    the page into an online-softmax partial per row; finally each CTA
-//    combines its rows' partials from every CTA of the cluster (distributed
-//    shared memory), writes the new o_p / L_p to the cache and merges them
-//    with the suffix partial.  K2 is launched only when some row is active.
+//    with programmatic dependent launch behind K1.  Each CTA stages the
+//    block's K/V before K1 has finished; then it merges the chunk candidates
+//    of its rows into the row's k pages and writes them into every CTA of the
+//    cluster (distributed shared memory).  Every CTA builds the group's page
+//    union (ascending, with a row mask per page); union slot u belongs to CTA
+//    u % CL, which copies the page's K and V once for the whole GQA group.
+//    While the copies fly the CTA computes the dense suffix of its share of
+//    the block's token rows (stable rows are merged with their untouched
+//    cache and finished here).  The pages are then folded into one
+//    online-softmax partial per row -- bf16: tensor cores, all rows of an
+//    m16 tile at once with a row mask, S = Q K^T and O += P V with P split
+//    into bf16 high and remainder parts; fp32: one warp per row on CUDA cores
+//    -- and each active row's owner CTA combines the partials of every CTA
+//    of the cluster, writes the new o_p / L_p and merges them with the
+//    row's suffix.
 //
-// Every wait on a bulk copy is bounded (clock64); a wait that gives up sets
-// LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA skips the rest of
-// its work but still takes part in every cluster barrier, so the cluster
-// never deadlocks.  There is no other cross-CTA wait.
+// K1's waits on bulk copies are bounded (clock64); a wait that gives up sets
+// LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA stops.  K2 waits on
+// cp.async groups and cluster barriers only; every CTA of a cluster takes
+// every cluster barrier.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -57,6 +60,7 @@ constexpr int kMaxStages = kMaxRingBytes / kStageBytes;
 constexpr int kCandCap = 64;                     // per-warp compaction buffer
 constexpr int kMaxCluster = 16;
 constexpr int kMaxGatherPages = 16;              // pages in flight per K2 CTA
+constexpr int kGatherSmemTarget = 113 * 1024;    // two gather CTAs per SM
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
   return a > b ? a : b;
@@ -77,7 +81,7 @@ __device__ __forceinline__ float4 row4(const char* base, int j, int lane) {
 // Online-softmax update of one row (lane owns 4 channels) with `ntok` <= 16
 // keys/values of a page held in shared memory in element type DT.
 template <int DT>
-__device__ __noinline__ void attend_page(float4 q, const char* Ks, const char* Vs, int ntok,
+__device__ __forceinline__ void attend_page(float4 q, const char* Ks, const char* Vs, int ntok,
                                             float scale_log2, float& m, float& l, float4& acc,
                                             float* Ps) {
   const int lane = threadIdx.x & 31;
@@ -138,6 +142,26 @@ __device__ __noinline__ void attend_page(float4 q, const char* Ks, const char* V
   m = m_new;
 }
 
+// The k-th largest (1 <= k <= W) of the values held by the W lanes of an
+// aligned lane group (W a power of two, the same for the whole warp): every
+// lane ranks its value against the group's (ties by lane), and the lane of
+// rank k-1 holds the answer.  The W shuffles are independent, so they
+// overlap instead of forming a chain.
+__device__ __forceinline__ unsigned long long group_kth_u64(unsigned long long v, int W, int k) {
+  const int lane = threadIdx.x & 31, j = lane & (W - 1), base = lane - j;
+  int rk = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    if (i < W) {
+      const unsigned long long o = __shfl_sync(0xffffffffu, v, base + i);
+      rk += (o > v) || (o == v && i < j);
+    }
+  }
+  const unsigned bal = __ballot_sync(0xffffffffu, rk == k - 1);
+  const unsigned grp = W == 32 ? bal : ((bal >> base) & ((1u << W) - 1u));
+  return __shfl_sync(0xffffffffu, v, base + __ffs(grp) - 1);
+}
+
 // ---------------------------------------------------------------------------
 // Warp top-k over n selection keys key(i), i in [0, n): writes the k largest
 // keys, descending, to out[0..k) (0 = empty slot when n < k).  Fast path:
@@ -153,19 +177,7 @@ __device__ void warp_topk(KeyFn key, int n, int k, unsigned long long* out,
   for (int i = lane; i < n; i += 32) lmax = umax64(lmax, key(i));
   bool done = false;
   if (k <= 32) {
-    // bitonic sort of the 32 local maxima, descending (lane 0 largest)
-    unsigned long long v = lmax;
-#pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
-        const bool dir = (lane & size) == 0;
-        const bool lower = (lane & stride) == 0;
-        v = (lower == dir) ? umax64(v, o) : (v < o ? v : o);
-      }
-    }
-    const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1);
+    const unsigned long long tau = group_kth_u64(lmax, 32, k);
     int cnt = 0;
     for (int i = lane; i < n; i += 32) cnt += key(i) >= tau && key(i) != 0;
     int incl = cnt;
@@ -309,17 +321,7 @@ __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long 
     kx[t] = i < n ? key(i) : 0ull;
     lmax = umax64(lmax, kx[t]);
   }
-  unsigned long long v = lmax;  // bitonic sort of the lane maxima, descending
-#pragma unroll 1
-  for (int size = 2; size <= W; size <<= 1) {
-#pragma unroll 1
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
-      const bool dir = (j & size) == 0, lower = (j & stride) == 0;
-      v = (lower == dir) ? umax64(v, o) : (v < o ? v : o);
-    }
-  }
-  const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1, W);
+  const unsigned long long tau = group_kth_u64(lmax, W, k);
   int cnt = 0;
 #pragma unroll
   for (int t = 0; t < kNV; ++t) cnt += (kx[t] >= tau && kx[t] != 0ull);
@@ -361,37 +363,49 @@ int pow2_floor(int x) {
 }
 int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
+// Byte offset of 16-byte chunk c of row j inside a [rows][kD] tile: bf16 tiles
+// XOR-swizzle the chunks by row (conflict-free ldmatrix), fp32 tiles are plain.
+template <int DT>
+__device__ __forceinline__ int tile_off(int j, int c) {
+  return DT == LOSA_BF16 ? j * 256 + ((c ^ (j & 7)) << 4) : j * 512 + c * 16;
+}
+
+// fp32 sum of squared differences of two bf16x2 / f32 words, in channel order.
+__device__ __forceinline__ float sqd_bf16x2(uint32_t a, uint32_t b, float acc) {
+  const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
+  acc = __fadd_rn(acc, __fmul_rn(d0, d0));
+  const float d1 = __fsub_rn(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u));
+  return __fadd_rn(acc, __fmul_rn(d1, d1));
+}
+__device__ __forceinline__ float sqd_f32(uint32_t a, uint32_t b, float acc) {
+  const float d0 = __fsub_rn(__uint_as_float(a), __uint_as_float(b));
+  return __fadd_rn(acc, __fmul_rn(d0, d0));
+}
+
 // ---------------------------------------------------------------------------
 // K1: scan
 // ---------------------------------------------------------------------------
 struct ScanLayout {
-  int ring, scores, kbv, qrows, misc, ps, fbuf, cbuf, mbar, total;
+  int ring, qc, qps, qrows, misc, fbuf, cbuf, mbar, total;
 };
 
 struct ScanParams {
   const void* qc;
   const void* qp;
   const char* meta;
-  const void* kb;
-  const void* vb;
-  const float* o_p;
-  const float* l_p;
-  float* out;
-  float* out_lse;
+  int32_t* act_g;                  // workspace [S*Hkv][R + G*B]: act_tok, then act_slot
   int32_t* active_idx;
-  int32_t* union_count;
-  int32_t* act_tok_g;              // workspace [S*Hkv][R]
-  float* sfx_g;                    // workspace [S*Hkv][R][kPartStride]: active rows' suffix
   unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
   int* status;
   Dims d;
+  int scan;       // this launch scores pages (else: the active set only)
   int rec;        // bytes per metadata record
   int tile;       // pages per ring stage
   int stages;     // ring stages
   int sc_stride;  // floats per score row
-  int qw;         // 32-bit words per staged query row (padded)
   int kp;         // register top-k width (2..16), 0 = warp fallback
   int tpr;        // threads per row for the chunk top-k
+  int mse_t;      // threads per row for the locality score
   ScanLayout lo;
 };
 
@@ -442,63 +456,72 @@ __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* s
   }
 }
 
+// Bound scores of one 8-page n-tile for the 16 rows of the A fragments:
+// acc[0..1] = rows g4, pages 2*t4, 2*t4+1; acc[2..3] = row g4 + 8.  `rec0`
+// points to the tile's first record; records are [kmin | kmax] with 16-byte
+// chunks swizzled by the page index (which is congruent to the record index
+// mod 8 inside a ring stage).
+__device__ __forceinline__ void bound_ntile(const uint32_t (&a)[16][4], const char* rec0,
+                                            float (&acc)[4]) {
+  const int lane = threadIdx.x & 31;
+  const int pg = lane & 7;
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 16; ks += 2) {
+    uint32_t b0, b1, b2, b3;
+    const int ch = ks * 2 + (lane >> 3);
+    ldsm_x4(su32(rec0 + pg * 512 + ((ch ^ pg) << 4)), b0, b1, b2, b3);
+    mma_bf16(acc, a[ks], b0, b1);
+    mma_bf16(acc, a[ks + 1], b2, b3);
+  }
+}
+
 template <int DT, int KP>
 __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams prm) {
   extern __shared__ __align__(1024) char smem[];
   const Dims& d = prm.d;
   const ScanLayout& lo = prm.lo;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, nchunk = gridDim.x;
+  const int chunk = blockIdx.x;
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
   const int GB = G * B;
-  const int qw = prm.qw;
-  const int esz = DT == LOSA_BF16 ? 2 : 4;
-  const int Bpad = (B + kPS - 1) / kPS * kPS;
+  constexpr int rowb = DT == LOSA_BF16 ? kD * 2 : kD * 4;
 
-  // let the gather kernel start its own preparation now; it waits for this
-  // grid's completion before it reads anything written here
+  // the gather kernel may start staging now; it waits for this grid's
+  // completion before it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   char* ring = smem + lo.ring;
-  float* sc = reinterpret_cast<float*>(smem + lo.scores);
-  uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + lo.scores);  // staging; aliases sc
-  uint32_t* qps = qcs + GB * qw;
-  char* kbv = smem + lo.kbv;  // the block's own K then V (element type)
+  const char* qcs = smem + lo.qc;
+  const char* qps = smem + lo.qps;
+  float* sc = reinterpret_cast<float*>(smem + lo.qps);  // scores, after the locality pass
   char* qrows = smem + lo.qrows;
-  float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   unsigned long long* fbuf = reinterpret_cast<unsigned long long*>(smem + lo.fbuf);
   unsigned long long* cbuf = reinterpret_cast<unsigned long long*>(smem + lo.cbuf);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
   int32_t* s_fail = misc;
   float* s_mse = reinterpret_cast<float*>(misc + 4);
-  int32_t* act_slot = misc + 4 + kMaxRowsPerGroup;
-  int32_t* act_tok = act_slot + kMaxRowsPerGroup;
+  int32_t* act_tok = misc + 4 + kMaxRowsPerGroup;
 
   const int p0 = chunk * d.chunk_pages;
-  const int npages = max(0, min(d.P, p0 + d.chunk_pages) - p0);
+  const int npages = prm.scan ? max(0, min(d.P, p0 + d.chunk_pages) - p0) : 0;
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.P * prm.rec;
-  const bool scan = A > 0 && !d.all_pages && npages > 0;
-  // token-rows of the group whose suffix this CTA computes: i = chunk + n * nchunk
-  const int n_mine = GB > chunk ? (GB - chunk + nchunk - 1) / nchunk : 0;
-  const uint32_t blk_bytes = static_cast<uint32_t>(B * kD * esz);
+  const uint32_t qbytes = static_cast<uint32_t>(GB * rowb);
 
   if (tid == 0) {
     for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    if (n_mine > 0) {
-      mbar_expect_tx(&mbar[kMaxStages], 2 * blk_bytes);
-      const size_t off = static_cast<size_t>(sg) * B * kD * esz;
-      bulk_g2s(kbv, static_cast<const char*>(prm.kb) + off, blk_bytes, &mbar[kMaxStages]);
-      bulk_g2s(kbv + Bpad * kD * esz, static_cast<const char*>(prm.vb) + off, blk_bytes,
-               &mbar[kMaxStages]);
-    }
+    const size_t qoff = (static_cast<size_t>(s) * d.Hq + g * G) * B * rowb;
+    mbar_expect_tx(&mbar[kMaxStages], 2 * qbytes);
+    bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, &mbar[kMaxStages]);
+    bulk_g2s(smem + lo.qps, static_cast<const char*>(prm.qp) + qoff, qbytes, &mbar[kMaxStages]);
 #pragma unroll 1
-    for (int t = 0; scan && t < min(ntiles, prm.stages); ++t) {
+    for (int t = 0; t < min(ntiles, prm.stages); ++t) {
       const int np = min(prm.tile, npages - t * prm.tile);
       const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
       mbar_expect_tx(&mbar[t], bytes);
@@ -506,132 +529,75 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
                bytes, &mbar[t]);
     }
   }
+  __syncthreads();
+  if (!mbar_wait(&mbar[kMaxStages], 0)) *s_fail = 1;
+  __syncthreads();
+  if (*s_fail) {
+    if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+    return;
+  }
 
-  // ---- stage the group's current / previous queries (coalesced), padded
-  // rows so that one thread walking its row in channel order hits every bank
+  // ---- locality score: mse_t lanes per row, each summing its channels in
+  // order (fp32, one rounding per operation), then a shuffle tree
   {
-    const int cpr = kD * esz / 16;  // 16-byte chunks per row
-    const size_t base = (static_cast<size_t>(s) * d.Hq + g * G) * B * kD * esz;
-    const uint4* gc = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + base);
-    const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qp) + base);
-#pragma unroll 2
-    for (int e = tid; e < GB * cpr; e += kThreads) {
-      const int row = e / cpr, c = e % cpr;
-      const uint4 a = gc[e], b = gp[e];
-      uint32_t* x = qcs + row * qw + 4 * c;
-      uint32_t* y = qps + row * qw + 4 * c;
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-      y[0] = b.x; y[1] = b.y; y[2] = b.z; y[3] = b.w;
-    }
-  }
-  __syncthreads();
-
-  // ---- locality score: fp32, one rounding per operation, channels in order
-  if (tid < GB) {
-    const uint32_t* x = qcs + tid * qw;
-    const uint32_t* y = qps + tid * qw;
+    const int T = prm.mse_t;
+    const int row = tid / T, part = tid % T;
     float acc = 0.f;
-    if (DT == LOSA_BF16) {
-#pragma unroll 8
-      for (int w = 0; w < kD / 2; ++w) {
-        const uint32_t a = x[w], b = y[w];
-        const float d0 = __fsub_rn(__uint_as_float(a << 16), __uint_as_float(b << 16));
-        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-        const float d1 = __fsub_rn(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u));
-        acc = __fadd_rn(acc, __fmul_rn(d1, d1));
-      }
-    } else {
-#pragma unroll 8
-      for (int w = 0; w < kD; ++w) {
-        const float d0 = __fsub_rn(__uint_as_float(x[w]), __uint_as_float(y[w]));
-        acc = __fadd_rn(acc, __fmul_rn(d0, d0));
-      }
-    }
-    s_mse[tid] = acc * (1.0f / kD);  // exact: kD is a power of two
-  }
-  __syncthreads();
-  if (tid < GB) {  // rank within the head: ties go to the lower token index
-    const int hl = tid / B, t = tid % B;
-    const float x = s_mse[tid];
-    int rk = 0;
+    if (row < GB) {
+      constexpr int cpr = rowb / 16;
+      const uint4* x = reinterpret_cast<const uint4*>(qcs + row * rowb);
+      const uint4* y = reinterpret_cast<const uint4*>(qps + row * rowb);
 #pragma unroll 4
-    for (int u = 0; u < B; ++u) {
-      const float y = s_mse[hl * B + u];
-      rk += (y > x) || (y == x && u < t);
+      for (int c = part; c < cpr; c += T) {
+        const uint4 a = x[c], b = y[c];
+        if (DT == LOSA_BF16) {
+          acc = sqd_bf16x2(a.x, b.x, acc);
+          acc = sqd_bf16x2(a.y, b.y, acc);
+          acc = sqd_bf16x2(a.z, b.z, acc);
+          acc = sqd_bf16x2(a.w, b.w, acc);
+        } else {
+          acc = sqd_f32(a.x, b.x, acc);
+          acc = sqd_f32(a.y, b.y, acc);
+          acc = sqd_f32(a.z, b.z, acc);
+          acc = sqd_f32(a.w, b.w, acc);
+        }
+      }
     }
-    act_slot[tid] = rk < A ? 1 : 0;
-  }
-  __syncthreads();
-  int my_slot = -1;
-  if (tid < GB && act_slot[tid]) {  // slot = active tokens before t in the head
-    const int hl = tid / B, t = tid % B;
-    my_slot = 0;
 #pragma unroll 1
-    for (int u = 0; u < t; ++u) my_slot += act_slot[hl * B + u];
+    for (int o = 1; o < T; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (row < GB && part == 0) s_mse[row] = acc * (1.0f / kD);  // exact: kD is a power of two
   }
-  __syncthreads();
-  if (tid < GB) act_slot[tid] = my_slot;
-  __syncthreads();
-  if (tid < GB && act_slot[tid] >= 0) {
-    const int hl = tid / B, r = hl * A + act_slot[tid];
-    act_tok[r] = tid % B;
-    if (chunk == 0) {
-      prm.act_tok_g[static_cast<size_t>(sg) * R + r] = tid % B;
-      if (prm.active_idx)
-        prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + hl) * A + act_slot[tid]] = tid % B;
-    }
-  }
-  if (chunk == 0 && tid == 0 && A == 0 && prm.union_count) prm.union_count[sg] = 0;
   __syncthreads();
 
-  // ---- suffix over the block of this CTA's token-rows (hidden under the
-  // metadata stream): stable rows are finished here (merge with their
-  // untouched cache); active rows leave (o_s, L_s) in the workspace
-  if (n_mine > 0) {
-    if (!mbar_wait(&mbar[kMaxStages], 0)) {
-      if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-    } else {
-      float* psw = Ps + warp * 16;
+  // ---- active set: one warp per head, lane = token; rank by (mse desc,
+  // token asc), slot = active tokens before it
+  {
+    int32_t* act_g = prm.act_g + static_cast<size_t>(sg) * (R + GB);
 #pragma unroll 1
-      for (int n = warp; n < n_mine; n += kWarps) {
-        const int i = chunk + n * nchunk;
-        const int slot = act_slot[i];
-        const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G) * B + i;
-        float4 q;
-        if (DT == LOSA_BF16) {
-          const uint32_t w0 = qcs[i * qw + 2 * lane], w1 = qcs[i * qw + 2 * lane + 1];
-          q = make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
-                          __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
-        } else {
-          const uint32_t* w = qcs + i * qw + 4 * lane;
-          q = make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
-                          __uint_as_float(w[3]));
-        }
-        float m = -INFINITY, l = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-        for (int j0 = 0; j0 < B; j0 += kPS)
-          attend_page<DT>(q, kbv + j0 * kD * esz, kbv + (Bpad + j0) * kD * esz, min(kPS, B - j0),
-                          d.scale_log2, m, l, acc, psw);
-        const float inv = __frcp_rn(l);
-        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        const float Ls = (m + __log2f(l)) * kLn2;
-        if (slot < 0) {
-          const float4 op = *reinterpret_cast<const float4*>(prm.o_p + grow * kD + 4 * lane);
-          float4 o;
-          float L;
-          lse_merge(op, prm.l_p[grow], os, Ls, o, L);
-          *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
-          if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
-        } else {
-          float* dst = prm.sfx_g + (static_cast<size_t>(sg) * R + (i / B) * A + slot) * kPartStride;
-          if (lane == 0) dst[0] = Ls;
-          *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
+    for (int h = warp; h < G; h += kWarps) {
+      const float x = lane < B ? s_mse[h * B + lane] : 0.f;
+      int rk = 0;
+#pragma unroll 4
+      for (int u = 0; u < B; ++u) {
+        const float y = s_mse[h * B + u];
+        rk += (y > x) || (y == x && u < lane);
+      }
+      const bool act = lane < B && rk < A;
+      const unsigned bal = __ballot_sync(0xffffffffu, act);
+      const int slot = __popc(bal & ((1u << lane) - 1u));
+      if (act) act_tok[h * A + slot] = lane;
+      if (chunk == 0) {
+        if (lane < B) act_g[R + h * B + lane] = act ? slot : -1;
+        if (act) {
+          act_g[h * A + slot] = lane;
+          if (prm.active_idx)
+            prm.active_idx[(static_cast<size_t>(s) * d.Hq + g * G + h) * A + slot] = lane;
         }
       }
     }
   }
-  if (!scan) return;
+  __syncthreads();
+  if (npages == 0) return;
 
   // ---- active rows' queries for the bound: bf16 -> [R16][256] = [q- | q+]
   // in swizzled 16-byte chunks (ldmatrix); fp32 -> [R][128]
@@ -643,12 +609,12 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (r < R) {
         const int row = (r / A) * B + act_tok[r];
-        const uint32_t* src = qcs + row * qw + 4 * (c & 15);
+        const uint4 w4 = *reinterpret_cast<const uint4*>(qcs + row * rowb + (c & 15) * 16);
+        const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t o[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t w = src[u];
-          uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
+          uint32_t lo16 = w[u] & 0xffffu, hi16 = w[u] >> 16;
           const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
           if (c < 16) {  // q- = min(q, 0)
             lo16 = nl ? lo16 : 0u;
@@ -668,62 +634,99 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     for (int e = tid; e < R * kD; e += kThreads) {
       const int r = e / kD, c = e % kD;
       const int row = (r / A) * B + act_tok[r];
-      reinterpret_cast<uint32_t*>(qrows)[r * kD + c] = qcs[row * qw + c];
+      reinterpret_cast<uint32_t*>(qrows)[r * kD + c] =
+          reinterpret_cast<const uint32_t*>(qcs + row * rowb)[c];
     }
   }
-  __syncthreads();  // the staging area becomes the score area below
+  __syncthreads();  // the previous queries' staging area becomes the score area
 
   // ---- bound scores of the chunk
-  const int ntm = R16 / 16;
-#pragma unroll 1
-  for (int t = 0; t < ntiles; ++t) {
-    const int st = t % prm.stages;
-    const uint32_t parity = (t / prm.stages) & 1;
-    if (!mbar_wait(&mbar[st], parity)) {
-      atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-      *s_fail = 1;
+  if (DT == LOSA_BF16) {
+    const int ntm = R16 / 16;         // 1..8
+    const int wpm = kWarps / ntm;     // warps per m16 tile
+    const int mt = warp / wpm, sub = warp % wpm;
+    const bool sw = mt < ntm;
+    const int g4 = lane >> 2, t4 = lane & 3;
+    uint32_t a[16][4];
+    if (sw) {
+      const int mi = lane >> 3, row = mt * 16 + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const int ch = ks * 2 + (mi >> 1);
+        ldsm_x4(su32(qrows + row * 512 + ((ch ^ (row & 7)) << 4)), a[ks][0], a[ks][1], a[ks][2],
+                a[ks][3]);
+      }
     }
-    __syncthreads();
-    if (*s_fail) return;  // no cluster here: leaving early is safe
-    const char* tile = ring + st * kStageBytes;
-    const int np = min(prm.tile, npages - t * prm.tile);
-    const int pl0 = t * prm.tile;
-    if (DT == LOSA_BF16) {
-      const int ntn = (np + 7) / 8;
-      const int g4 = lane >> 2, t4 = lane & 3;
+    const int r0 = mt * 16 + g4;
+    auto put = [&](const float (&acc)[4], int pc) {  // pc: chunk page of the lane's pair
+      if (r0 < R) {
+        sc[r0 * prm.sc_stride + pc] = acc[0];
+        sc[r0 * prm.sc_stride + pc + 1] = acc[1];
+      }
+      if (r0 + 8 < R) {
+        sc[(r0 + 8) * prm.sc_stride + pc] = acc[2];
+        sc[(r0 + 8) * prm.sc_stride + pc + 1] = acc[3];
+      }
+    };
+    if (ntiles <= prm.stages) {
+      // every stage was issued at launch: each warp runs through its n-tiles,
+      // two at a time, waiting only for the stage that holds them
+      const int nnt = (npages + 7) / 8;
+      const int ntpt = prm.tile / 8;  // n-tiles per stage
 #pragma unroll 1
-      for (int job = warp; job < ntn * ntm; job += kWarps) {
-        const int nt = job % ntn, mt = job / ntn;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 16; ks += 2) {
-          uint32_t b[4];
-          {
-            const int mi = lane >> 3, pg = nt * 8 + (lane & 7);
-            const int ch = ks * 2 + mi;
-            ldsm_x4(su32(tile + pg * 512 + ((ch ^ (pg & 7)) << 4)), b[0], b[1], b[2], b[3]);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            uint32_t a[4];
-            const int mi = lane >> 3;
-            const int row = mt * 16 + (mi & 1) * 8 + (lane & 7);
-            const int ch = (ks + kk) * 2 + (mi >> 1);
-            ldsm_x4(su32(qrows + row * 512 + ((ch ^ (row & 7)) << 4)), a[0], a[1], a[2], a[3]);
-            mma_bf16(acc, a, b[2 * kk], b[2 * kk + 1]);
-          }
+      for (int nt = sub; sw && nt < nnt; nt += 2 * wpm) {
+        const int nu = nt + wpm < nnt ? nt + wpm : nt;
+        const int t0 = nt / ntpt, t1 = nu / ntpt;
+        if (!mbar_wait(&mbar[t0], 0) || !mbar_wait(&mbar[t1], 0)) {
+          *s_fail = 1;
+          break;
         }
-        const int r0 = mt * 16 + g4, pc = pl0 + nt * 8 + 2 * t4;
-        if (r0 < R) {
-          sc[r0 * prm.sc_stride + pc] = acc[0];
-          sc[r0 * prm.sc_stride + pc + 1] = acc[1];
+        float acc0[4], acc1[4];
+        bound_ntile(a, ring + t0 * kStageBytes + (nt - t0 * ntpt) * 8 * 512, acc0);
+        bound_ntile(a, ring + t1 * kStageBytes + (nu - t1 * ntpt) * 8 * 512, acc1);
+        put(acc0, nt * 8 + 2 * t4);
+        if (nu != nt) put(acc1, nu * 8 + 2 * t4);
+      }
+      __syncthreads();
+    } else {
+#pragma unroll 1
+      for (int t = 0; t < ntiles; ++t) {
+        const int st = t % prm.stages;
+        const uint32_t parity = (t / prm.stages) & 1;
+        if (!mbar_wait(&mbar[st], parity)) *s_fail = 1;
+        __syncthreads();
+        if (*s_fail) break;
+        const int np = min(prm.tile, npages - t * prm.tile);
+        const int ntn = (np + 7) / 8;
+#pragma unroll 1
+        for (int nt = sub; sw && nt < ntn; nt += wpm) {
+          float acc[4];
+          bound_ntile(a, ring + st * kStageBytes + nt * 8 * 512, acc);
+          put(acc, t * prm.tile + nt * 8 + 2 * t4);
         }
-        if (r0 + 8 < R) {
-          sc[(r0 + 8) * prm.sc_stride + pc] = acc[2];
-          sc[(r0 + 8) * prm.sc_stride + pc + 1] = acc[3];
+        __syncthreads();
+        if (tid == 0 && t + prm.stages < ntiles) {  // refill the stage just consumed
+          const int tn = t + prm.stages;
+          const int npn = min(prm.tile, npages - tn * prm.tile);
+          const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
+          mbar_expect_tx(&mbar[st], bytes);
+          bulk_g2s(ring + st * kStageBytes,
+                   meta_g + static_cast<size_t>(p0 + tn * prm.tile) * prm.rec, bytes, &mbar[st]);
         }
       }
-    } else {
+      __syncthreads();
+    }
+  } else {
+#pragma unroll 1
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % prm.stages;
+      const uint32_t parity = (t / prm.stages) & 1;
+      if (!mbar_wait(&mbar[st], parity)) *s_fail = 1;
+      __syncthreads();
+      if (*s_fail) break;
+      const char* tile = ring + st * kStageBytes;
+      const int np = min(prm.tile, npages - t * prm.tile);
+      const int pl0 = t * prm.tile;
 #pragma unroll 1
       for (int e = tid; e < np * R; e += kThreads) {
         const int pl = e % np, r = e / np;
@@ -744,51 +747,217 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
         }
         sc[r * prm.sc_stride + pl0 + pl] = acc;
       }
+      __syncthreads();
+      if (tid == 0 && t + prm.stages < ntiles) {
+        const int tn = t + prm.stages;
+        const int npn = min(prm.tile, npages - tn * prm.tile);
+        const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
+        mbar_expect_tx(&mbar[st], bytes);
+        bulk_g2s(ring + st * kStageBytes, meta_g + static_cast<size_t>(p0 + tn * prm.tile) * prm.rec,
+                 bytes, &mbar[st]);
+      }
     }
     __syncthreads();
-    if (tid == 0 && t + prm.stages < ntiles) {  // refill the stage just consumed
-      const int tn = t + prm.stages;
-      const int npn = min(prm.tile, npages - tn * prm.tile);
-      const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
-      mbar_expect_tx(&mbar[st], bytes);
-      bulk_g2s(ring + st * kStageBytes, meta_g + static_cast<size_t>(p0 + tn * prm.tile) * prm.rec,
-               bytes, &mbar[st]);
-    }
+  }
+  if (*s_fail) {
+    if (tid == 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+    return;
   }
 
   // ---- chunk-local top-k per row -> workspace
-  unsigned long long* dst = prm.cand + (static_cast<size_t>(sg) * nchunk + chunk) * R * k;
+  unsigned long long* dst = prm.cand + (static_cast<size_t>(sg) * gridDim.x + chunk) * R * k;
   chunk_topk<DT, KP>(prm, sc, R, k, npages, p0, dst, fbuf, cbuf);
 }
 
 // ---------------------------------------------------------------------------
-// K2: select, union, gather, combine
+// Tensor-core attention of one m16 tile of query rows (bf16).  One warp holds
+// the tile's state: lane (g4 = lane / 4, t4 = lane % 4) keeps rows g4 and
+// g4 + 8 -- the running max m (base-2 units of the scaled score), its share
+// of the running sum l (the four lanes of a row are summed at the end), and
+// o[n][0..1] (row g4), o[n][2..3] (row g4 + 8) = channels 8n + 2*t4, +1 of
+// the unnormalised output.
+// ---------------------------------------------------------------------------
+struct TileAcc {
+  float m[2], l[2];
+  float o[16][4];
+};
+
+__device__ __forceinline__ void tile_init(TileAcc& t) {
+  t.m[0] = t.m[1] = -INFINITY;
+  t.l[0] = t.l[1] = 0.f;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) t.o[n][0] = t.o[n][1] = t.o[n][2] = t.o[n][3] = 0.f;
+}
+
+// Fold one page (K, V: [16][256 B] bf16, chunks swizzled by key) into the
+// state of the 16 query rows at q16 ([16][256 B], swizzled).  Row i of the
+// tile takes part iff bit i of `rows` is set; keys >= ntok are masked (their
+// V rows must be finite: the loaders zero-fill them).
+__device__ __forceinline__ void tile_attend(TileAcc& t, const char* q16, const char* Kp,
+                                         const char* Vp, uint32_t rows, int ntok, float sl2) {
+  const int lane = threadIdx.x & 31, g4 = lane >> 2, t4 = lane & 3;
+  float s[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ks += 2) {
+    uint32_t a0[4], a1[4];
+    {
+      const int mi = lane >> 3, row = (mi & 1) * 8 + (lane & 7);
+      const int ch0 = ks * 2 + (mi >> 1), ch1 = ch0 + 2;
+      ldsm_x4(su32(q16 + row * 256 + ((ch0 ^ (row & 7)) << 4)), a0[0], a0[1], a0[2], a0[3]);
+      ldsm_x4(su32(q16 + row * 256 + ((ch1 ^ (row & 7)) << 4)), a1[0], a1[1], a1[2], a1[3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t b0, b1, b2, b3;
+      const int key = nt * 8 + (lane & 7), ch = ks * 2 + (lane >> 3);
+      ldsm_x4(su32(Kp + key * 256 + ((ch ^ (key & 7)) << 4)), b0, b1, b2, b3);
+      mma_bf16(s[nt], a0, b0, b1);
+      mma_bf16(s[nt], a1, b2, b3);
+    }
+  }
+  const bool okA = (rows >> g4) & 1u, okB = (rows >> (g4 + 8)) & 1u;
+  float mxA = -INFINITY, mxB = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const bool kv = nt * 8 + 2 * t4 + c < ntok;
+      s[nt][c] = (okA && kv) ? s[nt][c] * sl2 : -INFINITY;
+      s[nt][2 + c] = (okB && kv) ? s[nt][2 + c] * sl2 : -INFINITY;
+      mxA = fmaxf(mxA, s[nt][c]);
+      mxB = fmaxf(mxB, s[nt][2 + c]);
+    }
+  }
+  mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 1));
+  mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 1));
+  mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 2));
+  mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 2));
+  const float mnA = fmaxf(t.m[0], mxA), mnB = fmaxf(t.m[1], mxB);
+  // a row that has seen no key yet keeps m = -inf and exponentiates against 0
+  const float uA = mnA == -INFINITY ? 0.f : mnA, uB = mnB == -INFINITY ? 0.f : mnB;
+  const float alA = exp2f(t.m[0] - uA), alB = exp2f(t.m[1] - uB);
+  t.m[0] = mnA;
+  t.m[1] = mnB;
+  float psA = 0.f, psB = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      s[nt][c] = exp2f(s[nt][c] - uA);
+      s[nt][2 + c] = exp2f(s[nt][2 + c] - uB);
+      psA += s[nt][c];
+      psB += s[nt][2 + c];
+    }
+  }
+  t.l[0] = t.l[0] * alA + psA;
+  t.l[1] = t.l[1] * alB + psB;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    t.o[n][0] *= alA;
+    t.o[n][1] *= alA;
+    t.o[n][2] *= alB;
+    t.o[n][3] *= alB;
+  }
+  // P (16 rows x 16 keys) as the A operand: bf16 high part and remainder
+  uint32_t ah[4], al[4];
+  {
+    const float pv[8] = {s[0][0], s[0][1], s[0][2], s[0][3], s[1][0], s[1][1], s[1][2], s[1][3]};
+    float rem[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rem[i] = pv[i] - __bfloat162float(__float2bfloat16_rn(pv[i]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ah[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+      al[i] = pack_bf16x2(rem[2 * i], rem[2 * i + 1]);
+    }
+  }
+#pragma unroll
+  for (int np = 0; np < 8; ++np) {
+    uint32_t b0, b1, b2, b3;
+    const int key = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int ch = 2 * np + (lane >> 4);
+    ldsm_x4_trans(su32(Vp + key * 256 + ((ch ^ (key & 7)) << 4)), b0, b1, b2, b3);
+    mma_bf16(t.o[2 * np], ah, b0, b1);
+    mma_bf16(t.o[2 * np + 1], ah, b2, b3);
+    mma_bf16(t.o[2 * np], al, b0, b1);
+    mma_bf16(t.o[2 * np + 1], al, b2, b3);
+  }
+}
+
+// Sum the four lanes' shares of l.
+__device__ __forceinline__ void tile_finish(TileAcc& t) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    t.l[h] += __shfl_xor_sync(0xffffffffu, t.l[h], 1);
+    t.l[h] += __shfl_xor_sync(0xffffffffu, t.l[h], 2);
+  }
+}
+
+// Partial of the tile's rows i < nrows -> base[i] = (m, l, -, -, o[128]).
+__device__ __forceinline__ void tile_store(const TileAcc& t, float* base, int nrows) {
+  const int lane = threadIdx.x & 31, g4 = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = g4 + 8 * h;
+    if (i >= nrows) continue;
+    float* pr = base + i * kPartStride;
+    if (t4 == 0) {
+      pr[0] = t.m[h];
+      pr[1] = t.l[h];
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(pr + 4 + n * 8 + 2 * t4) = make_float2(t.o[n][2 * h], t.o[n][2 * h + 1]);
+  }
+}
+
+// Merge of two normalised attentions (o1, L1), (o2, L2) (natural-log units).
+__device__ __forceinline__ void lse_weights(float L1, float L2, float& a, float& b, float& L) {
+  const float m = fmaxf(L1, L2);
+  const float x = __expf(L1 - m), y = __expf(L2 - m);
+  const float inv = __frcp_rn(x + y);
+  a = x * inv;
+  b = y * inv;
+  L = m + __logf(x + y);
+}
+
+// ---------------------------------------------------------------------------
+// K2: select, union, gather, suffix, combine
 // ---------------------------------------------------------------------------
 struct GatherLayout {
-  int stage, qa, sel_own, sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf, mbar,
-      total;
+  int region;   // gathered pages; afterwards the per-warp partials
+  int kbv;      // the block's K then V (bpad rows each)
+  int qa;       // active rows' queries (bf16: [R16][256 B] swizzled; fp32: [R][512 B])
+  int qs;       // this CTA's suffix rows' queries (same formats)
+  int ocache;   // cached o_p rows of this CTA's stable suffix rows
+  int lcache;   // their cached L_p
+  int sel_own, sel_all, bitmap, wbase, lpages, masks, part, sfx, misc, ps, mbuf, total;
 };
 
 struct GatherParams {
   const void* qc;
   const void* K;
   const void* V;
+  const void* kb;
+  const void* vb;
   float* o_p;
   float* l_p;
   float* out;
   float* out_lse;
-  int32_t* active_idx;
   int32_t* page_idx;
   int32_t* union_count;
-  const int32_t* act_tok_g;
-  const float* sfx_g;
+  const int32_t* act_g;
   const unsigned long long* cand;
   int* status;
   Dims d;
   int CL;        // CTAs per cluster
   int max_lp;    // max union pages per CTA
   int ngp;       // pages in flight per CTA
-  int qw;        // 32-bit words per staged query row (padded)
+  int n_oa;      // max active rows owned per CTA
+  int n_os;      // max stable suffix rows per CTA
+  int wpart;     // bf16: warps split pages and keep per-warp partials
   GatherLayout lo;
 };
 
@@ -819,22 +988,12 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg
       merge_top<KQ>(x, y);
     }
     // threshold from the list heads (every list is sorted, descending)
-    unsigned long long v = x[0];
-#pragma unroll 1
-    for (int size = 2; size <= 32; size <<= 1) {
-#pragma unroll 1
-      for (int stride = size >> 1; stride > 0; stride >>= 1) {
-        const unsigned long long o = __shfl_xor_sync(0xffffffffu, v, stride);
-        const bool dir = (lane & size) == 0, lower = (lane & stride) == 0;
-        v = (lower == dir) ? umax64(v, o) : (v < o ? v : o);
-      }
-    }
-    const unsigned long long tau = __shfl_sync(0xffffffffu, v, k - 1);
+    const unsigned long long tau = group_kth_u64(x[0], 32, k);
     int cnt = 0;
 #pragma unroll
     for (int i = 0; i < KQ; ++i) cnt += (x[i] >= tau && x[i] != 0ull);
     int incl = cnt;
-#pragma unroll 1
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
@@ -872,18 +1031,6 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg
   }
 }
 
-template <int DT>
-__device__ __forceinline__ float4 qrow4(const uint32_t* qs, int row, int qw, int lane) {
-  if (DT == LOSA_BF16) {
-    const uint32_t w0 = qs[row * qw + 2 * lane], w1 = qs[row * qw + 2 * lane + 1];
-    return make_float4(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
-                       __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u));
-  }
-  const uint32_t* w = qs + row * qw + 4 * lane;
-  return make_float4(__uint_as_float(w[0]), __uint_as_float(w[1]), __uint_as_float(w[2]),
-                     __uint_as_float(w[3]));
-}
-
 template <int DT, int KP>
 __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherParams prm) {
   extern __shared__ __align__(1024) char smem[];
@@ -891,17 +1038,26 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   const Dims& d = prm.d;
   const GatherLayout& lo = prm.lo;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g4 = lane >> 2, t4 = lane & 3;
   const int rank = static_cast<int>(cluster.block_rank());
   const int CL = prm.CL;
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
-  const int esz = DT == LOSA_BF16 ? 2 : 4;
-  const int pbytes = kPS * kD * esz;
+  const int GB = G * B;
+  constexpr int rowb = DT == LOSA_BF16 ? kD * 2 : kD * 4;
+  constexpr int cpr = rowb / 16;  // 16-byte chunks per row
+  constexpr int pbytes = kPS * rowb;
+  const int bpad = (B + kPS - 1) / kPS * kPS;
   const int nwords = (d.P + 31) / 32;
+  const size_t grow0 = (static_cast<size_t>(s) * d.Hq + g * G) * B;  // the group's first row
 
-  char* slots = smem + lo.stage;  // gather pages
-  char* qa = smem + lo.qa;  // [R][kD] active rows' queries, element type
+  char* region = smem + lo.region;
+  char* kbv = smem + lo.kbv;
+  char* qa = smem + lo.qa;
+  char* qs = smem + lo.qs;
+  float* ocache = reinterpret_cast<float*>(smem + lo.ocache);
+  float* lcache = reinterpret_cast<float*>(smem + lo.lcache);
   int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
   int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel_all);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + lo.bitmap);
@@ -909,20 +1065,35 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
+  float* sfx = reinterpret_cast<float*>(smem + lo.sfx);    // [n_oa][kPartStride]: (L_s, -, -, -, o_s)
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
-  int32_t* s_fail = misc;
-  int32_t* s_U = misc + 1;
-  int32_t* s_nlp = misc + 2;
-  int32_t* act_tok = misc + 4;  // [R]
+  int32_t* s_U = misc;
+  int32_t* s_nlp = misc + 1;
+  int32_t* s_wt = misc + 4;            // stable tokens per 32-token warp slice
+  int32_t* act_tok = misc + 8;         // [R], then act_slot [GB]
+  int32_t* act_slot = act_tok + R;
+  int32_t* sfx_tok = act_slot + GB;    // [n_oa + n_os]: token row of each suffix row
   float* psw = Ps + warp * 16;
 
-  if (tid == 0) {
-    for (int i = 0; i < kMaxGatherPages; ++i) mbar_init(&mbar[i], 1);
-    fence_mbar_init();
-    *s_fail = 0;
+  // barrier 0: before touching another CTA's shared memory, every CTA of the
+  // cluster must be running; the wait comes after the selection
+  cluster_arrive_relaxed();
+
+  // ---- the block's K and V (cp.async group 0; rows >= B are zero)
+  {
+    const char* kbg = static_cast<const char*>(prm.kb) + static_cast<size_t>(sg) * B * rowb;
+    const char* vbg = static_cast<const char*>(prm.vb) + static_cast<size_t>(sg) * B * rowb;
+    const int per = bpad * cpr;
+#pragma unroll 1
+    for (int e = tid; e < 2 * per; e += kThreads) {
+      const int h = e >= per ? 1 : 0, rem = e - h * per, j = rem / cpr, c = rem - j * cpr;
+      const bool ok = j < B;
+      const char* src = (h ? vbg : kbg) + static_cast<size_t>(ok ? j : 0) * rowb + c * 16;
+      cp_async16(su32(kbv + h * bpad * rowb + tile_off<DT>(j, c)), src, ok ? 16u : 0u);
+    }
+    cp_async_commit();
   }
 #pragma unroll 1
   for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
@@ -931,22 +1102,74 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   // everything below reads what the scan kernel wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
+  {
+    const int32_t* actg = prm.act_g + static_cast<size_t>(sg) * (R + GB);
 #pragma unroll 1
-  for (int r = tid; r < R; r += kThreads)
-    act_tok[r] = __ldcg(prm.act_tok_g + static_cast<size_t>(sg) * R + r);
+    for (int e = tid; e < R + GB; e += kThreads) act_tok[e] = __ldcg(actg + e);
+  }
   __syncthreads();
-  {  // active rows' queries (element type)
-    const int cpr = kD * esz / 16;
+
+  // ---- this CTA's suffix rows: its active rows r = rank + CL*j first, then
+  // every CL-th stable token row
+  const int n_oa = R > rank ? (R - rank + CL - 1) / CL : 0;
+  const int n_os = GB - R > rank ? (GB - R - rank + CL - 1) / CL : 0;
+  const int ns = n_oa + n_os;
+  {
+    bool st = false;
+    int pre = 0;
+    if (warp < 4) {  // G*B <= 128 token rows
+      st = tid < GB && act_slot[tid] < 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, st);
+      pre = __popc(bal & ((1u << lane) - 1u));
+      if (lane == 0) s_wt[warp] = __popc(bal);
+    }
 #pragma unroll 1
-    for (int e = tid; e < R * cpr; e += kThreads) {
-      const int r = e / cpr, c = e - r * cpr;
-      const size_t row = (static_cast<size_t>(s) * d.Hq + g * G + r / A) * B + act_tok[r];
-      reinterpret_cast<uint4*>(qa)[e] =
-          reinterpret_cast<const uint4*>(static_cast<const char*>(prm.qc) + row * kD * esz)[c];
+    for (int j = tid; j < n_oa; j += kThreads) {
+      const int r = rank + CL * j;
+      sfx_tok[j] = (r / A) * B + act_tok[r];
+    }
+    __syncthreads();
+    if (st) {
+      for (int w = 0; w < warp; ++w) pre += s_wt[w];
+      if (pre % CL == rank) sfx_tok[n_oa + pre / CL] = tid;
     }
   }
+  __syncthreads();
 
-  // ---- this CTA's rows (r % CL == rank): the row's k pages
+  // ---- cp.async group 1: queries of the suffix rows and of the active rows,
+  // cached state of the stable suffix rows
+  {
+    const char* qg = static_cast<const char*>(prm.qc) + grow0 * rowb;
+    const int nsr = DT == LOSA_BF16 ? (ns + 15) / 16 * 16 : ns;
+#pragma unroll 1
+    for (int e = tid; e < nsr * cpr; e += kThreads) {
+      const int n = e / cpr, c = e - n * cpr;
+      const bool ok = n < ns;
+      cp_async16(su32(qs + tile_off<DT>(n, c)),
+                 qg + static_cast<size_t>(ok ? sfx_tok[n] : 0) * rowb + c * 16, ok ? 16u : 0u);
+    }
+    const int nar = DT == LOSA_BF16 ? (R + 15) / 16 * 16 : R;
+#pragma unroll 1
+    for (int e = tid; e < nar * cpr; e += kThreads) {
+      const int r = e / cpr, c = e - r * cpr;
+      const bool ok = r < R;
+      const int tok = ok ? (r / A) * B + act_tok[r] : 0;
+      cp_async16(su32(qa + tile_off<DT>(r, c)), qg + static_cast<size_t>(tok) * rowb + c * 16,
+                 ok ? 16u : 0u);
+    }
+#pragma unroll 1
+    for (int e = tid; e < n_os * (kD / 4); e += kThreads) {
+      const int n = e / (kD / 4), c = e - n * (kD / 4);
+      const size_t grow = grow0 + sfx_tok[n_oa + n];
+      cp_async16(su32(ocache + n * kD + 4 * c), prm.o_p + grow * kD + 4 * c, 16u);
+    }
+#pragma unroll 1
+    for (int n = tid; n < n_os; n += kThreads)
+      cp_async4(su32(lcache + n), prm.l_p + grow0 + sfx_tok[n_oa + n]);
+    cp_async_commit();
+  }
+
+  // ---- this CTA's rows (r % CL == rank): the row's k pages, ascending
   if (!d.all_pages) {
 #pragma unroll 1
     for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
@@ -954,7 +1177,7 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       merge_row<KP>(prm, r, sg, best, mbuf + warp * kCandCap);
       int32_t* dst = sel_own + (r / CL) * k;
 #pragma unroll 1
-      for (int j = lane; j < k; j += 32) {  // pages in ascending order
+      for (int j = lane; j < k; j += 32) {
         const int pj = key_index(best[j]);
         int rk = 0;
 #pragma unroll 4
@@ -977,11 +1200,21 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
     }
   }
   __syncthreads();
-  cluster.sync();
+  cluster_wait();  // barrier 0
+  if (!d.all_pages) {  // this CTA's rows' pages -> every CTA of the cluster
+#pragma unroll 1
+    for (int e = tid; e < n_oa * CL * k; e += kThreads) {
+      const int j = e / (CL * k), rem = e - j * CL * k, c = rem / k, i = rem - c * k;
+      const int r = rank + CL * j;
+      cluster.map_shared_rank(sel_all, c)[r * k + i] = sel_own[j * k + i];
+    }
+  }
+  cluster_arrive();
+  cluster_wait();  // barrier 1: every row's pages are in every CTA
 
   // ---- union of the group's pages and this CTA's share
   if (d.all_pages) {
-    const int U = d.P;
+    const int U = R > 0 ? d.P : 0;
     const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
     if (tid == 0) {
       *s_nlp = nlp;
@@ -996,13 +1229,6 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
     }
   } else {
-    const int rows_own = (R + CL - 1) / CL;
-#pragma unroll 1
-    for (int e = tid; e < R * k; e += kThreads) {
-      const int r = e / k, j = e - r * k;
-      sel_all[e] = cluster.map_shared_rank(sel_own, r % CL)[(r / CL) * k + j];
-    }
-    (void)rows_own;
 #pragma unroll 1
     for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
     __syncthreads();
@@ -1020,7 +1246,7 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
 #pragma unroll 1
       for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
       int incl = sum;
-#pragma unroll 1
+#pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
@@ -1069,27 +1295,174 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   }
   __syncthreads();
 
-  // ---- gather: this CTA's union pages, in batches of ngp; warp w folds the
-  // pages of rows r = w, w + 8, ... into their partials (one writer per row)
-  {
-    const int nlp = min(*s_nlp, prm.max_lp);
+  // ---- gather copies (cp.async group 2): this CTA's union pages, in batches
+  // of ngp; rows past the prefix end are zero
+  const int nlp = min(*s_nlp, prm.max_lp);
+  auto issue_batch = [&](int b0) {
+    const int nb = min(prm.ngp, nlp - b0);
+    constexpr int per = kPS * cpr;
 #pragma unroll 1
-    for (int b0 = 0; b0 < nlp && !*s_fail; b0 += prm.ngp) {
-      const int nb = min(prm.ngp, nlp - b0);
-      const int batch = b0 / prm.ngp;
-      if (tid == 0) {
+    for (int e = tid; e < nb * 2 * per; e += kThreads) {
+      const int i = e / (2 * per), rem = e - i * 2 * per, h = rem / per, rr = rem - h * per;
+      const int j = rr / cpr, c = rr - j * cpr;
+      const int p = lpages[b0 + i];
+      const bool ok = p * kPS + j < d.L;
+      const size_t off =
+          (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS + (ok ? j : 0)) * rowb + c * 16;
+      cp_async16(su32(region + (2 * i + h) * pbytes + tile_off<DT>(j, c)),
+                 static_cast<const char*>(h ? prm.V : prm.K) + off, ok ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  issue_batch(0);
+
+  // ---- dense suffix of this CTA's rows (hidden behind the gather copies):
+  // stable rows merge with their cached state and are finished; active rows
+  // keep (L_s, o_s) for the combine
+  cp_async_wait<1>();  // groups 0 and 1
+  __syncthreads();
+  if (DT == LOSA_BF16) {
+    const int nmt = (ns + 15) / 16;
 #pragma unroll 1
-        for (int i = 0; i < nb; ++i) {
-          const int p = lpages[b0 + i];
-          const int ntok = min(kPS, d.L - p * kPS);
-          const uint32_t bytes = static_cast<uint32_t>(ntok * kD * esz);
-          const size_t off = (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS) * kD * esz;
-          char* dst = slots + i * 2 * pbytes;
-          mbar_expect_tx(&mbar[i], 2 * bytes);
-          bulk_g2s(dst, static_cast<const char*>(prm.K) + off, bytes, &mbar[i]);
-          bulk_g2s(dst + pbytes, static_cast<const char*>(prm.V) + off, bytes, &mbar[i]);
+    for (int mt = warp; mt < nmt; mt += kWarps) {
+      TileAcc t;
+      tile_init(t);
+#pragma unroll 1
+      for (int j0 = 0; j0 < B; j0 += kPS)
+        tile_attend(t, qs + mt * 16 * 256, kbv + j0 * 256, kbv + (bpad + j0) * 256, 0xffffu,
+                    min(kPS, B - j0), d.scale_log2);
+      tile_finish(t);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = mt * 16 + g4 + 8 * h;
+        if (n >= ns) continue;
+        const float inv = __frcp_rn(t.l[h]);
+        const float Ls = (t.m[h] + __log2f(t.l[h])) * kLn2;
+        if (n < n_oa) {
+          float* dst = sfx + n * kPartStride;
+          if (t4 == 0) dst[0] = Ls;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<float2*>(dst + 4 + c * 8 + 2 * t4) =
+                make_float2(t.o[c][2 * h] * inv, t.o[c][2 * h + 1] * inv);
+        } else {
+          const int m = n - n_oa;
+          const size_t grow = grow0 + sfx_tok[n];
+          float wa, wb, L;
+          lse_weights(lcache[m], Ls, wa, wb, L);
+          const float* op = ocache + m * kD;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int ch = c * 8 + 2 * t4;
+            const float2 o = *reinterpret_cast<const float2*>(op + ch);
+            *reinterpret_cast<float2*>(prm.out + grow * kD + ch) =
+                make_float2(wa * o.x + wb * (t.o[c][2 * h] * inv), wa * o.y + wb * (t.o[c][2 * h + 1] * inv));
+          }
+          if (prm.out_lse && t4 == 0) prm.out_lse[grow] = L;
         }
       }
+    }
+  } else {
+#pragma unroll 1
+    for (int n = warp; n < ns; n += kWarps) {
+      const float4 q = row4<DT>(qs, n, lane);
+      float m = -INFINITY, l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int j0 = 0; j0 < B; j0 += kPS)
+        attend_page<DT>(q, kbv + j0 * rowb, kbv + (bpad + j0) * rowb, min(kPS, B - j0),
+                        d.scale_log2, m, l, acc, psw);
+      const float inv = __frcp_rn(l);
+      const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      const float Ls = (m + __log2f(l)) * kLn2;
+      if (n < n_oa) {
+        float* dst = sfx + n * kPartStride;
+        if (lane == 0) dst[0] = Ls;
+        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
+      } else {
+        const int mm = n - n_oa;
+        const size_t grow = grow0 + sfx_tok[n];
+        float wa, wb, L;
+        lse_weights(lcache[mm], Ls, wa, wb, L);
+        const float4 op = *reinterpret_cast<const float4*>(ocache + mm * kD + 4 * lane);
+        *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+            make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                        wa * op.w + wb * os.w);
+        if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+      }
+    }
+  }
+
+  // ---- the union pages -> one partial per row (part)
+  cp_async_wait<0>();
+  __syncthreads();
+  if (DT == LOSA_BF16) {
+    const int ntm = (R + 15) / 16;
+    const int wpm = ntm > 0 ? kWarps / ntm : kWarps;
+    const int mt = warp / wpm, sub = warp % wpm;
+    const bool aw = mt < ntm;
+    TileAcc t;
+    tile_init(t);
+#pragma unroll 1
+    for (int b0 = 0; b0 < nlp; b0 += prm.ngp) {
+      const int nb = min(prm.ngp, nlp - b0);
+#pragma unroll 1
+      for (int i = sub; aw && i < nb; i += wpm) {
+        const uint32_t bits = (masks[(b0 + i) * d.MW + (mt >> 1)] >> ((mt & 1) * 16)) & 0xffffu;
+        if (!bits) continue;
+        const int p = lpages[b0 + i];
+        tile_attend(t, qa + mt * 16 * 256, region + 2 * i * pbytes, region + (2 * i + 1) * pbytes,
+                    bits, min(kPS, d.L - p * kPS), d.scale_log2);
+      }
+      if (b0 + prm.ngp < nlp) {  // next batch into the same slots
+        __syncthreads();
+        issue_batch(b0 + prm.ngp);
+        cp_async_wait<0>();
+        __syncthreads();
+      }
+    }
+    tile_finish(t);
+    if (wpm == 1) {  // one warp per m16 tile: its state is the CTA's partial
+      if (aw) tile_store(t, part + mt * 16 * kPartStride, min(16, R - mt * 16));
+    } else {
+      float* wp = reinterpret_cast<float*>(region);
+      __syncthreads();  // every page consumed: the region takes the warps' partials
+      if (aw) tile_store(t, wp + warp * 16 * kPartStride, 16);
+      __syncthreads();
+#pragma unroll 1
+      for (int r = warp; r < R; r += kWarps) {
+        const int m16 = r >> 4, i = r & 15;
+        float M = -INFINITY;
+#pragma unroll 1
+        for (int w = 0; w < wpm; ++w) M = fmaxf(M, wp[((m16 * wpm + w) * 16 + i) * kPartStride]);
+        if (M == -INFINITY) continue;  // none of this CTA's pages serve row r
+        float l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int w = 0; w < wpm; ++w) {
+          const float* pr = wp + ((m16 * wpm + w) * 16 + i) * kPartStride;
+          const float mw = pr[0];
+          if (mw == -INFINITY) continue;
+          const float wgt = exp2f(mw - M);
+          l += wgt * pr[1];
+          const float4 a = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+          acc.x += wgt * a.x;
+          acc.y += wgt * a.y;
+          acc.z += wgt * a.z;
+          acc.w += wgt * a.w;
+        }
+        float* dst = part + r * kPartStride;
+        if (lane == 0) {
+          dst[0] = M;
+          dst[1] = l;
+        }
+        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = acc;
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int b0 = 0; b0 < nlp; b0 += prm.ngp) {
+      const int nb = min(prm.ngp, nlp - b0);
 #pragma unroll 1
       for (int r = warp; r < R; r += kWarps) {
         bool have = false;
@@ -1103,17 +1476,9 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
 #pragma unroll 1
         for (int i = 0; i < nb; ++i) {
           if (!((masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u)) continue;
-          if (!__all_sync(0xffffffffu, mbar_wait(&mbar[i], batch & 1))) {
-            if (lane == 0) {
-              atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
-              *s_fail = 1;
-            }
-            break;
-          }
           const int p = lpages[b0 + i];
-          const char* Ks = slots + i * 2 * pbytes;
-          attend_page<DT>(q, Ks, Ks + pbytes, min(kPS, d.L - p * kPS), d.scale_log2, m, l, acc,
-                          psw);
+          attend_page<DT>(q, region + 2 * i * pbytes, region + (2 * i + 1) * pbytes,
+                          min(kPS, d.L - p * kPS), d.scale_log2, m, l, acc, psw);
         }
         __syncwarp();
         if (lane == 0) {
@@ -1122,64 +1487,90 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
         }
         *reinterpret_cast<float4*>(pr + 4 + 4 * lane) = acc;
       }
-      // every copy of this batch has landed before the slots are refilled
-#pragma unroll 1
-      for (int i = tid; i < nb; i += kThreads)
-        if (!mbar_wait(&mbar[i], batch & 1)) *s_fail = 1;
-      __syncthreads();
+      if (b0 + prm.ngp < nlp) {
+        __syncthreads();
+        issue_batch(b0 + prm.ngp);
+        cp_async_wait<0>();
+        __syncthreads();
+      }
     }
   }
   __syncthreads();
-  cluster.sync();
+  cluster_arrive();
+  cluster_wait();  // barrier 2: every CTA's partials are complete
 
-  // ---- combine every CTA's partial of this CTA's rows, cache write-back,
-  // merge with the suffix
-  if (!*s_fail) {
+  // ---- combine the partials of this CTA's rows from every CTA of the
+  // cluster (all loads issued before any is used), cache write-back, merge
+  // with the suffix
 #pragma unroll 1
-    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
-      float M = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < CL; ++c) M = fmaxf(M, cluster.map_shared_rank(part, c)[r * kPartStride]);
-      float lsum = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int c = 0; c < CL; ++c) {  // fixed order: deterministic
-        const float* pr = cluster.map_shared_rank(part, c) + r * kPartStride;
-        const float mc = pr[0];
-        if (mc == -INFINITY) continue;  // this CTA held none of the row's pages
-        const float w = exp2f(mc - M);
-        lsum += w * pr[1];
-        const float4 a = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
-        acc.x += w * a.x;
-        acc.y += w * a.y;
-        acc.z += w * a.z;
-        acc.w += w * a.w;
+  for (int j = warp; j < n_oa; j += kWarps) {
+    const int r = rank + CL * j;
+    // CTAs in fixed order (deterministic), eight partials in flight at a time
+    float M = -INFINITY, lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int h = 0; h < kMaxCluster; h += 8) {
+      if (h < CL) {
+        float mc[8], lc[8];
+        float4 ac[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          mc[i] = -INFINITY;
+          if (h + i < CL) {
+            const float* pr = cluster.map_shared_rank(part, h + i) + r * kPartStride;
+            mc[i] = pr[0];
+            lc[i] = pr[1];
+            ac[i] = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+          }
+        }
+        float Mh = M;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) Mh = fmaxf(Mh, mc[i]);
+        if (Mh != -INFINITY) {
+          const float rs = exp2f(M - Mh);  // 0 while nothing is accumulated
+          lsum *= rs;
+          acc.x *= rs;
+          acc.y *= rs;
+          acc.z *= rs;
+          acc.w *= rs;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (mc[i] != -INFINITY) {
+              const float w = exp2f(mc[i] - Mh);
+              lsum += w * lc[i];
+              acc.x += w * ac[i].x;
+              acc.y += w * ac[i].y;
+              acc.z += w * ac[i].z;
+              acc.w += w * ac[i].w;
+            }
+          }
+          M = Mh;
+        }
       }
-      const float inv = __frcp_rn(lsum);
-      const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      const float Lp = (M + __log2f(lsum)) * kLn2;
-      const int hl = r / A, t = act_tok[r];
-      const size_t grow = (static_cast<size_t>(s) * d.Hq + g * G + hl) * B + t;
-      *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
-      if (lane == 0) prm.l_p[grow] = Lp;
-      const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
-      const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4 + 4 * lane));
-      float4 o;
-      float L;
-      lse_merge(op, Lp, os, __ldcg(sx), o, L);
-      *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) = o;
-      if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
     }
+    const float inv = __frcp_rn(lsum);
+    const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    const float Lp = (M + __log2f(lsum)) * kLn2;
+    const size_t grow = grow0 + (r / A) * B + act_tok[r];
+    *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
+    if (lane == 0) prm.l_p[grow] = Lp;
+    const float* sx = sfx + j * kPartStride;
+    const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
+    float wa, wb, L;
+    lse_weights(Lp, sx[0], wa, wb, L);
+    *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+        make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                    wa * op.w + wb * os.w);
+    if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
   }
-  // no CTA may leave while others can still read its shared memory
-  cluster.sync();
+  // barrier 3: no CTA leaves while another may still read its partials
+  cluster_arrive();
+  cluster_wait();
 }
 
 // ---------------------------------------------------------------------------
 // host side: launch geometry, shared-memory layouts, attributes
 // ---------------------------------------------------------------------------
-constexpr int kGatherSmemTarget = 110 * 1024;  // two gather CTAs per SM
-
 int topk_width(int k) {
   if (k <= 2) return 2;
   if (k <= 4) return 4;
@@ -1188,86 +1579,107 @@ int topk_width(int k) {
   return 0;  // warp fallback
 }
 
+struct Taker {
+  int off = 0;
+  int operator()(long long bytes, int align) {
+    off = align_up(off, align);
+    const int o = off;
+    off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
+    return o;
+  }
+};
+
 bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   prm->d = d;
+  prm->scan = d.A > 0 && !d.all_pages;
   prm->rec = 2 * kD * d.esz;
   prm->tile = kStageBytes / prm->rec;  // 64 (bf16) or 32 (fp32) pages per stage
   prm->sc_stride = align_up(d.chunk_pages, 4) + 4;
-  prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
   prm->kp = topk_width(d.k);
+  const int GB = d.G * d.B;
   // a row's top-k group: at least k lanes, and enough lanes to cover the
   // CTA's rows in few passes
   prm->tpr = std::min(32, std::max(pow2_floor(std::max(1, kThreads / std::max(d.R, 1))),
                                    d.k <= 1 ? 1 : pow2_floor(2 * d.k - 1)));
-  const bool selects = d.A > 0 && !d.all_pages;
-  if (selects && prm->kp > 0 && prm->tpr < d.k) return false;
-  if (selects && prm->kp == 0 && d.k > kCandCap) return false;
+  prm->mse_t = std::min(16, pow2_floor(std::max(1, kThreads / std::max(GB, 1))));
+  if (prm->scan && prm->kp > 0 && prm->tpr < d.k) return false;
+  if (prm->scan && prm->kp == 0 && d.k > kCandCap) return false;
   const int R16 = (d.R + 15) / 16 * 16;
-  const int GB = d.G * d.B;
-  for (int ring = kMaxRingBytes; ring >= 64 * 1024; ring -= 32 * 1024) {
+  const long long qbytes = 1LL * GB * kD * d.esz;
+  for (int ring = prm->scan ? kMaxRingBytes : 0; ring >= 0; ring -= 32 * 1024) {
+    if (prm->scan && ring < 32 * 1024) break;
     ScanLayout& lo = prm->lo;
-    int off = 0;
-    auto take = [&](long long bytes, int align) {
-      off = align_up(off, align);
-      const int o = off;
-      off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
-      return o;
-    };
+    Taker take;
     lo.ring = take(ring, 1024);
-    // scores, or (before the scan) the staged queries
-    lo.scores = take(std::max(4LL * d.R * prm->sc_stride, 2LL * GB * prm->qw * 4), 16);
-    lo.kbv = take(2LL * ((d.B + kPS - 1) / kPS * kPS) * kD * d.esz, 16);
-    lo.qrows = take(R16 * 512, 128);
-    lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
-    lo.ps = take(kWarps * 16 * 4, 16);
-    lo.fbuf = take(prm->kp > 0 ? 8LL * (kThreads / prm->tpr) * kCandCap : 0, 16);
-    lo.cbuf = take(prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
+    lo.qc = take(qbytes, 128);
+    // the previous queries, then (after the locality pass) the scores
+    lo.qps = take(std::max(qbytes, prm->scan ? 4LL * d.R * prm->sc_stride : 0LL), 128);
+    lo.qrows = take(prm->scan ? (d.esz == 2 ? R16 : d.R) * 512LL : 0, 128);
+    lo.misc = take((4 + kMaxRowsPerGroup + d.R) * 4, 16);
+    lo.fbuf = take(prm->scan && prm->kp > 0 ? 8LL * (kThreads / prm->tpr) * kCandCap : 0, 16);
+    lo.cbuf = take(prm->scan && prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
     lo.mbar = take((kMaxStages + 1) * 8, 8);
-    lo.total = off;
+    lo.total = take.off;
     prm->stages = ring / kStageBytes;
     if (lo.total <= max_dyn) return true;
+    if (!prm->scan) break;
   }
   return false;
 }
 
-bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int max_cluster) {
+bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
   prm->d = d;
-  const int CL = std::min(max_cluster, std::max(1, std::max(d.Umax, 1)));
   prm->CL = CL;
   prm->max_lp = (d.Umax + CL - 1) / CL;
-  prm->qw = d.esz == 2 ? kD / 2 + 1 : kD + 1;
   if (!d.all_pages && d.A > 0 && topk_width(d.k) == 0 && d.k > kCandCap) return false;
+  const int GB = d.G * d.B;
+  prm->n_oa = (d.R + CL - 1) / CL;
+  prm->n_os = (GB - d.R + CL - 1) / CL;
+  const int ns = prm->n_oa + prm->n_os;
+  const bool bf = d.esz == 2;
+  const int ntm = (d.R + 15) / 16;
+  prm->wpart = bf && ntm > 0 && kWarps / ntm > 1;
+  const int rowb = kD * d.esz;
   const int nwords = (d.P + 31) / 32;
-  const int pbytes = kPS * kD * d.esz;
-  const int rows_per_cta = (d.R + CL - 1) / CL;
-  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
+  const int pbytes = kPS * rowb;
+  const int bpad = (d.B + kPS - 1) / kPS * kPS;
+  const bool sel = !d.all_pages && d.A > 0;
+  auto layout = [&](int ngp) {
     GatherLayout& lo = prm->lo;
-    int off = 0;
-    auto take = [&](long long bytes, int align) {
-      off = align_up(off, align);
-      const int o = off;
-      off += static_cast<int>(std::min<long long>(bytes, 1 << 30));
-      return o;
-    };
-    lo.stage = take(2LL * ngp * pbytes, 1024);
-    lo.qa = take(1LL * d.R * kD * d.esz, 16);
-    lo.sel_own = take(d.all_pages ? 0 : 4LL * rows_per_cta * d.k, 16);
-    lo.sel_all = take(d.all_pages ? 0 : 4LL * d.R * d.k, 16);
+    Taker take;
+    lo.region = take(std::max(2LL * ngp * pbytes, prm->wpart ? 4LL * kWarps * 16 * kPartStride : 0LL),
+                     1024);
+    lo.kbv = take(2LL * bpad * rowb, 128);
+    lo.qa = take(1LL * (bf ? ntm * 16 : d.R) * rowb, 128);
+    lo.qs = take(1LL * (bf ? (ns + 15) / 16 * 16 : ns) * rowb, 128);
+    lo.ocache = take(4LL * prm->n_os * kD, 16);
+    lo.lcache = take(4LL * prm->n_os, 16);
+    lo.sel_own = take(sel ? 4LL * prm->n_oa * d.k : 0, 16);
+    lo.sel_all = take(sel ? 4LL * d.R * d.k : 0, 16);
     lo.bitmap = take(nwords * 4, 16);
     lo.wbase = take(nwords * 4, 16);
     lo.lpages = take(prm->max_lp * 4, 16);
     lo.masks = take(4LL * prm->max_lp * d.MW, 16);
     lo.part = take(4LL * d.R * kPartStride, 16);
-    lo.misc = take((4 + kMaxRowsPerGroup) * 4, 16);
+    lo.sfx = take(4LL * prm->n_oa * kPartStride, 16);
+    lo.misc = take((8 + d.R + GB + ns) * 4, 16);
     lo.ps = take(kWarps * 16 * 4, 16);
-    lo.mbuf = take(2 * kWarps * kCandCap * 8, 16);
-    lo.mbar = take(kMaxGatherPages * 8, 8);
-    lo.total = off;
+    lo.mbuf = take(sel ? 2 * kWarps * kCandCap * 8 : 0, 16);
+    lo.total = take.off;
     prm->ngp = ngp;
-    if (lo.total <= std::min(max_dyn, kGatherSmemTarget) || (ngp == 1 && lo.total <= max_dyn))
-      return true;
+    return lo.total;
+  };
+  // the largest batch of pages in flight with two CTAs per SM, else the
+  // largest that fits one
+  int one = 0;
+  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
+    const int total = layout(ngp);
+    if (total <= std::min(max_dyn, kGatherSmemTarget)) return true;
+    if (total <= max_dyn && one == 0) one = ngp;
   }
-  return false;
+  if (one == 0) return false;
+  layout(one);
+  return true;
 }
 
 std::mutex g_attr_mu;
@@ -1353,15 +1765,15 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
 
 template <int DT, int KP>
 cudaError_t launch_pair(const cudaLaunchConfig_t& c1, const ScanParams& sp,
-                        const cudaLaunchConfig_t* c2, const GatherParams& gp) {
+                        const cudaLaunchConfig_t& c2, const GatherParams& gp) {
   const cudaError_t e = cudaLaunchKernelEx(&c1, losa_scan_kernel<DT, KP>, sp);
-  if (e != cudaSuccess || !c2) return e;
-  return cudaLaunchKernelEx(c2, losa_gather_kernel<DT, KP>, gp);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
 }
 
 template <int DT>
 cudaError_t launch_dt(int kp, const cudaLaunchConfig_t& c1, const ScanParams& sp,
-                      const cudaLaunchConfig_t* c2, const GatherParams& gp) {
+                      const cudaLaunchConfig_t& c2, const GatherParams& gp) {
   switch (kp) {
     case 2: return launch_pair<DT, 2>(c1, sp, c2, gp);
     case 4: return launch_pair<DT, 4>(c1, sp, c2, gp);
@@ -1374,9 +1786,10 @@ cudaError_t launch_dt(int kp, const cudaLaunchConfig_t& c1, const ScanParams& sp
 }  // namespace
 
 bool fused_step_fits(const Dims& d, int max_dyn) {
+  // sized for the smallest cluster the device may allow (the most rows per CTA)
   ScanParams sp;
   GatherParams gp;
-  return plan_scan(d, &sp, max_dyn) && (d.A == 0 || plan_gather(d, &gp, max_dyn, kMaxCluster));
+  return plan_scan(d, &sp, max_dyn) && plan_gather(d, &gp, max_dyn, 4);
 }
 
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
@@ -1390,31 +1803,22 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   ScanParams sp;
   GatherParams gp;
   if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
-  if (d.A > 0 && !plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
+  if (!plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
   if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
   char* ws = static_cast<char*>(workspace);
   int* status = reinterpret_cast<int*>(ws + d.off_status);
-  int32_t* act_tok = reinterpret_cast<int32_t*>(ws + d.off_act);
-  float* sfx = reinterpret_cast<float*>(ws + d.off_sfx);
+  int32_t* act = reinterpret_cast<int32_t*>(ws + d.off_act);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
 
   sp.qc = q_cur;
   sp.qp = q_prev;
   sp.meta = static_cast<const char*>(page_meta);
-  sp.kb = k_blk;
-  sp.vb = v_blk;
-  sp.o_p = o_p;
-  sp.l_p = l_p;
-  sp.out = out;
-  sp.out_lse = out_lse;
+  sp.act_g = act;
   sp.active_idx = active_idx;
-  sp.union_count = union_count;
-  sp.act_tok_g = act_tok;
-  sp.sfx_g = sfx;
   sp.cand = cand;
   sp.status = status;
   cudaLaunchConfig_t c1 = {};
-  c1.gridDim = dim3(d.nchunk, d.S * d.Hkv, 1);
+  c1.gridDim = dim3(sp.scan ? d.nchunk : 1, d.S * d.Hkv, 1);
   c1.blockDim = dim3(kThreads, 1, 1);
   c1.dynamicSmemBytes = static_cast<size_t>(sp.lo.total);
   c1.stream = st;
@@ -1422,38 +1826,36 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   gp.qc = q_cur;
   gp.K = k_prefix;
   gp.V = v_prefix;
+  gp.kb = k_blk;
+  gp.vb = v_blk;
   gp.o_p = o_p;
   gp.l_p = l_p;
   gp.out = out;
   gp.out_lse = out_lse;
   gp.page_idx = page_idx;
   gp.union_count = union_count;
-  gp.act_tok_g = act_tok;
-  gp.sfx_g = sfx;
+  gp.act_g = act;
   gp.cand = cand;
   gp.status = status;
   cudaLaunchConfig_t c2 = {};
   cudaLaunchAttribute attr[2];
-  if (d.A > 0) {
-    c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
-    c2.blockDim = dim3(kThreads, 1, 1);
-    c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
-    c2.stream = st;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = gp.CL;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
-    c2.attrs = attr;
-    c2.numAttrs = 2;
-  }
+  c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
+  c2.blockDim = dim3(kThreads, 1, 1);
+  c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
+  c2.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = gp.CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
+  c2.attrs = attr;
+  c2.numAttrs = 2;
   // one top-k width per compiled kernel: the selection code of the others is
   // never fetched
-  const int kp = (d.A > 0 && !d.all_pages) ? sp.kp : 2;
-  const cudaLaunchConfig_t* c2p = d.A > 0 ? &c2 : nullptr;
-  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, c1, sp, c2p, gp)
-                                             : launch_dt<LOSA_F32>(kp, c1, sp, c2p, gp);
+  const int kp = sp.scan ? sp.kp : 2;
+  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, c1, sp, c2, gp)
+                                             : launch_dt<LOSA_F32>(kp, c1, sp, c2, gp);
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
 
