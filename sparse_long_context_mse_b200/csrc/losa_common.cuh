@@ -19,6 +19,7 @@ constexpr int kMaxB = 32;       // block tokens (one warp lane per token)
 constexpr int kMaxRowsPerGroup = 128;  // G*B (and hence G*A) per KV head
 constexpr int kMaxK = 64;       // pages per active row unless every page is taken
 constexpr int kPartStride = kD + 4;    // floats per split-softmax partial: m, l, pad, pad, acc[d]
+constexpr int kGatherCtas = 16;        // CTAs per (sequence, KV head) in the step's gather kernel
 constexpr int kMaxDevices = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -35,7 +36,7 @@ struct Dims {
   int nsplit, split_pages;
   int nchunk, chunk_pages;
   // workspace byte offsets
-  size_t off_status, off_part, off_act, off_cand, total;
+  size_t off_status, off_part, off_act, off_cand, off_gpart, off_gsfx, off_cnt, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).

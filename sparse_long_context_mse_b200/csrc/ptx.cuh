@@ -1,6 +1,6 @@
 // ptx.cuh -- inline-PTX wrappers shared by the LoSA kernels (sm_100a):
 // mbarriers, non-multicast bulk copies (TMA), cp.async, ldmatrix, mma.sync,
-// cluster barriers.
+// named barriers.
 #pragma once
 
 #include <stdint.h>
@@ -89,18 +89,9 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// Thread-block-cluster barrier, split into its two halves.  Every thread of
-// every CTA of the cluster arrives, then waits; the release/acquire pair
-// orders shared-memory writes made before the arrive (including writes to
-// other CTAs' shared memory) before reads made after the wait.
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+// Named barrier `id` (1..15) over `n` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 // Two fp32 values -> packed bf16x2 (round to nearest even), low half first.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

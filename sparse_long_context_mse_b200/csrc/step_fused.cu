@@ -17,36 +17,29 @@
 //    A operand held in registers); fp32: CUDA cores, the sum in channel order
 //    with one rounding per operation -- and a chunk-local top-k per row into
 //    the workspace.  The first CTA of a group also stores the active set.
-// K2 `losa_gather_kernel` -- one thread-block cluster per group, launched
-//    with programmatic dependent launch behind K1.  Each CTA stages the
-//    block's K/V before K1 has finished; then it merges the chunk candidates
-//    of its rows into the row's k pages and writes them into every CTA of the
-//    cluster (distributed shared memory).  Every CTA builds the group's page
-//    union (ascending, with a row mask per page); union slot u belongs to CTA
-//    u % CL, which copies the page's K and V once for the whole GQA group.
-//    While the copies fly the CTA computes the dense suffix of its share of
-//    the block's token rows (stable rows are merged with their untouched
-//    cache and finished here).  The pages are then folded into one
-//    online-softmax partial per row -- bf16: tensor cores, all rows of an
-//    m16 tile at once with a row mask, S = Q K^T and O += P V with P split
-//    into bf16 high and remainder parts; fp32: one warp per row on CUDA cores
-//    -- and each active row's owner CTA combines the partials of every CTA
-//    of the cluster, writes the new o_p / L_p and merges them with the
-//    row's suffix.
+// K2 `losa_gather_kernel` -- CL CTAs per group, launched with programmatic
+//    dependent launch behind K1.  Each CTA stages the block's K/V before K1
+//    has finished; then it merges the chunk candidates of every active row
+//    into the row's k pages and builds the group's page union (ascending,
+//    with a row mask per page); union slot u belongs to CTA u % CL, which
+//    copies the page's K and V once for the whole GQA group.  While the
+//    copies fly the CTA computes the dense suffix of its share of the block's
+//    token rows (stable rows are merged with their untouched cache and
+//    finished here).  The pages are then folded into one online-softmax
+//    partial per row -- bf16: tensor cores, all rows of an m16 tile at once
+//    with a row mask, S = Q K^T and O += P V with P split into bf16 high and
+//    remainder parts; fp32: one warp per row on CUDA cores.  The partials go
+//    to the workspace (L2); the group's last CTA to arrive combines them,
+//    writes the new o_p / L_p and merges them with the rows' suffixes.
 //
 // K1's waits on bulk copies are bounded (clock64); a wait that gives up sets
 // LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA stops.  K2 waits on
-// cp.async groups and cluster barriers only; every CTA of a cluster takes
-// every cluster barrier.
-#include <cooperative_groups.h>
-
+// its own cp.async groups only; no CTA waits for another.
 #include <algorithm>
 #include <mutex>
 
 #include "losa_common.cuh"
 #include "ptx.cuh"
-
-namespace cg = cooperative_groups;
 
 namespace losa {
 
@@ -58,9 +51,12 @@ constexpr int kMaxRingBytes = 128 * 1024;
 constexpr int kStageBytes = 32 * 1024;
 constexpr int kMaxStages = kMaxRingBytes / kStageBytes;
 constexpr int kCandCap = 64;                     // per-warp compaction buffer
-constexpr int kMaxCluster = 16;
+constexpr int kThreadsG = 512;                   // gather kernel: one warp per merged row
+constexpr int kWarpsG = kThreadsG / 32;
+constexpr int kPageWarps = 8;                    // gather kernel: warps sharing an m16 tile's pages
+constexpr int kMaxGatherCtas = kGatherCtas;  // CTAs per group in the gather kernel
 constexpr int kMaxGatherPages = 16;              // pages in flight per K2 CTA
-constexpr int kGatherSmemTarget = 113 * 1024;    // two gather CTAs per SM
+constexpr int kGatherSmemTarget = 113 * 1024;    // room for another CTA on the SM
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
   return a > b ? a : b;
@@ -298,46 +294,61 @@ __device__ __forceinline__ void thread_topk(KeyFn key, int j, int stride, int n,
   }
 }
 
-// Top-k (k <= W) of the keys held by a group of W lanes (W a power of two;
-// groups are aligned inside the warp).  Lane j of a group holds the keys
-// key(i) for i = j, j + W, ... < n (0 = no key).  The threshold tau is the
-// k-th largest of the group's lane maxima: at least k keys reach it, so every
-// key of the top k does too.  The keys >= tau (at most `cap`) are compacted
-// into buf and rank-sorted into out[0..k).  Returns false, for every lane of
-// the warp and before writing anything, if an active group of the warp had
-// more than `cap` survivors.
-template <typename KeyFn>
-__device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long long* buf,
-                                  unsigned long long* out, int cap, bool active) {
-  constexpr int kNV = 32;  // keys a lane keeps in registers
+// Top-k (k <= W) of a row of n <= W * NV bound scores in shared memory
+// (score i is page p0 + i) by a group of W lanes (aligned inside the warp):
+// lane j holds scores j, j + W, ...  The threshold tau is the k-th largest of
+// the lanes' maxima: at least k scores reach it, so every score of the top k
+// does.  Only the scores >= tau (at most kCandCap) become selection keys;
+// they are compacted into buf and rank-sorted into out[0..k) (0 = empty when
+// n < k).  Returns false, for every lane of the warp and before writing
+// anything, if an active group of the warp had more than kCandCap survivors.
+// W and NV are compile-time so that every loop is unrolled without guards
+// (one copy per (W, NV) pair, shared by all kernels).
+template <int W, int NV>
+__device__ __noinline__ bool row_topk(const float* row, int n, int p0, int k,
+                                      unsigned long long* buf, unsigned long long* out,
+                                      bool active) {
   const int lane = threadIdx.x & 31;
-  const int j = lane & (W - 1);
-  if (n > W * kNV) return false;  // (uniform) the caller's other path handles it
-  unsigned long long kx[kNV];
-  unsigned long long lmax = 0ull;
+  const int j = lane & (W - 1), base = lane - j;
+  const unsigned gmask = W == 32 ? 0xffffffffu : (((1u << (W & 31)) - 1u) << base);
+  const unsigned lt = (1u << lane) - 1u;
+  float v[NV];
+  float lmax = -INFINITY;
 #pragma unroll
-  for (int t = 0; t < kNV; ++t) {
-    const int i = j + t * W;
-    kx[t] = i < n ? key(i) : 0ull;
-    lmax = umax64(lmax, kx[t]);
+  for (int t = 0; t < NV; ++t) {
+    v[t] = j + t * W < n ? row[j + t * W] : -INFINITY;
+    lmax = fmaxf(lmax, v[t]);
   }
-  const unsigned long long tau = group_kth_u64(lmax, W, k);
-  int cnt = 0;
+  // tau: the k-th largest lane maximum (rank by value, ties by lane), the
+  // maxima read back from shared memory (broadcast loads, no shuffle chain)
+  float* mx = reinterpret_cast<float*>(buf);
+  mx[j] = lmax;
+  __syncwarp();
+  int rk = 0;
 #pragma unroll
-  for (int t = 0; t < kNV; ++t) cnt += (kx[t] >= tau && kx[t] != 0ull);
-  int incl = cnt;
-#pragma unroll 1
-  for (int o = 1; o < W; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o, W);
-    if (j >= o) incl += y;
+  for (int i = 0; i < W; ++i) {
+    const float o = mx[i];
+    rk += (o > lmax) || (o == lmax && i < j);
   }
-  const int total = __shfl_sync(0xffffffffu, incl, W - 1, W);
-  if (!__all_sync(0xffffffffu, !active || total <= cap)) return false;
+  const unsigned bal = __ballot_sync(0xffffffffu, rk == k - 1) & gmask;
+  const float tau = mx[__ffs(bal) - 1 - base];
+  // survivors: one ballot per register slot gives every lane its positions
+  unsigned bl[NV];
+  int total = 0;
+#pragma unroll
+  for (int t = 0; t < NV; ++t) {
+    bl[t] = __ballot_sync(0xffffffffu, j + t * W < n && v[t] >= tau) & gmask;
+    total += __popc(bl[t]);
+  }
+  if (!__all_sync(0xffffffffu, !active || total <= kCandCap)) return false;
+  __syncwarp();  // the maxima are read before buf takes the survivors
   if (active) {
-    int pos = incl - cnt;
+    int pos = 0;
 #pragma unroll
-    for (int t = 0; t < kNV; ++t)
-      if (kx[t] >= tau && kx[t] != 0ull) buf[pos++] = kx[t];
+    for (int t = 0; t < NV; ++t) {
+      if ((bl[t] >> lane) & 1u) buf[pos + __popc(bl[t] & lt)] = sel_key(v[t], p0 + j + t * W);
+      pos += __popc(bl[t]);
+    }
   }
   __syncwarp();
   if (active) {
@@ -354,6 +365,21 @@ __device__ bool group_topk_filter(KeyFn key, int n, int W, int k, unsigned long 
   }
   __syncwarp();
   return true;
+}
+
+// row_topk for the (W, NV) pair of the launch; false if there is none (the
+// caller falls back to register sort-and-merge).
+__device__ __forceinline__ bool row_topk_dispatch(int W, int NV, const float* row, int n, int p0,
+                                                  int k, unsigned long long* buf,
+                                                  unsigned long long* out, bool active) {
+#define LOSA_ROW_TOPK(w, nv) \
+  if (W == w && NV == nv) return row_topk<w, nv>(row, n, p0, k, buf, out, active);
+  LOSA_ROW_TOPK(4, 8) LOSA_ROW_TOPK(4, 16) LOSA_ROW_TOPK(4, 32) LOSA_ROW_TOPK(4, 64)
+  LOSA_ROW_TOPK(8, 8) LOSA_ROW_TOPK(8, 16) LOSA_ROW_TOPK(8, 32) LOSA_ROW_TOPK(8, 64)
+  LOSA_ROW_TOPK(16, 8) LOSA_ROW_TOPK(16, 16) LOSA_ROW_TOPK(16, 32) LOSA_ROW_TOPK(16, 64)
+  LOSA_ROW_TOPK(32, 8) LOSA_ROW_TOPK(32, 16) LOSA_ROW_TOPK(32, 32) LOSA_ROW_TOPK(32, 64)
+#undef LOSA_ROW_TOPK
+  return false;
 }
 
 int pow2_floor(int x) {
@@ -396,6 +422,7 @@ struct ScanParams {
   int32_t* act_g;                  // workspace [S*Hkv][R + G*B]: act_tok, then act_slot
   int32_t* active_idx;
   unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
+  int* cnt;                        // workspace [S*Hkv]: the gather kernel's arrival counters
   int* status;
   Dims d;
   int scan;       // this launch scores pages (else: the active set only)
@@ -405,6 +432,7 @@ struct ScanParams {
   int sc_stride;  // floats per score row
   int kp;         // register top-k width (2..16), 0 = warp fallback
   int tpr;        // threads per row for the chunk top-k
+  int nv;         // scores per top-k lane (a power of two >= chunk_pages / tpr)
   int mse_t;      // threads per row for the locality score
   ScanLayout lo;
 };
@@ -428,7 +456,7 @@ __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* s
       const float* row = sc + (active ? r : 0) * prm.sc_stride;
       unsigned long long* out = dst_base + static_cast<size_t>(active ? r : 0) * k;
       auto key = [&](int i) { return sel_key(row[i], p0 + i); };
-      if (!group_topk_filter(key, npages, W, k, fbuf + (tid / W) * kCandCap, out, kCandCap,
+      if (!row_topk_dispatch(W, prm.nv, row, npages, p0, k, fbuf + (tid / W) * kCandCap, out,
                              active)) {
         unsigned long long x[KP > 0 ? KP : 1];
         thread_topk<(KP > 0 ? KP : 1)>(key, tid & (W - 1), W, npages, x);
@@ -492,6 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   // the gather kernel may start staging now; it waits for this grid's
   // completion before it reads anything written here
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (tid != 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   char* ring = smem + lo.ring;
   const char* qcs = smem + lo.qc;
@@ -516,6 +545,11 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
+    // launched behind the previous kernel of the stream (programmatic
+    // dependent launch): nothing it may still write or read is touched
+    // before it has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (chunk == 0) prm.cnt[sg] = 0;
     const size_t qoff = (static_cast<size_t>(s) * d.Hq + g * G) * B * rowb;
     mbar_expect_tx(&mbar[kMaxStages], 2 * qbytes);
     bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, &mbar[kMaxStages]);
@@ -933,7 +967,7 @@ struct GatherLayout {
   int qs;       // this CTA's suffix rows' queries (same formats)
   int ocache;   // cached o_p rows of this CTA's stable suffix rows
   int lcache;   // their cached L_p
-  int sel_own, sel_all, bitmap, wbase, lpages, masks, part, sfx, misc, ps, mbuf, total;
+  int sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf, total;
 };
 
 struct GatherParams {
@@ -950,9 +984,12 @@ struct GatherParams {
   int32_t* union_count;
   const int32_t* act_g;
   const unsigned long long* cand;
+  float* part_g;    // workspace [S*Hkv][CL][R][kPartStride]: every CTA's row partials
+  float* sfx_g;     // workspace [S*Hkv][R][kPartStride]: active rows' suffix (L_s, -, -, -, o_s)
+  int* cnt;         // workspace [S*Hkv]: CTAs of the group done (zeroed by the scan kernel)
   int* status;
   Dims d;
-  int CL;        // CTAs per cluster
+  int CL;        // CTAs per group
   int max_lp;    // max union pages per CTA
   int ngp;       // pages in flight per CTA
   int n_oa;      // max active rows owned per CTA
@@ -962,22 +999,34 @@ struct GatherParams {
 };
 
 // The k best chunk candidates of row r (keys, descending) -> out[0..k).
-// Fast path: lane c holds chunk c's sorted list; threshold = k-th largest
-// list head; the survivors are rank-sorted.  Fallback: sort-and-merge trees
-// or k rounds of warp argmax.
+// Fast path: lane c holds chunk c's sorted list; the threshold is the k-th
+// largest list head (ranked from shared memory, hb: 32 keys per warp); the
+// keys at or above it are placed by ballots and rank-sorted.  Fallback:
+// sort-and-merge trees or k rounds of warp argmax.
 template <int KP>
 __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg,
-                                          unsigned long long* out, unsigned long long* fb) {
+                                          unsigned long long* out, unsigned long long* fb,
+                                          unsigned long long* hb) {
   const Dims& d = prm.d;
   const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
   const unsigned long long* base = prm.cand + static_cast<size_t>(sg) * nc * R * k;
   if (KP > 0) {
     constexpr int KQ = KP > 0 ? KP : 1;
+    const unsigned lt = (1u << lane) - 1u;
     unsigned long long x[KQ];
     {
       const unsigned long long* lst = base + (static_cast<size_t>(lane) * R + r) * k;
+      if (KQ >= 2 && k == KQ && lane < nc) {  // 16-byte loads (k even: 16-byte aligned lists)
 #pragma unroll
-      for (int i = 0; i < KQ; ++i) x[i] = (lane < nc && i < k) ? __ldcg(lst + i) : 0ull;
+        for (int i = 0; i < KQ / 2; ++i) {
+          const ulonglong2 v = __ldcg(reinterpret_cast<const ulonglong2*>(lst) + i);
+          x[2 * i] = v.x;
+          x[(2 * i + 1) % KQ] = v.y;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < KQ; ++i) x[i] = (lane < nc && i < k) ? __ldcg(lst + i) : 0ull;
+      }
     }
 #pragma unroll 1
     for (int c = lane + 32; c < nc; c += 32) {  // more than 32 chunks: fold lists
@@ -987,23 +1036,30 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg
       for (int i = 0; i < KQ; ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
       merge_top<KQ>(x, y);
     }
-    // threshold from the list heads (every list is sorted, descending)
-    const unsigned long long tau = group_kth_u64(x[0], 32, k);
-    int cnt = 0;
+    // threshold: the k-th largest list head (every list is sorted, descending)
+    hb[lane] = x[0];
+    __syncwarp();
+    int rk = 0;
 #pragma unroll
-    for (int i = 0; i < KQ; ++i) cnt += (x[i] >= tau && x[i] != 0ull);
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+    for (int i = 0; i < 32; ++i) {
+      const unsigned long long o = hb[i];
+      rk += (o > x[0]) || (o == x[0] && i < lane);
     }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    if (total <= kCandCap) {
-      int pos = incl - cnt;
+    const unsigned long long tau = hb[__ffs(__ballot_sync(0xffffffffu, rk == k - 1)) - 1];
+    unsigned bl[KQ];
+    int total = 0;
 #pragma unroll
-      for (int i = 0; i < KQ; ++i)
-        if (x[i] >= tau && x[i] != 0ull) fb[pos++] = x[i];
+    for (int i = 0; i < KQ; ++i) {
+      bl[i] = __ballot_sync(0xffffffffu, x[i] >= tau && x[i] != 0ull);
+      total += __popc(bl[i]);
+    }
+    if (total <= kCandCap) {
+      int pos = 0;
+#pragma unroll
+      for (int i = 0; i < KQ; ++i) {
+        if ((bl[i] >> lane) & 1u) fb[pos + __popc(bl[i] & lt)] = x[i];
+        pos += __popc(bl[i]);
+      }
       __syncwarp();
 #pragma unroll 1
       for (int t = lane; t < total; t += 32) {
@@ -1032,15 +1088,15 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg
 }
 
 template <int DT, int KP>
-__global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherParams prm) {
+__global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherParams prm) {
   extern __shared__ __align__(1024) char smem[];
-  cg::cluster_group cluster = cg::this_cluster();
   const Dims& d = prm.d;
   const GatherLayout& lo = prm.lo;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g4 = lane >> 2, t4 = lane & 3;
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int CL = prm.CL;
+  const int rank = blockIdx.x;  // this CTA's place among the group's CL CTAs
+  constexpr int CL = kGatherCtas;
+  static_assert((CL & (CL - 1)) == 0, "CTAs per group: a power of two");
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
@@ -1058,14 +1114,12 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   char* qs = smem + lo.qs;
   float* ocache = reinterpret_cast<float*>(smem + lo.ocache);
   float* lcache = reinterpret_cast<float*>(smem + lo.lcache);
-  int32_t* sel_own = reinterpret_cast<int32_t*>(smem + lo.sel_own);
   int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel_all);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + lo.bitmap);
   int32_t* wbase = reinterpret_cast<int32_t*>(smem + lo.wbase);
   int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
-  float* sfx = reinterpret_cast<float*>(smem + lo.sfx);    // [n_oa][kPartStride]: (L_s, -, -, -, o_s)
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
@@ -1077,17 +1131,33 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   int32_t* sfx_tok = act_slot + GB;    // [n_oa + n_os]: token row of each suffix row
   float* psw = Ps + warp * 16;
 
-  // barrier 0: before touching another CTA's shared memory, every CTA of the
-  // cluster must be running; the wait comes after the selection
-  cluster_arrive_relaxed();
+  const int n_oa = R > rank ? (R - rank + CL - 1) / CL : 0;
+  const int n_os = GB - R > rank ? (GB - R - rank + CL - 1) / CL : 0;
+  const int ns = n_oa + n_os;
+  const bool sel = !d.all_pages;
+  // after the selection the CTA splits in two halves of kThreads threads:
+  // warps [0, 8) build the page union and issue the gather copies, warps
+  // [8, 16) stage the suffix rows and compute the suffix
+  const bool uhalf = tid < kThreads;
+  const int htid = uhalf ? tid : tid - kThreads;
+  // the next step's scan kernel may be scheduled now; it waits for this
+  // grid's completion before it touches anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // ---- the block's K and V (cp.async group 0; rows >= B are zero)
-  {
+#pragma unroll 1
+  for (int e = tid; e < R * kPartStride; e += kThreadsG)  // empty partials
+    part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+  if (sel) {
+#pragma unroll 1
+    for (int w = tid; w < nwords; w += kThreadsG) bitmap[w] = 0u;
+  }
+  // ---- the block's K and V (suffix half, cp.async group 0; rows >= B zero)
+  if (!uhalf) {
     const char* kbg = static_cast<const char*>(prm.kb) + static_cast<size_t>(sg) * B * rowb;
     const char* vbg = static_cast<const char*>(prm.vb) + static_cast<size_t>(sg) * B * rowb;
     const int per = bpad * cpr;
 #pragma unroll 1
-    for (int e = tid; e < 2 * per; e += kThreads) {
+    for (int e = htid; e < 2 * per; e += kThreads) {
       const int h = e >= per ? 1 : 0, rem = e - h * per, j = rem / cpr, c = rem - j * cpr;
       const bool ok = j < B;
       const char* src = (h ? vbg : kbg) + static_cast<size_t>(ok ? j : 0) * rowb + c * 16;
@@ -1095,9 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
     }
     cp_async_commit();
   }
-#pragma unroll 1
-  for (int e = tid; e < R * kPartStride; e += kThreads)  // empty partials
-    part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+  __syncthreads();
 
   // everything below reads what the scan kernel wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1105,77 +1173,20 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
   {
     const int32_t* actg = prm.act_g + static_cast<size_t>(sg) * (R + GB);
 #pragma unroll 1
-    for (int e = tid; e < R + GB; e += kThreads) act_tok[e] = __ldcg(actg + e);
-  }
-  __syncthreads();
-
-  // ---- this CTA's suffix rows: its active rows r = rank + CL*j first, then
-  // every CL-th stable token row
-  const int n_oa = R > rank ? (R - rank + CL - 1) / CL : 0;
-  const int n_os = GB - R > rank ? (GB - R - rank + CL - 1) / CL : 0;
-  const int ns = n_oa + n_os;
-  {
-    bool st = false;
-    int pre = 0;
-    if (warp < 4) {  // G*B <= 128 token rows
-      st = tid < GB && act_slot[tid] < 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, st);
-      pre = __popc(bal & ((1u << lane) - 1u));
-      if (lane == 0) s_wt[warp] = __popc(bal);
-    }
-#pragma unroll 1
-    for (int j = tid; j < n_oa; j += kThreads) {
-      const int r = rank + CL * j;
-      sfx_tok[j] = (r / A) * B + act_tok[r];
-    }
-    __syncthreads();
-    if (st) {
-      for (int w = 0; w < warp; ++w) pre += s_wt[w];
-      if (pre % CL == rank) sfx_tok[n_oa + pre / CL] = tid;
-    }
-  }
-  __syncthreads();
-
-  // ---- cp.async group 1: queries of the suffix rows and of the active rows,
-  // cached state of the stable suffix rows
-  {
-    const char* qg = static_cast<const char*>(prm.qc) + grow0 * rowb;
-    const int nsr = DT == LOSA_BF16 ? (ns + 15) / 16 * 16 : ns;
-#pragma unroll 1
-    for (int e = tid; e < nsr * cpr; e += kThreads) {
-      const int n = e / cpr, c = e - n * cpr;
-      const bool ok = n < ns;
-      cp_async16(su32(qs + tile_off<DT>(n, c)),
-                 qg + static_cast<size_t>(ok ? sfx_tok[n] : 0) * rowb + c * 16, ok ? 16u : 0u);
-    }
-    const int nar = DT == LOSA_BF16 ? (R + 15) / 16 * 16 : R;
-#pragma unroll 1
-    for (int e = tid; e < nar * cpr; e += kThreads) {
-      const int r = e / cpr, c = e - r * cpr;
-      const bool ok = r < R;
-      const int tok = ok ? (r / A) * B + act_tok[r] : 0;
-      cp_async16(su32(qa + tile_off<DT>(r, c)), qg + static_cast<size_t>(tok) * rowb + c * 16,
-                 ok ? 16u : 0u);
-    }
-#pragma unroll 1
-    for (int e = tid; e < n_os * (kD / 4); e += kThreads) {
-      const int n = e / (kD / 4), c = e - n * (kD / 4);
-      const size_t grow = grow0 + sfx_tok[n_oa + n];
-      cp_async16(su32(ocache + n * kD + 4 * c), prm.o_p + grow * kD + 4 * c, 16u);
-    }
-#pragma unroll 1
-    for (int n = tid; n < n_os; n += kThreads)
-      cp_async4(su32(lcache + n), prm.l_p + grow0 + sfx_tok[n_oa + n]);
-    cp_async_commit();
+    for (int e = tid; e < R + GB; e += kThreadsG) act_tok[e] = __ldcg(actg + e);
   }
 
-  // ---- this CTA's rows (r % CL == rank): the row's k pages, ascending
-  if (!d.all_pages) {
+  // ---- every row's k pages, ascending, into sel_all and the union bitmap
+  // (each CTA of the group merges all rows; the CTA with r % CL == rank
+  // reports row r)
+  if (sel) {
 #pragma unroll 1
-    for (int r = rank + CL * warp; r < R; r += CL * kWarps) {
-      unsigned long long* best = mbuf + (kWarps + warp) * kCandCap;
-      merge_row<KP>(prm, r, sg, best, mbuf + warp * kCandCap);
-      int32_t* dst = sel_own + (r / CL) * k;
+    for (int r = warp; r < R; r += kWarpsG) {
+      unsigned long long* best = mbuf + (kWarpsG + warp) * kCandCap;
+      merge_row<KP>(prm, r, sg, best, mbuf + warp * kCandCap,
+                    mbuf + 2 * kWarpsG * kCandCap + warp * 32);
+      int32_t* dst = sel_all + r * k;
+      const bool report = prm.page_idx && r % CL == rank;
 #pragma unroll 1
       for (int j = lane; j < k; j += 32) {
         const int pj = key_index(best[j]);
@@ -1183,7 +1194,9 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
 #pragma unroll 4
         for (int u = 0; u < k; ++u) rk += key_index(best[u]) < pj;
         dst[rk] = pj;
-        if (prm.page_idx) {
+        if (pj >= 0 && pj < d.P) atomicOr(&bitmap[pj >> 5], 1u << (pj & 31));
+        else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+        if (report) {
           const int hl = r / A, a = r % A;
           prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + rk] = pj;
         }
@@ -1195,210 +1208,255 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
     for (int r = rank; r < R; r += CL) {
       const int hl = r / A, a = r % A;
 #pragma unroll 1
-      for (int j = tid; j < k; j += kThreads)
+      for (int j = tid; j < k; j += kThreadsG)
         prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + j] = j;
     }
   }
   __syncthreads();
-  cluster_wait();  // barrier 0
-  if (!d.all_pages) {  // this CTA's rows' pages -> every CTA of the cluster
-#pragma unroll 1
-    for (int e = tid; e < n_oa * CL * k; e += kThreads) {
-      const int j = e / (CL * k), rem = e - j * CL * k, c = rem / k, i = rem - c * k;
-      const int r = rank + CL * j;
-      cluster.map_shared_rank(sel_all, c)[r * k + i] = sel_own[j * k + i];
-    }
-  }
-  cluster_arrive();
-  cluster_wait();  // barrier 1: every row's pages are in every CTA
 
-  // ---- union of the group's pages and this CTA's share
-  if (d.all_pages) {
-    const int U = R > 0 ? d.P : 0;
-    const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
-    if (tid == 0) {
-      *s_nlp = nlp;
-      if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
-    }
-#pragma unroll 1
-    for (int j = tid; j < min(nlp, prm.max_lp); j += kThreads) lpages[j] = rank + j * CL;
-#pragma unroll 1
-    for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) {
-      const int w = e % d.MW;
-      const int nb = min(32, R - 32 * w);
-      masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
-    }
-  } else {
-#pragma unroll 1
-    for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
-    __syncthreads();
-#pragma unroll 1
-    for (int e = tid; e < R * k; e += kThreads) {
-      const int p = sel_all[e];
-      if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
-      else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-    }
-    __syncthreads();
-    if (warp == 0) {  // exclusive prefix of word popcounts
-      const int per = (nwords + 31) / 32;
-      const int w0 = lane * per, w1 = min(nwords, w0 + per);
-      int sum = 0;
-#pragma unroll 1
-      for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
-      int incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int run = incl - sum;
-#pragma unroll 1
-      for (int w = w0; w < w1; ++w) {
-        wbase[w] = run;
-        run += __popc(bitmap[w]);
-      }
-      if (lane == 31) *s_U = incl;
-    }
-    __syncthreads();
-    const int U = *s_U;
-    const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
-    if (tid == 0) {
-      *s_nlp = nlp;
-      if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
-    }
-#pragma unroll 1
-    for (int w = tid; w < nwords; w += kThreads) {
-      uint32_t bits = bitmap[w];
-      int pos = wbase[w];
-#pragma unroll 1
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (pos % CL == rank && pos / CL < prm.max_lp) lpages[pos / CL] = w * 32 + b;
-        ++pos;
-      }
-    }
-#pragma unroll 1
-    for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) masks[e] = 0u;
-    __syncthreads();
-#pragma unroll 1
-    for (int e = tid; e < R * k; e += kThreads) {
-      const int p = sel_all[e];
-      if (p < 0 || p >= d.P) continue;
-      const int w = p >> 5;
-      const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
-      if (u % CL != rank) continue;
-      const int r = e / k;
-      if (u / CL < prm.max_lp) atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
-      else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-    }
-  }
-  __syncthreads();
-
-  // ---- gather copies (cp.async group 2): this CTA's union pages, in batches
-  // of ngp; rows past the prefix end are zero
-  const int nlp = min(*s_nlp, prm.max_lp);
-  auto issue_batch = [&](int b0) {
+  // gather copies (cp.async, union half): this CTA's union pages b0 ..
+  // b0 + ngp into the page slots; rows past the prefix end are zero
+  auto issue_batch = [&](int b0, int nlp, int t0, int nthr) {
     const int nb = min(prm.ngp, nlp - b0);
-    constexpr int per = kPS * cpr;
+    constexpr int per = kPS * cpr;  // chunks of one page's K (or V)
 #pragma unroll 1
-    for (int e = tid; e < nb * 2 * per; e += kThreads) {
-      const int i = e / (2 * per), rem = e - i * 2 * per, h = rem / per, rr = rem - h * per;
-      const int j = rr / cpr, c = rr - j * cpr;
+    for (int i = 0; i < nb; ++i) {
       const int p = lpages[b0 + i];
-      const bool ok = p * kPS + j < d.L;
-      const size_t off =
-          (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS + (ok ? j : 0)) * rowb + c * 16;
-      cp_async16(su32(region + (2 * i + h) * pbytes + tile_off<DT>(j, c)),
-                 static_cast<const char*>(h ? prm.V : prm.K) + off, ok ? 16u : 0u);
+      const size_t off = (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS) * rowb;
+      const char* kp = static_cast<const char*>(prm.K) + off;
+      const char* vp = static_cast<const char*>(prm.V) + off;
+      char* dk = region + 2 * i * pbytes;
+#pragma unroll 1
+      for (int e = t0; e < per; e += nthr) {
+        const int j = e / cpr, c = e - j * cpr;
+        const bool ok = p * kPS + j < d.L;
+        const int so = (ok ? j : 0) * rowb + c * 16;
+        cp_async16(su32(dk + tile_off<DT>(j, c)), kp + so, ok ? 16u : 0u);
+        cp_async16(su32(dk + pbytes + tile_off<DT>(j, c)), vp + so, ok ? 16u : 0u);
+      }
     }
     cp_async_commit();
   };
-  issue_batch(0);
 
-  // ---- dense suffix of this CTA's rows (hidden behind the gather copies):
-  // stable rows merge with their cached state and are finished; active rows
-  // keep (L_s, o_s) for the combine
-  cp_async_wait<1>();  // groups 0 and 1
-  __syncthreads();
-  if (DT == LOSA_BF16) {
-    const int nmt = (ns + 15) / 16;
+  if (uhalf) {
+    // ---- union of the group's pages and this CTA's share (slots u % CL)
+    if (d.all_pages) {
+      const int U = R > 0 ? d.P : 0;
+      const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
+      if (tid == 0) {
+        *s_nlp = nlp;
+        if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
+      }
 #pragma unroll 1
-    for (int mt = warp; mt < nmt; mt += kWarps) {
-      TileAcc t;
-      tile_init(t);
+      for (int j = tid; j < min(nlp, prm.max_lp); j += kThreads) lpages[j] = rank + j * CL;
 #pragma unroll 1
-      for (int j0 = 0; j0 < B; j0 += kPS)
-        tile_attend(t, qs + mt * 16 * 256, kbv + j0 * 256, kbv + (bpad + j0) * 256, 0xffffu,
-                    min(kPS, B - j0), d.scale_log2);
-      tile_finish(t);
+      for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) {
+        const int w = e % d.MW;
+        const int nb = min(32, R - 32 * w);
+        masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+      }
+    } else {
+      if (warp == 0) {  // exclusive prefix of word popcounts
+        const int per = (nwords + 31) / 32;
+        const int w0 = lane * per, w1 = min(nwords, w0 + per);
+        int sum = 0;
+#pragma unroll 1
+        for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
+        int incl = sum;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int n = mt * 16 + g4 + 8 * h;
-        if (n >= ns) continue;
-        const float inv = __frcp_rn(t.l[h]);
-        const float Ls = (t.m[h] + __log2f(t.l[h])) * kLn2;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+#pragma unroll 1
+        for (int w = w0; w < w1; ++w) {
+          wbase[w] = run;
+          run += __popc(bitmap[w]);
+        }
+        if (lane == 31) *s_U = incl;
+      }
+      bar_sync(1, kThreads);
+      const int U = *s_U;
+      const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
+      if (tid == 0) {
+        *s_nlp = nlp;
+        if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
+      }
+#pragma unroll 1
+      for (int w = tid; w < nwords; w += kThreads) {
+        uint32_t bits = bitmap[w];
+        int pos = wbase[w];
+#pragma unroll 1
+        while (bits) {
+          const int b = __ffs(bits) - 1;
+          bits &= bits - 1;
+          if (pos % CL == rank && pos / CL < prm.max_lp) lpages[pos / CL] = w * 32 + b;
+          ++pos;
+        }
+      }
+#pragma unroll 1
+      for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) masks[e] = 0u;
+      bar_sync(1, kThreads);
+#pragma unroll 1
+      for (int e = tid; e < R * k; e += kThreads) {
+        const int p = sel_all[e];
+        if (p < 0 || p >= d.P) continue;
+        const int w = p >> 5;
+        const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
+        if (u % CL != rank) continue;
+        const int r = e / k;
+        if (u / CL < prm.max_lp) atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
+        else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+      }
+    }
+    bar_sync(1, kThreads);
+    issue_batch(0, min(*s_nlp, prm.max_lp), tid, kThreads);
+    cp_async_wait<0>();  // this half's copies: the gathered pages
+  } else {
+    // ---- this CTA's suffix rows: its active rows r = rank + CL*j first, then
+    // every CL-th stable token row
+    {
+      const int hw = htid >> 5;
+      bool st = false;
+      int pre = 0;
+      if (hw < 4) {  // G*B <= 128 token rows
+        st = htid < GB && act_slot[htid] < 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, st);
+        pre = __popc(bal & ((1u << lane) - 1u));
+        if (lane == 0) s_wt[hw] = __popc(bal);
+      }
+#pragma unroll 1
+      for (int j = htid; j < n_oa; j += kThreads) {
+        const int r = rank + CL * j;
+        sfx_tok[j] = (r / A) * B + act_tok[r];
+      }
+      bar_sync(2, kThreads);
+      if (st) {
+        for (int w = 0; w < hw; ++w) pre += s_wt[w];
+        if (pre % CL == rank) sfx_tok[n_oa + pre / CL] = htid;
+      }
+    }
+    bar_sync(2, kThreads);
+    // ---- cp.async group 1: queries of the suffix rows and of the active
+    // rows, cached state of the stable suffix rows
+    {
+      const char* qg = static_cast<const char*>(prm.qc) + grow0 * rowb;
+      const int nsr = DT == LOSA_BF16 ? (ns + 15) / 16 * 16 : ns;
+#pragma unroll 1
+      for (int e = htid; e < nsr * cpr; e += kThreads) {
+        const int n = e / cpr, c = e - n * cpr;
+        const bool ok = n < ns;
+        cp_async16(su32(qs + tile_off<DT>(n, c)),
+                   qg + static_cast<size_t>(ok ? sfx_tok[n] : 0) * rowb + c * 16, ok ? 16u : 0u);
+      }
+      const int nar = DT == LOSA_BF16 ? (R + 15) / 16 * 16 : R;
+#pragma unroll 1
+      for (int e = htid; e < nar * cpr; e += kThreads) {
+        const int r = e / cpr, c = e - r * cpr;
+        const bool ok = r < R;
+        const int tok = ok ? (r / A) * B + act_tok[r] : 0;
+        cp_async16(su32(qa + tile_off<DT>(r, c)), qg + static_cast<size_t>(tok) * rowb + c * 16,
+                   ok ? 16u : 0u);
+      }
+#pragma unroll 1
+      for (int e = htid; e < n_os * (kD / 4); e += kThreads) {
+        const int n = e / (kD / 4), c = e - n * (kD / 4);
+        const size_t grow = grow0 + sfx_tok[n_oa + n];
+        cp_async16(su32(ocache + n * kD + 4 * c), prm.o_p + grow * kD + 4 * c, 16u);
+      }
+#pragma unroll 1
+      for (int n = htid; n < n_os; n += kThreads)
+        cp_async4(su32(lcache + n), prm.l_p + grow0 + sfx_tok[n_oa + n]);
+      cp_async_commit();
+    }
+    cp_async_wait<0>();  // this half's copies: block K/V, queries, cached state
+    bar_sync(2, kThreads);
+
+    // ---- dense suffix of this CTA's rows: stable rows merge with their
+    // cached state and are finished; active rows leave (L_s, o_s) for the
+    // combine
+    const int hw = htid >> 5;
+    if (DT == LOSA_BF16) {
+      const int nmt = (ns + 15) / 16;
+#pragma unroll 1
+      for (int mt = hw; mt < nmt; mt += kWarps) {
+        TileAcc t;
+        tile_init(t);
+#pragma unroll 1
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          tile_attend(t, qs + mt * 16 * 256, kbv + j0 * 256, kbv + (bpad + j0) * 256, 0xffffu,
+                      min(kPS, B - j0), d.scale_log2);
+        tile_finish(t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int n = mt * 16 + g4 + 8 * h;
+          if (n >= ns) continue;
+          const float inv = __frcp_rn(t.l[h]);
+          const float Ls = (t.m[h] + __log2f(t.l[h])) * kLn2;
+          if (n < n_oa) {
+            float* dst = prm.sfx_g + (static_cast<size_t>(sg) * R + rank + CL * n) * kPartStride;
+            if (t4 == 0) dst[0] = Ls;
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              *reinterpret_cast<float2*>(dst + 4 + c * 8 + 2 * t4) =
+                  make_float2(t.o[c][2 * h] * inv, t.o[c][2 * h + 1] * inv);
+          } else {
+            const int m = n - n_oa;
+            const size_t grow = grow0 + sfx_tok[n];
+            float wa, wb, L;
+            lse_weights(lcache[m], Ls, wa, wb, L);
+            const float* op = ocache + m * kD;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int ch = c * 8 + 2 * t4;
+              const float2 o = *reinterpret_cast<const float2*>(op + ch);
+              *reinterpret_cast<float2*>(prm.out + grow * kD + ch) =
+                  make_float2(wa * o.x + wb * (t.o[c][2 * h] * inv),
+                              wa * o.y + wb * (t.o[c][2 * h + 1] * inv));
+            }
+            if (prm.out_lse && t4 == 0) prm.out_lse[grow] = L;
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int n = hw; n < ns; n += kWarps) {
+        const float4 q = row4<DT>(qs, n, lane);
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          attend_page<DT>(q, kbv + j0 * rowb, kbv + (bpad + j0) * rowb, min(kPS, B - j0),
+                          d.scale_log2, m, l, acc, psw);
+        const float inv = __frcp_rn(l);
+        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        const float Ls = (m + __log2f(l)) * kLn2;
         if (n < n_oa) {
-          float* dst = sfx + n * kPartStride;
-          if (t4 == 0) dst[0] = Ls;
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<float2*>(dst + 4 + c * 8 + 2 * t4) =
-                make_float2(t.o[c][2 * h] * inv, t.o[c][2 * h + 1] * inv);
+          float* dst = prm.sfx_g + (static_cast<size_t>(sg) * R + rank + CL * n) * kPartStride;
+          if (lane == 0) dst[0] = Ls;
+          *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
         } else {
-          const int m = n - n_oa;
+          const int mm = n - n_oa;
           const size_t grow = grow0 + sfx_tok[n];
           float wa, wb, L;
-          lse_weights(lcache[m], Ls, wa, wb, L);
-          const float* op = ocache + m * kD;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int ch = c * 8 + 2 * t4;
-            const float2 o = *reinterpret_cast<const float2*>(op + ch);
-            *reinterpret_cast<float2*>(prm.out + grow * kD + ch) =
-                make_float2(wa * o.x + wb * (t.o[c][2 * h] * inv), wa * o.y + wb * (t.o[c][2 * h + 1] * inv));
-          }
-          if (prm.out_lse && t4 == 0) prm.out_lse[grow] = L;
+          lse_weights(lcache[mm], Ls, wa, wb, L);
+          const float4 op = *reinterpret_cast<const float4*>(ocache + mm * kD + 4 * lane);
+          *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+              make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                          wa * op.w + wb * os.w);
+          if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
         }
       }
     }
-  } else {
-#pragma unroll 1
-    for (int n = warp; n < ns; n += kWarps) {
-      const float4 q = row4<DT>(qs, n, lane);
-      float m = -INFINITY, l = 0.f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-      for (int j0 = 0; j0 < B; j0 += kPS)
-        attend_page<DT>(q, kbv + j0 * rowb, kbv + (bpad + j0) * rowb, min(kPS, B - j0),
-                        d.scale_log2, m, l, acc, psw);
-      const float inv = __frcp_rn(l);
-      const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      const float Ls = (m + __log2f(l)) * kLn2;
-      if (n < n_oa) {
-        float* dst = sfx + n * kPartStride;
-        if (lane == 0) dst[0] = Ls;
-        *reinterpret_cast<float4*>(dst + 4 + 4 * lane) = os;
-      } else {
-        const int mm = n - n_oa;
-        const size_t grow = grow0 + sfx_tok[n];
-        float wa, wb, L;
-        lse_weights(lcache[mm], Ls, wa, wb, L);
-        const float4 op = *reinterpret_cast<const float4*>(ocache + mm * kD + 4 * lane);
-        *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
-            make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
-                        wa * op.w + wb * os.w);
-        if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
-      }
-    }
   }
+  __syncthreads();
+  const int nlp = min(*s_nlp, prm.max_lp);
 
   // ---- the union pages -> one partial per row (part)
-  cp_async_wait<0>();
-  __syncthreads();
   if (DT == LOSA_BF16) {
     const int ntm = (R + 15) / 16;
-    const int wpm = ntm > 0 ? kWarps / ntm : kWarps;
+    const int wpm = ntm > 0 ? max(1, kPageWarps / ntm) : kWarpsG;  // page warps per m16 tile
     const int mt = warp / wpm, sub = warp % wpm;
     const bool aw = mt < ntm;
     TileAcc t;
@@ -1416,7 +1474,7 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       }
       if (b0 + prm.ngp < nlp) {  // next batch into the same slots
         __syncthreads();
-        issue_batch(b0 + prm.ngp);
+        issue_batch(b0 + prm.ngp, nlp, tid, kThreadsG);
         cp_async_wait<0>();
         __syncthreads();
       }
@@ -1430,26 +1488,35 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       if (aw) tile_store(t, wp + warp * 16 * kPartStride, 16);
       __syncthreads();
 #pragma unroll 1
-      for (int r = warp; r < R; r += kWarps) {
+      for (int r = warp; r < R; r += kWarpsG) {
         const int m16 = r >> 4, i = r & 15;
+        float mw[kPageWarps], lw[kPageWarps];
+        float4 aw4[kPageWarps];
+#pragma unroll
+        for (int w = 0; w < kPageWarps; ++w) {
+          mw[w] = -INFINITY;
+          if (w < wpm) {
+            const float* pr = wp + ((m16 * wpm + w) * 16 + i) * kPartStride;
+            mw[w] = pr[0];
+            lw[w] = pr[1];
+            aw4[w] = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+          }
+        }
         float M = -INFINITY;
-#pragma unroll 1
-        for (int w = 0; w < wpm; ++w) M = fmaxf(M, wp[((m16 * wpm + w) * 16 + i) * kPartStride]);
+#pragma unroll
+        for (int w = 0; w < kPageWarps; ++w) M = fmaxf(M, mw[w]);
         if (M == -INFINITY) continue;  // none of this CTA's pages serve row r
         float l = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-        for (int w = 0; w < wpm; ++w) {
-          const float* pr = wp + ((m16 * wpm + w) * 16 + i) * kPartStride;
-          const float mw = pr[0];
-          if (mw == -INFINITY) continue;
-          const float wgt = exp2f(mw - M);
-          l += wgt * pr[1];
-          const float4 a = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
-          acc.x += wgt * a.x;
-          acc.y += wgt * a.y;
-          acc.z += wgt * a.z;
-          acc.w += wgt * a.w;
+#pragma unroll
+        for (int w = 0; w < kPageWarps; ++w) {
+          if (mw[w] == -INFINITY) continue;
+          const float wgt = exp2f(mw[w] - M);
+          l += wgt * lw[w];
+          acc.x += wgt * aw4[w].x;
+          acc.y += wgt * aw4[w].y;
+          acc.z += wgt * aw4[w].z;
+          acc.w += wgt * aw4[w].w;
         }
         float* dst = part + r * kPartStride;
         if (lane == 0) {
@@ -1464,7 +1531,7 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
     for (int b0 = 0; b0 < nlp; b0 += prm.ngp) {
       const int nb = min(prm.ngp, nlp - b0);
 #pragma unroll 1
-      for (int r = warp; r < R; r += kWarps) {
+      for (int r = warp; r < R; r += kWarpsG) {
         bool have = false;
 #pragma unroll 1
         for (int i = 0; i < nb; ++i) have |= (masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u;
@@ -1489,27 +1556,43 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
       }
       if (b0 + prm.ngp < nlp) {
         __syncthreads();
-        issue_batch(b0 + prm.ngp);
+        issue_batch(b0 + prm.ngp, nlp, tid, kThreadsG);
         cp_async_wait<0>();
         __syncthreads();
       }
     }
   }
   __syncthreads();
-  cluster_arrive();
-  cluster_wait();  // barrier 2: every CTA's partials are complete
 
-  // ---- combine the partials of this CTA's rows from every CTA of the
-  // cluster (all loads issued before any is used), cache write-back, merge
-  // with the suffix
+  // ---- publish this CTA's row partials; the group's last CTA to finish
+  // combines every row
+  {
+    float4* dstp = reinterpret_cast<float4*>(
+        prm.part_g + (static_cast<size_t>(sg) * CL + rank) * R * kPartStride);
+    const float4* srcp = reinterpret_cast<const float4*>(part);
 #pragma unroll 1
-  for (int j = warp; j < n_oa; j += kWarps) {
-    const int r = rank + CL * j;
-    // CTAs in fixed order (deterministic), eight partials in flight at a time
+    for (int e = tid; e < R * kPartStride / 4; e += kThreadsG) dstp[e] = srcp[e];
+  }
+  __syncthreads();
+  int* s_last = misc + 2;
+  if (tid == 0) {
+    __threadfence();  // this CTA's partials and suffixes before its arrival
+    *s_last = atomicAdd(prm.cnt + sg, 1) == CL - 1;
+  }
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();  // every other CTA's writes are visible past its arrival
+
+  // ---- combine: per row, the partials of the CL CTAs in fixed order
+  // (deterministic), eight in flight at a time; cache write-back; merge with
+  // the suffix
+#pragma unroll 1
+  for (int r = warp; r < R; r += kWarpsG) {
+    const float* base = prm.part_g + (static_cast<size_t>(sg) * CL * R + r) * kPartStride;
     float M = -INFINITY, lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int h = 0; h < kMaxCluster; h += 8) {
+    for (int h = 0; h < kMaxGatherCtas; h += 8) {
       if (h < CL) {
         float mc[8], lc[8];
         float4 ac[8];
@@ -1517,10 +1600,10 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
         for (int i = 0; i < 8; ++i) {
           mc[i] = -INFINITY;
           if (h + i < CL) {
-            const float* pr = cluster.map_shared_rank(part, h + i) + r * kPartStride;
-            mc[i] = pr[0];
-            lc[i] = pr[1];
-            ac[i] = *reinterpret_cast<const float4*>(pr + 4 + 4 * lane);
+            const float* pr = base + static_cast<size_t>(h + i) * R * kPartStride;
+            mc[i] = __ldcg(pr);
+            lc[i] = __ldcg(pr + 1);
+            ac[i] = __ldcg(reinterpret_cast<const float4*>(pr + 4) + lane);
           }
         }
         float Mh = M;
@@ -1554,18 +1637,15 @@ __global__ void __launch_bounds__(kThreads, 2) losa_gather_kernel(const GatherPa
     const size_t grow = grow0 + (r / A) * B + act_tok[r];
     *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
     if (lane == 0) prm.l_p[grow] = Lp;
-    const float* sx = sfx + j * kPartStride;
-    const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
+    const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
+    const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4) + lane);
     float wa, wb, L;
-    lse_weights(Lp, sx[0], wa, wb, L);
+    lse_weights(Lp, __ldcg(sx), wa, wb, L);
     *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
         make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
                     wa * op.w + wb * os.w);
     if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
   }
-  // barrier 3: no CTA leaves while another may still read its partials
-  cluster_arrive();
-  cluster_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -1602,6 +1682,8 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   prm->tpr = std::min(32, std::max(pow2_floor(std::max(1, kThreads / std::max(d.R, 1))),
                                    d.k <= 1 ? 1 : pow2_floor(2 * d.k - 1)));
   prm->mse_t = std::min(16, pow2_floor(std::max(1, kThreads / std::max(GB, 1))));
+  prm->nv = 8;
+  while (prm->nv * prm->tpr < d.chunk_pages) prm->nv *= 2;
   if (prm->scan && prm->kp > 0 && prm->tpr < d.k) return false;
   if (prm->scan && prm->kp == 0 && d.k > kCandCap) return false;
   const int R16 = (d.R + 15) / 16 * 16;
@@ -1638,7 +1720,7 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
   const int ns = prm->n_oa + prm->n_os;
   const bool bf = d.esz == 2;
   const int ntm = (d.R + 15) / 16;
-  prm->wpart = bf && ntm > 0 && kWarps / ntm > 1;
+  prm->wpart = bf && ntm > 0 && kPageWarps / ntm > 1;
   const int rowb = kD * d.esz;
   const int nwords = (d.P + 31) / 32;
   const int pbytes = kPS * rowb;
@@ -1647,24 +1729,22 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
   auto layout = [&](int ngp) {
     GatherLayout& lo = prm->lo;
     Taker take;
-    lo.region = take(std::max(2LL * ngp * pbytes, prm->wpart ? 4LL * kWarps * 16 * kPartStride : 0LL),
+    lo.region = take(std::max(2LL * ngp * pbytes, prm->wpart ? 4LL * kPageWarps * 16 * kPartStride : 0LL),
                      1024);
     lo.kbv = take(2LL * bpad * rowb, 128);
     lo.qa = take(1LL * (bf ? ntm * 16 : d.R) * rowb, 128);
     lo.qs = take(1LL * (bf ? (ns + 15) / 16 * 16 : ns) * rowb, 128);
     lo.ocache = take(4LL * prm->n_os * kD, 16);
     lo.lcache = take(4LL * prm->n_os, 16);
-    lo.sel_own = take(sel ? 4LL * prm->n_oa * d.k : 0, 16);
     lo.sel_all = take(sel ? 4LL * d.R * d.k : 0, 16);
     lo.bitmap = take(nwords * 4, 16);
     lo.wbase = take(nwords * 4, 16);
     lo.lpages = take(prm->max_lp * 4, 16);
     lo.masks = take(4LL * prm->max_lp * d.MW, 16);
     lo.part = take(4LL * d.R * kPartStride, 16);
-    lo.sfx = take(4LL * prm->n_oa * kPartStride, 16);
     lo.misc = take((8 + d.R + GB + ns) * 4, 16);
-    lo.ps = take(kWarps * 16 * 4, 16);
-    lo.mbuf = take(sel ? 2 * kWarps * kCandCap * 8 : 0, 16);
+    lo.ps = take(kWarpsG * 16 * 4, 16);
+    lo.mbuf = take(sel ? (2 * kCandCap + 32) * kWarpsG * 8 : 0, 16);
     lo.total = take.off;
     prm->ngp = ngp;
     return lo.total;
@@ -1685,31 +1765,6 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
 std::mutex g_attr_mu;
 bool g_attr_done[kMaxDevices] = {};
 int g_attr_dyn[kMaxDevices] = {};
-int g_attr_cluster[kMaxDevices] = {};
-
-// Largest cluster size (16, 8, 4) of which at least one cluster of gather
-// CTAs can be resident on the device.
-int probe_cluster() {
-  for (int cl = kMaxCluster; cl >= 4; cl /= 2) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cl, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = static_cast<size_t>(kGatherSmemTarget);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, losa_gather_kernel<LOSA_BF16, 8>, &cfg) == cudaSuccess &&
-        n > 0)
-      return cl;
-    cudaGetLastError();  // clear a refused query
-  }
-  return 4;
-}
 
 template <int DT, int KP>
 cudaError_t set_attrs_one(int optin, int* dyn) {
@@ -1722,10 +1777,6 @@ cudaError_t set_attrs_one(int optin, int* dyn) {
     const int mine = optin - static_cast<int>(fa.sharedSizeBytes);
     e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
     if (e != cudaSuccess) return e;
-    if (i == 1) {
-      e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-    }
     *dyn = std::min(*dyn, mine);
   }
   return cudaSuccess;
@@ -1741,7 +1792,7 @@ cudaError_t set_attrs_dt(int optin, int* dyn) {
   return set_attrs_one<DT, 16>(optin, dyn);
 }
 
-int ensure_attributes(int* max_dyn, int* max_cluster) {
+int ensure_attributes(int* max_dyn) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
@@ -1755,11 +1806,9 @@ int ensure_attributes(int* max_dyn, int* max_cluster) {
     if ((e = set_attrs_dt<LOSA_BF16>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
     if ((e = set_attrs_dt<LOSA_F32>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
     g_attr_dyn[dev] = dyn;
-    g_attr_cluster[dev] = probe_cluster();
     g_attr_done[dev] = true;
   }
   *max_dyn = g_attr_dyn[dev];
-  *max_cluster = g_attr_cluster[dev];
   return LOSA_OK;
 }
 
@@ -1786,10 +1835,9 @@ cudaError_t launch_dt(int kp, const cudaLaunchConfig_t& c1, const ScanParams& sp
 }  // namespace
 
 bool fused_step_fits(const Dims& d, int max_dyn) {
-  // sized for the smallest cluster the device may allow (the most rows per CTA)
   ScanParams sp;
   GatherParams gp;
-  return plan_scan(d, &sp, max_dyn) && plan_gather(d, &gp, max_dyn, 4);
+  return plan_scan(d, &sp, max_dyn) && plan_gather(d, &gp, max_dyn, kGatherCtas);
 }
 
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
@@ -1797,18 +1845,21 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
                       const void* v_blk, float* o_p, float* l_p, float* out, float* out_lse,
                       int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
                       void* workspace, cudaStream_t st) {
-  int max_dyn = 0, max_cluster = kMaxCluster;
-  int rc = ensure_attributes(&max_dyn, &max_cluster);
+  int max_dyn = 0;
+  int rc = ensure_attributes(&max_dyn);
   if (rc != LOSA_OK) return rc;
   ScanParams sp;
   GatherParams gp;
   if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
-  if (!plan_gather(d, &gp, max_dyn, max_cluster)) return LOSA_ERR_UNSUPPORTED;
+  if (!plan_gather(d, &gp, max_dyn, kGatherCtas)) return LOSA_ERR_UNSUPPORTED;
   if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
   char* ws = static_cast<char*>(workspace);
   int* status = reinterpret_cast<int*>(ws + d.off_status);
   int32_t* act = reinterpret_cast<int32_t*>(ws + d.off_act);
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
+  float* part_g = reinterpret_cast<float*>(ws + d.off_gpart);
+  float* sfx_g = reinterpret_cast<float*>(ws + d.off_gsfx);
+  int* cnt = reinterpret_cast<int*>(ws + d.off_cnt);
 
   sp.qc = q_cur;
   sp.qp = q_prev;
@@ -1816,12 +1867,18 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   sp.act_g = act;
   sp.active_idx = active_idx;
   sp.cand = cand;
+  sp.cnt = cnt;
   sp.status = status;
   cudaLaunchConfig_t c1 = {};
+  cudaLaunchAttribute attr1[1];
   c1.gridDim = dim3(sp.scan ? d.nchunk : 1, d.S * d.Hkv, 1);
   c1.blockDim = dim3(kThreads, 1, 1);
   c1.dynamicSmemBytes = static_cast<size_t>(sp.lo.total);
   c1.stream = st;
+  attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr1[0].val.programmaticStreamSerializationAllowed = 1;  // overlaps the previous kernel's tail
+  c1.attrs = attr1;
+  c1.numAttrs = 1;
 
   gp.qc = q_cur;
   gp.K = k_prefix;
@@ -1836,21 +1893,20 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   gp.union_count = union_count;
   gp.act_g = act;
   gp.cand = cand;
+  gp.part_g = part_g;
+  gp.sfx_g = sfx_g;
+  gp.cnt = cnt;
   gp.status = status;
   cudaLaunchConfig_t c2 = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
-  c2.blockDim = dim3(kThreads, 1, 1);
+  c2.blockDim = dim3(kThreadsG, 1, 1);
   c2.dynamicSmemBytes = static_cast<size_t>(gp.lo.total);
   c2.stream = st;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = gp.CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
   c2.attrs = attr;
-  c2.numAttrs = 2;
+  c2.numAttrs = 1;
   // one top-k width per compiled kernel: the selection code of the others is
   // never fetched
   const int kp = sp.scan ? sp.kp : 2;
