@@ -73,13 +73,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest value of x over the ranks (every rank takes part)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, steps_per_rank, ms_max):
+    """Whole-job steps/s: each of `world` replicas ran `steps_per_rank` steps,
+    and the job took as long as its slowest rank."""
+    return world * steps_per_rank / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -292,7 +300,7 @@ def run_losa(args):
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, world)
     ms_per_step = ms_max / steps_timed
-    value = world * steps_timed / (ms_max / 1e3)
+    value = job_throughput(world, steps_timed, ms_max)
     bytes_per_step = sum(bytes_sched) / len(bytes_sched)
     achieved = bytes_per_step / (ms_per_step / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
