@@ -1000,7 +1000,7 @@ struct GatherParams {
 
 // The k best chunk candidates of row r (keys, descending) -> out[0..k).
 // Fast path: lane c holds chunk c's sorted list; the threshold is the k-th
-// largest list head (ranked from shared memory, hb: 32 keys per warp); the
+// largest list head (at least k keys reach it, so the top k all do); the
 // keys at or above it are placed by ballots and rank-sorted.  Fallback:
 // sort-and-merge trees or k rounds of warp argmax.
 template <int KP>
@@ -1036,14 +1036,18 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg
       for (int i = 0; i < KQ; ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
       merge_top<KQ>(x, y);
     }
-    // threshold: the k-th largest list head (every list is sorted, descending)
+    // threshold: the k-th largest list head (every list is sorted,
+    // descending), ranked from shared memory (hb: one key per lane)
     hb[lane] = x[0];
     __syncwarp();
+    const int nl = min(nc, 32);
     int rk = 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const unsigned long long o = hb[i];
-      rk += (o > x[0]) || (o == x[0] && i < lane);
+      if (i < nl) {
+        const unsigned long long o = hb[i];
+        rk += (o > x[0]) || (o == x[0] && i < lane);
+      }
     }
     const unsigned long long tau = hb[__ffs(__ballot_sync(0xffffffffu, rk == k - 1)) - 1];
     unsigned bl[KQ];
@@ -1119,14 +1123,15 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   int32_t* wbase = reinterpret_cast<int32_t*>(smem + lo.wbase);
   int32_t* lpages = reinterpret_cast<int32_t*>(smem + lo.lpages);
   uint32_t* masks = reinterpret_cast<uint32_t*>(smem + lo.masks);
-  float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride]
+  float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride] (fp32 path)
+  float* part_cta = prm.part_g + (static_cast<size_t>(sg) * CL + rank) * R * kPartStride;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
-  int32_t* s_U = misc;
   int32_t* s_nlp = misc + 1;
   int32_t* s_wt = misc + 4;            // stable tokens per 32-token warp slice
-  int32_t* act_tok = misc + 8;         // [R], then act_slot [GB]
+  int32_t* s_wsum = misc + 8;          // union words' popcounts per warp of the union half
+  int32_t* act_tok = misc + 16;        // [R], then act_slot [GB]
   int32_t* act_slot = act_tok + R;
   int32_t* sfx_tok = act_slot + GB;    // [n_oa + n_os]: token row of each suffix row
   float* psw = Ps + warp * 16;
@@ -1150,6 +1155,8 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   if (sel) {
 #pragma unroll 1
     for (int w = tid; w < nwords; w += kThreadsG) bitmap[w] = 0u;
+#pragma unroll 1
+    for (int e = tid; e < prm.max_lp * d.MW; e += kThreadsG) masks[e] = 0u;
   }
   // ---- the block's K and V (suffix half, cp.async group 0; rows >= B zero)
   if (!uhalf) {
@@ -1256,48 +1263,42 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
       }
     } else {
-      if (warp == 0) {  // exclusive prefix of word popcounts
-        const int per = (nwords + 31) / 32;
-        const int w0 = lane * per, w1 = min(nwords, w0 + per);
-        int sum = 0;
+      // exclusive prefix of the words' popcounts: each thread a run of words,
+      // a warp scan, then the warps' totals
+      const int per = (nwords + kThreads - 1) / kThreads;
+      const int w0 = tid * per, w1 = min(nwords, w0 + per);
+      int sum = 0;
 #pragma unroll 1
-        for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
-        int incl = sum;
+      for (int w = w0; w < w1; ++w) sum += __popc(bitmap[w]);
+      int incl = sum;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        int run = incl - sum;
-#pragma unroll 1
-        for (int w = w0; w < w1; ++w) {
-          wbase[w] = run;
-          run += __popc(bitmap[w]);
-        }
-        if (lane == 31) *s_U = incl;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
+      if (lane == 31) s_wsum[warp] = incl;
       bar_sync(1, kThreads);
-      const int U = *s_U;
+      int off = 0, U = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int c = s_wsum[w];
+        off += w < warp ? c : 0;
+        U += c;
+      }
+      int run = off + incl - sum;
+#pragma unroll 1
+      for (int w = w0; w < w1; ++w) {
+        wbase[w] = run;
+        run += __popc(bitmap[w]);
+      }
       const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
       if (tid == 0) {
         *s_nlp = nlp;
         if (rank == 0 && prm.union_count) prm.union_count[sg] = U;
       }
-#pragma unroll 1
-      for (int w = tid; w < nwords; w += kThreads) {
-        uint32_t bits = bitmap[w];
-        int pos = wbase[w];
-#pragma unroll 1
-        while (bits) {
-          const int b = __ffs(bits) - 1;
-          bits &= bits - 1;
-          if (pos % CL == rank && pos / CL < prm.max_lp) lpages[pos / CL] = w * 32 + b;
-          ++pos;
-        }
-      }
-#pragma unroll 1
-      for (int e = tid; e < min(nlp, prm.max_lp) * d.MW; e += kThreads) masks[e] = 0u;
       bar_sync(1, kThreads);
+      // one pass over every (row, page): this CTA's union slots u % CL ==
+      // rank get their page and the row's mask bit
 #pragma unroll 1
       for (int e = tid; e < R * k; e += kThreads) {
         const int p = sel_all[e];
@@ -1306,8 +1307,12 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
         if (u % CL != rank) continue;
         const int r = e / k;
-        if (u / CL < prm.max_lp) atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
-        else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+        if (u / CL < prm.max_lp) {
+          lpages[u / CL] = p;
+          atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
+        } else {
+          atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+        }
       }
     }
     bar_sync(1, kThreads);
@@ -1481,7 +1486,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
     }
     tile_finish(t);
     if (wpm == 1) {  // one warp per m16 tile: its state is the CTA's partial
-      if (aw) tile_store(t, part + mt * 16 * kPartStride, min(16, R - mt * 16));
+      if (aw) tile_store(t, part_cta + mt * 16 * kPartStride, min(16, R - mt * 16));
     } else {
       float* wp = reinterpret_cast<float*>(region);
       __syncthreads();  // every page consumed: the region takes the warps' partials
@@ -1505,7 +1510,11 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kPageWarps; ++w) M = fmaxf(M, mw[w]);
-        if (M == -INFINITY) continue;  // none of this CTA's pages serve row r
+        float* dst = part_cta + r * kPartStride;
+        if (M == -INFINITY) {  // none of this CTA's pages serve row r
+          if (lane == 0) dst[0] = -INFINITY;
+          continue;
+        }
         float l = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -1518,7 +1527,6 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
           acc.z += wgt * aw4[w].z;
           acc.w += wgt * aw4[w].w;
         }
-        float* dst = part + r * kPartStride;
         if (lane == 0) {
           dst[0] = M;
           dst[1] = l;
@@ -1564,16 +1572,15 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   }
   __syncthreads();
 
-  // ---- publish this CTA's row partials; the group's last CTA to finish
-  // combines every row
-  {
-    float4* dstp = reinterpret_cast<float4*>(
-        prm.part_g + (static_cast<size_t>(sg) * CL + rank) * R * kPartStride);
+  // ---- publish this CTA's row partials (bf16: already in the workspace);
+  // the group's last CTA to finish combines every row
+  if (DT != LOSA_BF16) {
+    float4* dstp = reinterpret_cast<float4*>(part_cta);
     const float4* srcp = reinterpret_cast<const float4*>(part);
 #pragma unroll 1
     for (int e = tid; e < R * kPartStride / 4; e += kThreadsG) dstp[e] = srcp[e];
+    __syncthreads();
   }
-  __syncthreads();
   int* s_last = misc + 2;
   if (tid == 0) {
     __threadfence();  // this CTA's partials and suffixes before its arrival
@@ -1589,6 +1596,9 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 #pragma unroll 1
   for (int r = warp; r < R; r += kWarpsG) {
     const float* base = prm.part_g + (static_cast<size_t>(sg) * CL * R + r) * kPartStride;
+    const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
+    const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4) + lane);  // the row's suffix
+    const float Ls = __ldcg(sx);
     float M = -INFINITY, lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -1637,10 +1647,8 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
     const size_t grow = grow0 + (r / A) * B + act_tok[r];
     *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
     if (lane == 0) prm.l_p[grow] = Lp;
-    const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
-    const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4) + lane);
     float wa, wb, L;
-    lse_weights(Lp, __ldcg(sx), wa, wb, L);
+    lse_weights(Lp, Ls, wa, wb, L);
     *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
         make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
                     wa * op.w + wb * os.w);
@@ -1742,7 +1750,7 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
     lo.lpages = take(prm->max_lp * 4, 16);
     lo.masks = take(4LL * prm->max_lp * d.MW, 16);
     lo.part = take(4LL * d.R * kPartStride, 16);
-    lo.misc = take((8 + d.R + GB + ns) * 4, 16);
+    lo.misc = take((16 + d.R + GB + ns) * 4, 16);
     lo.ps = take(kWarpsG * 16 * 4, 16);
     lo.mbuf = take(sel ? (2 * kCandCap + 32) * kWarpsG * 8 : 0, 16);
     lo.total = take.off;
