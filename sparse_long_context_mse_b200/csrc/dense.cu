@@ -97,14 +97,14 @@ __device__ __forceinline__ void suffix_row(float4 q, const float* Kb, const floa
   L = (m + __log2f(l)) * kLn2;
 }
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     dense_finish_kernel(const void* __restrict__ Q, const void* __restrict__ Kb,
                         const void* __restrict__ Vb, const float* __restrict__ part,
                         float* __restrict__ o_p, float* __restrict__ l_p, float* __restrict__ out,
                         float* __restrict__ out_lse, Dims d) {
   __shared__ __align__(16) float Ksb[kMaxB * kD];
   __shared__ __align__(16) float Vsb[kMaxB * kD];
-  __shared__ float Ps[4][kPS];
+  __shared__ float Ps[8][kPS];
   const int sh = blockIdx.x;  // s * Hq + h
   const int s = sh / d.Hq, h = sh % d.Hq, g = h / d.G;
   const int sg = s * d.Hkv + g;
@@ -123,20 +123,26 @@ __global__ void __launch_bounds__(128)
     *reinterpret_cast<float4*>(Vsb + j * kD + c) = vv;
   }
   __syncthreads();
-  for (int t = warp; t < d.B; t += 4) {
+  // one warp per row: rows blockIdx.y * 8 + warp of head h
+  for (int t = blockIdx.y * 8 + warp; t < min(d.B, blockIdx.y * 8 + 8); t += 8) {
     const size_t row = static_cast<size_t>(sh) * d.B + t;
     const int r = (h - g * d.G) * d.B + t;
-    // merge the prefix partials (base-2 units) of every split
+    // merge the prefix partials (base-2 units) of every split: the splits'
+    // maxima over the lanes, then the weighted sums with eight splits' loads
+    // in flight at a time
+    const float* p0 = part + (static_cast<size_t>(sg) * d.nsplit * rows + r) * kPartStride;
+    const size_t pstride = static_cast<size_t>(rows) * kPartStride;
     float M = -INFINITY;
-    for (int sp = 0; sp < d.nsplit; ++sp)
-      M = fmaxf(M, part[((static_cast<size_t>(sg) * d.nsplit + sp) * rows + r) * kPartStride]);
+    for (int sp = lane; sp < d.nsplit; sp += 32) M = fmaxf(M, __ldcg(p0 + sp * pstride));
+    M = warp_max(M);
     float lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int sp = 0; sp < d.nsplit; ++sp) {
-      const float* src = part + ((static_cast<size_t>(sg) * d.nsplit + sp) * rows + r) * kPartStride;
-      const float w = exp2f(src[0] - M);
-      lsum += w * src[1];
-      const float4 a = *reinterpret_cast<const float4*>(src + 4 + 4 * lane);
+      const float* src = p0 + sp * pstride;
+      const float w = exp2f(__ldcg(src) - M);
+      lsum += w * __ldcg(src + 1);
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(src + 4) + lane);
       acc.x += w * a.x;
       acc.y += w * a.y;
       acc.z += w * a.z;
@@ -405,8 +411,8 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);
   }
-  dense_finish_kernel<<<d.S * d.Hq, 128, 0, st>>>(q, k_blk, v_blk, part, o_p, l_p, out, out_lse,
-                                                  d);
+  dense_finish_kernel<<<dim3(d.S * d.Hq, (d.B + 7) / 8), 256, 0, st>>>(q, k_blk, v_blk, part, o_p,
+                                                                        l_p, out, out_lse, d);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
