@@ -333,6 +333,8 @@ def run_losa(args):
     }
     if not args.no_extras:
         res.update(extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched))
+        res["naive_quest_all_B"] = naive_quest(stream, dev, world,
+                                               statistics.mean(union_per_kv), ms_per_step)
         res["block"]["losa_vs_dense_step_speedup"] = round(
             res["dense_step_us"] / res["us_per_layer_step"], 3)
     if rank == 0:
@@ -341,6 +343,54 @@ def run_losa(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def naive_quest(stream, dev, world, losa_union, losa_ms):
+    """The same kernels with every block token active (|A| = B): QUEST page
+    selection for all B queries, the baseline LoSA's locality pruning is
+    measured against.  Reports the union (KV pages loaded per KV head), its
+    inflation over LoSA's, and the step time."""
+    import dataclasses
+    import torch
+    from sparse_long_context_mse_b200 import api, synth
+    cfg = synth.config(CONFIG_ID)
+    cfg = dataclasses.replace(cfg, n_active=cfg.block_size)
+    n_layers = 2  # 2 x ~280 MB of prefix K/V + metadata: larger than L2
+    sh, layers, _ = build_layers(cfg, n_layers, dev)
+    ws = api.alloc_workspace(sh, api.LOSA_WS_STEP, dev)
+    T = cfg.steps
+    sched = [(li, t) for t in range(1, T) for li in range(n_layers)]
+    unions = []
+    with torch.cuda.stream(stream):
+        for li, t in sched:
+            L = layers[li]
+            api.step(sh, L.q[t], L.q[t - 1], L.K, L.V, L.meta, L.kb[t], L.vb[t], L.o_p, L.l_p,
+                     L.out, L.lse, ws, union_count=L.ucount, stream=stream)
+            unions.append(L.ucount.sum().item() / (sh.num_seqs * sh.n_kv_heads))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for li, t in sched:
+            L = layers[li]
+            api.step(sh, L.q[t], L.q[t - 1], L.K, L.V, L.meta, L.kb[t], L.vb[t], L.o_p, L.l_p,
+                     L.out, L.lse, ws, stream=stream)
+    reps = 20
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / (reps * len(sched))
+    del g
+    u = statistics.mean(unions)
+    return {"n_active": cfg.n_active, "union_pages_per_kv_head": round(u, 2),
+            "density": round(u / sh.n_pages, 5), "us_per_step": round(ms * 1e3, 3),
+            "union_vs_losa": round(u / losa_union, 3), "step_time_vs_losa": round(ms / losa_ms, 3)}
 
 
 def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):

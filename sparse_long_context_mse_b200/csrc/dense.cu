@@ -7,8 +7,16 @@
 // range for all G*B query rows of the group and writes an unnormalised
 // online-softmax partial per row; the finish kernel merges the partials, adds
 // the dense suffix over the block's own keys and writes cache and output.
+// bf16 runs on the 5th-generation tensor cores (tcgen05, TMEM), fp32 on
+// CUDA cores.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "losa_common.cuh"
 #include "ptx.cuh"
+#include "umma.cuh"
 
 namespace losa {
 namespace {
@@ -166,206 +174,285 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// bf16: tensor cores.  CTA = (split, group); warp w owns query rows
-// [16w, 16w + 16) of the group's G*B rows.  Keys stream through a 3-stage
-// cp.async ring of 64-key K/V tiles (16-byte chunks XOR-swizzled by row, so
-// ldmatrix is conflict-free).  S = Q K^T and O += P V with mma.sync
-// m16n8k16 (bf16 operands, fp32 accumulation); P is split into a bf16 high
-// part and a bf16 remainder so the weights keep ~16 bits.  Online softmax in
-// base 2, one partial (m, l, acc) per row and split, as the fp32 kernel.
+// bf16: 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+// CTA = (split, group), 256 threads: two threads per query row of the group
+// (TMEM lane = row; rows >= G*B are padding), each with half of every tile's
+// keys and half of the output channels.  One thread drives the tensor core
+// and the TMA: 64-key K and V tiles arrive by 2-D tiled TMA loads in the
+// 128-byte-swizzled layout the matrix descriptors describe, K through a
+// 4-stage ring (a stage is free once the tile's scores are done), V through
+// a 3-stage ring (free once the tile's P V is done).  Per tile: S = Q K^T
+// (M=128, N=64, K=128) into one of two TMEM buffers, issued one tile ahead so
+// the tensor core runs while the threads do the softmax; every thread reads
+// its half row of S; the online softmax runs in base 2 (the halves exchange
+// row maxima through shared memory) against a reference max that moves only
+// when the row max grows by more than 2^8 (O and l are then rescaled in
+// TMEM); P goes to one of two shared-memory buffers as a bf16 high part and
+// a bf16 remainder, so the weights keep ~16 bits; then O += P_hi V + P_lo V
+// (M=128, N=128, K=64, V the MN-major operand).  A tile waits only for the
+// P V of two tiles back.  Every wait is bounded; a wait that gives up
+// records LOSA_ERR_DEVICE_TIMEOUT.
 // ---------------------------------------------------------------------------
-constexpr int kDKeys = 64;
-constexpr size_t kMaxDenseSmem = 128 * 256 + 3 * 2 * 64 * 128 * 2;
-constexpr int kDStages = 3;
-constexpr int kDTileBytes = kDKeys * kD * 2;
+constexpr int kUKeys = 64;                          // keys per tile
+constexpr int kUKst = 4;                            // K ring stages
+constexpr int kUVst = 3;                            // V ring stages
+constexpr int kUTile = kUKeys * kD * 2;             // 16 KB: one K (or V) tile
+constexpr int kUQ = 128 * kD * 2;                   // 32 KB: the query tile
+constexpr int kUP = 128 * kUKeys * 2;               // 16 KB: one P part
+constexpr int kUBars = 1 + 2 + 2 + kUKst + kUVst;   // Q, S[2], O[2], K[4], V[3]
+constexpr int kUSmem = 1024 + kUQ + (kUKst + kUVst) * kUTile + 4 * kUP + 1024 + kUBars * 8 + 16;
+constexpr uint32_t kUCols = 256;                    // TMEM: S [0, 128) (two tiles), O [128, 256)
 
-__global__ void __launch_bounds__(256) dense_mma_kernel(const __nv_bfloat16* __restrict__ Q,
-                                                        const __nv_bfloat16* __restrict__ K,
-                                                        const __nv_bfloat16* __restrict__ V,
-                                                        float* __restrict__ part, Dims d) {
-  extern __shared__ __align__(1024) char dsm[];
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(su32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(256, 1)
+    dense_umma_kernel(const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap, float* __restrict__ part,
+                      int* __restrict__ status, Dims d) {
+  extern __shared__ char dsm_raw[];
+  // 1024-byte alignment for the swizzled tiles
+  char* dsm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  char* qs = dsm;                                     // [128 rows], 2 atoms of 16 KB
+  char* kring = qs + kUQ;                             // kUKst K tiles (2 atoms of 8 KB)
+  char* vring = kring + kUKst * kUTile;               // kUVst V tiles
+  char* pbuf = vring + kUVst * kUTile;                // [2][hi, lo] P parts
+  float* xmax = reinterpret_cast<float*>(pbuf + 4 * kUP);     // [2][128]: the halves' row maxima
+  uint64_t* bars = reinterpret_cast<uint64_t*>(xmax + 256);
+  uint64_t* bQ = bars;
+  uint64_t* bS = bars + 1;     // [2] S buffer ready
+  uint64_t* bO = bars + 3;     // [2] O += P V of an even / odd tile done
+  uint64_t* bK = bars + 5;     // [kUKst] K tile landed
+  uint64_t* bV = bars + 5 + kUKst;  // [kUVst] V tile landed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + kUBars);
+  int* s_fail = reinterpret_cast<int*>(tslot + 1);
   const int sg = blockIdx.y, split = blockIdx.x;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int rows = d.G * d.B;
-  const int M16 = (rows + 15) / 16 * 16;
-  const int nthr = blockDim.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g4 = lane >> 2, t4 = lane & 3;
-  char* qs = dsm;                 // [M16][256 B]
-  char* kvs = dsm + M16 * 256;    // stages x (K tile, V tile)
+  // warp w reads TMEM lanes 32 (w % 4) ..: thread (w, lane) owns query row
+  // 32 (w % 4) + lane, the w / 4 half of each S tile's keys and of O
+  const int row = (warp & 3) * 32 + lane, half = warp >> 2;
+  const bool busy = (warp & 3) * 32 < rows;  // (warp-uniform) some row of this warp is real
   const int key0 = split * d.split_pages * kPS;
   const int key1 = min(d.L, key0 + d.split_pages * kPS);
-  const int ntile = (key1 - key0 + kDKeys - 1) / kDKeys;
-  const size_t kvbase = static_cast<size_t>(sg) * d.L * kD;
-  const size_t qbase = (static_cast<size_t>(s) * d.Hq + g * d.G) * d.B * kD;
+  const int n = (key1 - key0 + kUKeys - 1) / kUKeys;
+  const int kv_row0 = sg * d.L + key0;                 // first key of the split, as a tensor row
+  const int q_row0 = (s * d.Hq + g * d.G) * d.B;       // the group's first query row
 
-#pragma unroll 1
-  for (int e = tid; e < M16 * 16; e += nthr) {
-    const int r = e >> 4, c = e & 15;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < rows) v = *reinterpret_cast<const uint4*>(Q + qbase + static_cast<size_t>(r) * kD + c * 8);
-    *reinterpret_cast<uint4*>(qs + r * 256 + ((c ^ (r & 7)) << 4)) = v;
-  }
-  auto load_tile = [&](int t, int stage) {
-    char* kt = kvs + stage * 2 * kDTileBytes;
-    char* vt = kt + kDTileBytes;
-    const int kb = key0 + t * kDKeys;
-#pragma unroll 1
-    for (int e = tid; e < kDKeys * 16; e += nthr) {
-      const int j = e >> 4, c = e & 15;
-      const int key = kb + j;
-      const bool ok = key < key1;
-      const size_t off = kvbase + static_cast<size_t>(ok ? key : key0) * kD + c * 8;
-      const uint32_t o = j * 256 + ((c ^ (j & 7)) << 4);
-      cp_async16(su32(kt + o), K + off, ok ? 16u : 0u);
-      cp_async16(su32(vt + o), V + off, ok ? 16u : 0u);
-    }
+  auto load_k = [&](int t) {  // one thread
+    uint64_t* bar = &bK[t % kUKst];
+    char* dst = kring + (t % kUKst) * kUTile;
+    mbar_expect_tx(bar, kUTile);
+    tma_load_2d(dst, &kmap, 0, kv_row0 + t * kUKeys, bar);
+    tma_load_2d(dst + kUTile / 2, &kmap, 64, kv_row0 + t * kUKeys, bar);
   };
-#pragma unroll 1
-  for (int st = 0; st < kDStages - 1; ++st) {
-    if (st < ntile) load_tile(st, st);
-    cp_async_commit();
+  auto load_v = [&](int t) {
+    uint64_t* bar = &bV[t % kUVst];
+    char* dst = vring + (t % kUVst) * kUTile;
+    mbar_expect_tx(bar, kUTile);
+    tma_load_2d(dst, &vmap, 0, kv_row0 + t * kUKeys, bar);
+    tma_load_2d(dst + kUTile / 2, &vmap, 64, kv_row0 + t * kUKeys, bar);
+  };
+  constexpr uint32_t idesc_s = umma_idesc_bf16(128, kUKeys, 0);
+  constexpr uint32_t idesc_o = umma_idesc_bf16(128, kD, 1);
+  uint32_t tbase = 0;
+  auto issue_s = [&](int t) {  // S = Q K^T of tile t into S buffer t & 1 (one thread)
+    const char* kt = kring + (t % kUKst) * kUTile;
+    tc_fence_after();
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t ko = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+      const uint32_t kk = (ks >> 2) * (kUKeys * 128) + (ks & 3) * 32;
+      umma_bf16(tbase + (t & 1) * kUKeys, umma_desc(su32(qs) + ko, 16, 1024),
+                umma_desc(su32(kt) + kk, 16, 1024), idesc_s, ks > 0);
+    }
+    umma_commit(&bS[t & 1]);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kUBars; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+    *s_fail = 0;
+    mbar_expect_tx(bQ, kUQ);
+    tma_load_2d(qs, &qmap, 0, q_row0, bQ);
+    tma_load_2d(qs + kUQ / 2, &qmap, 64, q_row0, bQ);
+    for (int t = 0; t < min(n, kUKst); ++t) load_k(t);
+    for (int t = 0; t < min(n, kUVst); ++t) load_v(t);
   }
+  if (warp == 0) tmem_alloc(tslot, kUCols);
+  tc_fence_before();
   __syncthreads();
-  uint32_t qa[8][4];
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    const int mi = lane >> 3, row = warp * 16 + (mi & 1) * 8 + (lane & 7);
-    const int ch = ks * 2 + (mi >> 1);
-    ldsm_x4(su32(qs + row * 256 + ((ch ^ (row & 7)) << 4)), qa[ks][0], qa[ks][1], qa[ks][2],
-            qa[ks][3]);
-  }
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float o[16][4];
-#pragma unroll
-  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  tc_fence_after();
+  tbase = *tslot;
+  const uint32_t tO = tbase + 128;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
   const float sl2 = d.scale_log2;
+  float mref = -INFINITY, lrow = 0.f;  // lrow: this half's share of the row sum
+  bool ok = true;
+  if (tid == 0) {
+    if (!mbar_wait(bQ, 0) || !mbar_wait(&bK[0], 0)) ok = false;
+    issue_s(0);
+  }
 
 #pragma unroll 1
-  for (int t = 0; t < ntile; ++t) {
-    cp_async_wait<kDStages - 2>();
+  for (int t = 0; t < n; ++t) {
+    if (tid == 0 && t + 1 < n) {  // the next tile's scores run during this tile's softmax
+      if (!mbar_wait(&bK[(t + 1) % kUKst], ((t + 1) / kUKst) & 1)) ok = false;
+      issue_s(t + 1);
+    }
+    __syncwarp();
+    if (!mbar_wait(&bS[t & 1], (t >> 1) & 1)) ok = false;
+    if (tid == 0 && t + kUKst < n) load_k(t + kUKst);  // tile t's K stage is free again
+    // P V of two tiles back has finished: its P buffers and V stage are free
+    if (t >= 2 && !mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1)) ok = false;
+    if (tid == 0 && t >= 2 && t + 1 < n) load_v(t + 1);
+    tc_fence_after();
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
+
+    // this thread's 32 scores of the tile
+    const int kb = key0 + t * kUKeys + half * 32;
+    float sv[32];
+    float mx = -INFINITY;
+    if (busy) {
+      tmem_ld32(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
+      if (kb + 32 <= key1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] *= sl2;
+          mx = fmaxf(mx, sv[i]);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = kb + i < key1 ? sv[i] * sl2 : -INFINITY;
+          mx = fmaxf(mx, sv[i]);
+        }
+      }
+      xmax[half * 128 + row] = mx;
+    }
+    __syncthreads();  // both halves' maxima
+    char* phi = pbuf + (t & 1) * 2 * kUP;
+    char* plo = phi + kUP;
+    if (busy) {
+      mx = fmaxf(xmax[row], xmax[128 + row]);
+      const bool grow = mx > mref + 8.f;  // the same decision in both halves of the row
+      if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
+        const float nref = grow ? mx : mref;
+        const float alpha = grow ? exp2f(mref - nref) : 1.f;  // 0 while nothing is accumulated
+        lrow *= alpha;
+        if (t > 0) {
+          // O holds every P V up to tile t - 1
+          if (!mbar_wait(&bO[(t - 1) & 1], ((t - 1) >> 1) & 1)) ok = false;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+            float v[32];
+            tmem_ld32(tO + lane_off + c0, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st32(tO + lane_off + c0, v);
+          }
+        }
+        mref = nref;
+      }
+      // P = 2^(s - mref) <= 2^8: high part and remainder, [128 rows][64 keys]
+      // K-major, swizzled
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float p0 = exp2f(sv[c8 * 8 + 2 * u] - mref);
+          const float p1 = exp2f(sv[c8 * 8 + 2 * u + 1] - mref);
+          lrow += p0 + p1;
+          hi[u] = pack_bf16x2(p0, p1);
+          const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xffff0000u);
+          lo[u] = pack_bf16x2(p0 - h0, p1 - h1);
+        }
+        const uint32_t o = sw128_off(row, half * 32 + c8 * 8, 128);
+        *reinterpret_cast<uint4*>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
     __syncthreads();
-    {
-      const int tn = t + kDStages - 1;
-      if (tn < ntile) load_tile(tn, tn % kDStages);
-      cp_async_commit();
-    }
-    const char* kt = kvs + (t % kDStages) * 2 * kDTileBytes;
-    const char* vt = kt + kDTileBytes;
-    float sc[8][4];
+    if (tid == 0) {
+      if (!mbar_wait(&bV[t % kUVst], (t / kUVst) & 1)) ok = false;
+      tc_fence_after();
+      const char* vt = vring + (t % kUVst) * kUTile;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t pa = su32(h ? plo : phi);
 #pragma unroll
-      for (int ks = 0; ks < 8; ks += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int key = nt * 8 + (lane & 7), ch = ks * 2 + (lane >> 3);
-        ldsm_x4(su32(kt + key * 256 + ((ch ^ (key & 7)) << 4)), b0, b1, b2, b3);
-        mma_bf16(sc[nt], qa[ks], b0, b1);
-        mma_bf16(sc[nt], qa[ks + 1], b2, b3);
+        for (int ks = 0; ks < kUKeys / 16; ++ks)
+          umma_bf16(tO, umma_desc(pa + ks * 32, 16, 1024),
+                    umma_desc(su32(vt) + ks * 16 * 128, kUKeys * 128, 1024), idesc_o,
+                    (t > 0 || h > 0 || ks > 0) ? 1u : 0u);
       }
-    }
-    const int kb = key0 + t * kDKeys;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const bool ok = kb + nt * 8 + 2 * t4 + c < key1;
-        sc[nt][c] = ok ? sc[nt][c] * sl2 : -INFINITY;
-        sc[nt][2 + c] = ok ? sc[nt][2 + c] * sl2 : -INFINITY;
-        mx0 = fmaxf(mx0, sc[nt][c]);
-        mx1 = fmaxf(mx1, sc[nt][2 + c]);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      sc[nt][0] = exp2f(sc[nt][0] - mn0);
-      sc[nt][1] = exp2f(sc[nt][1] - mn0);
-      sc[nt][2] = exp2f(sc[nt][2] - mn1);
-      sc[nt][3] = exp2f(sc[nt][3] - mn1);
-      ps0 += sc[nt][0] + sc[nt][1];
-      ps1 += sc[nt][2] + sc[nt][3];
-    }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      o[n][0] *= al0;
-      o[n][1] *= al0;
-      o[n][2] *= al1;
-      o[n][3] *= al1;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      // P as the A operand: high bf16 part and the bf16 remainder
-      uint32_t ah[4], al[4];
-      const float* p0 = sc[2 * kk];
-      const float* p1 = sc[2 * kk + 1];
-      const float pv[8] = {p0[0], p0[1], p0[2], p0[3], p1[0], p1[1], p1[2], p1[3]};
-      float rem[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float hi = __bfloat162float(__float2bfloat16_rn(pv[i]));
-        rem[i] = pv[i] - hi;
-      }
-      ah[0] = pack_bf16x2(pv[0], pv[1]);
-      ah[1] = pack_bf16x2(pv[2], pv[3]);
-      ah[2] = pack_bf16x2(pv[4], pv[5]);
-      ah[3] = pack_bf16x2(pv[6], pv[7]);
-      al[0] = pack_bf16x2(rem[0], rem[1]);
-      al[1] = pack_bf16x2(rem[2], rem[3]);
-      al[2] = pack_bf16x2(rem[4], rem[5]);
-      al[3] = pack_bf16x2(rem[6], rem[7]);
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        uint32_t b0, b1, b2, b3;
-        const int key = 16 * kk + ((lane >> 3) & 1) * 8 + (lane & 7);
-        const int ch = 2 * np + (lane >> 4);
-        ldsm_x4_trans(su32(vt + key * 256 + ((ch ^ (key & 7)) << 4)), b0, b1, b2, b3);
-        mma_bf16(o[2 * np], ah, b0, b1);
-        mma_bf16(o[2 * np + 1], ah, b2, b3);
-        mma_bf16(o[2 * np], al, b0, b1);
-        mma_bf16(o[2 * np + 1], al, b2, b3);
-      }
+      umma_commit(&bO[t & 1]);
     }
   }
-  cp_async_wait<0>();
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const int r0 = warp * 16 + g4, r1 = r0 + 8;
-  const size_t pb = (static_cast<size_t>(sg) * d.nsplit + split) * rows;
-  if (r0 < rows) {
-    float* dst = part + (pb + r0) * kPartStride;
-    if (t4 == 0) {
-      dst[0] = m0;
-      dst[1] = l0;
-    }
+  __syncwarp();
+  if (!mbar_wait(&bO[(n - 1) & 1], ((n - 1) >> 1) & 1)) ok = false;
+  tc_fence_after();
+  if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
+  if (half == 1) xmax[row] = lrow;  // the second half's row sum
+  __syncthreads();
+  if (!*s_fail && busy) {
+    float* dst = part + ((static_cast<size_t>(sg) * d.nsplit + split) * rows + row) * kPartStride;
+#pragma unroll 1
+    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+      float v[32];
+      tmem_ld32(tO + lane_off + c0, v);
+      if (row < rows) {
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
-      *reinterpret_cast<float2*>(dst + 4 + n * 8 + 2 * t4) = make_float2(o[n][0], o[n][1]);
-  }
-  if (r1 < rows) {
-    float* dst = part + (pb + r1) * kPartStride;
-    if (t4 == 0) {
-      dst[0] = m1;
-      dst[1] = l1;
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + 4 + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
     }
-#pragma unroll
-    for (int n = 0; n < 16; ++n)
-      *reinterpret_cast<float2*>(dst + 4 + n * 8 + 2 * t4) = make_float2(o[n][2], o[n][3]);
+    if (row < rows && half == 0) {
+      dst[0] = mref;
+      dst[1] = lrow + xmax[row];
+    }
   }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *s_fail) atomicCAS(status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+  if (warp == 0) tmem_dealloc(tbase, kUCols);
+}
+
+// 2-D tensor map over a [rows][128] bf16 tensor for 128-byte-swizzled boxes
+// of 64 channels x box_rows rows.
+int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsigned box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return LOSA_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), nrows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  const cuuint32_t box[2] = {64u, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LOSA_OK : LOSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -392,21 +479,24 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* part = reinterpret_cast<float*>(static_cast<char*>(workspace) + d.off_part);
   if (d.dtype == LOSA_BF16) {
-    const int M16 = (d.G * d.B + 15) / 16 * 16;
-    const size_t smem = static_cast<size_t>(M16) * 256 + kDStages * 2 * kDTileBytes;
+    if (d.G * d.B > 128) return LOSA_ERR_UNSUPPORTED;
     static bool attr_done[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-      cudaError_t e0 = cudaFuncSetAttribute(dense_mma_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(kMaxDenseSmem));
+      cudaError_t e0 = cudaFuncSetAttribute(dense_umma_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
       if (e0 != cudaSuccess) return record_cuda_error(e0);
       attr_done[dev] = true;
     }
-    dense_mma_kernel<<<dim3(d.nsplit, d.S * d.Hkv), 32 * (M16 / 16), smem, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k_prefix),
-        static_cast<const __nv_bfloat16*>(v_prefix), part, d);
+    int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.off_status);
+    CUtensorMap qmap, kmap, vmap;
+    if (make_tmap(&qmap, q, rows, 128) != LOSA_OK ||
+        make_tmap(&kmap, k_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK ||
+        make_tmap(&vmap, v_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK)
+      return record_cuda_error(cudaErrorInvalidValue);
+    dense_umma_kernel<<<dim3(d.nsplit, d.S * d.Hkv), 256, kUSmem, st>>>(qmap, kmap, vmap, part,
+                                                                       status, d);
   } else {
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);

@@ -534,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   int32_t* s_fail = misc;
   float* s_mse = reinterpret_cast<float*>(misc + 4);
   int32_t* act_tok = misc + 4 + kMaxRowsPerGroup;
+  int32_t* act_row = act_tok + kMaxRowsPerGroup;
 
   const int p0 = chunk * d.chunk_pages;
   const int npages = prm.scan ? max(0, min(d.P, p0 + d.chunk_pages) - p0) : 0;
@@ -571,31 +572,34 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     return;
   }
 
-  // ---- locality score: mse_t lanes per row, each summing its channels in
-  // order (fp32, one rounding per operation), then a shuffle tree
+  // ---- locality score: mse_t lanes per row, each keeping four running
+  // sums over its channels (fp32, one rounding per operation), then a
+  // shuffle tree
   {
     const int T = prm.mse_t;
     const int row = tid / T, part = tid % T;
     float acc = 0.f;
-    if (row < GB) {
+    if (row < GB) {  // four running sums (one per 32-bit word of a chunk), added at the end
       constexpr int cpr = rowb / 16;
       const uint4* x = reinterpret_cast<const uint4*>(qcs + row * rowb);
       const uint4* y = reinterpret_cast<const uint4*>(qps + row * rowb);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 4
       for (int c = part; c < cpr; c += T) {
         const uint4 a = x[c], b = y[c];
         if (DT == LOSA_BF16) {
-          acc = sqd_bf16x2(a.x, b.x, acc);
-          acc = sqd_bf16x2(a.y, b.y, acc);
-          acc = sqd_bf16x2(a.z, b.z, acc);
-          acc = sqd_bf16x2(a.w, b.w, acc);
+          a0 = sqd_bf16x2(a.x, b.x, a0);
+          a1 = sqd_bf16x2(a.y, b.y, a1);
+          a2 = sqd_bf16x2(a.z, b.z, a2);
+          a3 = sqd_bf16x2(a.w, b.w, a3);
         } else {
-          acc = sqd_f32(a.x, b.x, acc);
-          acc = sqd_f32(a.y, b.y, acc);
-          acc = sqd_f32(a.z, b.z, acc);
-          acc = sqd_f32(a.w, b.w, acc);
+          a0 = sqd_f32(a.x, b.x, a0);
+          a1 = sqd_f32(a.y, b.y, a1);
+          a2 = sqd_f32(a.z, b.z, a2);
+          a3 = sqd_f32(a.w, b.w, a3);
         }
       }
+      acc = (a0 + a1) + (a2 + a3);
     }
 #pragma unroll 1
     for (int o = 1; o < T; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -619,7 +623,10 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
       const bool act = lane < B && rk < A;
       const unsigned bal = __ballot_sync(0xffffffffu, act);
       const int slot = __popc(bal & ((1u << lane) - 1u));
-      if (act) act_tok[h * A + slot] = lane;
+      if (act) {
+        act_tok[h * A + slot] = lane;
+        act_row[h * A + slot] = h * B + lane;  // the row's query in the staged group
+      }
       if (chunk == 0) {
         if (lane < B) act_g[R + h * B + lane] = act ? slot : -1;
         if (act) {
@@ -642,8 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
       const int r = e / 32, c = e % 32;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (r < R) {
-        const int row = (r / A) * B + act_tok[r];
-        const uint4 w4 = *reinterpret_cast<const uint4*>(qcs + row * rowb + (c & 15) * 16);
+        const uint4 w4 = *reinterpret_cast<const uint4*>(qcs + act_row[r] * rowb + (c & 15) * 16);
         const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t o[4];
 #pragma unroll
@@ -667,9 +673,8 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
 #pragma unroll 1
     for (int e = tid; e < R * kD; e += kThreads) {
       const int r = e / kD, c = e % kD;
-      const int row = (r / A) * B + act_tok[r];
       reinterpret_cast<uint32_t*>(qrows)[r * kD + c] =
-          reinterpret_cast<const uint32_t*>(qcs + row * rowb)[c];
+          reinterpret_cast<const uint32_t*>(qcs + act_row[r] * rowb)[c];
     }
   }
   __syncthreads();  // the previous queries' staging area becomes the score area
@@ -1705,7 +1710,7 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
     // the previous queries, then (after the locality pass) the scores
     lo.qps = take(std::max(qbytes, prm->scan ? 4LL * d.R * prm->sc_stride : 0LL), 128);
     lo.qrows = take(prm->scan ? (d.esz == 2 ? R16 : d.R) * 512LL : 0, 128);
-    lo.misc = take((4 + kMaxRowsPerGroup + d.R) * 4, 16);
+    lo.misc = take((4 + 3 * kMaxRowsPerGroup) * 4, 16);
     lo.fbuf = take(prm->scan && prm->kp > 0 ? 8LL * (kThreads / prm->tpr) * kCandCap : 0, 16);
     lo.cbuf = take(prm->scan && prm->kp == 0 ? 2 * kWarps * kCandCap * 8 : 0, 16);
     lo.mbar = take((kMaxStages + 1) * 8, 8);
