@@ -199,7 +199,7 @@ constexpr int kUVst = 3;                            // V ring stages
 constexpr int kUTile = kUKeys * kD * 2;             // 16 KB: one K (or V) tile
 constexpr int kUQ = 128 * kD * 2;                   // 32 KB: the query tile
 constexpr int kUP = 128 * kUKeys * 2;               // 16 KB: one P part
-constexpr int kUBars = 1 + 2 + 2 + kUKst + kUVst;   // Q, S[2], O[2], K[4], V[3]
+constexpr int kUBars = 1 + 2 + 2 + kUKst + kUVst + 2;  // Q, S[2], O[2], K[4], V[3], P[2]
 constexpr int kUSmem = 1024 + kUQ + (kUKst + kUVst) * kUTile + 4 * kUP + 1024 + kUBars * 8 + 16;
 constexpr uint32_t kUCols = 256;                    // TMEM: S [0, 128) (two tiles), O [128, 256)
 
@@ -212,7 +212,8 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-__global__ void __launch_bounds__(256, 1)
+template <int MR>
+__global__ void __launch_bounds__(288, 1)
     dense_umma_kernel(const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, float* __restrict__ part,
@@ -220,7 +221,8 @@ __global__ void __launch_bounds__(256, 1)
   extern __shared__ char dsm_raw[];
   // 1024-byte alignment for the swizzled tiles
   char* dsm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  char* qs = dsm;                                     // [128 rows], 2 atoms of 16 KB
+  // MR = MMA rows (64 or 128): the group's query rows, zero-padded
+  char* qs = dsm;                                     // [MR rows], 2 atoms of MR x 128 B
   char* kring = qs + kUQ;                             // kUKst K tiles (2 atoms of 8 KB)
   char* vring = kring + kUKst * kUTile;               // kUVst V tiles
   char* pbuf = vring + kUVst * kUTile;                // [2][hi, lo] P parts
@@ -231,197 +233,211 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* bO = bars + 3;     // [2] O += P V of an even / odd tile done
   uint64_t* bK = bars + 5;     // [kUKst] K tile landed
   uint64_t* bV = bars + 5 + kUKst;  // [kUVst] V tile landed
+  uint64_t* bP = bars + 5 + kUKst + kUVst;  // [2] P buffer written (256 arrivals)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + kUBars);
   int* s_fail = reinterpret_cast<int*>(tslot + 1);
   const int sg = blockIdx.y, split = blockIdx.x;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int rows = d.G * d.B;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // warp w reads TMEM lanes 32 (w % 4) ..: thread (w, lane) owns query row
-  // 32 (w % 4) + lane, the w / 4 half of each S tile's keys and of O
-  const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-  const bool busy = (warp & 3) * 32 < rows;  // (warp-uniform) some row of this warp is real
   const int key0 = split * d.split_pages * kPS;
   const int key1 = min(d.L, key0 + d.split_pages * kPS);
   const int n = (key1 - key0 + kUKeys - 1) / kUKeys;
-  const int kv_row0 = sg * d.L + key0;                 // first key of the split, as a tensor row
-  const int q_row0 = (s * d.Hq + g * d.G) * d.B;       // the group's first query row
-
-  auto load_k = [&](int t) {  // one thread
-    uint64_t* bar = &bK[t % kUKst];
-    char* dst = kring + (t % kUKst) * kUTile;
-    mbar_expect_tx(bar, kUTile);
-    tma_load_2d(dst, &kmap, 0, kv_row0 + t * kUKeys, bar);
-    tma_load_2d(dst + kUTile / 2, &kmap, 64, kv_row0 + t * kUKeys, bar);
-  };
-  auto load_v = [&](int t) {
-    uint64_t* bar = &bV[t % kUVst];
-    char* dst = vring + (t % kUVst) * kUTile;
-    mbar_expect_tx(bar, kUTile);
-    tma_load_2d(dst, &vmap, 0, kv_row0 + t * kUKeys, bar);
-    tma_load_2d(dst + kUTile / 2, &vmap, 64, kv_row0 + t * kUKeys, bar);
-  };
-  constexpr uint32_t idesc_s = umma_idesc_bf16(128, kUKeys, 0);
-  constexpr uint32_t idesc_o = umma_idesc_bf16(128, kD, 1);
-  uint32_t tbase = 0;
-  auto issue_s = [&](int t) {  // S = Q K^T of tile t into S buffer t & 1 (one thread)
-    const char* kt = kring + (t % kUKst) * kUTile;
-    tc_fence_after();
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t ko = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-      const uint32_t kk = (ks >> 2) * (kUKeys * 128) + (ks & 3) * 32;
-      umma_bf16(tbase + (t & 1) * kUKeys, umma_desc(su32(qs) + ko, 16, 1024),
-                umma_desc(su32(kt) + kk, 16, 1024), idesc_s, ks > 0);
-    }
-    umma_commit(&bS[t & 1]);
-  };
 
   if (tid == 0) {
-    for (int i = 0; i < kUBars; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < kUBars; ++i) mbar_init(&bars[i], i >= 5 + kUKst + kUVst ? 256 : 1);
     fence_mbar_init();
     *s_fail = 0;
-    mbar_expect_tx(bQ, kUQ);
-    tma_load_2d(qs, &qmap, 0, q_row0, bQ);
-    tma_load_2d(qs + kUQ / 2, &qmap, 64, q_row0, bQ);
-    for (int t = 0; t < min(n, kUKst); ++t) load_k(t);
-    for (int t = 0; t < min(n, kUVst); ++t) load_v(t);
   }
   if (warp == 0) tmem_alloc(tslot, kUCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  tbase = *tslot;
-  const uint32_t tO = tbase + 128;
-  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
-  const float sl2 = d.scale_log2;
-  float mref = -INFINITY, lrow = 0.f;  // lrow: this half's share of the row sum
+  const uint32_t tbase = *tslot;
+  const uint32_t tO = tbase + 128;  // S tiles: columns [0, 64) and [64, 128)
   bool ok = true;
-  if (tid == 0) {
-    if (!mbar_wait(bQ, 0) || !mbar_wait(&bK[0], 0)) ok = false;
-    issue_s(0);
-  }
 
+  if (warp == 8) {
+    // ---- producer: TMA loads and tensor-core MMAs, one thread
+    if (lane == 0) {
+      const int kv_row0 = sg * d.L + key0;            // first key of the split, as a tensor row
+      const int q_row0 = (s * d.Hq + g * d.G) * d.B;  // the group's first query row
+      auto load_k = [&](int t) {
+        uint64_t* bar = &bK[t % kUKst];
+        char* dst = kring + (t % kUKst) * kUTile;
+        mbar_expect_tx(bar, kUTile);
+        tma_load_2d(dst, &kmap, 0, kv_row0 + t * kUKeys, bar);
+        tma_load_2d(dst + kUTile / 2, &kmap, 64, kv_row0 + t * kUKeys, bar);
+      };
+      auto load_v = [&](int t) {
+        uint64_t* bar = &bV[t % kUVst];
+        char* dst = vring + (t % kUVst) * kUTile;
+        mbar_expect_tx(bar, kUTile);
+        tma_load_2d(dst, &vmap, 0, kv_row0 + t * kUKeys, bar);
+        tma_load_2d(dst + kUTile / 2, &vmap, 64, kv_row0 + t * kUKeys, bar);
+      };
+      constexpr uint32_t idesc_s = umma_idesc_bf16(MR, kUKeys, 0);
+      constexpr uint32_t idesc_o = umma_idesc_bf16(MR, kD, 1);
+      // descriptors at offset 0; a k-step adds its byte offset >> 4 to the
+      // start-address field (no carry: shared addresses stay below 256 KB)
+      const uint64_t dq = umma_desc(su32(qs), 16, 1024);
+      auto issue_s = [&](int t) {  // S = Q K^T of tile t into S buffer t & 1
+        const uint64_t dk = umma_desc(su32(kring + (t % kUKst) * kUTile), 16, 1024);
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ko = (ks >> 2) * (MR * 128) + (ks & 3) * 32;
+          const uint32_t kk = (ks >> 2) * (kUKeys * 128) + (ks & 3) * 32;
+          umma_bf16(tbase + (t & 1) * kUKeys, dq + (ko >> 4), dk + (kk >> 4), idesc_s, ks > 0);
+        }
+        umma_commit(&bS[t & 1]);
+      };
+      mbar_expect_tx(bQ, MR * 256);
+      tma_load_2d(qs, &qmap, 0, q_row0, bQ);
+      tma_load_2d(qs + MR * 128, &qmap, 64, q_row0, bQ);
+      for (int t = 0; t < min(n, kUKst); ++t) load_k(t);
+      for (int t = 0; t < min(n, kUVst); ++t) load_v(t);
+      ok = ok && mbar_wait(bQ, 0) && mbar_wait(&bK[0], 0);
+      issue_s(0);
 #pragma unroll 1
-  for (int t = 0; t < n; ++t) {
-    if (tid == 0 && t + 1 < n) {  // the next tile's scores run during this tile's softmax
-      if (!mbar_wait(&bK[(t + 1) % kUKst], ((t + 1) / kUKst) & 1)) ok = false;
-      issue_s(t + 1);
-    }
-    __syncwarp();
-    if (!mbar_wait(&bS[t & 1], (t >> 1) & 1)) ok = false;
-    if (tid == 0 && t + kUKst < n) load_k(t + kUKst);  // tile t's K stage is free again
-    // P V of two tiles back has finished: its P buffers and V stage are free
-    if (t >= 2 && !mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1)) ok = false;
-    if (tid == 0 && t >= 2 && t + 1 < n) load_v(t + 1);
-    tc_fence_after();
-    if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
-
-    // this thread's 32 scores of the tile
-    const int kb = key0 + t * kUKeys + half * 32;
-    float sv[32];
-    float mx = -INFINITY;
-    if (busy) {
-      tmem_ld32(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
-      if (kb + 32 <= key1) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] *= sl2;
-          mx = fmaxf(mx, sv[i]);
+      for (int t = 0; t < n && ok; ++t) {  // (a failed wait ends the stream; the softmax warps give up too)
+        if (t + 1 < n) {  // the next tile's scores run during this tile's softmax
+          ok = ok && mbar_wait(&bK[(t + 1) % kUKst], ((t + 1) / kUKst) & 1);
+          issue_s(t + 1);
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = kb + i < key1 ? sv[i] * sl2 : -INFINITY;
-          mx = fmaxf(mx, sv[i]);
+        ok = ok && mbar_wait(&bS[t & 1], (t >> 1) & 1);
+        if (t + kUKst < n) load_k(t + kUKst);  // tile t's K stage is free again
+        // P V of two tiles back has finished (before this barrier completes
+        // again): V stage (t + 1) % kUVst is free
+        if (t >= 2) {
+          ok = ok && mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1);
+          if (t + 1 < n) load_v(t + 1);
         }
+        ok = ok && mbar_wait(&bP[t & 1], (t >> 1) & 1) && mbar_wait(&bV[t % kUVst], (t / kUVst) & 1);
+        tc_fence_after();
+        const uint64_t dv = umma_desc(su32(vring + (t % kUVst) * kUTile), kUKeys * 128, 1024);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint64_t dp = umma_desc(su32(pbuf + ((t & 1) * 2 + h) * kUP), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kUKeys / 16; ++ks)
+            umma_bf16(tO, dp + ((ks * 32) >> 4), dv + ((ks * 16 * 128) >> 4), idesc_o,
+                      (t > 0 || h > 0 || ks > 0) ? 1u : 0u);
+        }
+        umma_commit(&bO[t & 1]);
       }
-      xmax[half * 128 + row] = mx;
+      if (!ok) *s_fail = 1;
     }
-    __syncthreads();  // both halves' maxima
-    char* phi = pbuf + (t & 1) * 2 * kUP;
-    char* plo = phi + kUP;
-    if (busy) {
-      mx = fmaxf(xmax[row], xmax[128 + row]);
-      const bool grow = mx > mref + 8.f;  // the same decision in both halves of the row
-      if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
-        const float nref = grow ? mx : mref;
-        const float alpha = grow ? exp2f(mref - nref) : 1.f;  // 0 while nothing is accumulated
-        lrow *= alpha;
-        if (t > 0) {
-          // O holds every P V up to tile t - 1
-          if (!mbar_wait(&bO[(t - 1) & 1], ((t - 1) >> 1) & 1)) ok = false;
-          tc_fence_after();
+  } else {
+    // ---- softmax warps: warp w reads TMEM lanes 32 (w % 4) .. (its
+    // sub-partition), where the accumulator rows (M = 128) 32 (w % 4) + lane
+    // or (M = 64) 16 (w % 4) + lane, lane < 16, live; a thread owns its row's
+    // w / 4 half of each S tile's keys and of O
+    constexpr int RPW = MR / 4;  // accumulator rows per sub-partition
+    const int row = (warp & 3) * RPW + lane, half = warp >> 2;
+    const bool mine = lane < RPW && row < rows;  // this thread's row is a real query row
+    const bool busy = (warp & 3) * RPW < rows;   // (warp-uniform) some row of this warp is real
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const float sl2 = d.scale_log2;
+    float mref = -INFINITY, lrow = 0.f;  // lrow: this half's share of the row sum
 #pragma unroll 1
-          for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-            float v[32];
-            tmem_ld32(tO + lane_off + c0, v);
+    for (int t = 0; t < n; ++t) {
+      ok = ok && mbar_wait(&bS[t & 1], (t >> 1) & 1);
+      // the P buffers of this parity are free once P V of two tiles back is done
+      ok = ok && (t < 2 || mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1));
+      tc_fence_after();
+      const int kb = key0 + t * kUKeys + half * 32;
+      float sv[32];
+      float mx = -INFINITY;
+      if (busy) {
+        tmem_ld32(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
+        if (kb + 32 <= key1) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= alpha;
-            tmem_st32(tO + lane_off + c0, v);
+          for (int i = 0; i < 32; ++i) {
+            sv[i] *= sl2;
+            mx = fmaxf(mx, sv[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            sv[i] = kb + i < key1 ? sv[i] * sl2 : -INFINITY;
+            mx = fmaxf(mx, sv[i]);
           }
         }
-        mref = nref;
+        if (lane < RPW) xmax[half * 128 + row] = mx;
       }
-      // P = 2^(s - mref) <= 2^8: high part and remainder, [128 rows][64 keys]
-      // K-major, swizzled
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float p0 = exp2f(sv[c8 * 8 + 2 * u] - mref);
-          const float p1 = exp2f(sv[c8 * 8 + 2 * u + 1] - mref);
-          lrow += p0 + p1;
-          hi[u] = pack_bf16x2(p0, p1);
-          const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xffff0000u);
-          lo[u] = pack_bf16x2(p0 - h0, p1 - h1);
-        }
-        const uint32_t o = sw128_off(row, half * 32 + c8 * 8, 128);
-        *reinterpret_cast<uint4*>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      if (!mbar_wait(&bV[t % kUVst], (t / kUVst) & 1)) ok = false;
-      tc_fence_after();
-      const char* vt = vring + (t % kUVst) * kUTile;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t pa = su32(h ? plo : phi);
-#pragma unroll
-        for (int ks = 0; ks < kUKeys / 16; ++ks)
-          umma_bf16(tO, umma_desc(pa + ks * 32, 16, 1024),
-                    umma_desc(su32(vt) + ks * 16 * 128, kUKeys * 128, 1024), idesc_o,
-                    (t > 0 || h > 0 || ks > 0) ? 1u : 0u);
-      }
-      umma_commit(&bO[t & 1]);
-    }
-  }
-  __syncwarp();
-  if (!mbar_wait(&bO[(n - 1) & 1], ((n - 1) >> 1) & 1)) ok = false;
-  tc_fence_after();
-  if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
-  if (half == 1) xmax[row] = lrow;  // the second half's row sum
-  __syncthreads();
-  if (!*s_fail && busy) {
-    float* dst = part + ((static_cast<size_t>(sg) * d.nsplit + split) * rows + row) * kPartStride;
+      bar_sync(1, 256);  // both halves' maxima
+      char* phi = pbuf + (t & 1) * 2 * kUP;
+      char* plo = phi + kUP;
+      if (busy) {
+        if (lane < RPW) mx = fmaxf(xmax[row], xmax[128 + row]);
+        // the same decision in both halves of the row; padding lanes never move
+        const bool grow = mine && mx > mref + 8.f;
+        if (__any_sync(0xffffffffu, grow)) {  // tcgen05.ld/st are warp-wide
+          const float nref = grow ? mx : mref;
+          const float alpha = grow ? exp2f(mref - nref) : 1.f;  // 0 while nothing is accumulated
+          lrow *= alpha;
+          if (t > 0) {
+            // O holds every P V up to tile t - 1
+            ok = ok && mbar_wait(&bO[(t - 1) & 1], ((t - 1) >> 1) & 1);
+            tc_fence_after();
 #pragma unroll 1
-    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-      float v[32];
-      tmem_ld32(tO + lane_off + c0, v);
-      if (row < rows) {
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+              float v[32];
+              tmem_ld32(tO + lane_off + c0, v);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4*>(dst + 4 + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+              for (int i = 0; i < 32; ++i) v[i] *= alpha;
+              tmem_st32(tO + lane_off + c0, v);
+            }
+          }
+          mref = nref;
+        }
+        // P = 2^(s - mref) <= 2^8: high part and remainder, [128 rows][64
+        // keys] K-major, swizzled
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float p0 = ex2_approx(sv[c8 * 8 + 2 * u] - mref);
+            const float p1 = ex2_approx(sv[c8 * 8 + 2 * u + 1] - mref);
+            lrow += p0 + p1;
+            hi[u] = pack_bf16x2(p0, p1);
+            const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xffff0000u);
+            lo[u] = pack_bf16x2(p0 - h0, p1 - h1);
+          }
+          if (lane < RPW) {
+            const uint32_t o = sw128_off(row, half * 32 + c8 * 8, MR);
+            *reinterpret_cast<uint4*>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+        }
       }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bP[t & 1]);
     }
-    if (row < rows && half == 0) {
-      dst[0] = mref;
-      dst[1] = lrow + xmax[row];
+    ok = ok && mbar_wait(&bO[(n - 1) & 1], ((n - 1) >> 1) & 1);
+    tc_fence_after();
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
+    if (half == 1 && lane < RPW) xmax[row] = lrow;  // the second half's row sum
+    bar_sync(1, 256);
+    if (!*s_fail && busy) {
+      float* dst = part + ((static_cast<size_t>(sg) * d.nsplit + split) * rows + row) * kPartStride;
+#pragma unroll 1
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+        float v[32];
+        tmem_ld32(tO + lane_off + c0, v);
+        if (mine) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + 4 + c0 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+      if (mine && half == 0) {
+        dst[0] = mref;
+        dst[1] = lrow + xmax[row];
+      }
     }
   }
   tc_fence_before();
@@ -484,19 +500,27 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-      cudaError_t e0 = cudaFuncSetAttribute(dense_umma_kernel,
+      cudaError_t e0 = cudaFuncSetAttribute(dense_umma_kernel<64>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
+      if (e0 == cudaSuccess)
+        e0 = cudaFuncSetAttribute(dense_umma_kernel<128>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
       if (e0 != cudaSuccess) return record_cuda_error(e0);
       attr_done[dev] = true;
     }
     int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.off_status);
+    const bool m64 = d.G * d.B <= 64;
     CUtensorMap qmap, kmap, vmap;
-    if (make_tmap(&qmap, q, rows, 128) != LOSA_OK ||
+    if (make_tmap(&qmap, q, rows, m64 ? 64 : 128) != LOSA_OK ||
         make_tmap(&kmap, k_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK ||
         make_tmap(&vmap, v_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK)
       return record_cuda_error(cudaErrorInvalidValue);
-    dense_umma_kernel<<<dim3(d.nsplit, d.S * d.Hkv), 256, kUSmem, st>>>(qmap, kmap, vmap, part,
-                                                                       status, d);
+    if (m64)
+      dense_umma_kernel<64><<<dim3(d.nsplit, d.S * d.Hkv), 288, kUSmem, st>>>(qmap, kmap, vmap,
+                                                                             part, status, d);
+    else
+      dense_umma_kernel<128><<<dim3(d.nsplit, d.S * d.Hkv), 288, kUSmem, st>>>(qmap, kmap, vmap,
+                                                                              part, status, d);
   } else {
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);
