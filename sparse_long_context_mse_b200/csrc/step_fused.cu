@@ -54,9 +54,7 @@ constexpr int kCandCap = 64;                     // per-warp compaction buffer
 constexpr int kThreadsG = 512;                   // gather kernel: one warp per merged row
 constexpr int kWarpsG = kThreadsG / 32;
 constexpr int kPageWarps = 8;                    // gather kernel: warps sharing an m16 tile's pages
-constexpr int kMaxGatherCtas = kGatherCtas;  // CTAs per group in the gather kernel
 constexpr int kMaxGatherPages = 16;              // pages in flight per K2 CTA
-constexpr int kGatherSmemTarget = 113 * 1024;    // room for another CTA on the SM
 
 __device__ __forceinline__ unsigned long long umax64(unsigned long long a, unsigned long long b) {
   return a > b ? a : b;
@@ -972,7 +970,9 @@ struct GatherLayout {
   int qs;       // this CTA's suffix rows' queries (same formats)
   int ocache;   // cached o_p rows of this CTA's stable suffix rows
   int lcache;   // their cached L_p
-  int sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf, total;
+  int sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf;
+  int comb;     // per row: the CTAs owning one of its pages (the non-empty partials)
+  int total;
 };
 
 struct GatherParams {
@@ -1000,6 +1000,7 @@ struct GatherParams {
   int n_oa;      // max active rows owned per CTA
   int n_os;      // max stable suffix rows per CTA
   int wpart;     // bf16: warps split pages and keep per-warp partials
+  int comb_rows; // rows per batch of the last CTA's combine (their partials staged in the region)
   GatherLayout lo;
 };
 
@@ -1008,13 +1009,15 @@ struct GatherParams {
 // largest list head (at least k keys reach it, so the top k all do); the
 // keys at or above it are placed by ballots and rank-sorted.  Fallback:
 // sort-and-merge trees or k rounds of warp argmax.
+// base: the group's lists [nc][R][k] (written by the scan kernel: read
+// through L2, not L1)
 template <int KP>
-__device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int sg,
+__device__ __forceinline__ void merge_row(const GatherParams& prm, int r,
+                                          const unsigned long long* base,
                                           unsigned long long* out, unsigned long long* fb,
                                           unsigned long long* hb) {
   const Dims& d = prm.d;
   const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
-  const unsigned long long* base = prm.cand + static_cast<size_t>(sg) * nc * R * k;
   if (KP > 0) {
     constexpr int KQ = KP > 0 ? KP : 1;
     const unsigned lt = (1u << lane) - 1u;
@@ -1105,7 +1108,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   const int g4 = lane >> 2, t4 = lane & 3;
   const int rank = blockIdx.x;  // this CTA's place among the group's CL CTAs
   constexpr int CL = kGatherCtas;
-  static_assert((CL & (CL - 1)) == 0, "CTAs per group: a power of two");
+  static_assert((CL & (CL - 1)) == 0 && CL <= 32, "CTAs per group: a power of two, at most a warp");
   const int sg = blockIdx.y;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int G = d.G, B = d.B, A = d.A, R = d.R, k = d.k;
@@ -1131,6 +1134,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride] (fp32 path)
   float* part_cta = prm.part_g + (static_cast<size_t>(sg) * CL + rank) * R * kPartStride;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
+  uint32_t* rmask = reinterpret_cast<uint32_t*>(smem + lo.comb);  // [R] CTAs owning the row's pages
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
   int32_t* s_nlp = misc + 1;
@@ -1157,6 +1161,9 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 #pragma unroll 1
   for (int e = tid; e < R * kPartStride; e += kThreadsG)  // empty partials
     part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+#pragma unroll 1
+  for (int r = tid; r < R; r += kThreadsG)  // every CTA holds a partial of every row
+    rmask[r] = sel ? 0u : (CL >= 32 ? 0xffffffffu : (1u << CL) - 1u);
   if (sel) {
 #pragma unroll 1
     for (int w = tid; w < nwords; w += kThreadsG) bitmap[w] = 0u;
@@ -1182,6 +1189,8 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   // everything below reads what the scan kernel wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
+  const unsigned long long* cand_sg =
+      prm.cand + static_cast<size_t>(sg) * d.nchunk * R * k;
   {
     const int32_t* actg = prm.act_g + static_cast<size_t>(sg) * (R + GB);
 #pragma unroll 1
@@ -1195,7 +1204,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 #pragma unroll 1
     for (int r = warp; r < R; r += kWarpsG) {
       unsigned long long* best = mbuf + (kWarpsG + warp) * kCandCap;
-      merge_row<KP>(prm, r, sg, best, mbuf + warp * kCandCap,
+      merge_row<KP>(prm, r, cand_sg, best, mbuf + warp * kCandCap,
                     mbuf + 2 * kWarpsG * kCandCap + warp * 32);
       int32_t* dst = sel_all + r * k;
       const bool report = prm.page_idx && r % CL == rank;
@@ -1310,8 +1319,9 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         if (p < 0 || p >= d.P) continue;
         const int w = p >> 5;
         const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
-        if (u % CL != rank) continue;
         const int r = e / k;
+        atomicOr(&rmask[r], 1u << (u % CL));  // the CTAs holding a partial of row r
+        if (u % CL != rank) continue;
         if (u / CL < prm.max_lp) {
           lpages[u / CL] = p;
           atomicOr(&masks[(u / CL) * d.MW + (r >> 5)], 1u << (r & 31));
@@ -1589,75 +1599,89 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   int* s_last = misc + 2;
   if (tid == 0) {
     __threadfence();  // this CTA's partials and suffixes before its arrival
-    *s_last = atomicAdd(prm.cnt + sg, 1) == CL - 1;
+    const bool last = atomicAdd(prm.cnt + sg, 1) == CL - 1;
+    if (last) __threadfence();  // the other CTAs' writes, seen past their arrivals
+    *s_last = last;
   }
   __syncthreads();
   if (!*s_last) return;
-  __threadfence();  // every other CTA's writes are visible past its arrival
 
-  // ---- combine: per row, the partials of the CL CTAs in fixed order
-  // (deterministic), eight in flight at a time; cache write-back; merge with
-  // the suffix
+  // ---- combine, in batches of comb_rows rows.  A CTA's partial of row r is
+  // non-empty only if it owns one of the row's pages (rmask); each warp
+  // stages its row's non-empty partials (ascending CTA) and its suffix in the
+  // row's CL + 1 slots of the region, then merges them in that order
+  // (deterministic), writes the cache back and merges with the suffix.
+  float* stg = reinterpret_cast<float*>(region);
+  const float* pg = prm.part_g + static_cast<size_t>(sg) * CL * R * kPartStride;
+  const float* sxg = prm.sfx_g + static_cast<size_t>(sg) * R * kPartStride;
+  constexpr int c16 = kPartStride / 4;  // 16-byte chunks per partial
 #pragma unroll 1
-  for (int r = warp; r < R; r += kWarpsG) {
-    const float* base = prm.part_g + (static_cast<size_t>(sg) * CL * R + r) * kPartStride;
-    const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
-    const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4) + lane);  // the row's suffix
-    const float Ls = __ldcg(sx);
-    float M = -INFINITY, lsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int h = 0; h < kMaxGatherCtas; h += 8) {
-      if (h < CL) {
-        float mc[8], lc[8];
-        float4 ac[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          mc[i] = -INFINITY;
-          if (h + i < CL) {
-            const float* pr = base + static_cast<size_t>(h + i) * R * kPartStride;
-            mc[i] = __ldcg(pr);
-            lc[i] = __ldcg(pr + 1);
-            ac[i] = __ldcg(reinterpret_cast<const float4*>(pr + 4) + lane);
-          }
-        }
-        float Mh = M;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) Mh = fmaxf(Mh, mc[i]);
-        if (Mh != -INFINITY) {
-          const float rs = exp2f(M - Mh);  // 0 while nothing is accumulated
-          lsum *= rs;
-          acc.x *= rs;
-          acc.y *= rs;
-          acc.z *= rs;
-          acc.w *= rs;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (mc[i] != -INFINITY) {
-              const float w = exp2f(mc[i] - Mh);
-              lsum += w * lc[i];
-              acc.x += w * ac[i].x;
-              acc.y += w * ac[i].y;
-              acc.z += w * ac[i].z;
-              acc.w += w * ac[i].w;
-            }
-          }
-          M = Mh;
+  for (int r0 = 0; r0 < R; r0 += prm.comb_rows) {
+    const int nr = min(prm.comb_rows, R - r0);
+#pragma unroll 1
+    for (int i = warp; i < nr; i += kWarpsG) {
+      const int r = r0 + i;
+      const uint32_t m = rmask[r];
+      const int np = __popc(m);
+      float* rs = stg + i * (CL + 1) * kPartStride;
+      const int own = lane < np ? static_cast<int>(__fns(m, 0u, lane + 1)) : 0;  // lane j: j-th owner
+#pragma unroll 1
+      for (int e0 = 0; e0 < (np + 1) * c16; e0 += 32) {
+        const int e = e0 + lane, j = e / c16, c = e - j * c16;
+        const int cj = __shfl_sync(0xffffffffu, own, min(j, 31));
+        if (e < (np + 1) * c16) {
+          const float* gsrc = j < np ? pg + (static_cast<size_t>(cj) * R + r) * kPartStride
+                                     : sxg + static_cast<size_t>(r) * kPartStride;
+          cp_async16(su32(rs + j * kPartStride + 4 * c), gsrc + 4 * c, 16u);
         }
       }
     }
-    const float inv = __frcp_rn(lsum);
-    const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    const float Lp = (M + __log2f(lsum)) * kLn2;
-    const size_t grow = grow0 + (r / A) * B + act_tok[r];
-    *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
-    if (lane == 0) prm.l_p[grow] = Lp;
-    float wa, wb, L;
-    lse_weights(Lp, Ls, wa, wb, L);
-    *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
-        make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
-                    wa * op.w + wb * os.w);
-    if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+#pragma unroll 1
+    for (int i = warp; i < nr; i += kWarpsG) {
+      const int r = r0 + i;
+      const int np = __popc(rmask[r]);
+      const float* rs = stg + i * (CL + 1) * kPartStride;
+      // lane j holds partial j's (m, l): the maximum and the weights in
+      // parallel, then the vectors accumulated in slot order
+      const float mj = lane < np ? rs[lane * kPartStride] : -INFINITY;
+      const float lj = lane < np ? rs[lane * kPartStride + 1] : 0.f;
+      float M = mj;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float wj = mj == -INFINITY ? 0.f : exp2f(mj - M);
+      float lsum = wj * lj;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int j = 0; j < np; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wj, j);
+        const float4 a4 = *reinterpret_cast<const float4*>(rs + j * kPartStride + 4 + 4 * lane);
+        acc.x += w * a4.x;
+        acc.y += w * a4.y;
+        acc.z += w * a4.z;
+        acc.w += w * a4.w;
+      }
+      const float* sx = rs + np * kPartStride;
+      const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
+      const float Ls = sx[0];
+      const float inv = __frcp_rn(lsum);
+      const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      const float Lp = (M + __log2f(lsum)) * kLn2;
+      const size_t grow = grow0 + (r / A) * B + act_tok[r];
+      *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
+      if (lane == 0) prm.l_p[grow] = Lp;
+      float wa, wb, L;
+      lse_weights(Lp, Ls, wa, wb, L);
+      *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+          make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                      wa * op.w + wb * os.w);
+      if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+    }
+    __syncthreads();  // the batch's slots are consumed before the next batch's copies
   }
 }
 
@@ -1739,10 +1763,15 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
   const int pbytes = kPS * rowb;
   const int bpad = (d.B + kPS - 1) / kPS * kPS;
   const bool sel = !d.all_pages && d.A > 0;
-  auto layout = [&](int ngp) {
+  // the region holds, in turn: the gathered pages, the page warps' partials,
+  // the partials staged for the combine
+  const long long slot = 4LL * kPartStride;  // one staged partial
+  auto layout = [&](int ngp, int crows) {
     GatherLayout& lo = prm->lo;
     Taker take;
-    lo.region = take(std::max(2LL * ngp * pbytes, prm->wpart ? 4LL * kPageWarps * 16 * kPartStride : 0LL),
+    lo.region = take(std::max({2LL * ngp * pbytes,
+                               prm->wpart ? 4LL * kPageWarps * 16 * kPartStride : 0LL,
+                               (CL + 1LL) * crows * slot}),
                      1024);
     lo.kbv = take(2LL * bpad * rowb, 128);
     lo.qa = take(1LL * (bf ? ntm * 16 : d.R) * rowb, 128);
@@ -1758,21 +1787,27 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
     lo.misc = take((16 + d.R + GB + ns) * 4, 16);
     lo.ps = take(kWarpsG * 16 * 4, 16);
     lo.mbuf = take(sel ? (2 * kCandCap + 32) * kWarpsG * 8 : 0, 16);
+    lo.comb = take(4LL * d.R, 16);
     lo.total = take.off;
     prm->ngp = ngp;
+    prm->comb_rows = crows;
     return lo.total;
   };
-  // the largest batch of pages in flight with two CTAs per SM, else the
-  // largest that fits one
-  int one = 0;
-  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
-    const int total = layout(ngp);
-    if (total <= std::min(max_dyn, kGatherSmemTarget)) return true;
-    if (total <= max_dyn && one == 0) one = ngp;
+  // the CTA holds an SM alone (512 threads at up to 128 registers): the
+  // largest batch of pages in flight, then as many combine rows per batch
+  // as fit
+  const int R1 = std::max(1, d.R);
+  bool ok = false;
+  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1 && !ok; ngp /= 2) {
+    for (int crows = R1; crows >= 1; crows = crows > 1 ? (crows + 1) / 2 : 0) {
+      if (layout(ngp, crows) <= max_dyn) {
+        ok = true;
+        break;
+      }
+      if (crows == 1) break;
+    }
   }
-  if (one == 0) return false;
-  layout(one);
-  return true;
+  return ok;
 }
 
 std::mutex g_attr_mu;
