@@ -37,18 +37,22 @@ class Shape(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
                 ("d", ctypes.c_int), ("L", ctypes.c_int), ("ps", ctypes.c_int),
                 ("B", ctypes.c_int), ("A", ctypes.c_int), ("budget", ctypes.c_int),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_int)]
 
 
-def shape(S, Hq, Hkv, d, L, ps, B, A, budget, scale=None) -> Shape:
+# variant bit: every active row attends to its GQA group's whole page union
+ATTEND_UNION = 1
+
+
+def shape(S, Hq, Hkv, d, L, ps, B, A, budget, scale=None, flags=0) -> Shape:
     if scale is None:
         scale = float(np.float32(1.0 / np.sqrt(d)))
-    return Shape(S, Hq, Hkv, d, L, ps, B, A, budget, scale)
+    return Shape(S, Hq, Hkv, d, L, ps, B, A, budget, scale, flags)
 
 
-def shape_of(cfg, scale=None) -> Shape:
+def shape_of(cfg, scale=None, flags=0) -> Shape:
     return shape(cfg.num_seqs, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.prefix_len,
-                 cfg.page_size, cfg.block_size, cfg.n_active, cfg.token_budget, scale)
+                 cfg.page_size, cfg.block_size, cfg.n_active, cfg.token_budget, scale, flags)
 
 
 def _load():
@@ -219,3 +223,22 @@ def step_forced(sh: Shape, Qc, K, V, Kb, Vb, active_idx, page_idx, o_p, l_p):
     _load().oracle_step_forced(ctypes.byref(sh), _f(Qc), _f(K), _f(V), _f(Kb), _f(Vb), _i(act),
                                _i(pidx), _f(o_p), _f(l_p), _f(out), _f(lse), _i(uc))
     return {"o_p": o_p, "l_p": l_p, "out": out, "lse": lse, "union_count": uc}
+
+
+def refresh_ref(sh: Shape, Qc, active_idx, q_ref):
+    """Drift-safe locality: ``q_ref`` with the active rows' current queries
+    moved in (a copy is returned)."""
+    Qc = f32(Qc)
+    q_ref = f32(q_ref).copy()
+    act = np.ascontiguousarray(active_idx, dtype=np.int32)
+    _load().oracle_refresh_ref(ctypes.byref(sh), _f(Qc), _i(act), _f(q_ref))
+    return q_ref
+
+
+def step_ref(sh: Shape, Qc, q_ref, K, V, kmin, kmax, Kb, Vb, o_p, l_p):
+    """One drift-safe LoSA step: locality against the reference queries, then
+    the reference refreshed for the recomputed rows.  Returns step()'s dict
+    plus ``q_ref`` (the updated reference)."""
+    res = step(sh, Qc, q_ref, K, V, kmin, kmax, Kb, Vb, o_p, l_p)
+    res["q_ref"] = refresh_ref(sh, Qc, res["active_idx"], q_ref)
+    return res

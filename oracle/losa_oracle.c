@@ -56,7 +56,13 @@ typedef struct {
     int A;        /* active tokens per query head, |A|          */
     int budget;   /* token budget per active query              */
     float scale;  /* softmax scale                              */
+    int flags;    /* variant bits, ORACLE_ATTEND_UNION below     */
 } oracle_shape;
+
+/* Variant: every active row attends to all pages of its GQA group's union
+ * (the pages that are loaded once per group, paper, methodology: sparse
+ * computation for active tokens) instead of only its own top-k pages. */
+#define ORACLE_ATTEND_UNION 1
 
 /* ---- planted-mistake switch (tests only) -------------------------------
  * 0 = the method as written.  A non-zero value plants one deliberate bug so
@@ -343,41 +349,45 @@ void oracle_step_forced(const oracle_shape* sh, const float* Qc, const float* K,
                         const int* page_idx, float* o_p, float* l_p, float* out, float* out_lse,
                         int* union_count) {
     int d = sh->d, B = sh->B, A = sh->A, k = pages_per_row(sh), P = n_pages(sh);
-    int* tok = (int*)malloc(sizeof(int) * (size_t)(k * sh->ps + 1));
+    int* tok = (int*)malloc(sizeof(int) * (size_t)(P * sh->ps + 1));
     double* o = (double*)malloc(sizeof(double) * (size_t)d);
     char* used = (char*)malloc((size_t)P);
-    for (int s = 0; s < sh->S; ++s) {
-        for (int h = 0; h < sh->Hq; ++h) {
-            int g = kv_head_of(sh, h);
+    int* ul = (int*)malloc(sizeof(int) * (size_t)P);
+    for (int s = 0; s < sh->S; ++s)
+        for (int g = 0; g < sh->Hkv; ++g) {
+            /* the group's union: every page some active row of the group selected */
+            memset(used, 0, (size_t)P);
+            int cnt = 0;
+            for (int h = 0; h < sh->Hq; ++h) {
+                if (kv_head_of(sh, h) != g) continue;
+                for (int a = 0; a < A; ++a)
+                    for (int c = 0; c < k; ++c) {
+                        int p = page_idx[(((size_t)s * sh->Hq + h) * A + a) * k + c];
+                        if (!used[p] || MUT(9)) { used[p] = 1; ++cnt; }
+                    }
+            }
+            if (union_count) union_count[s * sh->Hkv + g] = cnt;
+            int nu = 0;
+            for (int p = 0; p < P; ++p)
+                if (used[p]) ul[nu++] = p;
             const float* Kg = K + ((size_t)s * sh->Hkv + g) * (size_t)sh->L * d;
             const float* Vg = V + ((size_t)s * sh->Hkv + g) * (size_t)sh->L * d;
-            for (int a = 0; a < A; ++a) {
-                int t = active_idx[((size_t)s * sh->Hq + h) * A + a];
-                size_t r = ((size_t)s * sh->Hq + h) * B + t;
-                const int* pg = page_idx + (((size_t)s * sh->Hq + h) * A + a) * k;
-                int n = tokens_of_pages(sh, pg, k, tok);
-                double lse;
-                attend(d, (double)sh->scale, Qc + r * d, Kg, Vg, n, tok, o, &lse);
-                for (int i = 0; i < d; ++i) o_p[r * d + i] = (float)o[i];
-                l_p[r] = (float)lse;
+            for (int h = 0; h < sh->Hq; ++h) {
+                if (kv_head_of(sh, h) != g) continue;
+                for (int a = 0; a < A; ++a) {
+                    int t = active_idx[((size_t)s * sh->Hq + h) * A + a];
+                    size_t r = ((size_t)s * sh->Hq + h) * B + t;
+                    const int* pg = page_idx + (((size_t)s * sh->Hq + h) * A + a) * k;
+                    int n = ((sh->flags & ORACLE_ATTEND_UNION) && !MUT(12)) ? tokens_of_pages(sh, ul, nu, tok)
+                                                              : tokens_of_pages(sh, pg, k, tok);
+                    double lse;
+                    attend(d, (double)sh->scale, Qc + r * d, Kg, Vg, n, tok, o, &lse);
+                    for (int i = 0; i < d; ++i) o_p[r * d + i] = (float)o[i];
+                    l_p[r] = (float)lse;
+                }
             }
         }
-        if (union_count)
-            for (int g = 0; g < sh->Hkv; ++g) {
-                memset(used, 0, (size_t)P);
-                int cnt = 0;
-                for (int h = 0; h < sh->Hq; ++h) {
-                    if (kv_head_of(sh, h) != g) continue;
-                    for (int a = 0; a < A; ++a)
-                        for (int c = 0; c < k; ++c) {
-                            int p = page_idx[(((size_t)s * sh->Hq + h) * A + a) * k + c];
-                            if (!used[p] || MUT(9)) { used[p] = 1; ++cnt; }
-                        }
-                }
-                union_count[s * sh->Hkv + g] = cnt;
-            }
-    }
-    free(tok); free(o); free(used);
+    free(tok); free(o); free(used); free(ul);
     suffix_and_merge(sh, Qc, Kb, Vb, o_p, l_p, out, out_lse);
 }
 
@@ -422,4 +432,26 @@ void oracle_step(const oracle_shape* sh, const float* Qc, const float* Qp, const
     free(mse); free(U);
     oracle_step_forced(sh, Qc, K, V, Kb, Vb, active_idx, page_idx, o_p, l_p, out, out_lse,
                        union_count);
+}
+
+/* ------------------------------------------------------------------------
+ * Drift-safe locality (a variant; the pages score locality between steps
+ * t-1 and t, methodology: locality pruning).  A stable row keeps the prefix
+ * state computed from the query it had when it was last recomputed, so the
+ * variant scores each token against that reference query instead of the
+ * previous step's.  oracle_step is run with q_ref in place of Qp; this then
+ * moves the recomputed (active) rows' current queries into q_ref
+ * [S][Hq][B][d]; the other rows keep their reference.
+ * ---------------------------------------------------------------------- */
+void oracle_refresh_ref(const oracle_shape* sh, const float* Qc, const int* active_idx,
+                        float* q_ref) {
+    int d = sh->d, B = sh->B, A = sh->A;
+    for (int s = 0; s < sh->S; ++s)
+        for (int h = 0; h < sh->Hq; ++h)
+            for (int a = 0; a < A; ++a) {
+                int t = active_idx[((size_t)s * sh->Hq + h) * A + a];
+                size_t r = ((size_t)s * sh->Hq + h) * B + t;
+                if (MUT(11)) r = ((size_t)s * sh->Hq + h) * B + (t + 1) % B;
+                memcpy(q_ref + r * d, Qc + r * d, sizeof(float) * (size_t)d);
+            }
 }

@@ -38,9 +38,10 @@ def np_bound(q, kmin, kmax):
     return np.maximum(q * kmax.astype(np.float64), q * kmin.astype(np.float64)).sum(-1)
 
 
-def rand_shape(rng, S=2, Hq=4, Hkv=2, d=16, L=45, ps=4, B=6, A=2, budget=12, scale=None):
+def rand_shape(rng, S=2, Hq=4, Hkv=2, d=16, L=45, ps=4, B=6, A=2, budget=12, scale=None,
+               flags=0):
     return oracle.shape(S, Hq, Hkv, d, L, ps, B, A, budget,
-                        scale if scale is not None else float(np.float32(0.37)))
+                        scale if scale is not None else float(np.float32(0.37)), flags)
 
 
 def rand_inputs(rng, sh):
@@ -379,6 +380,111 @@ def pin_step_active_rows_bruteforce():
         for g in range(sh.Hkv):
             assert r["union_count"][s, g] == len(unions[g]), "union count vs set union"
             assert k <= r["union_count"][s, g] <= min(P, G * sh.A * k)
+
+
+def pin_step_attend_union_bruteforce():
+    """Variant: every active row attends to its group's whole page union.
+    The selection is the default's; o_p/L_p equal numpy attention over the
+    union's tokens (the union built here from page_idx); L_p is at least the
+    default's (log-sum-exp over a superset of the row's own tokens)."""
+    kw = dict(L=93, ps=4, B=8, A=3, budget=16)
+    sh, x, kmin, kmax, cache = _step_inputs(23, **kw)
+    shu, _, _, _, _ = _step_inputs(23, flags=oracle.ATTEND_UNION, **kw)
+    args = (x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"], cache["o_p"],
+            cache["l_p"])
+    r0 = oracle.step(sh, *args)
+    r = oracle.step(shu, *args)
+    for key in ("active_idx", "page_idx", "union_count"):
+        assert np.array_equal(r[key], r0[key]), key
+    G = sh.Hq // sh.Hkv
+    n_strict = 0
+    for s in range(sh.S):
+        for g in range(sh.Hkv):
+            pages = sorted(set(r["page_idx"][s, g * G:(g + 1) * G].reshape(-1).tolist()))
+            tok = np.concatenate([np.arange(p * sh.ps, min((p + 1) * sh.ps, sh.L)) for p in pages])
+            for h in range(g * G, (g + 1) * G):
+                for t in r["active_idx"][s, h]:
+                    o, l = np_attend(x["Qc"][s, h, t], x["K"][s, g][tok], x["V"][s, g][tok],
+                                     sh.scale)
+                    close(r["o_p"][s, h, t], o, 1e-6, "union row o_p")
+                    close(r["l_p"][s, h, t], l, 1e-5, "union row L_p")
+                    assert r["l_p"][s, h, t] >= r0["l_p"][s, h, t] - 1e-5
+                    n_strict += r["l_p"][s, h, t] > r0["l_p"][s, h, t] + 1e-4
+    assert n_strict > 0, "the union added no tokens anywhere: the case does not test the variant"
+
+
+def pin_step_attend_union_single_row():
+    """With one active row per group (G = 1, |A| = 1) the union is the row's
+    own pages: the variant equals the default step."""
+    kw = dict(Hq=2, Hkv=2, A=1, L=61, budget=12)
+    sh, x, kmin, kmax, cache = _step_inputs(24, **kw)
+    shu, _, _, _, _ = _step_inputs(24, flags=oracle.ATTEND_UNION, **kw)
+    args = (x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"], cache["o_p"],
+            cache["l_p"])
+    r0, r = oracle.step(sh, *args), oracle.step(shu, *args)
+    for key in ("o_p", "l_p", "out", "lse", "page_idx"):
+        assert np.array_equal(r[key], r0[key]), key
+
+
+def pin_refresh_ref_rows():
+    """Drift-safe reference: exactly the active rows take the current query
+    (bitwise); every other row keeps its reference."""
+    sh, x, kmin, kmax, cache = _step_inputs(25)
+    q_ref = x["Qp"] + np.float32(0.5)
+    r = oracle.step_ref(sh, x["Qc"], q_ref, x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                        cache["o_p"], cache["l_p"])
+    for s in range(sh.S):
+        for h in range(sh.Hq):
+            act = set(r["active_idx"][s, h].tolist())
+            for t in range(sh.B):
+                want = x["Qc"][s, h, t] if t in act else q_ref[s, h, t]
+                assert np.array_equal(r["q_ref"][s, h, t].view(np.uint32), want.view(np.uint32))
+
+
+def pin_drift_safe_slow_drift():
+    """A token drifting slowly in one direction: against the previous step it
+    never changes most, so plain locality never activates it; against its
+    reference (the query its cached state came from) the change grows as
+    n*delta and it becomes active at the first step with n*delta > the jump
+    size of the other tokens -- step 4 for delta = 0.3, jump = 1 (closed form
+    below)."""
+    d, B = 16, 4
+    sh = oracle.shape(1, 1, 1, d, 32, 4, B, 1, 8, float(np.float32(0.25)))
+    rng = np.random.default_rng(26)
+    u = np.zeros(d, np.float32)
+    u[0] = 1.0
+    K = rng.standard_normal((1, 1, 32, d)).astype(np.float32)
+    V = rng.standard_normal((1, 1, 32, d)).astype(np.float32)
+    Kb = rng.standard_normal((1, 1, B, d)).astype(np.float32)
+    Vb = rng.standard_normal((1, 1, B, d)).astype(np.float32)
+    kmin, kmax = oracle.build_meta(sh, K)
+    q1 = rng.standard_normal((1, 1, B, d)).astype(np.float32)
+    cache = oracle.dense_prefix(sh, q1, K, V, Kb, Vb)
+    delta, jump = np.float32(0.3), np.float32(1.0)
+    prev, ref = q1, q1.copy()
+    o_p, l_p = cache["o_p"], cache["l_p"]
+    o_p2, l_p2 = o_p, l_p
+    first_plain, first_safe = None, None
+    for n in range(1, 7):
+        cur = prev.copy()
+        cur[0, 0, 0] += delta * u                      # token 0: slow drift
+        j = 1 + (n - 1) % (B - 1)                      # one other token jumps by `jump`
+        e = np.zeros(d, np.float32)
+        e[1 + n % (d - 1)] = jump
+        cur[0, 0, j] += e
+        rp = oracle.step(sh, cur, prev, K, V, kmin, kmax, Kb, Vb, o_p, l_p)
+        rs = oracle.step_ref(sh, cur, ref, K, V, kmin, kmax, Kb, Vb, o_p2, l_p2)
+        if first_plain is None and 0 in rp["active_idx"][0, 0].tolist():
+            first_plain = n
+        if first_safe is None and 0 in rs["active_idx"][0, 0].tolist():
+            first_safe = n
+        prev, ref = cur, rs["q_ref"]
+        o_p, l_p, o_p2, l_p2 = rp["o_p"], rp["l_p"], rs["o_p"], rs["l_p"]
+    # token 0's change against its reference after n steps is n*delta in one
+    # channel; a jumping token changes by `jump`: first n with n*delta > jump
+    want = int(np.floor(float(jump) / float(delta))) + 1
+    assert first_plain is None, first_plain
+    assert first_safe == want, (first_safe, want)
 
 
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -16,6 +16,8 @@ MUTATIONS = {
     8: "page metadata drops the page's last token",
     9: "union count does not deduplicate",
     10: "log-normaliser misses the running max",
+    11: "drift-safe refresh writes the next token's row",
+    12: "union variant attends to the row's own pages only",
 }
 
 
