@@ -84,7 +84,18 @@ typedef struct {
     int32_t token_budget;  /* prefix tokens each active query may attend  */
     float   scale;         /* softmax scale; 0 selects 1/sqrt(d)          */
     int32_t dtype;         /* LOSA_F32 or LOSA_BF16                       */
+    int32_t flags;         /* 0, or LOSA_STEP_ATTEND_UNION (below)        */
 } losa_shape;
+
+/* ---- step variants (losa_shape.flags) ----------------------------------
+ * LOSA_STEP_ATTEND_UNION: each active row attends to every page of its GQA
+ *   group's union -- the pages the step loads once per (sequence, KV head),
+ *   paper, methodology: sparse computation for active tokens -- instead of
+ *   only its own top-k pages.  Selection (active_idx, page_idx) and the union
+ *   are unchanged; o_p/L_p of active rows cover more prefix tokens for the
+ *   same HBM traffic.  Only losa_step / losa_step_ref / losa_step_noalloc
+ *   read the flag; any other bit is LOSA_ERR_INVALID_ARG. */
+#define LOSA_STEP_ATTEND_UNION 1
 
 /* Bytes of page metadata for `shape` (the size of `page_meta` below). */
 size_t losa_page_meta_size(const losa_shape* shape);
@@ -166,6 +177,31 @@ int losa_step(const losa_shape* shape, const void* q_cur, const void* q_prev,
               const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
               float* out_lse, int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
               void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Drift-safe locality (a variant of losa_step).  The pages score a token's
+ * locality between denoising steps t-1 and t (methodology: locality
+ * pruning).  A stable token, though, keeps the prefix state computed from
+ * the query it had when it was last recomputed, and a slow drift in one
+ * direction never shows between two adjacent steps.  This entry point scores
+ * every token against that reference query instead:
+ *
+ *   q_ref  in/out [S][Hq][B][d], element type `dtype`: on entry, for each
+ *          row, the query its cached o_p/L_p were computed from (after the
+ *          cold-start dense pass: that pass's q).  The locality score is the
+ *          MSE of q_cur against q_ref.  On return the active rows hold
+ *          q_cur (their cache was recomputed from it); the other rows are
+ *          unchanged.  Must not overlap q_cur or any output.
+ *
+ * Every other argument, result and error is losa_step's (q_prev is replaced
+ * by q_ref).  The rewrite of q_ref happens after every read of it in this
+ * call, on `stream`.
+ */
+int losa_step_ref(const losa_shape* shape, const void* q_cur, void* q_ref,
+                  const void* k_prefix, const void* v_prefix, const void* page_meta,
+                  const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
+                  float* out_lse, int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
+                  void* workspace, size_t ws_bytes, void* stream);
 
 /* Size of the scratch array behind losa_step_noalloc: 8 MiB per GPU. */
 #define LOSA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)

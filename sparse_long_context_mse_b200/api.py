@@ -25,12 +25,14 @@ LOSA_ERR_DEVICE_TIMEOUT = 4
 LOSA_ERR_DEVICE_BOUNDS = 5
 LOSA_F32 = 0
 LOSA_BF16 = 1
+LOSA_STEP_ATTEND_UNION = 1  # losa_shape.flags: active rows attend to the group's whole union
 LOSA_WS_DENSE = 0
 LOSA_WS_STEP = 1
 
 #: every symbol ``include/losa.h`` declares
 EXPORTS = ("losa_page_meta_size", "losa_workspace_size", "losa_build_page_meta",
-           "losa_dense_prefix", "losa_step", "losa_step_noalloc", "losa_read_device_status",
+           "losa_dense_prefix", "losa_step", "losa_step_ref", "losa_step_noalloc",
+           "losa_read_device_status",
            "losa_status_string", "losa_last_error")
 
 #: size of the library-owned scratch behind ``losa_step_noalloc``
@@ -50,7 +52,7 @@ class Shape(ctypes.Structure):
                 ("prefix_len", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("n_active", ctypes.c_int32),
                 ("token_budget", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
     # derived sizes (same rules as the library's validation)
     @property
@@ -71,18 +73,19 @@ class Shape(ctypes.Structure):
 
 
 def make_shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
-               n_active, token_budget, dtype="bf16", scale: Optional[float] = None) -> Shape:
+               n_active, token_budget, dtype="bf16", scale: Optional[float] = None,
+               flags: int = 0) -> Shape:
     dt = {"bf16": LOSA_BF16, "f32": LOSA_F32, LOSA_BF16: LOSA_BF16, LOSA_F32: LOSA_F32}[dtype]
     sc = float(scale) if scale is not None else 0.0
     return Shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
-                 n_active, token_budget, sc, dt)
+                 n_active, token_budget, sc, dt, flags)
 
 
-def shape_of(cfg, scale: Optional[float] = None) -> Shape:
+def shape_of(cfg, scale: Optional[float] = None, flags: int = 0) -> Shape:
     """Shape of a :class:`synth.LosaConfig` (duck-typed)."""
     return make_shape(cfg.num_seqs, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.prefix_len,
                       cfg.page_size, cfg.block_size, cfg.n_active, cfg.token_budget, cfg.dtype,
-                      scale)
+                      scale, flags)
 
 
 _lib = None
@@ -108,6 +111,8 @@ def lib():
         L.losa_dense_prefix.restype = i32
         L.losa_step.argtypes = [sp] + [vp] * 14 + [vp, sz, vp]
         L.losa_step.restype = i32
+        L.losa_step_ref.argtypes = [sp] + [vp] * 14 + [vp, sz, vp]
+        L.losa_step_ref.restype = i32
         L.losa_step_noalloc.argtypes = [sp] + [vp] * 14 + [vp]
         L.losa_step_noalloc.restype = i32
         L.losa_read_device_status.argtypes = [vp, vp]
@@ -209,6 +214,22 @@ def dense_prefix(sh: Shape, q, k_prefix, v_prefix, k_blk, v_blk, o_p, l_p, out, 
 
 def step(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p, l_p, out,
          out_lse, workspace, active_idx=None, page_idx=None, union_count=None, stream=None):
+    _step_call("losa_step", sh, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
+               l_p, out, out_lse, workspace, active_idx, page_idx, union_count, stream)
+
+
+def step_ref(sh: Shape, q_cur, q_ref, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p, l_p,
+             out, out_lse, workspace, active_idx=None, page_idx=None, union_count=None,
+             stream=None):
+    """``losa_step_ref``: drift-safe locality.  ``q_ref`` holds each row's
+    reference query (the one its cached o_p/L_p came from); the active rows'
+    entries are overwritten with ``q_cur``."""
+    _step_call("losa_step_ref", sh, q_cur, q_ref, k_prefix, v_prefix, page_meta, k_blk, v_blk,
+               o_p, l_p, out, out_lse, workspace, active_idx, page_idx, union_count, stream)
+
+
+def _step_call(fn, sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
+               l_p, out, out_lse, workspace, active_idx, page_idx, union_count, stream):
     dev = _device_of(q_cur)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
@@ -227,7 +248,7 @@ def step(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, 
             _ptr(page_idx, (sh.num_seqs, sh.n_q_heads, A, k), torch.int32, "page_idx", dev),
             _ptr(union_count, (sh.num_seqs, sh.n_kv_heads), torch.int32, "union_count", dev),
             _ptr(workspace, None, torch.uint8, "workspace", dev)]
-    _check(lib().losa_step(ctypes.byref(sh), *args, workspace.numel(), _stream(stream)))
+    _check(getattr(lib(), fn)(ctypes.byref(sh), *args, workspace.numel(), _stream(stream)))
 
 
 def step_noalloc(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,

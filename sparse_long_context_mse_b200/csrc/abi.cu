@@ -44,6 +44,7 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   if (!(std::isfinite(sh->scale)) || sh->scale < 0.f) return LOSA_ERR_INVALID_ARG;
   if (sh->head_dim != kD || sh->page_size != kPS) return LOSA_ERR_UNSUPPORTED;
   if (sh->dtype != LOSA_F32 && sh->dtype != LOSA_BF16) return LOSA_ERR_UNSUPPORTED;
+  if (sh->flags & ~LOSA_STEP_ATTEND_UNION) return LOSA_ERR_INVALID_ARG;
   const int G = sh->n_q_heads / sh->n_kv_heads;
   if (sh->block_size > kMaxB || G * sh->block_size > kMaxRowsPerGroup) return LOSA_ERR_UNSUPPORTED;
   const long long P = (static_cast<long long>(sh->prefix_len) + kPS - 1) / kPS;
@@ -65,6 +66,7 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   d->dtype = sh->dtype;
   d->esz = sh->dtype == LOSA_BF16 ? 2 : 4;
   d->all_pages = (d->k == d->P);
+  d->attend_union = (sh->flags & LOSA_STEP_ATTEND_UNION) != 0;
   d->scale = sh->scale > 0.f ? sh->scale : 1.0f / std::sqrt(static_cast<float>(sh->head_dim));
   d->scale_log2 = d->scale * kLog2e;
   d->Umax = static_cast<int>(std::min<long long>(P, static_cast<long long>(d->R) * d->k));

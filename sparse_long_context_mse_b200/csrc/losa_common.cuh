@@ -30,6 +30,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 struct Dims {
   int S, Hq, Hkv, G, L, P, B, A, k, R, MW, Umax, dtype, esz;
   int all_pages;          // k == P: every page is selected, no scoring needed
+  int attend_union;       // LOSA_STEP_ATTEND_UNION: active rows attend to the group's union
   float scale;            // softmax scale (natural-log units)
   float scale_log2;       // scale * log2(e): scores in base-2 units
   // prefix splits (dense pass); page chunks of the step's scan
@@ -224,7 +225,7 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
                       const void* v_prefix, const void* page_meta, const void* k_blk,
                       const void* v_blk, float* o_p, float* l_p, float* out, float* out_lse,
                       int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
-                      void* workspace, cudaStream_t st);
+                      void* workspace, cudaStream_t st, void* q_ref_out = nullptr);
 int record_cuda_error(cudaError_t e);  // stores the message, returns LOSA_ERR_CUDA
 int num_sms();
 

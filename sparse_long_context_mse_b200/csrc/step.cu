@@ -1,12 +1,14 @@
-// step.cu -- C entry point of one LoSA denoising step: host validation, then
-// the fused single-launch kernel of step_fused.cu.
+// step.cu -- C entry points of one LoSA denoising step (plain and drift-safe):
+// host validation, then the two step kernels of step_fused.cu.
 #include "losa_common.cuh"
 
-extern "C" int losa_step(const losa_shape* shape, const void* q_cur, const void* q_prev,
-                         const void* k_prefix, const void* v_prefix, const void* page_meta,
-                         const void* k_blk, const void* v_blk, float* o_p, float* l_p,
-                         float* out, float* out_lse, int32_t* active_idx, int32_t* page_idx,
-                         int32_t* union_count, void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+
+int step_common(const losa_shape* shape, const void* q_cur, const void* q_prev, void* q_ref_out,
+                const void* k_prefix, const void* v_prefix, const void* page_meta,
+                const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
+                float* out_lse, int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
+                void* workspace, size_t ws_bytes, void* stream) {
   using namespace losa;
   Dims d;
   int rc = make_dims(shape, LOSA_WS_STEP, &d);
@@ -23,8 +25,39 @@ extern "C" int losa_step(const losa_shape* shape, const void* q_cur, const void*
   if (overlaps(out, ob, q_cur, qb) || overlaps(out, ob, q_prev, qb) || overlaps(out, ob, o_p, ob) ||
       overlaps(out, ob, l_p, rows * sizeof(float)))
     return LOSA_ERR_INVALID_ARG;
+  if (q_ref_out) {  // the reference is rewritten: it may alias nothing else
+    const size_t lb = rows * sizeof(float);
+    if (overlaps(q_ref_out, qb, q_cur, qb) || overlaps(q_ref_out, qb, o_p, ob) ||
+        overlaps(q_ref_out, qb, l_p, lb) || overlaps(q_ref_out, qb, out, ob) ||
+        (out_lse && overlaps(q_ref_out, qb, out_lse, lb)))
+      return LOSA_ERR_INVALID_ARG;
+  }
   if (d.S * d.Hkv > 65535) return LOSA_ERR_UNSUPPORTED;
-  return losa::launch_fused_step(d, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk,
-                                 o_p, l_p, out, out_lse, active_idx, page_idx, union_count,
-                                 workspace, static_cast<cudaStream_t>(stream));
+  return launch_fused_step(d, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
+                           l_p, out, out_lse, active_idx, page_idx, union_count, workspace,
+                           static_cast<cudaStream_t>(stream), q_ref_out);
+}
+
+}  // namespace
+
+extern "C" int losa_step(const losa_shape* shape, const void* q_cur, const void* q_prev,
+                         const void* k_prefix, const void* v_prefix, const void* page_meta,
+                         const void* k_blk, const void* v_blk, float* o_p, float* l_p,
+                         float* out, float* out_lse, int32_t* active_idx, int32_t* page_idx,
+                         int32_t* union_count, void* workspace, size_t ws_bytes, void* stream) {
+  return step_common(shape, q_cur, q_prev, nullptr, k_prefix, v_prefix, page_meta, k_blk, v_blk,
+                     o_p, l_p, out, out_lse, active_idx, page_idx, union_count, workspace,
+                     ws_bytes, stream);
+}
+
+extern "C" int losa_step_ref(const losa_shape* shape, const void* q_cur, void* q_ref,
+                             const void* k_prefix, const void* v_prefix, const void* page_meta,
+                             const void* k_blk, const void* v_blk, float* o_p, float* l_p,
+                             float* out, float* out_lse, int32_t* active_idx, int32_t* page_idx,
+                             int32_t* union_count, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  if (!q_ref) return LOSA_ERR_INVALID_ARG;
+  return step_common(shape, q_cur, q_ref, q_ref, k_prefix, v_prefix, page_meta, k_blk, v_blk,
+                     o_p, l_p, out, out_lse, active_idx, page_idx, union_count, workspace,
+                     ws_bytes, stream);
 }

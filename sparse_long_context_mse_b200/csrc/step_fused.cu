@@ -987,6 +987,7 @@ struct GatherParams {
   float* out_lse;
   int32_t* page_idx;
   int32_t* union_count;
+  void* qref;       // drift-safe locality: active rows' q_cur written here (may be null)
   const int32_t* act_g;
   const unsigned long long* cand;
   float* part_g;    // workspace [S*Hkv][CL][R][kPartStride]: every CTA's row partials
@@ -1331,6 +1332,23 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
       }
     }
     bar_sync(1, kThreads);
+    if (d.attend_union && sel) {
+      // every active row attends to the whole union: every row's bit on each
+      // of this CTA's pages, every CTA holding union pages in every row's
+      // combine
+      const int nlp = min(*s_nlp, prm.max_lp);
+#pragma unroll 1
+      for (int e = tid; e < nlp * d.MW; e += kThreads) {
+        const int nb = min(32, R - 32 * (e % d.MW));
+        masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+      }
+      int U = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) U += s_wsum[w];
+      const uint32_t own = U >= CL ? (CL >= 32 ? 0xffffffffu : (1u << CL) - 1u) : (1u << U) - 1u;
+#pragma unroll 1
+      for (int r = tid; r < R; r += kThreads) rmask[r] = own;
+    }
     issue_batch(0, min(*s_nlp, prm.max_lp), tid, kThreads);
     cp_async_wait<0>();  // this half's copies: the gathered pages
   } else {
@@ -1358,6 +1376,16 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
       }
     }
     bar_sync(2, kThreads);
+    if (prm.qref) {  // drift-safe locality: this CTA's active rows' reference := q_cur
+      const char* qg = static_cast<const char*>(prm.qc) + grow0 * rowb;
+      char* qr = static_cast<char*>(prm.qref) + grow0 * rowb;
+#pragma unroll 1
+      for (int e = htid; e < n_oa * cpr; e += kThreads) {
+        const int j = e / cpr, c = e - j * cpr;
+        const size_t o = static_cast<size_t>(sfx_tok[j]) * rowb + c * 16;
+        *reinterpret_cast<uint4*>(qr + o) = *reinterpret_cast<const uint4*>(qg + o);
+      }
+    }
     // ---- cp.async group 1: queries of the suffix rows and of the active
     // rows, cached state of the stable suffix rows
     {
@@ -1892,7 +1920,7 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
                       const void* v_prefix, const void* page_meta, const void* k_blk,
                       const void* v_blk, float* o_p, float* l_p, float* out, float* out_lse,
                       int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
-                      void* workspace, cudaStream_t st) {
+                      void* workspace, cudaStream_t st, void* q_ref_out) {
   int max_dyn = 0;
   int rc = ensure_attributes(&max_dyn);
   if (rc != LOSA_OK) return rc;
@@ -1938,6 +1966,7 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   gp.out = out;
   gp.out_lse = out_lse;
   gp.page_idx = page_idx;
+  gp.qref = q_ref_out;
   gp.union_count = union_count;
   gp.act_g = act;
   gp.cand = cand;

@@ -56,8 +56,10 @@ def unswizzle_page_meta(sh, page_meta):
 
 
 def oshape(sh):
+    flags = oracle.ATTEND_UNION if sh.flags & api.LOSA_STEP_ATTEND_UNION else 0
     return oracle.shape(sh.num_seqs, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, sh.prefix_len,
-                        sh.page_size, sh.block_size, sh.n_active, sh.token_budget, sh.scale)
+                        sh.page_size, sh.block_size, sh.n_active, sh.token_budget, sh.scale,
+                        flags)
 
 
 def maxabs(a, b):
@@ -146,8 +148,10 @@ def gpu_dense(sh, q, K, V, kb, vb, ws=None):
     return {"o_p": o_p, "l_p": l_p, "out": out, "lse": lse}
 
 
-def gpu_step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, ws=None):
-    """One step; o_p/l_p are updated in place (pass clones to keep inputs)."""
+def gpu_step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, ws=None, q_ref=None):
+    """One step; o_p/l_p are updated in place (pass clones to keep inputs).
+    With ``q_ref`` (drift-safe locality) ``qp`` is ignored and ``q_ref`` is
+    the in/out reference."""
     rows = (sh.num_seqs, sh.n_q_heads, sh.block_size)
     out = torch.empty(*rows, sh.head_dim, device=DEV)
     lse = torch.empty(*rows, device=DEV)
@@ -157,7 +161,10 @@ def gpu_step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, ws=None):
     uc = torch.full((sh.num_seqs, sh.n_kv_heads), -7, dtype=torch.int32, device=DEV)
     if ws is None:
         ws = api.alloc_workspace(sh, api.LOSA_WS_STEP, DEV)
-    api.step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, out, lse, ws, act, pidx, uc)
+    if q_ref is None:
+        api.step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, out, lse, ws, act, pidx, uc)
+    else:
+        api.step_ref(sh, qc, q_ref, K, V, meta, kb, vb, o_p, l_p, out, lse, ws, act, pidx, uc)
     return {"out": out, "lse": lse, "o_p": o_p, "l_p": l_p, "active_idx": act,
             "page_idx": pidx, "union_count": uc, "ws": ws}
 
@@ -272,13 +279,15 @@ def check_step_sampled(c, step_t, res, cache_in, kmin, kmax, n_stable=24, rng_se
     return err, near
 
 
-def check_step_full(c, step_t, res, cache_o_in, kmin, kmax, tag=""):
+def check_step_full(c, step_t, res, cache_o_in, kmin, kmax, tag="", qp=None):
     """Compare every output of one GPU step with the oracle's full step run on
     the oracle's own cache (``cache_o_in``: dict from oracle.dense_prefix or a
-    previous oracle.step)."""
+    previous oracle.step).  ``qp``: the locality reference (default: the
+    previous step's queries)."""
     sh = c.sh
     osh = oshape(sh)
-    r = oracle.step(osh, c.q[step_t], c.q[step_t - 1], c.host("K"), c.host("V"), kmin, kmax,
+    qp = c.q[step_t - 1] if qp is None else qp
+    r = oracle.step(osh, c.q[step_t], qp, c.host("K"), c.host("V"), kmin, kmax,
                     c.kb[step_t], c.vb[step_t], cache_o_in["o_p"], cache_o_in["l_p"],
                     want_bound=sh.pages_per_row < sh.n_pages)
     act_g = res["active_idx"].cpu().numpy()

@@ -139,6 +139,36 @@ def test_pointer_validation(L):
     assert L.losa_step(None, *_step_args(base), ws_n, None) == api.LOSA_ERR_INVALID_ARG
 
 
+def test_step_flags_validation(L):
+    # the union variant is a legal step shape; an unknown bit is refused
+    # before anything is launched
+    assert api.workspace_size(S(flags=api.LOSA_STEP_ATTEND_UNION), api.LOSA_WS_STEP) > 0
+    bad = S(flags=2)
+    assert api.workspace_size(bad, api.LOSA_WS_STEP) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.losa_step(ctypes.byref(bad), *([fake] * 10), None, None, None, None, fake,
+                       1 << 40, None) == api.LOSA_ERR_INVALID_ARG
+
+
+def test_step_ref_pointer_validation(L):
+    # losa_step_ref rewrites q_ref: null, or aliasing any output or q_cur, is
+    # refused before anything is launched
+    sh = S()
+    ws_n = api.workspace_size(sh, api.LOSA_WS_STEP)
+    base = [0x100000 * (i + 1) for i in range(10)] + [None, None, None, None, 0x7f0000000000]
+
+    def call(ptrs):
+        return L.losa_step_ref(ctypes.byref(sh), *_step_args(ptrs), ws_n, None)
+
+    for i, other in ((1, None), (1, 0), (1, 7), (1, 8), (1, 9)):
+        p = list(base)
+        p[i] = None if other is None else base[other]
+        assert call(p) == api.LOSA_ERR_INVALID_ARG, other
+    p = list(base)
+    p[10] = base[1]                      # out_lse aliases q_ref
+    assert call(p) == api.LOSA_ERR_INVALID_ARG
+
+
 def test_dense_pointer_validation(L):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)

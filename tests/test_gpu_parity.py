@@ -115,6 +115,71 @@ def test_step_sampled(n, layer):
 
 
 # ---------------------------------------------------------------------------
+# step variants
+# ---------------------------------------------------------------------------
+def _union_case(name):
+    if name == "cfg0":
+        return Case(synth.config(0))
+    if name == "cfg1":
+        return Case(synth.config(1))
+    if name == "groups_bf16":
+        return random_case(2, 8, 2, 1000, 16, 4, 64, "bf16", seed=5)
+    return random_case(1, 4, 1, 777, 8, 3, 48, "f32", seed=6)
+
+
+@pytest.mark.parametrize("name", ["cfg0", "cfg1", "groups_bf16", "ragged_f32"])
+def test_step_attend_union(name):
+    """Every active row attends to its group's whole page union: the
+    selection is the plain step's, o_p/L_p/out are the oracle's union
+    attention."""
+    c = _union_case(name)
+    c.sh.flags = api.LOSA_STEP_ATTEND_UNION
+    sh = c.sh
+    meta = gpu_meta(sh, c.K)
+    kmin, kmax = check_meta(sh, meta, c.host("K"))
+    cache_g = gpu_dense(sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])
+    cache_o = oracle.dense_prefix(oshape(sh), c.q[0], c.host("K"), c.host("V"), c.kb[0], c.vb[0])
+    res = gpu_step(sh, c.q[1], c.q[0], c.K, c.V, meta, c.kb[1], c.vb[1],
+                   cache_g["o_p"].clone(), cache_g["l_p"].clone())
+    ref, _, _ = check_step_full(c, 1, res, cache_o, kmin, kmax, tag=f"union {name}")
+    # the union rows differ from the plain step's wherever the union added pages
+    sh.flags = 0
+    plain = oracle.step_forced(oshape(sh), c.q[1], c.host("K"), c.host("V"), c.kb[1], c.vb[1],
+                               res["active_idx"].cpu().numpy(), res["page_idx"].cpu().numpy(),
+                               cache_o["o_p"], cache_o["l_p"])
+    if sh.n_active * sh.group > 1 and sh.pages_per_row < sh.n_pages:
+        assert maxabs(ref["l_p"], plain["l_p"]) > 10 * TOL, "the case does not exercise the union"
+    assert api.read_device_status(res["ws"]) == api.LOSA_OK
+
+
+@pytest.mark.parametrize("n", [0, 1])
+def test_step_ref_chain(n):
+    """Drift-safe locality over a denoising chain: each step scores against
+    the reference queries, the GPU's reference is rewritten exactly for the
+    active rows, and every output matches the oracle's drift-safe step."""
+    cfg = synth.config(n)
+    T = 4
+    c = Case(cfg, steps=T)
+    sh = c.sh
+    meta = gpu_meta(sh, c.K)
+    kmin, kmax = check_meta(sh, meta, c.host("K"))
+    cache_g = gpu_dense(sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])
+    cache_o = oracle.dense_prefix(oshape(sh), c.q[0], c.host("K"), c.host("V"), c.kb[0], c.vb[0])
+    q_ref_g = c.q[0].clone()
+    q_ref_o = oracle.f32(c.q[0])
+    ws = api.alloc_workspace(sh, api.LOSA_WS_STEP, DEV)
+    for t in range(1, T):
+        res = gpu_step(sh, c.q[t], None, c.K, c.V, meta, c.kb[t], c.vb[t], cache_g["o_p"],
+                       cache_g["l_p"], ws=ws, q_ref=q_ref_g)
+        ref, _, _ = check_step_full(c, t, res, cache_o, kmin, kmax, tag=f"ref{n} t{t}",
+                                    qp=q_ref_o)
+        q_ref_o = oracle.refresh_ref(oshape(sh), c.q[t], res["active_idx"].cpu().numpy(), q_ref_o)
+        assert np.array_equal(oracle.f32(q_ref_g).view(np.uint32), q_ref_o.view(np.uint32)), t
+        cache_o = {"o_p": ref["o_p"], "l_p": ref["l_p"]}
+    assert api.read_device_status(ws) == api.LOSA_OK
+
+
+# ---------------------------------------------------------------------------
 # denoising chains: step 1 dense, then LoSA steps, cache carried through
 # ---------------------------------------------------------------------------
 def test_chain_full_cfg1():
