@@ -187,21 +187,31 @@ __global__ void __launch_bounds__(256)
 // its half row of S; the online softmax runs in base 2 (the halves exchange
 // row maxima through shared memory) against a reference max that moves only
 // when the row max grows by more than 2^8 (O and l are then rescaled in
-// TMEM); P goes to one of two shared-memory buffers as a bf16 high part and
-// a bf16 remainder, so the weights keep ~16 bits; then O += P_hi V + P_lo V
-// (M=128, N=128, K=64, V the MN-major operand).  A tile waits only for the
+// TMEM); P goes to one of two shared-memory buffers in bf16, and the row sum
+// l adds the same rounded weights, so the output is an exactly normalised
+// average of the values under weights perturbed by at most 2^-9 relative;
+// then O += P V (M=128, N=128, K=64, V the MN-major operand).  A tile waits only for the
 // P V of two tiles back.  Every wait is bounded; a wait that gives up
 // records LOSA_ERR_DEVICE_TIMEOUT.
 // ---------------------------------------------------------------------------
 constexpr int kUKeys = 64;                          // keys per tile
-constexpr int kUKst = 4;                            // K ring stages
-constexpr int kUVst = 3;                            // V ring stages
 constexpr int kUTile = kUKeys * kD * 2;             // 16 KB: one K (or V) tile
-constexpr int kUQ = 128 * kD * 2;                   // 32 KB: the query tile
-constexpr int kUP = 128 * kUKeys * 2;               // 16 KB: one P part
-constexpr int kUBars = 1 + 2 + 2 + kUKst + kUVst + 2;  // Q, S[2], O[2], K[4], V[3], P[2]
-constexpr int kUSmem = 1024 + kUQ + (kUKst + kUVst) * kUTile + 4 * kUP + 1024 + kUBars * 8 + 16;
 constexpr uint32_t kUCols = 256;                    // TMEM: S [0, 128) (two tiles), O [128, 256)
+
+// Shared-memory plan per MMA row count MR (64 or 128): the query tile and the
+// P parts scale with MR; what a 64-row group saves goes to a deeper V ring,
+// so V tiles are requested several tiles before their P V MMAs.
+template <int MR>
+struct UPlan {
+  static constexpr int kst = 4;                    // K ring stages
+  static constexpr int vst = MR == 64 ? 6 : 5;     // V ring stages
+  static constexpr int qbytes = MR * kD * 2;       // the query tile
+  static constexpr int pbytes = MR * kUKeys * 2;   // one P buffer
+  static constexpr int nbars = 1 + 2 + 2 + kst + vst + 2;  // Q, S[2], O[2], K[kst], V[vst], P[2]
+  static constexpr int smem = 1024 + qbytes + (kst + vst) * kUTile + 2 * pbytes + 1024 +
+                              nbars * 8 + 16;
+};
+static_assert(UPlan<64>::smem <= 232448 && UPlan<128>::smem <= 232448, "dense plan > 227 KB");
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
@@ -218,6 +228,9 @@ __global__ void __launch_bounds__(288, 1)
                       const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, float* __restrict__ part,
                       int* __restrict__ status, Dims d) {
+  using C = UPlan<MR>;
+  constexpr int kUKst = C::kst, kUVst = C::vst, kUQ = C::qbytes, kUP = C::pbytes;
+  constexpr int kUBars = C::nbars;
   extern __shared__ char dsm_raw[];
   // 1024-byte alignment for the swizzled tiles
   char* dsm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
@@ -225,8 +238,8 @@ __global__ void __launch_bounds__(288, 1)
   char* qs = dsm;                                     // [MR rows], 2 atoms of MR x 128 B
   char* kring = qs + kUQ;                             // kUKst K tiles (2 atoms of 8 KB)
   char* vring = kring + kUKst * kUTile;               // kUVst V tiles
-  char* pbuf = vring + kUVst * kUTile;                // [2][hi, lo] P parts
-  float* xmax = reinterpret_cast<float*>(pbuf + 4 * kUP);     // [2][128]: the halves' row maxima
+  char* pbuf = vring + kUVst * kUTile;                // [2] P buffers
+  float* xmax = reinterpret_cast<float*>(pbuf + 2 * kUP);     // [2][128]: the halves' row maxima
   uint64_t* bars = reinterpret_cast<uint64_t*>(xmax + 256);
   uint64_t* bQ = bars;
   uint64_t* bS = bars + 1;     // [2] S buffer ready
@@ -296,7 +309,8 @@ __global__ void __launch_bounds__(288, 1)
       tma_load_2d(qs, &qmap, 0, q_row0, bQ);
       tma_load_2d(qs + MR * 128, &qmap, 64, q_row0, bQ);
       for (int t = 0; t < min(n, kUKst); ++t) load_k(t);
-      for (int t = 0; t < min(n, kUVst); ++t) load_v(t);
+      int vnext = 0;  // the next V tile to request
+      while (vnext < min(n, kUVst)) load_v(vnext++);
       ok = ok && mbar_wait(bQ, 0) && mbar_wait(&bK[0], 0);
       issue_s(0);
 #pragma unroll 1
@@ -308,25 +322,147 @@ __global__ void __launch_bounds__(288, 1)
         ok = ok && mbar_wait(&bS[t & 1], (t >> 1) & 1);
         if (t + kUKst < n) load_k(t + kUKst);  // tile t's K stage is free again
         // P V of two tiles back has finished (before this barrier completes
-        // again): V stage (t + 1) % kUVst is free
+        // again): the V stages of tiles <= t - 2 are free
         if (t >= 2) {
           ok = ok && mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1);
-          if (t + 1 < n) load_v(t + 1);
+          while (vnext < n && vnext <= t - 2 + kUVst) load_v(vnext++);
         }
         ok = ok && mbar_wait(&bP[t & 1], (t >> 1) & 1) && mbar_wait(&bV[t % kUVst], (t / kUVst) & 1);
         tc_fence_after();
         const uint64_t dv = umma_desc(su32(vring + (t % kUVst) * kUTile), kUKeys * 128, 1024);
+        const uint64_t dp = umma_desc(su32(pbuf + (t & 1) * kUP), 16, 1024);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint64_t dp = umma_desc(su32(pbuf + ((t & 1) * 2 + h) * kUP), 16, 1024);
-#pragma unroll
-          for (int ks = 0; ks < kUKeys / 16; ++ks)
-            umma_bf16(tO, dp + ((ks * 32) >> 4), dv + ((ks * 16 * 128) >> 4), idesc_o,
-                      (t > 0 || h > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kUKeys / 16; ++ks)
+          umma_bf16(tO, dp + ((ks * 32) >> 4), dv + ((ks * 16 * 128) >> 4), idesc_o,
+                    (t > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&bO[t & 1]);
       }
       if (!ok) *s_fail = 1;
+    }
+  } else if constexpr (MR == 64) {
+    // ---- softmax warps, 64 accumulator rows: rows 16q .. 16q + 15 of
+    // sub-partition q = w % 4 live in TMEM lanes 32q .. 32q + 15; the 16x256b
+    // fragment gives thread t rows 16q + t/4 and 16q + t/4 + 8, so every
+    // lane holds real scores.  Warp w takes key half w / 4 of each S tile
+    // (32 keys: 8 per row and thread) and the same half of O's columns.
+    const int q4 = warp & 3, half = warp >> 2, tq = lane & 3;
+    const int rr[2] = {16 * q4 + (lane >> 2), 16 * q4 + (lane >> 2) + 8};
+    const bool valid[2] = {rr[0] < rows, rr[1] < rows};
+    const bool busy = 16 * q4 < rows;  // (warp-uniform) some row of this warp is real
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const float sl2 = d.scale_log2;
+    float mref[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+#pragma unroll 1
+    for (int t = 0; t < n; ++t) {
+      ok = ok && mbar_wait(&bS[t & 1], (t >> 1) & 1);
+      // the P buffers of this parity are free once P V of two tiles back is done
+      ok = ok && (t < 2 || mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1));
+      tc_fence_after();
+      // register r: row rr[(r >> 1) & 1], key kb + 8 (r >> 2) + 2 tq + (r & 1)
+      const int kb = key0 + t * kUKeys + half * 32;
+      float sv[16];
+      float mx[2] = {-INFINITY, -INFINITY};
+      if (busy) {
+        tmem_ld16x256_x4(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int key = kb + 8 * (r >> 2) + 2 * tq + (r & 1);
+          sv[r] = key < key1 ? sv[r] * sl2 : -INFINITY;
+          mx[(r >> 1) & 1] = fmaxf(mx[(r >> 1) & 1], sv[r]);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {  // the row's four threads
+          mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+          mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+        }
+        if (tq == 0) {
+          xmax[half * 128 + rr[0]] = mx[0];
+          xmax[half * 128 + rr[1]] = mx[1];
+        }
+      }
+      bar_sync(1, 256);  // both halves' maxima
+      char* pb = pbuf + (t & 1) * kUP;
+      if (busy) {
+        bool grow[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          mx[i] = fmaxf(xmax[rr[i]], xmax[128 + rr[i]]);
+          // the same decision in both halves of the row; padding rows never move
+          grow[i] = valid[i] && mx[i] > mref[i] + 8.f;
+        }
+        if (__any_sync(0xffffffffu, grow[0] || grow[1])) {  // tcgen05.ld/st are warp-wide
+          float alpha[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float nref = grow[i] ? mx[i] : mref[i];
+            alpha[i] = grow[i] ? exp2f(mref[i] - nref) : 1.f;  // 0 while nothing is accumulated
+            lrow[i] *= alpha[i];
+            mref[i] = nref;
+          }
+          if (t > 0) {
+            // O holds every P V up to tile t - 1
+            ok = ok && mbar_wait(&bO[(t - 1) & 1], ((t - 1) >> 1) & 1);
+            tc_fence_after();
+#pragma unroll 1
+            for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+              float v[16];
+              tmem_ld16x256_x4(tO + lane_off + c0, v);
+#pragma unroll
+              for (int r = 0; r < 16; ++r) v[r] *= alpha[(r >> 1) & 1];
+              tmem_st16x256_x4(tO + lane_off + c0, v);
+            }
+          }
+        }
+        // P = 2^(s - mref) <= 2^8 in bf16, [64 rows][64 keys] K-major,
+        // swizzled, one 4-byte store per key pair; l adds the rounded weights
+#pragma unroll
+        for (int r = 0; r < 16; r += 2) {
+          const int i = (r >> 1) & 1;
+          const uint32_t pw = pack_bf16x2(ex2_approx(sv[r] - mref[i]), ex2_approx(sv[r + 1] - mref[i]));
+          lrow[i] += __uint_as_float(pw << 16) + __uint_as_float(pw & 0xffff0000u);
+          *reinterpret_cast<uint32_t*>(pb + sw128_off(rr[i], half * 32 + 8 * (r >> 2) + 2 * tq, MR)) = pw;
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bP[t & 1]);
+    }
+    ok = ok && mbar_wait(&bO[(n - 1) & 1], ((n - 1) >> 1) & 1);
+    tc_fence_after();
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) *s_fail = 1;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {  // the row's four threads' shares of this half's sum
+      lrow[i] += __shfl_xor_sync(0xffffffffu, lrow[i], 1);
+      lrow[i] += __shfl_xor_sync(0xffffffffu, lrow[i], 2);
+    }
+    if (busy && half == 1 && tq == 0) {  // the second half's row sums
+      xmax[rr[0]] = lrow[0];
+      xmax[rr[1]] = lrow[1];
+    }
+    bar_sync(1, 256);
+    if (!*s_fail && busy) {
+      float* dst0 = part + ((static_cast<size_t>(sg) * d.nsplit + split) * rows) * kPartStride;
+#pragma unroll 1
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+        float v[16];
+        tmem_ld16x256_x4(tO + lane_off + c0, v);
+#pragma unroll
+        for (int r = 0; r < 16; r += 2) {
+          const int i = (r >> 1) & 1;
+          if (valid[i])
+            *reinterpret_cast<float2*>(dst0 + rr[i] * kPartStride + 4 + c0 + 8 * (r >> 2) +
+                                       2 * tq) = make_float2(v[r], v[r + 1]);
+        }
+      }
+      if (half == 0 && tq == 0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (!valid[i]) continue;
+          float* dst = dst0 + rr[i] * kPartStride;
+          dst[0] = mref[i];
+          dst[1] = lrow[i] + xmax[rr[i]];
+        }
+      }
     }
   } else {
     // ---- softmax warps: warp w reads TMEM lanes 32 (w % 4) .. (its
@@ -367,8 +503,7 @@ __global__ void __launch_bounds__(288, 1)
         if (lane < RPW) xmax[half * 128 + row] = mx;
       }
       bar_sync(1, 256);  // both halves' maxima
-      char* phi = pbuf + (t & 1) * 2 * kUP;
-      char* plo = phi + kUP;
+      char* pb = pbuf + (t & 1) * kUP;
       if (busy) {
         if (lane < RPW) mx = fmaxf(xmax[row], xmax[128 + row]);
         // the same decision in both halves of the row; padding lanes never move
@@ -392,25 +527,20 @@ __global__ void __launch_bounds__(288, 1)
           }
           mref = nref;
         }
-        // P = 2^(s - mref) <= 2^8: high part and remainder, [128 rows][64
-        // keys] K-major, swizzled
+        // P = 2^(s - mref) <= 2^8 in bf16, [128 rows][64 keys] K-major,
+        // swizzled; l adds the rounded weights
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t hi[4], lo[4];
+          uint32_t pw[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float p0 = ex2_approx(sv[c8 * 8 + 2 * u] - mref);
-            const float p1 = ex2_approx(sv[c8 * 8 + 2 * u + 1] - mref);
-            lrow += p0 + p1;
-            hi[u] = pack_bf16x2(p0, p1);
-            const float h0 = __uint_as_float(hi[u] << 16), h1 = __uint_as_float(hi[u] & 0xffff0000u);
-            lo[u] = pack_bf16x2(p0 - h0, p1 - h1);
+            pw[u] = pack_bf16x2(ex2_approx(sv[c8 * 8 + 2 * u] - mref),
+                                ex2_approx(sv[c8 * 8 + 2 * u + 1] - mref));
+            lrow += __uint_as_float(pw[u] << 16) + __uint_as_float(pw[u] & 0xffff0000u);
           }
-          if (lane < RPW) {
-            const uint32_t o = sw128_off(row, half * 32 + c8 * 8, MR);
-            *reinterpret_cast<uint4*>(phi + o) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(plo + o) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-          }
+          if (lane < RPW)
+            *reinterpret_cast<uint4*>(pb + sw128_off(row, half * 32 + c8 * 8, MR)) =
+                make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
       }
       fence_async_smem();
@@ -500,11 +630,11 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-      cudaError_t e0 = cudaFuncSetAttribute(dense_umma_kernel<64>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
+      cudaError_t e0 = cudaFuncSetAttribute(
+          dense_umma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, UPlan<64>::smem);
       if (e0 == cudaSuccess)
         e0 = cudaFuncSetAttribute(dense_umma_kernel<128>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, UPlan<128>::smem);
       if (e0 != cudaSuccess) return record_cuda_error(e0);
       attr_done[dev] = true;
     }
@@ -516,11 +646,11 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
         make_tmap(&vmap, v_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK)
       return record_cuda_error(cudaErrorInvalidValue);
     if (m64)
-      dense_umma_kernel<64><<<dim3(d.nsplit, d.S * d.Hkv), 288, kUSmem, st>>>(qmap, kmap, vmap,
-                                                                             part, status, d);
+      dense_umma_kernel<64><<<dim3(d.nsplit, d.S * d.Hkv), 288, UPlan<64>::smem, st>>>(
+          qmap, kmap, vmap, part, status, d);
     else
-      dense_umma_kernel<128><<<dim3(d.nsplit, d.S * d.Hkv), 288, kUSmem, st>>>(qmap, kmap, vmap,
-                                                                              part, status, d);
+      dense_umma_kernel<128><<<dim3(d.nsplit, d.S * d.Hkv), 288, UPlan<128>::smem, st>>>(
+          qmap, kmap, vmap, part, status, d);
   } else {
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);
