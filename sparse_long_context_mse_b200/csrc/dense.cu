@@ -194,17 +194,18 @@ __global__ void __launch_bounds__(256)
 // P V of two tiles back.  Every wait is bounded; a wait that gives up
 // records LOSA_ERR_DEVICE_TIMEOUT.
 // ---------------------------------------------------------------------------
-constexpr int kUKeys = 64;                          // keys per tile
-constexpr int kUTile = kUKeys * kD * 2;             // 16 KB: one K (or V) tile
-constexpr uint32_t kUCols = 256;                    // TMEM: S [0, 128) (two tiles), O [128, 256)
+constexpr int kUKeys = 128;                         // keys per tile (the S MMA's N)
+constexpr int kUHalf = kUKeys / 2;                  // keys of a tile per softmax warp
+constexpr int kUTile = kUKeys * kD * 2;             // 32 KB: one K (or V) tile
+constexpr uint32_t kUCols = 512;                    // TMEM: S [0, 256) (two tiles), O [256, 384)
 
 // Shared-memory plan per MMA row count MR (64 or 128): the query tile and the
-// P parts scale with MR; what a 64-row group saves goes to a deeper V ring,
-// so V tiles are requested several tiles before their P V MMAs.
+// P buffers scale with MR; what a 64-row group saves goes to a deeper V ring,
+// so V tiles are requested a tile before their P V MMAs.
 template <int MR>
 struct UPlan {
-  static constexpr int kst = 4;                    // K ring stages
-  static constexpr int vst = MR == 64 ? 6 : 5;     // V ring stages
+  static constexpr int kst = 2;                    // K ring stages
+  static constexpr int vst = MR == 64 ? 3 : 2;     // V ring stages
   static constexpr int qbytes = MR * kD * 2;       // the query tile
   static constexpr int pbytes = MR * kUKeys * 2;   // one P buffer
   static constexpr int nbars = 1 + 2 + 2 + kst + vst + 2;  // Q, S[2], O[2], K[kst], V[vst], P[2]
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(288, 1)
   char* dsm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   // MR = MMA rows (64 or 128): the group's query rows, zero-padded
   char* qs = dsm;                                     // [MR rows], 2 atoms of MR x 128 B
-  char* kring = qs + kUQ;                             // kUKst K tiles (2 atoms of 8 KB)
+  char* kring = qs + kUQ;                             // kUKst K tiles (2 atoms of 16 KB)
   char* vring = kring + kUKst * kUTile;               // kUVst V tiles
   char* pbuf = vring + kUVst * kUTile;                // [2] P buffers
   float* xmax = reinterpret_cast<float*>(pbuf + 2 * kUP);     // [2][128]: the halves' row maxima
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(288, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  const uint32_t tO = tbase + 128;  // S tiles: columns [0, 64) and [64, 128)
+  const uint32_t tO = tbase + 2 * kUKeys;  // S tiles: columns [0, 128) and [128, 256)
   bool ok = true;
 
   if (warp == 8) {
@@ -332,9 +333,9 @@ __global__ void __launch_bounds__(288, 1)
         const uint64_t dv = umma_desc(su32(vring + (t % kUVst) * kUTile), kUKeys * 128, 1024);
         const uint64_t dp = umma_desc(su32(pbuf + (t & 1) * kUP), 16, 1024);
 #pragma unroll
-        for (int ks = 0; ks < kUKeys / 16; ++ks)
-          umma_bf16(tO, dp + ((ks * 32) >> 4), dv + ((ks * 16 * 128) >> 4), idesc_o,
-                    (t > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kUKeys / 16; ++ks)  // P: two K-major atoms of 64 keys
+          umma_bf16(tO, dp + (((ks >> 2) * (MR * 128) + (ks & 3) * 32) >> 4),
+                    dv + ((ks * 16 * 128) >> 4), idesc_o, (t > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&bO[t & 1]);
       }
       if (!ok) *s_fail = 1;
@@ -344,7 +345,8 @@ __global__ void __launch_bounds__(288, 1)
     // sub-partition q = w % 4 live in TMEM lanes 32q .. 32q + 15; the 16x256b
     // fragment gives thread t rows 16q + t/4 and 16q + t/4 + 8, so every
     // lane holds real scores.  Warp w takes key half w / 4 of each S tile
-    // (32 keys: 8 per row and thread) and the same half of O's columns.
+    // (64 keys: 16 per row and thread, two 32-column blocks) and the same
+    // half of O's columns.
     const int q4 = warp & 3, half = warp >> 2, tq = lane & 3;
     const int rr[2] = {16 * q4 + (lane >> 2), 16 * q4 + (lane >> 2) + 8};
     const bool valid[2] = {rr[0] < rows, rr[1] < rows};
@@ -358,17 +360,21 @@ __global__ void __launch_bounds__(288, 1)
       // the P buffers of this parity are free once P V of two tiles back is done
       ok = ok && (t < 2 || mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1));
       tc_fence_after();
-      // register r: row rr[(r >> 1) & 1], key kb + 8 (r >> 2) + 2 tq + (r & 1)
-      const int kb = key0 + t * kUKeys + half * 32;
-      float sv[16];
+      // block b, register r: row rr[(r >> 1) & 1], key kb + 32 b + 8 (r >> 2)
+      // + 2 tq + (r & 1)
+      const int kb = key0 + t * kUKeys + half * kUHalf;
+      float sv[2][16];
       float mx[2] = {-INFINITY, -INFINITY};
       if (busy) {
-        tmem_ld16x256_x4(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-          const int key = kb + 8 * (r >> 2) + 2 * tq + (r & 1);
-          sv[r] = key < key1 ? sv[r] * sl2 : -INFINITY;
-          mx[(r >> 1) & 1] = fmaxf(mx[(r >> 1) & 1], sv[r]);
+        for (int b = 0; b < 2; ++b) {
+          tmem_ld16x256_x4(tbase + (t & 1) * kUKeys + half * kUHalf + 32 * b + lane_off, sv[b]);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const int key = kb + 32 * b + 8 * (r >> 2) + 2 * tq + (r & 1);
+            sv[b][r] = key < key1 ? sv[b][r] * sl2 : -INFINITY;
+            mx[(r >> 1) & 1] = fmaxf(mx[(r >> 1) & 1], sv[b][r]);
+          }
         }
 #pragma unroll
         for (int i = 0; i < 2; ++i) {  // the row's four threads
@@ -413,14 +419,20 @@ __global__ void __launch_bounds__(288, 1)
             }
           }
         }
-        // P = 2^(s - mref) <= 2^8 in bf16, [64 rows][64 keys] K-major,
-        // swizzled, one 4-byte store per key pair; l adds the rounded weights
+        // P = 2^(s - mref) <= 2^8 in bf16, [64 rows][128 keys] K-major (two
+        // atoms of 64 keys), swizzled, one 4-byte store per key pair; l adds
+        // the rounded weights
 #pragma unroll
-        for (int r = 0; r < 16; r += 2) {
-          const int i = (r >> 1) & 1;
-          const uint32_t pw = pack_bf16x2(ex2_approx(sv[r] - mref[i]), ex2_approx(sv[r + 1] - mref[i]));
-          lrow[i] += __uint_as_float(pw << 16) + __uint_as_float(pw & 0xffff0000u);
-          *reinterpret_cast<uint32_t*>(pb + sw128_off(rr[i], half * 32 + 8 * (r >> 2) + 2 * tq, MR)) = pw;
+        for (int b = 0; b < 2; ++b) {
+#pragma unroll
+          for (int r = 0; r < 16; r += 2) {
+            const int i = (r >> 1) & 1;
+            const uint32_t pw = pack_bf16x2(ex2_approx(sv[b][r] - mref[i]),
+                                            ex2_approx(sv[b][r + 1] - mref[i]));
+            lrow[i] += __uint_as_float(pw << 16) + __uint_as_float(pw & 0xffff0000u);
+            *reinterpret_cast<uint32_t*>(
+                pb + sw128_off(rr[i], half * kUHalf + 32 * b + 8 * (r >> 2) + 2 * tq, MR)) = pw;
+          }
         }
       }
       fence_async_smem();
@@ -482,22 +494,17 @@ __global__ void __launch_bounds__(288, 1)
       // the P buffers of this parity are free once P V of two tiles back is done
       ok = ok && (t < 2 || mbar_wait(&bO[t & 1], ((t - 2) >> 1) & 1));
       tc_fence_after();
-      const int kb = key0 + t * kUKeys + half * 32;
-      float sv[32];
+      const int kb = key0 + t * kUKeys + half * kUHalf;
+      float sv[2][32];
       float mx = -INFINITY;
       if (busy) {
-        tmem_ld32(tbase + (t & 1) * kUKeys + half * 32 + lane_off, sv);
-        if (kb + 32 <= key1) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          tmem_ld32(tbase + (t & 1) * kUKeys + half * kUHalf + 32 * b + lane_off, sv[b]);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            sv[i] *= sl2;
-            mx = fmaxf(mx, sv[i]);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            sv[i] = kb + i < key1 ? sv[i] * sl2 : -INFINITY;
-            mx = fmaxf(mx, sv[i]);
+            sv[b][i] = kb + 32 * b + i < key1 ? sv[b][i] * sl2 : -INFINITY;
+            mx = fmaxf(mx, sv[b][i]);
           }
         }
         if (lane < RPW) xmax[half * 128 + row] = mx;
@@ -527,19 +534,19 @@ __global__ void __launch_bounds__(288, 1)
           }
           mref = nref;
         }
-        // P = 2^(s - mref) <= 2^8 in bf16, [128 rows][64 keys] K-major,
-        // swizzled; l adds the rounded weights
+        // P = 2^(s - mref) <= 2^8 in bf16, [128 rows][128 keys] K-major (two
+        // atoms of 64 keys), swizzled; l adds the rounded weights
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
+        for (int c8 = 0; c8 < 8; ++c8) {
           uint32_t pw[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            pw[u] = pack_bf16x2(ex2_approx(sv[c8 * 8 + 2 * u] - mref),
-                                ex2_approx(sv[c8 * 8 + 2 * u + 1] - mref));
+            pw[u] = pack_bf16x2(ex2_approx(sv[c8 >> 2][(c8 & 3) * 8 + 2 * u] - mref),
+                                ex2_approx(sv[c8 >> 2][(c8 & 3) * 8 + 2 * u + 1] - mref));
             lrow += __uint_as_float(pw[u] << 16) + __uint_as_float(pw[u] & 0xffff0000u);
           }
           if (lane < RPW)
-            *reinterpret_cast<uint4*>(pb + sw128_off(row, half * 32 + c8 * 8, MR)) =
+            *reinterpret_cast<uint4*>(pb + sw128_off(row, half * kUHalf + c8 * 8, MR)) =
                 make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
       }
