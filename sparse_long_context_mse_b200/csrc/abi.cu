@@ -76,11 +76,15 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   d->off_status = off;
   off += 256;
   if (which == LOSA_WS_DENSE) {
-    const int target = 2 * kSizingSms;
-    int nsplit = static_cast<int>((target + SG - 1) / SG);
+    // bf16 (tensor cores, one 211-227 KB CTA per SM): one wave of whole
+    // 128-key tiles; fp32: two CTAs' worth of splits per SM
+    const bool tc = sh->dtype == LOSA_BF16;
+    int nsplit = tc ? static_cast<int>(kSizingSms / SG)
+                    : static_cast<int>((2 * kSizingSms + SG - 1) / SG);
     if (nsplit < 1) nsplit = 1;
     if (nsplit > d->P) nsplit = d->P;
     d->split_pages = (d->P + nsplit - 1) / nsplit;
+    if (tc) d->split_pages = (d->split_pages + 7) / 8 * 8;
     d->nsplit = (d->P + d->split_pages - 1) / d->split_pages;
     d->off_part = off;
     off += align256(SG * d->nsplit * static_cast<size_t>(G * d->B) * kPartStride * sizeof(float));

@@ -105,14 +105,17 @@ __device__ __forceinline__ void suffix_row(float4 q, const float* Kb, const floa
   L = (m + __log2f(l)) * kLn2;
 }
 
-__global__ void __launch_bounds__(256)
+constexpr int kFinishWarps = 4;   // rows (one per warp) per CTA of the dense finish
+constexpr int kFinishBatch = 16;  // splits' partials in flight per row
+
+__global__ void __launch_bounds__(kFinishWarps * 32)
     dense_finish_kernel(const void* __restrict__ Q, const void* __restrict__ Kb,
                         const void* __restrict__ Vb, const float* __restrict__ part,
                         float* __restrict__ o_p, float* __restrict__ l_p, float* __restrict__ out,
                         float* __restrict__ out_lse, Dims d) {
   __shared__ __align__(16) float Ksb[kMaxB * kD];
   __shared__ __align__(16) float Vsb[kMaxB * kD];
-  __shared__ float Ps[8][kPS];
+  __shared__ float Ps[kFinishWarps][kPS];
   const int sh = blockIdx.x;  // s * Hq + h
   const int s = sh / d.Hq, h = sh % d.Hq, g = h / d.G;
   const int sg = s * d.Hkv + g;
@@ -131,30 +134,53 @@ __global__ void __launch_bounds__(256)
     *reinterpret_cast<float4*>(Vsb + j * kD + c) = vv;
   }
   __syncthreads();
-  // one warp per row: rows blockIdx.y * 8 + warp of head h
-  for (int t = blockIdx.y * 8 + warp; t < min(d.B, blockIdx.y * 8 + 8); t += 8) {
+  // one warp per row: rows blockIdx.y * kFinishWarps + warp of head h
+  for (int t = blockIdx.y * kFinishWarps + warp;
+       t < min(d.B, (blockIdx.y + 1) * kFinishWarps); t += kFinishWarps) {
     const size_t row = static_cast<size_t>(sh) * d.B + t;
     const int r = (h - g * d.G) * d.B + t;
-    // merge the prefix partials (base-2 units) of every split: the splits'
-    // maxima over the lanes, then the weighted sums with eight splits' loads
-    // in flight at a time
+    // merge the prefix partials (base-2 units) of every split in one pass,
+    // 16 splits' loads in flight at a time, the running sums rescaled when
+    // a batch raises the maximum
     const float* p0 = part + (static_cast<size_t>(sg) * d.nsplit * rows + r) * kPartStride;
     const size_t pstride = static_cast<size_t>(rows) * kPartStride;
-    float M = -INFINITY;
-    for (int sp = lane; sp < d.nsplit; sp += 32) M = fmaxf(M, __ldcg(p0 + sp * pstride));
-    M = warp_max(M);
-    float lsum = 0.f;
+    float M = -INFINITY, lsum = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int sp = 0; sp < d.nsplit; ++sp) {
-      const float* src = p0 + sp * pstride;
-      const float w = exp2f(__ldcg(src) - M);
-      lsum += w * __ldcg(src + 1);
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(src + 4) + lane);
-      acc.x += w * a.x;
-      acc.y += w * a.y;
-      acc.z += w * a.z;
-      acc.w += w * a.w;
+#pragma unroll 1
+    for (int s0 = 0; s0 < d.nsplit; s0 += kFinishBatch) {
+      float mc[kFinishBatch], lc[kFinishBatch];
+      float4 ac[kFinishBatch];
+#pragma unroll
+      for (int i = 0; i < kFinishBatch; ++i) {
+        mc[i] = -INFINITY;
+        if (s0 + i < d.nsplit) {
+          const float* src = p0 + (s0 + i) * pstride;
+          mc[i] = __ldcg(src);
+          lc[i] = __ldcg(src + 1);
+          ac[i] = __ldcg(reinterpret_cast<const float4*>(src + 4) + lane);
+        }
+      }
+      float Mh = M;
+#pragma unroll
+      for (int i = 0; i < kFinishBatch; ++i) Mh = fmaxf(Mh, mc[i]);
+      const float rs = exp2f(M - Mh);  // 0 while nothing is accumulated
+      lsum *= rs;
+      acc.x *= rs;
+      acc.y *= rs;
+      acc.z *= rs;
+      acc.w *= rs;
+#pragma unroll
+      for (int i = 0; i < kFinishBatch; ++i) {
+        if (s0 + i < d.nsplit) {
+          const float w = exp2f(mc[i] - Mh);
+          lsum += w * lc[i];
+          acc.x += w * ac[i].x;
+          acc.y += w * ac[i].y;
+          acc.z += w * ac[i].z;
+          acc.w += w * ac[i].w;
+        }
+      }
+      M = Mh;
     }
     const float inv = 1.f / lsum;
     const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
@@ -662,8 +688,9 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);
   }
-  dense_finish_kernel<<<dim3(d.S * d.Hq, (d.B + 7) / 8), 256, 0, st>>>(q, k_blk, v_blk, part, o_p,
-                                                                        l_p, out, out_lse, d);
+  dense_finish_kernel<<<dim3(d.S * d.Hq, (d.B + kFinishWarps - 1) / kFinishWarps),
+                        kFinishWarps * 32, 0, st>>>(q, k_blk, v_blk, part, o_p, l_p, out,
+                                                    out_lse, d);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
