@@ -157,13 +157,18 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+# the sources the two step kernels are compiled from (their launch code and
+# shared headers included)
+STEP_SOURCES = ("step_fused.cu", "step.cu", "losa_common.cuh", "ptx.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_long_context_mse_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for path in [os.path.join(csrc, n) for n in STEP_SOURCES] + [
+            os.path.join(ROOT, "include", "losa.h")]:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -436,9 +441,44 @@ def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):
                 api.step(sh, L.q[t], L.q[t - 1], L.K, L.V, L.meta, L.kb[t], L.vb[t], L.o_p,
                          L.l_p, L.out, L.lse, ws, stream=stream)
 
+    # the two step variants on the same schedule: every active row over its
+    # group's whole union; drift-safe locality against per-row references
+    import copy
+    sh_u = copy.copy(sh)
+    sh_u.flags = api.LOSA_STEP_ATTEND_UNION
+    q_ref = [L.q[0].clone() for L in layers]
+
+    def union_all():
+        for li, t in sched:
+            L = layers[li]
+            api.step(sh_u, L.q[t], L.q[t - 1], L.K, L.V, L.meta, L.kb[t], L.vb[t], L.o_p, L.l_p,
+                     L.out, L.lse, ws, stream=stream)
+
+    def ref_all():
+        for li, t in sched:
+            L = layers[li]
+            api.step_ref(sh, L.q[t], q_ref[li], L.K, L.V, L.meta, L.kb[t], L.vb[t], L.o_p,
+                         L.l_p, L.out, L.lse, ws, stream=stream)
+
+    out["variants"] = {
+        "attend_union_us_per_step": round(time_graph(union_all, 10) / len(sched) * 1e3, 3),
+        "drift_safe_us_per_step": round(time_graph(ref_all, 10) / len(sched) * 1e3, 3)}
+
     dense_ms = time_graph(dense_all, 3) / nL
     block_ms = time_graph(block_all, 3) / nL
     out["dense_step_us"] = dense_ms * 1e3
+    # the cold-start dense pass against the HBM roofline: the whole prefix's
+    # K and V once, the block's queries, the cache and output rows written
+    esz = 2
+    rows = sh.num_seqs * sh.n_q_heads * sh.block_size
+    dense_bytes = (2 * sh.num_seqs * sh.n_kv_heads * sh.prefix_len * sh.head_dim * esz
+                   + rows * sh.head_dim * esz + 2 * rows * (sh.head_dim + 1) * 4)
+    peak, peak_kind = measured_peaks()
+    achieved = dense_bytes / (dense_ms / 1e3) / 1e9
+    out["dense_roofline"] = {"bound": "hbm", "kernel": "losa_dense_prefix (tcgen05 pass + split combine)",
+                             "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                             "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                             "algorithmic_bytes": dense_bytes}
     out["block"] = {"T": T, "block_us": block_ms * 1e3,
                     "steps_per_s_over_block": T / (block_ms / 1e3),
                     "losa_vs_dense_step_speedup": None}
