@@ -41,6 +41,10 @@
  *   heads share KV head g = h / G), d = head_dim, L = prefix_len,
  *   ps = page_size, P = ceil(L / ps) pages (the last may be partial),
  *   B = block_size, A = n_active, k = min(token_budget / ps, P).
+ * - Prefix buffers have a capacity Lc = prefix_capacity (>= L; 0 means L):
+ *   prefix K/V are [S][Hkv][Lc][d] (tokens L..Lc-1 of each (s, g) are
+ *   unused), and the page metadata has Pc = ceil(Lc / ps) records per
+ *   (s, g).  losa_append_block grows L inside that capacity.
  */
 #ifndef LOSA_H_
 #define LOSA_H_
@@ -85,6 +89,8 @@ typedef struct {
     float   scale;         /* softmax scale; 0 selects 1/sqrt(d)          */
     int32_t dtype;         /* LOSA_F32 or LOSA_BF16                       */
     int32_t flags;         /* 0, or LOSA_STEP_ATTEND_UNION (below)        */
+    int32_t prefix_capacity; /* Lc >= L tokens per (s, g) in the prefix
+                                buffers; 0 selects L                       */
 } losa_shape;
 
 /* ---- step variants (losa_shape.flags) ----------------------------------
@@ -109,10 +115,10 @@ size_t losa_workspace_size(const losa_shape* shape, int which);
  * and max of the keys of the page's valid tokens -- what the QUEST bound
  * needs (paper, methodology: QUEST-style page selection over KV pages).
  *
- *   k_prefix   [S][Hkv][L][d]   keys, element type `dtype`
+ *   k_prefix   [S][Hkv][Lc][d]  keys, element type `dtype` (tokens < L read)
  *   page_meta  out, losa_page_meta_size() bytes, element type `dtype`:
  *              for page p of (s, g), a record of 2*d elements -- kmin[0..d)
- *              then kmax[0..d) -- at record index (s*Hkv + g)*P + p.  Inside
+ *              then kmax[0..d) -- at record index (s*Hkv + g)*Pc + p.  Inside
  *              a record the 16-byte chunks are stored XOR-swizzled: logical
  *              chunk c sits at chunk position c ^ (p & 7).  (This keeps the
  *              scoring kernel's shared-memory reads free of bank conflicts.)
@@ -122,6 +128,28 @@ int losa_build_page_meta(const losa_shape* shape, const void* k_prefix, void* pa
                          void* stream);
 
 /*
+ * Prefix growth: commit a finished block to the prefix.  When a block's last
+ * denoising step is done its tokens become prefix tokens for the blocks
+ * after it (paper, block-wise generation: each block is generated
+ * conditioned on the committed prefix).  This copies the block's keys and
+ * values into prefix positions L .. L+B-1 of every (s, g) and rebuilds the
+ * min/max records of the pages those positions touch (the old last page, if
+ * it was partial, and the new ones), exactly as losa_build_page_meta would
+ * on the grown prefix.  Afterwards the caller uses prefix_len = L + B.
+ *
+ *   shape      the shape BEFORE the append (prefix_len = L); requires
+ *              L + B <= prefix capacity (LOSA_ERR_INVALID_ARG otherwise)
+ *   k_blk,
+ *   v_blk      [S][Hkv][B][d]   the committed block's keys/values
+ *   k_prefix,
+ *   v_prefix   in/out [S][Hkv][Lc][d]
+ *   page_meta  in/out, built for the prefix of length L
+ * Other pages' records and prefix tokens < L are not written.
+ */
+int losa_append_block(const losa_shape* shape, const void* k_blk, const void* v_blk,
+                      void* k_prefix, void* v_prefix, void* page_meta, void* stream);
+
+/*
  * Cold-start dense pass (first denoising step of a block; paper,
  * limitations): every block token attends to the whole prefix, which fills
  * the cached prefix state of every row; then dense suffix attention over the
@@ -129,7 +157,7 @@ int losa_build_page_meta(const losa_shape* shape, const void* k_prefix, void* pa
  *
  *   q          [S][Hq][B][d]    queries of this step
  *   k_prefix,
- *   v_prefix   [S][Hkv][L][d]
+ *   v_prefix   [S][Hkv][Lc][d]
  *   k_blk,
  *   v_blk      [S][Hkv][B][d]   the block's own keys/values
  *   o_p        out [S][Hq][B][d] fp32  prefix output, all rows
@@ -150,7 +178,7 @@ int losa_dense_prefix(const losa_shape* shape, const void* q, const void* k_pref
  *   q_cur      [S][Hq][B][d]    this step's queries
  *   q_prev     [S][Hq][B][d]    the previous step's queries (caller rotates)
  *   k_prefix,
- *   v_prefix   [S][Hkv][L][d]
+ *   v_prefix   [S][Hkv][Lc][d]
  *   page_meta  from losa_build_page_meta on the same k_prefix
  *   k_blk,
  *   v_blk      [S][Hkv][B][d]

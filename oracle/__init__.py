@@ -242,3 +242,10 @@ def step_ref(sh: Shape, Qc, q_ref, K, V, kmin, kmax, Kb, Vb, o_p, l_p):
     res = step(sh, Qc, q_ref, K, V, kmin, kmax, Kb, Vb, o_p, l_p)
     res["q_ref"] = refresh_ref(sh, Qc, res["active_idx"], q_ref)
     return res
+
+def append_block(K, V, Kb, Vb):
+    """Prefix growth: the committed block's keys/values become prefix tokens
+    L .. L+B-1 of every (sequence, KV head) -- a concatenation along the token
+    axis of ``[S][Hkv][L][d]`` and ``[S][Hkv][B][d]``.  The grown prefix's
+    page metadata is ``build_meta`` over the result."""
+    return (np.concatenate([f32(K), f32(Kb)], axis=2), np.concatenate([f32(V), f32(Vb)], axis=2))

@@ -32,6 +32,7 @@ LOSA_WS_STEP = 1
 #: every symbol ``include/losa.h`` declares
 EXPORTS = ("losa_page_meta_size", "losa_workspace_size", "losa_build_page_meta",
            "losa_dense_prefix", "losa_step", "losa_step_ref", "losa_step_noalloc",
+           "losa_append_block",
            "losa_read_device_status",
            "losa_status_string", "losa_last_error")
 
@@ -52,7 +53,8 @@ class Shape(ctypes.Structure):
                 ("prefix_len", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("n_active", ctypes.c_int32),
                 ("token_budget", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("prefix_capacity", ctypes.c_int32)]
 
     # derived sizes (same rules as the library's validation)
     @property
@@ -62,6 +64,11 @@ class Shape(ctypes.Structure):
     @property
     def n_pages(self):
         return (self.prefix_len + self.page_size - 1) // self.page_size
+
+    @property
+    def capacity(self):
+        """Tokens per (sequence, KV head) in the prefix buffers."""
+        return self.prefix_capacity if self.prefix_capacity > 0 else self.prefix_len
 
     @property
     def pages_per_row(self):
@@ -74,11 +81,11 @@ class Shape(ctypes.Structure):
 
 def make_shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
                n_active, token_budget, dtype="bf16", scale: Optional[float] = None,
-               flags: int = 0) -> Shape:
+               flags: int = 0, prefix_capacity: int = 0) -> Shape:
     dt = {"bf16": LOSA_BF16, "f32": LOSA_F32, LOSA_BF16: LOSA_BF16, LOSA_F32: LOSA_F32}[dtype]
     sc = float(scale) if scale is not None else 0.0
     return Shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
-                 n_active, token_budget, sc, dt, flags)
+                 n_active, token_budget, sc, dt, flags, prefix_capacity)
 
 
 def shape_of(cfg, scale: Optional[float] = None, flags: int = 0) -> Shape:
@@ -111,6 +118,8 @@ def lib():
         L.losa_dense_prefix.restype = i32
         L.losa_step.argtypes = [sp] + [vp] * 14 + [vp, sz, vp]
         L.losa_step.restype = i32
+        L.losa_append_block.argtypes = [sp] + [vp] * 6
+        L.losa_append_block.restype = i32
         L.losa_step_ref.argtypes = [sp] + [vp] * 14 + [vp, sz, vp]
         L.losa_step_ref.restype = i32
         L.losa_step_noalloc.argtypes = [sp] + [vp] * 14 + [vp]
@@ -189,10 +198,25 @@ def alloc_workspace(sh: Shape, which: int, device) -> torch.Tensor:
 
 def build_page_meta(sh: Shape, k_prefix: torch.Tensor, page_meta: torch.Tensor, stream=None):
     dev = _device_of(k_prefix)
-    kv = (sh.num_seqs, sh.n_kv_heads, sh.prefix_len, sh.head_dim)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     a = _ptr(k_prefix, kv, sh.torch_dtype, "k_prefix", dev)
     b = _ptr(page_meta, (page_meta_size(sh),), torch.uint8, "page_meta", dev)
     _check(lib().losa_build_page_meta(ctypes.byref(sh), a, b, _stream(stream)))
+
+
+def append_block(sh: Shape, k_blk, v_blk, k_prefix, v_prefix, page_meta, stream=None):
+    """``losa_append_block``: commit a finished block to the prefix (tokens
+    L .. L+B-1 of every (sequence, KV head)) and rebuild the page records it
+    touches.  ``sh`` is the shape before the append; the prefix buffers need
+    room for L + B tokens (``prefix_capacity``)."""
+    dev = _device_of(k_blk)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
+    kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
+    args = [_ptr(k_blk, kb, sh.torch_dtype, "k_blk", dev), _ptr(v_blk, kb, sh.torch_dtype, "v_blk", dev),
+            _ptr(k_prefix, kv, sh.torch_dtype, "k_prefix", dev),
+            _ptr(v_prefix, kv, sh.torch_dtype, "v_prefix", dev),
+            _ptr(page_meta, (page_meta_size(sh),), torch.uint8, "page_meta", dev)]
+    _check(lib().losa_append_block(ctypes.byref(sh), *args, _stream(stream)))
 
 
 def dense_prefix(sh: Shape, q, k_prefix, v_prefix, k_blk, v_blk, o_p, l_p, out, out_lse,
@@ -200,7 +224,7 @@ def dense_prefix(sh: Shape, q, k_prefix, v_prefix, k_blk, v_blk, o_p, l_p, out, 
     dev = _device_of(q)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
-    kv = (sh.num_seqs, sh.n_kv_heads, sh.prefix_len, sh.head_dim)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
     rs = qs[:3]
     args = [_ptr(q, qs, dt, "q", dev), _ptr(k_prefix, kv, dt, "k_prefix", dev),
@@ -233,7 +257,7 @@ def _step_call(fn, sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_bl
     dev = _device_of(q_cur)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
-    kv = (sh.num_seqs, sh.n_kv_heads, sh.prefix_len, sh.head_dim)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
     rs = qs[:3]
     A, k = sh.n_active, sh.pages_per_row
@@ -261,7 +285,7 @@ def step_noalloc(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk,
     dev = _device_of(q_cur)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
-    kv = (sh.num_seqs, sh.n_kv_heads, sh.prefix_len, sh.head_dim)
+    kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
     rs = qs[:3]
     A, k = sh.n_active, sh.pages_per_row

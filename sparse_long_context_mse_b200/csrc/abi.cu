@@ -45,6 +45,7 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   if (sh->head_dim != kD || sh->page_size != kPS) return LOSA_ERR_UNSUPPORTED;
   if (sh->dtype != LOSA_F32 && sh->dtype != LOSA_BF16) return LOSA_ERR_UNSUPPORTED;
   if (sh->flags & ~LOSA_STEP_ATTEND_UNION) return LOSA_ERR_INVALID_ARG;
+  if (sh->prefix_capacity != 0 && sh->prefix_capacity < sh->prefix_len) return LOSA_ERR_INVALID_ARG;
   const int G = sh->n_q_heads / sh->n_kv_heads;
   if (sh->block_size > kMaxB || G * sh->block_size > kMaxRowsPerGroup) return LOSA_ERR_UNSUPPORTED;
   const long long P = (static_cast<long long>(sh->prefix_len) + kPS - 1) / kPS;
@@ -58,6 +59,8 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   d->G = G;
   d->L = sh->prefix_len;
   d->P = static_cast<int>(P);
+  d->Lc = sh->prefix_capacity > 0 ? sh->prefix_capacity : sh->prefix_len;
+  d->Pc = (d->Lc + kPS - 1) / kPS;
   d->B = sh->block_size;
   d->A = sh->n_active;
   d->k = static_cast<int>(kk);
@@ -132,7 +135,7 @@ extern "C" {
 size_t losa_page_meta_size(const losa_shape* shape) {
   losa::Dims d;
   if (losa::make_dims(shape, LOSA_WS_DENSE, &d) != LOSA_OK) return 0;
-  return static_cast<size_t>(d.S) * d.Hkv * d.P * 2 * losa::kD * d.esz;
+  return static_cast<size_t>(d.S) * d.Hkv * d.Pc * 2 * losa::kD * d.esz;
 }
 
 size_t losa_workspace_size(const losa_shape* shape, int which) {

@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kDenseWarps * 32)
   const int rows = d.G * d.B;
   const int p0 = split * d.split_pages;
   const int p1 = min(d.P, p0 + d.split_pages);
-  const size_t kv0 = static_cast<size_t>(sg) * d.L * kD;
+  const size_t kv0 = static_cast<size_t>(sg) * d.Lc * kD;
 
   for (int rbase = 0; rbase < rows; rbase += kDenseWarps * kRowsPerWarp) {
     float4 q[kRowsPerWarp], acc[kRowsPerWarp];
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(288, 1)
   if (warp == 8) {
     // ---- producer: TMA loads and tensor-core MMAs, one thread
     if (lane == 0) {
-      const int kv_row0 = sg * d.L + key0;            // first key of the split, as a tensor row
+      const int kv_row0 = sg * d.Lc + key0;           // first key of the split, as a tensor row
       const int q_row0 = (s * d.Hq + g * d.G) * d.B;  // the group's first query row
       auto load_k = [&](int t) {
         uint64_t* bar = &bK[t % kUKst];
@@ -675,8 +675,8 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     const bool m64 = d.G * d.B <= 64;
     CUtensorMap qmap, kmap, vmap;
     if (make_tmap(&qmap, q, rows, m64 ? 64 : 128) != LOSA_OK ||
-        make_tmap(&kmap, k_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK ||
-        make_tmap(&vmap, v_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.L, kUKeys) != LOSA_OK)
+        make_tmap(&kmap, k_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.Lc, kUKeys) != LOSA_OK ||
+        make_tmap(&vmap, v_prefix, static_cast<unsigned long long>(d.S) * d.Hkv * d.Lc, kUKeys) != LOSA_OK)
       return record_cuda_error(cudaErrorInvalidValue);
     if (m64)
       dense_umma_kernel<64><<<dim3(d.nsplit, d.S * d.Hkv), 288, UPlan<64>::smem, st>>>(

@@ -29,6 +29,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // ---------------------------------------------------------------------------
 struct Dims {
   int S, Hq, Hkv, G, L, P, B, A, k, R, MW, Umax, dtype, esz;
+  int Lc, Pc;             // prefix capacity: tokens (K/V row stride) and page records per (s, g)
   int all_pages;          // k == P: every page is selected, no scoring needed
   int attend_union;       // LOSA_STEP_ATTEND_UNION: active rows attend to the group's union
   float scale;            // softmax scale (natural-log units)

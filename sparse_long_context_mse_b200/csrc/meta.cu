@@ -1,4 +1,5 @@
-// meta.cu -- page min/max metadata build (once per prefix).
+// meta.cu -- page min/max metadata: the build (once per prefix) and prefix
+// growth (a committed block appended, its pages' records rebuilt).
 //
 // QUEST's bound needs, per page and channel, the min and max key value over
 // the page's tokens (LoSA paper, methodology: QUEST-style selection over KV
@@ -11,18 +12,14 @@ namespace {
 
 constexpr int kMetaWarps = 8;
 
-__global__ void __launch_bounds__(kMetaWarps * 32)
-    meta_build_kernel(const void* __restrict__ K, void* __restrict__ meta, Dims d) {
-  const int sg = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p = blockIdx.x * kMetaWarps + warp;
-  if (p >= d.P) return;
-  const int j0 = p * kPS;
-  const int n = min(kPS, d.L - j0);
-  const size_t base = (static_cast<size_t>(sg) * d.L + j0) * kD + 4 * lane;
-  float4 lo = ld4(K, base, d.dtype), hi = lo;
+// Min and max over n >= 1 tokens of channels [4 lane, 4 lane + 4) (key4(j):
+// token j's four channels as floats), stored as page p's record of group sg.
+template <typename Key4>
+__device__ __forceinline__ void page_record(Key4 key4, int n, void* meta, int sg, int p,
+                                            const Dims& d, int lane) {
+  float4 lo = key4(0), hi = lo;
   for (int j = 1; j < n; ++j) {
-    const float4 x = ld4(K, base + static_cast<size_t>(j) * kD, d.dtype);
+    const float4 x = key4(j);
     // strict comparisons: the first of equal values (e.g. -0 vs +0) is kept
     lo.x = x.x < lo.x ? x.x : lo.x;
     lo.y = x.y < lo.y ? x.y : lo.y;
@@ -33,7 +30,7 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
     hi.z = x.z > hi.z ? x.z : hi.z;
     hi.w = x.w > hi.w ? x.w : hi.w;
   }
-  char* rec = static_cast<char*>(meta) + (static_cast<size_t>(sg) * d.P + p) * (2 * kD * d.esz);
+  char* rec = static_cast<char*>(meta) + (static_cast<size_t>(sg) * d.Pc + p) * (2 * kD * d.esz);
   if (d.dtype == LOSA_BF16) {
     // the values are bf16 numbers held in fp32: the top 16 bits are exact
     uint2 mn, mx;
@@ -49,6 +46,58 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
   }
 }
 
+__global__ void __launch_bounds__(kMetaWarps * 32)
+    meta_build_kernel(const void* __restrict__ K, void* __restrict__ meta, Dims d) {
+  const int sg = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = blockIdx.x * kMetaWarps + warp;
+  if (p >= d.P) return;
+  const int j0 = p * kPS;
+  const size_t base = (static_cast<size_t>(sg) * d.Lc + j0) * kD + 4 * lane;
+  page_record([&](int j) { return ld4(K, base + static_cast<size_t>(j) * kD, d.dtype); },
+              min(kPS, d.L - j0), meta, sg, p, d, lane);
+}
+
+// Prefix growth: one warp per page touched by tokens L .. L+B-1 (pages
+// p0 .. p0+np-1): the page's block tokens are copied into the prefix K and V
+// (16-byte chunks), and its record is rebuilt over its tokens < L+B, each
+// read from where it lives before the copy (old prefix below L, the block
+// from L on), so no thread reads what another writes.
+__global__ void __launch_bounds__(kMetaWarps * 32)
+    append_kernel(const void* __restrict__ kb, const void* __restrict__ vb, void* __restrict__ K,
+                  void* __restrict__ V, void* __restrict__ meta, Dims d, int p0, int np) {
+  const int sg = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kMetaWarps + warp;
+  if (i >= np) return;
+  const int p = p0 + i;
+  const int L1 = d.L + d.B;
+  const int j0 = p * kPS, j1 = min(j0 + kPS, L1);
+  const size_t rowb = static_cast<size_t>(kD) * d.esz;
+  const int c16 = static_cast<int>(rowb / 16);  // 16-byte chunks per token row
+  const char* kbs = static_cast<const char*>(kb) + static_cast<size_t>(sg) * d.B * rowb;
+  const char* vbs = static_cast<const char*>(vb) + static_cast<size_t>(sg) * d.B * rowb;
+  char* Kd = static_cast<char*>(K) + static_cast<size_t>(sg) * d.Lc * rowb;
+  char* Vd = static_cast<char*>(V) + static_cast<size_t>(sg) * d.Lc * rowb;
+  const int jb = max(j0, d.L);
+  for (int e = lane; e < (j1 - jb) * c16; e += 32) {
+    const int j = jb + e / c16, c = e % c16;
+    const size_t src = static_cast<size_t>(j - d.L) * rowb + 16 * c;
+    const size_t dst = static_cast<size_t>(j) * rowb + 16 * c;
+    *reinterpret_cast<uint4*>(Kd + dst) = *reinterpret_cast<const uint4*>(kbs + src);
+    *reinterpret_cast<uint4*>(Vd + dst) = *reinterpret_cast<const uint4*>(vbs + src);
+  }
+  const size_t kbase = (static_cast<size_t>(sg) * d.Lc) * kD + 4 * lane;
+  const size_t bbase = (static_cast<size_t>(sg) * d.B) * kD + 4 * lane;
+  page_record(
+      [&](int t) {
+        const int j = j0 + t;
+        return j < d.L ? ld4(K, kbase + static_cast<size_t>(j) * kD, d.dtype)
+                       : ld4(kb, bbase + static_cast<size_t>(j - d.L) * kD, d.dtype);
+      },
+      j1 - j0, meta, sg, p, d, lane);
+}
+
 }  // namespace
 }  // namespace losa
 
@@ -59,12 +108,40 @@ extern "C" int losa_build_page_meta(const losa_shape* shape, const void* k_prefi
   int rc = make_dims(shape, LOSA_WS_DENSE, &d);
   if (rc != LOSA_OK) return rc;
   if (bad_ptr(k_prefix) || bad_ptr(page_meta)) return LOSA_ERR_INVALID_ARG;
-  const size_t kbytes = static_cast<size_t>(d.S) * d.Hkv * d.L * kD * d.esz;
+  const size_t kbytes = static_cast<size_t>(d.S) * d.Hkv * d.Lc * kD * d.esz;
   if (overlaps(k_prefix, kbytes, page_meta, losa_page_meta_size(shape))) return LOSA_ERR_INVALID_ARG;
   dim3 grid((d.P + kMetaWarps - 1) / kMetaWarps, d.S * d.Hkv);
   if (grid.y > 65535u) return LOSA_ERR_UNSUPPORTED;
   meta_build_kernel<<<grid, kMetaWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
       k_prefix, page_meta, d);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
+}
+
+extern "C" int losa_append_block(const losa_shape* shape, const void* k_blk, const void* v_blk,
+                                 void* k_prefix, void* v_prefix, void* page_meta, void* stream) {
+  using namespace losa;
+  Dims d;
+  int rc = make_dims(shape, LOSA_WS_DENSE, &d);
+  if (rc != LOSA_OK) return rc;
+  if (bad_ptr(k_blk) || bad_ptr(v_blk) || bad_ptr(k_prefix) || bad_ptr(v_prefix) ||
+      bad_ptr(page_meta))
+    return LOSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(d.L) + d.B > d.Lc) return LOSA_ERR_INVALID_ARG;  // no room
+  const size_t pb = static_cast<size_t>(d.S) * d.Hkv * d.Lc * kD * d.esz;
+  const size_t bb = static_cast<size_t>(d.S) * d.Hkv * d.B * kD * d.esz;
+  const size_t mb = losa_page_meta_size(shape);
+  if (overlaps(k_prefix, pb, v_prefix, pb) || overlaps(k_prefix, pb, page_meta, mb) ||
+      overlaps(v_prefix, pb, page_meta, mb) || overlaps(k_blk, bb, k_prefix, pb) ||
+      overlaps(k_blk, bb, v_prefix, pb) || overlaps(v_blk, bb, k_prefix, pb) ||
+      overlaps(v_blk, bb, v_prefix, pb) || overlaps(k_blk, bb, page_meta, mb) ||
+      overlaps(v_blk, bb, page_meta, mb))
+    return LOSA_ERR_INVALID_ARG;
+  const int p0 = d.L / kPS, np = (d.L + d.B - 1) / kPS - p0 + 1;
+  dim3 grid((np + kMetaWarps - 1) / kMetaWarps, d.S * d.Hkv);
+  if (grid.y > 65535u) return LOSA_ERR_UNSUPPORTED;
+  append_kernel<<<grid, kMetaWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      k_blk, v_blk, k_prefix, v_prefix, page_meta, d, p0, np);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }

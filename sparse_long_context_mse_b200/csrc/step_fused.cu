@@ -537,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int p0 = chunk * d.chunk_pages;
   const int npages = prm.scan ? max(0, min(d.P, p0 + d.chunk_pages) - p0) : 0;
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
-  const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.P * prm.rec;
+  const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.Pc * prm.rec;
   const uint32_t qbytes = static_cast<uint32_t>(GB * rowb);
 
   if (tid == 0) {
@@ -1244,7 +1244,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 #pragma unroll 1
     for (int i = 0; i < nb; ++i) {
       const int p = lpages[b0 + i];
-      const size_t off = (static_cast<size_t>(sg) * d.L + static_cast<size_t>(p) * kPS) * rowb;
+      const size_t off = (static_cast<size_t>(sg) * d.Lc + static_cast<size_t>(p) * kPS) * rowb;
       const char* kp = static_cast<const char*>(prm.K) + off;
       const char* vp = static_cast<const char*>(prm.V) + off;
       char* dk = region + 2 * i * pbytes;

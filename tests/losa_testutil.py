@@ -44,9 +44,10 @@ def unswizzle_page_meta(sh, page_meta):
     at chunk c ^ (p & 7).  Pure index permutation."""
     esz = 2 if sh.dtype == api.LOSA_BF16 else 4
     P, d = sh.n_pages, sh.head_dim
+    Pc = (sh.capacity + sh.page_size - 1) // sh.page_size  # records per (s, g)
     nchunk = 2 * d * esz // 16
-    raw = page_meta.detach().cpu().view(torch.uint8).reshape(sh.num_seqs * sh.n_kv_heads, P,
-                                                             nchunk, 16)
+    raw = page_meta.detach().cpu().view(torch.uint8).reshape(sh.num_seqs * sh.n_kv_heads, Pc,
+                                                             nchunk, 16)[:, :P]
     pages = torch.arange(P)
     phys = torch.arange(nchunk)[None, :] ^ (pages[:, None] & 7)
     idx = phys[None, :, :, None].expand(raw.shape[0], P, nchunk, 16)

@@ -487,4 +487,30 @@ def pin_drift_safe_slow_drift():
     assert first_safe == want, (first_safe, want)
 
 
+def pin_append_then_meta():
+    """Prefix growth: the grown prefix holds the old tokens then the block's
+    (bitwise); pages entirely below the old length keep their records; the
+    rebuilt pages bound every token they hold (brute force)."""
+    rng = np.random.default_rng(27)
+    S, Hkv, d, L, ps, B = 2, 2, 16, 45, 4, 6
+    f = lambda *s_: rng.standard_normal(s_).astype(np.float32)
+    K, V, Kb, Vb = f(S, Hkv, L, d), f(S, Hkv, L, d), f(S, Hkv, B, d), f(S, Hkv, B, d)
+    K2, V2 = oracle.append_block(K, V, Kb, Vb)
+    assert K2.shape == (S, Hkv, L + B, d)
+    assert np.array_equal(K2[:, :, :L].view(np.uint32), K.view(np.uint32))
+    assert np.array_equal(K2[:, :, L:].view(np.uint32), Kb.view(np.uint32))
+    assert np.array_equal(V2[:, :, L:].view(np.uint32), Vb.view(np.uint32))
+    sh1 = oracle.shape(S, 2 * Hkv, Hkv, d, L, ps, B, 2, 8)
+    sh2 = oracle.shape(S, 2 * Hkv, Hkv, d, L + B, ps, B, 2, 8)
+    mn1, mx1 = oracle.build_meta(sh1, K)
+    mn2, mx2 = oracle.build_meta(sh2, K2)
+    full = L // ps  # pages entirely below L
+    assert np.array_equal(mn2[:, :, :full], mn1[:, :, :full])
+    assert np.array_equal(mx2[:, :, :full], mx1[:, :, :full])
+    for p in range(full, oracle.n_pages(sh2)):
+        tok = K2[:, :, p * ps:min((p + 1) * ps, L + B)]
+        assert np.array_equal(mn2[:, :, p], tok.min(axis=2))
+        assert np.array_equal(mx2[:, :, p], tok.max(axis=2))
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

@@ -169,6 +169,21 @@ def test_step_ref_pointer_validation(L):
     assert call(p) == api.LOSA_ERR_INVALID_ARG
 
 
+def test_prefix_capacity_validation(L):
+    # a capacity below the prefix length is refused; a larger one grows the
+    # metadata to ceil(capacity / ps) records per (s, g)
+    assert api.workspace_size(S(prefix_capacity=65535), api.LOSA_WS_STEP) == 0
+    assert api.page_meta_size(S(prefix_capacity=65536 + 33)) == 8 * (4096 + 3) * 2 * 128 * 2
+    # appending a block needs room for B more tokens: refused before any launch
+    fake = [ctypes.c_void_p((i + 1) << 36) for i in range(5)]  # far apart: no overlaps
+    assert L.losa_append_block(ctypes.byref(S(prefix_capacity=65536 + 15)), *fake,
+                               None) == api.LOSA_ERR_INVALID_ARG
+    assert L.losa_append_block(ctypes.byref(S()), *fake, None) == api.LOSA_ERR_INVALID_ARG
+    fake[2] = fake[0]                    # k_prefix aliases k_blk
+    assert L.losa_append_block(ctypes.byref(S(prefix_capacity=65536 + 16)), *fake,
+                               None) == api.LOSA_ERR_INVALID_ARG
+
+
 def test_dense_pointer_validation(L):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)
