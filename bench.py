@@ -464,6 +464,26 @@ def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):
         "attend_union_us_per_step": round(time_graph(union_all, 10) / len(sched) * 1e3, 3),
         "drift_safe_us_per_step": round(time_graph(ref_all, 10) / len(sched) * 1e3, 3)}
 
+    # prefix growth: a committed block appended inside the buffers' capacity
+    # (one layer copy with room for one more block; the same append repeated)
+    import copy as _copy
+    L0 = layers[0]
+    sh_a = _copy.copy(sh)
+    sh_a.prefix_capacity = sh.prefix_len + sh.block_size
+    Kc = torch.empty(sh.num_seqs, sh.n_kv_heads, sh_a.prefix_capacity, sh.head_dim,
+                     dtype=L0.K.dtype, device=dev)
+    Vc = torch.empty_like(Kc)
+    Kc[:, :, :sh.prefix_len] = L0.K
+    Vc[:, :, :sh.prefix_len] = L0.V
+    meta_c = api.alloc_page_meta(sh_a, dev)
+    api.build_page_meta(sh_a, Kc, meta_c, stream=stream)
+
+    def append_one():
+        api.append_block(sh_a, L0.kb[0], L0.vb[0], Kc, Vc, meta_c, stream=stream)
+
+    out["append_block_us"] = round(time_graph(append_one, 50) * 1e3, 3)
+    del Kc, Vc, meta_c
+
     dense_ms = time_graph(dense_all, 3) / nL
     block_ms = time_graph(block_all, 3) / nL
     out["dense_step_us"] = dense_ms * 1e3
