@@ -113,8 +113,7 @@ __global__ void __launch_bounds__(kFinishWarps * 32)
                         const void* __restrict__ Vb, const float* __restrict__ part,
                         float* __restrict__ o_p, float* __restrict__ l_p, float* __restrict__ out,
                         float* __restrict__ out_lse, Dims d) {
-  __shared__ __align__(16) float Ksb[kMaxB * kD];
-  __shared__ __align__(16) float Vsb[kMaxB * kD];
+  extern __shared__ __align__(16) float fsm[];  // the block's K then V, [Bpad][d] each
   __shared__ float Ps[kFinishWarps][kPS];
   const int sh = blockIdx.x;  // s * Hq + h
   const int s = sh / d.Hq, h = sh % d.Hq, g = h / d.G;
@@ -122,6 +121,8 @@ __global__ void __launch_bounds__(kFinishWarps * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = d.G * d.B;
   const int Bpad = (d.B + kPS - 1) / kPS * kPS;
+  float* Ksb = fsm;
+  float* Vsb = fsm + Bpad * kD;
   for (int e = threadIdx.x; e < Bpad * kD / 4; e += blockDim.x) {
     const int j = e / (kD / 4), c = (e % (kD / 4)) * 4;
     float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
@@ -134,6 +135,9 @@ __global__ void __launch_bounds__(kFinishWarps * 32)
     *reinterpret_cast<float4*>(Vsb + j * kD + c) = vv;
   }
   __syncthreads();
+  // launched behind the split kernel (programmatic dependent launch): its
+  // partials are read only after it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // one warp per row: rows blockIdx.y * kFinishWarps + warp of head h
   for (int t = blockIdx.y * kFinishWarps + warp;
        t < min(d.B, (blockIdx.y + 1) * kFinishWarps); t += kFinishWarps) {
@@ -259,6 +263,9 @@ __global__ void __launch_bounds__(288, 1)
   constexpr int kUKst = C::kst, kUVst = C::vst, kUQ = C::qbytes, kUP = C::pbytes;
   constexpr int kUBars = C::nbars;
   extern __shared__ char dsm_raw[];
+  // the finish kernel may be scheduled now; it waits for this grid's
+  // completion before it reads a partial
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // 1024-byte alignment for the swizzled tiles
   char* dsm = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   // MR = MMA rows (64 or 128): the group's query rows, zero-padded
@@ -688,9 +695,24 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
         q, k_prefix, v_prefix, part, d);
   }
-  dense_finish_kernel<<<dim3(d.S * d.Hq, (d.B + kFinishWarps - 1) / kFinishWarps),
-                        kFinishWarps * 32, 0, st>>>(q, k_blk, v_blk, part, o_p, l_p, out,
-                                                    out_lse, d);
+  {
+    // behind the split kernel with programmatic dependent launch: the finish
+    // CTAs stage the block's K/V while the split kernel drains
+    cudaLaunchConfig_t cf = {};
+    cudaLaunchAttribute at[1];
+    cf.gridDim = dim3(d.S * d.Hq, (d.B + kFinishWarps - 1) / kFinishWarps, 1);
+    cf.blockDim = dim3(kFinishWarps * 32, 1, 1);
+    cf.dynamicSmemBytes = 2u * ((d.B + kPS - 1) / kPS * kPS) * kD * sizeof(float);
+    cf.stream = st;
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cf.attrs = at;
+    cf.numAttrs = 1;
+    const cudaError_t ef = cudaLaunchKernelEx(&cf, dense_finish_kernel, q, k_blk, v_blk,
+                                              static_cast<const float*>(part), o_p, l_p, out,
+                                              out_lse, d);
+    if (ef != cudaSuccess) return record_cuda_error(ef);
+  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
