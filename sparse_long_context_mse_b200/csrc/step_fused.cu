@@ -1006,10 +1006,9 @@ struct GatherParams {
 };
 
 // The k best chunk candidates of row r (keys, descending) -> out[0..k).
-// Fast path: lane c holds chunk c's sorted list; the threshold is the k-th
-// largest list head (at least k keys reach it, so the top k all do); the
-// keys at or above it are placed by ballots and rank-sorted.  Fallback:
-// sort-and-merge trees or k rounds of warp argmax.
+// Fast path: lane c holds chunk c's sorted list (lists past 32 folded in by
+// bitonic merges), then a k-way merge by warp max-reductions over the list
+// heads.  Fallback (k > 16): k rounds of warp argmax over all candidates.
 // base: the group's lists [nc][R][k] (written by the scan kernel: read
 // through L2, not L1)
 template <int KP>
@@ -1021,7 +1020,6 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r,
   const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
   if (KP > 0) {
     constexpr int KQ = KP > 0 ? KP : 1;
-    const unsigned lt = (1u << lane) - 1u;
     unsigned long long x[KQ];
     {
       const unsigned long long* lst = base + (static_cast<size_t>(lane) * R + r) * k;
@@ -1045,51 +1043,19 @@ __device__ __forceinline__ void merge_row(const GatherParams& prm, int r,
       for (int i = 0; i < KQ; ++i) y[i] = i < k ? __ldcg(lst + i) : 0ull;
       merge_top<KQ>(x, y);
     }
-    // threshold: the k-th largest list head (every list is sorted,
-    // descending), ranked from shared memory (hb: one key per lane)
-    hb[lane] = x[0];
-    __syncwarp();
-    const int nl = min(nc, 32);
-    int rk = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i < nl) {
-        const unsigned long long o = hb[i];
-        rk += (o > x[0]) || (o == x[0] && i < lane);
-      }
-    }
-    const unsigned long long tau = hb[__ffs(__ballot_sync(0xffffffffu, rk == k - 1)) - 1];
-    unsigned bl[KQ];
-    int total = 0;
-#pragma unroll
-    for (int i = 0; i < KQ; ++i) {
-      bl[i] = __ballot_sync(0xffffffffu, x[i] >= tau && x[i] != 0ull);
-      total += __popc(bl[i]);
-    }
-    if (total <= kCandCap) {
-      int pos = 0;
-#pragma unroll
-      for (int i = 0; i < KQ; ++i) {
-        if ((bl[i] >> lane) & 1u) fb[pos + __popc(bl[i] & lt)] = x[i];
-        pos += __popc(bl[i]);
-      }
-      __syncwarp();
+    // k-way merge of the sorted lists (one per lane, descending): each round
+    // a warp maximum over the list heads (high then low key half; keys are
+    // unique) is the next key, and the list that held it pops its head
 #pragma unroll 1
-      for (int t = lane; t < total; t += 32) {
-        const unsigned long long y = fb[t];
-        int rank = 0;
-#pragma unroll 4
-        for (int m = 0; m < total; ++m) rank += fb[m] > y;
-        if (rank < k) out[rank] = y;
-      }
-#pragma unroll 1
-      for (int t = total + lane; t < k; t += 32) out[t] = 0ull;
-    } else {
-      group_merge<KQ>(x, 32);
-      if (lane == 0) {
+    for (int it = 0; it < k; ++it) {
+      const uint32_t hhi = static_cast<uint32_t>(x[0] >> 32), hlo = static_cast<uint32_t>(x[0]);
+      const uint32_t mhi = __reduce_max_sync(0xffffffffu, hhi);
+      const uint32_t mlo = __reduce_max_sync(0xffffffffu, hhi == mhi ? hlo : 0u);
+      if (lane == 0) out[it] = (static_cast<unsigned long long>(mhi) << 32) | mlo;
+      if (x[0] != 0ull && hhi == mhi && hlo == mlo) {
 #pragma unroll
-        for (int i = 0; i < KQ; ++i)
-          if (i < k) out[i] = x[i];
+        for (int i = 0; i + 1 < KQ; ++i) x[i] = x[i + 1];
+        x[KQ - 1] = 0ull;
       }
     }
     __syncwarp();
