@@ -51,6 +51,7 @@ constexpr int kMaxRingBytes = 128 * 1024;
 constexpr int kStageBytes = 32 * 1024;
 constexpr int kMaxStages = kMaxRingBytes / kStageBytes;
 constexpr int kCandCap = 64;                     // per-warp compaction buffer
+constexpr int kTopkW = 16;                       // lanes per row in the chunk top-k
 constexpr int kThreadsG = 512;                   // gather kernel: one warp per merged row
 constexpr int kWarpsG = kThreadsG / 32;
 constexpr int kPageWarps = 8;                    // gather kernel: warps sharing an m16 tile's pages
@@ -365,21 +366,6 @@ __device__ __noinline__ bool row_topk(const float* row, int n, int p0, int k,
   return true;
 }
 
-// row_topk for the (W, NV) pair of the launch; false if there is none (the
-// caller falls back to register sort-and-merge).
-__device__ __forceinline__ bool row_topk_dispatch(int W, int NV, const float* row, int n, int p0,
-                                                  int k, unsigned long long* buf,
-                                                  unsigned long long* out, bool active) {
-#define LOSA_ROW_TOPK(w, nv) \
-  if (W == w && NV == nv) return row_topk<w, nv>(row, n, p0, k, buf, out, active);
-  LOSA_ROW_TOPK(4, 8) LOSA_ROW_TOPK(4, 16) LOSA_ROW_TOPK(4, 32) LOSA_ROW_TOPK(4, 64)
-  LOSA_ROW_TOPK(8, 8) LOSA_ROW_TOPK(8, 16) LOSA_ROW_TOPK(8, 32) LOSA_ROW_TOPK(8, 64)
-  LOSA_ROW_TOPK(16, 8) LOSA_ROW_TOPK(16, 16) LOSA_ROW_TOPK(16, 32) LOSA_ROW_TOPK(16, 64)
-  LOSA_ROW_TOPK(32, 8) LOSA_ROW_TOPK(32, 16) LOSA_ROW_TOPK(32, 32) LOSA_ROW_TOPK(32, 64)
-#undef LOSA_ROW_TOPK
-  return false;
-}
-
 int pow2_floor(int x) {
   int p = 1;
   while (p * 2 <= x) p *= 2;
@@ -439,13 +425,13 @@ struct ScanParams {
 // (k <= 16): the threshold filter over a group of W >= k lanes per row, rows
 // in passes of kThreads / W; a warp whose groups overflow the filter buffer
 // falls back to register sort-and-merge.  k > 16: one warp per row.
-template <int DT, int KP>
+template <int DT, int KP, int NV>
 __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* sc, int R, int k,
                                            int npages, int p0, unsigned long long* dst_base,
                                            unsigned long long* fbuf, unsigned long long* cbuf) {
   const int tid = threadIdx.x;
   if (KP > 0) {
-    const int W = prm.tpr;
+    constexpr int W = kTopkW;
     const int rows_per_pass = kThreads / W;
 #pragma unroll 1
     for (int r0 = 0; r0 < R; r0 += rows_per_pass) {
@@ -454,8 +440,10 @@ __device__ __forceinline__ void chunk_topk(const ScanParams& prm, const float* s
       const float* row = sc + (active ? r : 0) * prm.sc_stride;
       unsigned long long* out = dst_base + static_cast<size_t>(active ? r : 0) * k;
       auto key = [&](int i) { return sel_key(row[i], p0 + i); };
-      if (!row_topk_dispatch(W, prm.nv, row, npages, p0, k, fbuf + (tid / W) * kCandCap, out,
-                             active)) {
+      bool done = false;
+      if constexpr (NV > 0)
+        done = row_topk<W, NV>(row, npages, p0, k, fbuf + (tid / W) * kCandCap, out, active);
+      if (!done) {
         unsigned long long x[KP > 0 ? KP : 1];
         thread_topk<(KP > 0 ? KP : 1)>(key, tid & (W - 1), W, npages, x);
         group_merge<(KP > 0 ? KP : 1)>(x, W);
@@ -502,7 +490,7 @@ __device__ __forceinline__ void bound_ntile(const uint32_t (&a)[16][4], const ch
   }
 }
 
-template <int DT, int KP>
+template <int DT, int KP, int NV>
 __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams prm) {
   extern __shared__ __align__(1024) char smem[];
   const Dims& d = prm.d;
@@ -803,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
 
   // ---- chunk-local top-k per row -> workspace
   unsigned long long* dst = prm.cand + (static_cast<size_t>(sg) * gridDim.x + chunk) * R * k;
-  chunk_topk<DT, KP>(prm, sc, R, k, npages, p0, dst, fbuf, cbuf);
+  chunk_topk<DT, KP, NV>(prm, sc, R, k, npages, p0, dst, fbuf, cbuf);
 }
 
 // ---------------------------------------------------------------------------
@@ -1710,8 +1698,7 @@ bool plan_scan(const Dims& d, ScanParams* prm, int max_dyn) {
   const int GB = d.G * d.B;
   // a row's top-k group: at least k lanes, and enough lanes to cover the
   // CTA's rows in few passes
-  prm->tpr = std::min(32, std::max(pow2_floor(std::max(1, kThreads / std::max(d.R, 1))),
-                                   d.k <= 1 ? 1 : pow2_floor(2 * d.k - 1)));
+  prm->tpr = kTopkW;  // k <= 16 whenever the specialised top-k runs
   prm->mse_t = std::min(16, pow2_floor(std::max(1, kThreads / std::max(GB, 1))));
   prm->nv = 8;
   while (prm->nv * prm->tpr < d.chunk_pages) prm->nv *= 2;
@@ -1810,9 +1797,13 @@ int g_attr_dyn[kMaxDevices] = {};
 
 template <int DT, int KP>
 cudaError_t set_attrs_one(int optin, int* dyn) {
-  const void* fns[2] = {reinterpret_cast<const void*>(losa_scan_kernel<DT, KP>),
-                        reinterpret_cast<const void*>(losa_gather_kernel<DT, KP>)};
-  for (int i = 0; i < 2; ++i) {
+  const void* fns[6] = {reinterpret_cast<const void*>(losa_gather_kernel<DT, KP>),
+                        reinterpret_cast<const void*>(losa_scan_kernel<DT, KP, 0>),
+                        reinterpret_cast<const void*>(losa_scan_kernel<DT, KP, KP ? 8 : 0>),
+                        reinterpret_cast<const void*>(losa_scan_kernel<DT, KP, KP ? 16 : 0>),
+                        reinterpret_cast<const void*>(losa_scan_kernel<DT, KP, KP ? 32 : 0>),
+                        reinterpret_cast<const void*>(losa_scan_kernel<DT, KP, KP ? 64 : 0>)};
+  for (int i = 0; i < 6; ++i) {
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, fns[i]);
     if (e != cudaSuccess) return e;
@@ -1854,12 +1845,30 @@ int ensure_attributes(int* max_dyn) {
   return LOSA_OK;
 }
 
+// One scan kernel per (top-k width, scores per lane): each carries the one
+// row top-k it runs, which keeps its code small (instruction fetch is a
+// measurable part of a step); NV = 0 is the general fallback.
+template <int DT, int KP, int NV>
+cudaError_t launch_pair_nv(const cudaLaunchConfig_t& c1, const ScanParams& sp,
+                           const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+  const cudaError_t e = cudaLaunchKernelEx(&c1, losa_scan_kernel<DT, KP, NV>, sp);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
+}
+
 template <int DT, int KP>
 cudaError_t launch_pair(const cudaLaunchConfig_t& c1, const ScanParams& sp,
                         const cudaLaunchConfig_t& c2, const GatherParams& gp) {
-  const cudaError_t e = cudaLaunchKernelEx(&c1, losa_scan_kernel<DT, KP>, sp);
-  if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
+  if constexpr (KP > 0) {
+    switch (sp.nv) {
+      case 8: return launch_pair_nv<DT, KP, 8>(c1, sp, c2, gp);
+      case 16: return launch_pair_nv<DT, KP, 16>(c1, sp, c2, gp);
+      case 32: return launch_pair_nv<DT, KP, 32>(c1, sp, c2, gp);
+      case 64: return launch_pair_nv<DT, KP, 64>(c1, sp, c2, gp);
+      default: break;
+    }
+  }
+  return launch_pair_nv<DT, KP, 0>(c1, sp, c2, gp);
 }
 
 template <int DT>
