@@ -201,9 +201,9 @@ def step_bytes(sh, union_counts, esz):
 
 
 def launches_per_step(sh):
-    """Kernels one losa_step launches: the scan kernel always, the gather
-    kernel whenever some query row is active."""
-    return 2 if sh.n_active > 0 else 1
+    """Kernels one losa_step launches: the scan and gather kernels always, the
+    combine kernel whenever some query row is active."""
+    return 3 if sh.n_active > 0 else 2
 
 
 # ---------------------------------------------------------------------------

@@ -115,13 +115,11 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   d->off_cand = off;
   off += align256(SG * d->nchunk * R * K * sizeof(unsigned long long));
   // the gather kernel's row partials (every CTA of a group), the active
-  // rows' suffixes, and one arrival counter per group
+  // rows' suffixes
   d->off_gpart = off;
   off += align256(SG * kGatherCtas * R * kPartStride * sizeof(float));
   d->off_gsfx = off;
   off += align256(SG * R * kPartStride * sizeof(float));
-  d->off_cnt = off;
-  off += align256(SG * sizeof(int));
   d->total = off;
   // the fused step keeps each group's selection state in shared memory
   if (!fused_step_fits(*d, kB200MaxDynSmem)) return LOSA_ERR_UNSUPPORTED;

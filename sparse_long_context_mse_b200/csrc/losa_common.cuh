@@ -38,7 +38,7 @@ struct Dims {
   int nsplit, split_pages;
   int nchunk, chunk_pages;
   // workspace byte offsets
-  size_t off_status, off_part, off_act, off_cand, off_gpart, off_gsfx, off_cnt, total;
+  size_t off_status, off_part, off_act, off_cand, off_gpart, off_gsfx, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).

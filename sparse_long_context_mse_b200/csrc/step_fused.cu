@@ -1,4 +1,4 @@
-// step_fused.cu -- one LoSA denoising step in two kernel launches.
+// step_fused.cu -- one LoSA denoising step in three kernel launches.
 //
 // LoSA paper, methodology: locality pruning (MSE of Q_t vs Q_{t-1}, top-|A|
 // per head), reuse of the cached prefix state for stable tokens, QUEST page
@@ -29,8 +29,11 @@
 //    partial per row -- bf16: tensor cores, all rows of an m16 tile at once
 //    with a row mask, S = Q K^T and O += P V with P split into bf16 high and
 //    remainder parts; fp32: one warp per row on CUDA cores.  The partials go
-//    to the workspace (L2); the group's last CTA to arrive combines them,
-//    writes the new o_p / L_p and merges them with the rows' suffixes.
+//    to the workspace (L2).
+// K3 `losa_combine_kernel` -- one warp per active row, launched with
+//    programmatic dependent launch behind K2: merges the row's non-empty
+//    partials, writes the new o_p / L_p and merges them with the row's
+//    suffix into the output.
 //
 // K1's waits on bulk copies are bounded (clock64); a wait that gives up sets
 // LOSA_ERR_DEVICE_TIMEOUT in the status word and the CTA stops.  K2 waits on
@@ -406,7 +409,6 @@ struct ScanParams {
   int32_t* act_g;                  // workspace [S*Hkv][R + G*B]: act_tok, then act_slot
   int32_t* active_idx;
   unsigned long long* cand;        // workspace [S*Hkv][nchunk][R][k]
-  int* cnt;                        // workspace [S*Hkv]: the gather kernel's arrival counters
   int* status;
   Dims d;
   int scan;       // this launch scores pages (else: the active set only)
@@ -536,7 +538,6 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     // dependent launch): nothing it may still write or read is touched
     // before it has completed
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (chunk == 0) prm.cnt[sg] = 0;
     const size_t qoff = (static_cast<size_t>(s) * d.Hq + g * G) * B * rowb;
     mbar_expect_tx(&mbar[kMaxStages], 2 * qbytes);
     bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, &mbar[kMaxStages]);
@@ -959,7 +960,6 @@ struct GatherLayout {
   int ocache;   // cached o_p rows of this CTA's stable suffix rows
   int lcache;   // their cached L_p
   int sel_all, bitmap, wbase, lpages, masks, part, misc, ps, mbuf;
-  int comb;     // per row: the CTAs owning one of its pages (the non-empty partials)
   int total;
 };
 
@@ -980,7 +980,6 @@ struct GatherParams {
   const unsigned long long* cand;
   float* part_g;    // workspace [S*Hkv][CL][R][kPartStride]: every CTA's row partials
   float* sfx_g;     // workspace [S*Hkv][R][kPartStride]: active rows' suffix (L_s, -, -, -, o_s)
-  int* cnt;         // workspace [S*Hkv]: CTAs of the group done (zeroed by the scan kernel)
   int* status;
   Dims d;
   int CL;        // CTAs per group
@@ -989,7 +988,6 @@ struct GatherParams {
   int n_oa;      // max active rows owned per CTA
   int n_os;      // max stable suffix rows per CTA
   int wpart;     // bf16: warps split pages and keep per-warp partials
-  int comb_rows; // rows per batch of the last CTA's combine (their partials staged in the region)
   GatherLayout lo;
 };
 
@@ -1089,7 +1087,6 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   float* part = reinterpret_cast<float*>(smem + lo.part);  // [R][kPartStride] (fp32 path)
   float* part_cta = prm.part_g + (static_cast<size_t>(sg) * CL + rank) * R * kPartStride;
   int32_t* misc = reinterpret_cast<int32_t*>(smem + lo.misc);
-  uint32_t* rmask = reinterpret_cast<uint32_t*>(smem + lo.comb);  // [R] CTAs owning the row's pages
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
   int32_t* s_nlp = misc + 1;
@@ -1116,9 +1113,6 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 #pragma unroll 1
   for (int e = tid; e < R * kPartStride; e += kThreadsG)  // empty partials
     part[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
-#pragma unroll 1
-  for (int r = tid; r < R; r += kThreadsG)  // every CTA holds a partial of every row
-    rmask[r] = sel ? 0u : (CL >= 32 ? 0xffffffffu : (1u << CL) - 1u);
   if (sel) {
 #pragma unroll 1
     for (int w = tid; w < nwords; w += kThreadsG) bitmap[w] = 0u;
@@ -1275,7 +1269,6 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         const int w = p >> 5;
         const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
         const int r = e / k;
-        atomicOr(&rmask[r], 1u << (u % CL));  // the CTAs holding a partial of row r
         if (u % CL != rank) continue;
         if (u / CL < prm.max_lp) {
           lpages[u / CL] = p;
@@ -1288,20 +1281,13 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
     bar_sync(1, kThreads);
     if (d.attend_union && sel) {
       // every active row attends to the whole union: every row's bit on each
-      // of this CTA's pages, every CTA holding union pages in every row's
-      // combine
+      // of this CTA's pages
       const int nlp = min(*s_nlp, prm.max_lp);
 #pragma unroll 1
       for (int e = tid; e < nlp * d.MW; e += kThreads) {
         const int nb = min(32, R - 32 * (e % d.MW));
         masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
       }
-      int U = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) U += s_wsum[w];
-      const uint32_t own = U >= CL ? (CL >= 32 ? 0xffffffffu : (1u << CL) - 1u) : (1u << U) - 1u;
-#pragma unroll 1
-      for (int r = tid; r < R; r += kThreads) rmask[r] = own;
     }
     issue_batch(0, min(*s_nlp, prm.max_lp), tid, kThreads);
     cp_async_wait<0>();  // this half's copies: the gathered pages
@@ -1569,102 +1555,95 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   }
   __syncthreads();
 
-  // ---- publish this CTA's row partials (bf16: already in the workspace);
-  // the group's last CTA to finish combines every row
+  // ---- this CTA's row partials to the workspace (bf16: already there); the
+  // combine kernel merges them once every CTA of the grid has finished
   if (DT != LOSA_BF16) {
     float4* dstp = reinterpret_cast<float4*>(part_cta);
     const float4* srcp = reinterpret_cast<const float4*>(part);
 #pragma unroll 1
     for (int e = tid; e < R * kPartStride / 4; e += kThreadsG) dstp[e] = srcp[e];
-    __syncthreads();
   }
-  int* s_last = misc + 2;
-  if (tid == 0) {
-    __threadfence();  // this CTA's partials and suffixes before its arrival
-    const bool last = atomicAdd(prm.cnt + sg, 1) == CL - 1;
-    if (last) __threadfence();  // the other CTAs' writes, seen past their arrivals
-    *s_last = last;
-  }
-  __syncthreads();
-  if (!*s_last) return;
+}
 
-  // ---- combine, in batches of comb_rows rows.  A CTA's partial of row r is
-  // non-empty only if it owns one of the row's pages (rmask); each warp
-  // stages its row's non-empty partials (ascending CTA) and its suffix in the
-  // row's CL + 1 slots of the region, then merges them in that order
-  // (deterministic), writes the cache back and merges with the suffix.
-  float* stg = reinterpret_cast<float*>(region);
-  const float* pg = prm.part_g + static_cast<size_t>(sg) * CL * R * kPartStride;
-  const float* sxg = prm.sfx_g + static_cast<size_t>(sg) * R * kPartStride;
-  constexpr int c16 = kPartStride / 4;  // 16-byte chunks per partial
-#pragma unroll 1
-  for (int r0 = 0; r0 < R; r0 += prm.comb_rows) {
-    const int nr = min(prm.comb_rows, R - r0);
-#pragma unroll 1
-    for (int i = warp; i < nr; i += kWarpsG) {
-      const int r = r0 + i;
-      const uint32_t m = rmask[r];
-      const int np = __popc(m);
-      float* rs = stg + i * (CL + 1) * kPartStride;
-      const int own = lane < np ? static_cast<int>(__fns(m, 0u, lane + 1)) : 0;  // lane j: j-th owner
-#pragma unroll 1
-      for (int e0 = 0; e0 < (np + 1) * c16; e0 += 32) {
-        const int e = e0 + lane, j = e / c16, c = e - j * c16;
-        const int cj = __shfl_sync(0xffffffffu, own, min(j, 31));
-        if (e < (np + 1) * c16) {
-          const float* gsrc = j < np ? pg + (static_cast<size_t>(cj) * R + r) * kPartStride
-                                     : sxg + static_cast<size_t>(r) * kPartStride;
-          cp_async16(su32(rs + j * kPartStride + 4 * c), gsrc + 4 * c, 16u);
-        }
-      }
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-#pragma unroll 1
-    for (int i = warp; i < nr; i += kWarpsG) {
-      const int r = r0 + i;
-      const int np = __popc(rmask[r]);
-      const float* rs = stg + i * (CL + 1) * kPartStride;
-      // lane j holds partial j's (m, l): the maximum and the weights in
-      // parallel, then the vectors accumulated in slot order
-      const float mj = lane < np ? rs[lane * kPartStride] : -INFINITY;
-      const float lj = lane < np ? rs[lane * kPartStride + 1] : 0.f;
-      float M = mj;
+// ---------------------------------------------------------------------------
+// K3: combine.  One warp per active row, launched behind the gather kernel by
+// programmatic dependent launch: lane c reads CTA c's partial maximum and
+// sum, the non-empty partials' vectors are loaded together (a CTA that owns
+// none of the row's pages left m = -inf), merged in ascending CTA order
+// (deterministic); the new o_p / L_p are written back and merged with the
+// row's suffix into the output.
+// ---------------------------------------------------------------------------
+struct CombineParams {
+  const int32_t* act_g;
+  const float* part_g;
+  const float* sfx_g;
+  float* o_p;
+  float* l_p;
+  float* out;
+  float* out_lse;
+  Dims d;
+};
+
+constexpr int kCombineWarps = 4;
+
+__global__ void __launch_bounds__(kCombineWarps * 32) losa_combine_kernel(const CombineParams prm) {
+  // the next kernel of the stream may be scheduled now; it waits for this
+  // grid's completion before it touches anything this grid reads or writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const Dims& d = prm.d;
+  constexpr int CL = kGatherCtas;
+  const int lane = threadIdx.x & 31;
+  const int sg = blockIdx.y, r = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int R = d.R, A = d.A, B = d.B, GB = d.G * d.B;
+  // everything below reads what the gather kernel (and before it the scan
+  // kernel) wrote
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (r >= R) return;
+  const int s = sg / d.Hkv, g = sg % d.Hkv;
+  const size_t grow0 = (static_cast<size_t>(s) * d.Hq + g * d.G) * B;
+  const int tok = __ldcg(prm.act_g + static_cast<size_t>(sg) * (R + GB) + r);
+  const size_t cstride = static_cast<size_t>(R) * kPartStride;  // between CTAs' partials
+  const float* pg = prm.part_g + (static_cast<size_t>(sg) * CL * R + r) * kPartStride;
+  const float* sx = prm.sfx_g + (static_cast<size_t>(sg) * R + r) * kPartStride;
+  const float mj = lane < CL ? __ldcg(pg + lane * cstride) : -INFINITY;
+  const float lj = lane < CL ? __ldcg(pg + lane * cstride + 1) : 0.f;
+  const float4 os = __ldcg(reinterpret_cast<const float4*>(sx + 4) + lane);
+  const float Ls = __ldcg(sx);
+  const uint32_t nz = __ballot_sync(0xffffffffu, mj != -INFINITY);
+  float4 ac[CL];
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      const float wj = mj == -INFINITY ? 0.f : exp2f(mj - M);
-      float lsum = wj * lj;
+  for (int j = 0; j < CL; ++j)
+    if ((nz >> j) & 1u) ac[j] = __ldcg(reinterpret_cast<const float4*>(pg + j * cstride + 4) + lane);
+  float M = mj;
 #pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int j = 0; j < np; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wj, j);
-        const float4 a4 = *reinterpret_cast<const float4*>(rs + j * kPartStride + 4 + 4 * lane);
-        acc.x += w * a4.x;
-        acc.y += w * a4.y;
-        acc.z += w * a4.z;
-        acc.w += w * a4.w;
-      }
-      const float* sx = rs + np * kPartStride;
-      const float4 os = *reinterpret_cast<const float4*>(sx + 4 + 4 * lane);
-      const float Ls = sx[0];
-      const float inv = __frcp_rn(lsum);
-      const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      const float Lp = (M + __log2f(lsum)) * kLn2;
-      const size_t grow = grow0 + (r / A) * B + act_tok[r];
-      *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
-      if (lane == 0) prm.l_p[grow] = Lp;
-      float wa, wb, L;
-      lse_weights(Lp, Ls, wa, wb, L);
-      *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
-          make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
-                      wa * op.w + wb * os.w);
-      if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float wj = mj == -INFINITY ? 0.f : exp2f(mj - M);
+  float lsum = wj * lj;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < CL; ++j) {
+    const float w = __shfl_sync(0xffffffffu, wj, j);
+    if ((nz >> j) & 1u) {
+      acc.x += w * ac[j].x;
+      acc.y += w * ac[j].y;
+      acc.z += w * ac[j].z;
+      acc.w += w * ac[j].w;
     }
-    __syncthreads();  // the batch's slots are consumed before the next batch's copies
   }
+  const float inv = __frcp_rn(lsum);
+  const float4 op = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  const float Lp = (M + __log2f(lsum)) * kLn2;
+  const size_t grow = grow0 + (r / A) * B + tok;
+  *reinterpret_cast<float4*>(prm.o_p + grow * kD + 4 * lane) = op;
+  if (lane == 0) prm.l_p[grow] = Lp;
+  float wa, wb, L;
+  lse_weights(Lp, Ls, wa, wb, L);
+  *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+      make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                  wa * op.w + wb * os.w);
+  if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
 }
 
 // ---------------------------------------------------------------------------
@@ -1744,15 +1723,12 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
   const int pbytes = kPS * rowb;
   const int bpad = (d.B + kPS - 1) / kPS * kPS;
   const bool sel = !d.all_pages && d.A > 0;
-  // the region holds, in turn: the gathered pages, the page warps' partials,
-  // the partials staged for the combine
-  const long long slot = 4LL * kPartStride;  // one staged partial
-  auto layout = [&](int ngp, int crows) {
+  // the region holds, in turn: the gathered pages, the page warps' partials
+  auto layout = [&](int ngp) {
     GatherLayout& lo = prm->lo;
     Taker take;
-    lo.region = take(std::max({2LL * ngp * pbytes,
-                               prm->wpart ? 4LL * kPageWarps * 16 * kPartStride : 0LL,
-                               (CL + 1LL) * crows * slot}),
+    lo.region = take(std::max(2LL * ngp * pbytes,
+                              prm->wpart ? 4LL * kPageWarps * 16 * kPartStride : 0LL),
                      1024);
     lo.kbv = take(2LL * bpad * rowb, 128);
     lo.qa = take(1LL * (bf ? ntm * 16 : d.R) * rowb, 128);
@@ -1768,27 +1744,14 @@ bool plan_gather(const Dims& d, GatherParams* prm, int max_dyn, int CL) {
     lo.misc = take((16 + d.R + GB + ns) * 4, 16);
     lo.ps = take(kWarpsG * 16 * 4, 16);
     lo.mbuf = take(sel ? (2 * kCandCap + 32) * kWarpsG * 8 : 0, 16);
-    lo.comb = take(4LL * d.R, 16);
     lo.total = take.off;
     prm->ngp = ngp;
-    prm->comb_rows = crows;
     return lo.total;
   };
-  // the CTA holds an SM alone (512 threads at up to 128 registers): the
-  // largest batch of pages in flight, then as many combine rows per batch
-  // as fit
-  const int R1 = std::max(1, d.R);
-  bool ok = false;
-  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1 && !ok; ngp /= 2) {
-    for (int crows = R1; crows >= 1; crows = crows > 1 ? (crows + 1) / 2 : 0) {
-      if (layout(ngp, crows) <= max_dyn) {
-        ok = true;
-        break;
-      }
-      if (crows == 1) break;
-    }
-  }
-  return ok;
+  // the largest batch of pages in flight that fits
+  for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2)
+    if (layout(ngp) <= max_dyn) return true;
+  return false;
 }
 
 std::mutex g_attr_mu;
@@ -1848,38 +1811,44 @@ int ensure_attributes(int* max_dyn) {
 // One scan kernel per (top-k width, scores per lane): each carries the one
 // row top-k it runs, which keeps its code small (instruction fetch is a
 // measurable part of a step); NV = 0 is the general fallback.
+struct StepLaunch {
+  cudaLaunchConfig_t c1, c2, c3;
+  ScanParams sp;
+  GatherParams gp;
+  CombineParams cp;
+};
+
 template <int DT, int KP, int NV>
-cudaError_t launch_pair_nv(const cudaLaunchConfig_t& c1, const ScanParams& sp,
-                           const cudaLaunchConfig_t& c2, const GatherParams& gp) {
-  const cudaError_t e = cudaLaunchKernelEx(&c1, losa_scan_kernel<DT, KP, NV>, sp);
+cudaError_t launch_step_nv(const StepLaunch& L) {
+  cudaError_t e = cudaLaunchKernelEx(&L.c1, losa_scan_kernel<DT, KP, NV>, L.sp);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&c2, losa_gather_kernel<DT, KP>, gp);
+  e = cudaLaunchKernelEx(&L.c2, losa_gather_kernel<DT, KP>, L.gp);
+  if (e != cudaSuccess || L.c3.gridDim.x == 0) return e;  // no active row: nothing to combine
+  return cudaLaunchKernelEx(&L.c3, losa_combine_kernel, L.cp);
 }
 
 template <int DT, int KP>
-cudaError_t launch_pair(const cudaLaunchConfig_t& c1, const ScanParams& sp,
-                        const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+cudaError_t launch_step_kp(const StepLaunch& L) {
   if constexpr (KP > 0) {
-    switch (sp.nv) {
-      case 8: return launch_pair_nv<DT, KP, 8>(c1, sp, c2, gp);
-      case 16: return launch_pair_nv<DT, KP, 16>(c1, sp, c2, gp);
-      case 32: return launch_pair_nv<DT, KP, 32>(c1, sp, c2, gp);
-      case 64: return launch_pair_nv<DT, KP, 64>(c1, sp, c2, gp);
+    switch (L.sp.nv) {
+      case 8: return launch_step_nv<DT, KP, 8>(L);
+      case 16: return launch_step_nv<DT, KP, 16>(L);
+      case 32: return launch_step_nv<DT, KP, 32>(L);
+      case 64: return launch_step_nv<DT, KP, 64>(L);
       default: break;
     }
   }
-  return launch_pair_nv<DT, KP, 0>(c1, sp, c2, gp);
+  return launch_step_nv<DT, KP, 0>(L);
 }
 
 template <int DT>
-cudaError_t launch_dt(int kp, const cudaLaunchConfig_t& c1, const ScanParams& sp,
-                      const cudaLaunchConfig_t& c2, const GatherParams& gp) {
+cudaError_t launch_dt(int kp, const StepLaunch& L) {
   switch (kp) {
-    case 2: return launch_pair<DT, 2>(c1, sp, c2, gp);
-    case 4: return launch_pair<DT, 4>(c1, sp, c2, gp);
-    case 8: return launch_pair<DT, 8>(c1, sp, c2, gp);
-    case 16: return launch_pair<DT, 16>(c1, sp, c2, gp);
-    default: return launch_pair<DT, 0>(c1, sp, c2, gp);
+    case 2: return launch_step_kp<DT, 2>(L);
+    case 4: return launch_step_kp<DT, 4>(L);
+    case 8: return launch_step_kp<DT, 8>(L);
+    case 16: return launch_step_kp<DT, 16>(L);
+    default: return launch_step_kp<DT, 0>(L);
   }
 }
 
@@ -1899,8 +1868,9 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   int max_dyn = 0;
   int rc = ensure_attributes(&max_dyn);
   if (rc != LOSA_OK) return rc;
-  ScanParams sp;
-  GatherParams gp;
+  StepLaunch L = {};
+  ScanParams& sp = L.sp;
+  GatherParams& gp = L.gp;
   if (!plan_scan(d, &sp, max_dyn)) return LOSA_ERR_UNSUPPORTED;
   if (!plan_gather(d, &gp, max_dyn, kGatherCtas)) return LOSA_ERR_UNSUPPORTED;
   if (d.S * d.Hkv > 65535 || d.nchunk > 65535) return LOSA_ERR_UNSUPPORTED;
@@ -1910,7 +1880,6 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + d.off_cand);
   float* part_g = reinterpret_cast<float*>(ws + d.off_gpart);
   float* sfx_g = reinterpret_cast<float*>(ws + d.off_gsfx);
-  int* cnt = reinterpret_cast<int*>(ws + d.off_cnt);
 
   sp.qc = q_cur;
   sp.qp = q_prev;
@@ -1918,9 +1887,8 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   sp.act_g = act;
   sp.active_idx = active_idx;
   sp.cand = cand;
-  sp.cnt = cnt;
   sp.status = status;
-  cudaLaunchConfig_t c1 = {};
+  cudaLaunchConfig_t& c1 = L.c1;
   cudaLaunchAttribute attr1[1];
   c1.gridDim = dim3(sp.scan ? d.nchunk : 1, d.S * d.Hkv, 1);
   c1.blockDim = dim3(kThreads, 1, 1);
@@ -1947,9 +1915,8 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   gp.cand = cand;
   gp.part_g = part_g;
   gp.sfx_g = sfx_g;
-  gp.cnt = cnt;
   gp.status = status;
-  cudaLaunchConfig_t c2 = {};
+  cudaLaunchConfig_t& c2 = L.c2;
   cudaLaunchAttribute attr[1];
   c2.gridDim = dim3(gp.CL, d.S * d.Hkv, 1);
   c2.blockDim = dim3(kThreadsG, 1, 1);
@@ -1959,11 +1926,31 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;  // overlaps the scan kernel
   c2.attrs = attr;
   c2.numAttrs = 1;
+
+  CombineParams& cp = L.cp;
+  cp.act_g = act;
+  cp.part_g = part_g;
+  cp.sfx_g = sfx_g;
+  cp.o_p = o_p;
+  cp.l_p = l_p;
+  cp.out = out;
+  cp.out_lse = out_lse;
+  cp.d = d;
+  cudaLaunchConfig_t& c3 = L.c3;
+  cudaLaunchAttribute attr3[1];
+  c3.gridDim = dim3((d.R + kCombineWarps - 1) / kCombineWarps, d.S * d.Hkv, 1);
+  c3.blockDim = dim3(kCombineWarps * 32, 1, 1);
+  c3.dynamicSmemBytes = 0;
+  c3.stream = st;
+  attr3[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr3[0].val.programmaticStreamSerializationAllowed = 1;  // overlaps the gather kernel
+  c3.attrs = attr3;
+  c3.numAttrs = 1;
   // one top-k width per compiled kernel: the selection code of the others is
   // never fetched
   const int kp = sp.scan ? sp.kp : 2;
-  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, c1, sp, c2, gp)
-                                             : launch_dt<LOSA_F32>(kp, c1, sp, c2, gp);
+  const cudaError_t e = d.dtype == LOSA_BF16 ? launch_dt<LOSA_BF16>(kp, L)
+                                             : launch_dt<LOSA_F32>(kp, L);
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }
 
