@@ -1106,8 +1106,8 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   // [8, 16) stage the suffix rows and compute the suffix
   const bool uhalf = tid < kThreads;
   const int htid = uhalf ? tid : tid - kThreads;
-  // the next step's scan kernel may be scheduled now; it waits for this
-  // grid's completion before it touches anything
+  // the combine kernel may be scheduled now (its CTAs are small); it waits
+  // for this grid's completion before it reads anything
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
 #pragma unroll 1
@@ -1587,9 +1587,6 @@ struct CombineParams {
 constexpr int kCombineWarps = 4;
 
 __global__ void __launch_bounds__(kCombineWarps * 32) losa_combine_kernel(const CombineParams prm) {
-  // the next kernel of the stream may be scheduled now; it waits for this
-  // grid's completion before it touches anything this grid reads or writes
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const Dims& d = prm.d;
   constexpr int CL = kGatherCtas;
   const int lane = threadIdx.x & 31;
@@ -1598,6 +1595,11 @@ __global__ void __launch_bounds__(kCombineWarps * 32) losa_combine_kernel(const 
   // everything below reads what the gather kernel (and before it the scan
   // kernel) wrote
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the next kernel of the stream (the next step's scan kernel) may be
+  // scheduled now, not earlier: its CTAs would sit on SMs the gather kernel
+  // still needs; it waits for this grid's completion before it touches
+  // anything this grid reads or writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (r >= R) return;
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const size_t grow0 = (static_cast<size_t>(s) * d.Hq + g * d.G) * B;
