@@ -106,7 +106,7 @@ __device__ __forceinline__ void suffix_row(float4 q, const float* Kb, const floa
 }
 
 constexpr int kFinishWarps = 4;   // rows (one per warp) per CTA of the dense finish
-constexpr int kFinishBatch = 16;  // splits' partials in flight per row
+constexpr int kFinishBatch = 18;  // splits' partials in flight per row (one round at 18 splits)
 
 __global__ void __launch_bounds__(kFinishWarps * 32)
     dense_finish_kernel(const void* __restrict__ Q, const void* __restrict__ Kb,
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kFinishWarps * 32)
     const size_t row = static_cast<size_t>(sh) * d.B + t;
     const int r = (h - g * d.G) * d.B + t;
     // merge the prefix partials (base-2 units) of every split in one pass,
-    // 16 splits' loads in flight at a time, the running sums rescaled when
+    // kFinishBatch splits' loads in flight at a time, the running sums rescaled when
     // a batch raises the maximum
     const float* p0 = part + (static_cast<size_t>(sg) * d.nsplit * rows + r) * kPartStride;
     const size_t pstride = static_cast<size_t>(rows) * kPartStride;
