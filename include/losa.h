@@ -34,6 +34,10 @@
  *   legacy default stream).  Host-side validation happens before any launch;
  *   a call that returns an error has launched nothing, except LOSA_ERR_CUDA
  *   after a failed launch.
+ * - Stream order holds for every input, including one written by the
+ *   kernel right before the call: the step's kernels are chained by
+ *   programmatic dependent launch, and none reads an argument before the
+ *   work queued ahead of the call has completed.
  * - Element types: LOSA_BF16 (bfloat16) or LOSA_F32 (float) for Q, K, V and
  *   the page metadata; the cached prefix state, the outputs and all
  *   accumulation are fp32.

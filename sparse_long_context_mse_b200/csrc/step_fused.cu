@@ -505,10 +505,15 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   const int GB = G * B;
   constexpr int rowb = DT == LOSA_BF16 ? kD * 2 : kD * 4;
 
-  // the gather kernel may start staging now; it waits for this grid's
-  // completion before it reads anything written here
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (tid != 0) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // launched behind the previous kernel of the stream (programmatic
+  // dependent launch): every thread waits for it to complete before touching
+  // anything it may write; only then may the gather kernel be scheduled,
+  // since that kernel stages the block's K/V (an input of this call) before
+  // its own wait
+  if (tid != 0) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
 
   char* ring = smem + lo.ring;
   const char* qcs = smem + lo.qc;
@@ -534,10 +539,8 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    // launched behind the previous kernel of the stream (programmatic
-    // dependent launch): nothing it may still write or read is touched
-    // before it has completed
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const size_t qoff = (static_cast<size_t>(s) * d.Hq + g * G) * B * rowb;
     mbar_expect_tx(&mbar[kMaxStages], 2 * qbytes);
     bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, &mbar[kMaxStages]);
