@@ -263,6 +263,47 @@ def test_edge(name):
     assert api.read_device_status(res["ws"]) == api.LOSA_OK
 
 
+@pytest.mark.parametrize("variant", ["union", "ref", "capacity"])
+@pytest.mark.parametrize("name", ["ragged_bf16", "one_page", "rows128", "all_pages_big_k",
+                                  "zero_active", "k64"])
+def test_edge_variants(name, variant):
+    """The edge shapes under each variant: attending to the whole union,
+    drift-safe locality against a reference, prefix buffers with a capacity
+    beyond the prefix (unaligned, never read)."""
+    S, Hq, Hkv, L, B, A, budget, dt = EDGE[name]
+    c = random_case(S, Hq, Hkv, L, B, A, budget, dt, seed=zlib.crc32((name + variant).encode()) % 1000)
+    sh = c.sh
+    Kh, Vh = c.host("K"), c.host("V")
+    if variant == "union":
+        sh.flags = api.LOSA_STEP_ATTEND_UNION
+    if variant == "capacity":
+        cap = L + 37
+        K = torch.full((S, Hkv, cap, 128), 3.0, dtype=c.K.dtype, device=DEV)
+        V = torch.full_like(K, -3.0)
+        K[:, :, :L] = c.K
+        V[:, :, :L] = c.V
+        sh.prefix_capacity = cap
+        c.K, c.V = K, V
+    meta = gpu_meta(sh, c.K)
+    kmin, kmax = check_meta(sh, meta, Kh)
+    cache_g = gpu_dense(sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])
+    cache_o = oracle.dense_prefix(oshape(sh), c.q[0], Kh, Vh, c.kb[0], c.vb[0])
+    for k in ("o_p", "l_p", "out", "lse"):
+        assert maxabs(cache_g[k].cpu().numpy(), cache_o[k]) <= TOL, (name, variant, "dense", k)
+    q_ref = c.q[0].clone() + 0.25 if variant == "ref" else None
+    if q_ref is not None:
+        q_ref = q_ref.to(c.q[0].dtype)
+        q_ref_o = oracle.f32(q_ref)
+    res = gpu_step(sh, c.q[1], c.q[0], c.K, c.V, meta, c.kb[1], c.vb[1], cache_g["o_p"],
+                   cache_g["l_p"], q_ref=q_ref)
+    check_step_full(c, 1, res, cache_o, kmin, kmax, tag=f"{name}/{variant}",
+                    qp=q_ref_o if q_ref is not None else None)
+    if q_ref is not None:
+        want = oracle.refresh_ref(oshape(sh), c.q[1], res["active_idx"].cpu().numpy(), q_ref_o)
+        assert np.array_equal(oracle.f32(q_ref).view(np.uint32), want.view(np.uint32))
+    assert api.read_device_status(res["ws"]) == api.LOSA_OK
+
+
 def test_deterministic():
     c = Case(synth.config(1))
     sh = c.sh
