@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LoSA attention steps/s and achieved HBM GB/s (frac of peak) at 64K ctx, B=16"
 UNIT = "steps/s"
-CONFIG_ID = 2
+WORKLOAD = "gqa32x8_L65536_B16"  # the 64K-context, B=16 layer
 
 
 def parse_args():
@@ -246,7 +246,7 @@ def run_losa(args):
     from sparse_long_context_mse_b200 import api, synth
     rank, world, local = dist_setup(args)
     dev = torch.device("cuda", local)
-    cfg = synth.config(CONFIG_ID)
+    cfg = synth.workload(WORKLOAD)
     T = cfg.steps
     sh, layers, ws_dense = build_layers(cfg, args.layers, dev)
     ws = api.alloc_workspace(sh, api.LOSA_WS_STEP, dev)
@@ -358,7 +358,7 @@ def naive_quest(stream, dev, world, losa_union, losa_ms):
     import dataclasses
     import torch
     from sparse_long_context_mse_b200 import api, synth
-    cfg = synth.config(CONFIG_ID)
+    cfg = synth.workload(WORKLOAD)
     cfg = dataclasses.replace(cfg, n_active=cfg.block_size)
     n_layers = 2  # 2 x ~280 MB of prefix K/V + metadata: larger than L2
     sh, layers, _ = build_layers(cfg, n_layers, dev)
@@ -546,7 +546,7 @@ def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):
 # ---------------------------------------------------------------------------
 # the oracle (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample_setup(cfg_id=CONFIG_ID, device="cpu", layer0=None):
+def oracle_sample_setup(name=WORKLOAD, device="cpu", layer0=None):
     """Host arrays of one layer of the workload, restricted to query head 0
     and its KV head (1/Hq of a step's rows; the step's work is uniform over
     heads).  The incoming cache is zeros: the step's cost does not depend on
@@ -554,7 +554,7 @@ def oracle_sample_setup(cfg_id=CONFIG_ID, device="cpu", layer0=None):
     import numpy as np
     import oracle
     from sparse_long_context_mse_b200 import synth
-    cfg = synth.config(cfg_id)
+    cfg = synth.workload(name)
     if layer0 is None:
         pre = synth.gen_prefix(cfg, 0, device=device)
         q = synth.gen_queries(cfg, 0, steps=2, device=device, hot_u=pre["hot_u"])["q"]

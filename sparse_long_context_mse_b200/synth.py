@@ -92,26 +92,32 @@ def _outer_inner_profile(n_layers=36, outer=4, a_outer=2, s_outer=0.005, a_mid=6
     return tuple(prof)
 
 
-#: The five workloads.  0: tiny fp32 single head; 1: one 8B-class GQA layer
-#: at 16K; 2: the same layer at the 64K / B=16 point the pages time;
-#: 3: 8 independent 32K sequences with B=32; 4: a 36-layer stack at 128K.
-CONFIGS = {
-    0: LosaConfig("tiny_f32_L2048", 1, 1, 1, 128, 2048, 16, 16, 4, 128, F32,
-                  n_hot=32, sigma_stable=0.01, sigma_active=1.0, seed=0),
-    1: LosaConfig("gqa32x8_L16384_B16", 1, 32, 8, 128, 16384, 16, 16, 4, 256, BF16,
-                  n_hot=64, sigma_stable=0.01, sigma_active=1.0, seed=1),
-    2: LosaConfig("gqa32x8_L65536_B16", 1, 32, 8, 128, 65536, 16, 16, 4, 128, BF16,
-                  n_hot=64, sigma_stable=0.01, sigma_active=1.0, seed=2, steps=8),
-    3: LosaConfig("batch8_gqa32x8_L32768_B32", 8, 32, 8, 128, 32768, 16, 32, 8, 256, BF16,
-                  n_hot=327, sigma_stable=0.02, sigma_active=1.0, seed=300),
-    4: LosaConfig("stack36_gqa32x8_L131072_B16", 1, 32, 8, 128, 131072, 16, 16, 6, 256, BF16,
-                  n_hot=64, sigma_stable=0.02, sigma_active=1.0, seed=400, steps=8,
-                  layers=36, layer_profile=_outer_inner_profile()),
-}
+#: Workload names: a tiny fp32 single head; one 8B-class GQA layer (32 query,
+#: 8 KV heads) at 16K; the same layer at the 64K / B=16 point the pages time;
+#: 8 independent 32K sequences with B=32; a 36-layer stack at 128K.
+TINY = "tiny_f32_L2048"
+GQA16K = "gqa32x8_L16384_B16"
+GQA64K = "gqa32x8_L65536_B16"
+BATCH8 = "batch8_gqa32x8_L32768_B32"
+STACK36 = "stack36_gqa32x8_L131072_B16"
+
+WORKLOADS = {c.name: c for c in (
+    LosaConfig(TINY, 1, 1, 1, 128, 2048, 16, 16, 4, 128, F32,
+               n_hot=32, sigma_stable=0.01, sigma_active=1.0, seed=0),
+    LosaConfig(GQA16K, 1, 32, 8, 128, 16384, 16, 16, 4, 256, BF16,
+               n_hot=64, sigma_stable=0.01, sigma_active=1.0, seed=1),
+    LosaConfig(GQA64K, 1, 32, 8, 128, 65536, 16, 16, 4, 128, BF16,
+               n_hot=64, sigma_stable=0.01, sigma_active=1.0, seed=2, steps=8),
+    LosaConfig(BATCH8, 8, 32, 8, 128, 32768, 16, 32, 8, 256, BF16,
+               n_hot=327, sigma_stable=0.02, sigma_active=1.0, seed=300),
+    LosaConfig(STACK36, 1, 32, 8, 128, 131072, 16, 16, 6, 256, BF16,
+               n_hot=64, sigma_stable=0.02, sigma_active=1.0, seed=400, steps=8,
+               layers=36, layer_profile=_outer_inner_profile()),
+)}
 
 
-def config(n: int) -> LosaConfig:
-    return CONFIGS[n]
+def workload(name: str) -> LosaConfig:
+    return WORKLOADS[name]
 
 
 # ---------------------------------------------------------------------------

@@ -213,9 +213,9 @@ def pin_planted_recovery():
     """Planted actives (drift 1.0 vs 0.01) are recovered exactly on the tiny
     workload and on the first heads of the GQA workload."""
     from sparse_long_context_mse_b200 import synth
-    for n in (0, 1):
-        cfg = synth.config(n)
-        if n == 1:
+    for w in (synth.TINY, synth.GQA16K):
+        cfg = synth.workload(w)
+        if w == synth.GQA16K:
             cfg = cfg.with_(prefix_len=64)
         q = synth.gen_queries(cfg)
         sh = oracle.shape_of(cfg)
@@ -225,7 +225,7 @@ def pin_planted_recovery():
         for s in range(cfg.num_seqs):
             for h in range(cfg.n_q_heads):
                 want = list(np.nonzero(planted[s, h])[0])
-                assert list(act[s, h]) == want, f"cfg{n} s{s} h{h}: {list(act[s, h])} != {want}"
+                assert list(act[s, h]) == want, f"{w} s{s} h{h}: {list(act[s, h])} != {want}"
 
 
 def _np_dense_all(sh, x):

@@ -21,15 +21,15 @@ def clone_cache(d):
 # ---------------------------------------------------------------------------
 # page metadata: bit-exact
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("n", [0, 1, 2, 3])
-def test_meta_exact(n):
-    c = Case(synth.config(n), gen_device="cpu" if n < 2 else DEV)
+@pytest.mark.parametrize("w", [synth.TINY, synth.GQA16K, synth.GQA64K, synth.BATCH8])
+def test_meta_exact(w):
+    c = Case(synth.workload(w), gen_device="cpu" if w in (synth.TINY, synth.GQA16K) else DEV)
     meta = gpu_meta(c.sh, c.K)
     check_meta(c.sh, meta, c.host("K"))
 
 
 def test_meta_exact_stack_layer():
-    c = Case(synth.config(4), layer=35, gen_device=DEV)
+    c = Case(synth.workload(synth.STACK36), layer=35, gen_device=DEV)
     meta = gpu_meta(c.sh, c.K)
     check_meta(c.sh, meta, c.host("K"))
 
@@ -37,9 +37,9 @@ def test_meta_exact_stack_layer():
 # ---------------------------------------------------------------------------
 # cold-start dense pass
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("n", [0, 1])
-def test_dense_full(n):
-    c = Case(synth.config(n))
+@pytest.mark.parametrize("w", [synth.TINY, synth.GQA16K])
+def test_dense_full(w):
+    c = Case(synth.workload(w))
     g = gpu_dense(c.sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])
     o = oracle.dense_prefix(oshape(c.sh), c.q[0], c.host("K"), c.host("V"), c.kb[0], c.vb[0])
     for k in ("o_p", "l_p", "out", "lse"):
@@ -47,9 +47,9 @@ def test_dense_full(n):
         assert e <= TOL, (k, e)
 
 
-@pytest.mark.parametrize("n", [2, 3])
-def test_dense_sampled(n):
-    c = Case(synth.config(n), gen_device=DEV)
+@pytest.mark.parametrize("w", [synth.GQA64K, synth.BATCH8])
+def test_dense_sampled(w):
+    c = Case(synth.workload(w), gen_device=DEV)
     g = gpu_dense(c.sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])
     sh = c.sh
     osh = oshape(sh)
@@ -75,9 +75,9 @@ def test_dense_sampled(n):
 # ---------------------------------------------------------------------------
 # one LoSA step
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("n", [0, 1])
-def test_step_full(n):
-    c = Case(synth.config(n))
+@pytest.mark.parametrize("w", [synth.TINY, synth.GQA16K])
+def test_step_full(w):
+    c = Case(synth.workload(w))
     sh = c.sh
     meta = gpu_meta(sh, c.K)
     kmin, kmax = check_meta(sh, meta, c.host("K"))
@@ -85,7 +85,7 @@ def test_step_full(n):
     cache_o = oracle.dense_prefix(oshape(sh), c.q[0], c.host("K"), c.host("V"), c.kb[0], c.vb[0])
     res = gpu_step(sh, c.q[1], c.q[0], c.K, c.V, meta, c.kb[1], c.vb[1],
                    cache_g["o_p"].clone(), cache_g["l_p"].clone())
-    _, errs, exact = check_step_full(c, 1, res, cache_o, kmin, kmax, tag=f"cfg{n}")
+    _, errs, exact = check_step_full(c, 1, res, cache_o, kmin, kmax, tag=w)
     # stable rows untouched
     act = res["active_idx"].cpu().numpy()
     for s in range(sh.num_seqs):
@@ -100,9 +100,10 @@ def test_step_full(n):
     assert api.read_device_status(res["ws"]) == api.LOSA_OK
 
 
-@pytest.mark.parametrize("n,layer", [(2, 0), (3, 0), (4, 0), (4, 17), (4, 35)])
-def test_step_sampled(n, layer):
-    c = Case(synth.config(n), layer=layer, gen_device=DEV)
+@pytest.mark.parametrize("w,layer", [(synth.GQA64K, 0), (synth.BATCH8, 0), (synth.STACK36, 0),
+                                     (synth.STACK36, 17), (synth.STACK36, 35)])
+def test_step_sampled(w, layer):
+    c = Case(synth.workload(w), layer=layer, gen_device=DEV)
     sh = c.sh
     meta = gpu_meta(sh, c.K)
     kmin, kmax = check_meta(sh, meta, c.host("K"))
@@ -110,7 +111,7 @@ def test_step_sampled(n, layer):
     cache_in = clone_cache(cache_g)
     res = gpu_step(sh, c.q[1], c.q[0], c.K, c.V, meta, c.kb[1], c.vb[1], cache_g["o_p"],
                    cache_g["l_p"])
-    check_step_sampled(c, 1, res, cache_in, kmin, kmax, tag=f"cfg{n}/L{layer}")
+    check_step_sampled(c, 1, res, cache_in, kmin, kmax, tag=f"{w}/L{layer}")
     assert api.read_device_status(res["ws"]) == api.LOSA_OK
 
 
@@ -118,16 +119,14 @@ def test_step_sampled(n, layer):
 # step variants
 # ---------------------------------------------------------------------------
 def _union_case(name):
-    if name == "cfg0":
-        return Case(synth.config(0))
-    if name == "cfg1":
-        return Case(synth.config(1))
+    if name in (synth.TINY, synth.GQA16K):
+        return Case(synth.workload(name))
     if name == "groups_bf16":
         return random_case(2, 8, 2, 1000, 16, 4, 64, "bf16", seed=5)
     return random_case(1, 4, 1, 777, 8, 3, 48, "f32", seed=6)
 
 
-@pytest.mark.parametrize("name", ["cfg0", "cfg1", "groups_bf16", "ragged_f32"])
+@pytest.mark.parametrize("name", [synth.TINY, synth.GQA16K, "groups_bf16", "ragged_f32"])
 def test_step_attend_union(name):
     """Every active row attends to its group's whole page union: the
     selection is the plain step's, o_p/L_p/out are the oracle's union
@@ -152,12 +151,12 @@ def test_step_attend_union(name):
     assert api.read_device_status(res["ws"]) == api.LOSA_OK
 
 
-@pytest.mark.parametrize("n", [0, 1])
-def test_step_ref_chain(n):
+@pytest.mark.parametrize("w", [synth.TINY, synth.GQA16K])
+def test_step_ref_chain(w):
     """Drift-safe locality over a denoising chain: each step scores against
     the reference queries, the GPU's reference is rewritten exactly for the
     active rows, and every output matches the oracle's drift-safe step."""
-    cfg = synth.config(n)
+    cfg = synth.workload(w)
     T = 4
     c = Case(cfg, steps=T)
     sh = c.sh
@@ -171,7 +170,7 @@ def test_step_ref_chain(n):
     for t in range(1, T):
         res = gpu_step(sh, c.q[t], None, c.K, c.V, meta, c.kb[t], c.vb[t], cache_g["o_p"],
                        cache_g["l_p"], ws=ws, q_ref=q_ref_g)
-        ref, _, _ = check_step_full(c, t, res, cache_o, kmin, kmax, tag=f"ref{n} t{t}",
+        ref, _, _ = check_step_full(c, t, res, cache_o, kmin, kmax, tag=f"ref {w} t{t}",
                                     qp=q_ref_o)
         q_ref_o = oracle.refresh_ref(oshape(sh), c.q[t], res["active_idx"].cpu().numpy(), q_ref_o)
         assert np.array_equal(oracle.f32(q_ref_g).view(np.uint32), q_ref_o.view(np.uint32)), t
@@ -182,8 +181,8 @@ def test_step_ref_chain(n):
 # ---------------------------------------------------------------------------
 # denoising chains: step 1 dense, then LoSA steps, cache carried through
 # ---------------------------------------------------------------------------
-def test_chain_full_cfg1():
-    cfg = synth.config(1)
+def test_chain_full_16k():
+    cfg = synth.workload(synth.GQA16K)
     T = 4
     c = Case(cfg, steps=T)
     sh = c.sh
@@ -199,8 +198,8 @@ def test_chain_full_cfg1():
         cache_o = {"o_p": ref["o_p"], "l_p": ref["l_p"]}
 
 
-def test_chain_sampled_cfg2():
-    cfg = synth.config(2)
+def test_chain_sampled_64k():
+    cfg = synth.workload(synth.GQA64K)
     T = cfg.steps
     c = Case(cfg, steps=T, gen_device=DEV)
     sh = c.sh
@@ -305,7 +304,7 @@ def test_edge_variants(name, variant):
 
 
 def test_deterministic():
-    c = Case(synth.config(1))
+    c = Case(synth.workload(synth.GQA16K))
     sh = c.sh
     meta = gpu_meta(sh, c.K)
     cache = gpu_dense(sh, c.q[0], c.K, c.V, c.kb[0], c.vb[0])

@@ -32,7 +32,7 @@ def _outputs(sh):
 
 def test_noalloc_matches_workspace_step_on_two_calls():
     import torch
-    c = Case(synth.config(1))
+    c = Case(synth.workload(synth.GQA16K))
     sh = c.sh
     assert api.workspace_size(sh, api.LOSA_WS_STEP) <= api.NOALLOC_SCRATCH_BYTES
     meta = gpu_meta(sh, c.K)
