@@ -484,6 +484,49 @@ def extras(args, sh, layers, ws, ws_dense, stream, dev, world, sched):
     out["append_block_us"] = round(time_graph(append_one, 50) * 1e3, 3)
     del Kc, Vc, meta_c
 
+    # a variable-length batch: four sequences of 1, 1/2, 1/4 and 1/8 (+5
+    # tokens) of the prefix length in one call, against the same batch with
+    # every sequence at the longest length; NC copies rotated so that the
+    # bytes of a rotation exceed L2
+    lens = [sh.prefix_len, sh.prefix_len // 2, sh.prefix_len // 4, sh.prefix_len // 8 + 5]
+    S4, NC = len(lens), 4
+    lens_t = torch.tensor(lens, dtype=torch.int32, device=dev)
+    geo = (S4, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, sh.prefix_len, sh.page_size,
+           sh.block_size, sh.n_active, sh.token_budget, sh.dtype)
+    sh_v = api.make_shape(*geo, scale=sh.scale, prefix_lens=lens_t)
+    sh_f = api.make_shape(*geo, scale=sh.scale)
+
+    def rep(t):
+        return t.repeat(S4, *([1] * (t.dim() - 1)))
+
+    copies = []
+    for _ in range(NC):
+        K4, V4 = rep(L0.K), rep(L0.V)
+        mv, mf = api.alloc_page_meta(sh_v, dev), api.alloc_page_meta(sh_f, dev)
+        api.build_page_meta(sh_v, K4, mv, stream=stream)
+        api.build_page_meta(sh_f, K4, mf, stream=stream)
+        copies.append((K4, V4, mv, mf))
+    q1, q0, kb4, vb4 = rep(L0.q[1]), rep(L0.q[0]), rep(L0.kb[1]), rep(L0.vb[1])
+    o_p4 = torch.zeros(S4, sh.n_q_heads, sh.block_size, sh.head_dim, device=dev)
+    l_p4 = torch.zeros(S4, sh.n_q_heads, sh.block_size, device=dev)
+    out4, lse4 = torch.empty_like(o_p4), torch.empty_like(l_p4)
+    ws_v = api.alloc_workspace(sh_v, api.LOSA_WS_STEP, dev)
+    ws_f = api.alloc_workspace(sh_f, api.LOSA_WS_STEP, dev)
+
+    def batch_steps(shx, wsx, varlen):
+        def run():
+            for K4, V4, mv, mf in copies:
+                api.step(shx, q1, q0, K4, V4, mv if varlen else mf, kb4, vb4, o_p4, l_p4, out4,
+                         lse4, wsx, stream=stream)
+        return run
+
+    us_v = time_graph(batch_steps(sh_v, ws_v, True), 10) / NC * 1e3
+    us_f = time_graph(batch_steps(sh_f, ws_f, False), 10) / NC * 1e3
+    out["varlen_batch"] = {"prefix_lens": lens, "us_per_step": round(us_v, 3),
+                           "all_at_longest_us_per_step": round(us_f, 3),
+                           "device_status": api.read_device_status(ws_v)}
+    del copies
+
     dense_ms = time_graph(dense_all, 3) / nL
     block_ms = time_graph(block_all, 3) / nL
     out["dense_step_us"] = dense_ms * 1e3

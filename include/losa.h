@@ -49,6 +49,17 @@
  *   prefix K/V are [S][Hkv][Lc][d] (tokens L..Lc-1 of each (s, g) are
  *   unused), and the page metadata has Pc = ceil(Lc / ps) records per
  *   (s, g).  losa_append_block grows L inside that capacity.
+ * - Variable-length batches: with losa_shape.prefix_lens set, sequence s has
+ *   its own prefix length L_s (P_s = ceil(L_s / ps) pages); prefix_len is
+ *   then the largest length and sizes the buffers, the workspaces and k.
+ *   Every sequence gets what a one-sequence call with prefix_len = L_s
+ *   gives (up to rounding order), except that its rows of page_idx are
+ *   padded with -1 past min(k, P_s) entries; tokens L_s..Lc-1 of its prefix
+ *   buffers are never used, whatever they hold.  The array is read on the
+ *   device in stream order (it may be written by the kernel right before the
+ *   call, and a captured graph reads its current contents).  An entry
+ *   outside [1, L] is clamped into it; losa_dense_prefix and the step calls
+ *   also report it as LOSA_ERR_DEVICE_BOUNDS through losa_read_device_status.
  */
 #ifndef LOSA_H_
 #define LOSA_H_
@@ -95,6 +106,9 @@ typedef struct {
     int32_t flags;         /* 0, or LOSA_STEP_ATTEND_UNION (below)        */
     int32_t prefix_capacity; /* Lc >= L tokens per (s, g) in the prefix
                                 buffers; 0 selects L                       */
+    const int32_t* prefix_lens; /* NULL, or a DEVICE array [S] (4-byte
+                                aligned) of per-sequence prefix lengths
+                                1 <= L_s <= L: a variable-length batch   */
 } losa_shape;
 
 /* ---- step variants (losa_shape.flags) ----------------------------------
@@ -142,7 +156,9 @@ int losa_build_page_meta(const losa_shape* shape, const void* k_prefix, void* pa
  * on the grown prefix.  Afterwards the caller uses prefix_len = L + B.
  *
  *   shape      the shape BEFORE the append (prefix_len = L); requires
- *              L + B <= prefix capacity (LOSA_ERR_INVALID_ARG otherwise)
+ *              L + B <= prefix capacity (LOSA_ERR_INVALID_ARG otherwise).
+ *              With prefix_lens, sequence s appends at its own L_s (and the
+ *              caller then adds B to every entry and to prefix_len).
  *   k_blk,
  *   v_blk      [S][Hkv][B][d]   the committed block's keys/values
  *   k_prefix,
@@ -193,7 +209,7 @@ int losa_dense_prefix(const losa_shape* shape, const void* q, const void* k_pref
  *   out_lse    out [S][Hq][B] fp32; may be NULL
  *   active_idx optional out [S][Hq][A] int32: active tokens, ascending
  *   page_idx   optional out [S][Hq][A][k] int32: each active row's pages,
- *              ascending
+ *              ascending (then -1 past a short sequence's P_s pages)
  *   union_count optional out [S][Hkv] int32: distinct pages loaded per
  *              (sequence, KV head) -- the union over its G*A active rows
  *   workspace  >= losa_workspace_size(shape, LOSA_WS_STEP) bytes, 256-byte

@@ -249,3 +249,58 @@ def append_block(K, V, Kb, Vb):
     axis of ``[S][Hkv][L][d]`` and ``[S][Hkv][B][d]``.  The grown prefix's
     page metadata is ``build_meta`` over the result."""
     return (np.concatenate([f32(K), f32(Kb)], axis=2), np.concatenate([f32(V), f32(Vb)], axis=2))
+
+# ---------------------------------------------------------------------------
+# Variable-length batches.  The pages define the step for one sequence; a
+# batch whose sequences have different prefix lengths is read as what the
+# definition gives for each sequence on its own (prefix length lens[s], its
+# own pages P_s = ceil(lens[s] / ps) and k_s = min(budget / ps, P_s)), laid
+# side by side.  Inputs are the batch's capacity-strided arrays
+# ([S][Hkv][>= max lens][d]); tokens past a sequence's length are not read.
+# Page lists are padded to the batch's k = min(budget / ps, P_max) with -1.
+# ---------------------------------------------------------------------------
+def seq_shape(sh: Shape, L: int) -> Shape:
+    """The one-sequence shape of a sequence of prefix length ``L``."""
+    return shape(1, sh.Hq, sh.Hkv, sh.d, int(L), sh.ps, sh.B, sh.A, sh.budget, sh.scale,
+                 sh.flags)
+
+
+def _seq_prefix(X, s, L):
+    return f32(X[s:s + 1, :, :int(L)])
+
+
+def build_meta_varlen(sh: Shape, lens, K):
+    """Per-sequence page metadata: a list of (kmin, kmax), ``[1][Hkv][P_s][d]``."""
+    return [build_meta(seq_shape(sh, L), _seq_prefix(K, s, L)) for s, L in enumerate(lens)]
+
+
+def dense_prefix_varlen(sh: Shape, lens, Q, K, V, Kb, Vb):
+    parts = [dense_prefix(seq_shape(sh, L), f32(Q[s:s + 1]), _seq_prefix(K, s, L),
+                          _seq_prefix(V, s, L), f32(Kb[s:s + 1]), f32(Vb[s:s + 1]))
+             for s, L in enumerate(lens)]
+    return {key: np.concatenate([p[key] for p in parts]) for key in parts[0]}
+
+
+def step_varlen(sh: Shape, lens, Qc, Qp, K, V, Kb, Vb, o_p, l_p):
+    """One LoSA step of a variable-length batch (metadata built from K per
+    sequence).  Returns step()'s dict, page_idx padded with -1."""
+    k = pages_per_row(sh)
+    parts = []
+    for s, L in enumerate(lens):
+        ssh = seq_shape(sh, L)
+        Ks = _seq_prefix(K, s, L)
+        kmin, kmax = build_meta(ssh, Ks)
+        r = step(ssh, f32(Qc[s:s + 1]), f32(Qp[s:s + 1]), Ks, _seq_prefix(V, s, L), kmin, kmax,
+                 f32(Kb[s:s + 1]), f32(Vb[s:s + 1]), f32(o_p[s:s + 1]), f32(l_p[s:s + 1]))
+        pidx = np.full(r["page_idx"].shape[:-1] + (k,), -1, np.int32)
+        pidx[..., :r["page_idx"].shape[-1]] = r["page_idx"]
+        r["page_idx"] = pidx
+        parts.append(r)
+    return {key: np.concatenate([p[key] for p in parts]) for key in parts[0]}
+
+
+def append_block_varlen(lens, K, V, Kb, Vb):
+    """Each sequence's block appended at its own length: a list of the grown
+    ``(K_s, V_s)``, ``[1][Hkv][lens[s] + B][d]``."""
+    return [append_block(_seq_prefix(K, s, L), _seq_prefix(V, s, L), f32(Kb[s:s + 1]),
+                         f32(Vb[s:s + 1])) for s, L in enumerate(lens)]

@@ -54,7 +54,14 @@ class Shape(ctypes.Structure):
                 ("block_size", ctypes.c_int32), ("n_active", ctypes.c_int32),
                 ("token_budget", ctypes.c_int32), ("scale", ctypes.c_float),
                 ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32),
-                ("prefix_capacity", ctypes.c_int32)]
+                ("prefix_capacity", ctypes.c_int32), ("prefix_lens", ctypes.c_void_p)]
+
+    def __copy__(self):
+        """A field-by-field copy (ctypes cannot pickle a structure that holds a
+        pointer); it shares the per-sequence length array."""
+        sh = Shape(*(getattr(self, f) for f, _ in self._fields_))
+        sh._prefix_lens = getattr(self, "_prefix_lens", None)
+        return sh
 
     # derived sizes (same rules as the library's validation)
     @property
@@ -81,11 +88,23 @@ class Shape(ctypes.Structure):
 
 def make_shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
                n_active, token_budget, dtype="bf16", scale: Optional[float] = None,
-               flags: int = 0, prefix_capacity: int = 0) -> Shape:
+               flags: int = 0, prefix_capacity: int = 0, prefix_lens=None) -> Shape:
+    """``prefix_lens``: None, or an int32 device tensor of ``num_seqs`` per-sequence
+    prefix lengths (a variable-length batch; ``prefix_len`` is then the largest).
+    The shape keeps a reference to it and passes its address: the library reads
+    its current contents at every call."""
     dt = {"bf16": LOSA_BF16, "f32": LOSA_F32, LOSA_BF16: LOSA_BF16, LOSA_F32: LOSA_F32}[dtype]
     sc = float(scale) if scale is not None else 0.0
-    return Shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
-                 n_active, token_budget, sc, dt, flags, prefix_capacity)
+    lens_ptr = None
+    if prefix_lens is not None:
+        if (prefix_lens.dtype != torch.int32 or not prefix_lens.is_contiguous()
+                or prefix_lens.numel() != num_seqs or prefix_lens.device.type != "cuda"):
+            raise ValueError("prefix_lens: a contiguous int32 CUDA tensor of num_seqs entries")
+        lens_ptr = prefix_lens.data_ptr()
+    sh = Shape(num_seqs, n_q_heads, n_kv_heads, head_dim, prefix_len, page_size, block_size,
+               n_active, token_budget, sc, dt, flags, prefix_capacity, lens_ptr)
+    sh._prefix_lens = prefix_lens  # keeps the array alive as long as the shape
+    return sh
 
 
 def shape_of(cfg, scale: Optional[float] = None, flags: int = 0) -> Shape:

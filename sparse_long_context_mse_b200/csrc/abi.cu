@@ -46,6 +46,7 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   if (sh->dtype != LOSA_F32 && sh->dtype != LOSA_BF16) return LOSA_ERR_UNSUPPORTED;
   if (sh->flags & ~LOSA_STEP_ATTEND_UNION) return LOSA_ERR_INVALID_ARG;
   if (sh->prefix_capacity != 0 && sh->prefix_capacity < sh->prefix_len) return LOSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(sh->prefix_lens) & 3u) return LOSA_ERR_INVALID_ARG;
   const int G = sh->n_q_heads / sh->n_kv_heads;
   if (sh->block_size > kMaxB || G * sh->block_size > kMaxRowsPerGroup) return LOSA_ERR_UNSUPPORTED;
   const long long P = (static_cast<long long>(sh->prefix_len) + kPS - 1) / kPS;
@@ -70,6 +71,7 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
   d->esz = sh->dtype == LOSA_BF16 ? 2 : 4;
   d->all_pages = (d->k == d->P);
   d->attend_union = (sh->flags & LOSA_STEP_ATTEND_UNION) != 0;
+  d->lens = sh->prefix_lens;
   d->scale = sh->scale > 0.f ? sh->scale : 1.0f / std::sqrt(static_cast<float>(sh->head_dim));
   d->scale_log2 = d->scale * kLog2e;
   d->Umax = static_cast<int>(std::min<long long>(P, static_cast<long long>(d->R) * d->k));

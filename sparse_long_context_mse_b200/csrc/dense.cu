@@ -38,7 +38,8 @@ __device__ __forceinline__ void load_page_f32(const void* src, size_t elem0, int
 
 __global__ void __launch_bounds__(kDenseWarps * 32)
     dense_partial_kernel(const void* __restrict__ Q, const void* __restrict__ K,
-                         const void* __restrict__ V, float* __restrict__ part, Dims d) {
+                         const void* __restrict__ V, float* __restrict__ part,
+                         int* __restrict__ status, Dims d) {
   __shared__ __align__(16) float Ks[kPS * kD];
   __shared__ __align__(16) float Vs[kPS * kD];
   __shared__ float Ps[kDenseWarps][kPS];
@@ -46,9 +47,11 @@ __global__ void __launch_bounds__(kDenseWarps * 32)
   const int s = sg / d.Hkv, g = sg % d.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rows = d.G * d.B;
+  const int L = seq_len(d, s);  // this sequence's prefix length
   const int p0 = split * d.split_pages;
-  const int p1 = min(d.P, p0 + d.split_pages);
+  const int p1 = min((L + kPS - 1) / kPS, p0 + d.split_pages);  // none past its end
   const size_t kv0 = static_cast<size_t>(sg) * d.Lc * kD;
+  if (split == 0 && threadIdx.x == 0 && seq_len_bad(d, s)) atomicCAS(status, 0, LOSA_ERR_DEVICE_BOUNDS);
 
   for (int rbase = 0; rbase < rows; rbase += kDenseWarps * kRowsPerWarp) {
     float4 q[kRowsPerWarp], acc[kRowsPerWarp];
@@ -64,7 +67,7 @@ __global__ void __launch_bounds__(kDenseWarps * 32)
       l[i] = 0.f;
     }
     for (int p = p0; p < p1; ++p) {
-      const int ntok = min(kPS, d.L - p * kPS);
+      const int ntok = min(kPS, L - p * kPS);
       __syncthreads();
       load_page_f32(K, kv0 + static_cast<size_t>(p) * kPS * kD, ntok, d.dtype, Ks, threadIdx.x,
                     blockDim.x);
@@ -288,8 +291,15 @@ __global__ void __launch_bounds__(288, 1)
   const int rows = d.G * d.B;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int key0 = split * d.split_pages * kPS;
-  const int key1 = min(d.L, key0 + d.split_pages * kPS);
-  const int n = (key1 - key0 + kUKeys - 1) / kUKeys;
+  const int key1 = min(seq_len(d, s), key0 + d.split_pages * kPS);
+  const int n = key1 > key0 ? (key1 - key0 + kUKeys - 1) / kUKeys : 0;
+  if (split == 0 && tid == 0 && seq_len_bad(d, s)) atomicCAS(status, 0, LOSA_ERR_DEVICE_BOUNDS);
+  if (n == 0) {  // a split past a shorter sequence's end: an empty partial per row
+    float* dst0 = part + (static_cast<size_t>(sg) * d.nsplit + split) * rows * kPartStride;
+    for (int e = tid; e < rows * kPartStride; e += blockDim.x)
+      dst0[e] = (e % kPartStride) == 0 ? -INFINITY : 0.f;
+    return;
+  }
 
   if (tid == 0) {
     for (int i = 0; i < kUBars; ++i) mbar_init(&bars[i], i >= 5 + kUKst + kUVst ? 256 : 1);
@@ -303,6 +313,23 @@ __global__ void __launch_bounds__(288, 1)
   const uint32_t tbase = *tslot;
   const uint32_t tO = tbase + 2 * kUKeys;  // S tiles: columns [0, 128) and [128, 256)
   bool ok = true;
+  // V rows of a partial last tile past the split's end are outside the
+  // prefix (a capacity region or a shorter sequence's unused tokens) and may
+  // hold anything; P is 0 there, but 0 times a NaN or Inf of V would still
+  // reach O, so the softmax warps zero those rows once the tile has landed
+  // and before they publish P (rows r of both 64-channel atoms are the bytes
+  // [128 r, 128 r + 128): the swizzle permutes chunks inside a row)
+  auto zero_v_tail = [&](int t) {
+    const int nv = key1 - (key0 + t * kUKeys);  // real keys of the tile, 1 .. 127
+    ok = ok && mbar_wait(&bV[t % kUVst], (t / kUVst) & 1);
+    char* vt = vring + (t % kUVst) * kUTile;
+    const int per = (kUKeys - nv) * 8;  // 16-byte chunks past the real rows, per atom
+    for (int e = tid; e < 2 * per; e += 256) {
+      const int a = e >= per ? 1 : 0;
+      *reinterpret_cast<uint4*>(vt + a * (kUTile / 2) + nv * 128 + (e - a * per) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
 
   if (warp == 8) {
     // ---- producer: TMA loads and tensor-core MMAs, one thread
@@ -468,6 +495,7 @@ __global__ void __launch_bounds__(288, 1)
           }
         }
       }
+      if (key0 + (t + 1) * kUKeys > key1) zero_v_tail(t);
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bP[t & 1]);
@@ -583,6 +611,7 @@ __global__ void __launch_bounds__(288, 1)
                 make_uint4(pw[0], pw[1], pw[2], pw[3]);
         }
       }
+      if (key0 + (t + 1) * kUKeys > key1) zero_v_tail(t);
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(&bP[t & 1]);
@@ -664,6 +693,7 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
   if (d.S * d.Hkv > 65535) return LOSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* part = reinterpret_cast<float*>(static_cast<char*>(workspace) + d.off_part);
+  int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.off_status);
   if (d.dtype == LOSA_BF16) {
     if (d.G * d.B > 128) return LOSA_ERR_UNSUPPORTED;
     static bool attr_done[kMaxDevices] = {};
@@ -678,7 +708,6 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
       if (e0 != cudaSuccess) return record_cuda_error(e0);
       attr_done[dev] = true;
     }
-    int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.off_status);
     const bool m64 = d.G * d.B <= 64;
     CUtensorMap qmap, kmap, vmap;
     if (make_tmap(&qmap, q, rows, m64 ? 64 : 128) != LOSA_OK ||
@@ -693,7 +722,7 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
           qmap, kmap, vmap, part, status, d);
   } else {
     dense_partial_kernel<<<dim3(d.nsplit, d.S * d.Hkv), kDenseWarps * 32, 0, st>>>(
-        q, k_prefix, v_prefix, part, d);
+        q, k_prefix, v_prefix, part, status, d);
   }
   {
     // behind the split kernel with programmatic dependent launch: the finish

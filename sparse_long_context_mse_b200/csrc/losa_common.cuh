@@ -32,6 +32,7 @@ struct Dims {
   int Lc, Pc;             // prefix capacity: tokens (K/V row stride) and page records per (s, g)
   int all_pages;          // k == P: every page is selected, no scoring needed
   int attend_union;       // LOSA_STEP_ATTEND_UNION: active rows attend to the group's union
+  const int32_t* lens;    // per-sequence prefix lengths (device, [S]) or null: every one is L
   float scale;            // softmax scale (natural-log units)
   float scale_log2;       // scale * log2(e): scores in base-2 units
   // prefix splits (dense pass); page chunks of the step's scan
@@ -107,6 +108,16 @@ __device__ __forceinline__ int key_index(unsigned long long key) {
 // (16-byte chunks XOR-swizzled by the page index).
 __host__ __device__ __forceinline__ uint32_t meta_swz(uint32_t b, int page) {
   return ((((b >> 4) ^ static_cast<uint32_t>(page & 7)) << 4) | (b & 15u));
+}
+
+// Prefix length of sequence s: its entry of the per-sequence lengths, clamped
+// into [1, L] (so that every access stays inside the buffers), else L.
+__device__ __forceinline__ int seq_len(const Dims& d, int s) {
+  return d.lens ? min(max(d.lens[s], 1), d.L) : d.L;
+}
+// The entry of sequence s lies outside [1, L] (seq_len clamped it).
+__device__ __forceinline__ bool seq_len_bad(const Dims& d, int s) {
+  return d.lens && (d.lens[s] < 1 || d.lens[s] > d.L);
 }
 
 __device__ __forceinline__ void set_status(void* ws, int code) {

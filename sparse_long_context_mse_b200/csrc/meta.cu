@@ -51,27 +51,31 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
   const int sg = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p = blockIdx.x * kMetaWarps + warp;
-  if (p >= d.P) return;
+  const int L = seq_len(d, sg / d.Hkv);  // this sequence's prefix length
+  if (p * kPS >= L) return;
   const int j0 = p * kPS;
   const size_t base = (static_cast<size_t>(sg) * d.Lc + j0) * kD + 4 * lane;
   page_record([&](int j) { return ld4(K, base + static_cast<size_t>(j) * kD, d.dtype); },
-              min(kPS, d.L - j0), meta, sg, p, d, lane);
+              min(kPS, L - j0), meta, sg, p, d, lane);
 }
 
 // Prefix growth: one warp per page touched by tokens L .. L+B-1 (pages
-// p0 .. p0+np-1): the page's block tokens are copied into the prefix K and V
-// (16-byte chunks), and its record is rebuilt over its tokens < L+B, each
-// read from where it lives before the copy (old prefix below L, the block
-// from L on), so no thread reads what another writes.
+// L/ps .. (L+B-1)/ps, L the sequence's own length): the page's block tokens
+// are copied into the prefix K and V (16-byte chunks), and its record is
+// rebuilt over its tokens < L+B, each read from where it lives before the
+// copy (old prefix below L, the block from L on), so no thread reads what
+// another writes.
 __global__ void __launch_bounds__(kMetaWarps * 32)
     append_kernel(const void* __restrict__ kb, const void* __restrict__ vb, void* __restrict__ K,
-                  void* __restrict__ V, void* __restrict__ meta, Dims d, int p0, int np) {
+                  void* __restrict__ V, void* __restrict__ meta, Dims d) {
   const int sg = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = seq_len(d, sg / d.Hkv);
+  const int p0 = L / kPS, np = (L + d.B - 1) / kPS - p0 + 1;
   const int i = blockIdx.x * kMetaWarps + warp;
   if (i >= np) return;
   const int p = p0 + i;
-  const int L1 = d.L + d.B;
+  const int L1 = L + d.B;
   const int j0 = p * kPS, j1 = min(j0 + kPS, L1);
   const size_t rowb = static_cast<size_t>(kD) * d.esz;
   const int c16 = static_cast<int>(rowb / 16);  // 16-byte chunks per token row
@@ -79,10 +83,10 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
   const char* vbs = static_cast<const char*>(vb) + static_cast<size_t>(sg) * d.B * rowb;
   char* Kd = static_cast<char*>(K) + static_cast<size_t>(sg) * d.Lc * rowb;
   char* Vd = static_cast<char*>(V) + static_cast<size_t>(sg) * d.Lc * rowb;
-  const int jb = max(j0, d.L);
+  const int jb = max(j0, L);
   for (int e = lane; e < (j1 - jb) * c16; e += 32) {
     const int j = jb + e / c16, c = e % c16;
-    const size_t src = static_cast<size_t>(j - d.L) * rowb + 16 * c;
+    const size_t src = static_cast<size_t>(j - L) * rowb + 16 * c;
     const size_t dst = static_cast<size_t>(j) * rowb + 16 * c;
     *reinterpret_cast<uint4*>(Kd + dst) = *reinterpret_cast<const uint4*>(kbs + src);
     *reinterpret_cast<uint4*>(Vd + dst) = *reinterpret_cast<const uint4*>(vbs + src);
@@ -92,8 +96,8 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
   page_record(
       [&](int t) {
         const int j = j0 + t;
-        return j < d.L ? ld4(K, kbase + static_cast<size_t>(j) * kD, d.dtype)
-                       : ld4(kb, bbase + static_cast<size_t>(j - d.L) * kD, d.dtype);
+        return j < L ? ld4(K, kbase + static_cast<size_t>(j) * kD, d.dtype)
+                     : ld4(kb, bbase + static_cast<size_t>(j - L) * kD, d.dtype);
       },
       j1 - j0, meta, sg, p, d, lane);
 }
@@ -137,11 +141,12 @@ extern "C" int losa_append_block(const losa_shape* shape, const void* k_blk, con
       overlaps(v_blk, bb, v_prefix, pb) || overlaps(k_blk, bb, page_meta, mb) ||
       overlaps(v_blk, bb, page_meta, mb))
     return LOSA_ERR_INVALID_ARG;
-  const int p0 = d.L / kPS, np = (d.L + d.B - 1) / kPS - p0 + 1;
+  // pages touched: (L+B-1)/ps - L/ps + 1 <= (B-1)/ps + 2, whatever L is
+  const int np = (d.B - 1) / kPS + 2;
   dim3 grid((np + kMetaWarps - 1) / kMetaWarps, d.S * d.Hkv);
   if (grid.y > 65535u) return LOSA_ERR_UNSUPPORTED;
   append_kernel<<<grid, kMetaWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      k_blk, v_blk, k_prefix, v_prefix, page_meta, d, p0, np);
+      k_blk, v_blk, k_prefix, v_prefix, page_meta, d);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LOSA_OK : record_cuda_error(e);
 }

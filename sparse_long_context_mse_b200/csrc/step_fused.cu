@@ -506,14 +506,12 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   constexpr int rowb = DT == LOSA_BF16 ? kD * 2 : kD * 4;
 
   // launched behind the previous kernel of the stream (programmatic
-  // dependent launch): every thread waits for it to complete before touching
-  // anything it may write; only then may the gather kernel be scheduled,
-  // since that kernel stages the block's K/V (an input of this call) before
-  // its own wait
-  if (tid != 0) {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  }
+  // dependent launch): every thread waits for it to complete before reading
+  // any input (the sequence's length included) or touching anything it may
+  // write; only then may the gather kernel be scheduled, since that kernel
+  // stages the block's K/V (an input of this call) before its own wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   char* ring = smem + lo.ring;
   const char* qcs = smem + lo.qc;
@@ -530,7 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
   int32_t* act_row = act_tok + kMaxRowsPerGroup;
 
   const int p0 = chunk * d.chunk_pages;
-  const int npages = prm.scan ? max(0, min(d.P, p0 + d.chunk_pages) - p0) : 0;
+  // this chunk's pages of the sequence
+  const int npages =
+      prm.scan ? max(0, min((seq_len(d, s) + kPS - 1) / kPS, p0 + d.chunk_pages) - p0) : 0;
   const int ntiles = (npages + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.Pc * prm.rec;
   const uint32_t qbytes = static_cast<uint32_t>(GB * rowb);
@@ -539,8 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     for (int i = 0; i < kMaxStages + 1; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     *s_fail = 0;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (chunk == 0 && g == 0 && seq_len_bad(d, s)) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
     const size_t qoff = (static_cast<size_t>(s) * d.Hq + g * G) * B * rowb;
     mbar_expect_tx(&mbar[kMaxStages], 2 * qbytes);
     bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, &mbar[kMaxStages]);
@@ -628,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1) losa_scan_kernel(const ScanParams
     }
   }
   __syncthreads();
-  if (npages == 0) return;
+  if (npages == 0) return;  // past the sequence's end: the gather kernel reads no list of it
 
   // ---- active rows' queries for the bound: bf16 -> [R16][256] = [q- | q+]
   // in swizzled 16-byte chunks (ldmatrix); fp32 -> [R][128]
@@ -998,15 +997,15 @@ struct GatherParams {
 // Fast path: lane c holds chunk c's sorted list (lists past 32 folded in by
 // bitonic merges), then a k-way merge by warp max-reductions over the list
 // heads.  Fallback (k > 16): k rounds of warp argmax over all candidates.
-// base: the group's lists [nc][R][k] (written by the scan kernel: read
-// through L2, not L1)
+// base: the group's lists [nchunk][R][k] (written by the scan kernel: read
+// through L2, not L1), of which the first nc cover the sequence's pages
 template <int KP>
-__device__ __forceinline__ void merge_row(const GatherParams& prm, int r,
+__device__ __forceinline__ void merge_row(const GatherParams& prm, int r, int nc,
                                           const unsigned long long* base,
                                           unsigned long long* out, unsigned long long* fb,
                                           unsigned long long* hb) {
   const Dims& d = prm.d;
-  const int lane = threadIdx.x & 31, k = d.k, nc = d.nchunk, R = d.R;
+  const int lane = threadIdx.x & 31, k = d.k, R = d.R;
   if (KP > 0) {
     constexpr int KQ = KP > 0 ? KP : 1;
     unsigned long long x[KQ];
@@ -1093,6 +1092,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   float* Ps = reinterpret_cast<float*>(smem + lo.ps);
   unsigned long long* mbuf = reinterpret_cast<unsigned long long*>(smem + lo.mbuf);
   int32_t* s_nlp = misc + 1;
+  int32_t* s_len = misc + 2;           // the sequence's prefix length (kept out of registers)
   int32_t* s_wt = misc + 4;            // stable tokens per 32-token warp slice
   int32_t* s_wsum = misc + 8;          // union words' popcounts per warp of the union half
   int32_t* act_tok = misc + 16;        // [R], then act_slot [GB]
@@ -1143,6 +1143,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
 
   const unsigned long long* cand_sg =
       prm.cand + static_cast<size_t>(sg) * d.nchunk * R * k;
+  if (tid == 0) *s_len = seq_len(d, s);  // read after the selection's barrier
   {
     const int32_t* actg = prm.act_g + static_cast<size_t>(sg) * (R + GB);
 #pragma unroll 1
@@ -1153,22 +1154,31 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   // (each CTA of the group merges all rows; the CTA with r % CL == rank
   // reports row r)
   if (sel) {
+    // the scan chunks that hold the sequence's pages
+    const int ncs = ((seq_len(d, s) + kPS - 1) / kPS + d.chunk_pages - 1) / d.chunk_pages;
 #pragma unroll 1
     for (int r = warp; r < R; r += kWarpsG) {
       unsigned long long* best = mbuf + (kWarpsG + warp) * kCandCap;
-      merge_row<KP>(prm, r, cand_sg, best, mbuf + warp * kCandCap,
+      merge_row<KP>(prm, r, ncs, cand_sg, best, mbuf + warp * kCandCap,
                     mbuf + 2 * kWarpsG * kCandCap + warp * 32);
       int32_t* dst = sel_all + r * k;
       const bool report = prm.page_idx && r % CL == rank;
 #pragma unroll 1
       for (int j = lane; j < k; j += 32) {
-        const int pj = key_index(best[j]);
-        int rk = 0;
+        // an empty key (a sequence of fewer than k pages) sorts after every
+        // real one, keeps its slot and reports page -1
+        const bool real = best[j] != 0ull;
+        const int pj = real ? key_index(best[j]) : -1;
+        int rk = j;
+        if (real) {
+          rk = 0;
 #pragma unroll 4
-        for (int u = 0; u < k; ++u) rk += key_index(best[u]) < pj;
+          for (int u = 0; u < k; ++u)  // (empty keys map to index 0xffffffff: never below)
+            rk += static_cast<uint32_t>(key_index(best[u])) < static_cast<uint32_t>(pj);
+        }
         dst[rk] = pj;
         if (pj >= 0 && pj < d.P) atomicOr(&bitmap[pj >> 5], 1u << (pj & 31));
-        else atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+        else if (real) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
         if (report) {
           const int hl = r / A, a = r % A;
           prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + rk] = pj;
@@ -1177,12 +1187,14 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
       __syncwarp();
     }
   } else if (prm.page_idx) {
+    const int Pseq = (seq_len(d, s) + kPS - 1) / kPS;  // every page of the sequence, then -1
 #pragma unroll 1
     for (int r = rank; r < R; r += CL) {
       const int hl = r / A, a = r % A;
 #pragma unroll 1
       for (int j = tid; j < k; j += kThreadsG)
-        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + j] = j;
+        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + a) * k + j] =
+            j < Pseq ? j : -1;
     }
   }
   __syncthreads();
@@ -1199,10 +1211,11 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
       const char* kp = static_cast<const char*>(prm.K) + off;
       const char* vp = static_cast<const char*>(prm.V) + off;
       char* dk = region + 2 * i * pbytes;
+      const int ntok = min(kPS, *s_len - p * kPS);
 #pragma unroll 1
       for (int e = t0; e < per; e += nthr) {
         const int j = e / cpr, c = e - j * cpr;
-        const bool ok = p * kPS + j < d.L;
+        const bool ok = j < ntok;
         const int so = (ok ? j : 0) * rowb + c * 16;
         cp_async16(su32(dk + tile_off<DT>(j, c)), kp + so, ok ? 16u : 0u);
         cp_async16(su32(dk + pbytes + tile_off<DT>(j, c)), vp + so, ok ? 16u : 0u);
@@ -1214,7 +1227,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
   if (uhalf) {
     // ---- union of the group's pages and this CTA's share (slots u % CL)
     if (d.all_pages) {
-      const int U = R > 0 ? d.P : 0;
+      const int U = R > 0 ? (*s_len + kPS - 1) / kPS : 0;
       const int nlp = U > rank ? (U - rank + CL - 1) / CL : 0;
       if (tid == 0) {
         *s_nlp = nlp;
@@ -1461,7 +1474,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
         if (!bits) continue;
         const int p = lpages[b0 + i];
         tile_attend(t, qa + mt * 16 * 256, region + 2 * i * pbytes, region + (2 * i + 1) * pbytes,
-                    bits, min(kPS, d.L - p * kPS), d.scale_log2);
+                    bits, min(kPS, *s_len - p * kPS), d.scale_log2);
       }
       if (b0 + prm.ngp < nlp) {  // next batch into the same slots
         __syncthreads();
@@ -1539,7 +1552,7 @@ __global__ void __launch_bounds__(kThreadsG, 1) losa_gather_kernel(const GatherP
           if (!((masks[(b0 + i) * d.MW + (r >> 5)] >> (r & 31)) & 1u)) continue;
           const int p = lpages[b0 + i];
           attend_page<DT>(q, region + 2 * i * pbytes, region + (2 * i + 1) * pbytes,
-                          min(kPS, d.L - p * kPS), d.scale_log2, m, l, acc, psw);
+                          min(kPS, *s_len - p * kPS), d.scale_log2, m, l, acc, psw);
         }
         __syncwarp();
         if (lane == 0) {

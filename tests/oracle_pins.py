@@ -513,4 +513,82 @@ def pin_append_then_meta():
         assert np.array_equal(mx2[:, :, p], tok.max(axis=2))
 
 
+def pin_varlen_equal_lengths():
+    """A variable-length batch whose lengths all equal L is the batched call,
+    bit for bit (metadata, dense pass and step)."""
+    sh, x, kmin, kmax, cache = _step_inputs(31, S=3)
+    lens = [sh.L] * sh.S
+    for (mn, mx), s in zip(oracle.build_meta_varlen(sh, lens, x["K"]), range(sh.S)):
+        assert np.array_equal(mn, kmin[s:s + 1]) and np.array_equal(mx, kmax[s:s + 1])
+    dv = oracle.dense_prefix_varlen(sh, lens, x["Qp"], x["K"], x["V"], x["Kb"], x["Vb"])
+    for key in cache:
+        assert np.array_equal(dv[key], cache[key]), key
+    r = oracle.step(sh, x["Qc"], x["Qp"], x["K"], x["V"], kmin, kmax, x["Kb"], x["Vb"],
+                    cache["o_p"], cache["l_p"])
+    rv = oracle.step_varlen(sh, lens, x["Qc"], x["Qp"], x["K"], x["V"], x["Kb"], x["Vb"],
+                            cache["o_p"], cache["l_p"])
+    for key in rv:
+        assert np.array_equal(rv[key], r[key]), key
+
+
+def pin_varlen_short_sequences():
+    """Sequences of different lengths (NaN past each): every value is finite;
+    the dense pass is numpy attention over each sequence's own tokens; a
+    sequence shorter than the budget selects all of its pages (its active rows'
+    o_p is then its dense prefix attention) with the page lists padded by -1;
+    a one-token prefix attends to that token alone (o_p = its value row)."""
+    rng = np.random.default_rng(32)
+    sh = rand_shape(rng, S=3, L=45, ps=4, B=6, A=2, budget=12)  # k = 3 pages
+    x = rand_inputs(rng, sh)
+    lens = [45, 7, 1]
+    K, V = x["K"].copy(), x["V"].copy()
+    for s, L in enumerate(lens):
+        K[s, :, L:] = np.nan
+        V[s, :, L:] = np.nan
+    G = sh.Hq // sh.Hkv
+    cache = oracle.dense_prefix_varlen(sh, lens, x["Qp"], K, V, x["Kb"], x["Vb"])
+    for key in cache:
+        assert np.isfinite(cache[key]).all(), key
+    for s, L in enumerate(lens):
+        for h in range(sh.Hq):
+            for t in range(sh.B):
+                o, l = np_attend(x["Qp"][s, h, t], K[s, h // G, :L], V[s, h // G, :L], sh.scale)
+                close(cache["o_p"][s, h, t], o, 1e-6, "varlen dense o_p")
+                close(cache["l_p"][s, h, t], l, 1e-5, "varlen dense L_p")
+    r = oracle.step_varlen(sh, lens, x["Qc"], x["Qp"], K, V, x["Kb"], x["Vb"],
+                           cache["o_p"], cache["l_p"])
+    for key in ("o_p", "l_p", "out", "lse"):
+        assert np.isfinite(r[key]).all(), key
+    assert r["page_idx"].shape[-1] == 3
+    assert np.all(r["page_idx"][1] == np.array([0, 1, -1])), "7 tokens: both pages, then -1"
+    assert np.all(r["page_idx"][2] == np.array([0, -1, -1])), "1 token: page 0, then -1"
+    assert np.all(r["union_count"][1] == 2) and np.all(r["union_count"][2] == 1)
+    for s, L in ((1, 7), (2, 1)):
+        for h in range(sh.Hq):
+            for t in r["active_idx"][s, h]:
+                o, l = np_attend(x["Qc"][s, h, t], K[s, h // G, :L], V[s, h // G, :L], sh.scale)
+                close(r["o_p"][s, h, t], o, 1e-6, "short sequence: dense over its tokens")
+                if L == 1:
+                    close(r["o_p"][s, h, t], V[s, h // G, 0], 1e-6, "one token: its value")
+    s0 = oracle.seq_shape(sh, 45)
+    kmin, kmax = oracle.build_meta(s0, x["K"][:1])
+    alone = oracle.step(s0, x["Qc"][:1], x["Qp"][:1], x["K"][:1], x["V"][:1], kmin, kmax,
+                        x["Kb"][:1], x["Vb"][:1], cache["o_p"][:1], cache["l_p"][:1])
+    for key in alone:
+        assert np.array_equal(r[key][:1], alone[key]), key
+
+
+def pin_varlen_append():
+    """Each sequence's block lands at its own length (bitwise concatenation)."""
+    rng = np.random.default_rng(33)
+    f = lambda *s_: rng.standard_normal(s_).astype(np.float32)
+    K, V, Kb, Vb = f(3, 2, 20, 8), f(3, 2, 20, 8), f(3, 2, 5, 8), f(3, 2, 5, 8)
+    lens = [20, 9, 1]
+    for s, (K2, V2) in enumerate(oracle.append_block_varlen(lens, K, V, Kb, Vb)):
+        L = lens[s]
+        assert K2.shape == (1, 2, L + 5, 8)
+        assert np.array_equal(K2[0, :, :L], K[s, :, :L]) and np.array_equal(K2[0, :, L:], Kb[s])
+        assert np.array_equal(V2[0, :, :L], V[s, :, :L]) and np.array_equal(V2[0, :, L:], Vb[s])
+
+
 PINS = [v for n, v in sorted(globals().items()) if n.startswith("pin_")]

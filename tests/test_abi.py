@@ -184,6 +184,29 @@ def test_prefix_capacity_validation(L):
                                None) == api.LOSA_ERR_INVALID_ARG
 
 
+def test_prefix_lens_validation(L):
+    # the per-sequence length array is a device pointer read by the kernels:
+    # the host checks only its alignment, and the sizes follow prefix_len
+    # (the largest length)
+    sh = S()
+    sh.prefix_lens = 0x100002
+    assert api.workspace_size(sh, api.LOSA_WS_STEP) == 0
+    assert api.page_meta_size(sh) == 0
+    sh.prefix_lens = 0x100004
+    for which in (api.LOSA_WS_STEP, api.LOSA_WS_DENSE):
+        assert api.workspace_size(sh, which) == api.workspace_size(S(), which) > 0
+    assert api.page_meta_size(sh) == api.page_meta_size(S())
+    assert ctypes.sizeof(api.Shape) == 13 * 4 + 4 + 8  # 8-byte aligned pointer last
+    import copy
+    c = copy.copy(sh)
+    c.prefix_len = 7
+    assert c.prefix_lens == sh.prefix_lens and sh.prefix_len == 65536
+    import torch
+    with pytest.raises(ValueError):  # a host tensor is refused by the binding
+        api.make_shape(2, 8, 2, 128, 100, 16, 16, 4, 64,
+                       prefix_lens=torch.tensor([100, 50], dtype=torch.int32))
+
+
 def test_dense_pointer_validation(L):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)
