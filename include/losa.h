@@ -141,6 +141,8 @@ size_t losa_workspace_size(const losa_shape* shape, int which);
  *              chunk c sits at chunk position c ^ (p & 7).  (This keeps the
  *              scoring kernel's shared-memory reads free of bank conflicts.)
  * Min/max introduce no rounding: the values are exact copies of key values.
+ * With prefix_lens, sequence s gets records for its own P_s pages (the last
+ * over its tokens < L_s only); its records from P_s on are not written.
  */
 int losa_build_page_meta(const losa_shape* shape, const void* k_prefix, void* page_meta,
                          void* stream);
