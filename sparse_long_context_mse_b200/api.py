@@ -201,6 +201,16 @@ def _device_of(t: torch.Tensor):
     return t.device
 
 
+def _call_device(sh: Shape, t: torch.Tensor):
+    """The call's device (its first tensor's).  The shape's per-sequence length
+    array, when it has one, must live there too: the kernels dereference it."""
+    dev = _device_of(t)
+    lens = getattr(sh, "_prefix_lens", None)
+    if sh.prefix_lens and lens is not None and lens.device != dev:
+        raise ValueError(f"prefix_lens lives on {lens.device}, the call's tensors on {dev}")
+    return dev
+
+
 def alloc_page_meta(sh: Shape, device) -> torch.Tensor:
     n = page_meta_size(sh)
     if n == 0:
@@ -216,7 +226,7 @@ def alloc_workspace(sh: Shape, which: int, device) -> torch.Tensor:
 
 
 def build_page_meta(sh: Shape, k_prefix: torch.Tensor, page_meta: torch.Tensor, stream=None):
-    dev = _device_of(k_prefix)
+    dev = _call_device(sh, k_prefix)
     kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     a = _ptr(k_prefix, kv, sh.torch_dtype, "k_prefix", dev)
     b = _ptr(page_meta, (page_meta_size(sh),), torch.uint8, "page_meta", dev)
@@ -228,7 +238,7 @@ def append_block(sh: Shape, k_blk, v_blk, k_prefix, v_prefix, page_meta, stream=
     L .. L+B-1 of every (sequence, KV head)) and rebuild the page records it
     touches.  ``sh`` is the shape before the append; the prefix buffers need
     room for L + B tokens (``prefix_capacity``)."""
-    dev = _device_of(k_blk)
+    dev = _call_device(sh, k_blk)
     kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
     kb = (sh.num_seqs, sh.n_kv_heads, sh.block_size, sh.head_dim)
     args = [_ptr(k_blk, kb, sh.torch_dtype, "k_blk", dev), _ptr(v_blk, kb, sh.torch_dtype, "v_blk", dev),
@@ -240,7 +250,7 @@ def append_block(sh: Shape, k_blk, v_blk, k_prefix, v_prefix, page_meta, stream=
 
 def dense_prefix(sh: Shape, q, k_prefix, v_prefix, k_blk, v_blk, o_p, l_p, out, out_lse,
                  workspace, stream=None):
-    dev = _device_of(q)
+    dev = _call_device(sh, q)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
     kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
@@ -273,7 +283,7 @@ def step_ref(sh: Shape, q_cur, q_ref, k_prefix, v_prefix, page_meta, k_blk, v_bl
 
 def _step_call(fn, sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
                l_p, out, out_lse, workspace, active_idx, page_idx, union_count, stream):
-    dev = _device_of(q_cur)
+    dev = _call_device(sh, q_cur)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
     kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)
@@ -301,7 +311,7 @@ def step_noalloc(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk,
     that cannot allocate device memory (the library's own fixed scratch array
     is used; shapes needing more than ``NOALLOC_SCRATCH_BYTES`` are refused).
     Calls that may overlap on the GPU race on that array."""
-    dev = _device_of(q_cur)
+    dev = _call_device(sh, q_cur)
     dt = sh.torch_dtype
     qs = (sh.num_seqs, sh.n_q_heads, sh.block_size, sh.head_dim)
     kv = (sh.num_seqs, sh.n_kv_heads, sh.capacity, sh.head_dim)

@@ -207,6 +207,22 @@ def test_prefix_lens_validation(L):
                        prefix_lens=torch.tensor([100, 50], dtype=torch.int32))
 
 
+def test_prefix_lens_on_another_device_is_refused(L):
+    # the binding refuses, before any launch, a length array that lives on
+    # another GPU than the call's tensors (no GPU is needed to check this)
+    import types
+    import torch
+    sh = S()
+    sh.prefix_lens = 0x100000
+    sh._prefix_lens = types.SimpleNamespace(device=torch.device("cuda", 1))
+    t = types.SimpleNamespace(device=torch.device("cuda", 0))
+    with pytest.raises(ValueError):
+        api._call_device(sh, t)
+    sh._prefix_lens = types.SimpleNamespace(device=torch.device("cuda", 0))
+    assert api._call_device(sh, t) == torch.device("cuda", 0)
+    assert api._call_device(S(), t) == torch.device("cuda", 0)
+
+
 def test_dense_pointer_validation(L):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)
