@@ -315,7 +315,9 @@ void oracle_dense_prefix(const oracle_shape* sh, const float* Q, const float* K,
 }
 
 /* Dense prefix attention of selected rows only (rows[] index [S][Hq][B]
- * flattened); for spot checks at sizes where the full pass is too slow. */
+ * flattened: r = (s*Hq + h)*B + t); for spot checks at sizes where the full
+ * pass is too slow.  The same cold-start pass as oracle_dense_prefix (paper,
+ * limitations: the forced dense first iteration of a block), row by row. */
 void oracle_dense_rows(const oracle_shape* sh, const float* Q, const float* K, const float* V,
                        int n_rows, const int* rows, float* o_p, float* l_p) {
     int d = sh->d, L = sh->L;
@@ -324,7 +326,7 @@ void oracle_dense_rows(const oracle_shape* sh, const float* Q, const float* K, c
     for (int j = 0; j < L; ++j) tok[j] = j;
     for (int a = 0; a < n_rows; ++a) {
         int r = rows[a];
-        int h = (r / sh->B) % sh->Hq, s = r / (sh->B * sh->Hq);
+        int h = (r / sh->B) % (MUT(13) ? sh->Hkv : sh->Hq), s = r / (sh->B * sh->Hq);
         int g = kv_head_of(sh, h);
         const float* Kg = K + ((size_t)s * sh->Hkv + g) * (size_t)L * d;
         const float* Vg = V + ((size_t)s * sh->Hkv + g) * (size_t)L * d;

@@ -259,6 +259,35 @@ def pin_dense_prefix_numpy():
     close(r["lse"], full_l, 1e-5, "dense lse == logsumexp over prefix+block")
 
 
+def pin_dense_rows_numpy():
+    """Row-by-row dense prefix attention (the checker of sampled stable rows
+    at sizes where the full pass is too slow): rows from several sequences and
+    heads of a GQA shape, in shuffled order, against numpy over each row's own
+    KV head, and bitwise against the same rows of the full pass."""
+    rng = np.random.default_rng(23)
+    sh = rand_shape(rng, S=3, Hq=6, Hkv=2, L=37, B=5)
+    x = rand_inputs(rng, sh)
+    for g in range(sh.Hkv):  # very different KV heads: a wrong head shows at once
+        x["V"][:, g] += np.float32(7.0 * (g + 1))
+    for s in range(sh.S):
+        x["V"][s] += np.float32(50.0 * s)
+    n = sh.S * sh.Hq * sh.B
+    rows = rng.permutation(n)[: n - 7].astype(np.int32)
+    o_r, l_r = oracle.dense_rows(sh, x["Qc"], x["K"], x["V"], rows)
+    G = sh.Hq // sh.Hkv
+    for a, r in enumerate(rows):
+        s, rem = divmod(int(r), sh.Hq * sh.B)
+        h, t = divmod(rem, sh.B)
+        o, L = np_attend(x["Qc"][s, h, t], x["K"][s, h // G], x["V"][s, h // G], sh.scale)
+        close(o_r[a], o, 1e-6 * max(1.0, float(np.abs(o).max())), f"dense row {r} o_p vs numpy")
+        close(l_r[a], L, 1e-5, f"dense row {r} L_p vs numpy")
+    full = oracle.dense_prefix(sh, x["Qc"], x["K"], x["V"], x["Kb"], x["Vb"])
+    fo = full["o_p"].reshape(n, sh.d)[rows]
+    fl = full["l_p"].reshape(n)[rows]
+    assert np.array_equal(o_r.view(np.uint32), fo.view(np.uint32)), "dense rows != full pass"
+    assert np.array_equal(l_r.view(np.uint32), fl.view(np.uint32)), "dense rows L != full pass"
+
+
 def pin_gqa_mapping():
     """Query head h reads KV head h // G: make the KV heads very different."""
     rng = np.random.default_rng(18)

@@ -18,6 +18,7 @@ MUTATIONS = {
     10: "log-normaliser misses the running max",
     11: "drift-safe refresh writes the next token's row",
     12: "union variant attends to the row's own pages only",
+    13: "row-by-row dense pass decodes the head modulo Hkv instead of Hq",
 }
 
 
