@@ -276,16 +276,28 @@ int losa_step_ref(const losa_shape* shape, const void* q_cur, void* q_ref,
  *    per device, with that device current); make that first call before any
  *    stream capture on that device.
  *  - All calls on a device share the one array, which keeps whatever the
- *    last call left in it (losa_step needs nothing there to start at zero).
+ *    last call left in it.  losa_step needs nothing there to start at zero,
+ *    so those leftovers are harmless while every call ends with LOSA_OK;
+ *    read the device-side status with losa_noalloc_read_status.
  *    Calls that can overlap on the GPU -- on different streams without an
  *    ordering between them -- race on the array and give wrong results;
  *    order them on one stream or with events.
+ *  - The array's address is looked up once per device and kept; after a
+ *    cudaDeviceReset on that device the library's module (and the array)
+ *    is gone, and later calls in the same process are invalid.
  */
 int losa_step_noalloc(const losa_shape* shape, const void* q_cur, const void* q_prev,
                       const void* k_prefix, const void* v_prefix, const void* page_meta,
                       const void* k_blk, const void* v_blk, float* o_p, float* l_p, float* out,
                       float* out_lse, int32_t* active_idx, int32_t* page_idx,
                       int32_t* union_count, void* stream);
+
+/* losa_read_device_status for the scratch array of losa_step_noalloc on the
+ * current device: synchronises `stream`, returns the status the noalloc
+ * calls recorded there (LOSA_OK, LOSA_ERR_DEVICE_TIMEOUT or
+ * LOSA_ERR_DEVICE_BOUNDS) and clears it.  Allocates nothing.  The paper has
+ * no counterpart to this entry point either. */
+int losa_noalloc_read_status(void* stream);
 
 /* Synchronises `stream`, then returns the device-side status recorded in the
  * workspace by the last call that used it (LOSA_OK, LOSA_ERR_DEVICE_TIMEOUT

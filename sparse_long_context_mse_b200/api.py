@@ -33,7 +33,7 @@ LOSA_WS_STEP = 1
 EXPORTS = ("losa_page_meta_size", "losa_workspace_size", "losa_build_page_meta",
            "losa_dense_prefix", "losa_step", "losa_step_ref", "losa_step_noalloc",
            "losa_append_block",
-           "losa_read_device_status",
+           "losa_read_device_status", "losa_noalloc_read_status",
            "losa_status_string", "losa_last_error")
 
 #: size of the library-owned scratch behind ``losa_step_noalloc``
@@ -143,6 +143,8 @@ def lib():
         L.losa_step_ref.restype = i32
         L.losa_step_noalloc.argtypes = [sp] + [vp] * 14 + [vp]
         L.losa_step_noalloc.restype = i32
+        L.losa_noalloc_read_status.argtypes = [vp]
+        L.losa_noalloc_read_status.restype = i32
         L.losa_read_device_status.argtypes = [vp, vp]
         L.losa_read_device_status.restype = i32
         L.losa_status_string.argtypes = [i32]
@@ -333,3 +335,9 @@ def step_noalloc(sh: Shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk,
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:
     return lib().losa_read_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream(stream))
+
+
+def noalloc_read_status(stream=None) -> int:
+    """Device-side status of the ``losa_step_noalloc`` calls on the current
+    device (read and cleared; synchronises the stream)."""
+    return lib().losa_noalloc_read_status(_stream(stream))

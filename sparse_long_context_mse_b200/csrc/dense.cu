@@ -208,24 +208,27 @@ __global__ void __launch_bounds__(kFinishWarps * 32)
 
 // ---------------------------------------------------------------------------
 // bf16: 5th-generation tensor cores (tcgen05, accumulators in TMEM).
-// CTA = (split, group), 256 threads: two threads per query row of the group
-// (TMEM lane = row; rows >= G*B are padding), each with half of every tile's
-// keys and half of the output channels.  One thread drives the tensor core
-// and the TMA: 64-key K and V tiles arrive by 2-D tiled TMA loads in the
-// 128-byte-swizzled layout the matrix descriptors describe, K through a
-// 4-stage ring (a stage is free once the tile's scores are done), V through
-// a 3-stage ring (free once the tile's P V is done).  Per tile: S = Q K^T
-// (M=128, N=64, K=128) into one of two TMEM buffers, issued one tile ahead so
-// the tensor core runs while the threads do the softmax; every thread reads
-// its half row of S; the online softmax runs in base 2 (the halves exchange
-// row maxima through shared memory) against a reference max that moves only
-// when the row max grows by more than 2^8 (O and l are then rescaled in
-// TMEM); P goes to one of two shared-memory buffers in bf16, and the row sum
-// l adds the same rounded weights, so the output is an exactly normalised
-// average of the values under weights perturbed by at most 2^-9 relative;
-// then O += P V (M=128, N=128, K=64, V the MN-major operand).  A tile waits only for the
-// P V of two tiles back.  Every wait is bounded; a wait that gives up
-// records LOSA_ERR_DEVICE_TIMEOUT.
+// CTA = (split, group), 288 threads, one CTA per SM: eight softmax warps
+// (0-7) and a producer warp (8) whose lane 0 drives the TMA and the tensor
+// core.  The group's G*B query rows, zero-padded to MR = 64 or 128 MMA rows,
+// arrive once by 2-D tiled TMA in the 128-byte-swizzled layout the matrix
+// descriptors describe; 128-key K and V tiles stream through a 2-stage K
+// ring and a 2- (MR = 128) or 3-stage (MR = 64) V ring (the tensor maps'
+// 64-channel x 128-row boxes).  Per tile: S = Q K^T (M = MR, N = 128,
+// K = 128) into one of two TMEM score buffers, issued a tile ahead so the
+// tensor core runs while the softmax warps work; the softmax warps read S
+// from TMEM (MR = 64: the 16x256b fragment, two real rows per thread), run
+// the online softmax in base 2 (the two halves of a row exchange maxima
+// through shared memory) against a reference max that moves only when the
+// row max grows by more than 2^8 (O and l are then rescaled in TMEM), and
+// write P in bf16 to one of two shared-memory buffers; the row sum l adds the
+// same rounded weights, so the output is an exactly normalised average of
+// the values under weights perturbed by at most 2^-9 relative.  Then
+// O += P V (N = 128, K = 128: P in two K-major 64-key atoms, V the MN-major
+// operand) into a TMEM accumulator; every MMA group commits to an mbarrier.
+// At the end each thread writes its rows' O, m and l to the split partials.
+// Every wait is bounded; a wait that gives up records
+// LOSA_ERR_DEVICE_TIMEOUT.
 // ---------------------------------------------------------------------------
 constexpr int kUKeys = 128;                         // keys per tile (the S MMA's N)
 constexpr int kUHalf = kUKeys / 2;                  // keys of a tile per softmax warp
@@ -687,8 +690,14 @@ extern "C" int losa_dense_prefix(const losa_shape* shape, const void* q, const v
     return LOSA_ERR_INVALID_ARG;
   if (ws_bytes < d.total) return LOSA_ERR_INVALID_ARG;
   const size_t rows = static_cast<size_t>(d.S) * d.Hq * d.B;
-  const size_t qb = rows * kD * d.esz;
-  if (overlaps(out, rows * kD * 4, q, qb) || overlaps(out, rows * kD * 4, o_p, rows * kD * 4))
+  const size_t SG = static_cast<size_t>(d.S) * d.Hkv;
+  const size_t qb = rows * kD * d.esz, ob = rows * kD * sizeof(float), lb = rows * sizeof(float);
+  const size_t kvb = SG * d.Lc * kD * d.esz, kbb = SG * d.B * kD * d.esz;
+  const Region reg[] = {{q, qb, false},       {k_prefix, kvb, false}, {v_prefix, kvb, false},
+                        {k_blk, kbb, false},  {v_blk, kbb, false},    {o_p, ob, true},
+                        {l_p, lb, true},      {out, ob, true},        {out_lse, lb, true},
+                        {workspace, d.total, true}};
+  if (any_write_alias(reg, static_cast<int>(sizeof(reg) / sizeof(reg[0]))))
     return LOSA_ERR_INVALID_ARG;
   if (d.S * d.Hkv > 65535) return LOSA_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -227,6 +227,21 @@ inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// A buffer an entry point reads or writes: base, bytes, whether it is written.
+struct Region {
+  const void* p;
+  size_t n;
+  bool w;
+};
+// Whether two of the regions overlap where at least one of the two is written
+// (read-only inputs may alias each other; a null region is skipped).
+inline bool any_write_alias(const Region* r, int n) {
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j)
+      if ((r[i].w || r[j].w) && overlaps(r[i].p, r[i].n, r[j].p, r[j].n)) return true;
+  return false;
+}
+
 int make_dims(const losa_shape* sh, int which, Dims* d);
 // Whether the fused step kernel's shared-memory plan fits in `max_dyn` bytes.
 bool fused_step_fits(const Dims& d, int max_dyn);

@@ -66,8 +66,19 @@ extern "C" int losa_step_noalloc(const losa_shape* shape, const void* q_cur, con
   const int rc = scratch_address(&scratch);
   if (rc != LOSA_OK) return rc;
   // losa_step needs nothing in its workspace to start at zero, so the
-  // previous call's leftovers are harmless
+  // previous call's leftovers are harmless as long as the calls ended with
+  // LOSA_OK (losa_noalloc_read_status tells)
   return losa_step(shape, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p, l_p,
                    out, out_lse, active_idx, page_idx, union_count, scratch,
                    static_cast<size_t>(LOSA_NOALLOC_SCRATCH_BYTES), stream);
+}
+
+extern "C" int losa_noalloc_read_status(void* stream) {
+  using namespace losa;
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != LOSA_OK) return rc;
+  // the status word sits at the start of a step workspace, and so at the
+  // start of the scratch array
+  return losa_read_device_status(scratch, stream);
 }

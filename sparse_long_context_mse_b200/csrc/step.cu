@@ -1,5 +1,5 @@
 // step.cu -- C entry points of one LoSA denoising step (plain and drift-safe):
-// host validation, then the two step kernels of step_fused.cu.
+// host validation, then the step kernels of step_fused.cu.
 #include "losa_common.cuh"
 
 namespace {
@@ -20,18 +20,24 @@ int step_common(const losa_shape* shape, const void* q_cur, const void* q_prev, 
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return LOSA_ERR_INVALID_ARG;
   if (ws_bytes < d.total) return LOSA_ERR_INVALID_ARG;
+  // no written buffer may overlap another buffer of the call (q_ref is
+  // q_prev, read and then rewritten, in the drift-safe variant)
   const size_t rows = static_cast<size_t>(d.S) * d.Hq * d.B;
-  const size_t ob = rows * kD * sizeof(float), qb = rows * kD * d.esz;
-  if (overlaps(out, ob, q_cur, qb) || overlaps(out, ob, q_prev, qb) || overlaps(out, ob, o_p, ob) ||
-      overlaps(out, ob, l_p, rows * sizeof(float)))
+  const size_t SG = static_cast<size_t>(d.S) * d.Hkv;
+  const size_t ob = rows * kD * sizeof(float), lb = rows * sizeof(float);
+  const size_t qb = rows * kD * d.esz, kvb = SG * d.Lc * kD * d.esz, kbb = SG * d.B * kD * d.esz;
+  const size_t mb = SG * d.Pc * 2 * kD * d.esz;
+  const size_t ab = static_cast<size_t>(d.S) * d.Hq * d.A * sizeof(int32_t);
+  const Region reg[] = {{q_cur, qb, false},       {q_prev, qb, q_ref_out != nullptr},
+                        {k_prefix, kvb, false},   {v_prefix, kvb, false},
+                        {page_meta, mb, false},   {k_blk, kbb, false},
+                        {v_blk, kbb, false},      {o_p, ob, true},
+                        {l_p, lb, true},          {out, ob, true},
+                        {out_lse, lb, true},      {active_idx, ab, true},
+                        {page_idx, ab * d.k, true}, {union_count, SG * sizeof(int32_t), true},
+                        {workspace, d.total, true}};
+  if (any_write_alias(reg, static_cast<int>(sizeof(reg) / sizeof(reg[0]))))
     return LOSA_ERR_INVALID_ARG;
-  if (q_ref_out) {  // the reference is rewritten: it may alias nothing else
-    const size_t lb = rows * sizeof(float);
-    if (overlaps(q_ref_out, qb, q_cur, qb) || overlaps(q_ref_out, qb, o_p, ob) ||
-        overlaps(q_ref_out, qb, l_p, lb) || overlaps(q_ref_out, qb, out, ob) ||
-        (out_lse && overlaps(q_ref_out, qb, out_lse, lb)))
-      return LOSA_ERR_INVALID_ARG;
-  }
   if (d.S * d.Hkv > 65535) return LOSA_ERR_UNSUPPORTED;
   return launch_fused_step(d, q_cur, q_prev, k_prefix, v_prefix, page_meta, k_blk, v_blk, o_p,
                            l_p, out, out_lse, active_idx, page_idx, union_count, workspace,

@@ -49,6 +49,15 @@ def S(**kw):
     return api.make_shape(**base)
 
 
+@pytest.fixture
+def no_device():
+    """Validation tests that pass fake addresses: a call that wrongly passed
+    validation would launch on them, so they run only without a GPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses: CPU-only validation test")
+
+
 def test_status_strings(L):
     for code in range(6):
         assert api.status_string(code)
@@ -112,10 +121,14 @@ def _step_args(ptrs):
     return [ctypes.c_void_p(p) if p is not None else None for p in ptrs]
 
 
-def test_pointer_validation(L):
+# fake device addresses 64 GiB apart: no two buffers of a call overlap
+FAR = [(i + 1) << 36 for i in range(16)]
+
+
+def test_pointer_validation(L, no_device):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_STEP)
-    base = [0x100000 * (i + 1) for i in range(10)] + [None, None, None, None, 0x7f0000000000]
+    base = FAR[:10] + [None, None, None, None, FAR[14]]
 
     def call(ptrs, ws_bytes=ws_n):
         return L.losa_step(ctypes.byref(sh), *_step_args(ptrs), ws_bytes, None)
@@ -133,13 +146,32 @@ def test_pointer_validation(L):
     p = list(base)
     p[11] = 0x900004                     # optional output misaligned
     assert call(p) == api.LOSA_ERR_INVALID_ARG
-    p = list(base)
-    p[9] = p[0]                          # out aliases q_cur
-    assert call(p) == api.LOSA_ERR_INVALID_ARG
     assert L.losa_step(None, *_step_args(base), ws_n, None) == api.LOSA_ERR_INVALID_ARG
 
 
-def test_step_flags_validation(L):
+# (written buffer, other buffer) index pairs of losa_step's pointer list:
+# 0 q_cur 1 q_prev 2 k_prefix 3 v_prefix 4 page_meta 5 k_blk 6 v_blk 7 o_p
+# 8 l_p 9 out 10 out_lse 11 active_idx 12 page_idx 13 union_count 14 workspace
+STEP_ALIASES = [(9, 0), (9, 2), (9, 3), (9, 4), (9, 5), (9, 6), (9, 7), (9, 14), (10, 1),
+                (10, 8), (10, 14), (7, 14), (8, 14), (7, 2), (8, 4), (11, 12), (12, 14),
+                (13, 3), (11, 7)]
+
+
+@pytest.mark.parametrize("w,o", STEP_ALIASES)
+def test_step_refuses_written_aliases(L, w, o, no_device):
+    # a written buffer overlapping any other buffer of the call is refused
+    # before anything is launched; the address sits inside the other buffer
+    # (with fake addresses a call that passed validation would launch, so the
+    # test only runs where there is no device to launch on)
+    sh = S()
+    ws_n = api.workspace_size(sh, api.LOSA_WS_STEP)
+    p = list(FAR[:15])
+    p[w] = p[o] + 16             # 16 bytes into the other buffer (every one is larger)
+    rc = L.losa_step(ctypes.byref(sh), *_step_args(p), ws_n, None)
+    assert rc == api.LOSA_ERR_INVALID_ARG
+
+
+def test_step_flags_validation(L, no_device):
     # the union variant is a legal step shape; an unknown bit is refused
     # before anything is launched
     assert api.workspace_size(S(flags=api.LOSA_STEP_ATTEND_UNION), api.LOSA_WS_STEP) > 0
@@ -150,12 +182,12 @@ def test_step_flags_validation(L):
                        1 << 40, None) == api.LOSA_ERR_INVALID_ARG
 
 
-def test_step_ref_pointer_validation(L):
+def test_step_ref_pointer_validation(L, no_device):
     # losa_step_ref rewrites q_ref: null, or aliasing any output or q_cur, is
     # refused before anything is launched
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_STEP)
-    base = [0x100000 * (i + 1) for i in range(10)] + [None, None, None, None, 0x7f0000000000]
+    base = FAR[:10] + [None, None, None, None, FAR[14]]
 
     def call(ptrs):
         return L.losa_step_ref(ctypes.byref(sh), *_step_args(ptrs), ws_n, None)
@@ -169,7 +201,7 @@ def test_step_ref_pointer_validation(L):
     assert call(p) == api.LOSA_ERR_INVALID_ARG
 
 
-def test_prefix_capacity_validation(L):
+def test_prefix_capacity_validation(L, no_device):
     # a capacity below the prefix length is refused; a larger one grows the
     # metadata to ceil(capacity / ps) records per (s, g)
     assert api.workspace_size(S(prefix_capacity=65535), api.LOSA_WS_STEP) == 0
@@ -223,10 +255,10 @@ def test_prefix_lens_on_another_device_is_refused(L):
     assert api._call_device(S(), t) == torch.device("cuda", 0)
 
 
-def test_dense_pointer_validation(L):
+def test_dense_pointer_validation(L, no_device):
     sh = S()
     ws_n = api.workspace_size(sh, api.LOSA_WS_DENSE)
-    base = [0x100000 * (i + 1) for i in range(9)] + [0x7f0000000000]
+    base = FAR[:9] + [FAR[14]]
     for i in range(8):
         p = list(base)
         p[i] = None
@@ -234,6 +266,12 @@ def test_dense_pointer_validation(L):
         assert rc == api.LOSA_ERR_INVALID_ARG
     rc = L.losa_dense_prefix(ctypes.byref(sh), *_step_args(base), ws_n - 256, None)
     assert rc == api.LOSA_ERR_INVALID_ARG
+    # 0 q 1 k_prefix 2 v_prefix 3 k_blk 4 v_blk 5 o_p 6 l_p 7 out 8 out_lse 9 workspace
+    for w, o in ((7, 0), (7, 1), (7, 5), (8, 9), (5, 2), (6, 3), (5, 9), (8, 6)):
+        p = list(base)
+        p[w] = p[o] + 16
+        rc = L.losa_dense_prefix(ctypes.byref(sh), *_step_args(p), ws_n, None)
+        assert rc == api.LOSA_ERR_INVALID_ARG, (w, o)
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
