@@ -1,8 +1,11 @@
 // abi.cu -- host side of the C ABI: shape validation, workspace layout,
 // status reporting.  No kernel lives here.
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "losa_common.cuh"
@@ -22,6 +25,29 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 int record_cuda_error(cudaError_t e) {
   g_last_error = std::string(cudaGetErrorName(e)) + ": " + cudaGetErrorString(e);
   return LOSA_ERR_CUDA;
+}
+
+int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsigned box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return LOSA_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), nrows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  const cuuint32_t box[2] = {64u, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LOSA_OK : LOSA_ERR_CUDA;
 }
 
 int num_sms() {
@@ -97,31 +123,8 @@ int make_dims(const losa_shape* sh, int which, Dims* d) {
     return LOSA_OK;
   }
   if (which != LOSA_WS_STEP) return LOSA_ERR_INVALID_ARG;
-  // step: the scan splits each group's pages into chunks so that the whole
-  // grid covers the SMs once; a chunk's bound scores live in shared memory
-  const size_t R = static_cast<size_t>(d->R), K = static_cast<size_t>(d->k);
-  {
-    const long long per_group = std::max<long long>(1, kSizingSms / static_cast<long long>(SG));
-    long long chunk = (P + per_group - 1) / per_group;
-    chunk = (chunk + 7) / 8 * 8;
-    const long long cap = std::max<long long>(8, (16384 / std::max(d->R, 1)) / 8 * 8);
-    chunk = std::min(chunk, cap);
-    d->chunk_pages = static_cast<int>(chunk);
-    d->nchunk = static_cast<int>((P + chunk - 1) / chunk);
-  }
-  // workspace: status word, the active set of every group (active tokens,
-  // then every token's active slot or -1), and the chunk candidates
-  // (selection keys) of every (group, chunk, active row)
-  d->off_act = off;
-  off += align256(SG * (R + static_cast<size_t>(G) * d->B) * sizeof(int32_t));
-  d->off_cand = off;
-  off += align256(SG * d->nchunk * R * K * sizeof(unsigned long long));
-  // the gather kernel's row partials (every CTA of a group), the active
-  // rows' suffixes
-  d->off_gpart = off;
-  off += align256(SG * kGatherCtas * R * kPartStride * sizeof(float));
-  d->off_gsfx = off;
-  off += align256(SG * R * kPartStride * sizeof(float));
+  // step: one cluster per group keeps its whole state in shared memory; the
+  // workspace holds only the status word
   d->total = off;
   // the fused step keeps each group's selection state in shared memory
   if (!fused_step_fits(*d, kB200MaxDynSmem)) return LOSA_ERR_UNSUPPORTED;

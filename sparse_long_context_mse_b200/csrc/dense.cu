@@ -9,9 +9,6 @@
 // the dense suffix over the block's own keys and writes cache and output.
 // bf16 runs on the 5th-generation tensor cores (tcgen05, TMEM), fp32 on
 // CUDA cores.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "losa_common.cuh"
@@ -249,15 +246,6 @@ struct UPlan {
                               nbars * 8 + 16;
 };
 static_assert(UPlan<64>::smem <= 232448 && UPlan<128>::smem <= 232448, "dense plan > 227 KB");
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
-      "{%2, %3}], [%4];" ::"r"(su32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(su32(bar))
-      : "memory");
-}
 
 template <int MR>
 __global__ void __launch_bounds__(288, 1)
@@ -646,31 +634,6 @@ __global__ void __launch_bounds__(288, 1)
   __syncthreads();
   if (tid == 0 && *s_fail) atomicCAS(status, 0, LOSA_ERR_DEVICE_TIMEOUT);
   if (warp == 0) tmem_dealloc(tbase, kUCols);
-}
-
-// 2-D tensor map over a [rows][128] bf16 tensor for 128-byte-swizzled boxes
-// of 64 channels x box_rows rows.
-int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsigned box_rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  if (!encode) return LOSA_ERR_CUDA;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), nrows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
-  const cuuint32_t box[2] = {64u, box_rows};
-  const cuuint32_t estr[2] = {1u, 1u};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? LOSA_OK : LOSA_ERR_CUDA;
 }
 
 }  // namespace

@@ -5,6 +5,7 @@
 // selection keys).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -19,7 +20,6 @@ constexpr int kMaxB = 32;       // block tokens (one warp lane per token)
 constexpr int kMaxRowsPerGroup = 128;  // G*B (and hence G*A) per KV head
 constexpr int kMaxK = 64;       // pages per active row unless every page is taken
 constexpr int kPartStride = kD + 4;    // floats per split-softmax partial: m, l, pad, pad, acc[d]
-constexpr int kGatherCtas = 16;        // CTAs per (sequence, KV head) in the step's gather kernel
 constexpr int kMaxDevices = 64;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -35,11 +35,10 @@ struct Dims {
   const int32_t* lens;    // per-sequence prefix lengths (device, [S]) or null: every one is L
   float scale;            // softmax scale (natural-log units)
   float scale_log2;       // scale * log2(e): scores in base-2 units
-  // prefix splits (dense pass); page chunks of the step's scan
+  // prefix splits (dense pass)
   int nsplit, split_pages;
-  int nchunk, chunk_pages;
   // workspace byte offsets
-  size_t off_status, off_part, off_act, off_cand, off_gpart, off_gsfx, total;
+  size_t off_status, off_part, total;
 };
 
 // Element load as float (bf16 -> f32 is exact).
@@ -254,6 +253,10 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
                       int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
                       void* workspace, cudaStream_t st, void* q_ref_out = nullptr);
 int record_cuda_error(cudaError_t e);  // stores the message, returns LOSA_ERR_CUDA
+// 2-D tensor map over a [nrows][128] bf16 tensor at `base`, for
+// 128-byte-swizzled boxes of 64 channels x box_rows rows (rows past nrows
+// read as zero).  LOSA_OK, or LOSA_ERR_CUDA if the driver refuses it.
+int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsigned box_rows);
 int num_sms();
 
 }  // namespace losa
