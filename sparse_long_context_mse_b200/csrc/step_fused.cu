@@ -64,10 +64,9 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kStageBytes = 32 * 1024;
 constexpr int kMinStages = 2;
 constexpr int kMaxStages = 6;
-constexpr int kListSlack = 8;       // list entries beyond k before an exact refinement
-constexpr int kEpl = 16;            // list entries per lane in a list update
+constexpr int kListSlack = 4;       // buffer entries beyond k kept after a compaction before an exact refinement
 constexpr int kMaxGatherPages = 16; // union pages in flight per CTA
-constexpr int kEpsExp = -14;        // interval half-width: 2^-14 * sum of the terms' magnitudes
+constexpr float kEpsScale = 6.103515625e-05f;  // 2^-14: interval half-width per unit of sum |terms|
 constexpr int kRecSlots = 8;        // records staged at once per merge warp for exact rescoring
 
 typedef unsigned long long u64;
@@ -146,26 +145,6 @@ __device__ __forceinline__ void attend_page(float4 q, const char* Ks, const char
   acc = o;
   l = l * alpha + psum;
   m = m_new;
-}
-
-// The k-th largest (1 <= k <= W) of the values held by the W lanes of an
-// aligned lane group (W a power of two, the same for the whole warp): every
-// lane ranks its value against the group's (ties by lane), and the lane of
-// rank k-1 holds the answer.  The W shuffles are independent, so they
-// overlap instead of forming a chain.
-__device__ __forceinline__ unsigned long long group_kth_u64(unsigned long long v, int W, int k) {
-  const int lane = threadIdx.x & 31, j = lane & (W - 1), base = lane - j;
-  int rk = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    if (i < W) {
-      const unsigned long long o = __shfl_sync(0xffffffffu, v, base + i);
-      rk += (o > v) || (o == v && i < j);
-    }
-  }
-  const unsigned bal = __ballot_sync(0xffffffffu, rk == k - 1);
-  const unsigned grp = W == 32 ? bal : ((bal >> base) & ((1u << W) - 1u));
-  return __shfl_sync(0xffffffffu, v, base + __ffs(grp) - 1);
 }
 
 // Byte offset of 16-byte chunk c of row j inside a [rows][kD] tile: bf16 tiles
@@ -332,7 +311,7 @@ __device__ __forceinline__ void lse_weights(float L1, float L2, float& a, float&
 // (rounded outward), so lk <= the page's true key <= uk.  t = 0 (an exact
 // score) gives lk == uk == the exact key.
 __device__ __forceinline__ void entry_keys(float u, float t, int p, u64& lk, u64& uk) {
-  const float e = ldexpf(t, kEpsExp);
+  const float e = __fmul_ru(t, kEpsScale);  // >= 2^-14 t (exact unless subnormal)
   lk = sel_key(__fsub_rd(u, e), p);
   uk = sel_key(__fadd_ru(u, e), p);
 }
@@ -380,6 +359,9 @@ __device__ __forceinline__ void bound_ntile2(const uint32_t (&a)[16][4], const c
   const int lane = threadIdx.x & 31;
   const int pg = lane & 7;
   constexpr uint32_t kAbs = 0x7fff7fffu;
+  // two accumulator chains each (even / odd k-steps), added at the end: half
+  // the dependent MMA latency
+  float u1[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
   u[0] = u[1] = u[2] = u[3] = 0.f;
   t[0] = t[1] = t[2] = t[3] = 0.f;
 #pragma unroll
@@ -388,63 +370,194 @@ __device__ __forceinline__ void bound_ntile2(const uint32_t (&a)[16][4], const c
     const int ch = ks * 2 + (lane >> 3);
     ldsm_x4(su32(rec0 + pg * 512 + ((ch ^ pg) << 4)), b0, b1, b2, b3);
     mma_bf16(u, a[ks], b0, b1);
-    mma_bf16(u, a[ks + 1], b2, b3);
+    mma_bf16(u1, a[ks + 1], b2, b3);
     const uint32_t x0[4] = {a[ks][0] & kAbs, a[ks][1] & kAbs, a[ks][2] & kAbs, a[ks][3] & kAbs};
     const uint32_t x1[4] = {a[ks + 1][0] & kAbs, a[ks + 1][1] & kAbs, a[ks + 1][2] & kAbs,
                             a[ks + 1][3] & kAbs};
     mma_bf16(t, x0, b0 & kAbs, b1 & kAbs);
-    mma_bf16(t, x1, b2 & kAbs, b3 & kAbs);
+    mma_bf16(t1, x1, b2 & kAbs, b3 & kAbs);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    u[i] += u1[i];
+    t[i] += t1[i];
   }
 }
 
 // ---------------------------------------------------------------------------
-// Per-row candidate lists.  Row r's list holds, sorted by lower key
-// (descending), every page seen so far whose upper key reaches the k-th
-// largest lower key seen so far (thr[r]; 0 while fewer than k pages were
-// seen): the pages that can still be among the row's top k.
+// Per-row candidate buffers.  Row r's buffer holds, unsorted, every page seen
+// so far whose upper key reaches thr[r], a lower bound of the k-th largest
+// lower key seen so far (0 while fewer than k pages were seen): a superset of
+// the pages that can still be among the row's top k.  A group of w lanes
+// (aligned in its warp) serves each row: rows r = pass * (threads / w) +
+// tid / w, in as many passes as the rows need.
 // ---------------------------------------------------------------------------
 struct ListCtx {
-  u64* lk;   // [R][lb] lower keys
-  u64* uk;   // [R][lb] upper keys
-  int* n;    // [R] entries
-  u64* thr;  // [R] k-th largest lower key
-  int lb;    // entries per row buffer (cap + pages per update)
-  int cap;   // entries kept before the list's inexact entries are rescored
-  int w;     // lanes per row (a power of two); rows r = tid / w
+  u64* lk;    // [R][lb] lower keys
+  u64* uk;    // [R][lb] upper keys
+  int* n;     // [R] entries
+  u64* thr;   // [R] threshold
+  u64* scr;   // [threads / w][sstride] per-group scratch (sub-maxima, survivors, broadcast)
+  int lb;     // entries per row buffer
+  int cap;    // entries kept after the last compaction before an exact refinement
+  int sstride;
+  int w;      // lanes per row (a power of two)
 };
 
-// Add np newly scored pages pbase .. pbase + np - 1 (scores u = sU[r][e],
-// magnitudes t = sT[r][e]) to the lists of rows 0..R-1.  Every thread of the
-// CTA calls it.
+// The k-th largest of the keys a[0..n) (distinct; 0 if n < k), computed by
+// the w lanes of a row group.  A lower bound first -- the k-th largest of
+// the lanes' sub-maxima (each lane keeps V = ceil(k / w) of them, so there
+// are at least k) -- then an exact rank among the keys at or above it, which
+// are few.  Every lane of the warp calls it (`act` false for a group without
+// a row); scr holds w * V + 1 + n keys.
+__device__ u64 group_kth(const u64* a, int n, int k, int w, bool act, u64* scr) {
+  const int lane = threadIdx.x & 31, j = lane & (w - 1);
+  const unsigned gmask = w == 32 ? 0xffffffffu : (((1u << w) - 1u) << (lane & ~(w - 1)));
+  const unsigned lt = (1u << lane) - 1u;
+  const int V = (k + w - 1) / w;
+  const int nw = __reduce_max_sync(0xffffffffu, act ? n : 0);
+  u64* sub = scr;
+  u64* bc = scr + w * V;
+  u64* sv = bc + 1;
+  if (act) {
+    for (int v = 0; v < V; ++v) {
+      u64 m = 0;
+      for (int i = j + w * v; i < n; i += w * V) m = a[i] > m ? a[i] : m;
+      sub[j * V + v] = m;
+    }
+    if (j == 0) *bc = 0ull;
+  }
+  __syncwarp();
+  if (act && n >= k) {
+    for (int v = 0; v < V; ++v) {
+      const u64 x = sub[j * V + v];
+      int rk = 0;
+      for (int q = 0; q < w * V; ++q) {
+        const u64 y = sub[q];
+        rk += (y > x) || (y == x && q < j * V + v);
+      }
+      if (rk == k - 1) *bc = x;
+    }
+  }
+  __syncwarp();
+  const u64 t1 = act ? *bc : 0ull;
+  // the keys at or above the lower bound (they hold the k largest)
+  int ns = 0;
+  for (int i0 = 0; i0 < nw; i0 += w) {
+    const int i = i0 + j;
+    const bool in = act && i < n && a[i] >= t1;
+    const unsigned bal = __ballot_sync(0xffffffffu, in) & gmask;
+    if (in) sv[ns + __popc(bal & lt)] = a[i];
+    ns += __popc(bal);
+  }
+  __syncwarp();
+  if (act && j == 0) *bc = 0ull;
+  __syncwarp();
+  if (act && n >= k) {
+    for (int i = j; i < ns; i += w) {
+      const u64 x = sv[i];
+      int rk = 0;
+      for (int q = 0; q < ns; ++q) rk += sv[q] > x;
+      if (rk == k - 1) *bc = x;
+    }
+  }
+  __syncwarp();
+  const u64 r = act ? *bc : 0ull;
+  __syncwarp();
+  return r;
+}
+
+// Keep the entries of a row's buffer whose upper key reaches `thr`
+// (compaction in place, order kept); returns the new count.
+__device__ int buffer_keep(u64* lk, u64* uk, int n, u64 thr, int w, bool act) {
+  const int lane = threadIdx.x & 31, j = lane & (w - 1);
+  const unsigned gmask = w == 32 ? 0xffffffffu : (((1u << w) - 1u) << (lane & ~(w - 1)));
+  const unsigned lt = (1u << lane) - 1u;
+  const int nw = __reduce_max_sync(0xffffffffu, act ? n : 0);
+  int kept = 0;
+  for (int i0 = 0; i0 < nw; i0 += w) {
+    const int i = i0 + j;
+    u64 a = 0, b = 0;
+    bool keep = false;
+    if (act && i < n) {
+      a = lk[i];
+      b = uk[i];
+      keep = b >= thr;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep) & gmask;
+    __syncwarp();
+    if (keep) {
+      const int pos = kept + __popc(bal & lt);
+      lk[pos] = a;
+      uk[pos] = b;
+    }
+    kept += __popc(bal);
+    __syncwarp();
+  }
+  return kept;
+}
+
+// Compaction of the rows with `act`: the exact k-th largest lower key
+// becomes the threshold and only the entries whose upper key reaches it stay;
+// a row left with more than `cap` entries (near-ties at the boundary) has its
+// inexact entries rescored exactly (the oracle's arithmetic) and is compacted
+// again, which leaves min(k, n) exact entries.
 template <int DT>
-__device__ __noinline__ void list_update(const ListCtx L, int R, int k, const float* sU,
-                                         const float* sT, int ts, int np, int pbase,
-                                         const char* qa, const char* meta_g) {
+__device__ void buffer_compact(const ListCtx& L, int r, int k, bool act, const char* qa,
+                               const char* meta_g) {
+  const int j = (threadIdx.x & 31) & (L.w - 1);
+  const int rr = act ? r : 0;
+  u64* lk = L.lk + static_cast<size_t>(rr) * L.lb;
+  u64* uk = L.uk + static_cast<size_t>(rr) * L.lb;
+  u64* scr = L.scr + static_cast<size_t>(threadIdx.x / L.w) * L.sstride;
+  int n = act ? L.n[r] : 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const u64 th = group_kth(lk, n, k, L.w, act, scr);
+    const int nk = buffer_keep(lk, uk, n, th, L.w, act);
+    if (act) n = nk;
+    if (act && j == 0) L.thr[r] = th > L.thr[r] ? th : L.thr[r];
+    const bool over = act && n > L.cap;
+    if (DT != LOSA_BF16 || !__any_sync(0xffffffffu, over)) break;
+    if (over) {
+      for (int i = j; i < n; i += L.w)
+        if (lk[i] != uk[i]) {
+          const int p = key_index(lk[i]);
+          const float v = exact_bound_bf16(qa + r * 256, r, meta_g + static_cast<size_t>(p) * 512, p);
+          lk[i] = uk[i] = sel_key(v, p);
+        }
+    }
+    __syncwarp();
+  }
+  __syncwarp();
+  if (act && j == 0) L.n[r] = n;
+  __syncwarp();
+}
+
+// Add np newly scored pages pbase .. pbase + np - 1 (score u = sU[r][e],
+// magnitude t = sT[r][e]) to the buffers of rows 0..R-1: the threshold
+// rises to the k-th largest sub-maximum of the new lower keys (a lower bound
+// of their k-th largest), the new pages whose upper key reaches it join the
+// buffer, and a buffer that could not take another np pages is compacted.
+// Every thread of the CTA calls it.
+template <int DT>
+__device__ __forceinline__ void list_add_rows(const ListCtx& L, int r, int R, int k,
+                                              const float* sU, const float* sT, int ts, int np,
+                                              int pbase, const char* qa, const char* meta_g) {
   const int tid = threadIdx.x, lane = tid & 31, W = L.w;
-  const int j = tid & (W - 1), r = tid / W;
+  const int j = tid & (W - 1);
   const bool act = r < R;
   const unsigned gmask = W == 32 ? 0xffffffffu : (((1u << W) - 1u) << (lane & ~(W - 1)));
   const unsigned lt = (1u << lane) - 1u;
   const int rr = act ? r : 0;
   u64* lk = L.lk + static_cast<size_t>(rr) * L.lb;
   u64* uk = L.uk + static_cast<size_t>(rr) * L.lb;
+  u64* scr = L.scr + static_cast<size_t>(tid / W) * L.sstride;
   const float* ur = sU + rr * ts;
   const float* tr = sT + rr * ts;
-  const int n = act ? L.n[r] : 0;
-  // 1. filter: the running threshold, tightened by the k-th largest lane
-  //    maximum of the new lower keys (at most the new pages' k-th largest)
-  u64 tau = act ? L.thr[r] : 0ull;
-  if (k <= W && np >= k) {
-    u64 lmax = 0;
-    for (int e = j; e < np; e += W) {
-      u64 a, b;
-      entry_keys(ur[e], tr[e], pbase + e, a, b);
-      lmax = a > lmax ? a : lmax;
-    }
-    const u64 tl = group_kth_u64(act ? lmax : 0ull, W, k);
-    tau = tl > tau ? tl : tau;
-  }
-  // 2. the new pages whose upper key reaches it join the list
+  int n = act ? L.n[r] : 0;
+  u64 thr = act ? L.thr[r] : 0ull;
+  // 1. the new pages whose upper key reaches the running threshold join
   int m = 0;
   for (int e0 = 0; e0 < np; e0 += W) {
     const int e = e0 + j;
@@ -452,7 +565,7 @@ __device__ __noinline__ void list_update(const ListCtx L, int R, int k, const fl
     bool sv = false;
     if (act && e < np) {
       entry_keys(ur[e], tr[e], pbase + e, a, b);
-      sv = b >= tau;
+      sv = b >= thr;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, sv) & gmask;
     if (sv) {
@@ -462,80 +575,60 @@ __device__ __noinline__ void list_update(const ListCtx L, int R, int k, const fl
     }
     m += __popc(bal);
   }
+  n += m;
   __syncwarp();
-  int N = n + m;
-  u64 nthr = 0;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    // 3. rank sort by lower key, descending (keys are distinct: they hold
-    //    the page index)
-    u64 rl[kEpl], ru[kEpl];
-    int rk[kEpl];
-#pragma unroll
-    for (int t = 0; t < kEpl; ++t) {
-      const int i = j + t * W;
-      rk[t] = -1;
-      rl[t] = ru[t] = 0;
-      if (act && i < N) {
-        rl[t] = lk[i];
-        ru[t] = uk[i];
-        int cnt = 0;
-#pragma unroll 4
-        for (int i2 = 0; i2 < N; ++i2) cnt += lk[i2] > rl[t];
-        rk[t] = cnt;
+  // 2. a buffer that could not take another np pages: the threshold rises to
+  //    the k-th largest of the lanes' V sub-maxima of its lower keys (a lower
+  //    bound of its k-th largest) and only the entries reaching it stay
+  const bool full = act && n + ts > L.lb;
+  if (__any_sync(0xffffffffu, full)) {
+    const int V = (k + W - 1) / W;
+    if (full) {
+      for (int v = 0; v < V; ++v) {
+        u64 mx = 0;
+        for (int i = j + W * v; i < n; i += W * V) mx = lk[i] > mx ? lk[i] : mx;
+        scr[j * V + v] = mx;
       }
     }
     __syncwarp();
-#pragma unroll
-    for (int t = 0; t < kEpl; ++t)
-      if (rk[t] >= 0) {
-        lk[rk[t]] = rl[t];
-        uk[rk[t]] = ru[t];
-      }
-    __syncwarp();
-    // 4. the k-th largest lower key, and the entries whose upper key reaches it
-    nthr = (act && N >= k) ? lk[k - 1] : 0ull;
-    const int Nw = __reduce_max_sync(0xffffffffu, act ? N : 0);
-    int kept = 0;
-    for (int i0 = 0; i0 < Nw; i0 += W) {
-      const int i = i0 + j;
-      u64 a = 0, b = 0;
-      bool keep = false;
-      if (act && i < N) {
-        a = lk[i];
-        b = uk[i];
-        keep = b >= nthr;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep) & gmask;
-      __syncwarp();
-      if (keep) {
-        const int pos = kept + __popc(bal & lt);
-        lk[pos] = a;
-        uk[pos] = b;
-      }
-      kept += __popc(bal);
-      __syncwarp();
-    }
-    N = kept;
-    // 5. a list longer than its capacity (near-ties at the boundary): its
-    //    inexact entries are rescored exactly, then it is sorted and pruned
-    //    again and holds exactly min(k, N) exact entries
-    const bool over = act && N > L.cap;
-    if (!__any_sync(0xffffffffu, over)) break;
-    if (DT == LOSA_BF16 && over) {
-      for (int i = j; i < N; i += W)
-        if (lk[i] != uk[i]) {
-          const int p = key_index(lk[i]);
-          const float v = exact_bound_bf16(qa + r * 256, r, meta_g + static_cast<size_t>(p) * 512, p);
-          lk[i] = uk[i] = sel_key(v, p);
+    u64 t2 = 0;
+    if (full && n >= k) {
+      for (int v = 0; v < V; ++v) {
+        const u64 x = scr[j * V + v];
+        int rk = 0;
+        for (int q = 0; q < W * V; ++q) {
+          const u64 y = scr[q];
+          rk += (y > x) || (y == x && q < j * V + v);
         }
+        if (rk == k - 1) t2 = x;
+      }
     }
-    __syncwarp();
+    for (int o = 1; o < W; o <<= 1) {
+      const u64 y = __shfl_xor_sync(0xffffffffu, t2, o);
+      t2 = y > t2 ? y : t2;
+    }
+    thr = t2 > thr ? t2 : thr;
+    const int nk = buffer_keep(lk, uk, n, thr, W, full);
+    if (full) n = nk;
   }
   if (act && j == 0) {
-    L.n[r] = N;
-    L.thr[r] = nthr;
+    L.n[r] = n;
+    L.thr[r] = thr;
   }
+  __syncwarp();
+  // 3. still too full (many near-equal keys): exact compaction
+  const bool still = act && n + ts > L.lb;
+  if (__any_sync(0xffffffffu, still)) buffer_compact<DT>(L, r, k, still, qa, meta_g);
+}
+
+template <int DT>
+__device__ __forceinline__ void list_add(const ListCtx& L, int R, int k, const float* sU,
+                                         const float* sT, int ts, int np, int pbase,
+                                         const char* qa, const char* meta_g) {
+#pragma unroll 1
+  for (int r0 = 0; r0 < R; r0 += kThreads / L.w)
+    list_add_rows<DT>(L, r0 + static_cast<int>(threadIdx.x) / L.w, R, k, sU, sT, ts, np, pbase,
+                      qa, meta_g);
 }
 
 // ---------------------------------------------------------------------------
@@ -543,7 +636,8 @@ __device__ __noinline__ void list_update(const ListCtx L, int R, int k, const fl
 // the row's k pages, exactly the oracle's top k (value descending, lower page
 // first), written ascending to sel[0..k) (then -1 when the sequence has fewer
 // pages).  `buf` is the warp's scratch: lk[cap_all], uk[cap_all],
-// kRecSlots staged records of 512 bytes, flag[cap_all].
+// kRecSlots staged records of 512 bytes, flag[cap_all], then the k-th
+// selection's scratch (32 * ceil(k / 32) + 1 + cap_all keys).
 // ---------------------------------------------------------------------------
 struct MergeCtx {
   const u64* lk;   // this CTA's list arrays (the same offsets in every CTA)
@@ -557,13 +651,14 @@ struct MergeCtx {
 
 template <int DT>
 __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf, int32_t* sel,
-                                       u64* bcast, const char* qa, const char* meta_g) {
+                                       const char* qa, const char* meta_g) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
   u64* blk = reinterpret_cast<u64*>(buf);
   u64* buk = blk + M.cap_all;
   char* recs = reinterpret_cast<char*>(buk + M.cap_all);
   int* flag = reinterpret_cast<int*>(recs + kRecSlots * 512);
+  u64* kscr = reinterpret_cast<u64*>(flag + ((M.cap_all + 1) & ~1));
   // 1. the largest of the CTAs' thresholds bounds the group's k-th largest
   //    lower key from below; only entries whose upper key reaches it matter
   int nc = 0;
@@ -612,18 +707,7 @@ __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf
   __syncwarp();
   // 2. the group's k-th largest lower key (0: fewer than k pages in all)
   const int N = cnt;
-  if (lane == 0) *bcast = 0ull;
-  __syncwarp();
-  if (N >= k) {
-    for (int e = lane; e < N; e += 32) {
-      const u64 x = blk[e];
-      int rk = 0;
-      for (int e2 = 0; e2 < N; ++e2) rk += blk[e2] > x;
-      if (rk == k - 1) *bcast = x;
-    }
-  }
-  __syncwarp();
-  const u64 lkth = *bcast;
+  const u64 lkth = group_kth(blk, N, k, 32, true, kscr);
   // 3. candidates: upper key at or above it (they hold the true top k),
   //    compacted to the front in place
   int nca = 0;
@@ -731,7 +815,7 @@ __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf
 struct StepLayout {
   int ring;     // metadata ring; afterwards merge scratch, gathered pages, warp partials
   int qc, qp;   // the group's queries (current, previous) [GB][rowb]
-  int lists;    // list keys lk [R][lb], uk [R][lb]
+  int lists;    // candidate buffers lk [R][lb], uk [R][lb], then their scratch [R][sstride]
   int sc;       // scores of the pages being added: sU [R][ts], sT [R][ts]
   int part_o;   // the CTA's partial outputs [R16][kD] floats (bf16: in the ring)
   int part_ml;  // the CTA's partial (m, l) [R16][2] (bf16: in the ring)
@@ -745,7 +829,6 @@ struct StepLayout {
   int bitmap, wbase;   // union bitmap and its words' prefix counts
   int lpages, masks;   // this CTA's union pages and their row masks
   int misc;            // per-token / per-row ints and scalars
-  int bcast;           // per-warp u64 broadcast slots
   int mbar;            // kMaxStages ring barriers, the queries', the gather's
   int total;
 };
@@ -775,7 +858,9 @@ struct StepParams {
   int rec;         // bytes per metadata record
   int ts;          // pages per list update (a multiple of 8)
   int lw;          // lanes per row in a list update
-  int lb, lcap;    // list buffer entries per row; entries before an exact refinement
+  int lb, lcap;    // buffer entries per row; entries left after a compaction before an exact refinement
+  int sstride;     // scratch keys per row (sub-maxima, survivors, broadcast)
+  int qstride;     // bytes per staged query row (padded: no bank conflicts between rows)
   int nmw;         // merge warps
   int mstride;     // bytes of a merge warp's scratch (in the ring area)
   int max_lp;      // union pages per CTA, at most
@@ -840,6 +925,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* part_ml = reinterpret_cast<float*>(smem + lo.part_ml);
   u64* l_lk = reinterpret_cast<u64*>(smem + lo.lists);
   u64* l_uk = l_lk + static_cast<size_t>(R) * prm.lb;
+  u64* l_scr = l_uk + static_cast<size_t>(R) * prm.lb;
+  const int qst = prm.qstride;
   float* sU = reinterpret_cast<float*>(smem + lo.sc);
   float* sT = sU + R * prm.ts;
   int* l_n = reinterpret_cast<int*>(smem + lo.l_n);
@@ -856,10 +943,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* act_slot = misc + kMiscActSlot;
   int32_t* sfx_tok = misc + kMiscSfxTok;
   int32_t* scal = misc + kMiscScal;
-  u64* bcast = reinterpret_cast<u64*>(smem + lo.bcast);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
-  uint64_t* qbar = mbar + kMaxStages;
-  uint64_t* gbar = mbar + kMaxStages + 1;
+  uint64_t* gbar = mbar + kMaxStages;  // [2]: the gather's two page buffers
 
   // the next kernel of the stream may be scheduled now when this grid fits
   // one wave (it waits for this grid's completion before it reads anything);
@@ -875,17 +960,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int npg = sel ? max(0, min(Ps, pr0 + prm.cp) - pr0) : 0;
   const int nstg = (npg + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.Pc * prm.rec;
-  const uint32_t qbytes = static_cast<uint32_t>(GB * rowb);
 
   if (tid == 0) {
     for (int i = 0; i < kMaxStages + 2; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
     scal[kSFail] = 0;
     if (c == 0 && g == 0 && seq_len_bad(d, s)) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-    const size_t qoff = grow0 * rowb;
-    mbar_expect_tx(qbar, 2 * qbytes);
-    bulk_g2s(smem + lo.qc, static_cast<const char*>(prm.qc) + qoff, qbytes, qbar);
-    bulk_g2s(smem + lo.qp, static_cast<const char*>(prm.qp) + qoff, qbytes, qbar);
 #pragma unroll 1
     for (int t = 0; t < min(nstg, prm.stages); ++t) {
       const int np = min(prm.tile, npg - t * prm.tile);
@@ -895,7 +975,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                bytes, &mbar[t]);
     }
   }
+  // the group's current and previous queries (cp.async group 0), rows
+  // padded to qst bytes
+  {
+    const char* qcg = static_cast<const char*>(prm.qc) + grow0 * rowb;
+    const char* qpg = static_cast<const char*>(prm.qp) + grow0 * rowb;
+    const int per = GB * cpr;
+#pragma unroll 1
+    for (int e = tid; e < 2 * per; e += kThreads) {
+      const int h = e >= per ? 1 : 0, rem = e - h * per, row = rem / cpr, cc = rem - row * cpr;
+      cp_async16(su32(smem + (h ? lo.qp : lo.qc) + row * qst + cc * 16),
+                 (h ? qpg : qcg) + static_cast<size_t>(row) * rowb + cc * 16, 16u);
+    }
+    cp_async_commit();
+  }
   // the block's K and V (rows >= B zero), chunks swizzled for ldmatrix
+  // (cp.async group 1)
   {
     const char* kbg = static_cast<const char*>(prm.kb) + static_cast<size_t>(sg) * B * rowb;
     const char* vbg = static_cast<const char*>(prm.vb) + static_cast<size_t>(sg) * B * rowb;
@@ -909,18 +1004,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_commit();
   }
+  cp_async_wait<1>();  // the queries
   __syncthreads();
-  if (!mbar_wait(qbar, 0)) scal[kSFail] = 1;
-  __syncthreads();
-  const bool qok = scal[kSFail] == 0;
+  const bool qok = true;
 
   // ---- locality: one thread per token row, the oracle's arithmetic exactly
   // (channels in order, fp32, one rounding per operation)
   if (tid < GB) {
     float acc = 0.f;
     if (qok) {
-      const char* x = qcs + tid * rowb;
-      const char* y = qps + tid * rowb;
+      const char* x = qcs + tid * qst;
+      const char* y = qps + tid * qst;
 #pragma unroll 2
       for (int cc = 0; cc < cpr; ++cc) {
         const uint4 a = *reinterpret_cast<const uint4*>(x + cc * 16);
@@ -976,7 +1070,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (int e = tid; e < R16 * 16; e += kThreads) {
       const int r = e / 16, cc = e % 16;
-      const uint4 v = r < R ? *reinterpret_cast<const uint4*>(qcs + act_row[r] * rowb + cc * 16)
+      const uint4 v = r < R ? *reinterpret_cast<const uint4*>(qcs + act_row[r] * qst + cc * 16)
                             : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(qa + tile_off<DT>(r, cc)) = v;
     }
@@ -985,7 +1079,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int e = tid; e < R * cpr; e += kThreads) {
       const int r = e / cpr, cc = e % cpr;
       *reinterpret_cast<uint4*>(qa + r * rowb + cc * 16) =
-          *reinterpret_cast<const uint4*>(qcs + act_row[r] * rowb + cc * 16);
+          *reinterpret_cast<const uint4*>(qcs + act_row[r] * qst + cc * 16);
     }
   }
 
@@ -1017,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (int e = tid; e < nsr * cpr; e += kThreads) {
       const int n = e / cpr, cc = e - n * cpr;
-      const uint4 v = n < ns ? *reinterpret_cast<const uint4*>(qcs + sfx_tok[n] * rowb + cc * 16)
+      const uint4 v = n < ns ? *reinterpret_cast<const uint4*>(qcs + sfx_tok[n] * qst + cc * 16)
                              : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(sq + tile_off<DT>(n, cc)) = v;
     }
@@ -1032,7 +1126,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_async4(su32(lcache + n), prm.l_p + grow0 + sfx_tok[n_oa + n]);
     cp_async_commit();
   }
-  cp_async_wait<0>();  // the block's K/V, the cached state
   __syncthreads();
 
   // ---- the bound's A operand stays in registers for the whole scan (one
@@ -1048,8 +1141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // columns + 8; column j < 128 is q-_j = min(q_j, 0), column 128 + j is
     // q+_j = max(q_j, 0) (sign bit tests, exact)
     const int rA = mt * 16 + g4, rB = rA + 8;
-    const char* qrA = rA < R ? qcs + act_row[rA] * rowb : nullptr;
-    const char* qrB = rB < R ? qcs + act_row[rB] * rowb : nullptr;
+    const char* qrA = rA < R ? qcs + act_row[rA] * qst : nullptr;
+    const char* qrB = rB < R ? qcs + act_row[rB] * qst : nullptr;
     auto part = [](uint32_t w, bool neg) {
       uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
       const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
@@ -1072,82 +1165,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // ---- dense suffix of this CTA's rows over the block's own keys: stable
-  // rows merge with their untouched cache and are finished; active rows keep
-  // (o_s, L_s) for the combine
-  if (qok) {
-    if (DT == LOSA_BF16) {
-      const int nmt = (ns + 15) / 16;
-#pragma unroll 1
-      for (int m2 = warp; m2 < nmt; m2 += kWarps) {
-        TileAcc t;
-        tile_init(t);
-#pragma unroll 1
-        for (int j0 = 0; j0 < B; j0 += kPS)
-          tile_attend<false>(t, sq + m2 * 16 * 256, kbv + j0 * 256, kbv + (bpad + j0) * 256,
-                             0xffffu, min(kPS, B - j0), d.scale_log2);
-        tile_finish(t);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int n = m2 * 16 + g4 + 8 * h;
-          if (n >= ns) continue;
-          const float inv = __frcp_rn(t.l[h]);
-          const float Lsx = (t.m[h] + __log2f(t.l[h])) * kLn2;
-          if (n < n_oa) {
-            if (t4 == 0) sfx_l[n] = Lsx;
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc)
-              *reinterpret_cast<float2*>(sfx_o + n * kD + cc * 8 + 2 * t4) =
-                  make_float2(t.o[cc][2 * h] * inv, t.o[cc][2 * h + 1] * inv);
-          } else {
-            const int m = n - n_oa;
-            const size_t grow = grow0 + sfx_tok[n];
-            float wa, wb, L;
-            lse_weights(lcache[m], Lsx, wa, wb, L);
-            const float* op = ocache + m * kD;
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const int ch = cc * 8 + 2 * t4;
-              const float2 o = *reinterpret_cast<const float2*>(op + ch);
-              *reinterpret_cast<float2*>(prm.out + grow * kD + ch) =
-                  make_float2(wa * o.x + wb * (t.o[cc][2 * h] * inv),
-                              wa * o.y + wb * (t.o[cc][2 * h + 1] * inv));
-            }
-            if (prm.out_lse && t4 == 0) prm.out_lse[grow] = L;
-          }
-        }
-      }
-    } else {
-      float* Ps = reinterpret_cast<float*>(sU) + warp * 16;  // (the score area is free now)
-#pragma unroll 1
-      for (int n = warp; n < ns; n += kWarps) {
-        const float4 q = row4<DT>(sq, n, lane);
-        float m = -INFINITY, l = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-        for (int j0 = 0; j0 < B; j0 += kPS)
-          attend_page<DT>(q, kbv + j0 * rowb, kbv + (bpad + j0) * rowb, min(kPS, B - j0),
-                          d.scale_log2, m, l, acc, Ps);
-        const float inv = __frcp_rn(l);
-        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-        const float Lsx = (m + __log2f(l)) * kLn2;
-        if (n < n_oa) {
-          if (lane == 0) sfx_l[n] = Lsx;
-          *reinterpret_cast<float4*>(sfx_o + n * kD + 4 * lane) = os;
-        } else {
-          const int mm = n - n_oa;
-          const size_t grow = grow0 + sfx_tok[n];
-          float wa, wb, L;
-          lse_weights(lcache[mm], Lsx, wa, wb, L);
-          const float4 op = *reinterpret_cast<const float4*>(ocache + mm * kD + 4 * lane);
-          *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
-              make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
-                          wa * op.w + wb * os.w);
-          if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
-        }
-      }
-    }
-  }
   for (int r = tid; r < R; r += kThreads) {
     l_n[r] = 0;
     l_thr[r] = 0ull;
@@ -1156,7 +1173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- bound scores of this CTA's pages, stage by stage, into the rows'
   // candidate lists
-  const ListCtx LC = {l_lk, l_uk, l_n, l_thr, prm.lb, prm.lcap, prm.lw};
+  const ListCtx LC = {l_lk, l_uk, l_n, l_thr, l_scr, prm.lb, prm.lcap, prm.sstride, prm.lw};
 #pragma unroll 1
   for (int t = 0; t < nstg; ++t) {
     const int st = t % prm.stages;
@@ -1228,39 +1245,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_g2s(ring + st * kStageBytes,
                  meta_g + static_cast<size_t>(pr0 + tn * prm.tile) * prm.rec, bytes, &mbar[st]);
       }
-      if (ok) list_update<DT>(LC, R, k, sU, sT, prm.ts, np, pbase, qa, meta_g);
+      if (ok) list_add<DT>(LC, R, k, sU, sT, prm.ts, np, pbase, qa, meta_g);
       __syncthreads();
     }
   }
+
+  // the exact k-th largest lower key of each row's pages becomes its
+  // threshold; the buffer keeps the pages whose upper key reaches it
+  if (sel && scal[kSFail] == 0) {
+#pragma unroll 1
+    for (int r0 = 0; r0 < R; r0 += kThreads / prm.lw)
+      buffer_compact<DT>(LC, r0 + tid / prm.lw, k, r0 + tid / prm.lw < R, qa, meta_g);
+  }
+  __syncthreads();
 
   // ================= cluster barrier 1: every CTA's lists are final ========
   cluster_sync();
   const bool ok1 = scal[kSFail] == 0;
 
-  // ---- every row's k pages from the lists of all CTAs of the cluster
+  // ---- each row's k pages from the lists of all CTAs of the cluster: CTA c
+  // merges rows r = c (mod C), one warp per row
   const int nwords = (d.P + 31) / 32;
   if (sel) {
-#pragma unroll 1
-    for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
-    if (ok1 && warp < prm.nmw) {
+    if (ok1) {
       const MergeCtx MC = {l_lk, l_uk, l_n, l_thr, prm.lb, C * prm.lcap, C};
       char* buf = ring + warp * prm.mstride;
 #pragma unroll 1
-      for (int r = warp; r < R; r += prm.nmw)
-        merge_row<DT>(MC, r, k, buf, sel_all + r * k, bcast + warp, qa, meta_g);
+      for (int i = warp; warp < prm.nmw && c + C * i < R; i += prm.nmw)
+        merge_row<DT>(MC, c + C * i, k, buf, sel_all + (c + C * i) * k, qa, meta_g);
     }
     __syncthreads();
-    // union bitmap; every CTA reports its rows r = c (mod C)
+    if (prm.page_idx) {
+#pragma unroll 1
+      for (int e = tid; e < R * k; e += kThreads) {
+        const int r = e / k, j = e - r * k;
+        if (r % C != c) continue;
+        const int hl = r / A, aa = r % A;
+        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + aa) * k + j] = sel_all[e];
+      }
+    }
+  }
+
+  // ================= cluster barrier 1b: every row's selection is final =====
+  cluster_sync();
+
+  // ---- every CTA takes the other rows' selections from their CTAs and
+  // builds the group's union bitmap
+  if (sel) {
+#pragma unroll 1
+    for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
 #pragma unroll 1
     for (int e = tid; e < R * k; e += kThreads) {
-      const int r = e / k, j = e - r * k;
+      const int r = e / k;
+      if (r % C != c) sel_all[e] = ld_dsmem_s32(dsmem(sel_all + e, r % C));
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int e = tid; e < R * k; e += kThreads) {
       const int p = sel_all[e];
       if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
       else if (p >= 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-      if (prm.page_idx && r % C == c) {
-        const int hl = r / A, aa = r % A;
-        prm.page_idx[((static_cast<size_t>(s) * d.Hq + g * G + hl) * A + aa) * k + j] = p;
-      }
     }
   } else if (R > 0 && prm.page_idx) {
     // every page of the sequence, then -1
@@ -1372,6 +1416,127 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nlp = R > 0 ? scal[kSNlp] : 0;
   const bool ok2 = scal[kSFail] == 0;
   const float sl2 = d.scale_log2;
+  // two page buffers of ngp pages: batch b lands in buffer b & 1 while the
+  // previous batch is folded in
+  const int nbat = (nlp + prm.ngp - 1) / prm.ngp;
+  auto issue = [&](int bt) {
+    const int b0 = bt * prm.ngp, nb = min(prm.ngp, nlp - b0);
+    char* bufp = ring + (bt & 1) * prm.ngp * 2 * pbytes;
+    if (DT == LOSA_BF16) {
+      mbar_expect_tx(&gbar[bt & 1], static_cast<uint32_t>(nb * 2 * pbytes));
+#pragma unroll 1
+      for (int i = 0; i < nb; ++i) {
+        const int p = lpages[b0 + i];
+        const int row = sg * d.Lc + p * kPS;
+        char* dk = bufp + 2 * i * pbytes;
+        tma_load_2d(dk, &kmap, 0, row, &gbar[bt & 1]);
+        tma_load_2d(dk + 2048, &kmap, 64, row, &gbar[bt & 1]);
+        tma_load_2d(dk + pbytes, &vmap, 0, row, &gbar[bt & 1]);
+        tma_load_2d(dk + pbytes + 2048, &vmap, 64, row, &gbar[bt & 1]);
+      }
+    } else {
+      uint32_t bytes = 0;
+      for (int i = 0; i < nb; ++i) bytes += 2u * min(kPS, Ls - lpages[b0 + i] * kPS) * rowb;
+      mbar_expect_tx(&gbar[bt & 1], bytes);
+#pragma unroll 1
+      for (int i = 0; i < nb; ++i) {
+        const int p = lpages[b0 + i];
+        const uint32_t nbytes = static_cast<uint32_t>(min(kPS, Ls - p * kPS) * rowb);
+        const size_t off = (static_cast<size_t>(sg) * d.Lc + static_cast<size_t>(p) * kPS) * rowb;
+        bulk_g2s(bufp + 2 * i * pbytes, static_cast<const char*>(prm.K) + off, nbytes,
+                 &gbar[bt & 1]);
+        bulk_g2s(bufp + (2 * i + 1) * pbytes, static_cast<const char*>(prm.V) + off, nbytes,
+                 &gbar[bt & 1]);
+      }
+    }
+  };
+  if (tid == 0 && ok2) {
+    if (nbat > 0) issue(0);
+    if (nbat > 1) issue(1);
+  }
+
+  // ---- while the pages land: the block's K/V and the cached state are in
+  // (cp.async groups 1 and 2)
+  cp_async_wait<0>();
+  __syncthreads();
+  // ---- dense suffix of this CTA's rows over the block's own keys: stable
+  // rows merge with their untouched cache and are finished; active rows keep
+  // (o_s, L_s) for the combine
+  if (qok) {
+    if (DT == LOSA_BF16) {
+      const int nmt = (ns + 15) / 16;
+#pragma unroll 1
+      for (int m2 = warp; m2 < nmt; m2 += kWarps) {
+        TileAcc t;
+        tile_init(t);
+#pragma unroll 1
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          tile_attend<false>(t, sq + m2 * 16 * 256, kbv + j0 * 256, kbv + (bpad + j0) * 256,
+                             0xffffu, min(kPS, B - j0), d.scale_log2);
+        tile_finish(t);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int n = m2 * 16 + g4 + 8 * h;
+          if (n >= ns) continue;
+          const float inv = __frcp_rn(t.l[h]);
+          const float Lsx = (t.m[h] + __log2f(t.l[h])) * kLn2;
+          if (n < n_oa) {
+            if (t4 == 0) sfx_l[n] = Lsx;
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc)
+              *reinterpret_cast<float2*>(sfx_o + n * kD + cc * 8 + 2 * t4) =
+                  make_float2(t.o[cc][2 * h] * inv, t.o[cc][2 * h + 1] * inv);
+          } else {
+            const int m = n - n_oa;
+            const size_t grow = grow0 + sfx_tok[n];
+            float wa, wb, L;
+            lse_weights(lcache[m], Lsx, wa, wb, L);
+            const float* op = ocache + m * kD;
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int ch = cc * 8 + 2 * t4;
+              const float2 o = *reinterpret_cast<const float2*>(op + ch);
+              *reinterpret_cast<float2*>(prm.out + grow * kD + ch) =
+                  make_float2(wa * o.x + wb * (t.o[cc][2 * h] * inv),
+                              wa * o.y + wb * (t.o[cc][2 * h + 1] * inv));
+            }
+            if (prm.out_lse && t4 == 0) prm.out_lse[grow] = L;
+          }
+        }
+      }
+    } else {
+      float* Ps = reinterpret_cast<float*>(sU) + warp * 16;  // (the score area is free now)
+#pragma unroll 1
+      for (int n = warp; n < ns; n += kWarps) {
+        const float4 q = row4<DT>(sq, n, lane);
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+        for (int j0 = 0; j0 < B; j0 += kPS)
+          attend_page<DT>(q, kbv + j0 * rowb, kbv + (bpad + j0) * rowb, min(kPS, B - j0),
+                          d.scale_log2, m, l, acc, Ps);
+        const float inv = __frcp_rn(l);
+        const float4 os = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        const float Lsx = (m + __log2f(l)) * kLn2;
+        if (n < n_oa) {
+          if (lane == 0) sfx_l[n] = Lsx;
+          *reinterpret_cast<float4*>(sfx_o + n * kD + 4 * lane) = os;
+        } else {
+          const int mm = n - n_oa;
+          const size_t grow = grow0 + sfx_tok[n];
+          float wa, wb, L;
+          lse_weights(lcache[mm], Lsx, wa, wb, L);
+          const float4 op = *reinterpret_cast<const float4*>(ocache + mm * kD + 4 * lane);
+          *reinterpret_cast<float4*>(prm.out + grow * kD + 4 * lane) =
+              make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
+                          wa * op.w + wb * os.w);
+          if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
   if (DT == LOSA_BF16) {
     const int wpg = ntm > 0 ? kWarps / ntm : 1;
     const int mtg = warp / wpg, subg = warp % wpg;
@@ -1379,22 +1544,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     TileAcc t;
     tile_init(t);
 #pragma unroll 1
-    for (int b = 0, b0 = 0; b0 < nlp; ++b, b0 += prm.ngp) {
-      const int nb = min(prm.ngp, nlp - b0);
-      if (tid == 0 && ok2) {
-        mbar_expect_tx(gbar, static_cast<uint32_t>(nb * 2 * pbytes));
-#pragma unroll 1
-        for (int i = 0; i < nb; ++i) {
-          const int p = lpages[b0 + i];
-          const int row = sg * d.Lc + p * kPS;
-          char* dk = ring + 2 * i * pbytes;
-          tma_load_2d(dk, &kmap, 0, row, gbar);
-          tma_load_2d(dk + 2048, &kmap, 64, row, gbar);
-          tma_load_2d(dk + pbytes, &vmap, 0, row, gbar);
-          tma_load_2d(dk + pbytes + 2048, &vmap, 64, row, gbar);
-        }
-      }
-      if (ok2 && !mbar_wait(gbar, b & 1)) scal[kSFail] = 1;
+    for (int bt = 0; bt < nbat; ++bt) {
+      const int b0 = bt * prm.ngp, nb = min(prm.ngp, nlp - b0);
+      char* bufp = ring + (bt & 1) * prm.ngp * 2 * pbytes;
+      if (ok2 && scal[kSFail] == 0 && !mbar_wait(&gbar[bt & 1], (bt >> 1) & 1)) scal[kSFail] = 1;
       // V rows past the sequence's end of its partial last page may hold
       // anything (P is 0 there, but 0 times NaN is NaN): zero them
       if (Ls % kPS) {
@@ -1403,7 +1556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int p = lpages[b0 + i];
           if (p != Ps - 1) continue;
           const int ntok = Ls - p * kPS;
-          char* dv = ring + (2 * i + 1) * pbytes;
+          char* dv = bufp + (2 * i + 1) * pbytes;
           for (int e = tid; e < 2 * (kPS - ntok) * 8; e += kThreads) {
             const int h = e / ((kPS - ntok) * 8), rem = e % ((kPS - ntok) * 8);
             *reinterpret_cast<uint4*>(dv + h * 2048 + ntok * 128 + rem * 16) =
@@ -1418,11 +1571,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t bits = (masks[(b0 + i) * MW + (mtg >> 1)] >> ((mtg & 1) * 16)) & 0xffffu;
           if (!bits) continue;
           const int p = lpages[b0 + i];
-          tile_attend<true>(t, qa + mtg * 16 * 256, ring + 2 * i * pbytes,
-                            ring + (2 * i + 1) * pbytes, bits, min(kPS, Ls - p * kPS), sl2);
+          tile_attend<true>(t, qa + mtg * 16 * 256, bufp + 2 * i * pbytes,
+                            bufp + (2 * i + 1) * pbytes, bits, min(kPS, Ls - p * kPS), sl2);
         }
       }
-      __syncthreads();  // before the next batch overwrites the pages
+      __syncthreads();  // the buffer is free: the batch after next may land in it
+      if (tid == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
     }
     tile_finish(t);
     if (R > 0 && wpg == 1) {
@@ -1502,22 +1656,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* Ps = sU + warp * 16;
     __syncthreads();
 #pragma unroll 1
-    for (int b = 0, b0 = 0; b0 < nlp; ++b, b0 += prm.ngp) {
-      const int nb = min(prm.ngp, nlp - b0);
-      if (tid == 0 && ok2) {
-        uint32_t bytes = 0;
-        for (int i = 0; i < nb; ++i) bytes += 2u * min(kPS, Ls - lpages[b0 + i] * kPS) * rowb;
-        mbar_expect_tx(gbar, bytes);
-#pragma unroll 1
-        for (int i = 0; i < nb; ++i) {
-          const int p = lpages[b0 + i];
-          const uint32_t nbytes = static_cast<uint32_t>(min(kPS, Ls - p * kPS) * rowb);
-          const size_t off = (static_cast<size_t>(sg) * d.Lc + static_cast<size_t>(p) * kPS) * rowb;
-          bulk_g2s(ring + 2 * i * pbytes, static_cast<const char*>(prm.K) + off, nbytes, gbar);
-          bulk_g2s(ring + (2 * i + 1) * pbytes, static_cast<const char*>(prm.V) + off, nbytes, gbar);
-        }
-      }
-      if (ok2 && !mbar_wait(gbar, b & 1)) scal[kSFail] = 1;
+    for (int bt = 0; bt < nbat; ++bt) {
+      const int b0 = bt * prm.ngp, nb = min(prm.ngp, nlp - b0);
+      char* bufp = ring + (bt & 1) * prm.ngp * 2 * pbytes;
+      if (ok2 && scal[kSFail] == 0 && !mbar_wait(&gbar[bt & 1], (bt >> 1) & 1)) scal[kSFail] = 1;
       __syncthreads();
       if (scal[kSFail] == 0) {
 #pragma unroll 1
@@ -1533,7 +1675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < nb; ++i) {
             if (!((masks[(b0 + i) * MW + (r >> 5)] >> (r & 31)) & 1u)) continue;
             const int p = lpages[b0 + i];
-            attend_page<DT>(q, ring + 2 * i * pbytes, ring + (2 * i + 1) * pbytes,
+            attend_page<DT>(q, bufp + 2 * i * pbytes, bufp + (2 * i + 1) * pbytes,
                             min(kPS, Ls - p * kPS), sl2, m, l, acc, Ps);
           }
           __syncwarp();
@@ -1545,6 +1687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
+      if (tid == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
     }
   }
 
@@ -1644,17 +1787,18 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   if (R == 0) C = 1;
   prm->C = C;
   prm->cp = align_up((d.P + C - 1) / C, 8);
-  // candidate lists: lanes per row, refinement cap, pages per update
-  prm->lw = std::min(32, pow2_floor(kThreads / std::max(R16, 16)));
+  // candidate buffers: lanes per row, entries kept after a compaction
+  prm->lw = std::min(32, std::max(4, pow2_floor(kThreads / std::max(R16, 16))));
   prm->lcap = d.k + kListSlack;
-  prm->ts = std::min(prm->tile, (kEpl * prm->lw - prm->lcap) / 8 * 8);
-  if (sel && prm->ts < 8) return false;
-  if (!sel) prm->ts = 8;
-  prm->lb = prm->lcap + prm->ts;
+  const int ts_max = prm->tile;
   const long long cap_all = static_cast<long long>(C) * prm->lcap;
+  // merge warp scratch: keys, staged records, flags, the k-th selection's
+  const long long kv32 = 32LL * ((d.k + 31) / 32) + 1 + cap_all;
   prm->mstride = align_up(static_cast<int>(std::min<long long>(
-                              2 * cap_all * 8 + kRecSlots * 512 + cap_all * 4, 1 << 30)),
+                              2 * cap_all * 8 + kRecSlots * 512 + ((cap_all + 1) & ~1LL) * 4 +
+                                  kv32 * 8, 1 << 30)),
                           16);
+  prm->qstride = rowb + 16;  // rows 16 bytes apart in bank order
   // union pages per CTA
   const int Umax = d.all_pages ? d.P : std::min(d.P, R * d.k);
   prm->max_lp = R > 0 ? (Umax + C - 1) / C : 0;
@@ -1665,12 +1809,21 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   const int MW = (R + 31) / 32;
   prm->early = static_cast<long long>(d.S) * d.Hkv * C <= kEarlyTriggerCtas;
 
+  // the largest plan that fits: most pages per list update, then most union
+  // pages in flight, then most ring stages
+  for (int ts = sel ? ts_max : 8; ts >= 8; ts = (ts / 2 >= 8 ? ts / 2 / 8 * 8 : 0)) {
+  prm->ts = ts;
+  // room for a page tile's survivors beside the entries kept between
+  // prunings: ~3k when it fits, at least the cap after an exact compaction
+  for (int lbx = ts + 3 * d.k + 8; lbx >= ts + prm->lcap; lbx = (lbx > ts + prm->lcap ? std::max(ts + prm->lcap, lbx - d.k - 4) : 0)) {
+  prm->lb = lbx;
+  prm->sstride = prm->lw * ((d.k + prm->lw - 1) / prm->lw) + 1 + prm->lb;
   for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
     for (int stages = kMaxStages; stages >= kMinStages; --stages) {
       long long ring = 0;
       if (sel) ring = std::max(ring, static_cast<long long>(stages) * kStageBytes);
       if (sel) ring = std::max(ring, static_cast<long long>(prm->mstride));  // one merge warp
-      if (R > 0) ring = std::max(ring, 2LL * ngp * pbytes);
+      if (R > 0) ring = std::max(ring, 4LL * ngp * pbytes);  // two buffers of ngp pages
       // bf16: the warps' partials (when several warps share an m16 tile),
       // then the CTA's partial per row
       const int ntm = R16 / 16;
@@ -1680,12 +1833,13 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       Taker take;
       lo.ring = take(ring, 1024);
       // the queries, then (after the suffix) the lists and the scores
-      const long long qarea = 2LL * GB * rowb;
-      const long long larea = sel ? 2LL * R * prm->lb * 8 : 0;
+      const long long qarea = 2LL * GB * prm->qstride;
+      const long long larea =
+          sel ? (2LL * prm->lb * R + 1LL * (kThreads / prm->lw) * prm->sstride) * 8 : 0;
       const long long sarea = std::max(sel ? 2LL * R * prm->ts * 4 : 0LL, bf ? 0LL : 512LL);
       const int qbase = take(std::max(qarea, larea + sarea), 1024);
       lo.qc = qbase;
-      lo.qp = qbase + GB * rowb;
+      lo.qp = qbase + GB * prm->qstride;
       lo.lists = qbase;
       lo.sc = qbase + static_cast<int>(larea);
       if (bf) {  // after the gather: the warps' partials, then the CTA's
@@ -1710,7 +1864,6 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       lo.lpages = take(4LL * prm->max_lp, 16);
       lo.masks = take(4LL * prm->max_lp * MW, 16);
       lo.misc = take(4LL * kMiscInts, 16);
-      lo.bcast = take(8LL * kWarps, 16);
       lo.mbar = take(8LL * (kMaxStages + 2), 16);
       // + 1 KB: the kernel aligns its shared-memory base to 1024 bytes
       lo.total = static_cast<int>(std::min<long long>(take.off + 1024, 1LL << 30));
@@ -1721,6 +1874,8 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       if (sel && prm->nmw < 1) continue;
       return true;
     }
+  }
+  }
   }
   return false;
 }
