@@ -121,7 +121,8 @@ typedef struct {
  *   read the flag; any other bit is LOSA_ERR_INVALID_ARG. */
 #define LOSA_STEP_ATTEND_UNION 1
 
-/* Bytes of page metadata for `shape` (the size of `page_meta` below). */
+/* Bytes of page metadata for `shape` (the size of `page_meta` below): the
+ * records, then the page-norm rows. */
 size_t losa_page_meta_size(const losa_shape* shape);
 
 /* Bytes of workspace needed by losa_dense_prefix (which = LOSA_WS_DENSE) or
@@ -140,6 +141,12 @@ size_t losa_workspace_size(const losa_shape* shape, int which);
  *              a record the 16-byte chunks are stored XOR-swizzled: logical
  *              chunk c sits at chunk position c ^ (p & 7).  (This keeps the
  *              scoring kernel's shared-memory reads free of bank conflicts.)
+ *              After the S*Hkv*Pc records: for every (s, g) a row of
+ *              Pn = ceil(Pc / 8) * 8 float pairs, pair p = (||kmin||_2,
+ *              ||kmax||_2) of page p, computed in fp32 with every operation
+ *              rounded up (upper bounds of the exact norms; the step uses them
+ *              to bound the rounding error of its tensor-core page scores).
+ *              The row padding past a sequence's pages is never written.
  * Min/max introduce no rounding: the values are exact copies of key values.
  * With prefix_lens, sequence s gets records for its own P_s pages (the last
  * over its tokens < L_s only); its records from P_s on are not written.

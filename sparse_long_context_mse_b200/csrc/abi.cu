@@ -138,7 +138,8 @@ extern "C" {
 size_t losa_page_meta_size(const losa_shape* shape) {
   losa::Dims d;
   if (losa::make_dims(shape, LOSA_WS_DENSE, &d) != LOSA_OK) return 0;
-  return static_cast<size_t>(d.S) * d.Hkv * d.Pc * 2 * losa::kD * d.esz;
+  return losa::meta_norm_offset(d) +
+         static_cast<size_t>(d.S) * d.Hkv * losa::meta_norm_stride(d) * 2 * sizeof(float);
 }
 
 size_t losa_workspace_size(const losa_shape* shape, int which) {

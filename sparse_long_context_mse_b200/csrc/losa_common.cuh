@@ -109,6 +109,18 @@ __host__ __device__ __forceinline__ uint32_t meta_swz(uint32_t b, int page) {
   return ((((b >> 4) ^ static_cast<uint32_t>(page & 7)) << 4) | (b & 15u));
 }
 
+// The page-norm section of the page metadata, after the S*Hkv*Pc records:
+// for every (s, g) a row of meta_norm_stride(d) float2 entries, entry p =
+// (||kmin||_2, ||kmax||_2) of page p over the d channels, each rounded up (an
+// upper bound of the exact norm).  The row stride is a multiple of 8 entries
+// so that every 8-page run starts on a 64-byte boundary.
+__host__ __device__ __forceinline__ size_t meta_norm_offset(const Dims& d) {
+  return static_cast<size_t>(d.S) * d.Hkv * d.Pc * 2 * kD * d.esz;
+}
+__host__ __device__ __forceinline__ int meta_norm_stride(const Dims& d) {
+  return (d.Pc + 7) / 8 * 8;
+}
+
 // Prefix length of sequence s: its entry of the per-sequence lengths, clamped
 // into [1, L] (so that every access stays inside the buffers), else L.
 __device__ __forceinline__ int seq_len(const Dims& d, int s) {

@@ -4,7 +4,9 @@
 // QUEST's bound needs, per page and channel, the min and max key value over
 // the page's tokens (LoSA paper, methodology: QUEST-style selection over KV
 // pages).  One warp per page; lane l owns channels [4l, 4l+4).  Min/max are
-// exact, so the result is bit-identical to any correct implementation.
+// exact, so the records are bit-identical to any correct implementation.
+// Each page also gets the norms of its kmin and kmax rows, rounded up: the
+// scoring kernel bounds the error of its tensor-core sums with them.
 #include "losa_common.cuh"
 
 namespace losa {
@@ -29,6 +31,26 @@ __device__ __forceinline__ void page_record(Key4 key4, int n, void* meta, int sg
     hi.y = x.y > hi.y ? x.y : hi.y;
     hi.z = x.z > hi.z ? x.z : hi.z;
     hi.w = x.w > hi.w ? x.w : hi.w;
+  }
+  // the norms of kmin and kmax, every operation rounded up (all terms are
+  // non-negative, so each partial sum bounds the exact one from above)
+  float sl = 0.f, sh = 0.f;
+  sl = __fmaf_ru(lo.x, lo.x, sl);
+  sl = __fmaf_ru(lo.y, lo.y, sl);
+  sl = __fmaf_ru(lo.z, lo.z, sl);
+  sl = __fmaf_ru(lo.w, lo.w, sl);
+  sh = __fmaf_ru(hi.x, hi.x, sh);
+  sh = __fmaf_ru(hi.y, hi.y, sh);
+  sh = __fmaf_ru(hi.z, hi.z, sh);
+  sh = __fmaf_ru(hi.w, hi.w, sh);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sl = __fadd_ru(sl, __shfl_xor_sync(0xffffffffu, sl, o));
+    sh = __fadd_ru(sh, __shfl_xor_sync(0xffffffffu, sh, o));
+  }
+  if (lane == 0) {
+    float2* nrm = reinterpret_cast<float2*>(static_cast<char*>(meta) + meta_norm_offset(d));
+    nrm[static_cast<size_t>(sg) * meta_norm_stride(d) + p] = make_float2(__fsqrt_ru(sl), __fsqrt_ru(sh));
   }
   char* rec = static_cast<char*>(meta) + (static_cast<size_t>(sg) * d.Pc + p) * (2 * kD * d.esz);
   if (d.dtype == LOSA_BF16) {

@@ -304,25 +304,22 @@ __device__ __forceinline__ void lse_weights(float L1, float L2, float& a, float&
 
 
 // ---------------------------------------------------------------------------
-// Selection keys with error intervals.
+// Selection keys with error intervals.  A page scored u on the tensor cores
+// has its oracle score (the channel-order fp32 sum) in [u - e, u + e], with
+// e = 2^-14 T rounded up and T >= the sum of the terms' magnitudes.  The
+// terms are q-_i kmin_i and q+_i kmax_i, so by Cauchy-Schwarz on each half
+// T = ||q-|| ||kmin|| + ||q+|| ||kmax|| (every norm and operation rounded
+// up) bounds it.  The lower key lk and the upper key uk of [u - e, u + e]
+// bracket the page's true key; e = 0 (an exact score) gives lk == uk == the
+// exact key.
 // ---------------------------------------------------------------------------
-// Keys of a page scored u (tensor-core sum) with terms of total magnitude t:
-// the oracle's channel-order fp32 sum lies in [u - e, u + e], e = 2^-14 t
-// (rounded outward), so lk <= the page's true key <= uk.  t = 0 (an exact
-// score) gives lk == uk == the exact key.
-__device__ __forceinline__ void entry_keys(float u, float t, int p, u64& lk, u64& uk) {
-  const float e = __fmul_ru(t, kEpsScale);  // >= 2^-14 t (exact unless subnormal)
-  lk = sel_key(__fsub_rd(u, e), p);
-  uk = sel_key(__fadd_ru(u, e), p);
-}
-
 // The oracle's bound of page p for one active row, bit for bit: channels in
 // order 0..d-1, fp32, one rounding per operation,
 //   acc = acc + max(q_i * kmax_i, q_i * kmin_i).
 // qrow: the row's q (bf16, 16-byte chunks swizzled by r & 7, as staged for
 // the tensor cores); rec: page p's metadata record (global or shared memory;
 // chunks swizzled by p & 7 as losa_build_page_meta stores them).
-__device__ float exact_bound_bf16(const char* qrow, int r, const char* rec, int p) {
+__device__ __noinline__ float exact_bound_bf16(const char* qrow, int r, const char* rec, int p) {
   const int rs = r & 7, ps = p & 7;
   float acc = 0.f;
 #pragma unroll 4
@@ -348,22 +345,18 @@ __device__ float exact_bound_bf16(const char* qrow, int r, const char* rec, int 
 }
 
 // Bound scores of one 8-page n-tile for the 16 rows of the A fragments
-// ([q- | q+], bf16): u = [q- | q+] . [kmin ; kmax] and t = the same product of
-// the operands' magnitudes (the sum of the terms' magnitudes: one of q-_i,
-// q+_i is zero).  u[0..1]: row g4, pages 2*t4, 2*t4+1; u[2..3]: row g4 + 8.
-// `rec0` points to the tile's first record; records are [kmin | kmax] with
-// 16-byte chunks swizzled by the page index (congruent to the record index
-// mod 8 inside a ring stage).
-__device__ __forceinline__ void bound_ntile2(const uint32_t (&a)[16][4], const char* rec0,
-                                             float (&u)[4], float (&t)[4]) {
+// ([q- | q+], bf16): u = [q- | q+] . [kmin ; kmax].  u[0..1]: row g4, pages
+// 2*t4, 2*t4+1; u[2..3]: row g4 + 8.  `rec0` points to the tile's first
+// record; records are [kmin | kmax] with 16-byte chunks swizzled by the page
+// index (congruent to the record index mod 8 inside a ring stage).
+__device__ __forceinline__ void bound_ntile(const uint32_t (&a)[16][4], const char* rec0,
+                                            float (&u)[4]) {
   const int lane = threadIdx.x & 31;
   const int pg = lane & 7;
-  constexpr uint32_t kAbs = 0x7fff7fffu;
-  // two accumulator chains each (even / odd k-steps), added at the end: half
-  // the dependent MMA latency
-  float u1[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+  // two accumulator chains (even / odd k-steps), added at the end: half the
+  // dependent MMA latency
+  float u1[4] = {0.f, 0.f, 0.f, 0.f};
   u[0] = u[1] = u[2] = u[3] = 0.f;
-  t[0] = t[1] = t[2] = t[3] = 0.f;
 #pragma unroll
   for (int ks = 0; ks < 16; ks += 2) {
     uint32_t b0, b1, b2, b3;
@@ -371,120 +364,240 @@ __device__ __forceinline__ void bound_ntile2(const uint32_t (&a)[16][4], const c
     ldsm_x4(su32(rec0 + pg * 512 + ((ch ^ pg) << 4)), b0, b1, b2, b3);
     mma_bf16(u, a[ks], b0, b1);
     mma_bf16(u1, a[ks + 1], b2, b3);
-    const uint32_t x0[4] = {a[ks][0] & kAbs, a[ks][1] & kAbs, a[ks][2] & kAbs, a[ks][3] & kAbs};
-    const uint32_t x1[4] = {a[ks + 1][0] & kAbs, a[ks + 1][1] & kAbs, a[ks + 1][2] & kAbs,
-                            a[ks + 1][3] & kAbs};
-    mma_bf16(t, x0, b0 & kAbs, b1 & kAbs);
-    mma_bf16(t1, x1, b2 & kAbs, b3 & kAbs);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    u[i] += u1[i];
-    t[i] += t1[i];
-  }
+  for (int i = 0; i < 4; ++i) u[i] += u1[i];
 }
 
 // ---------------------------------------------------------------------------
-// Per-row candidate buffers.  Row r's buffer holds, unsorted, every page seen
-// so far whose upper key reaches thr[r], a lower bound of the k-th largest
-// lower key seen so far (0 while fewer than k pages were seen): a superset of
-// the pages that can still be among the row's top k.  A group of w lanes
-// (aligned in its warp) serves each row: rows r = pass * (threads / w) +
-// tid / w, in as many passes as the rows need.
+// Per-row candidate buffers.  Row r's buffer lk/uk [r][0..lb) holds, unsorted,
+// every page of the CTA scored so far whose upper key reached thr[r] when it
+// was scored.  thr[r] is the k-th largest lower key of k scored pages (0 until
+// the row's first compaction), so it never exceeds the k-th largest lower key
+// of all the CTA's pages: every page that can be among the row's top k is in
+// the buffer.  One warp compacts a row.
 // ---------------------------------------------------------------------------
-struct ListCtx {
-  u64* lk;    // [R][lb] lower keys
-  u64* uk;    // [R][lb] upper keys
-  int* n;     // [R] entries
-  u64* thr;   // [R] threshold
-  u64* scr;   // [threads / w][sstride] per-group scratch (sub-maxima, survivors, broadcast)
-  int lb;     // entries per row buffer
-  int cap;    // entries kept after the last compaction before an exact refinement
-  int sstride;
-  int w;      // lanes per row (a power of two)
-};
 
-// The k-th largest of the keys a[0..n) (distinct; 0 if n < k), computed by
-// the w lanes of a row group.  A lower bound first -- the k-th largest of
-// the lanes' sub-maxima (each lane keeps V = ceil(k / w) of them, so there
-// are at least k) -- then an exact rank among the keys at or above it, which
-// are few.  Every lane of the warp calls it (`act` false for a group without
-// a row); scr holds w * V + 1 + n keys.
-__device__ u64 group_kth(const u64* a, int n, int k, int w, bool act, u64* scr) {
-  const int lane = threadIdx.x & 31, j = lane & (w - 1);
-  const unsigned gmask = w == 32 ? 0xffffffffu : (((1u << w) - 1u) << (lane & ~(w - 1)));
+// The k-th largest of the distinct keys a[0..n) (0 if n < k), by one warp.  A
+// lower bound first -- the k-th largest of the lanes' sub-maxima (lane j keeps
+// V = ceil(k / 32) of them, so there are at least k) -- then the exact rank
+// among the keys at or above it, which are few.  scr holds 32 V + n keys.
+__device__ __noinline__ u64 warp_kth(const u64* a, int n, int k, u64* scr) {
+  const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  const int V = (k + w - 1) / w;
-  const int nw = __reduce_max_sync(0xffffffffu, act ? n : 0);
-  u64* sub = scr;
-  u64* bc = scr + w * V;
-  u64* sv = bc + 1;
-  if (act) {
-    for (int v = 0; v < V; ++v) {
-      u64 m = 0;
-      for (int i = j + w * v; i < n; i += w * V) m = a[i] > m ? a[i] : m;
-      sub[j * V + v] = m;
-    }
-    if (j == 0) *bc = 0ull;
+  if (n < k) return 0ull;
+  const int V = (k + 31) >> 5;
+  u64* sv = scr + 32 * V;
+#pragma unroll 1
+  for (int v = 0; v < V; ++v) {
+    u64 m = 0;
+    for (int i = lane + 32 * v; i < n; i += 32 * V) m = a[i] > m ? a[i] : m;
+    scr[lane * V + v] = m;
   }
   __syncwarp();
-  if (act && n >= k) {
-    for (int v = 0; v < V; ++v) {
-      const u64 x = sub[j * V + v];
-      int rk = 0;
-      for (int q = 0; q < w * V; ++q) {
-        const u64 y = sub[q];
-        rk += (y > x) || (y == x && q < j * V + v);
-      }
-      if (rk == k - 1) *bc = x;
+  u64 t1 = 0;
+#pragma unroll 1
+  for (int v = 0; v < V; ++v) {
+    const u64 x = scr[lane * V + v];
+    int rk = 0;
+    for (int q = 0; q < 32 * V; ++q) {
+      const u64 y = scr[q];
+      rk += (y > x) || (y == x && q < lane * V + v);
     }
+    if (rk == k - 1) t1 = x;
   }
-  __syncwarp();
-  const u64 t1 = act ? *bc : 0ull;
-  // the keys at or above the lower bound (they hold the k largest)
+  t1 = warp_max_u64(t1);
   int ns = 0;
-  for (int i0 = 0; i0 < nw; i0 += w) {
-    const int i = i0 + j;
-    const bool in = act && i < n && a[i] >= t1;
-    const unsigned bal = __ballot_sync(0xffffffffu, in) & gmask;
-    if (in) sv[ns + __popc(bal & lt)] = a[i];
+#pragma unroll 1
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    const u64 x = i < n ? a[i] : 0ull;
+    const bool in = i < n && x >= t1;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in) sv[ns + __popc(bal & lt)] = x;
     ns += __popc(bal);
   }
   __syncwarp();
-  if (act && j == 0) *bc = 0ull;
-  __syncwarp();
-  if (act && n >= k) {
-    for (int i = j; i < ns; i += w) {
-      const u64 x = sv[i];
-      int rk = 0;
-      for (int q = 0; q < ns; ++q) rk += sv[q] > x;
-      if (rk == k - 1) *bc = x;
-    }
+  u64 r = 0;
+#pragma unroll 1
+  for (int i = lane; i < ns; i += 32) {
+    const u64 x = sv[i];
+    int rk = 0;
+    for (int q = 0; q < ns; ++q) rk += sv[q] > x;
+    if (rk == k - 1) r = x;
   }
-  __syncwarp();
-  const u64 r = act ? *bc : 0ull;
+  r = warp_max_u64(r);
   __syncwarp();
   return r;
 }
 
-// Keep the entries of a row's buffer whose upper key reaches `thr`
-// (compaction in place, order kept); returns the new count.
-__device__ int buffer_keep(u64* lk, u64* uk, int n, u64 thr, int w, bool act) {
-  const int lane = threadIdx.x & 31, j = lane & (w - 1);
-  const unsigned gmask = w == 32 ? 0xffffffffu : (((1u << w) - 1u) << (lane & ~(w - 1)));
+// Compaction of one row's buffer by a warp (any n, in shared memory): the
+// exact k-th largest lower key becomes the threshold and only the entries
+// whose upper key reaches it stay.  A row left with more than `cap` entries
+// (near-ties at the boundary) has its inexact entries rescored exactly (the
+// oracle's arithmetic) and is compacted again, which leaves min(k, n) exact
+// entries.
+template <int DT>
+__device__ __noinline__ void row_compact_slow(u64* lk, u64* uk, int* cnt, u64* thr, int k,
+                                              int cap, u64* scr, const char* qrow, int r,
+                                              const char* meta_g) {
+  const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  const int nw = __reduce_max_sync(0xffffffffu, act ? n : 0);
+  int n = *cnt;
+  u64 th_old = *thr;
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    const u64 th = warp_kth(lk, n, k, scr);
+    int kept = 0;
+#pragma unroll 1
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      u64 a = 0, b = 0;
+      bool keep = false;
+      if (i < n) {
+        a = lk[i];
+        b = uk[i];
+        keep = b >= th;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      __syncwarp();
+      if (keep) {
+        const int pos = kept + __popc(bal & lt);
+        lk[pos] = a;
+        uk[pos] = b;
+      }
+      kept += __popc(bal);
+      __syncwarp();
+    }
+    n = kept;
+    th_old = th > th_old ? th : th_old;
+    if (DT == LOSA_BF16 && n > cap) {
+#pragma unroll 1
+      for (int i = lane; i < n; i += 32)
+        if (lk[i] != uk[i]) {
+          const int p = key_index(lk[i]);
+          const float v = exact_bound_bf16(qrow, r, meta_g + static_cast<size_t>(p) * 512, p);
+          lk[i] = uk[i] = sel_key(v, p);
+        }
+      __syncwarp();
+    } else {
+      break;
+    }
+  }
+  if (lane == 0) {
+    *cnt = n;
+    *thr = th_old;
+  }
+  __syncwarp();
+}
+
+// The k-th largest of the 32-bit values the warp's lanes hold (E per lane,
+// 0 = none), counting repeats: the value x with fewer than k values above it
+// and at least k at or above it (0 when there are fewer than k values).  Each
+// lane orders its values; each round then takes the largest head over the
+// lanes and pops it from every lane holding it (at most k rounds).
+template <int E>
+__device__ __forceinline__ uint32_t warp_kth_u32(uint32_t (&v)[E], int k) {
+#pragma unroll
+  for (int i = 1; i < E; ++i) {
+#pragma unroll
+    for (int j = i; j > 0; --j) {
+      const uint32_t x = max(v[j - 1], v[j]), y = min(v[j - 1], v[j]);
+      v[j - 1] = x;
+      v[j] = y;
+    }
+  }
+  int got = 0;
+#pragma unroll 1
+  for (int it = 0; it < k; ++it) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, v[0]);
+    if (m == 0u) return 0u;
+    const bool mine = v[0] == m;
+    got += __popc(__ballot_sync(0xffffffffu, mine));
+    if (got >= k) return m;
+    if (mine) {
+#pragma unroll
+      for (int e = 0; e + 1 < E; ++e) v[e] = v[e + 1];
+      v[E - 1] = 0u;
+    }
+  }
+  return 0u;
+}
+
+// The k-th largest of the 64 values v0, v1 of the warp's lanes (0 = none),
+// counting repeats, or 0 when there are fewer than k: every value counts the
+// values above it (independent shuffles), and the answer is the smallest
+// value with fewer than k above it.
+__device__ __forceinline__ uint32_t warp_kth64(uint32_t v0, uint32_t v1, int k) {
+  int g0 = 0, g1 = 0;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const uint32_t y0 = __shfl_sync(0xffffffffu, v0, q), y1 = __shfl_sync(0xffffffffu, v1, q);
+    g0 += (y0 > v0) + (y1 > v0);
+    g1 += (y0 > v1) + (y1 > v1);
+  }
+  const uint32_t c0 = g0 < k ? v0 : 0xffffffffu, c1 = g1 < k ? v1 : 0xffffffffu;
+  const uint32_t m = __reduce_min_sync(0xffffffffu, min(c0, c1));
+  return m == 0xffffffffu ? 0u : m;
+}
+
+// A lower bound of the k-th largest of the 64 values v0, v1 of the warp's
+// lanes (0 = none): k rounds each take the largest head over the lanes
+// (redux) and pop it from every lane holding it.  Repeats can pop several
+// values in a round, which only lowers the result; 0 when fewer than k
+// rounds find a value.
+__device__ __forceinline__ uint32_t warp_kth64_lb(uint32_t v0, uint32_t v1, int k) {
+  uint32_t h0 = max(v0, v1), h1 = min(v0, v1);
+  uint32_t m = 0u;
+#pragma unroll 1
+  for (int i = 0; i < k; ++i) {
+    m = __reduce_max_sync(0xffffffffu, h0);
+    const bool pop = h0 == m;
+    h0 = pop ? h1 : h0;
+    h1 = pop ? 0u : h1;
+  }
+  return m;
+}
+
+// The float whose ordered value bits are x (x != 0).
+__device__ __forceinline__ float ordered_value(uint32_t x) {
+  return __uint_as_float((x & 0x80000000u) ? (x & 0x7fffffffu) : ~x);
+}
+
+// A row's threshold from its buffer (one warp, n <= 32 E entries): th = the
+// k-th largest of the entries' lower-key value words, so that the k-th
+// largest lower key of the CTA's pages is at least th << 32, to which thr
+// rises.  With `compact`, only the entries whose upper-key value word
+// reaches th stay -- every entry whose upper key reaches that k-th largest
+// lower key, and at least k.
+template <int E>
+__device__ __forceinline__ void row_threshold(u64* lk, u64* uk, int& n, u64& thr, int k,
+                                              bool compact) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane + 32 * e;
+    v[e] = i < n ? static_cast<uint32_t>(lk[i] >> 32) : 0u;
+  }
+  uint32_t th = 0u;
+  if (n >= k) th = E == 2 ? warp_kth64(v[0], v[E > 1 ? 1 : 0], k) : warp_kth_u32<E>(v, k);
+  const u64 th64 = static_cast<u64>(th) << 32;
+  thr = th64 > thr ? th64 : thr;
+  if (!compact) return;
   int kept = 0;
-  for (int i0 = 0; i0 < nw; i0 += w) {
-    const int i = i0 + j;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane + 32 * e;
     u64 a = 0, b = 0;
     bool keep = false;
-    if (act && i < n) {
-      a = lk[i];
+    if (i < n) {
       b = uk[i];
-      keep = b >= thr;
+      keep = static_cast<uint32_t>(b >> 32) >= th;
+      if (keep) a = lk[i];
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep) & gmask;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
     __syncwarp();
     if (keep) {
       const int pos = kept + __popc(bal & lt);
@@ -492,152 +605,216 @@ __device__ int buffer_keep(u64* lk, u64* uk, int n, u64 thr, int w, bool act) {
       uk[pos] = b;
     }
     kept += __popc(bal);
-    __syncwarp();
-  }
-  return kept;
-}
-
-// Compaction of the rows with `act`: the exact k-th largest lower key
-// becomes the threshold and only the entries whose upper key reaches it stay;
-// a row left with more than `cap` entries (near-ties at the boundary) has its
-// inexact entries rescored exactly (the oracle's arithmetic) and is compacted
-// again, which leaves min(k, n) exact entries.
-template <int DT>
-__device__ void buffer_compact(const ListCtx& L, int r, int k, bool act, const char* qa,
-                               const char* meta_g) {
-  const int j = (threadIdx.x & 31) & (L.w - 1);
-  const int rr = act ? r : 0;
-  u64* lk = L.lk + static_cast<size_t>(rr) * L.lb;
-  u64* uk = L.uk + static_cast<size_t>(rr) * L.lb;
-  u64* scr = L.scr + static_cast<size_t>(threadIdx.x / L.w) * L.sstride;
-  int n = act ? L.n[r] : 0;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const u64 th = group_kth(lk, n, k, L.w, act, scr);
-    const int nk = buffer_keep(lk, uk, n, th, L.w, act);
-    if (act) n = nk;
-    if (act && j == 0) L.thr[r] = th > L.thr[r] ? th : L.thr[r];
-    const bool over = act && n > L.cap;
-    if (DT != LOSA_BF16 || !__any_sync(0xffffffffu, over)) break;
-    if (over) {
-      for (int i = j; i < n; i += L.w)
-        if (lk[i] != uk[i]) {
-          const int p = key_index(lk[i]);
-          const float v = exact_bound_bf16(qa + r * 256, r, meta_g + static_cast<size_t>(p) * 512, p);
-          lk[i] = uk[i] = sel_key(v, p);
-        }
-    }
-    __syncwarp();
   }
   __syncwarp();
-  if (act && j == 0) L.n[r] = n;
-  __syncwarp();
+  n = kept;
 }
 
-// Add np newly scored pages pbase .. pbase + np - 1 (score u = sU[r][e],
-// magnitude t = sT[r][e]) to the buffers of rows 0..R-1: the threshold
-// rises to the k-th largest sub-maximum of the new lower keys (a lower bound
-// of their k-th largest), the new pages whose upper key reaches it join the
-// buffer, and a buffer that could not take another np pages is compacted.
-// Every thread of the CTA calls it.
+// Candidates of one active row after another chunk of np of the CTA's
+// pages (one warp): su[p] the page's tensor-core score (exact for fp32),
+// its interval half-width e = q2.x ||kmin_p|| + q2.y ||kmax_p|| (bf16; every
+// operation rounded up).  The row's list lk/uk[0..cnt) holds every page of
+// the chunks before whose upper key can reach thr, and thr is at most the
+// k-th largest lower key of those pages; afterwards the same holds with this
+// chunk's pages included (cnt <= cap).
+//   1. tau0: the larger of thr's value word and (a lower bound of) the k-th
+//      largest of group maxima of the lower-key value words -- a lower bound
+//      of the k-th largest lower key.  The groups: gm[0..ng) kept by the scoring
+//      threads over all the pages so far (bf16), else (gm null) 64
+//      sub-maxima of this chunk's pages (lane l, pages l + 32 i, one for
+//      even and one for odd i);
+//   2. the list and the chunk's pages whose upper value word reaches tau0
+//      (few) go to the warp's buffer wl/wu (lb entries); a page is tested
+//      with u + emax first (emax >= every page's half-width);
+//   3. more than cap of them: th, the exact k-th largest lower value word
+//      among them, and only the entries whose upper value word reaches it
+//      stay (row_threshold).
+// More than lb entries in step 2 (many near-equal scores) or more than cap
+// left after step 3 take the exact paths.
+struct ListCount {
+  int n;     // entries
+  u64 thr;   // their threshold key
+};
+
 template <int DT>
-__device__ __forceinline__ void list_add_rows(const ListCtx& L, int r, int R, int k,
-                                              const float* sU, const float* sT, int ts, int np,
-                                              int pbase, const char* qa, const char* meta_g) {
-  const int tid = threadIdx.x, lane = tid & 31, W = L.w;
-  const int j = tid & (W - 1);
-  const bool act = r < R;
-  const unsigned gmask = W == 32 ? 0xffffffffu : (((1u << W) - 1u) << (lane & ~(W - 1)));
+__device__ __noinline__ ListCount row_candidates_exact(float* su, int np, int pbase, int k,
+                                                       u64* lk, u64* uk, const char* qrow, int r,
+                                                       const char* meta_g);
+
+template <int DT>
+__device__ __forceinline__ void row_candidates(float* su, const float2* pn, float2 q2, int np,
+                                               int pbase, int k, int cap, int lb, u64* wl,
+                                               u64* wu, u64* lk, u64* uk, int* cnt, u64* thr,
+                                               u64* scr, const char* qrow, int r,
+                                               const char* meta_g, const uint32_t* gm, int ng,
+                                               float emax) {
+  const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  const int rr = act ? r : 0;
-  u64* lk = L.lk + static_cast<size_t>(rr) * L.lb;
-  u64* uk = L.uk + static_cast<size_t>(rr) * L.lb;
-  u64* scr = L.scr + static_cast<size_t>(tid / W) * L.sstride;
-  const float* ur = sU + rr * ts;
-  const float* tr = sT + rr * ts;
-  int n = act ? L.n[r] : 0;
-  u64 thr = act ? L.thr[r] : 0ull;
-  // 1. the new pages whose upper key reaches the running threshold join
-  int m = 0;
-  for (int e0 = 0; e0 < np; e0 += W) {
-    const int e = e0 + j;
-    u64 a = 0, b = 0;
-    bool sv = false;
-    if (act && e < np) {
-      entry_keys(ur[e], tr[e], pbase + e, a, b);
-      sv = b >= thr;
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, sv) & gmask;
-    if (sv) {
-      const int pos = n + m + __popc(bal & lt);
-      lk[pos] = a;
-      uk[pos] = b;
-    }
-    m += __popc(bal);
+  auto half_width = [&](int p) {
+    if (DT != LOSA_BF16) return 0.f;
+    const float2 nk = pn[p];
+    return __fadd_ru(__fmul_ru(q2.x, nk.x), __fmul_ru(q2.y, nk.y));
+  };
+  const int n0 = *cnt;
+  const u64 thr0 = *thr;
+  for (int i = lane; i < n0; i += 32) {
+    wl[i] = lk[i];
+    wu[i] = uk[i];
   }
-  n += m;
-  __syncwarp();
-  // 2. a buffer that could not take another np pages: the threshold rises to
-  //    the k-th largest of the lanes' V sub-maxima of its lower keys (a lower
-  //    bound of its k-th largest) and only the entries reaching it stay
-  const bool full = act && n + ts > L.lb;
-  if (__any_sync(0xffffffffu, full)) {
-    const int V = (k + W - 1) / W;
-    if (full) {
-      for (int v = 0; v < V; ++v) {
-        u64 mx = 0;
-        for (int i = j + W * v; i < n; i += W * V) mx = lk[i] > mx ? lk[i] : mx;
-        scr[j * V + v] = mx;
+  uint32_t gmax[2] = {0u, 0u};
+  if (gm) {
+    gmax[0] = lane < ng ? gm[lane] : 0u;
+    gmax[1] = lane + 32 < ng ? gm[lane + 32] : 0u;
+  } else {
+    int i = 0;
+#pragma unroll 1
+    for (int p = lane; p < np; p += 32, ++i) {
+      const uint32_t lo = ordered_bits(__fsub_rd(su[p], half_width(p)));
+      if (i & 1)
+        gmax[1] = max(gmax[1], lo);
+      else
+        gmax[0] = max(gmax[0], lo);
+    }
+  }
+  const uint32_t t0 = max(warp_kth64_lb(gmax[0], gmax[1], k), static_cast<uint32_t>(thr0 >> 32));
+  const float t0f = t0 ? ordered_value(t0) : -INFINITY;
+  // step 2, 16 pages per lane at a time (pages p00 + 32 i + lane): a mask
+  // of the pages whose u + emax reaches tau0, the exact test of those (few),
+  // then the survivors' places by a prefix sum over the lanes
+  int ns = n0;
+#pragma unroll 1
+  for (int p00 = 0; p00 < np; p00 += 32 * 16) {
+    uint32_t mask = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int p = p00 + 32 * i + lane;
+      if (p < np && __fadd_ru(su[p], emax) >= t0f) mask |= 1u << i;
+    }
+    uint32_t keep = 0u;
+    for (uint32_t m = mask; m; m &= m - 1) {
+      const int i = __ffs(m) - 1, p = p00 + 32 * i + lane;
+      if (ordered_bits(__fadd_ru(su[p], half_width(p))) >= t0) keep |= 1u << i;
+    }
+    const int c = __popc(keep);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = ns + incl - c;
+    for (uint32_t m = keep; m; m &= m - 1, ++pos) {
+      const int i = __ffs(m) - 1, p = p00 + 32 * i + lane;
+      const float u = su[p], e = half_width(p);
+      if (pos < lb) {
+        wl[pos] = sel_key(__fsub_rd(u, e), pbase + p);
+        wu[pos] = sel_key(__fadd_ru(u, e), pbase + p);
       }
+    }
+    ns += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  int n;
+  u64 th = thr0;
+  if (ns > lb || ns > 256) {
+    // this chunk's exact top k beside the list (n0 + k <= lb by the plan)
+    n = n0 + row_candidates_exact<DT>(su, np, pbase, k, wl + n0, wu + n0, qrow, r, meta_g).n;
+  } else {
+    n = ns;
+    th = static_cast<u64>(t0) << 32 > thr0 ? static_cast<u64>(t0) << 32 : thr0;
+  }
+  // more than cap: the exact k-th largest lower value word becomes the
+  // threshold (step 3)
+  if (n > cap) {
+    if (n <= 64)
+      row_threshold<2>(wl, wu, n, th, k, true);
+    else if (n <= 128)
+      row_threshold<4>(wl, wu, n, th, k, true);
+    else
+      row_threshold<8>(wl, wu, n, th, k, true);
+  }
+  if (n > cap) {
+    int* cs = reinterpret_cast<int*>(scr);  // (the slow path's own scratch follows)
+    u64* ts = scr + 1;
+    if (lane == 0) {
+      *cs = n;
+      *ts = th;
     }
     __syncwarp();
-    u64 t2 = 0;
-    if (full && n >= k) {
-      for (int v = 0; v < V; ++v) {
-        const u64 x = scr[j * V + v];
-        int rk = 0;
-        for (int q = 0; q < W * V; ++q) {
-          const u64 y = scr[q];
-          rk += (y > x) || (y == x && q < j * V + v);
-        }
-        if (rk == k - 1) t2 = x;
-      }
-    }
-    for (int o = 1; o < W; o <<= 1) {
-      const u64 y = __shfl_xor_sync(0xffffffffu, t2, o);
-      t2 = y > t2 ? y : t2;
-    }
-    thr = t2 > thr ? t2 : thr;
-    const int nk = buffer_keep(lk, uk, n, thr, W, full);
-    if (full) n = nk;
+    row_compact_slow<DT>(wl, wu, cs, ts, k, cap, scr + 2, qrow, r, meta_g);
+    n = *cs;
+    th = *ts;
+    __syncwarp();
   }
-  if (act && j == 0) {
-    L.n[r] = n;
-    L.thr[r] = thr;
+  // the row's list (at most cap entries)
+  for (int i = lane; i < n; i += 32) {
+    lk[i] = wl[i];
+    uk[i] = wu[i];
+  }
+  if (lane == 0) {
+    *cnt = n;
+    *thr = th;
   }
   __syncwarp();
-  // 3. still too full (many near-equal keys): exact compaction
-  const bool still = act && n + ts > L.lb;
-  if (__any_sync(0xffffffffu, still)) buffer_compact<DT>(L, r, k, still, qa, meta_g);
 }
 
+// The exact path (many near-equal scores): every page of the row is
+// rescored exactly (the oracle's arithmetic; fp32 scores are exact already)
+// and the row's list gets exactly its top min(k, np) pages by exact key
+// (value descending, lower page first), thr the k-th of them.
 template <int DT>
-__device__ __forceinline__ void list_add(const ListCtx& L, int R, int k, const float* sU,
-                                         const float* sT, int ts, int np, int pbase,
-                                         const char* qa, const char* meta_g) {
+__device__ __noinline__ ListCount row_candidates_exact(float* su, int np, int pbase, int k,
+                                                       u64* lk, u64* uk, const char* qrow, int r,
+                                                       const char* meta_g) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  if (DT == LOSA_BF16) {
 #pragma unroll 1
-  for (int r0 = 0; r0 < R; r0 += kThreads / L.w)
-    list_add_rows<DT>(L, r0 + static_cast<int>(threadIdx.x) / L.w, R, k, sU, sT, ts, np, pbase,
-                      qa, meta_g);
+    for (int p = lane; p < np; p += 32)
+      su[p] = exact_bound_bf16(qrow, r, meta_g + static_cast<size_t>(pbase + p) * 512, pbase + p);
+    __syncwarp();
+  }
+  const int kk = min(k, np);
+  // X: the largest value word with at least kk pages at or above it
+  uint32_t X = 0u;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = X | (1u << bit);
+    int c = 0;
+    for (int p = lane; p < np; p += 32) c += ordered_bits(su[p]) >= cand;
+    if (__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)) >= static_cast<unsigned>(kk)) X = cand;
+  }
+  int above = 0;
+  for (int p = lane; p < np; p += 32) above += ordered_bits(su[p]) > X;
+  const int need_eq = kk - static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(above)));
+  // every page above X, then the first need_eq pages (in page order) at X
+  int n = 0, eq = 0;
+#pragma unroll 1
+  for (int p0 = 0; p0 < np; p0 += 32) {
+    const int p = p0 + lane;
+    const uint32_t x = p < np ? ordered_bits(su[p]) : 0u;
+    const bool at = p < np && x == X;
+    const unsigned bal_eq = __ballot_sync(0xffffffffu, at);
+    const bool in = (p < np && x > X) || (at && eq + __popc(bal_eq & lt) < need_eq);
+    eq += __popc(bal_eq);
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in) {
+      const int pos = n + __popc(bal & lt);
+      lk[pos] = uk[pos] = sel_key(su[p], pbase + p);
+    }
+    n += __popc(bal);
+  }
+  __syncwarp();
+  return ListCount{n, static_cast<u64>(X) << 32};  // (warp-uniform)
 }
 
 // ---------------------------------------------------------------------------
 // Merge of one active row's lists from the C CTAs of the cluster (one warp):
 // the row's k pages, exactly the oracle's top k (value descending, lower page
 // first), written ascending to sel[0..k) (then -1 when the sequence has fewer
-// pages).  `buf` is the warp's scratch: lk[cap_all], uk[cap_all],
-// kRecSlots staged records of 512 bytes, flag[cap_all], then the k-th
-// selection's scratch (32 * ceil(k / 32) + 1 + cap_all keys).
+// pages).  `buf` is the warp's scratch for the rare paths: lk[cap_all],
+// uk[cap_all], kRecSlots staged records of 512 bytes, flag[cap_all], then the
+// k-th selection's scratch (32 * ceil(k / 32) + cap_all keys).
 // ---------------------------------------------------------------------------
 struct MergeCtx {
   const u64* lk;   // this CTA's list arrays (the same offsets in every CTA)
@@ -649,51 +826,154 @@ struct MergeCtx {
   int C;
 };
 
+struct CtaOffsets {
+  int v[8];  // first entry of each CTA's list in the concatenation (unused CTAs: INT_MAX)
+};
+
+// More candidates than k (near-ties at the boundary; blk/buk[0..nca) hold
+// them).  lkth: a key that no page outside the candidates reaches with its
+// upper key (the candidates' lower bound and the merge's tau0, whichever is
+// larger).  A candidate whose lower key reaches lkth and that at most k - 1
+// other candidates can beat (their upper key above its lower key) is in; the
+// others are rescored exactly (the oracle's arithmetic) and the best of them
+// by exact key fill the rest.  (The true top k are all candidates, so this
+// is exactly the top k.)  Writes sel[0..k).
 template <int DT>
-__device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf, int32_t* sel,
-                                       const char* qa, const char* meta_g) {
+__device__ __noinline__ void merge_resolve(u64* blk, u64* buk, int* flag, char* recs, int nca,
+                                           int k, u64 lkth, int32_t* sel, const char* qrow, int r,
+                                           const char* meta_g) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  u64* blk = reinterpret_cast<u64*>(buf);
-  u64* buk = blk + M.cap_all;
-  char* recs = reinterpret_cast<char*>(buk + M.cap_all);
-  int* flag = reinterpret_cast<int*>(recs + kRecSlots * 512);
-  u64* kscr = reinterpret_cast<u64*>(flag + ((M.cap_all + 1) & ~1));
-  // 1. the largest of the CTAs' thresholds bounds the group's k-th largest
-  //    lower key from below; only entries whose upper key reaches it matter
-  int nc = 0;
-  u64 th = 0;
-  if (lane < M.C) {
-    nc = ld_dsmem_s32(dsmem(M.n + r, lane));
-    th = ld_dsmem_u64(dsmem(M.thr + r, lane));
+  int ncert = 0;
+#pragma unroll 1
+  for (int e0 = 0; e0 < nca; e0 += 32) {
+    const int e = e0 + lane;
+    bool cert = false;
+    if (e < nca && blk[e] >= lkth) {
+      int beat = 0;
+      for (int e2 = 0; e2 < nca; ++e2) beat += (e2 != e) && (buk[e2] > blk[e]);
+      cert = beat <= k - 1;
+    }
+    if (e < nca) flag[e] = cert ? 1 : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, cert);
+    if (cert) sel[ncert + __popc(bal & lt)] = key_index(blk[e]);
+    ncert += __popc(bal);
   }
-  const u64 tau0 = warp_max_u64(th);
-  int incl = nc;
+  __syncwarp();
+  if (DT == LOSA_BF16) {  // fp32 scores are exact already
+#pragma unroll 1
+    for (int e0 = 0; e0 < nca; e0 += kRecSlots) {
+#pragma unroll 1
+      for (int q = 0; q < kRecSlots && e0 + q < nca; ++q) {
+        const int e = e0 + q;
+        if (!flag[e] && blk[e] != buk[e]) {
+          const int p = key_index(blk[e]);
+          reinterpret_cast<uint4*>(recs + q * 512)[lane] =
+              reinterpret_cast<const uint4*>(meta_g + static_cast<size_t>(p) * 512)[lane];
+        }
+      }
+      __syncwarp();
+      if (lane < kRecSlots && e0 + lane < nca) {
+        const int e = e0 + lane;
+        if (!flag[e] && blk[e] != buk[e]) {
+          const int p = key_index(blk[e]);
+          const float v = exact_bound_bf16(qrow, r, recs + lane * 512, p);
+          blk[e] = buk[e] = sel_key(v, p);
+        }
+      }
+      __syncwarp();
+    }
+  }
+  const int need = k - ncert;
+#pragma unroll 1
+  for (int e = lane; e < nca; e += 32) {
+    if (flag[e]) continue;
+    int rk = 0;
+    for (int e2 = 0; e2 < nca; ++e2) rk += !flag[e2] && blk[e2] > blk[e];
+    if (rk < need) sel[ncert + rk] = key_index(blk[e]);
+  }
+  __syncwarp();
+}
+
+// The row's entries whose upper key reaches tau0, gathered from the C CTAs
+// into registers (E per lane; lane l takes entries l, l + 32, ... of the
+// CTAs' lists in CTA order), a lower bound lkth of their k-th largest lower
+// key, and its candidates (upper key >= lkth: a superset of the true top k):
+// sel when there are at most k of them, else blk/buk for merge_resolve.
+// Returns the number of candidates.
+template <int E>
+__device__ __forceinline__ int merge_gather(const MergeCtx& M, int r, int k, u64 tau0, int total,
+                                            const CtaOffsets& offs, int32_t* sel, u64* blk,
+                                            u64* buk, u64& lkth) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  u64 a[E], b[E];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, 31);
-  int offs[8];
+  for (int e = 0; e < E; ++e) {
+    const int f = lane + 32 * e;
+    a[e] = b[e] = 0ull;
+    if (f < total) {
+      int cf = 0;
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const int v = __shfl_sync(0xffffffffu, incl - nc, q);
-    offs[q] = q < M.C ? v : 0x7fffffff;
+      for (int q = 1; q < 8; ++q) cf += f >= offs.v[q];
+      const size_t i = static_cast<size_t>(r) * M.lb + (f - offs.v[cf]);
+      const u64 y = ld_dsmem_u64(dsmem(M.uk + i, cf));
+      const u64 x = ld_dsmem_u64(dsmem(M.lk + i, cf));
+      if (y >= tau0) {
+        a[e] = x;
+        b[e] = y;
+      }
+    }
   }
+  // lkth: the k-th largest lower-key value word, as a key (at most the k-th
+  // largest lower key: the candidates below are a superset of the exact ones)
+  uint32_t v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = static_cast<uint32_t>(a[e] >> 32);
+  lkth = static_cast<u64>(warp_kth_u32<E>(v, k)) << 32;
+  int nca = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) nca += __popc(__ballot_sync(0xffffffffu, b[e] != 0ull && b[e] >= lkth));
+  int pos = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const bool c = b[e] != 0ull && b[e] >= lkth;
+    const unsigned bal = __ballot_sync(0xffffffffu, c);
+    if (c) {
+      const int at = pos + __popc(bal & lt);
+      if (nca <= k) {
+        sel[at] = key_index(a[e]);
+      } else {
+        blk[at] = a[e];
+        buk[at] = b[e];
+      }
+    }
+    pos += __popc(bal);
+  }
+  __syncwarp();
+  return nca;
+}
+
+// The same for a row with more than 256 entries reaching tau0 (large k):
+// gathered into shared memory.
+
+__device__ __noinline__ int merge_gather_smem(const MergeCtx M, int r, int k, u64 tau0,
+                                              int total, const CtaOffsets offs, int32_t* sel,
+                                              u64* blk, u64* buk, u64* kscr, u64* lkth_out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
   int cnt = 0;
+#pragma unroll 1
   for (int f0 = 0; f0 < total; f0 += 32) {
     const int f = f0 + lane;
     u64 a = 0, b = 0;
     bool in = false;
     if (f < total) {
       int cf = 0;
-#pragma unroll
-      for (int q = 1; q < 8; ++q) cf += f >= offs[q];
-      const int i = f - offs[cf];
-      const size_t e = static_cast<size_t>(r) * M.lb + i;
-      b = ld_dsmem_u64(dsmem(M.uk + e, cf));
-      a = ld_dsmem_u64(dsmem(M.lk + e, cf));
+      for (int q = 1; q < 8; ++q) cf += f >= offs.v[q];
+      const size_t i = static_cast<size_t>(r) * M.lb + (f - offs.v[cf]);
+      b = ld_dsmem_u64(dsmem(M.uk + i, cf));
+      a = ld_dsmem_u64(dsmem(M.lk + i, cf));
       in = b >= tau0;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, in);
@@ -705,17 +985,14 @@ __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf
     cnt += __popc(bal);
   }
   __syncwarp();
-  // 2. the group's k-th largest lower key (0: fewer than k pages in all)
-  const int N = cnt;
-  const u64 lkth = group_kth(blk, N, k, 32, true, kscr);
-  // 3. candidates: upper key at or above it (they hold the true top k),
-  //    compacted to the front in place
+  const u64 lkth = warp_kth(blk, cnt, k, kscr);
   int nca = 0;
-  for (int e0 = 0; e0 < N; e0 += 32) {
+#pragma unroll 1
+  for (int e0 = 0; e0 < cnt; e0 += 32) {
     const int e = e0 + lane;
     u64 a = 0, b = 0;
     bool c = false;
-    if (e < N) {
+    if (e < cnt) {
       a = blk[e];
       b = buk[e];
       c = b >= lkth;
@@ -730,64 +1007,57 @@ __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf
     nca += __popc(bal);
     __syncwarp();
   }
-  // 4. more candidates than k.  A candidate whose lower key reaches the k-th
-  //    largest lower key and that at most k - 1 others can beat (their upper
-  //    key above its lower key) is in; the others are rescored exactly (the
-  //    oracle's arithmetic) and the best of them by exact key fill the rest.
-  //    (The true top k are all candidates, so this is exactly the top k.)
-  int nsel = 0;
-  if (nca <= k) {
+  if (nca <= k)
     for (int e = lane; e < nca; e += 32) sel[e] = key_index(blk[e]);
-    nsel = nca;
-  } else {
-    int ncert = 0;
-    for (int e0 = 0; e0 < nca; e0 += 32) {
-      const int e = e0 + lane;
-      bool cert = false;
-      if (e < nca && blk[e] >= lkth) {
-        int beat = 0;
-        for (int e2 = 0; e2 < nca; ++e2) beat += (e2 != e) && (buk[e2] > blk[e]);
-        cert = beat <= k - 1;
-      }
-      if (e < nca) flag[e] = cert ? 1 : 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, cert);
-      if (cert) sel[ncert + __popc(bal & lt)] = key_index(blk[e]);
-      ncert += __popc(bal);
-    }
-    __syncwarp();
-    if (DT == LOSA_BF16) {  // fp32 scores are exact already
-      for (int e0 = 0; e0 < nca; e0 += kRecSlots) {
-        for (int q = 0; q < kRecSlots && e0 + q < nca; ++q) {
-          const int e = e0 + q;
-          if (!flag[e] && blk[e] != buk[e]) {
-            const int p = key_index(blk[e]);
-            reinterpret_cast<uint4*>(recs + q * 512)[lane] =
-                reinterpret_cast<const uint4*>(meta_g + static_cast<size_t>(p) * 512)[lane];
-          }
-        }
-        __syncwarp();
-        if (lane < kRecSlots && e0 + lane < nca) {
-          const int e = e0 + lane;
-          if (!flag[e] && blk[e] != buk[e]) {
-            const int p = key_index(blk[e]);
-            const float v = exact_bound_bf16(qa + r * 256, r, recs + lane * 512, p);
-            blk[e] = buk[e] = sel_key(v, p);
-          }
-        }
-        __syncwarp();
-      }
-    }
-    const int need = k - ncert;
-    for (int e = lane; e < nca; e += 32) {
-      if (flag[e]) continue;
-      int rk = 0;
-      for (int e2 = 0; e2 < nca; ++e2) rk += !flag[e2] && blk[e2] > blk[e];
-      if (rk < need) sel[ncert + rk] = key_index(blk[e]);
-    }
-    nsel = k;
-  }
   __syncwarp();
-  // 5. ascending page order, then -1 past the selection
+  *lkth_out = lkth;
+  return nca;
+}
+
+template <int DT>
+__device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, char* buf,
+                                          int32_t* sel, const char* qa, const char* meta_g) {
+  const int lane = threadIdx.x & 31;
+  u64* blk = reinterpret_cast<u64*>(buf);
+  u64* buk = blk + M.cap_all;
+  char* recs = reinterpret_cast<char*>(buk + M.cap_all);
+  int* flag = reinterpret_cast<int*>(recs + kRecSlots * 512);
+  u64* kscr = reinterpret_cast<u64*>(flag + ((M.cap_all + 1) & ~1));
+  // the largest of the CTAs' thresholds bounds the group's k-th largest
+  // lower key from below: only entries whose upper key reaches it matter
+  int nc = 0;
+  u64 th = 0;
+  if (lane < M.C) {
+    nc = ld_dsmem_s32(dsmem(M.n + r, lane));
+    th = ld_dsmem_u64(dsmem(M.thr + r, lane));
+  }
+  const u64 tau0 = warp_max_u64(th);
+  int incl = nc;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 7);
+  CtaOffsets offs;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int v = __shfl_sync(0xffffffffu, incl - nc, q);
+    offs.v[q] = q < M.C ? v : 0x7fffffff;
+  }
+  u64 lkth = 0;
+  int nca;
+  if (total <= 128)
+    nca = merge_gather<4>(M, r, k, tau0, total, offs, sel, blk, buk, lkth);
+  else if (total <= 256)
+    nca = merge_gather<8>(M, r, k, tau0, total, offs, sel, blk, buk, lkth);
+  else
+    nca = merge_gather_smem(M, r, k, tau0, total, offs, sel, blk, buk, kscr, &lkth);
+  if (nca > k)
+    merge_resolve<DT>(blk, buk, flag, recs, nca, k, lkth > tau0 ? lkth : tau0, sel, qa + r * 256,
+                      r, meta_g);
+  const int nsel = min(nca, k);
+  // ascending page order, then -1 past the selection
   int pv[4];
   int pr[4];
 #pragma unroll
@@ -815,8 +1085,8 @@ __device__ __noinline__ void merge_row(const MergeCtx M, int r, int k, char* buf
 struct StepLayout {
   int ring;     // metadata ring; afterwards merge scratch, gathered pages, warp partials
   int qc, qp;   // the group's queries (current, previous) [GB][rowb]
-  int lists;    // candidate buffers lk [R][lb], uk [R][lb], then their scratch [R][sstride]
-  int sc;       // scores of the pages being added: sU [R][ts], sT [R][ts]
+  int lists;    // candidate lists lk, uk [R][lcap]; per warp survivors [2][lb] and scratch [sstride]
+  int sc;       // fp32: the warps' probability rows (16 floats each)
   int part_o;   // the CTA's partial outputs [R16][kD] floats (bf16: in the ring)
   int part_ml;  // the CTA's partial (m, l) [R16][2] (bf16: in the ring)
   int qa;       // active rows' q_cur [R16][rowb] (bf16 chunks swizzled by row)
@@ -829,6 +1099,11 @@ struct StepLayout {
   int bitmap, wbase;   // union bitmap and its words' prefix counts
   int lpages, masks;   // this CTA's union pages and their row masks
   int misc;            // per-token / per-row ints and scalars
+  int scores;          // the active rows' bound scores of the CTA's pages [R][cp] floats
+  int pnorm;           // the CTA's page norms [cp] float2 (bf16)
+  int gmx, emx;        // bf16: the rows' group maxima [R16][8 * warps per m16 tile] and
+                       // largest half-widths [R16]
+  int qn;              // active rows' 2^-14 ||q-||, 2^-14 ||q+|| [R16] float2
   int mbar;            // kMaxStages ring barriers, the queries', the gather's
   int total;
 };
@@ -837,6 +1112,7 @@ struct StepParams {
   const void* qc;
   const void* qp;
   const char* meta;
+  const float2* norms;  // the page-norm section of the metadata (row stride pn)
   const void* K;
   const void* V;
   const void* kb;
@@ -856,16 +1132,16 @@ struct StepParams {
   int tile;        // pages per ring stage
   int stages;      // ring stages
   int rec;         // bytes per metadata record
-  int ts;          // pages per list update (a multiple of 8)
-  int lw;          // lanes per row in a list update
-  int lb, lcap;    // buffer entries per row; entries left after a compaction before an exact refinement
-  int sstride;     // scratch keys per row (sub-maxima, survivors, broadcast)
+  int spc;         // pages per score chunk (a multiple of the stage's pages)
+  int lb, lcap;    // survivor buffer entries per warp; list entries per row (k + slack)
+  int sstride;     // scratch keys per warp for the exact paths
   int qstride;     // bytes per staged query row (padded: no bank conflicts between rows)
   int nmw;         // merge warps
   int mstride;     // bytes of a merge warp's scratch (in the ring area)
   int max_lp;      // union pages per CTA, at most
   int ngp;         // union pages in flight per CTA
   int early;       // release the dependent launch at the start (the grid fits one wave)
+  int pn;          // page-norm entries per (sequence, KV head)
   StepLayout lo;
 };
 
@@ -923,12 +1199,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   // pages are consumed, fp32 in its own area (its running state lives there)
   float* part_o = reinterpret_cast<float*>(smem + lo.part_o);
   float* part_ml = reinterpret_cast<float*>(smem + lo.part_ml);
+  // the rows' candidate lists [R][lcap], then per warp its survivor buffer
+  // [lb] (lower and upper keys) and the exact paths' scratch [sstride]
   u64* l_lk = reinterpret_cast<u64*>(smem + lo.lists);
-  u64* l_uk = l_lk + static_cast<size_t>(R) * prm.lb;
-  u64* l_scr = l_uk + static_cast<size_t>(R) * prm.lb;
+  u64* l_uk = l_lk + static_cast<size_t>(R) * prm.lcap;
+  u64* w_lk = l_uk + static_cast<size_t>(R) * prm.lcap + static_cast<size_t>(warp) * 2 * prm.lb;
+  u64* w_uk = w_lk + prm.lb;
+  u64* w_scr = l_uk + static_cast<size_t>(R) * prm.lcap + static_cast<size_t>(kWarps) * 2 * prm.lb +
+               static_cast<size_t>(warp) * prm.sstride;
   const int qst = prm.qstride;
-  float* sU = reinterpret_cast<float*>(smem + lo.sc);
-  float* sT = sU + R * prm.ts;
+  float* fscr = reinterpret_cast<float*>(smem + lo.sc);
   int* l_n = reinterpret_cast<int*>(smem + lo.l_n);
   u64* l_thr = reinterpret_cast<u64*>(smem + lo.l_thr);
   int32_t* sel_all = reinterpret_cast<int32_t*>(smem + lo.sel);
@@ -944,6 +1224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* sfx_tok = misc + kMiscSfxTok;
   int32_t* scal = misc + kMiscScal;
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + lo.mbar);
+  float* scores = reinterpret_cast<float*>(smem + lo.scores);
+  float2* pnorm = reinterpret_cast<float2*>(smem + lo.pnorm);
+  uint32_t* gmx = reinterpret_cast<uint32_t*>(smem + lo.gmx);
+  uint32_t* emx = reinterpret_cast<uint32_t*>(smem + lo.emx);
+  float2* qn = reinterpret_cast<float2*>(smem + lo.qn);
   uint64_t* gbar = mbar + kMaxStages;  // [2]: the gather's two page buffers
 
   // the next kernel of the stream may be scheduled now when this grid fits
@@ -960,6 +1245,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int npg = sel ? max(0, min(Ps, pr0 + prm.cp) - pr0) : 0;
   const int nstg = (npg + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.Pc * prm.rec;
+  const float2* norm_g = prm.norms + static_cast<size_t>(sg) * prm.pn;
+  // ring stage t (slot t % stages): its records; stage 0 also brings (bf16)
+  // the norms of all the CTA's pages, rounded up to a 16-byte copy (the norm
+  // rows are padded to 8 entries)
+  auto issue_stage = [&](int t) {
+    const int st = t % prm.stages;
+    const int np = min(prm.tile, npg - t * prm.tile);
+    const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
+    const uint32_t nbytes =
+        DT == LOSA_BF16 && t == 0 ? static_cast<uint32_t>((npg + 1) / 2 * 16) : 0u;
+    mbar_expect_tx(&mbar[st], bytes + nbytes);
+    bulk_g2s(ring + st * kStageBytes, meta_g + static_cast<size_t>(pr0 + t * prm.tile) * prm.rec,
+             bytes, &mbar[st]);
+    if (nbytes) bulk_g2s(pnorm, norm_g + pr0, nbytes, &mbar[st]);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < kMaxStages + 2; ++i) mbar_init(&mbar[i], 1);
@@ -967,13 +1267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     scal[kSFail] = 0;
     if (c == 0 && g == 0 && seq_len_bad(d, s)) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
 #pragma unroll 1
-    for (int t = 0; t < min(nstg, prm.stages); ++t) {
-      const int np = min(prm.tile, npg - t * prm.tile);
-      const uint32_t bytes = static_cast<uint32_t>(np * prm.rec);
-      mbar_expect_tx(&mbar[t], bytes);
-      bulk_g2s(ring + t * kStageBytes, meta_g + static_cast<size_t>(pr0 + t * prm.tile) * prm.rec,
-               bytes, &mbar[t]);
-    }
+    for (int t = 0; t < min(nstg, prm.stages); ++t) issue_stage(t);
   }
   // the group's current and previous queries (cp.async group 0), rows
   // padded to qst bytes
@@ -1065,6 +1359,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
+  // ---- the active rows' interval factors 2^-14 ||q-||, 2^-14 ||q+|| (bf16;
+  // one warp per row, every operation rounded up)
+  if (DT == LOSA_BF16) {
+#pragma unroll 1
+    for (int r = warp; r < R; r += kWarps) {
+      const uint2 w = *reinterpret_cast<const uint2*>(qcs + act_row[r] * qst + 8 * lane);
+      const float x[4] = {__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                          __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u)};
+      float sn = 0.f, sp = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (__float_as_uint(x[i]) & 0x80000000u)
+          sn = __fmaf_ru(x[i], x[i], sn);
+        else
+          sp = __fmaf_ru(x[i], x[i], sp);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        sn = __fadd_ru(sn, __shfl_xor_sync(0xffffffffu, sn, o));
+        sp = __fadd_ru(sp, __shfl_xor_sync(0xffffffffu, sp, o));
+      }
+      if (lane == 0)
+        qn[r] = make_float2(__fmul_ru(__fsqrt_ru(sn), kEpsScale), __fmul_ru(__fsqrt_ru(sp), kEpsScale));
+    }
+  }
+
   // ---- active rows' q_cur for the page tiles and the exact rescoring
   if (DT == LOSA_BF16) {
 #pragma unroll 1
@@ -1136,31 +1456,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool sw = sel && mt < ntm;
   uint32_t a[16][4];
   if (DT == LOSA_BF16 && sw) {
-    // m16n8k16 A fragment of [q- | q+] (K = 256): a[ks][0] row g4 and a[ks][1]
-    // row g4 + 8 at columns 16 ks + 2 t4 (+1), a[ks][2..3] the same rows at
-    // columns + 8; column j < 128 is q-_j = min(q_j, 0), column 128 + j is
-    // q+_j = max(q_j, 0) (sign bit tests, exact)
-    const int rA = mt * 16 + g4, rB = rA + 8;
-    const char* qrA = rA < R ? qcs + act_row[rA] * qst : nullptr;
-    const char* qrB = rB < R ? qcs + act_row[rB] * qst : nullptr;
-    auto part = [](uint32_t w, bool neg) {
-      uint32_t lo16 = w & 0xffffu, hi16 = w >> 16;
-      const bool nl = lo16 & 0x8000u, nh = hi16 & 0x8000u;
-      lo16 = (nl == neg) ? lo16 : 0u;
-      hi16 = (nh == neg) ? hi16 : 0u;
-      return lo16 | (hi16 << 16);
-    };
+    // m16n8k16 A fragments of [q- | q+] (K = 256): ldmatrix of the active
+    // rows' q_cur (8 channel steps of 16), then a[kc] = the negative part
+    // and a[kc + 8] = the non-negative part (sign bit tests, exact; -0 goes
+    // to q-).  a[.][0] and a[.][2] hold row g4, a[.][1] and a[.][3] row g4 + 8.
+    const int mi = lane >> 3, trow = mt * 16 + (mi & 1) * 8 + (lane & 7);
+    const char* qsrc = qcs + act_row[trow < R ? trow : 0] * qst + (mi >> 1) * 16;
+    const bool okA = mt * 16 + g4 < R, okB = mt * 16 + g4 + 8 < R;
 #pragma unroll
-    for (int ks = 0; ks < 16; ++ks) {
+    for (int kc = 0; kc < 8; ++kc) {
+      uint32_t w[4];
+      ldsm_x4(su32(qsrc + kc * 32), w[0], w[1], w[2], w[3]);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int col = ks * 16 + 2 * t4 + 8 * hf;
-        const int ch = col & 127;
-        const bool neg = col < 128;
-        const uint32_t wA = qrA ? *reinterpret_cast<const uint32_t*>(qrA + ch * 2) : 0u;
-        const uint32_t wB = qrB ? *reinterpret_cast<const uint32_t*>(qrB + ch * 2) : 0u;
-        a[ks][2 * hf] = part(wA, neg);
-        a[ks][2 * hf + 1] = part(wB, neg);
+      for (int j = 0; j < 4; ++j) {
+        const bool okr = (j & 1) ? okB : okA;
+        const uint32_t x = okr ? w[j] : 0u;
+        const uint32_t neg = ((x >> 15) & 0x00010001u) * 0xffffu;
+        a[kc][j] = x & neg;
+        a[kc + 8][j] = x & ~neg;
       }
     }
   }
@@ -1168,96 +1481,127 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int r = tid; r < R; r += kThreads) {
     l_n[r] = 0;
     l_thr[r] = 0ull;
+    if (DT == LOSA_BF16 && sel) emx[r] = 0u;
   }
-  __syncthreads();  // the query area becomes the list area
+  __syncthreads();  // the query area becomes the buffer area
 
-  // ---- bound scores of this CTA's pages, stage by stage, into the rows'
-  // candidate lists
-  const ListCtx LC = {l_lk, l_uk, l_n, l_thr, l_scr, prm.lb, prm.lcap, prm.sstride, prm.lw};
+  // ---- bound scores of this CTA's pages, stage by stage, stored per row
+  // for a chunk of spc pages (scores[r][p - chunk start]); a stage's slot is
+  // refilled once every warp has read it, and after a chunk's last stage
+  // each active row's candidates take in the chunk's pages (one warp per
+  // row)
+  const int rA = mt * 16 + g4, rB = rA + 8;
+  const int spc = prm.spc;
+  // bf16: each scoring thread keeps, for its two rows, the maxima of the
+  // lower-key value words of its pages in two groups (n-tile parity) and the
+  // largest half-width; they go to gmx [R16][ng] and emx [R16] before each
+  // chunk's selection
+  const int ng = 8 * wpm;
+  uint32_t gA0 = 0u, gA1 = 0u, gB0 = 0u, gB1 = 0u;
+  float eA = 0.f, eB = 0.f;
+  const float2 qnA = DT == LOSA_BF16 && sw && rA < R ? qn[rA] : make_float2(0.f, 0.f);
+  const float2 qnB = DT == LOSA_BF16 && sw && rB < R ? qn[rB] : make_float2(0.f, 0.f);
 #pragma unroll 1
   for (int t = 0; t < nstg; ++t) {
     const int st = t % prm.stages;
     const uint32_t parity = (t / prm.stages) & 1;
-    if (scal[kSFail] == 0 && !mbar_wait(&mbar[st], parity)) scal[kSFail] = 1;
-    __syncthreads();
-    const bool ok = scal[kSFail] == 0;
     const char* stage = ring + st * kStageBytes;
     const int nps = min(prm.tile, npg - t * prm.tile);
+    const int pl0 = t * prm.tile;  // the stage's first page (CTA-local)
+    // each thread waits for the stage itself (the wait makes the bytes the
+    // copy wrote visible to it)
+    if (scal[kSFail] == 0 && mbar_wait(&mbar[st], parity)) {
+      if (DT == LOSA_BF16) {
+        const int nnt = (nps + 7) / 8;
 #pragma unroll 1
-    for (int o = 0; o < nps; o += prm.ts) {
-      const int np = min(prm.ts, nps - o);
-      const int pbase = pr0 + t * prm.tile + o;
-      if (ok) {
-        if (DT == LOSA_BF16) {
-          const int nt0 = o / 8, nnt = (np + 7) / 8;
-#pragma unroll 1
-          for (int nt = sub; sw && nt < nnt; nt += wpm) {
-            float u[4], tt[4];
-            bound_ntile2(a, stage + (nt0 + nt) * 8 * 512, u, tt);
-            const int e = nt * 8 + 2 * t4;
-            const int r0 = mt * 16 + g4;
-            if (r0 < R) {
-              sU[r0 * prm.ts + e] = u[0];
-              sU[r0 * prm.ts + e + 1] = u[1];
-              sT[r0 * prm.ts + e] = tt[0];
-              sT[r0 * prm.ts + e + 1] = tt[1];
+        for (int nt = sub; sw && nt < nnt; nt += wpm) {
+          float u[4];
+          bound_ntile(a, stage + nt * 8 * 512, u);
+          const int pl = pl0 + nt * 8 + 2 * t4;  // this lane's pages pl, pl + 1 (pl even)
+          if (pl < npg) {  // (pl + 1 stays inside the chunk's row: spc is even)
+            const int ps = pl % spc;
+            if (rA < R) *reinterpret_cast<float2*>(scores + rA * spc + ps) = make_float2(u[0], u[1]);
+            if (rB < R) *reinterpret_cast<float2*>(scores + rB * spc + ps) = make_float2(u[2], u[3]);
+            const float4 nk = *reinterpret_cast<const float4*>(pnorm + pl);
+            const bool v1 = pl + 1 < npg;
+            const float e0 = __fadd_ru(__fmul_ru(qnA.x, nk.x), __fmul_ru(qnA.y, nk.y));
+            const float e1 = v1 ? __fadd_ru(__fmul_ru(qnA.x, nk.z), __fmul_ru(qnA.y, nk.w)) : 0.f;
+            const float e2 = __fadd_ru(__fmul_ru(qnB.x, nk.x), __fmul_ru(qnB.y, nk.y));
+            const float e3 = v1 ? __fadd_ru(__fmul_ru(qnB.x, nk.z), __fmul_ru(qnB.y, nk.w)) : 0.f;
+            const uint32_t lA = max(ordered_bits(__fsub_rd(u[0], e0)),
+                                    v1 ? ordered_bits(__fsub_rd(u[1], e1)) : 0u);
+            const uint32_t lB = max(ordered_bits(__fsub_rd(u[2], e2)),
+                                    v1 ? ordered_bits(__fsub_rd(u[3], e3)) : 0u);
+            if (nt & 1) {
+              gA1 = max(gA1, lA);
+              gB1 = max(gB1, lB);
+            } else {
+              gA0 = max(gA0, lA);
+              gB0 = max(gB0, lB);
             }
-            if (r0 + 8 < R) {
-              sU[(r0 + 8) * prm.ts + e] = u[2];
-              sU[(r0 + 8) * prm.ts + e + 1] = u[3];
-              sT[(r0 + 8) * prm.ts + e] = tt[2];
-              sT[(r0 + 8) * prm.ts + e + 1] = tt[3];
-            }
-          }
-        } else {
-          // fp32: exact scores on CUDA cores (the oracle's arithmetic)
-#pragma unroll 1
-          for (int e = tid; e < np * R; e += kThreads) {
-            const int pl = e % np, r = e / np;
-            const int pg = pbase + pl;
-            const char* recp = stage + (o + pl) * prm.rec;
-            const float* q = reinterpret_cast<const float*>(qa + r * rowb);
-            float acc = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < kD / 4; ++cc) {
-              const float4 mn = *reinterpret_cast<const float4*>(recp + meta_swz(16u * cc, pg));
-              const float4 mx =
-                  *reinterpret_cast<const float4*>(recp + meta_swz(16u * (cc + kD / 4), pg));
-              const float mns[4] = {mn.x, mn.y, mn.z, mn.w}, mxs[4] = {mx.x, mx.y, mx.z, mx.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const float qi = q[4 * cc + u];
-                acc = __fadd_rn(acc, fmaxf(__fmul_rn(qi, mxs[u]), __fmul_rn(qi, mns[u])));
-              }
-            }
-            sU[r * prm.ts + pl] = acc;
-            sT[r * prm.ts + pl] = 0.f;
+            eA = fmaxf(eA, fmaxf(e0, e1));
+            eB = fmaxf(eB, fmaxf(e2, e3));
           }
         }
+      } else {
+        // fp32: exact scores on CUDA cores (the oracle's arithmetic)
+#pragma unroll 1
+        for (int e = tid; e < nps * R; e += kThreads) {
+          const int pl = e % nps, r = e / nps;
+          const int pg = pr0 + pl0 + pl;
+          const char* recp = stage + pl * prm.rec;
+          const float* q = reinterpret_cast<const float*>(qa + r * rowb);
+          float acc = 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < kD / 4; ++cc) {
+            const float4 mn = *reinterpret_cast<const float4*>(recp + meta_swz(16u * cc, pg));
+            const float4 mx =
+                *reinterpret_cast<const float4*>(recp + meta_swz(16u * (cc + kD / 4), pg));
+            const float mns[4] = {mn.x, mn.y, mn.z, mn.w}, mxs[4] = {mx.x, mx.y, mx.z, mx.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float qi = q[4 * cc + u];
+              acc = __fadd_rn(acc, fmaxf(__fmul_rn(qi, mxs[u]), __fmul_rn(qi, mns[u])));
+            }
+          }
+          scores[r * spc + (pl0 + pl) % spc] = acc;
+        }
       }
-      __syncthreads();
-      // the stage is consumed once its last page is scored: refill it
-      if (tid == 0 && ok && o + prm.ts >= nps && t + prm.stages < nstg) {
-        const int tn = t + prm.stages;
-        const int npn = min(prm.tile, npg - tn * prm.tile);
-        const uint32_t bytes = static_cast<uint32_t>(npn * prm.rec);
-        mbar_expect_tx(&mbar[st], bytes);
-        bulk_g2s(ring + st * kStageBytes,
-                 meta_g + static_cast<size_t>(pr0 + tn * prm.tile) * prm.rec, bytes, &mbar[st]);
+    } else {
+      scal[kSFail] = 1;
+    }
+    const bool chunk_end = ((t + 1) * prm.tile) % spc == 0 || t == nstg - 1;
+    if (DT == LOSA_BF16 && chunk_end && sw) {
+      const int slot = ((sub * 4) + t4) * 2;
+      if (rA < R) {
+        gmx[rA * ng + slot] = gA0;
+        gmx[rA * ng + slot + 1] = gA1;
+        atomicMax(emx + rA, __float_as_uint(eA));
       }
-      if (ok) list_add<DT>(LC, R, k, sU, sT, prm.ts, np, pbase, qa, meta_g);
+      if (rB < R) {
+        gmx[rB * ng + slot] = gB0;
+        gmx[rB * ng + slot + 1] = gB1;
+        atomicMax(emx + rB, __float_as_uint(eB));
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && scal[kSFail] == 0 && t + prm.stages < nstg) issue_stage(t + prm.stages);
+    if (chunk_end) {
+      const int cb = t * prm.tile / spc * spc;  // the chunk's first page
+      const int cn = min(npg, cb + spc) - cb;
+      if (sel && scal[kSFail] == 0) {
+#pragma unroll 1
+        for (int r = warp; r < R; r += kWarps)
+          row_candidates<DT>(scores + r * spc, pnorm + cb,
+                             DT == LOSA_BF16 ? qn[r] : make_float2(0.f, 0.f), cn, pr0 + cb, k,
+                             prm.lcap, prm.lb, w_lk, w_uk, l_lk + static_cast<size_t>(r) * prm.lcap,
+                             l_uk + static_cast<size_t>(r) * prm.lcap, l_n + r, l_thr + r, w_scr,
+                             qa + r * rowb, r, meta_g, DT == LOSA_BF16 ? gmx + r * ng : nullptr,
+                             ng, DT == LOSA_BF16 ? __uint_as_float(emx[r]) : 0.f);
+      }
       __syncthreads();
     }
   }
-
-  // the exact k-th largest lower key of each row's pages becomes its
-  // threshold; the buffer keeps the pages whose upper key reaches it
-  if (sel && scal[kSFail] == 0) {
-#pragma unroll 1
-    for (int r0 = 0; r0 < R; r0 += kThreads / prm.lw)
-      buffer_compact<DT>(LC, r0 + tid / prm.lw, k, r0 + tid / prm.lw < R, qa, meta_g);
-  }
-  __syncthreads();
 
   // ================= cluster barrier 1: every CTA's lists are final ========
   cluster_sync();
@@ -1268,7 +1612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nwords = (d.P + 31) / 32;
   if (sel) {
     if (ok1) {
-      const MergeCtx MC = {l_lk, l_uk, l_n, l_thr, prm.lb, C * prm.lcap, C};
+      const MergeCtx MC = {l_lk, l_uk, l_n, l_thr, prm.lcap, C * prm.lcap, C};
       char* buf = ring + warp * prm.mstride;
 #pragma unroll 1
       for (int i = warp; warp < prm.nmw && c + C * i < R; i += prm.nmw)
@@ -1505,7 +1849,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      float* Ps = reinterpret_cast<float*>(sU) + warp * 16;  // (the score area is free now)
+      float* Ps = fscr + warp * 16;
 #pragma unroll 1
       for (int n = warp; n < ns; n += kWarps) {
         const float4 q = row4<DT>(sq, n, lane);
@@ -1653,7 +1997,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       part_ml[2 * r] = -INFINITY;
       part_ml[2 * r + 1] = 0.f;
     }
-    float* Ps = sU + warp * 16;
+    float* Ps = fscr + warp * 16;
     __syncthreads();
 #pragma unroll 1
     for (int bt = 0; bt < nbat; ++bt) {
@@ -1749,11 +2093,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side: cluster geometry, shared-memory plan, attributes, launch
 // ---------------------------------------------------------------------------
-int pow2_floor(int x) {
-  int p = 1;
-  while (p * 2 <= x) p *= 2;
-  return p;
-}
 int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
 struct Taker {
@@ -1787,10 +2126,14 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   if (R == 0) C = 1;
   prm->C = C;
   prm->cp = align_up((d.P + C - 1) / C, 8);
-  // candidate buffers: lanes per row, entries kept after a compaction
-  prm->lw = std::min(32, std::max(4, pow2_floor(kThreads / std::max(R16, 16))));
+  // candidate lists: entries per row left for the merge, and room for the
+  // survivors of the first bound
   prm->lcap = d.k + kListSlack;
-  const int ts_max = prm->tile;
+  // (the survivor buffer takes a row's list beside a chunk's exact top k)
+  prm->lb = std::max(prm->lcap + 64, prm->lcap + d.k);
+  if (sel && prm->lb > 256) return false;
+  prm->sstride = 2 + 32 * ((d.k + 31) / 32) + prm->lb;
+  const int cp_t = align_up(prm->cp, prm->tile);
   const long long cap_all = static_cast<long long>(C) * prm->lcap;
   // merge warp scratch: keys, staged records, flags, the k-th selection's
   const long long kv32 = 32LL * ((d.k + 31) / 32) + 1 + cap_all;
@@ -1809,17 +2152,15 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   const int MW = (R + 31) / 32;
   prm->early = static_cast<long long>(d.S) * d.Hkv * C <= kEarlyTriggerCtas;
 
-  // the largest plan that fits: most pages per list update, then most union
-  // pages in flight, then most ring stages
-  for (int ts = sel ? ts_max : 8; ts >= 8; ts = (ts / 2 >= 8 ? ts / 2 / 8 * 8 : 0)) {
-  prm->ts = ts;
-  // room for a page tile's survivors beside the entries kept between
-  // prunings: ~3k when it fits, at least the cap after an exact compaction
-  for (int lbx = ts + 3 * d.k + 8; lbx >= ts + prm->lcap; lbx = (lbx > ts + prm->lcap ? std::max(ts + prm->lcap, lbx - d.k - 4) : 0)) {
-  prm->lb = lbx;
-  prm->sstride = prm->lw * ((d.k + prm->lw - 1) / prm->lw) + 1 + prm->lb;
+  // the largest plan that fits, with at least 4 ring stages when any plan
+  // allows it: most pages per score chunk, then most union pages in flight,
+  // then most ring stages
+  for (int pass = 0; pass < 2; ++pass) {
+  const int smin = pass == 0 ? std::min(4, kMaxStages) : kMinStages;
+  for (int spc = cp_t; spc >= prm->tile; spc = (spc / 2 >= prm->tile ? align_up(spc / 2, prm->tile) : 0)) {
+  prm->spc = spc;
   for (int ngp = std::min(kMaxGatherPages, std::max(1, prm->max_lp)); ngp >= 1; ngp /= 2) {
-    for (int stages = kMaxStages; stages >= kMinStages; --stages) {
+    for (int stages = kMaxStages; stages >= smin; --stages) {
       long long ring = 0;
       if (sel) ring = std::max(ring, static_cast<long long>(stages) * kStageBytes);
       if (sel) ring = std::max(ring, static_cast<long long>(prm->mstride));  // one merge warp
@@ -1832,16 +2173,19 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       StepLayout& lo = prm->lo;
       Taker take;
       lo.ring = take(ring, 1024);
-      // the queries, then (after the suffix) the lists and the scores
+      // the queries; once they are staged, the lists, the scores and the
+      // fp32 probability rows in the same bytes
       const long long qarea = 2LL * GB * prm->qstride;
       const long long larea =
-          sel ? (2LL * prm->lb * R + 1LL * (kThreads / prm->lw) * prm->sstride) * 8 : 0;
-      const long long sarea = std::max(sel ? 2LL * R * prm->ts * 4 : 0LL, bf ? 0LL : 512LL);
-      const int qbase = take(std::max(qarea, larea + sarea), 1024);
+          sel ? (2LL * prm->lcap * R + kWarps * (2LL * prm->lb + prm->sstride)) * 8 : 0;
+      const long long carea = sel ? 4LL * R * prm->spc : 0;
+      const long long sarea = bf ? 0LL : kWarps * 16LL * 4;
+      const int qbase = take(std::max(qarea, larea + carea + sarea), 1024);
       lo.qc = qbase;
       lo.qp = qbase + GB * prm->qstride;
       lo.lists = qbase;
-      lo.sc = qbase + static_cast<int>(larea);
+      lo.scores = qbase + static_cast<int>(larea);
+      lo.sc = qbase + static_cast<int>(larea + carea);
       if (bf) {  // after the gather: the warps' partials, then the CTA's
         lo.part_o = lo.ring + static_cast<int>(wpart);
         lo.part_ml = lo.part_o + R16 * kD * 4;
@@ -1864,6 +2208,11 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       lo.lpages = take(4LL * prm->max_lp, 16);
       lo.masks = take(4LL * prm->max_lp * MW, 16);
       lo.misc = take(4LL * kMiscInts, 16);
+      lo.pnorm = take(bf && sel ? 8LL * prm->cp : 0, 128);
+      const int ntm_ = std::max(1, R16 / 16);
+      lo.gmx = take(bf && sel ? 4LL * R16 * 8 * std::max(1, kWarps / ntm_) : 0, 16);
+      lo.emx = take(bf && sel ? 4LL * R16 : 0, 16);
+      lo.qn = take(8LL * R16, 16);
       lo.mbar = take(8LL * (kMaxStages + 2), 16);
       // + 1 KB: the kernel aligns its shared-memory base to 1024 bytes
       lo.total = static_cast<int>(std::min<long long>(take.off + 1024, 1LL << 30));
@@ -1939,6 +2288,9 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   prm.qc = q_cur;
   prm.qp = q_prev;
   prm.meta = static_cast<const char*>(page_meta);
+  prm.norms = reinterpret_cast<const float2*>(static_cast<const char*>(page_meta) +
+                                              meta_norm_offset(d));
+  prm.pn = meta_norm_stride(d);
   prm.K = k_prefix;
   prm.V = v_prefix;
   prm.kb = k_blk;

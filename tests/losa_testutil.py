@@ -35,8 +35,9 @@ def unswizzle_page_meta(sh, page_meta):
     P, d = sh.n_pages, sh.head_dim
     Pc = (sh.capacity + sh.page_size - 1) // sh.page_size  # records per (s, g)
     nchunk = 2 * d * esz // 16
-    raw = page_meta.detach().cpu().view(torch.uint8).reshape(sh.num_seqs * sh.n_kv_heads, Pc,
-                                                             nchunk, 16)[:, :P]
+    nrec = sh.num_seqs * sh.n_kv_heads * Pc
+    raw = page_meta.detach().cpu().view(torch.uint8)[:nrec * nchunk * 16].reshape(
+        sh.num_seqs * sh.n_kv_heads, Pc, nchunk, 16)[:, :P]
     pages = torch.arange(P)
     phys = torch.arange(nchunk)[None, :] ^ (pages[:, None] & 7)
     idx = phys[None, :, :, None].expand(raw.shape[0], P, nchunk, 16)
@@ -162,11 +163,31 @@ def gpu_step(sh, qc, qp, K, V, meta, kb, vb, o_p, l_p, ws=None, q_ref=None):
 # ---------------------------------------------------------------------------
 # comparisons
 # ---------------------------------------------------------------------------
+def page_norms(sh, page_meta):
+    """The metadata's page-norm rows ``[S][Hkv][P][2]`` (||kmin||, ||kmax||):
+    after the records, float2 per page, rows padded to a multiple of 8 pages."""
+    esz = 2 if sh.dtype == api.LOSA_BF16 else 4
+    P, d = sh.n_pages, sh.head_dim
+    Pc = (sh.capacity + sh.page_size - 1) // sh.page_size
+    Pn = (Pc + 7) // 8 * 8
+    nrec = sh.num_seqs * sh.n_kv_heads * Pc
+    raw = page_meta.detach().cpu().view(torch.uint8)[nrec * 2 * d * esz:]
+    nrm = raw[:sh.num_seqs * sh.n_kv_heads * Pn * 8].view(torch.float32)
+    return nrm.reshape(sh.num_seqs, sh.n_kv_heads, Pn, 2)[:, :, :P].numpy()
+
+
 def check_meta(sh, meta, K_host):
     kmin_g, kmax_g = unswizzle_page_meta(sh, meta)
     kmin_o, kmax_o = oracle.build_meta(oshape(sh), K_host)
     assert np.array_equal(kmin_g.float().numpy().view(np.uint32), kmin_o.view(np.uint32))
     assert np.array_equal(kmax_g.float().numpy().view(np.uint32), kmax_o.view(np.uint32))
+    # the page norms bound the exact norms of the (exact) records from above,
+    # and closely: fp32 sums of 128 squares with every rounding upward
+    nrm = page_norms(sh, meta).astype(np.float64)
+    for j, m in enumerate((kmin_o, kmax_o)):
+        exact = np.sqrt(np.sum(np.asarray(m, np.float64) ** 2, axis=-1))
+        assert np.all(nrm[..., j] >= exact)
+        assert np.all(nrm[..., j] <= exact * (1 + 2.0 ** -15) + 1e-30)
     return kmin_o, kmax_o
 
 

@@ -67,9 +67,13 @@ def test_status_strings(L):
 def test_sizes(L):
     sh = S()
     P = 4096
-    assert api.page_meta_size(sh) == 8 * P * 2 * 128 * 2
-    assert api.page_meta_size(S(dtype="f32")) == 8 * P * 2 * 128 * 4
-    assert api.page_meta_size(S(prefix_len=65537)) == 8 * (P + 1) * 2 * 128 * 2
+
+    def norms(Pc):  # the page-norm rows: float2 per page, rows padded to 8 pages
+        return 8 * ((Pc + 7) // 8 * 8) * 8
+
+    assert api.page_meta_size(sh) == 8 * P * 2 * 128 * 2 + norms(P)
+    assert api.page_meta_size(S(dtype="f32")) == 8 * P * 2 * 128 * 4 + norms(P)
+    assert api.page_meta_size(S(prefix_len=65537)) == 8 * (P + 1) * 2 * 128 * 2 + norms(P + 1)
     for which in (api.LOSA_WS_DENSE, api.LOSA_WS_STEP):
         n = api.workspace_size(sh, which)
         assert n > 0 and n % 256 == 0
@@ -205,7 +209,8 @@ def test_prefix_capacity_validation(L, no_device):
     # a capacity below the prefix length is refused; a larger one grows the
     # metadata to ceil(capacity / ps) records per (s, g)
     assert api.workspace_size(S(prefix_capacity=65535), api.LOSA_WS_STEP) == 0
-    assert api.page_meta_size(S(prefix_capacity=65536 + 33)) == 8 * (4096 + 3) * 2 * 128 * 2
+    assert api.page_meta_size(S(prefix_capacity=65536 + 33)) == (8 * (4096 + 3) * 2 * 128 * 2 +
+                                                                 8 * 4104 * 8)
     # appending a block needs room for B more tokens: refused before any launch
     fake = [ctypes.c_void_p((i + 1) << 36) for i in range(5)]  # far apart: no overlaps
     assert L.losa_append_block(ctypes.byref(S(prefix_capacity=65536 + 15)), *fake,

@@ -72,7 +72,16 @@ def _check_meta(c, meta):
                                                 sh.prefix_len, 16, sh.block_size, sh.n_active,
                                                 sh.token_budget, sh.scale), c.lens, c.K)
     Pc = (sh.capacity + 15) // 16
-    raw = meta.view(torch.uint8).reshape(sh.num_seqs * sh.n_kv_heads, Pc, -1).cpu()
+    esz = 2 if sh.dtype == api.LOSA_BF16 else 4
+    nrec = sh.num_seqs * sh.n_kv_heads * Pc
+    raw = meta.view(torch.uint8)[:nrec * 2 * 128 * esz].reshape(
+        sh.num_seqs * sh.n_kv_heads, Pc, -1).cpu()
+    # the page norms: upper bounds of the records' exact norms, close to them;
+    # entries past a sequence's pages never written
+    Pn = (Pc + 7) // 8 * 8
+    nrm_raw = meta.view(torch.uint8)[nrec * 2 * 128 * esz:].cpu()
+    nrm = nrm_raw.view(torch.float32).reshape(sh.num_seqs, sh.n_kv_heads, Pn, 2).numpy()
+    nrm_bytes = nrm_raw.reshape(sh.num_seqs, sh.n_kv_heads, Pn, 8)
     per_seq = []
     for s, (kmin_o, kmax_o) in enumerate(ref):
         P = kmin_o.shape[2]
@@ -82,6 +91,11 @@ def _check_meta(c, meta):
                               kmax_o.view(np.uint32)), s
         rows = raw[s * sh.n_kv_heads:(s + 1) * sh.n_kv_heads, P:]
         assert bool((rows == META_FILL).all()), f"records past sequence {s}'s pages written"
+        for j, m in enumerate((kmin_o, kmax_o)):
+            exact = np.sqrt(np.sum(np.asarray(m[0], np.float64) ** 2, axis=-1))
+            got = nrm[s, :, :P, j].astype(np.float64)
+            assert np.all(got >= exact) and np.all(got <= exact * (1 + 2.0 ** -15) + 1e-30), s
+        assert bool((nrm_bytes[s, :, P:] == META_FILL).all()), f"norms past sequence {s}'s pages"
         per_seq.append((kmin_o, kmax_o))
     return per_seq
 
@@ -174,7 +188,14 @@ def test_varlen_equal_lengths_match_uniform_call():
     res_u = gpu_step(sh_u, c.q[1], c.q[0], c.K, c.V, meta_u, c.kb[1], c.vb[1],
                      cache_u["o_p"].clone(), cache_u["l_p"].clone())
     torch.cuda.synchronize()
-    assert torch.equal(meta, meta_u)
+    # the written bytes agree: every record and every page's norms (the norm
+    # rows' padding is never written)
+    Pc = (700 + 15) // 16
+    nrec_bytes = 3 * 2 * Pc * 2 * 128 * 2
+    assert torch.equal(meta[:nrec_bytes], meta_u[:nrec_bytes])
+    nrm = meta[nrec_bytes:].view(torch.float32).reshape(3, 2, -1, 2)[:, :, :Pc]
+    nrm_u = meta_u[nrec_bytes:].view(torch.float32).reshape(3, 2, -1, 2)[:, :, :Pc]
+    assert torch.equal(nrm, nrm_u)
     for key in ("o_p", "l_p", "out", "lse"):
         assert torch.equal(cache[key], cache_u[key]), key
     for key in ("out", "lse", "o_p", "l_p", "active_idx", "page_idx", "union_count"):
