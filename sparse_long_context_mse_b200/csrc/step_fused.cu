@@ -67,7 +67,6 @@ constexpr int kMaxStages = 6;
 constexpr int kListSlack = 4;       // buffer entries beyond k kept after a compaction before an exact refinement
 constexpr int kMaxGatherPages = 16; // union pages in flight per CTA
 constexpr float kEpsScale = 6.103515625e-05f;  // 2^-14: interval half-width per unit of sum |terms|
-constexpr int kRecSlots = 8;        // records staged at once per merge warp for exact rescoring
 
 typedef unsigned long long u64;
 
@@ -321,15 +320,20 @@ __device__ __forceinline__ void lse_weights(float L1, float L2, float& a, float&
 // chunks swizzled by p & 7 as losa_build_page_meta stores them).
 __device__ __noinline__ float exact_bound_bf16(const char* qrow, int r, const char* rec, int p) {
   const int rs = r & 7, ps = p & 7;
+  // the whole record first (its 32 loads in flight together), then the sum
+  uint4 mn[16], mx[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    mn[c] = *reinterpret_cast<const uint4*>(rec + ((c ^ ps) << 4));
+    mx[c] = *reinterpret_cast<const uint4*>(rec + ((16 + (c ^ ps)) << 4));
+  }
   float acc = 0.f;
-#pragma unroll 4
+#pragma unroll
   for (int c = 0; c < 16; ++c) {  // 16-byte chunks of 8 channels, in channel order
     const uint4 q4 = *reinterpret_cast<const uint4*>(qrow + ((c ^ rs) << 4));
-    const uint4 mn = *reinterpret_cast<const uint4*>(rec + ((c ^ ps) << 4));
-    const uint4 mx = *reinterpret_cast<const uint4*>(rec + ((16 + (c ^ ps)) << 4));
     const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
-    const uint32_t nw[4] = {mn.x, mn.y, mn.z, mn.w};
-    const uint32_t xw[4] = {mx.x, mx.y, mx.z, mx.w};
+    const uint32_t nw[4] = {mn[c].x, mn[c].y, mn[c].z, mn[c].w};
+    const uint32_t xw[4] = {mx[c].x, mx[c].y, mx[c].z, mx[c].w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
 #pragma unroll
@@ -370,176 +374,11 @@ __device__ __forceinline__ void bound_ntile(const uint32_t (&a)[16][4], const ch
 }
 
 // ---------------------------------------------------------------------------
-// Per-row candidate buffers.  Row r's buffer lk/uk [r][0..lb) holds, unsorted,
-// every page of the CTA scored so far whose upper key reached thr[r] when it
-// was scored.  thr[r] is the k-th largest lower key of k scored pages (0 until
-// the row's first compaction), so it never exceeds the k-th largest lower key
-// of all the CTA's pages: every page that can be among the row's top k is in
-// the buffer.  One warp compacts a row.
+// Per-row candidate lists.  After the CTA's pages are scored, row r's list
+// holds its exact top min(k, pages) among the CTA's pages (exact keys), and
+// thr[r] the k-th of them; the cluster merge takes the row's top k from the
+// C lists.  One warp selects a row.
 // ---------------------------------------------------------------------------
-
-// The k-th largest of the distinct keys a[0..n) (0 if n < k), by one warp.  A
-// lower bound first -- the k-th largest of the lanes' sub-maxima (lane j keeps
-// V = ceil(k / 32) of them, so there are at least k) -- then the exact rank
-// among the keys at or above it, which are few.  scr holds 32 V + n keys.
-__device__ __noinline__ u64 warp_kth(const u64* a, int n, int k, u64* scr) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  if (n < k) return 0ull;
-  const int V = (k + 31) >> 5;
-  u64* sv = scr + 32 * V;
-#pragma unroll 1
-  for (int v = 0; v < V; ++v) {
-    u64 m = 0;
-    for (int i = lane + 32 * v; i < n; i += 32 * V) m = a[i] > m ? a[i] : m;
-    scr[lane * V + v] = m;
-  }
-  __syncwarp();
-  u64 t1 = 0;
-#pragma unroll 1
-  for (int v = 0; v < V; ++v) {
-    const u64 x = scr[lane * V + v];
-    int rk = 0;
-    for (int q = 0; q < 32 * V; ++q) {
-      const u64 y = scr[q];
-      rk += (y > x) || (y == x && q < lane * V + v);
-    }
-    if (rk == k - 1) t1 = x;
-  }
-  t1 = warp_max_u64(t1);
-  int ns = 0;
-#pragma unroll 1
-  for (int i0 = 0; i0 < n; i0 += 32) {
-    const int i = i0 + lane;
-    const u64 x = i < n ? a[i] : 0ull;
-    const bool in = i < n && x >= t1;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (in) sv[ns + __popc(bal & lt)] = x;
-    ns += __popc(bal);
-  }
-  __syncwarp();
-  u64 r = 0;
-#pragma unroll 1
-  for (int i = lane; i < ns; i += 32) {
-    const u64 x = sv[i];
-    int rk = 0;
-    for (int q = 0; q < ns; ++q) rk += sv[q] > x;
-    if (rk == k - 1) r = x;
-  }
-  r = warp_max_u64(r);
-  __syncwarp();
-  return r;
-}
-
-// Compaction of one row's buffer by a warp (any n, in shared memory): the
-// exact k-th largest lower key becomes the threshold and only the entries
-// whose upper key reaches it stay.  A row left with more than `cap` entries
-// (near-ties at the boundary) has its inexact entries rescored exactly (the
-// oracle's arithmetic) and is compacted again, which leaves min(k, n) exact
-// entries.
-template <int DT>
-__device__ __noinline__ void row_compact_slow(u64* lk, u64* uk, int* cnt, u64* thr, int k,
-                                              int cap, u64* scr, const char* qrow, int r,
-                                              const char* meta_g) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  int n = *cnt;
-  u64 th_old = *thr;
-#pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-    const u64 th = warp_kth(lk, n, k, scr);
-    int kept = 0;
-#pragma unroll 1
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      u64 a = 0, b = 0;
-      bool keep = false;
-      if (i < n) {
-        a = lk[i];
-        b = uk[i];
-        keep = b >= th;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, keep);
-      __syncwarp();
-      if (keep) {
-        const int pos = kept + __popc(bal & lt);
-        lk[pos] = a;
-        uk[pos] = b;
-      }
-      kept += __popc(bal);
-      __syncwarp();
-    }
-    n = kept;
-    th_old = th > th_old ? th : th_old;
-    if (DT == LOSA_BF16 && n > cap) {
-#pragma unroll 1
-      for (int i = lane; i < n; i += 32)
-        if (lk[i] != uk[i]) {
-          const int p = key_index(lk[i]);
-          const float v = exact_bound_bf16(qrow, r, meta_g + static_cast<size_t>(p) * 512, p);
-          lk[i] = uk[i] = sel_key(v, p);
-        }
-      __syncwarp();
-    } else {
-      break;
-    }
-  }
-  if (lane == 0) {
-    *cnt = n;
-    *thr = th_old;
-  }
-  __syncwarp();
-}
-
-// The k-th largest of the 32-bit values the warp's lanes hold (E per lane,
-// 0 = none), counting repeats: the value x with fewer than k values above it
-// and at least k at or above it (0 when there are fewer than k values).  Each
-// lane orders its values; each round then takes the largest head over the
-// lanes and pops it from every lane holding it (at most k rounds).
-template <int E>
-__device__ __forceinline__ uint32_t warp_kth_u32(uint32_t (&v)[E], int k) {
-#pragma unroll
-  for (int i = 1; i < E; ++i) {
-#pragma unroll
-    for (int j = i; j > 0; --j) {
-      const uint32_t x = max(v[j - 1], v[j]), y = min(v[j - 1], v[j]);
-      v[j - 1] = x;
-      v[j] = y;
-    }
-  }
-  int got = 0;
-#pragma unroll 1
-  for (int it = 0; it < k; ++it) {
-    const uint32_t m = __reduce_max_sync(0xffffffffu, v[0]);
-    if (m == 0u) return 0u;
-    const bool mine = v[0] == m;
-    got += __popc(__ballot_sync(0xffffffffu, mine));
-    if (got >= k) return m;
-    if (mine) {
-#pragma unroll
-      for (int e = 0; e + 1 < E; ++e) v[e] = v[e + 1];
-      v[E - 1] = 0u;
-    }
-  }
-  return 0u;
-}
-
-// The k-th largest of the 64 values v0, v1 of the warp's lanes (0 = none),
-// counting repeats, or 0 when there are fewer than k: every value counts the
-// values above it (independent shuffles), and the answer is the smallest
-// value with fewer than k above it.
-__device__ __forceinline__ uint32_t warp_kth64(uint32_t v0, uint32_t v1, int k) {
-  int g0 = 0, g1 = 0;
-#pragma unroll
-  for (int q = 0; q < 32; ++q) {
-    const uint32_t y0 = __shfl_sync(0xffffffffu, v0, q), y1 = __shfl_sync(0xffffffffu, v1, q);
-    g0 += (y0 > v0) + (y1 > v0);
-    g1 += (y0 > v1) + (y1 > v1);
-  }
-  const uint32_t c0 = g0 < k ? v0 : 0xffffffffu, c1 = g1 < k ? v1 : 0xffffffffu;
-  const uint32_t m = __reduce_min_sync(0xffffffffu, min(c0, c1));
-  return m == 0xffffffffu ? 0u : m;
-}
 
 // A lower bound of the k-th largest of the 64 values v0, v1 of the warp's
 // lanes (0 = none): k rounds each take the largest head over the lanes
@@ -564,73 +403,26 @@ __device__ __forceinline__ float ordered_value(uint32_t x) {
   return __uint_as_float((x & 0x80000000u) ? (x & 0x7fffffffu) : ~x);
 }
 
-// A row's threshold from its buffer (one warp, n <= 32 E entries): th = the
-// k-th largest of the entries' lower-key value words, so that the k-th
-// largest lower key of the CTA's pages is at least th << 32, to which thr
-// rises.  With `compact`, only the entries whose upper-key value word
-// reaches th stay -- every entry whose upper key reaches that k-th largest
-// lower key, and at least k.
-template <int E>
-__device__ __forceinline__ void row_threshold(u64* lk, u64* uk, int& n, u64& thr, int k,
-                                              bool compact) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  uint32_t v[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = lane + 32 * e;
-    v[e] = i < n ? static_cast<uint32_t>(lk[i] >> 32) : 0u;
-  }
-  uint32_t th = 0u;
-  if (n >= k) th = E == 2 ? warp_kth64(v[0], v[E > 1 ? 1 : 0], k) : warp_kth_u32<E>(v, k);
-  const u64 th64 = static_cast<u64>(th) << 32;
-  thr = th64 > thr ? th64 : thr;
-  if (!compact) return;
-  int kept = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int i = lane + 32 * e;
-    u64 a = 0, b = 0;
-    bool keep = false;
-    if (i < n) {
-      b = uk[i];
-      keep = static_cast<uint32_t>(b >> 32) >= th;
-      if (keep) a = lk[i];
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    __syncwarp();
-    if (keep) {
-      const int pos = kept + __popc(bal & lt);
-      lk[pos] = a;
-      uk[pos] = b;
-    }
-    kept += __popc(bal);
-  }
-  __syncwarp();
-  n = kept;
-}
-
 // Candidates of one active row after another chunk of np of the CTA's
-// pages (one warp): su[p] the page's tensor-core score (exact for fp32),
-// its interval half-width e = q2.x ||kmin_p|| + q2.y ||kmax_p|| (bf16; every
-// operation rounded up).  The row's list lk/uk[0..cnt) holds every page of
-// the chunks before whose upper key can reach thr, and thr is at most the
-// k-th largest lower key of those pages; afterwards the same holds with this
-// chunk's pages included (cnt <= cap).
-//   1. tau0: the larger of thr's value word and (a lower bound of) the k-th
-//      largest of group maxima of the lower-key value words -- a lower bound
-//      of the k-th largest lower key.  The groups: gm[0..ng) kept by the scoring
-//      threads over all the pages so far (bf16), else (gm null) 64
-//      sub-maxima of this chunk's pages (lane l, pages l + 32 i, one for
-//      even and one for odd i);
-//   2. the list and the chunk's pages whose upper value word reaches tau0
-//      (few) go to the warp's buffer wl/wu (lb entries); a page is tested
-//      with u + emax first (emax >= every page's half-width);
-//   3. more than cap of them: th, the exact k-th largest lower value word
-//      among them, and only the entries whose upper value word reaches it
-//      stay (row_threshold).
-// More than lb entries in step 2 (many near-equal scores) or more than cap
-// left after step 3 take the exact paths.
+// pages (one warp), in three steps so that a warp can rescore the
+// candidates of two rows together.  su[p] is the page's tensor-core score
+// (exact for fp32), its interval half-width e = q2.x ||kmin_p|| +
+// q2.y ||kmax_p|| (bf16; every operation rounded up).  Before: the row's
+// list lk[0..cnt) holds its exact top min(k, pages) over the chunks before,
+// thr the k-th key.  After: the same over this chunk's pages too.
+//   row_survivors: into the warp's buffer wl/wu go the list and the chunk's
+//     pages whose upper key's value word reaches tau0 -- the larger of
+//     thr's value word and (a lower bound of) the k-th largest of group
+//     maxima of lower-key value words (gm[0..ng), kept by the scoring
+//     threads over all pages so far (bf16), else (gm null) 64 sub-maxima of
+//     this chunk's pages: lane l, pages l + 32 i, one for even and one for
+//     odd i).  A page is tested with u + emax first (emax >= every page's
+//     half-width).  More than lb of them (many near-equal scores): the
+//     exact path for the chunk.  Returns the buffer's entry count;
+//   the caller rescores the inexact entries exactly (the oracle's
+//     arithmetic);
+//   row_topk: the list keeps the exact top min(k, n) by key, thr the k-th.
+// ---------------------------------------------------------------------------
 struct ListCount {
   int n;     // entries
   u64 thr;   // their threshold key
@@ -642,25 +434,18 @@ __device__ __noinline__ ListCount row_candidates_exact(float* su, int np, int pb
                                                        const char* meta_g);
 
 template <int DT>
-__device__ __forceinline__ void row_candidates(float* su, const float2* pn, float2 q2, int np,
-                                               int pbase, int k, int cap, int lb, u64* wl,
-                                               u64* wu, u64* lk, u64* uk, int* cnt, u64* thr,
-                                               u64* scr, const char* qrow, int r,
-                                               const char* meta_g, const uint32_t* gm, int ng,
-                                               float emax) {
+__device__ __forceinline__ int row_survivors(float* su, const float2* pn, float2 q2, int np,
+                                             int pbase, int k, int lb, u64* wl, u64* wu,
+                                             const u64* lk, int n0, u64 thr0, const char* qrow,
+                                             int r, const char* meta_g, const uint32_t* gm,
+                                             int ng, float emax) {
   const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
   auto half_width = [&](int p) {
     if (DT != LOSA_BF16) return 0.f;
     const float2 nk = pn[p];
     return __fadd_ru(__fmul_ru(q2.x, nk.x), __fmul_ru(q2.y, nk.y));
   };
-  const int n0 = *cnt;
-  const u64 thr0 = *thr;
-  for (int i = lane; i < n0; i += 32) {
-    wl[i] = lk[i];
-    wu[i] = uk[i];
-  }
+  for (int i = lane; i < n0; i += 32) wl[i] = wu[i] = lk[i];
   uint32_t gmax[2] = {0u, 0u};
   if (gm) {
     gmax[0] = lane < ng ? gm[lane] : 0u;
@@ -678,9 +463,9 @@ __device__ __forceinline__ void row_candidates(float* su, const float2* pn, floa
   }
   const uint32_t t0 = max(warp_kth64_lb(gmax[0], gmax[1], k), static_cast<uint32_t>(thr0 >> 32));
   const float t0f = t0 ? ordered_value(t0) : -INFINITY;
-  // step 2, 16 pages per lane at a time (pages p00 + 32 i + lane): a mask
-  // of the pages whose u + emax reaches tau0, the exact test of those (few),
-  // then the survivors' places by a prefix sum over the lanes
+  // 16 pages per lane at a time (pages p00 + 32 i + lane): a mask of the
+  // pages whose u + emax reaches tau0, the exact test of those (few), then
+  // the survivors' places by a prefix sum over the lanes
   int ns = n0;
 #pragma unroll 1
   for (int p00 = 0; p00 < np; p00 += 32 * 16) {
@@ -714,46 +499,33 @@ __device__ __forceinline__ void row_candidates(float* su, const float2* pn, floa
     ns += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
-  int n;
-  u64 th = thr0;
   if (ns > lb || ns > 256) {
     // this chunk's exact top k beside the list (n0 + k <= lb by the plan)
-    n = n0 + row_candidates_exact<DT>(su, np, pbase, k, wl + n0, wu + n0, qrow, r, meta_g).n;
-  } else {
-    n = ns;
-    th = static_cast<u64>(t0) << 32 > thr0 ? static_cast<u64>(t0) << 32 : thr0;
+    return n0 + row_candidates_exact<DT>(su, np, pbase, k, wl + n0, wu + n0, qrow, r, meta_g).n;
   }
-  // more than cap: the exact k-th largest lower value word becomes the
-  // threshold (step 3)
-  if (n > cap) {
-    if (n <= 64)
-      row_threshold<2>(wl, wu, n, th, k, true);
-    else if (n <= 128)
-      row_threshold<4>(wl, wu, n, th, k, true);
-    else
-      row_threshold<8>(wl, wu, n, th, k, true);
-  }
-  if (n > cap) {
-    int* cs = reinterpret_cast<int*>(scr);  // (the slow path's own scratch follows)
-    u64* ts = scr + 1;
-    if (lane == 0) {
-      *cs = n;
-      *ts = th;
-    }
-    __syncwarp();
-    row_compact_slow<DT>(wl, wu, cs, ts, k, cap, scr + 2, qrow, r, meta_g);
-    n = *cs;
-    th = *ts;
-    __syncwarp();
-  }
-  // the row's list (at most cap entries)
+  return ns;
+}
+
+// The exact top min(k, n) of the (exact, distinct) keys wl[0..n): an
+// entry's rank is the number of entries above it; the list takes ranks < k
+// in rank order, thr the larger of thr0 and the k-th key (if there are k).
+__device__ __forceinline__ void row_topk(const u64* wl, int n, int k, u64* lk, int* cnt, u64* thr,
+                                         u64 thr0) {
+  const int lane = threadIdx.x & 31;
+  u64 kth = 0;
+#pragma unroll 1
   for (int i = lane; i < n; i += 32) {
-    lk[i] = wl[i];
-    uk[i] = wu[i];
+    const u64 x = wl[i];
+    int rk = 0;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) rk += wl[j] > x;
+    if (rk < k) lk[rk] = x;
+    if (rk == k - 1) kth = x;
   }
+  kth = warp_max_u64(kth);
   if (lane == 0) {
-    *cnt = n;
-    *thr = th;
+    *cnt = min(n, k);
+    *thr = kth > thr0 ? kth : thr0;
   }
   __syncwarp();
 }
@@ -809,222 +581,25 @@ __device__ __noinline__ ListCount row_candidates_exact(float* su, int np, int pb
 }
 
 // ---------------------------------------------------------------------------
-// Merge of one active row's lists from the C CTAs of the cluster (one warp):
-// the row's k pages, exactly the oracle's top k (value descending, lower page
-// first), written ascending to sel[0..k) (then -1 when the sequence has fewer
-// pages).  `buf` is the warp's scratch for the rare paths: lk[cap_all],
-// uk[cap_all], kRecSlots staged records of 512 bytes, flag[cap_all], then the
-// k-th selection's scratch (32 * ceil(k / 32) + cap_all keys).
+// Merge of one active row's lists from the C CTAs of the cluster (one warp).
+// Every CTA's list holds its exact top min(k, its pages) by exact key, and
+// thr its k-th key; the row's top k over all pages is among them, at or
+// above the largest thr.  The row's k pages (value descending, lower page
+// first) go to sel[0..k) in ascending page order (then -1 when the sequence
+// has fewer pages).  `buf` holds the gathered keys (C * lcap of them).
 // ---------------------------------------------------------------------------
 struct MergeCtx {
-  const u64* lk;   // this CTA's list arrays (the same offsets in every CTA)
-  const u64* uk;
+  const u64* lk;   // this CTA's list keys [R][lcap] (the same offsets in every CTA)
   const int* n;
   const u64* thr;
-  int lb;          // entries per row buffer
-  int cap_all;     // C * cap: entries the warp's buffer holds
+  int lcap;        // entries per row list
   int C;
 };
 
-struct CtaOffsets {
-  int v[8];  // first entry of each CTA's list in the concatenation (unused CTAs: INT_MAX)
-};
-
-// More candidates than k (near-ties at the boundary; blk/buk[0..nca) hold
-// them).  lkth: a key that no page outside the candidates reaches with its
-// upper key (the candidates' lower bound and the merge's tau0, whichever is
-// larger).  A candidate whose lower key reaches lkth and that at most k - 1
-// other candidates can beat (their upper key above its lower key) is in; the
-// others are rescored exactly (the oracle's arithmetic) and the best of them
-// by exact key fill the rest.  (The true top k are all candidates, so this
-// is exactly the top k.)  Writes sel[0..k).
-template <int DT>
-__device__ __noinline__ void merge_resolve(u64* blk, u64* buk, int* flag, char* recs, int nca,
-                                           int k, u64 lkth, int32_t* sel, const char* qrow, int r,
-                                           const char* meta_g) {
+__device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, u64* blk,
+                                          int32_t* sel) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  int ncert = 0;
-#pragma unroll 1
-  for (int e0 = 0; e0 < nca; e0 += 32) {
-    const int e = e0 + lane;
-    bool cert = false;
-    if (e < nca && blk[e] >= lkth) {
-      int beat = 0;
-      for (int e2 = 0; e2 < nca; ++e2) beat += (e2 != e) && (buk[e2] > blk[e]);
-      cert = beat <= k - 1;
-    }
-    if (e < nca) flag[e] = cert ? 1 : 0;
-    const unsigned bal = __ballot_sync(0xffffffffu, cert);
-    if (cert) sel[ncert + __popc(bal & lt)] = key_index(blk[e]);
-    ncert += __popc(bal);
-  }
-  __syncwarp();
-  if (DT == LOSA_BF16) {  // fp32 scores are exact already
-#pragma unroll 1
-    for (int e0 = 0; e0 < nca; e0 += kRecSlots) {
-#pragma unroll 1
-      for (int q = 0; q < kRecSlots && e0 + q < nca; ++q) {
-        const int e = e0 + q;
-        if (!flag[e] && blk[e] != buk[e]) {
-          const int p = key_index(blk[e]);
-          reinterpret_cast<uint4*>(recs + q * 512)[lane] =
-              reinterpret_cast<const uint4*>(meta_g + static_cast<size_t>(p) * 512)[lane];
-        }
-      }
-      __syncwarp();
-      if (lane < kRecSlots && e0 + lane < nca) {
-        const int e = e0 + lane;
-        if (!flag[e] && blk[e] != buk[e]) {
-          const int p = key_index(blk[e]);
-          const float v = exact_bound_bf16(qrow, r, recs + lane * 512, p);
-          blk[e] = buk[e] = sel_key(v, p);
-        }
-      }
-      __syncwarp();
-    }
-  }
-  const int need = k - ncert;
-#pragma unroll 1
-  for (int e = lane; e < nca; e += 32) {
-    if (flag[e]) continue;
-    int rk = 0;
-    for (int e2 = 0; e2 < nca; ++e2) rk += !flag[e2] && blk[e2] > blk[e];
-    if (rk < need) sel[ncert + rk] = key_index(blk[e]);
-  }
-  __syncwarp();
-}
-
-// The row's entries whose upper key reaches tau0, gathered from the C CTAs
-// into registers (E per lane; lane l takes entries l, l + 32, ... of the
-// CTAs' lists in CTA order), a lower bound lkth of their k-th largest lower
-// key, and its candidates (upper key >= lkth: a superset of the true top k):
-// sel when there are at most k of them, else blk/buk for merge_resolve.
-// Returns the number of candidates.
-template <int E>
-__device__ __forceinline__ int merge_gather(const MergeCtx& M, int r, int k, u64 tau0, int total,
-                                            const CtaOffsets& offs, int32_t* sel, u64* blk,
-                                            u64* buk, u64& lkth) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  u64 a[E], b[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int f = lane + 32 * e;
-    a[e] = b[e] = 0ull;
-    if (f < total) {
-      int cf = 0;
-#pragma unroll
-      for (int q = 1; q < 8; ++q) cf += f >= offs.v[q];
-      const size_t i = static_cast<size_t>(r) * M.lb + (f - offs.v[cf]);
-      const u64 y = ld_dsmem_u64(dsmem(M.uk + i, cf));
-      const u64 x = ld_dsmem_u64(dsmem(M.lk + i, cf));
-      if (y >= tau0) {
-        a[e] = x;
-        b[e] = y;
-      }
-    }
-  }
-  // lkth: the k-th largest lower-key value word, as a key (at most the k-th
-  // largest lower key: the candidates below are a superset of the exact ones)
-  uint32_t v[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) v[e] = static_cast<uint32_t>(a[e] >> 32);
-  lkth = static_cast<u64>(warp_kth_u32<E>(v, k)) << 32;
-  int nca = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) nca += __popc(__ballot_sync(0xffffffffu, b[e] != 0ull && b[e] >= lkth));
-  int pos = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const bool c = b[e] != 0ull && b[e] >= lkth;
-    const unsigned bal = __ballot_sync(0xffffffffu, c);
-    if (c) {
-      const int at = pos + __popc(bal & lt);
-      if (nca <= k) {
-        sel[at] = key_index(a[e]);
-      } else {
-        blk[at] = a[e];
-        buk[at] = b[e];
-      }
-    }
-    pos += __popc(bal);
-  }
-  __syncwarp();
-  return nca;
-}
-
-// The same for a row with more than 256 entries reaching tau0 (large k):
-// gathered into shared memory.
-
-__device__ __noinline__ int merge_gather_smem(const MergeCtx M, int r, int k, u64 tau0,
-                                              int total, const CtaOffsets offs, int32_t* sel,
-                                              u64* blk, u64* buk, u64* kscr, u64* lkth_out) {
-  const int lane = threadIdx.x & 31;
-  const unsigned lt = (1u << lane) - 1u;
-  int cnt = 0;
-#pragma unroll 1
-  for (int f0 = 0; f0 < total; f0 += 32) {
-    const int f = f0 + lane;
-    u64 a = 0, b = 0;
-    bool in = false;
-    if (f < total) {
-      int cf = 0;
-      for (int q = 1; q < 8; ++q) cf += f >= offs.v[q];
-      const size_t i = static_cast<size_t>(r) * M.lb + (f - offs.v[cf]);
-      b = ld_dsmem_u64(dsmem(M.uk + i, cf));
-      a = ld_dsmem_u64(dsmem(M.lk + i, cf));
-      in = b >= tau0;
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (in) {
-      const int pos = cnt + __popc(bal & lt);
-      blk[pos] = a;
-      buk[pos] = b;
-    }
-    cnt += __popc(bal);
-  }
-  __syncwarp();
-  const u64 lkth = warp_kth(blk, cnt, k, kscr);
-  int nca = 0;
-#pragma unroll 1
-  for (int e0 = 0; e0 < cnt; e0 += 32) {
-    const int e = e0 + lane;
-    u64 a = 0, b = 0;
-    bool c = false;
-    if (e < cnt) {
-      a = blk[e];
-      b = buk[e];
-      c = b >= lkth;
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, c);
-    __syncwarp();
-    if (c) {
-      const int pos = nca + __popc(bal & lt);
-      blk[pos] = a;
-      buk[pos] = b;
-    }
-    nca += __popc(bal);
-    __syncwarp();
-  }
-  if (nca <= k)
-    for (int e = lane; e < nca; e += 32) sel[e] = key_index(blk[e]);
-  __syncwarp();
-  *lkth_out = lkth;
-  return nca;
-}
-
-template <int DT>
-__device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, char* buf,
-                                          int32_t* sel, const char* qa, const char* meta_g) {
-  const int lane = threadIdx.x & 31;
-  u64* blk = reinterpret_cast<u64*>(buf);
-  u64* buk = blk + M.cap_all;
-  char* recs = reinterpret_cast<char*>(buk + M.cap_all);
-  int* flag = reinterpret_cast<int*>(recs + kRecSlots * 512);
-  u64* kscr = reinterpret_cast<u64*>(flag + ((M.cap_all + 1) & ~1));
-  // the largest of the CTAs' thresholds bounds the group's k-th largest
-  // lower key from below: only entries whose upper key reaches it matter
   int nc = 0;
   u64 th = 0;
   if (lane < M.C) {
@@ -1032,6 +607,8 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, char*
     th = ld_dsmem_u64(dsmem(M.thr + r, lane));
   }
   const u64 tau0 = warp_max_u64(th);
+  // the CTAs' entries at or above tau0 (lane l takes entries l, l + 32, ...
+  // of the lists in CTA order)
   int incl = nc;
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) {
@@ -1039,24 +616,40 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, char*
     if (lane >= o) incl += y;
   }
   const int total = __shfl_sync(0xffffffffu, incl, 7);
-  CtaOffsets offs;
+  int offs[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const int v = __shfl_sync(0xffffffffu, incl - nc, q);
-    offs.v[q] = q < M.C ? v : 0x7fffffff;
+    offs[q] = q < M.C ? v : 0x7fffffff;
   }
-  u64 lkth = 0;
-  int nca;
-  if (total <= 128)
-    nca = merge_gather<4>(M, r, k, tau0, total, offs, sel, blk, buk, lkth);
-  else if (total <= 256)
-    nca = merge_gather<8>(M, r, k, tau0, total, offs, sel, blk, buk, lkth);
-  else
-    nca = merge_gather_smem(M, r, k, tau0, total, offs, sel, blk, buk, kscr, &lkth);
-  if (nca > k)
-    merge_resolve<DT>(blk, buk, flag, recs, nca, k, lkth > tau0 ? lkth : tau0, sel, qa + r * 256,
-                      r, meta_g);
-  const int nsel = min(nca, k);
+  int cnt = 0;
+#pragma unroll 1
+  for (int f0 = 0; f0 < total; f0 += 32) {
+    const int f = f0 + lane;
+    u64 x = 0;
+    if (f < total) {
+      int cf = 0;
+#pragma unroll
+      for (int q = 1; q < 8; ++q) cf += f >= offs[q];
+      x = ld_dsmem_u64(dsmem(M.lk + static_cast<size_t>(r) * M.lcap + (f - offs[cf]), cf));
+    }
+    const bool in = f < total && x >= tau0;
+    const unsigned bal = __ballot_sync(0xffffffffu, in);
+    if (in) blk[cnt + __popc(bal & lt)] = x;
+    cnt += __popc(bal);
+  }
+  __syncwarp();
+  // the top min(k, cnt) by rank (distinct keys)
+#pragma unroll 1
+  for (int i = lane; i < cnt; i += 32) {
+    const u64 x = blk[i];
+    int rk = 0;
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) rk += blk[j] > x;
+    if (rk < k) sel[rk] = key_index(x);
+  }
+  __syncwarp();
+  const int nsel = min(cnt, k);
   // ascending page order, then -1 past the selection
   int pv[4];
   int pr[4];
@@ -1085,7 +678,7 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, char*
 struct StepLayout {
   int ring;     // metadata ring; afterwards merge scratch, gathered pages, warp partials
   int qc, qp;   // the group's queries (current, previous) [GB][rowb]
-  int lists;    // candidate lists lk, uk [R][lcap]; per warp survivors [2][lb] and scratch [sstride]
+  int lists;    // candidate lists [R][lcap] (exact keys); per warp survivor keys [2][2][lb]
   int sc;       // fp32: the warps' probability rows (16 floats each)
   int part_o;   // the CTA's partial outputs [R16][kD] floats (bf16: in the ring)
   int part_ml;  // the CTA's partial (m, l) [R16][2] (bf16: in the ring)
@@ -1134,7 +727,6 @@ struct StepParams {
   int rec;         // bytes per metadata record
   int spc;         // pages per score chunk (a multiple of the stage's pages)
   int lb, lcap;    // survivor buffer entries per warp; list entries per row (k + slack)
-  int sstride;     // scratch keys per warp for the exact paths
   int qstride;     // bytes per staged query row (padded: no bank conflicts between rows)
   int nmw;         // merge warps
   int mstride;     // bytes of a merge warp's scratch (in the ring area)
@@ -1199,14 +791,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // pages are consumed, fp32 in its own area (its running state lives there)
   float* part_o = reinterpret_cast<float*>(smem + lo.part_o);
   float* part_ml = reinterpret_cast<float*>(smem + lo.part_ml);
-  // the rows' candidate lists [R][lcap], then per warp its survivor buffer
-  // [lb] (lower and upper keys) and the exact paths' scratch [sstride]
+  // the rows' candidate lists [R][lcap] (exact keys), then per warp its
+  // survivor buffers for two rows: lower keys [2][lb], upper keys [2][lb]
   u64* l_lk = reinterpret_cast<u64*>(smem + lo.lists);
-  u64* l_uk = l_lk + static_cast<size_t>(R) * prm.lcap;
-  u64* w_lk = l_uk + static_cast<size_t>(R) * prm.lcap + static_cast<size_t>(warp) * 2 * prm.lb;
-  u64* w_uk = w_lk + prm.lb;
-  u64* w_scr = l_uk + static_cast<size_t>(R) * prm.lcap + static_cast<size_t>(kWarps) * 2 * prm.lb +
-               static_cast<size_t>(warp) * prm.sstride;
+  u64* w_lk = l_lk + static_cast<size_t>(R) * prm.lcap + static_cast<size_t>(warp) * 4 * prm.lb;
+  u64* w_uk = w_lk + 2 * prm.lb;
   const int qst = prm.qstride;
   float* fscr = reinterpret_cast<float*>(smem + lo.sc);
   int* l_n = reinterpret_cast<int*>(smem + lo.l_n);
@@ -1230,12 +819,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* emx = reinterpret_cast<uint32_t*>(smem + lo.emx);
   float2* qn = reinterpret_cast<float2*>(smem + lo.qn);
   uint64_t* gbar = mbar + kMaxStages;  // [2]: the gather's two page buffers
+  uint64_t* ebar = gbar + 2;            // [kMaxStages]: ring slot released by every warp
 
   // the next kernel of the stream may be scheduled now when this grid fits
   // one wave (it waits for this grid's completion before it reads anything);
   // otherwise at exit, so that its CTAs never take SMs this grid's later
   // clusters need
   if (prm.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (DT == LOSA_BF16 && tid == 0 && d.R > 0) {  // (the page gather's maps; no data read)
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+  }
   // nothing is read before the work queued ahead of the step has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
@@ -1261,14 +855,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (nbytes) bulk_g2s(pnorm, norm_g + pr0, nbytes, &mbar[st]);
   };
 
-  if (tid == 0) {
-    for (int i = 0; i < kMaxStages + 2; ++i) mbar_init(&mbar[i], 1);
-    fence_mbar_init();
-    scal[kSFail] = 0;
-    if (c == 0 && g == 0 && seq_len_bad(d, s)) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-#pragma unroll 1
-    for (int t = 0; t < min(nstg, prm.stages); ++t) issue_stage(t);
-  }
   // the group's current and previous queries (cp.async group 0), rows
   // padded to qst bytes
   {
@@ -1282,6 +868,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (h ? qpg : qcg) + static_cast<size_t>(row) * rowb + cc * 16, 16u);
     }
     cp_async_commit();
+  }
+  // the metadata ring (after the queries: they are needed first)
+  if (tid == 0) {
+    for (int i = 0; i < kMaxStages + 2; ++i) mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxStages; ++i) mbar_init(&ebar[i], kWarps);
+    fence_mbar_init();
+    scal[kSFail] = 0;
+    if (c == 0 && g == 0 && seq_len_bad(d, s)) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+#pragma unroll 1
+    for (int t = 0; t < min(nstg, prm.stages); ++t) issue_stage(t);
   }
   // the block's K and V (rows >= B zero), chunks swizzled for ldmatrix
   // (cp.async group 1)
@@ -1486,10 +1082,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();  // the query area becomes the buffer area
 
   // ---- bound scores of this CTA's pages, stage by stage, stored per row
-  // for a chunk of spc pages (scores[r][p - chunk start]); a stage's slot is
-  // refilled once every warp has read it, and after a chunk's last stage
-  // each active row's candidates take in the chunk's pages (one warp per
-  // row)
+  // for a chunk of spc pages (scores[r][p - chunk start]).  Each warp goes
+  // through the stages at its own pace: it waits for a stage's bytes, scores
+  // its tiles and releases the slot; thread 0 refills a slot once all warps
+  // have released it.  After a chunk's last stage (a barrier) each active
+  // row's candidates take in the chunk's pages (one warp per row).
   const int rA = mt * 16 + g4, rB = rA + 8;
   const int spc = prm.spc;
   // bf16: each scoring thread keeps, for its two rows, the maxima of the
@@ -1508,6 +1105,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const char* stage = ring + st * kStageBytes;
     const int nps = min(prm.tile, npg - t * prm.tile);
     const int pl0 = t * prm.tile;  // the stage's first page (CTA-local)
+    // the producer (thread 0) refills the slot of the stage before this one
+    // once every warp has released it
+    if (tid == 0 && t >= 1 && t - 1 + prm.stages < nstg && scal[kSFail] == 0) {
+      if (mbar_wait(&ebar[(t - 1) % prm.stages], ((t - 1) / prm.stages) & 1))
+        issue_stage(t - 1 + prm.stages);
+      else
+        scal[kSFail] = 1;
+    }
     // each thread waits for the stage itself (the wait makes the bytes the
     // copy wrote visible to it)
     if (scal[kSFail] == 0 && mbar_wait(&mbar[st], parity)) {
@@ -1570,6 +1175,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       scal[kSFail] = 1;
     }
+    // the warp has read the stage: release its slot
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ebar[st]);
     const bool chunk_end = ((t + 1) * prm.tile) % spc == 0 || t == nstg - 1;
     if (DT == LOSA_BF16 && chunk_end && sw) {
       const int slot = ((sub * 4) + t4) * 2;
@@ -1584,20 +1192,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         atomicMax(emx + rB, __float_as_uint(eB));
       }
     }
-    __syncthreads();
-    if (tid == 0 && scal[kSFail] == 0 && t + prm.stages < nstg) issue_stage(t + prm.stages);
     if (chunk_end) {
+      __syncthreads();  // every warp's scores and maxima of the chunk are in
       const int cb = t * prm.tile / spc * spc;  // the chunk's first page
       const int cn = min(npg, cb + spc) - cb;
       if (sel && scal[kSFail] == 0) {
+        // rows r0 and r0 + 8 per warp: their survivors, rescored together,
+        // then each row's exact top k
 #pragma unroll 1
-        for (int r = warp; r < R; r += kWarps)
-          row_candidates<DT>(scores + r * spc, pnorm + cb,
-                             DT == LOSA_BF16 ? qn[r] : make_float2(0.f, 0.f), cn, pr0 + cb, k,
-                             prm.lcap, prm.lb, w_lk, w_uk, l_lk + static_cast<size_t>(r) * prm.lcap,
-                             l_uk + static_cast<size_t>(r) * prm.lcap, l_n + r, l_thr + r, w_scr,
-                             qa + r * rowb, r, meta_g, DT == LOSA_BF16 ? gmx + r * ng : nullptr,
-                             ng, DT == LOSA_BF16 ? __uint_as_float(emx[r]) : 0.f);
+        for (int r0 = warp; r0 < R; r0 += 2 * kWarps) {
+          const int r1 = r0 + kWarps;
+          auto survivors = [&](int r, int h) {
+            return row_survivors<DT>(
+                scores + r * spc, pnorm + cb, DT == LOSA_BF16 ? qn[r] : make_float2(0.f, 0.f), cn,
+                pr0 + cb, k, prm.lb, w_lk + h * prm.lb, w_uk + h * prm.lb,
+                l_lk + static_cast<size_t>(r) * prm.lcap, l_n[r], l_thr[r], qa + r * rowb, r,
+                meta_g, DT == LOSA_BF16 ? gmx + r * ng : nullptr, ng,
+                DT == LOSA_BF16 ? __uint_as_float(emx[r]) : 0.f);
+          };
+          const int nA = survivors(r0, 0);
+          const int nB = r1 < R ? survivors(r1, 1) : 0;
+          if (DT == LOSA_BF16) {
+#pragma unroll 1
+            for (int i = lane; i < nA + nB; i += 32) {
+              const bool b = i >= nA;
+              const int j = b ? prm.lb + i - nA : i;
+              if (w_lk[j] != w_uk[j]) {
+                const int p = key_index(w_lk[j]), r = b ? r1 : r0;
+                const float v = exact_bound_bf16(qa + r * rowb, r, meta_g + static_cast<size_t>(p) * 512, p);
+                w_lk[j] = sel_key(v, p);
+              }
+            }
+            __syncwarp();
+          }
+          row_topk(w_lk, nA, k, l_lk + static_cast<size_t>(r0) * prm.lcap, l_n + r0, l_thr + r0,
+                   l_thr[r0]);
+          if (r1 < R)
+            row_topk(w_lk + prm.lb, nB, k, l_lk + static_cast<size_t>(r1) * prm.lcap, l_n + r1,
+                     l_thr + r1, l_thr[r1]);
+        }
       }
       __syncthreads();
     }
@@ -1612,11 +1245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nwords = (d.P + 31) / 32;
   if (sel) {
     if (ok1) {
-      const MergeCtx MC = {l_lk, l_uk, l_n, l_thr, prm.lcap, C * prm.lcap, C};
-      char* buf = ring + warp * prm.mstride;
+      const MergeCtx MC = {l_lk, l_n, l_thr, prm.lcap, C};
+      u64* buf = reinterpret_cast<u64*>(ring + warp * prm.mstride);
 #pragma unroll 1
       for (int i = warp; warp < prm.nmw && c + C * i < R; i += prm.nmw)
-        merge_row<DT>(MC, c + C * i, k, buf, sel_all + (c + C * i) * k, qa, meta_g);
+        merge_row(MC, c + C * i, k, buf, sel_all + (c + C * i) * k);
     }
     __syncthreads();
     if (prm.page_idx) {
@@ -1763,13 +1396,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // two page buffers of ngp pages: batch b lands in buffer b & 1 while the
   // previous batch is folded in
   const int nbat = (nlp + prm.ngp - 1) / prm.ngp;
+  // (warp 0 issues a batch: lane i the pages i, i + 32, ...)
   auto issue = [&](int bt) {
     const int b0 = bt * prm.ngp, nb = min(prm.ngp, nlp - b0);
     char* bufp = ring + (bt & 1) * prm.ngp * 2 * pbytes;
     if (DT == LOSA_BF16) {
-      mbar_expect_tx(&gbar[bt & 1], static_cast<uint32_t>(nb * 2 * pbytes));
+      if (lane == 0) mbar_expect_tx(&gbar[bt & 1], static_cast<uint32_t>(nb * 2 * pbytes));
+      __syncwarp();
 #pragma unroll 1
-      for (int i = 0; i < nb; ++i) {
+      for (int i = lane; i < nb; i += 32) {
         const int p = lpages[b0 + i];
         const int row = sg * d.Lc + p * kPS;
         char* dk = bufp + 2 * i * pbytes;
@@ -1778,7 +1413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(dk + pbytes, &vmap, 0, row, &gbar[bt & 1]);
         tma_load_2d(dk + pbytes + 2048, &vmap, 64, row, &gbar[bt & 1]);
       }
-    } else {
+    } else if (lane == 0) {
       uint32_t bytes = 0;
       for (int i = 0; i < nb; ++i) bytes += 2u * min(kPS, Ls - lpages[b0 + i] * kPS) * rowb;
       mbar_expect_tx(&gbar[bt & 1], bytes);
@@ -1794,7 +1429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
-  if (tid == 0 && ok2) {
+  if (warp == 0 && ok2) {
     if (nbat > 0) issue(0);
     if (nbat > 1) issue(1);
   }
@@ -1920,7 +1555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();  // the buffer is free: the batch after next may land in it
-      if (tid == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
+      if (warp == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
     }
     tile_finish(t);
     if (R > 0 && wpg == 1) {
@@ -2031,7 +1666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
-      if (tid == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
+      if (warp == 0 && ok2 && scal[kSFail] == 0 && bt + 2 < nbat) issue(bt + 2);
     }
   }
 
@@ -2132,15 +1767,10 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   // (the survivor buffer takes a row's list beside a chunk's exact top k)
   prm->lb = std::max(prm->lcap + 64, prm->lcap + d.k);
   if (sel && prm->lb > 256) return false;
-  prm->sstride = 2 + 32 * ((d.k + 31) / 32) + prm->lb;
   const int cp_t = align_up(prm->cp, prm->tile);
   const long long cap_all = static_cast<long long>(C) * prm->lcap;
-  // merge warp scratch: keys, staged records, flags, the k-th selection's
-  const long long kv32 = 32LL * ((d.k + 31) / 32) + 1 + cap_all;
-  prm->mstride = align_up(static_cast<int>(std::min<long long>(
-                              2 * cap_all * 8 + kRecSlots * 512 + ((cap_all + 1) & ~1LL) * 4 +
-                                  kv32 * 8, 1 << 30)),
-                          16);
+  // merge warp scratch: the gathered keys
+  prm->mstride = align_up(static_cast<int>(std::min<long long>(cap_all * 8, 1 << 30)), 16);
   prm->qstride = rowb + 16;  // rows 16 bytes apart in bank order
   // union pages per CTA
   const int Umax = d.all_pages ? d.P : std::min(d.P, R * d.k);
@@ -2176,8 +1806,7 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       // the queries; once they are staged, the lists, the scores and the
       // fp32 probability rows in the same bytes
       const long long qarea = 2LL * GB * prm->qstride;
-      const long long larea =
-          sel ? (2LL * prm->lcap * R + kWarps * (2LL * prm->lb + prm->sstride)) * 8 : 0;
+      const long long larea = sel ? (1LL * prm->lcap * R + kWarps * 4LL * prm->lb) * 8 : 0;
       const long long carea = sel ? 4LL * R * prm->spc : 0;
       const long long sarea = bf ? 0LL : kWarps * 16LL * 4;
       const int qbase = take(std::max(qarea, larea + carea + sarea), 1024);
@@ -2213,7 +1842,7 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
       lo.gmx = take(bf && sel ? 4LL * R16 * 8 * std::max(1, kWarps / ntm_) : 0, 16);
       lo.emx = take(bf && sel ? 4LL * R16 : 0, 16);
       lo.qn = take(8LL * R16, 16);
-      lo.mbar = take(8LL * (kMaxStages + 2), 16);
+      lo.mbar = take(8LL * (2 * kMaxStages + 2), 16);
       // + 1 KB: the kernel aligns its shared-memory base to 1024 bytes
       lo.total = static_cast<int>(std::min<long long>(take.off + 1024, 1LL << 30));
       if (take.off + 1024 > max_dyn) continue;
