@@ -48,15 +48,26 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+TRACE_LIB = os.path.join(PKG, "liblosa_trace.so")
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False,
+          trace: bool = False) -> str:
+    """The library; with ``trace`` a separate copy, ``liblosa_trace.so``,
+    whose step kernel records per-phase timestamps (``phase_trace.py``)."""
+    lib = TRACE_LIB if trace else LIB
+    if not force and os.path.exists(lib) and all(
+            os.path.getmtime(p) <= os.path.getmtime(lib) for p in _deps()):
+        return lib
+    objdir = os.path.join(OBJDIR, "trace") if trace else OBJDIR
+    os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_v else []
+    if trace:
+        extra.append("-DLOSA_PHASE_TRACE")
 
     def compile_one(src):
-        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [cc, *NVCC_FLAGS, *ARCH, *extra, "-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
@@ -67,11 +78,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> 
 
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(compile_one, _sources()))
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     subprocess.check_call([cc, *ARCH, "-shared", "-o", tmp, *objs])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True, ptxas_v="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose=True, ptxas_v="-v" in sys.argv,
+                trace="--trace" in sys.argv))

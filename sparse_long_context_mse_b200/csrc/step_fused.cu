@@ -57,6 +57,31 @@
 
 namespace losa {
 
+// Phase timestamps of the step kernel, compiled in only for the tracing
+// build of the library (-DLOSA_PHASE_TRACE; phase_trace.py reads them):
+// thread 0 of each of the first kPhaseCtas CTAs stamps the %globaltimer at
+// each phase boundary.  The product build has none of this.
+constexpr int kPhases = 24;
+constexpr int kPhaseCtas = 512;
+#ifdef LOSA_PHASE_TRACE
+__device__ unsigned long long g_phase[kPhaseCtas * kPhases];
+#define LOSA_PHASE(i)                                                                   \
+  do {                                                                                  \
+    if (threadIdx.x == 0) {                                                             \
+      const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                        \
+      if (cta_ < static_cast<unsigned>(kPhaseCtas)) {                                   \
+        unsigned long long t_;                                                          \
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                          \
+        g_phase[cta_ * kPhases + (i)] = t_;                                             \
+      }                                                                                 \
+    }                                                                                   \
+  } while (0)
+#else
+#define LOSA_PHASE(i) \
+  do {                \
+  } while (0)
+#endif
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -832,6 +857,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // nothing is read before the work queued ahead of the step has completed
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  LOSA_PHASE(0);
 
   const int Ls = seq_len(d, s);                 // this sequence's prefix length
   const int Ps = (Ls + kPS - 1) / kPS;
@@ -897,6 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   cp_async_wait<1>();  // the queries
   __syncthreads();
   const bool qok = true;
+  LOSA_PHASE(1);
 
   // ---- locality: one thread per token row, the oracle's arithmetic exactly
   // (channels in order, fp32, one rounding per operation)
@@ -929,6 +956,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
+  LOSA_PHASE(2);
   // ---- active set: one warp per head, lane = token; rank by (mse desc,
   // token asc); an active row is r = h * A + (its rank among the head's
   // active tokens in token order)
@@ -1044,6 +1072,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
+  LOSA_PHASE(3);
   // ---- the bound's A operand stays in registers for the whole scan (one
   // m16 tile of active rows per warp)
   const int ntm = R16 / 16;
@@ -1080,6 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (DT == LOSA_BF16 && sel) emx[r] = 0u;
   }
   __syncthreads();  // the query area becomes the buffer area
+  LOSA_PHASE(4);
 
   // ---- bound scores of this CTA's pages, stage by stage, stored per row
   // for a chunk of spc pages (scores[r][p - chunk start]).  Each warp goes
@@ -1116,6 +1146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // each thread waits for the stage itself (the wait makes the bytes the
     // copy wrote visible to it)
     if (scal[kSFail] == 0 && mbar_wait(&mbar[st], parity)) {
+      if (t == 0) LOSA_PHASE(5);
+      if (t == nstg - 1) LOSA_PHASE(6);
       if (DT == LOSA_BF16) {
         const int nnt = (nps + 7) / 8;
 #pragma unroll 1
@@ -1196,6 +1228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();  // every warp's scores and maxima of the chunk are in
       const int cb = t * prm.tile / spc * spc;  // the chunk's first page
       const int cn = min(npg, cb + spc) - cb;
+      if (t == nstg - 1) LOSA_PHASE(7);
       if (sel && scal[kSFail] == 0) {
         // rows r0 and r0 + 8 per warp: their survivors, rescored together,
         // then each row's exact top k
@@ -1236,9 +1269,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  LOSA_PHASE(8);
   // ================= cluster barrier 1: every CTA's lists are final ========
   cluster_sync();
   const bool ok1 = scal[kSFail] == 0;
+  LOSA_PHASE(9);
 
   // ---- each row's k pages from the lists of all CTAs of the cluster: CTA c
   // merges rows r = c (mod C), one warp per row
@@ -1263,6 +1298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  LOSA_PHASE(10);
   // ================= cluster barrier 1b: every row's selection is final =====
   cluster_sync();
 
@@ -1388,6 +1424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
+  LOSA_PHASE(11);
   // ---- gather: the union pages of this CTA (TMA, no multicast), each
   // folded into the active rows whose mask has it
   const int nlp = R > 0 ? scal[kSNlp] : 0;
@@ -1433,6 +1470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (nbat > 0) issue(0);
     if (nbat > 1) issue(1);
   }
+  LOSA_PHASE(12);
 
   // ---- while the pages land: the block's K/V and the cached state are in
   // (cp.async groups 1 and 2)
@@ -1516,6 +1554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
+  LOSA_PHASE(13);
   if (DT == LOSA_BF16) {
     const int wpg = ntm > 0 ? kWarps / ntm : 1;
     const int mtg = warp / wpg, subg = warp % wpg;
@@ -1527,6 +1566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b0 = bt * prm.ngp, nb = min(prm.ngp, nlp - b0);
       char* bufp = ring + (bt & 1) * prm.ngp * 2 * pbytes;
       if (ok2 && scal[kSFail] == 0 && !mbar_wait(&gbar[bt & 1], (bt >> 1) & 1)) scal[kSFail] = 1;
+      if (bt == 0) LOSA_PHASE(14);
       // V rows past the sequence's end of its partial last page may hold
       // anything (P is 0 there, but 0 times NaN is NaN): zero them
       if (Ls % kPS) {
@@ -1670,9 +1710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  LOSA_PHASE(15);
   // ================= cluster barrier 2: every CTA's partials are final =====
   cluster_sync();
 
+  LOSA_PHASE(16);
   // ---- combine: CTA c finishes its active rows r = c + C*j
   if (scal[kSFail] == 0) {
 #pragma unroll 1
@@ -1719,10 +1761,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  LOSA_PHASE(17);
   // ================= cluster barrier 3: no CTA leaves while another may
   // still read its shared memory
   cluster_sync();
   if (tid == 0 && scal[kSFail]) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
+  LOSA_PHASE(18);
 }
 
 // ---------------------------------------------------------------------------
@@ -1963,3 +2007,18 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
 }
 
 }  // namespace losa
+
+#ifdef LOSA_PHASE_TRACE
+// (tracing build only) copy out / clear the phase timestamps
+extern "C" int losa_phase_read(unsigned long long* host, int n) {
+  if (!host || n < 0 || n > losa::kPhaseCtas * losa::kPhases) return LOSA_ERR_INVALID_ARG;
+  return cudaMemcpyFromSymbol(host, losa::g_phase, sizeof(unsigned long long) * n) == cudaSuccess
+             ? LOSA_OK
+             : LOSA_ERR_CUDA;
+}
+extern "C" int losa_phase_clear(void) {
+  static unsigned long long zero[losa::kPhaseCtas * losa::kPhases] = {};
+  return cudaMemcpyToSymbol(losa::g_phase, zero, sizeof(zero)) == cudaSuccess ? LOSA_OK
+                                                                            : LOSA_ERR_CUDA;
+}
+#endif

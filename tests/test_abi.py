@@ -284,3 +284,9 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_product_library_has_no_phase_trace(L):
+    # the per-phase timestamps exist only in the separate tracing build
+    assert not hasattr(L, "losa_phase_read")
+    assert not hasattr(L, "losa_phase_clear")
