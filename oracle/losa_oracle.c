@@ -340,8 +340,7 @@ void oracle_dense_rows(const oracle_shape* sh, const float* Q, const float* K, c
 
 /* ------------------------------------------------------------------------
  * One LoSA step with the active set and page lists given (shared tail of
- * oracle_step; also used directly when a near-tie makes two selections
- * equally correct).
+ * oracle_step; also used directly by tests that fix the selection).
  *   active_idx [S][Hq][A] ascending, page_idx [S][Hq][A][k] ascending.
  * Updates o_p, l_p of active rows in place (stable rows untouched), then
  * writes out/out_lse for all rows, and union_count [S][Hkv] (may be NULL).
