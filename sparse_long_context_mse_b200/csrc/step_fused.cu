@@ -1299,22 +1299,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   LOSA_PHASE(10);
-  // ================= cluster barrier 1b: every row's selection is final =====
-  cluster_sync();
+  // Which pages this CTA attends.  By default (own): the pages of the rows
+  // it merged -- every active row is finished by one CTA, with no union
+  // round and no cross-CTA combine; a page two of its rows share is read
+  // once, a page rows of two CTAs share is read by both.  With the
+  // whole-union variant, or when every page is selected: the CTA's share of
+  // the group's union (slots u = c mod C), and the CTAs' partials are
+  // combined through distributed shared memory.
+  const bool own = sel && !d.attend_union;
+  if (!own) {
+    // ================= cluster barrier 1b: every row's selection is final ====
+    cluster_sync();
+  }
 
-  // ---- every CTA takes the other rows' selections from their CTAs and
-  // builds the group's union bitmap
+  // ---- the page bitmap: this CTA's rows' selections (own), or every row's,
+  // read from their CTAs
   if (sel) {
 #pragma unroll 1
     for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
+    if (!own) {
 #pragma unroll 1
-    for (int e = tid; e < R * k; e += kThreads) {
-      const int r = e / k;
-      if (r % C != c) sel_all[e] = ld_dsmem_s32(dsmem(sel_all + e, r % C));
+      for (int e = tid; e < R * k; e += kThreads) {
+        const int r = e / k;
+        if (r % C != c) sel_all[e] = ld_dsmem_s32(dsmem(sel_all + e, r % C));
+      }
     }
     __syncthreads();
 #pragma unroll 1
     for (int e = tid; e < R * k; e += kThreads) {
+      if (own && (e / k) % C != c) continue;
       const int p = sel_all[e];
       if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
       else if (p >= 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
@@ -1335,7 +1348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int e = tid; e < prm.max_lp * MW; e += kThreads) masks[e] = 0u;
   __syncthreads();
 
-  // ---- the group's union and this CTA's share (union slots u = c mod C)
+  // ---- the slots: own, every page of the bitmap (u = slot); else the
+  // group's union and this CTA's share (union slots u = c mod C)
+  const int Cs = own ? 1 : C, cs = own ? 0 : c;
   if (R == 0 && c == 0 && tid == 0 && prm.union_count) prm.union_count[sg] = 0;
   if (R > 0) {
     if (!sel) {
@@ -1381,23 +1396,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         wbase[w] = run;
         run += __popc(bitmap[w]);
       }
-      const int nlp = U > c ? (U - c + C - 1) / C : 0;
+      const int nlp = U > cs ? (U - cs + Cs - 1) / Cs : 0;
       if (tid == 0) {
         scal[kSNlp] = min(nlp, prm.max_lp);
         if (nlp > prm.max_lp) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
-        if (c == 0 && prm.union_count) prm.union_count[sg] = U;
+        if (!own && c == 0 && prm.union_count) prm.union_count[sg] = U;
       }
       __syncthreads();
 #pragma unroll 1
       for (int e = tid; e < R * k; e += kThreads) {
+        const int r = e / k;
+        if (own && r % C != c) continue;
         const int p = sel_all[e];
         if (p < 0 || p >= d.P) continue;
         const int w = p >> 5;
         const int u = wbase[w] + __popc(bitmap[w] & ((1u << (p & 31)) - 1u));
-        if (u % C != c || u / C >= prm.max_lp) continue;
-        const int r = e / k;
-        lpages[u / C] = p;
-        atomicOr(&masks[(u / C) * MW + (r >> 5)], 1u << (r & 31));
+        if (u % Cs != cs || u / Cs >= prm.max_lp) continue;
+        lpages[u / Cs] = p;
+        atomicOr(&masks[(u / Cs) * MW + (r >> 5)], 1u << (r & 31));
       }
       __syncthreads();
       if (d.attend_union) {
@@ -1712,7 +1728,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   LOSA_PHASE(15);
   // ================= cluster barrier 2: every CTA's partials are final =====
-  cluster_sync();
+  // (own pages: each CTA's partial of its rows is the whole prefix result)
+  if (!own) cluster_sync();
+  __syncthreads();
 
   LOSA_PHASE(16);
   // ---- combine: CTA c finishes its active rows r = c + C*j
@@ -1721,12 +1739,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = warp; j < n_oa; j += kWarps) {
       const int r = c + C * j;
       float2 mlj = make_float2(-INFINITY, 0.f);
-      if (lane < C) mlj = ld_dsmem_f2(dsmem(part_ml + 2 * r, lane));
+      if (own) {
+        if (lane == 0) mlj = *reinterpret_cast<const float2*>(part_ml + 2 * r);
+      } else if (lane < C) {
+        mlj = ld_dsmem_f2(dsmem(part_ml + 2 * r, lane));
+      }
       const uint32_t nz = __ballot_sync(0xffffffffu, mlj.x != -INFINITY);
       float4 ac[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if ((nz >> q) & 1u) ac[q] = ld_dsmem_f4(dsmem(part_o + r * kD + 4 * lane, q));
+        if ((nz >> q) & 1u)
+          ac[q] = own ? *reinterpret_cast<const float4*>(part_o + r * kD + 4 * lane)
+                      : ld_dsmem_f4(dsmem(part_o + r * kD + 4 * lane, q));
       float M = mlj.x;
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -1758,6 +1782,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           make_float4(wa * op.x + wb * os.x, wa * op.y + wb * os.y, wa * op.z + wb * os.z,
                       wa * op.w + wb * os.w);
       if (prm.out_lse && lane == 0) prm.out_lse[grow] = L;
+    }
+  }
+
+  // own pages: the group's union size, if asked for, from every row's
+  // selection once all merges are done
+  if (own && prm.union_count) {
+    cluster_sync();
+    if (c == 0) {
+#pragma unroll 1
+      for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
+      __syncthreads();
+#pragma unroll 1
+      for (int e = tid; e < R * k; e += kThreads) {
+        const int r = e / k;
+        const int p = r % C == c ? sel_all[e] : ld_dsmem_s32(dsmem(sel_all + e, r % C));
+        if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
+      }
+      __syncthreads();
+      int cnt = 0;
+#pragma unroll 1
+      for (int w = tid; w < nwords; w += kThreads) cnt += __popc(bitmap[w]);
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (lane == 0) scal[kSWsum + warp] = cnt;
+      __syncthreads();
+      if (tid == 0) {
+        int U = 0;
+        for (int w = 0; w < kWarps; ++w) U += scal[kSWsum + w];
+        prm.union_count[sg] = U;
+      }
     }
   }
 
@@ -1819,6 +1872,9 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   // union pages per CTA
   const int Umax = d.all_pages ? d.P : std::min(d.P, R * d.k);
   prm->max_lp = R > 0 ? (Umax + C - 1) / C : 0;
+  // (own pages: the pages of the CTA's ceil(R / C) rows)
+  if (R > 0 && !d.all_pages)
+    prm->max_lp = std::max(prm->max_lp, std::min(d.P, (R + C - 1) / C * d.k));
   const int n_oa = (R + C - 1) / C;
   const int n_os = (GB - R + C - 1) / C;
   const int ns = n_oa + n_os;
