@@ -1315,22 +1315,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- the page bitmap: this CTA's rows' selections (own), or every row's,
   // read from their CTAs
   if (sel) {
-#pragma unroll 1
-    for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
     if (!own) {
+#pragma unroll 1
+      for (int w = tid; w < nwords; w += kThreads) bitmap[w] = 0u;
 #pragma unroll 1
       for (int e = tid; e < R * k; e += kThreads) {
         const int r = e / k;
         if (r % C != c) sel_all[e] = ld_dsmem_s32(dsmem(sel_all + e, r % C));
       }
-    }
-    __syncthreads();
+      __syncthreads();
 #pragma unroll 1
-    for (int e = tid; e < R * k; e += kThreads) {
-      if (own && (e / k) % C != c) continue;
-      const int p = sel_all[e];
-      if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
-      else if (p >= 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+      for (int e = tid; e < R * k; e += kThreads) {
+        const int p = sel_all[e];
+        if (p >= 0 && p < d.P) atomicOr(&bitmap[p >> 5], 1u << (p & 31));
+        else if (p >= 0) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+      }
     }
   } else if (R > 0 && prm.page_idx) {
     // every page of the sequence, then -1
@@ -1366,6 +1365,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = tid; e < min(nlp, prm.max_lp) * MW; e += kThreads) {
         const int nb = min(32, R - 32 * (e % MW));
         masks[e] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+      }
+    } else if (own) {
+      // the CTA's rows' pages, once each (warp 0): entry e is position
+      // e % k of its j = e / k -th row (r = c + C j); an entry takes the slot
+      // of its page if an earlier chunk made one, else the lowest lane with
+      // the same page makes a new slot; every entry sets its row's bit in
+      // its slot's mask
+      if (warp == 0) {
+        const int ne = n_oa * k;
+        int nu = 0;
+#pragma unroll 1
+        for (int e0 = 0; e0 < ne; e0 += 32) {
+          const int e = e0 + lane;
+          const int r = c + C * (e / k);
+          int p = e < ne ? sel_all[r * k + e % k] : -1;
+          if (p >= d.P) {
+            atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+            p = -1;
+          }
+          int slot = -1;
+          if (p >= 0)
+            for (int u = 0; u < nu && slot < 0; ++u) slot = lpages[u] == p ? u : -1;
+          const bool fresh = p >= 0 && slot < 0;
+          const unsigned same = __match_any_sync(0xffffffffu, fresh ? p : -1);
+          const int leader = __ffs(same) - 1;
+          const bool lead = fresh && leader == lane;
+          const unsigned bal = __ballot_sync(0xffffffffu, lead);
+          const int mine = nu + __popc(bal & lt);
+          const int from_leader = __shfl_sync(0xffffffffu, mine, leader);
+          if (fresh) slot = from_leader;
+          if (lead && slot < prm.max_lp) lpages[slot] = p;
+          if (p >= 0 && slot < prm.max_lp) atomicOr(&masks[slot * MW + (r >> 5)], 1u << (r & 31));
+          nu += __popc(bal);
+          __syncwarp();
+        }
+        if (lane == 0) {
+          scal[kSNlp] = min(nu, prm.max_lp);
+          if (nu > prm.max_lp) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_BOUNDS);
+        }
       }
     } else {
       // exclusive prefix of the words' popcounts: a run of words per thread,
