@@ -58,11 +58,25 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for phase `parity` of `bar`; false if it gave up.
+// The same, but a thread whose phase is not complete sleeps until it
+// completes or `ns` nanoseconds pass (it takes no issue slots meanwhile).
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(su32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase `parity` of `bar`; false if it gave up.  The
+// waiting thread sleeps between tests, so that it does not take issue slots
+// from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try(bar, parity))
+  while (!mbar_try_sleep(bar, parity, 20000u))
     if (clock64() - t0 > kWaitCycles) return false;
   return true;
 }
@@ -126,6 +140,22 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 // before it are visible to the cluster's reads after it.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// prmt.b32 in its default mode: byte n of the result is byte (c >> 4n) & 7
+// of {b, a} (a = bytes 0..3), or, when bit 3 of that nibble is set, that
+// byte's sign bit replicated over all 8 bits.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+// The two halves of cluster_sync, for a barrier whose arrival can be made
+// early (every thread of the CTA arrives once, then waits once).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Address, in the cluster's shared window, of `local` (a shared-memory

@@ -6,13 +6,16 @@
 // prefix attention, dense intra-block suffix, online-softmax merge, cache
 // update.
 //
-// One thread-block cluster of C <= 8 CTAs per (sequence, KV head) group; the
-// CTAs of a cluster exchange what they found through distributed shared
-// memory and meet at three cluster barriers.  Per CTA:
+// One thread-block cluster of C CTAs per (sequence, KV head) group: up to 16
+// (the non-portable cluster size) when every CTA attends the pages of its
+// own rows, up to 8 when the whole union is attended and the CTAs' partials
+// are combined across the cluster.  The CTAs exchange what they found
+// through distributed shared memory at cluster barriers.  Per CTA:
 //
-//  1. TMA bulk copies of the group's current and previous queries and of the
-//     metadata records of the CTA's contiguous range of prefix pages (a ring
-//     of 32 KB stages); the block's own K/V by cp.async.
+//  1. The group's current and previous queries (cp.async), then a ring of
+//     32 KB TMA bulk stages over the metadata records of the CTA's
+//     contiguous range of prefix pages (with the pages' rounded-up norms),
+//     the block's own K/V by cp.async.
 //  2. Locality: one thread per token row sums (Qc - Qp)^2 over the channels
 //     in channel order, one fp32 rounding per operation -- the oracle's
 //     arithmetic exactly, so the active set (top-|A| per head, ties to the
@@ -20,30 +23,28 @@
 //  3. Dense suffix of the CTA's share of the block's token rows on tensor
 //     cores (stable rows are merged with their untouched cache and written).
 //  4. QUEST bound of every page of the range for the R = G*|A| active rows on
-//     tensor cores: U' = [q- | q+] . [kmin ; kmax] (bf16 products are exact,
-//     the sum is the tensor core's), and T' = |[q- | q+]| . |[kmin ; kmax]|,
-//     the sum of the terms' magnitudes.  The channel-order fp32 sum U of the
-//     oracle lies within 2^-14 T of U', which gives every page an interval
-//     [lb, ub] and two keys LK <= true key <= UK (value, then lower page
-//     first).  Per row the CTA keeps every page whose UK reaches the k-th
-//     largest LK seen so far (a list that grows by stages, rank-sorted,
-//     pruned; if it ever holds more than k + 8 pages, its inexact entries are
-//     rescored exactly).  fp32 inputs are scored exactly on CUDA cores.
-//  5. Cluster barrier.  Every CTA merges every row's lists from all CTAs of
-//     the cluster (distributed shared memory): the k-th largest LK over all
-//     pages gives the candidates (UK at or above it); if they are more than
-//     k, the inexact ones are rescored in channel order exactly as the oracle
-//     does and the top k by exact key win.  The selection is therefore the
-//     oracle's, exactly, by construction.  Then the group's union (ascending
-//     page order, a row mask per page); union slot u belongs to CTA u % C.
-//  6. The CTA's union pages arrive by 2-D tiled TMA (no multicast, 128-byte
-//     swizzle), each page's K and V once for the whole GQA group, and are
-//     folded into one online-softmax partial per active row on tensor cores
-//     (P split into bf16 high and remainder parts).
-//  7. Cluster barrier.  CTA c combines the active rows r = c (mod C): the
-//     partials of every CTA (distributed shared memory) and the row's suffix
-//     give the new o_p / L_p and the output.  A last cluster barrier keeps
-//     every CTA's shared memory alive until the others have read it.
+//     tensor cores, U' = [q- | q+] . [kmin ; kmax] (bf16 products exact, the
+//     sum the tensor core's).  The channel-order fp32 sum U of the oracle
+//     lies within e = |q-| |kmin| + |q+| |kmax| (times 2^-14, every factor
+//     rounded up) of U'.  Per row and score chunk: a lower bound of the k-th
+//     largest U from group maxima, the pages whose U' + e reaches it, those
+//     rescored in the oracle's channel-order arithmetic, and the exact top k
+//     by key (value, then lower page first).  fp32 inputs are scored
+//     exactly on CUDA cores.
+//  5. Cluster barrier.  CTA c merges the rows r = c (mod C) from every CTA's
+//     exact list (distributed shared memory): the row's top k over all pages
+//     is among the keys at or above the largest k-th key of the lists.  The
+//     selection is the oracle's, exactly, by construction.
+//  6. Own pages (the default): CTA c gathers the pages of its rows, once
+//     each, by 2-D tiled TMA (no multicast, 128-byte swizzle) and folds them
+//     into one online-softmax partial per row on tensor cores (P split into
+//     bf16 high and remainder parts); with the row's suffix that gives the
+//     new o_p / L_p and the output, with no further exchange.  Whole union
+//     (an option): the group's union in ascending page order, slot u on CTA
+//     u % C, then a cluster barrier and CTA c combines rows r = c (mod C)
+//     from every CTA's partial.
+//  7. A last cluster barrier keeps every CTA's shared memory alive until the
+//     others have read it.
 //
 // Every wait on a TMA copy is bounded (clock64); a wait that gives up sets
 // LOSA_ERR_DEVICE_TIMEOUT in the status word, and the CTA skips the work
@@ -61,7 +62,7 @@ namespace losa {
 // build of the library (-DLOSA_PHASE_TRACE; phase_trace.py reads them):
 // thread 0 of each of the first kPhaseCtas CTAs stamps the %globaltimer at
 // each phase boundary.  The product build has none of this.
-constexpr int kPhases = 24;
+constexpr int kPhases = 48;
 constexpr int kPhaseCtas = 512;
 #ifdef LOSA_PHASE_TRACE
 __device__ unsigned long long g_phase[kPhaseCtas * kPhases];
@@ -76,9 +77,24 @@ __device__ unsigned long long g_phase[kPhaseCtas * kPhases];
       }                                                                                 \
     }                                                                                   \
   } while (0)
+// (the same from another thread: `th` instead of thread 0)
+#define LOSA_PHASE_BY(i, th)                                                            \
+  do {                                                                                  \
+    if (threadIdx.x == (th)) {                                                          \
+      const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                        \
+      if (cta_ < static_cast<unsigned>(kPhaseCtas)) {                                   \
+        unsigned long long t_;                                                          \
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                          \
+        g_phase[cta_ * kPhases + (i)] = t_;                                             \
+      }                                                                                 \
+    }                                                                                   \
+  } while (0)
 #else
 #define LOSA_PHASE(i) \
   do {                \
+  } while (0)
+#define LOSA_PHASE_BY(i, th) \
+  do {                       \
   } while (0)
 #endif
 
@@ -86,6 +102,11 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// CTAs per cluster at most: 8 (the portable size) when the CTAs' partials
+// are combined across the cluster, 16 (the non-portable size) when every CTA
+// attends the pages of its own rows and nothing is combined across CTAs
+constexpr int kMaxCombineCtas = 8;
+constexpr int kMaxClusterCtas = 16;
 constexpr int kStageBytes = 32 * 1024;
 constexpr int kMinStages = 2;
 constexpr int kMaxStages = 6;
@@ -340,6 +361,13 @@ __device__ __forceinline__ void lse_weights(float L1, float L2, float& a, float&
 // The oracle's bound of page p for one active row, bit for bit: channels in
 // order 0..d-1, fp32, one rounding per operation,
 //   acc = acc + max(q_i * kmax_i, q_i * kmin_i).
+// kmin_i <= kmax_i and rounding is monotone, so for finite values the max is
+// q_i * kmax_i when q_i >= 0 and q_i * kmin_i otherwise (a zero product of
+// either sign leaves acc unchanged: acc starts at +0 and a sum in
+// round-to-nearest is never -0 unless both addends are).  Per 32-bit word of
+// two channels, a byte permute that replicates each channel's q sign bit
+// gives a 16-bit mask per channel, and one logic op picks kmin under it and
+// kmax elsewhere.
 // qrow: the row's q (bf16, 16-byte chunks swizzled by r & 7, as staged for
 // the tensor cores); rec: page p's metadata record (global or shared memory;
 // chunks swizzled by p & 7 as losa_build_page_meta stores them).
@@ -361,13 +389,13 @@ __device__ __noinline__ float exact_bound_bf16(const char* qrow, int r, const ch
     const uint32_t xw[4] = {mx[c].x, mx[c].y, mx[c].z, mx[c].w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {  // low half = the lower channel
-        const float q = h ? __uint_as_float(qw[u] & 0xffff0000u) : __uint_as_float(qw[u] << 16);
-        const float kn = h ? __uint_as_float(nw[u] & 0xffff0000u) : __uint_as_float(nw[u] << 16);
-        const float kx = h ? __uint_as_float(xw[u] & 0xffff0000u) : __uint_as_float(xw[u] << 16);
-        acc = __fadd_rn(acc, fmaxf(__fmul_rn(q, kx), __fmul_rn(q, kn)));
-      }
+      // bytes 0-1: the sign of byte 1 (channel 2u's q), bytes 2-3: of byte 3
+      const uint32_t neg = prmt(qw[u], 0u, 0xbb99u);
+      const uint32_t kw = (nw[u] & neg) | (xw[u] & ~neg);
+      // low half = the lower channel
+      acc = __fadd_rn(acc, __fmul_rn(__uint_as_float(qw[u] << 16), __uint_as_float(kw << 16)));
+      acc = __fadd_rn(acc, __fmul_rn(__uint_as_float(qw[u] & 0xffff0000u),
+                                     __uint_as_float(kw & 0xffff0000u)));
     }
   }
   return acc;
@@ -462,8 +490,8 @@ template <int DT>
 __device__ __forceinline__ int row_survivors(float* su, const float2* pn, float2 q2, int np,
                                              int pbase, int k, int lb, u64* wl, u64* wu,
                                              const u64* lk, int n0, u64 thr0, const char* qrow,
-                                             int r, const char* meta_g, const uint32_t* gm,
-                                             int ng, float emax) {
+                                             int r, const char* meta_g, const uint32_t* gm, int ng,
+                                             float emax) {
   const int lane = threadIdx.x & 31;
   auto half_width = [&](int p) {
     if (DT != LOSA_BF16) return 0.f;
@@ -606,6 +634,149 @@ __device__ __noinline__ ListCount row_candidates_exact(float* su, int np, int pb
 }
 
 // ---------------------------------------------------------------------------
+// bf16: the same for a warp's two rows at once (A and B; B absent when
+// !hasB), each step of the two rows interleaved so that their latencies
+// overlap.  Per row: tau0 = the larger of thr's value word and a lower bound
+// of the k-th largest lower-key value word (k rounds over the 64 group
+// maxima of the scan); the survivors are the chunk's pages with
+// u + emax >= tau0 (rounded up: emax bounds every page's half-width, so no
+// page of the row's true top k is dropped); they are rescored exactly (the
+// oracle's arithmetic), and with the list they give the exact top k by key.
+// More than lb survivors: that row takes the exact path for the chunk.
+// ---------------------------------------------------------------------------
+struct PairRow {
+  const float* su;       // the chunk's tensor-core scores of the row
+  u64* w;                // the warp's buffer for the row [lb]
+  u64* lk;               // the row's list [lcap]
+  int* n;                // its entry count
+  u64* thr;              // its threshold key
+  const uint32_t* gm;    // group maxima of lower-key value words [ng]
+  float emax;            // the largest half-width of the row's pages so far
+  const char* qrow;      // the row's staged q
+  int r;                 // the active row
+};
+
+__device__ __forceinline__ void select_pair_bf16(const PairRow& A, const PairRow& B, bool hasB,
+                                                 int np, int pbase, int k, int lb, int ng,
+                                                 const char* meta_g) {
+  const int lane = threadIdx.x & 31;
+  const int n0A = *A.n, n0B = hasB ? *B.n : 0;
+  const u64 thr0A = *A.thr, thr0B = hasB ? *B.thr : 0ull;
+  for (int i = lane; i < n0A; i += 32) A.w[i] = A.lk[i];
+  for (int i = lane; i < n0B; i += 32) B.w[i] = B.lk[i];
+  // tau0 of both rows: k rounds, each popping every lane's head equal to
+  // the round's maximum (repeats pop together, which only lowers the bound)
+  uint32_t tA, tB;
+  {
+    const uint32_t a0 = lane < ng ? A.gm[lane] : 0u, a1 = lane + 32 < ng ? A.gm[lane + 32] : 0u;
+    const uint32_t b0 = hasB && lane < ng ? B.gm[lane] : 0u;
+    const uint32_t b1 = hasB && lane + 32 < ng ? B.gm[lane + 32] : 0u;
+    uint32_t ha0 = max(a0, a1), ha1 = min(a0, a1), hb0 = max(b0, b1), hb1 = min(b0, b1);
+    uint32_t ma = 0u, mb = 0u;
+#pragma unroll 2
+    for (int i = 0; i < k; ++i) {
+      ma = __reduce_max_sync(0xffffffffu, ha0);
+      mb = __reduce_max_sync(0xffffffffu, hb0);
+      const bool pa = ha0 == ma, pb = hb0 == mb;
+      ha0 = pa ? ha1 : ha0;
+      ha1 = pa ? 0u : ha1;
+      hb0 = pb ? hb1 : hb0;
+      hb1 = pb ? 0u : hb1;
+    }
+    tA = max(ma, static_cast<uint32_t>(thr0A >> 32));
+    tB = max(mb, static_cast<uint32_t>(thr0B >> 32));
+  }
+  const float tAf = tA ? ordered_value(tA) : -INFINITY;
+  const float tBf = tB ? ordered_value(tB) : -INFINITY;
+  // survivors: 16 pages per lane and row at a time (pages p00 + 32 i +
+  // lane), all loads first, then the places by a prefix sum over the lanes
+  int nA = n0A, nB = n0B;
+#pragma unroll 1
+  for (int p00 = 0; p00 < np; p00 += 32 * 16) {
+    float va[16], vb[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int p = min(p00 + 32 * i + lane, np - 1);
+      va[i] = A.su[p];
+      vb[i] = B.su[p];  // (B's pointers are A's when B is absent)
+    }
+    uint32_t ma = 0u, mb = 0u;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const bool in = p00 + 32 * i + lane < np;
+      if (in && __fadd_ru(va[i], A.emax) >= tAf) ma |= 1u << i;
+      if (in && hasB && __fadd_ru(vb[i], B.emax) >= tBf) mb |= 1u << i;
+    }
+    const int ca = __popc(ma), cb = __popc(mb);
+    int ia = ca, ib = cb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int ya = __shfl_up_sync(0xffffffffu, ia, o);
+      const int yb = __shfl_up_sync(0xffffffffu, ib, o);
+      if (lane >= o) {
+        ia += ya;
+        ib += yb;
+      }
+    }
+    int pa = nA + ia - ca, pb = nB + ib - cb;
+    for (uint32_t m = ma; m; m &= m - 1, ++pa)
+      if (pa < lb) A.w[pa] = sel_key(0.f, pbase + p00 + 32 * (__ffs(m) - 1) + lane);
+    for (uint32_t m = mb; m; m &= m - 1, ++pb)
+      if (pb < lb) B.w[pb] = sel_key(0.f, pbase + p00 + 32 * (__ffs(m) - 1) + lane);
+    nA += __shfl_sync(0xffffffffu, ia, 31);
+    nB += __shfl_sync(0xffffffffu, ib, 31);
+  }
+  __syncwarp();
+  LOSA_PHASE(19);
+  // too many survivors (many near-equal scores): the row's exact path
+  // (its list and this chunk's exact top k, n0 + k <= lb by the plan)
+  int fA = n0A, fB = n0B;  // first entry to rescore
+  if (nA > lb) {
+    nA = n0A + row_candidates_exact<LOSA_BF16>(const_cast<float*>(A.su), np, pbase, k, A.w + n0A,
+                                               A.w + n0A, A.qrow, A.r, meta_g).n;
+    fA = nA;
+  }
+  if (nB > lb) {
+    nB = n0B + row_candidates_exact<LOSA_BF16>(const_cast<float*>(B.su), np, pbase, k, B.w + n0B,
+                                               B.w + n0B, B.qrow, B.r, meta_g).n;
+    fB = nB;
+  }
+  // the survivors rescored exactly, both rows' entries over the lanes
+  const int xa = nA - fA, xt = xa + nB - fB;
+#pragma unroll 1
+  for (int i = lane; i < xt; i += 32) {
+    const bool b = i >= xa;
+    u64* slot = b ? B.w + fB + (i - xa) : A.w + fA + i;
+    const int p = key_index(*slot);
+    const float v = exact_bound_bf16(b ? B.qrow : A.qrow, b ? B.r : A.r,
+                                     meta_g + static_cast<size_t>(p) * 512, p);
+    *slot = sel_key(v, p);
+  }
+  __syncwarp();
+  LOSA_PHASE(20);
+  // each row's exact top min(k, n) by rank (keys are distinct); the entry
+  // of rank k - 1 sets the threshold
+#pragma unroll 1
+  for (int i = lane; i < nA + nB; i += 32) {
+    const bool b = i >= nA;
+    const int n = b ? nB : nA;
+    const u64* w = b ? B.w : A.w;
+    const u64 x = w[b ? i - nA : i];
+    int rk = 0;
+#pragma unroll 4
+    for (int j = 0; j < n; ++j) rk += w[j] > x;
+    if (rk < k) (b ? B.lk : A.lk)[rk] = x;
+    const u64 t0 = b ? thr0B : thr0A;
+    if (rk == k - 1) *(b ? B.thr : A.thr) = x > t0 ? x : t0;
+  }
+  if (lane == 0) {
+    *A.n = min(nA, k);
+    if (hasB) *B.n = min(nB, k);
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // Merge of one active row's lists from the C CTAs of the cluster (one warp).
 // Every CTA's list holds its exact top min(k, its pages) by exact key, and
 // thr its k-th key; the row's top k over all pages is among them, at or
@@ -636,14 +807,14 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, u64* 
   // of the lists in CTA order)
   int incl = nc;
 #pragma unroll
-  for (int o = 1; o < 8; o <<= 1) {
+  for (int o = 1; o < kMaxClusterCtas; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += y;
   }
-  const int total = __shfl_sync(0xffffffffu, incl, 7);
-  int offs[8];
+  const int total = __shfl_sync(0xffffffffu, incl, kMaxClusterCtas - 1);
+  int offs[kMaxClusterCtas];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
+  for (int q = 0; q < kMaxClusterCtas; ++q) {
     const int v = __shfl_sync(0xffffffffu, incl - nc, q);
     offs[q] = q < M.C ? v : 0x7fffffff;
   }
@@ -653,10 +824,17 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, u64* 
     const int f = f0 + lane;
     u64 x = 0;
     if (f < total) {
-      int cf = 0;
+      // the CTA whose entries hold f: the last with its offset at or below f
+      // (offsets are non-decreasing; an empty CTA shares the next one's)
+      int cf = 0, base = 0;
 #pragma unroll
-      for (int q = 1; q < 8; ++q) cf += f >= offs[q];
-      x = ld_dsmem_u64(dsmem(M.lk + static_cast<size_t>(r) * M.lcap + (f - offs[cf]), cf));
+      for (int q = 1; q < kMaxClusterCtas; ++q) {
+        if (f >= offs[q]) {
+          cf = q;
+          base = offs[q];
+        }
+      }
+      x = ld_dsmem_u64(dsmem(M.lk + static_cast<size_t>(r) * M.lcap + (f - base), cf));
     }
     const bool in = f < total && x >= tau0;
     const unsigned bal = __ballot_sync(0xffffffffu, in);
@@ -1138,14 +1316,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the producer (thread 0) refills the slot of the stage before this one
     // once every warp has released it
     if (tid == 0 && t >= 1 && t - 1 + prm.stages < nstg && scal[kSFail] == 0) {
-      if (mbar_wait(&ebar[(t - 1) % prm.stages], ((t - 1) / prm.stages) & 1))
+      if (mbar_wait(&ebar[(t - 1) % prm.stages], ((t - 1) / prm.stages) & 1)) {
         issue_stage(t - 1 + prm.stages);
+        if (t - 1 + prm.stages < 8) LOSA_PHASE(32 + t - 1 + prm.stages);
+      }
       else
         scal[kSFail] = 1;
     }
     // each thread waits for the stage itself (the wait makes the bytes the
     // copy wrote visible to it)
     if (scal[kSFail] == 0 && mbar_wait(&mbar[st], parity)) {
+      if (t < 8) LOSA_PHASE(24 + t);
       if (t == 0) LOSA_PHASE(5);
       if (t == nstg - 1) LOSA_PHASE(6);
       if (DT == LOSA_BF16) {
@@ -1210,6 +1391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the warp has read the stage: release its slot
     __syncwarp();
     if (lane == 0) mbar_arrive(&ebar[st]);
+    if (t < 8) LOSA_PHASE_BY(40 + t, 4 * 32);  // (warp 4: warp 0's scheduler partner)
     const bool chunk_end = ((t + 1) * prm.tile) % spc == 0 || t == nstg - 1;
     if (DT == LOSA_BF16 && chunk_end && sw) {
       const int slot = ((sub * 4) + t4) * 2;
@@ -1235,34 +1417,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int r0 = warp; r0 < R; r0 += 2 * kWarps) {
           const int r1 = r0 + kWarps;
-          auto survivors = [&](int r, int h) {
-            return row_survivors<DT>(
-                scores + r * spc, pnorm + cb, DT == LOSA_BF16 ? qn[r] : make_float2(0.f, 0.f), cn,
-                pr0 + cb, k, prm.lb, w_lk + h * prm.lb, w_uk + h * prm.lb,
-                l_lk + static_cast<size_t>(r) * prm.lcap, l_n[r], l_thr[r], qa + r * rowb, r,
-                meta_g, DT == LOSA_BF16 ? gmx + r * ng : nullptr, ng,
-                DT == LOSA_BF16 ? __uint_as_float(emx[r]) : 0.f);
-          };
-          const int nA = survivors(r0, 0);
-          const int nB = r1 < R ? survivors(r1, 1) : 0;
           if (DT == LOSA_BF16) {
-#pragma unroll 1
-            for (int i = lane; i < nA + nB; i += 32) {
-              const bool b = i >= nA;
-              const int j = b ? prm.lb + i - nA : i;
-              if (w_lk[j] != w_uk[j]) {
-                const int p = key_index(w_lk[j]), r = b ? r1 : r0;
-                const float v = exact_bound_bf16(qa + r * rowb, r, meta_g + static_cast<size_t>(p) * 512, p);
-                w_lk[j] = sel_key(v, p);
-              }
-            }
-            __syncwarp();
+            auto row = [&](int r, int h) {
+              return PairRow{scores + r * spc,
+                             w_lk + h * prm.lb,
+                             l_lk + static_cast<size_t>(r) * prm.lcap,
+                             l_n + r,
+                             l_thr + r,
+                             gmx + r * ng,
+                             __uint_as_float(emx[r]),
+                             qa + r * rowb,
+                             r};
+            };
+            const bool hasB = r1 < R;
+            select_pair_bf16(row(r0, 0), row(hasB ? r1 : r0, 1), hasB, cn, pr0 + cb, k, prm.lb,
+                             ng, meta_g);
+          } else {
+            auto survivors = [&](int r, int h) {
+              return row_survivors<DT>(scores + r * spc, pnorm + cb, make_float2(0.f, 0.f), cn,
+                                       pr0 + cb, k, prm.lb, w_lk + h * prm.lb, w_uk + h * prm.lb,
+                                       l_lk + static_cast<size_t>(r) * prm.lcap, l_n[r], l_thr[r],
+                                       qa + r * rowb, r, meta_g, nullptr, ng, 0.f);
+            };
+            const int nA = survivors(r0, 0);
+            const int nB = r1 < R ? survivors(r1, 1) : 0;
+            row_topk(w_lk, nA, k, l_lk + static_cast<size_t>(r0) * prm.lcap, l_n + r0,
+                     l_thr + r0, l_thr[r0]);
+            if (r1 < R)
+              row_topk(w_lk + prm.lb, nB, k, l_lk + static_cast<size_t>(r1) * prm.lcap, l_n + r1,
+                       l_thr + r1, l_thr[r1]);
           }
-          row_topk(w_lk, nA, k, l_lk + static_cast<size_t>(r0) * prm.lcap, l_n + r0, l_thr + r0,
-                   l_thr[r0]);
-          if (r1 < R)
-            row_topk(w_lk + prm.lb, nB, k, l_lk + static_cast<size_t>(r1) * prm.lcap, l_n + r1,
-                     l_thr + r1, l_thr[r1]);
         }
       }
       __syncthreads();
@@ -1307,9 +1491,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the group's union (slots u = c mod C), and the CTAs' partials are
   // combined through distributed shared memory.
   const bool own = sel && !d.attend_union;
+  // (own pages, no union count asked for: this CTA reads no other CTA's
+  // shared memory from here on, so it arrives at the last cluster barrier
+  // now and only waits there at the end)
+  const bool early_exit_arrival = own && !prm.union_count;
   if (!own) {
     // ================= cluster barrier 1b: every row's selection is final ====
     cluster_sync();
+  } else if (early_exit_arrival) {
+    cluster_arrive();
   }
 
   // ---- the page bitmap: this CTA's rows' selections (own), or every row's,
@@ -1855,7 +2045,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   LOSA_PHASE(17);
   // ================= cluster barrier 3: no CTA leaves while another may
   // still read its shared memory
-  cluster_sync();
+  if (early_exit_arrival) cluster_wait();
+  else cluster_sync();
   if (tid == 0 && scal[kSFail]) atomicCAS(prm.status, 0, LOSA_ERR_DEVICE_TIMEOUT);
   LOSA_PHASE(18);
 }
@@ -1875,10 +2066,12 @@ struct Taker {
   }
 };
 
-constexpr int kMaxCta = 8;             // CTAs per cluster (the portable cluster size)
-constexpr int kEarlyTriggerCtas = 64;  // grids up to this size fit one wave
+// clusters of 8 and of 16 CTAs that can be resident at once (1 CTA per SM)
+struct ClusterRoom {
+  int c8 = 0, c16 = 0;
+};
 
-bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
+bool plan_step(const Dims& d, StepParams* prm, int max_dyn, const ClusterRoom& room) {
   *prm = StepParams();
   prm->d = d;
   const bool bf = d.esz == 2;
@@ -1891,8 +2084,13 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   prm->tile = kStageBytes / prm->rec;  // 64 (bf16) or 32 (fp32) pages per ring stage
   // CTAs per cluster: a ring stage of pages each at least, more when many
   // active rows share the combine
+  // (up to 16 when the CTAs attend their own rows' pages and the 16-CTA
+  // clusters of the whole grid fit one wave)
+  const long long NG = static_cast<long long>(d.S) * d.Hkv;
+  const bool own = bf && sel && !d.attend_union;
+  const int cmax = own && NG <= room.c16 ? kMaxClusterCtas : kMaxCombineCtas;
   int C = std::max((d.P + prm->tile - 1) / prm->tile, (R + 15) / 16);
-  C = std::max(1, std::min(kMaxCta, C));
+  C = std::max(1, std::min(cmax, C));
   if (R == 0) C = 1;
   prm->C = C;
   prm->cp = align_up((d.P + C - 1) / C, 8);
@@ -1918,7 +2116,9 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
   const int ns = n_oa + n_os;
   const int nwords = (d.P + 31) / 32;
   const int MW = (R + 31) / 32;
-  prm->early = static_cast<long long>(d.S) * d.Hkv * C <= kEarlyTriggerCtas;
+  // one wave: every cluster resident at once (the next launch may then be
+  // scheduled from the start)
+  prm->early = NG <= (C > kMaxCombineCtas ? room.c16 : room.c8);
 
   // the largest plan that fits, with at least 4 ring stages when any plan
   // allows it: most pages per score chunk, then most union pages in flight,
@@ -1999,6 +2199,7 @@ bool plan_step(const Dims& d, StepParams* prm, int max_dyn) {
 std::mutex g_attr_mu;
 bool g_attr_done[kMaxDevices] = {};
 int g_attr_dyn[kMaxDevices] = {};
+ClusterRoom g_attr_room[kMaxDevices];
 
 template <int DT>
 cudaError_t set_attrs(int optin, int* dyn) {
@@ -2009,11 +2210,35 @@ cudaError_t set_attrs(int optin, int* dyn) {
   const int mine = optin - static_cast<int>(fa.sharedSizeBytes);
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, mine);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e != cudaSuccess) return e;
   *dyn = std::min(*dyn, mine);
   return cudaSuccess;
 }
 
-int ensure_attributes(int* max_dyn) {
+// clusters of `csize` step CTAs (the largest shared-memory plan) resident at
+// once; 0 when the device cannot place one
+int room_for(int csize, int dyn) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(csize, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, losa_step_kernel<LOSA_BF16>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();  // (not sticky) a size the device cannot place
+    return 0;
+  }
+  return n;
+}
+
+int ensure_attributes(int* max_dyn, ClusterRoom* room) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return record_cuda_error(e);
@@ -2027,17 +2252,21 @@ int ensure_attributes(int* max_dyn) {
     if ((e = set_attrs<LOSA_BF16>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
     if ((e = set_attrs<LOSA_F32>(optin, &dyn)) != cudaSuccess) return record_cuda_error(e);
     g_attr_dyn[dev] = dyn;
+    g_attr_room[dev].c8 = room_for(kMaxCombineCtas, dyn);
+    g_attr_room[dev].c16 = room_for(kMaxClusterCtas, dyn);
     g_attr_done[dev] = true;
   }
   *max_dyn = g_attr_dyn[dev];
+  if (room) *room = g_attr_room[dev];
   return LOSA_OK;
 }
 
 }  // namespace
 
 bool fused_step_fits(const Dims& d, int max_dyn) {
+  // (the 8-CTA plan; a 16-CTA plan of the same shape needs less per CTA)
   StepParams p;
-  return plan_step(d, &p, max_dyn);
+  return plan_step(d, &p, max_dyn, ClusterRoom());
 }
 
 int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, const void* k_prefix,
@@ -2046,10 +2275,12 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
                       int32_t* active_idx, int32_t* page_idx, int32_t* union_count,
                       void* workspace, cudaStream_t st, void* q_ref_out) {
   int max_dyn = 0;
-  int rc = ensure_attributes(&max_dyn);
+  ClusterRoom room;
+  int rc = ensure_attributes(&max_dyn, &room);
   if (rc != LOSA_OK) return rc;
   StepParams prm;
-  if (!plan_step(d, &prm, max_dyn)) return LOSA_ERR_UNSUPPORTED;
+  if (!plan_step(d, &prm, max_dyn, room) && !plan_step(d, &prm, max_dyn, ClusterRoom()))
+    return LOSA_ERR_UNSUPPORTED;
   const long long NG = static_cast<long long>(d.S) * d.Hkv;
   if (NG > 65535) return LOSA_ERR_UNSUPPORTED;
   prm.qc = q_cur;

@@ -38,8 +38,14 @@ PHASES = {
     16: "cluster barrier 2 passed",
     17: "combine done (before cluster barrier 3)",
     18: "end",
+    19: "(warp 0, last chunk) survivors of its two rows found",
+    20: "(warp 0, last chunk) survivors rescored exactly",
 }
-K_PHASES, K_CTAS = 24, 512
+for _t in range(8):
+    PHASES[24 + _t] = f"stage {_t} ready (thread 0)"
+    PHASES[32 + _t] = f"stage {_t} refill issued"
+    PHASES[40 + _t] = f"stage {_t} released by warp 4"
+K_PHASES, K_CTAS = 48, 512
 
 
 def _lib():
