@@ -50,6 +50,29 @@ int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsi
   return r == CUDA_SUCCESS ? LOSA_OK : LOSA_ERR_CUDA;
 }
 
+int make_page_tmap(CUtensorMap* map, const void* base, unsigned long long nrows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!encode) return LOSA_ERR_CUDA;
+  const cuuint64_t dims[3] = {64u, nrows, 2u};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, 128u};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(kPS), 2u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LOSA_OK : LOSA_ERR_CUDA;
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return kSizingSms;

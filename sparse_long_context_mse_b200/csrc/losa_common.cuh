@@ -269,6 +269,12 @@ int record_cuda_error(cudaError_t e);  // stores the message, returns LOSA_ERR_C
 // 128-byte-swizzled boxes of 64 channels x box_rows rows (rows past nrows
 // read as zero).  LOSA_OK, or LOSA_ERR_CUDA if the driver refuses it.
 int make_tmap(CUtensorMap* map, const void* base, unsigned long long nrows, unsigned box_rows);
+// A 3-D map over the same [nrows][kD] bf16 rows whose box is one page of
+// kPS rows, both 64-channel halves: dims (channel within the half, row,
+// half), so that one copy lands the page as [half][row][64 channels] with
+// the 128-byte swizzle (the layout of two 2-D boxes at offsets 0 and
+// kPS * 128).  LOSA_ERR_CUDA if the driver refuses the map.
+int make_page_tmap(CUtensorMap* map, const void* base, unsigned long long nrows);
 int num_sms();
 
 }  // namespace losa

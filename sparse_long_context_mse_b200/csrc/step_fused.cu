@@ -936,6 +936,7 @@ struct StepParams {
   int max_lp;      // union pages per CTA, at most
   int ngp;         // union pages in flight per CTA
   int early;       // release the dependent launch at the start (the grid fits one wave)
+  int page3d;      // bf16 gather: kmap/vmap are 3-D page maps (one copy per page of K or V)
   int pn;          // page-norm entries per (sequence, KV head)
   StepLayout lo;
 };
@@ -1689,10 +1690,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int p = lpages[b0 + i];
         const int row = sg * d.Lc + p * kPS;
         char* dk = bufp + 2 * i * pbytes;
-        tma_load_2d(dk, &kmap, 0, row, &gbar[bt & 1]);
-        tma_load_2d(dk + 2048, &kmap, 64, row, &gbar[bt & 1]);
-        tma_load_2d(dk + pbytes, &vmap, 0, row, &gbar[bt & 1]);
-        tma_load_2d(dk + pbytes + 2048, &vmap, 64, row, &gbar[bt & 1]);
+        if (prm.page3d) {
+          tma_load_3d(dk, &kmap, 0, row, 0, &gbar[bt & 1]);
+          tma_load_3d(dk + pbytes, &vmap, 0, row, 0, &gbar[bt & 1]);
+        } else {
+          tma_load_2d(dk, &kmap, 0, row, &gbar[bt & 1]);
+          tma_load_2d(dk + 2048, &kmap, 64, row, &gbar[bt & 1]);
+          tma_load_2d(dk + pbytes, &vmap, 0, row, &gbar[bt & 1]);
+          tma_load_2d(dk + pbytes + 2048, &vmap, 64, row, &gbar[bt & 1]);
+        }
       }
     } else if (lane == 0) {
       uint32_t bytes = 0;
@@ -2306,9 +2312,13 @@ int launch_fused_step(const Dims& d, const void* q_cur, const void* q_prev, cons
   std::memset(&kmap, 0, sizeof(kmap));
   std::memset(&vmap, 0, sizeof(vmap));
   if (d.dtype == LOSA_BF16 && d.R > 0) {
+    // one 3-D copy per page when the driver takes the page map, else two
+    // 2-D copies (one per 64-channel half)
     const unsigned long long rows = static_cast<unsigned long long>(NG) * d.Lc;
-    if (make_tmap(&kmap, k_prefix, rows, kPS) != LOSA_OK ||
-        make_tmap(&vmap, v_prefix, rows, kPS) != LOSA_OK)
+    prm.page3d = make_page_tmap(&kmap, k_prefix, rows) == LOSA_OK &&
+                 make_page_tmap(&vmap, v_prefix, rows) == LOSA_OK;
+    if (!prm.page3d && (make_tmap(&kmap, k_prefix, rows, kPS) != LOSA_OK ||
+                        make_tmap(&vmap, v_prefix, rows, kPS) != LOSA_OK))
       return record_cuda_error(cudaErrorInvalidValue);
   }
   cudaLaunchConfig_t cfg = {};
