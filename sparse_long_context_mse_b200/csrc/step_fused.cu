@@ -1494,13 +1494,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool own = sel && !d.attend_union;
   // (own pages, no union count asked for: this CTA reads no other CTA's
   // shared memory from here on, so it arrives at the last cluster barrier
-  // now and only waits there at the end)
+  // now and only waits there at the end.  The arrival is relaxed: the only
+  // thing it has to follow is the merge's loads from the other CTAs, and
+  // their values are already in this CTA's selections -- a release would
+  // also wait for the page_idx stores to become visible, for nothing)
   const bool early_exit_arrival = own && !prm.union_count;
   if (!own) {
     // ================= cluster barrier 1b: every row's selection is final ====
     cluster_sync();
   } else if (early_exit_arrival) {
-    cluster_arrive();
+    cluster_arrive_relaxed();
   }
 
   // ---- the page bitmap: this CTA's rows' selections (own), or every row's,
@@ -1885,8 +1888,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncthreads();
+      // (own pages: only the rows this CTA finishes, r = c + C j)
+      const int nmr = own ? n_oa : R;
 #pragma unroll 1
-      for (int r = warp; r < R; r += kWarps) {
+      for (int jr = warp; jr < nmr; jr += kWarps) {
+        const int r = own ? c + C * jr : jr;
         const int m16 = r >> 4, i = r & 15;
         float M = -INFINITY;
         for (int w = 0; w < wpg; ++w) M = fmaxf(M, wp[((m16 * wpg + w) * 16 + i) * ws]);
