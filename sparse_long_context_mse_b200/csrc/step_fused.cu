@@ -796,50 +796,43 @@ __device__ __forceinline__ void merge_row(const MergeCtx& M, int r, int k, u64* 
                                           int32_t* sel) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
+  // one round of remote loads: every CTA's count and threshold (lane = CTA)
+  // and every slot of every CTA's list (lane l: slots l, l + 32, ...; slot
+  // s is entry s % lcap of CTA s / lcap, the lists at the same offsets in
+  // every CTA); slots at or past their CTA's count are dropped below
   int nc = 0;
   u64 th = 0;
   if (lane < M.C) {
     nc = ld_dsmem_s32(dsmem(M.n + r, lane));
     th = ld_dsmem_u64(dsmem(M.thr + r, lane));
   }
-  const u64 tau0 = warp_max_u64(th);
-  // the CTAs' entries at or above tau0 (lane l takes entries l, l + 32, ...
-  // of the lists in CTA order)
-  int incl = nc;
-#pragma unroll
-  for (int o = 1; o < kMaxClusterCtas; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int total = __shfl_sync(0xffffffffu, incl, kMaxClusterCtas - 1);
-  int offs[kMaxClusterCtas];
-#pragma unroll
-  for (int q = 0; q < kMaxClusterCtas; ++q) {
-    const int v = __shfl_sync(0xffffffffu, incl - nc, q);
-    offs[q] = q < M.C ? v : 0x7fffffff;
-  }
+  const int slots = M.C * M.lcap;
+  const u64* row = M.lk + static_cast<size_t>(r) * M.lcap;
   int cnt = 0;
+  u64 tau0 = 0;
 #pragma unroll 1
-  for (int f0 = 0; f0 < total; f0 += 32) {
-    const int f = f0 + lane;
-    u64 x = 0;
-    if (f < total) {
-      // the CTA whose entries hold f: the last with its offset at or below f
-      // (offsets are non-decreasing; an empty CTA shares the next one's)
-      int cf = 0, base = 0;
+  for (int s0 = 0; s0 < slots; s0 += 4 * 32) {
+    u64 x[4];
+    int cta[4], idx[4];
 #pragma unroll
-      for (int q = 1; q < kMaxClusterCtas; ++q) {
-        if (f >= offs[q]) {
-          cf = q;
-          base = offs[q];
-        }
-      }
-      x = ld_dsmem_u64(dsmem(M.lk + static_cast<size_t>(r) * M.lcap + (f - base), cf));
+    for (int i = 0; i < 4; ++i) {
+      const int sl = s0 + 32 * i + lane;
+      cta[i] = sl < slots ? sl / M.lcap : 0;
+      idx[i] = sl - cta[i] * M.lcap;
+      x[i] = sl < slots ? ld_dsmem_u64(dsmem(row + idx[i], cta[i])) : 0ull;
     }
-    const bool in = f < total && x >= tau0;
-    const unsigned bal = __ballot_sync(0xffffffffu, in);
-    if (in) blk[cnt + __popc(bal & lt)] = x;
-    cnt += __popc(bal);
+    // the row's top k over all pages is among the keys at or above the
+    // largest k-th key of the lists
+    if (s0 == 0) tau0 = warp_max_u64(th);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int sl = s0 + 32 * i + lane;
+      const int ncta = __shfl_sync(0xffffffffu, nc, cta[i]);
+      const bool in = sl < slots && idx[i] < ncta && x[i] >= tau0;
+      const unsigned bal = __ballot_sync(0xffffffffu, in);
+      if (in) blk[cnt + __popc(bal & lt)] = x[i];
+      cnt += __popc(bal);
+    }
   }
   __syncwarp();
   // the top min(k, cnt) by rank (distinct keys)
