@@ -29,14 +29,14 @@ PHASES = {
     7: "last chunk's candidate selection starts",
     8: "candidate lists final (before cluster barrier 1)",
     9: "cluster barrier 1 passed",
-    10: "merge done (before cluster barrier 1b)",
-    11: "union and slots done",
+    10: "merge done",
+    11: "the CTA's page list done (own rows' pages, or its union slots)",
     12: "page gather issued",
     13: "suffix attention done",
     14: "first gathered pages landed",
-    15: "page attention done (before cluster barrier 2)",
-    16: "cluster barrier 2 passed",
-    17: "combine done (before cluster barrier 3)",
+    15: "page attention done",
+    16: "partials final (own rows merged, or cluster barrier 2 passed)",
+    17: "outputs written (before the last cluster barrier)",
     18: "end",
     19: "(warp 0, last chunk) survivors of its two rows found",
     20: "(warp 0, last chunk) survivors rescored exactly",
