@@ -1033,8 +1033,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int Ls = seq_len(d, s);                 // this sequence's prefix length
   const int Ps = (Ls + kPS - 1) / kPS;
-  const int pr0 = c * prm.cp;                   // this CTA's range of pages to score
-  const int npg = sel ? max(0, min(Ps, pr0 + prm.cp) - pr0) : 0;
+  // this CTA's range of pages to score: the sequence's own pages split over
+  // the cluster (a sequence shorter than the longest gives each CTA fewer;
+  // the plan's buffers are sized for the longest)
+  const int cps = min(prm.cp, (((Ps + C - 1) / C) + 7) / 8 * 8);
+  const int pr0 = c * cps;
+  const int npg = sel ? max(0, min(Ps, pr0 + cps) - pr0) : 0;
   const int nstg = (npg + prm.tile - 1) / prm.tile;
   const char* meta_g = prm.meta + static_cast<size_t>(sg) * d.Pc * prm.rec;
   const float2* norm_g = prm.norms + static_cast<size_t>(sg) * prm.pn;
