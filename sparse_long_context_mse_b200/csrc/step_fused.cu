@@ -50,6 +50,7 @@
 // LOSA_ERR_DEVICE_TIMEOUT in the status word, and the CTA skips the work
 // that needs the copy but still takes every cluster barrier.
 #include <algorithm>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -656,9 +657,24 @@ struct PairRow {
   int r;                 // the active row
 };
 
+// Records still in the metadata ring (the last chunk: its last stages are
+// not refilled) are read from shared memory by the rescoring.
+struct RingView {
+  const char* ring;  // the ring's first slot
+  int first;         // CTA-local index of the first page still in the ring (or INT_MAX)
+  int pr0;           // the CTA's first page
+  int tile, stages;  // pages per stage, slots
+  __device__ __forceinline__ const char* rec(const char* meta_g, int p) const {
+    const int pl = p - pr0;
+    if (pl >= first)
+      return ring + (pl / tile % stages) * kStageBytes + (pl % tile) * 512;
+    return meta_g + static_cast<size_t>(p) * 512;
+  }
+};
+
 __device__ __forceinline__ void select_pair_bf16(const PairRow& A, const PairRow& B, bool hasB,
                                                  int np, int pbase, int k, int lb, int ng,
-                                                 const char* meta_g) {
+                                                 const char* meta_g, const RingView& rv) {
   const int lane = threadIdx.x & 31;
   const int n0A = *A.n, n0B = hasB ? *B.n : 0;
   const u64 thr0A = *A.thr, thr0B = hasB ? *B.thr : 0ull;
@@ -748,8 +764,7 @@ __device__ __forceinline__ void select_pair_bf16(const PairRow& A, const PairRow
     const bool b = i >= xa;
     u64* slot = b ? B.w + fB + (i - xa) : A.w + fA + i;
     const int p = key_index(*slot);
-    const float v = exact_bound_bf16(b ? B.qrow : A.qrow, b ? B.r : A.r,
-                                     meta_g + static_cast<size_t>(p) * 512, p);
+    const float v = exact_bound_bf16(b ? B.qrow : A.qrow, b ? B.r : A.r, rv.rec(meta_g, p), p);
     *slot = sel_key(v, p);
   }
   __syncwarp();
@@ -1428,8 +1443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                              r};
             };
             const bool hasB = r1 < R;
+            // (the last chunk: the pages of the ring's last stages are still there)
+            const RingView rv{ring, t == nstg - 1 ? max(0, nstg - prm.stages) * prm.tile : INT_MAX,
+                              pr0, prm.tile, prm.stages};
             select_pair_bf16(row(r0, 0), row(hasB ? r1 : r0, 1), hasB, cn, pr0 + cb, k, prm.lb,
-                             ng, meta_g);
+                             ng, meta_g, rv);
           } else {
             auto survivors = [&](int r, int h) {
               return row_survivors<DT>(scores + r * spc, pnorm + cb, make_float2(0.f, 0.f), cn,
